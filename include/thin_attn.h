@@ -1,0 +1,156 @@
+/*
+ * thin_attn -- Thinformer and Thinformer Express attention on NVIDIA B200 (sm_100a).
+ *
+ * C ABI of the library.  Every entry point takes plain pointers and sizes; no
+ * framework types cross this boundary.
+ *
+ * The operation (Thinformer README, "Getting Started"; "Express Language
+ * Modeling" summary, Methodology):
+ *   non-causal  out = attention of every query against a kernel-halving coreset
+ *               C of the S key/value pairs of its (b,h), each coreset point
+ *               weighted S/|C|  ("Thinformer" for unmasked attention);
+ *   causal      Thinformer Express prefill: an exact phase of n_exact tokens,
+ *               then batches of `batch` tokens thinned to coresets as they
+ *               complete, then HALVE merges of four equal-level coresets into
+ *               one of four times the weight.
+ *
+ * Tensor layouts (README, "Getting Started"), all row-major and contiguous:
+ *   q   (B, T, H, E)        k (B, S, H, E)        v (B, S, H, D)
+ *   out (B, T, H, D)        lse (B, H, T) fp32    (causal: S = T)
+ * q, k, v and out share the handle's element type (fp32 or bf16).
+ *
+ * Ownership: the caller owns every tensor it passes; the library never frees
+ * caller memory.  A handle owns its device workspace (allocated on first use
+ * of a (causal, g) plan, or by thin_attn_reserve) and releases it in
+ * thin_attn_destroy.
+ *
+ * Execution: device entry points enqueue kernels on the caller's stream and
+ * return without synchronising.  The host-buffer entry point synchronises.
+ *
+ * Errors: every entry point returns a thin_attn_status; on failure the
+ * calling thread's message is available from thin_attn_last_error().  Invalid
+ * arguments are rejected on the host before anything is enqueued.
+ */
+#ifndef THIN_ATTN_H_
+#define THIN_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define THIN_ATTN_API __attribute__((visibility("default")))
+#else
+#define THIN_ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct thin_attn_s* thin_attn_t;
+
+typedef enum {
+  THIN_ATTN_OK = 0,
+  THIN_ATTN_EINVAL = 1,        /* bad argument: null pointer, shape, g out of range */
+  THIN_ATTN_ENOMEM = 2,        /* device or host allocation failed */
+  THIN_ATTN_ECUDA = 3,         /* a CUDA call failed (message holds the CUDA error) */
+  THIN_ATTN_ETIMEOUT = 4,      /* a bounded device-side wait gave up */
+  THIN_ATTN_EUNSUPPORTED = 5   /* valid request outside what this build implements */
+} thin_attn_status;
+
+typedef enum { THIN_ATTN_FP32 = 0, THIN_ATTN_BF16 = 1 } thin_attn_dtype;
+
+typedef struct {
+  int dtype;       /* thin_attn_dtype of q, k, v, out */
+  int B, T, S, H;  /* batch, queries, keys (ignored when causal: S = T), heads */
+  int E, D;        /* key/query width, value width: multiples of 8, E <= 256, D <= 256 */
+  float scale;     /* softmax scale s; <= 0 selects 1/sqrt(E) */
+  int n_exact;     /* Express exact phase length (causal only) */
+  int batch;       /* Express thin batch length (causal only; > 0) */
+  int device;      /* CUDA device ordinal the handle's memory lives on */
+} thin_attn_config;
+
+/* Sizes of one (causal, g) plan. */
+typedef struct {
+  int levels;                  /* halving levels r of KH-Compress (per sequence or per batch) */
+  int leaf;                    /* leaf size L (points per leaf run) */
+  int subsampled;              /* S' = L 4^r points kept by the systematic subsample */
+  int coreset_rows;            /* non-causal: |C| per (b,h); causal: c per node */
+  int n_batches;               /* causal: completed thin batches n_b */
+  int n_nodes;                 /* causal: node slots (level-0 nodes, then level 1, ...) */
+  int n_halvings;              /* halving instances (entries of the trace layout) */
+  int reserved;
+  uint64_t trace_words;        /* uint32 words of the decision trace */
+  uint64_t coreset_idx_elems;  /* int32 elements of coreset_idx_opt */
+  uint64_t workspace_bytes;    /* device workspace the plan needs */
+} thin_attn_plan_info;
+
+/* Where the decisions of one halving instance sit in the trace. */
+typedef struct {
+  uint32_t bh;           /* b * H + h */
+  uint32_t round_id;     /* Philox round identifier of the halving */
+  uint32_t pair0;        /* Philox pair index of the instance's first pair */
+  uint32_t n_pairs;      /* pairs m of the instance */
+  uint64_t word_offset;  /* first uint32 word; bit i%32 of word i/32 = 1 iff pair i kept its first point */
+} thin_attn_trace_entry;
+
+/* Library version string. */
+THIN_ATTN_API const char* thin_attn_version(void);
+
+/* Message of the last failure on the calling thread ("" when none). */
+THIN_ATTN_API const char* thin_attn_last_error(void);
+
+/* Create a handle for one problem shape.  *out receives the handle. */
+THIN_ATTN_API thin_attn_status thin_attn_create(thin_attn_t* out, const thin_attn_config* cfg);
+
+/* Release the handle and its workspace.  Null is accepted. */
+THIN_ATTN_API thin_attn_status thin_attn_destroy(thin_attn_t h);
+
+/* Sizes of the (causal, g) plan; 0 <= g <= 6. */
+THIN_ATTN_API thin_attn_status thin_attn_plan(thin_attn_t h, int causal, int g, thin_attn_plan_info* info);
+
+/* Allocate the workspace of the (causal, g) plan now (so the first forward allocates nothing). */
+THIN_ATTN_API thin_attn_status thin_attn_reserve(thin_attn_t h, int causal, int g);
+
+/* Copy the trace layout of the (causal, g) plan into entries[0 .. min(capacity, n)-1];
+ * *count receives n (the number of halving instances). */
+THIN_ATTN_API thin_attn_status thin_attn_trace_layout(thin_attn_t h, int causal, int g,
+                                        thin_attn_trace_entry* entries, size_t capacity,
+                                        size_t* count);
+
+/*
+ * Forward pass on device memory.
+ *   q, k, v, out      device pointers in the layouts above
+ *   causal            0: Thinformer; 1: Thinformer Express prefill
+ *   g                 oversampling parameter of KH-Compress, 0..6 (coreset ~ 2^g sqrt(S))
+ *   seed              Philox key of the thinning decisions
+ *   lse_opt           device (B,H,T) fp32 log-sum-exp ln sum_j w_j e^{s q.k_j}, or NULL
+ *   coreset_idx_opt   device int32: non-causal (B,H,|C|) token indices of the coreset;
+ *                     causal (B,H,n_nodes,c) token indices of every node; or NULL
+ *   trace_opt         device uint32[trace_words] decision bits (thin_attn_trace_layout), or NULL
+ *   stream            cudaStream_t to enqueue on (NULL = legacy default stream)
+ * Allocates the plan's workspace on first use (not inside stream capture).
+ */
+THIN_ATTN_API thin_attn_status thin_attn_forward(thin_attn_t h, const void* q, const void* k, const void* v,
+                                   void* out, int causal, int g, uint64_t seed, float* lse_opt,
+                                   int32_t* coreset_idx_opt, uint32_t* trace_opt, void* stream);
+
+/*
+ * Forward pass on host memory: copies q, k, v to device staging owned by the
+ * handle, runs thin_attn_forward on `stream`, copies out (and lse when
+ * lse_opt is not NULL) back, and synchronises the stream.  Page-locked host
+ * buffers give asynchronous copies; pageable ones work too.
+ */
+THIN_ATTN_API thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void* k,
+                                        const void* v, void* out, int causal, int g,
+                                        uint64_t seed, float* lse_opt, void* stream);
+
+/* Synchronise `stream` and report a device-side failure recorded by the
+ * handle's kernels since the last call (THIN_ATTN_ETIMEOUT, ...). */
+THIN_ATTN_API thin_attn_status thin_attn_check(thin_attn_t h, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* THIN_ATTN_H_ */

@@ -1,0 +1,117 @@
+"""The C-ABI library loads, exports what include/thin_attn.h declares, and plans on the host.
+
+No GPU: handles are created and planned only (thin_attn_create and the plan
+queries touch no device); no compute entry point is called.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import thinned_softmax_attention_b200 as T
+import workloads as W
+from oracle import compress_sizes, express_layout, round_batch, round_merge, round_noncausal
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "thin_attn.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(thin_attn_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    T.lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", T.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (thin_attn_\w+)", out))
+    declared = set(_declared())
+    assert declared, "no declarations parsed"
+    assert declared <= exported, declared - exported
+    assert set(T.EXPORTS) <= exported
+    # nothing else leaks out of the library (hidden visibility)
+    assert all(s.startswith("thin_attn_") for s in exported)
+
+
+def test_version_and_error_strings():
+    assert b"thin_attn" in T.lib().thin_attn_version()
+    assert T.lib().thin_attn_last_error() is not None
+
+
+def _handle(w, **kw):
+    return T.ThinAttention(w.B, w.T, w.T if w.causal else w.S, w.H, w.E, w.D, w.torch_dtype,
+                           n_exact=w.n_exact, batch=w.batch, **kw)
+
+
+@pytest.mark.parametrize("name", ["tiny", "vit", "biggan"])
+def test_noncausal_plan_matches_oracle_sizes(name):
+    w = W.WORKLOADS[name]
+    h = _handle(w)
+    p = h.plan(False, w.g)
+    r, L, Ss, C = compress_sizes(w.S, w.g)
+    assert (p["levels"], p["leaf"], p["subsampled"], p["coreset_rows"]) == (r, L, Ss, C)
+    assert p["coreset_idx_elems"] == w.B * w.H * C
+    lay = h.trace_layout(False, w.g)
+    # one entry per (b,h, level, group); every (b,h, level) covers all its pairs exactly once
+    pairs = {}
+    for bh, rid, pair0, m, off in lay:
+        pairs.setdefault((bh, rid), []).append((pair0, m))
+    assert len(pairs) == w.B * w.H * r
+    for (bh, rid), parts in pairs.items():
+        lv = rid
+        assert rid == round_noncausal(lv) and 1 <= lv <= r
+        parts.sort()
+        assert parts[0][0] == 0 and all(a[0] + a[1] == b[0] for a, b in zip(parts, parts[1:]))
+        assert parts[-1][0] + parts[-1][1] == Ss >> lv
+    offs = sorted(e[4] for e in lay)
+    assert len(set(offs)) == len(offs) and p["trace_words"] >= offs[-1] + 1
+
+
+@pytest.mark.parametrize("name", ["express32k", "express128k"])
+def test_express_plan_matches_oracle_layout(name):
+    w = W.WORKLOADS[name]
+    h = _handle(w)
+    p = h.plan(True, w.g)
+    n_b, slots = express_layout(w.T, w.n_exact, w.batch)
+    r, L, Ss, c = compress_sizes(w.batch, w.g)
+    assert (p["n_batches"], p["n_nodes"], p["coreset_rows"], p["levels"]) == (n_b, len(slots), c, r)
+    assert p["coreset_idx_elems"] == w.B * w.H * len(slots) * c
+    lay = h.trace_layout(True, w.g)
+    rounds = {rid for _, rid, _, _, _ in lay}
+    want = {round_batch(k, lv) for k in range(n_b) for lv in range(1, r + 1)}
+    lv = 0
+    while n_b // 4 ** (lv + 1):
+        want |= {round_merge(lv + 1, j, s) for j in range(n_b // 4 ** (lv + 1)) for s in (0, 1)}
+        lv += 1
+    assert rounds == want
+    assert len({e[0] for e in lay}) == w.B * w.H
+
+
+def test_bad_arguments_are_rejected_on_the_host():
+    w = W.WORKLOADS["tiny"]
+    with pytest.raises(T.ThinAttnError, match="EINVAL"):
+        T.ThinAttention(1, 8, 8, 1, 12, 64, w.torch_dtype)          # E not a multiple of 8
+    h = _handle(w)
+    for g in (-1, 7):
+        with pytest.raises(T.ThinAttnError, match="EINVAL"):
+            h.plan(False, g)
+    with pytest.raises(T.ThinAttnError, match="EINVAL"):
+        h.plan(True, 2)                                              # causal needs batch >= 1
+    cfg = T.Config(0, 1, 8, 8, 1, 64, 64, 0.0, 0, 0, 0)
+    hh = ctypes.c_void_p()
+    assert T.lib().thin_attn_create(None, ctypes.byref(cfg)) == 1
+    assert T.lib().thin_attn_create(ctypes.byref(hh), None) == 1
+    assert T.lib().thin_attn_forward(None, None, None, None, None, 0, 2, 0, None, None, None, None) == 1
+    assert T.lib().thin_attn_destroy(None) == 0
+
+
+def test_decode_trace_bit_order():
+    lay = [(3, 7, 0, 40, 0), (3, 7, 40, 40, 2)]
+    words = np.array([0b101, 1 << 7, 1, 0], dtype=np.uint32)
+    d = T.decode_trace(words, lay)
+    bits = d[(3, 7)]
+    assert bits.shape == (80,)
+    assert list(np.nonzero(bits)[0]) == [0, 2, 39, 40]

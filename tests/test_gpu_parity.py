@@ -1,0 +1,206 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+For every case the library runs with its decision trace; the oracle then
+replays the same thinning in follow mode: a decision whose swap margin is
+below 1e-4 of the instance's kernel scale is a near tie and takes the GPU's
+choice, every other decision must agree (mismatches == 0).  Given identical
+coresets the outputs must agree within 1e-2 (bf16) / 1e-5 (fp32) max relative
+error per (b,h) slice (max |o_gpu - o_ref| / max |o_ref|).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import thinned_softmax_attention_b200 as TA
+import workloads as W
+from oracle import express, thinformer
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp32": 1e-5, "bf16": 1e-2}
+LSE_TOL = {"fp32": 1e-5, "bf16": 2e-3}
+
+
+def _rel_err_per_slice(o, ref):
+    """max over (b,h) of max|o - ref| / max|ref| on (B, rows, H, D) arrays."""
+    err = np.abs(o - ref).max(axis=(1, 3))
+    scale = np.abs(ref).max(axis=(1, 3))
+    return float((err / scale).max())
+
+
+def run_case(w, T=None, S=None, heads=None, rows=None, g=None, seed=None, check_heads=None):
+    """Run GPU + oracle on workload ``w`` (optionally resized); returns a dict of measurements."""
+    T = w.T if T is None else T
+    S = (T if w.causal else w.S) if S is None else S
+    g = w.g if g is None else g
+    seed = w.seed if seed is None else seed
+    q, k, v = W.make_qkv(w, T=T, S=S)
+    dev = torch.device("cuda", 0)
+    h = TA.ThinAttention(w.B, T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
+    r = h.forward(q.to(dev), k.to(dev), v.to(dev), causal=w.causal, g=g, seed=seed, return_lse=True,
+                  return_coreset=True, return_trace=True)
+    torch.cuda.synchronize()
+    h.check()
+    follow = TA.decode_trace(r["trace"], h.trace_layout(w.causal, g))
+    hs = list(range(w.H)) if check_heads is None else list(check_heads)
+    rsel = np.arange(T) if rows is None else np.sort(np.asarray(rows))
+    qh, kh, vh = q[:, :, hs], k[:, :, hs], v[:, :, hs]
+    if w.causal:
+        ref = express(qh, kh, vh, w.n_exact, w.batch, g, seed, follow=follow, rows=rsel, heads=(w.H, hs))
+    else:
+        ref = thinformer(qh, kh, vh, g, seed, follow=follow, rows=rsel, heads=(w.H, hs))
+    o = r["out"].float().cpu().numpy()[:, rsel][:, :, hs]
+    lse = r["lse"].cpu().numpy()[:, hs][:, :, rsel]
+    cs = r["coreset"].cpu().numpy()[:, hs]
+    return {
+        "mismatches": ref.stats.mismatches,
+        "near_ties": ref.stats.near_ties,
+        "decisions": ref.stats.decisions,
+        "coreset_equal": bool(np.array_equal(cs, ref.coreset)),
+        "coreset_shape": cs.shape,
+        "out_err": _rel_err_per_slice(o, ref.out),
+        "lse_err": float(np.abs(lse - ref.lse).max()),
+        "ref": ref,
+        "gpu": r,
+    }
+
+
+def assert_parity(res, dtype):
+    assert res["mismatches"] == 0, res
+    assert res["coreset_equal"]
+    assert res["out_err"] <= TOL[dtype], res["out_err"]
+    assert res["lse_err"] <= LSE_TOL[dtype], res["lse_err"]
+
+
+# ------------------------------------------------------------------ non-causal
+
+
+def test_tiny_fp32_full():
+    w = W.WORKLOADS["tiny"]
+    res = run_case(w)
+    assert res["coreset_shape"] == (1, 1, 64)
+    assert_parity(res, "fp32")
+
+
+@pytest.mark.parametrize("name,B", [("vit", 2), ("biggan", 2)])
+def test_reduced_batch_full_length(name, B):
+    w = W.WORKLOADS[name].with_(B=B)
+    res = run_case(w)
+    assert_parity(res, w.dtype)
+
+
+@pytest.mark.parametrize("name", ["vit", "biggan"])
+def test_full_workload_sampled_rows(name):
+    """The full workload in the launch configuration the bench times; outputs checked on sampled rows."""
+    w = W.WORKLOADS[name]
+    rows = np.random.default_rng(0).choice(w.T, 192, replace=False)
+    res = run_case(w, rows=rows)
+    assert_parity(res, w.dtype)
+
+
+@pytest.mark.parametrize("B,H,T,S,E,D,g,dtype", [
+    (2, 3, 77, 1000, 64, 128, 2, "bf16"),    # ragged: S' = 960, groups of 60 (m = 30, not a multiple of 32)
+    (1, 2, 130, 200, 64, 64, 0, "bf16"),     # g = 0: r clamped so leaves are non-empty
+    (1, 1, 40, 64, 64, 64, 3, "fp32"),       # S <= 4^g: coreset = all keys, exact attention
+    (2, 2, 300, 513, 128, 128, 1, "fp32"),   # odd S, fp32
+    (1, 1, 1, 4096, 64, 64, 2, "bf16"),      # a single query
+])
+def test_noncausal_edge_cases(B, H, T, S, E, D, g, dtype):
+    w = W.Workload("edge", B, H, T, S, E, D, dtype, False, g, 11, 5, "iid")
+    res = run_case(w)
+    assert_parity(res, dtype)
+
+
+def test_coreset_equal_to_full_set_is_exact_attention():
+    w = W.Workload("exact", 1, 2, 50, 60, 64, 64, "fp32", False, 3, 1, 9, "iid")
+    res = run_case(w)
+    q, k, v = W.make_qkv(w)
+    ex = torch.nn.functional.scaled_dot_product_attention(
+        q.double().transpose(1, 2), k.double().transpose(1, 2), v.double().transpose(1, 2)).transpose(1, 2)
+    o = res["gpu"]["out"].double().cpu()
+    assert float((o - ex).abs().max() / ex.abs().max()) < 1e-5
+
+
+# ------------------------------------------------------------------ causal (Express)
+
+
+def test_express_reduced():
+    w = W.WORKLOADS["express32k"].with_(H=2, n_exact=512, batch=512)
+    res = run_case(w, T=4608)   # 7 batches + a trailing partial batch; one level-1 merge
+    assert_parity(res, "bf16")
+
+
+@pytest.mark.parametrize("T,n_e,bsz,g,dtype", [
+    (300, 512, 256, 2, "bf16"),     # T < n_e: everything in the exact phase
+    (1000, 0, 64, 1, "bf16"),       # no exact phase; 15 batches, three level-1 merges
+    (700, 100, 16, 2, "fp32"),      # batch <= 4^g: batches are stored whole, merges still halve
+    (2048, 256, 96, 2, "bf16"),     # batch not a power of 4: subsample inside every batch
+])
+def test_express_edge_cases(T, n_e, bsz, g, dtype):
+    w = W.Workload("edge", 1, 2, T, T, 128 if dtype == "bf16" else 64, 128 if dtype == "bf16" else 64, dtype,
+                   True, g, 7, 4, "rope", n_exact=n_e, batch=bsz)
+    res = run_case(w)
+    assert_parity(res, dtype)
+
+
+def test_express_exact_phase_equals_exact_causal_attention():
+    w = W.WORKLOADS["express32k"].with_(H=2, n_exact=256, batch=256)
+    q, k, v = W.make_qkv(w, T=1024)
+    res = run_case(w, T=1024)
+    ex = torch.nn.functional.scaled_dot_product_attention(
+        q.double().transpose(1, 2), k.double().transpose(1, 2), v.double().transpose(1, 2),
+        is_causal=True).transpose(1, 2)
+    o = res["gpu"]["out"].double().cpu()
+    # exact phase and the first batch (no node exists yet) are exact causal attention
+    assert float((o[:, :512] - ex[:, :512]).abs().max() / ex[:, :512].abs().max()) < 1e-2
+
+
+def test_express32k_full_sampled_rows():
+    w = W.WORKLOADS["express32k"]
+    rows = np.random.default_rng(1).choice(w.T, 256, replace=False)
+    res = run_case(w, rows=rows, check_heads=[0, 7, 31])
+    assert_parity(res, "bf16")
+
+
+@pytest.mark.slow
+def test_express128k_full_sampled_rows():
+    w = W.WORKLOADS["express128k"]
+    rows = np.random.default_rng(2).choice(w.T, 128, replace=False)
+    res = run_case(w, rows=rows, check_heads=[5, 30])
+    assert_parity(res, "bf16")
+
+
+# ------------------------------------------------------------------ API paths
+
+
+def test_host_buffer_entry_point_matches_device_path():
+    w = W.WORKLOADS["biggan"].with_(B=2)
+    q, k, v = W.make_qkv(w)
+    h = TA.ThinAttention(w.B, w.T, w.S, w.H, w.E, w.D, w.torch_dtype)
+    dev = torch.device("cuda", 0)
+    r = h.forward(q.to(dev), k.to(dev), v.to(dev), causal=False, g=w.g, seed=w.seed, return_lse=True)
+    out = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype).pin_memory()
+    lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32).pin_memory()
+    h.forward_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), out, causal=False, g=w.g, seed=w.seed, lse=lse)
+    assert torch.equal(out, r["out"].cpu())
+    assert torch.equal(lse, r["lse"].cpu())
+
+
+def test_repeat_calls_are_deterministic():
+    w = W.WORKLOADS["express32k"].with_(H=2, n_exact=256, batch=256)
+    q, k, v = (x.cuda() for x in W.make_qkv(w, T=2048))
+    h = TA.ThinAttention(w.B, 2048, 2048, w.H, w.E, w.D, w.torch_dtype, n_exact=256, batch=256)
+    a = h.forward(q, k, v, causal=True, g=2, seed=3, return_coreset=True)
+    b = h.forward(q, k, v, causal=True, g=2, seed=3, return_coreset=True)
+    c = h.forward(q, k, v, causal=True, g=2, seed=4, return_coreset=True)
+    assert torch.equal(a["out"], b["out"]) and torch.equal(a["coreset"], b["coreset"])
+    assert not torch.equal(a["coreset"], c["coreset"])
+
+
+def test_dropin_call_returns_output_and_none():
+    w = W.WORKLOADS["tiny"]
+    q, k, v = (x.cuda() for x in W.make_qkv(w))
+    out, weights = TA.thinformer_attention(q, k, v, g=2, seed=1)
+    assert weights is None and out.shape == (1, 256, 1, 64)

@@ -1,0 +1,222 @@
+"""thinned_softmax_attention_b200 -- Thinformer and Thinformer Express attention on B200 (sm_100a).
+
+A thin Python binding over the C ABI declared in ``include/thin_attn.h``: it
+only marshals arguments (device pointers of torch tensors, the current CUDA
+stream).  Every step of the computation runs in the CUDA library
+``libthin_attn.so``; if that library is missing the binding raises instead of
+falling back to anything else.
+
+Layouts follow the Thinformer README ("Getting Started"):
+    query (B, T, H, E), key (B, S, H, E), value (B, S, H, D)  ->  attn_output (B, T, H, D)
+with ``causal=True`` meaning Thinformer Express prefill (S = T).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Dict, Optional, Tuple
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libthin_attn.so")
+
+FP32, BF16 = 0, 1
+_STATUS = {0: "OK", 1: "EINVAL", 2: "ENOMEM", 3: "ECUDA", 4: "ETIMEOUT", 5: "EUNSUPPORTED"}
+
+
+class ThinAttnError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"thin_attn {_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("B", ctypes.c_int), ("T", ctypes.c_int), ("S", ctypes.c_int),
+                ("H", ctypes.c_int), ("E", ctypes.c_int), ("D", ctypes.c_int), ("scale", ctypes.c_float),
+                ("n_exact", ctypes.c_int), ("batch", ctypes.c_int), ("device", ctypes.c_int)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("levels", ctypes.c_int), ("leaf", ctypes.c_int), ("subsampled", ctypes.c_int),
+                ("coreset_rows", ctypes.c_int), ("n_batches", ctypes.c_int), ("n_nodes", ctypes.c_int),
+                ("n_halvings", ctypes.c_int), ("reserved", ctypes.c_int), ("trace_words", ctypes.c_uint64),
+                ("coreset_idx_elems", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64)]
+
+
+class TraceEntry(ctypes.Structure):
+    _fields_ = [("bh", ctypes.c_uint32), ("round_id", ctypes.c_uint32), ("pair0", ctypes.c_uint32),
+                ("n_pairs", ctypes.c_uint32), ("word_offset", ctypes.c_uint64)]
+
+
+_lib = None
+EXPORTS = ("thin_attn_version", "thin_attn_last_error", "thin_attn_create", "thin_attn_destroy",
+           "thin_attn_plan", "thin_attn_reserve", "thin_attn_trace_layout", "thin_attn_forward",
+           "thin_attn_forward_host", "thin_attn_check")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libthin_attn.so (built in-tree by ``python -m thinned_softmax_attention_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m thinned_softmax_attention_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
+    L.thin_attn_version.restype = ctypes.c_char_p
+    L.thin_attn_last_error.restype = ctypes.c_char_p
+    L.thin_attn_create.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(Config)]
+    L.thin_attn_destroy.argtypes = [vp]
+    L.thin_attn_plan.argtypes = [vp, i, i, ctypes.POINTER(PlanInfo)]
+    L.thin_attn_reserve.argtypes = [vp, i, i]
+    L.thin_attn_trace_layout.argtypes = [vp, i, i, ctypes.POINTER(TraceEntry), ctypes.c_size_t,
+                                         ctypes.POINTER(ctypes.c_size_t)]
+    L.thin_attn_forward.argtypes = [vp, vp, vp, vp, vp, i, i, u64, vp, vp, vp, vp]
+    L.thin_attn_forward_host.argtypes = [vp, vp, vp, vp, vp, i, i, u64, vp, vp]
+    L.thin_attn_check.argtypes = [vp, vp]
+    for f in EXPORTS[2:]:
+        getattr(L, f).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status != 0:
+        raise ThinAttnError(status, lib().thin_attn_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class ThinAttention:
+    """One problem shape on one device: Thinformer (non-causal) and Thinformer Express (causal).
+
+    ``forward(q, k, v, causal, g, seed)`` returns ``(attn_output, None)``: the dense
+    attention weights are never formed; pass ``return_lse=True`` for the
+    log-sum-exp ln sum_j w_j e^{s q.k_j} instead.
+    """
+
+    def __init__(self, B: int, T: int, S: int, H: int, E: int, D: int, dtype: torch.dtype,
+                 scale: Optional[float] = None, n_exact: int = 0, batch: int = 0, device: int = 0):
+        self.cfg = Config(FP32 if dtype == torch.float32 else BF16, B, T, S, H, E, D,
+                          0.0 if scale is None else float(scale), n_exact, batch, device)
+        self.dtype = dtype
+        self.device = torch.device("cuda", device)
+        self._h = ctypes.c_void_p()
+        _check(lib().thin_attn_create(ctypes.byref(self._h), ctypes.byref(self.cfg)))
+
+    def close(self):
+        if self._h:
+            lib().thin_attn_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def plan(self, causal: bool, g: int) -> Dict[str, int]:
+        info = PlanInfo()
+        _check(lib().thin_attn_plan(self._h, int(causal), g, ctypes.byref(info)))
+        return {f: getattr(info, f) for f, _ in PlanInfo._fields_}
+
+    def reserve(self, causal: bool, g: int):
+        _check(lib().thin_attn_reserve(self._h, int(causal), g))
+
+    def trace_layout(self, causal: bool, g: int):
+        n = ctypes.c_size_t()
+        _check(lib().thin_attn_trace_layout(self._h, int(causal), g, None, 0, ctypes.byref(n)))
+        arr = (TraceEntry * max(1, n.value))()
+        _check(lib().thin_attn_trace_layout(self._h, int(causal), g, arr, n.value, ctypes.byref(n)))
+        return [(e.bh, e.round_id, e.pair0, e.n_pairs, e.word_offset) for e in arr[:n.value]]
+
+    def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, g: int = 2,
+                seed: int = 0, return_lse: bool = False, return_coreset: bool = False,
+                return_trace: bool = False, out: Optional[torch.Tensor] = None):
+        c = self.cfg
+        L = c.T if causal else c.S
+        for name, t, shape in (("q", q, (c.B, c.T, c.H, c.E)), ("k", k, (c.B, L, c.H, c.E)),
+                               ("v", v, (c.B, L, c.H, c.D))):
+            if tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous() or t.device != self.device:
+                raise ValueError(f"{name}: expected contiguous {self.dtype} {shape} on {self.device}, "
+                                 f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+        if out is None:
+            out = torch.empty(c.B, c.T, c.H, c.D, dtype=self.dtype, device=self.device)
+        info = self.plan(causal, g)
+        lse = torch.empty(c.B, c.H, c.T, dtype=torch.float32, device=self.device) if return_lse else None
+        cidx = (torch.empty(max(1, info["coreset_idx_elems"]), dtype=torch.int32, device=self.device)
+                if return_coreset else None)
+        trace = (torch.zeros(max(1, info["trace_words"]), dtype=torch.int32, device=self.device)
+                 if return_trace else None)
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_forward(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), int(causal), g,
+                                       ctypes.c_uint64(seed & (2 ** 64 - 1)), _ptr(lse), _ptr(cidx), _ptr(trace),
+                                       ctypes.c_void_p(stream)))
+        res = {"out": out}
+        if return_lse:
+            res["lse"] = lse
+        if return_coreset:
+            n = info["coreset_idx_elems"]
+            if causal:
+                res["coreset"] = cidx[:n].view(c.B, c.H, info["n_nodes"], info["coreset_rows"])
+            else:
+                res["coreset"] = cidx[:n].view(c.B, c.H, info["coreset_rows"])
+        if return_trace:
+            res["trace"] = trace
+        return res
+
+    def forward_host(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                     causal: bool = False, g: int = 2, seed: int = 0, lse: Optional[torch.Tensor] = None):
+        """Host tensors in, host tensors out (copies included); synchronises the current stream."""
+        for t in (q, k, v, out):
+            if t.device.type != "cpu" or not t.is_contiguous():
+                raise ValueError("forward_host takes contiguous CPU tensors")
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_forward_host(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), int(causal), g,
+                                            ctypes.c_uint64(seed & (2 ** 64 - 1)), _ptr(lse),
+                                            ctypes.c_void_p(stream)))
+        return out
+
+    def check(self):
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_check(self._h, ctypes.c_void_p(stream)))
+
+
+def decode_trace(words, layout) -> Dict[Tuple[int, int], np.ndarray]:
+    """Decision bits of every halving, keyed by (b*H+h, round id), over the Philox pair index."""
+    w = np.asarray(words.cpu().numpy() if isinstance(words, torch.Tensor) else words).view(np.uint32)
+    acc: Dict[Tuple[int, int], Dict[int, np.ndarray]] = {}
+    for bh, rid, pair0, m, off in layout:
+        nw = (m + 31) // 32
+        bits = np.unpackbits(w[off:off + nw].astype("<u4").view(np.uint8), bitorder="little")[:m].astype(bool)
+        acc.setdefault((bh, rid), {})[pair0] = bits
+    return {key: np.concatenate([parts[p0] for p0 in sorted(parts)]) for key, parts in acc.items()}
+
+
+_cache: Dict[tuple, ThinAttention] = {}
+
+
+def thinformer_attention(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, causal: bool = False,
+                         g: int = 2, seed: int = 0, n_exact: int = 1024, batch: int = 1024,
+                         scale: Optional[float] = None):
+    """Drop-in attention layer call: ``attn_output, attn_output_weights = thinformer_attention(q, k, v)``.
+
+    ``attn_output_weights`` is always None (the dense weights are never formed).
+    """
+    B, T, H, E = query.shape
+    S, D = key.shape[1], value.shape[3]
+    dev = query.device.index or 0
+    k_ = (B, T, S, H, E, D, query.dtype, scale, n_exact if causal else 0, batch if causal else 0, dev)
+    if k_ not in _cache:
+        _cache[k_] = ThinAttention(B, T, S, H, E, D, query.dtype, scale, n_exact if causal else 0,
+                                   batch if causal else 0, dev)
+    return _cache[k_].forward(query, key, value, causal=causal, g=g, seed=seed)["out"], None
+
+
+__all__ = ["ThinAttention", "ThinAttnError", "thinformer_attention", "decode_trace", "lib", "LIB_PATH",
+           "EXPORTS"]

@@ -1,0 +1,740 @@
+// C ABI of thin_attn: argument checks, the (causal, g) plans, workspace, launch sequence.
+//
+// Plan of the non-causal path (Thinformer; README "Getting Started" layouts):
+//   per (b,h): systematic subsample of the S keys to S' = L 4^r, then r halving
+//   levels over groups of 4 L 2^(l-1) consecutive points (KH-Compress), then
+//   attention of every query against the |C| = L 2^r survivors, weight S/|C|.
+// Plan of the causal path (Thinformer Express; "Express Language Modeling",
+// "The EXPRESS Meta-Procedure"):
+//   exact phase [0, n_e); batch k = [n_e + k b, n_e + (k+1) b) compressed to c
+//   points (weight b/c); a 4-ary counter merges four level-l nodes by two
+//   halvings (4c -> 2c -> c, weight x4); a query of batch k attends to the exact
+//   prefix, the nodes present after k completed batches, and its batch causally.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "thin_attn.h"
+
+using namespace thin;
+
+namespace {
+
+thread_local std::string g_err;
+
+thin_attn_status fail(thin_attn_status s, const char* fmt, ...) {
+  char buf[1024];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+#define CK(call)                                                                               \
+  do {                                                                                         \
+    cudaError_t e_ = (call);                                                                   \
+    if (e_ != cudaSuccess) return fail(THIN_ATTN_ECUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+struct Sizes {
+  int r, L, S_sub, C;
+};
+
+// Least r with 4^(g+r) >= S, lowered (g = 0 only) until 4^r <= S; L = floor(S/4^r).
+Sizes compress_sizes(int64_t S, int g) {
+  if (S <= 0) return {0, 0, 0, 0};
+  int r = 0;
+  auto p4 = [](int e) { return (int64_t)1 << (2 * e); };
+  while (p4(g + r) < S) ++r;
+  while (r > 0 && p4(r) > S) --r;
+  const int64_t L = S / p4(r);
+  return {r, (int)L, (int)(L * p4(r)), (int)(L << r)};
+}
+
+uint32_t round_noncausal(int level) { return (uint32_t)level; }
+uint32_t round_batch(int k, int level) { return 0x40000000u | ((uint32_t)k << 4) | (uint32_t)level; }
+uint32_t round_merge(int level, int node, int step) {
+  return 0x80000000u | ((uint32_t)level << 24) | ((uint32_t)node << 1) | (uint32_t)step;
+}
+uint32_t round_subsample(int k) { return 0xC0000000u | (uint32_t)k; }
+
+enum : int { BUF_TOKENS = -1, BUF_NODES = -2, BUF_MTEMP = -3 };
+
+struct BufSpec {
+  int64_t rows = 0;
+  size_t k_off = 0, v_off = 0, idx_off = 0;
+};
+
+struct StepPlan {
+  bool copy_only = false;
+  int src_buf = BUF_TOKENS, dst_buf = 0;
+  int n = 0, m = 0, m_pad = 0;
+  int S_full = 0, S_sub = 0;
+  std::vector<HalveInst> inst;
+  size_t inst_off = 0;
+  uint64_t trace_base = 0;
+};
+
+struct AttnTables {
+  int rows_per_tile = 0;
+  std::vector<AttnTile> tiles;
+  std::vector<AttnSeg> segs;
+  size_t tiles_off = 0, segs_off = 0;
+};
+
+struct Plan {
+  int causal = 0, g = 0;
+  Sizes sz{};
+  int n_b = 0, n_slots = 0, c = 0;
+  std::vector<int> level_base;   // causal: first slot of each node level
+  std::vector<StepPlan> steps;
+  std::vector<BufSpec> levels;   // intermediate halving outputs
+  BufSpec nodes, mtemp;
+  std::vector<thin_attn_trace_entry> trace;
+  uint64_t trace_words = 0;
+  uint64_t coreset_idx_elems = 0;
+  int final_buf = BUF_TOKENS;    // compact buffer holding the coreset / nodes
+  int att_slots = 1, att_slot_rows = 0;
+  AttnTables simt, tc;
+  size_t delta_off = 0, c2_off = 0, delta_floats = 0, c2_floats = 0;
+  size_t bytes = 0;
+  void* d_mem = nullptr;
+};
+
+}  // namespace
+
+struct thin_attn_s {
+  thin_attn_config cfg{};
+  float scale = 0.f;
+  std::mutex mu;
+  std::map<std::pair<int, int>, Plan*> plans;
+  int* d_status = nullptr;
+  // host-buffer staging
+  void* st_mem = nullptr;
+  size_t st_bytes = 0;
+};
+
+namespace {
+
+size_t elt(const thin_attn_config& c) { return c.dtype == THIN_ATTN_FP32 ? 4 : 2; }
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (dev < 0) return;   // nothing on a device to touch
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+void build_attn_tables(const thin_attn_config& cf, const Plan& p, int QT, AttnTables& t) {
+  t.rows_per_tile = QT;
+  t.tiles.clear();
+  t.segs.clear();
+  if (!p.causal) {
+    AttnSeg s{};
+    if (p.sz.r == 0) {
+      s.kind = SEG_TOKENS;
+      s.first = 0;
+      s.len = cf.S;
+      s.logw = 0.f;
+    } else {
+      s.kind = SEG_COMPACT;
+      s.first = 0;
+      s.len = p.sz.C;
+      s.logw = (float)std::log((double)cf.S / (double)p.sz.C);
+    }
+    t.segs.push_back(s);
+    for (int q0 = 0; q0 < cf.T; q0 += QT) t.tiles.push_back({q0, std::min(QT, cf.T - q0), 0, 1});
+    return;
+  }
+  const int T = cf.T, ne = std::min(cf.n_exact, T), bsz = cf.batch;
+  for (int q0 = 0; q0 < ne; q0 += QT) {
+    const int ql = std::min(QT, ne - q0);
+    t.tiles.push_back({q0, ql, (int)t.segs.size(), 1});
+    t.segs.push_back({SEG_TOKENS, 0, q0 + ql, 1, 0.f, 0});
+  }
+  for (int k = 0;; ++k) {
+    const int64_t start = (int64_t)ne + (int64_t)k * bsz;
+    if (start >= T) break;
+    const int end = (int)std::min<int64_t>(start + bsz, T);
+    // nodes after k completed batches: base-4 digit d_l of k -> d_l nodes of level l
+    std::vector<std::pair<int, int>> snap;
+    for (int lv = 0; ((int64_t)1 << (2 * lv)) <= k; ++lv) {
+      const int64_t p4 = (int64_t)1 << (2 * lv);
+      const int d = (int)((k / p4) % 4);
+      const int base = (int)((k / (p4 * 4)) * 4);
+      for (int j = 0; j < d; ++j) snap.push_back({lv, base + j});
+    }
+    for (int q0 = (int)start; q0 < end; q0 += QT) {
+      const int ql = std::min(QT, end - q0);
+      const int seg0 = (int)t.segs.size();
+      if (ne > 0) t.segs.push_back({SEG_TOKENS, 0, ne, 0, 0.f, 0});
+      for (auto& nd : snap) {
+        const double w = std::ldexp((double)bsz / p.c, 2 * nd.first);
+        t.segs.push_back({SEG_COMPACT, p.level_base[nd.first] + nd.second, p.c, 0, (float)std::log(w), 0});
+      }
+      t.segs.push_back({SEG_TOKENS, (int)start, q0 + ql - (int)start, 1, 0.f, 0});
+      t.tiles.push_back({q0, ql, seg0, (int)t.segs.size() - seg0});
+    }
+  }
+}
+
+// Append the halving steps of KH-Compress of `runs` token runs of length S_run each.
+// run r: (bh, b*L_seq + tok0, tok0, batch id k for round ids, dst rows of the final level).
+struct RunDesc {
+  uint32_t bh;
+  int64_t src_row;
+  uint32_t tok0;
+  int k;                 // -1: non-causal (round = level), else Express batch index
+  int64_t final_dst;     // first destination row of the level-r output (buffer final_buf)
+};
+
+void add_compress_steps(Plan& p, const std::vector<RunDesc>& runs, int S_run, int final_buf,
+                        std::vector<int64_t>& level_rows_per_run) {
+  const Sizes sz = compress_sizes(S_run, p.g);
+  level_rows_per_run.clear();
+  const int nr = (int)runs.size();
+  for (int lv = 1; lv <= sz.r; ++lv) {
+    StepPlan st;
+    st.n = 4 * sz.L * (1 << (lv - 1));
+    st.m = st.n / 2;
+    st.m_pad = (st.m + 31) / 32 * 32;
+    const int in_rows = sz.S_sub >> (lv - 1);   // points per run entering this level
+    const int G = in_rows / st.n;
+    const int out_rows = in_rows / 2;
+    st.src_buf = lv == 1 ? BUF_TOKENS : (int)p.levels.size() - 1;
+    if (lv == sz.r) {
+      st.dst_buf = final_buf;
+    } else {
+      BufSpec b;
+      b.rows = (int64_t)nr * out_rows;
+      p.levels.push_back(b);
+      st.dst_buf = (int)p.levels.size() - 1;
+    }
+    st.S_full = S_run;
+    st.S_sub = sz.S_sub;
+    for (int r = 0; r < nr; ++r) {
+      const RunDesc& rd = runs[r];
+      for (int gi = 0; gi < G; ++gi) {
+        HalveInst in{};
+        in.src_row = lv == 1 ? rd.src_row : (int64_t)r * in_rows + (int64_t)gi * st.n;
+        in.dst_row = (lv == sz.r ? rd.final_dst : (int64_t)r * out_rows) + (int64_t)gi * st.m;
+        in.bh = rd.bh;
+        in.round_id = rd.k < 0 ? round_noncausal(lv) : round_batch(rd.k, lv);
+        in.pair0 = (uint32_t)(gi * st.m);
+        in.sub_round = round_subsample(rd.k < 0 ? 0 : rd.k);
+        in.tok0 = rd.tok0;
+        st.inst.push_back(in);
+      }
+    }
+    p.steps.push_back(std::move(st));
+  }
+}
+
+thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
+  const thin_attn_config& cf = h->cfg;
+  Plan* p = new Plan();
+  p->causal = causal;
+  p->g = g;
+  const int BH = cf.B * cf.H;
+  if (!causal) {
+    p->sz = compress_sizes(cf.S, g);
+    p->final_buf = BUF_TOKENS;
+    if (p->sz.r > 0) {
+      p->levels.reserve(p->sz.r + 1);
+      std::vector<RunDesc> runs;
+      for (int bh = 0; bh < BH; ++bh) {
+        const int b = bh / cf.H;
+        runs.push_back({(uint32_t)bh, (int64_t)b * cf.S, 0u, -1, (int64_t)bh * p->sz.C});
+      }
+      // the final level writes into its own buffer appended after the intermediates
+      std::vector<int64_t> lr;
+      const int final_index = p->sz.r - 1;   // levels 1..r-1 are intermediates -> indices 0..r-2
+      add_compress_steps(*p, runs, cf.S, final_index, lr);
+      BufSpec fb;
+      fb.rows = (int64_t)BH * p->sz.C;
+      p->levels.push_back(fb);
+      p->final_buf = final_index;
+      p->att_slots = 1;
+      p->att_slot_rows = p->sz.C;
+    }
+    p->coreset_idx_elems = (uint64_t)BH * (p->sz.r > 0 ? p->sz.C : cf.S);
+  } else {
+    const int T = cf.T, ne = std::min(cf.n_exact, T), bsz = cf.batch;
+    p->n_b = T > ne ? (T - ne) / bsz : 0;
+    p->sz = compress_sizes(bsz, g);
+    p->c = p->sz.C;
+    for (int lv = 0; (p->n_b >> (2 * lv)) > 0; ++lv) {
+      p->level_base.push_back(p->n_slots);
+      p->n_slots += p->n_b >> (2 * lv);
+    }
+    p->nodes.rows = (int64_t)BH * p->n_slots * p->c;
+    p->final_buf = BUF_NODES;
+    p->att_slots = p->n_slots;
+    p->att_slot_rows = p->c;
+    if (p->n_b > 0) {
+      std::vector<RunDesc> runs;
+      for (int bh = 0; bh < BH; ++bh)
+        for (int k = 0; k < p->n_b; ++k) {
+          const int b = bh / cf.H;
+          const uint32_t tok0 = (uint32_t)(ne + k * bsz);
+          runs.push_back({(uint32_t)bh, (int64_t)b * T + tok0, tok0, k,
+                          ((int64_t)bh * p->n_slots + k) * p->c});
+        }
+      if (p->sz.r == 0) {
+        StepPlan st;
+        st.copy_only = true;
+        st.n = bsz;
+        st.src_buf = BUF_TOKENS;
+        st.dst_buf = BUF_NODES;
+        st.S_full = st.S_sub = bsz;
+        for (auto& rd : runs) {
+          HalveInst in{};
+          in.src_row = rd.src_row;
+          in.dst_row = rd.final_dst;
+          in.bh = rd.bh;
+          in.tok0 = rd.tok0;
+          st.inst.push_back(in);
+        }
+        p->steps.push_back(std::move(st));
+      } else {
+        std::vector<int64_t> lr;
+        add_compress_steps(*p, runs, bsz, BUF_NODES, lr);
+      }
+      // HALVE merges: target level L' takes level L'-1 slots 4j'..4j'+3
+      const int nj1 = p->n_b / 4;
+      p->mtemp.rows = (int64_t)BH * nj1 * 2 * p->c;
+      for (int lv = 1; (p->n_b >> (2 * lv)) > 0; ++lv) {
+        const int nj = p->n_b >> (2 * lv);
+        for (int step = 0; step < 2; ++step) {
+          StepPlan st;
+          st.n = (step == 0 ? 4 : 2) * p->c;
+          st.m = st.n / 2;
+          st.m_pad = (st.m + 31) / 32 * 32;
+          st.src_buf = step == 0 ? BUF_NODES : BUF_MTEMP;
+          st.dst_buf = step == 0 ? BUF_MTEMP : BUF_NODES;
+          st.S_full = st.S_sub = st.n;
+          for (int bh = 0; bh < BH; ++bh)
+            for (int j = 0; j < nj; ++j) {
+              HalveInst in{};
+              const int64_t mt = ((int64_t)bh * nj + j) * 2 * p->c;
+              if (step == 0) {
+                in.src_row = ((int64_t)bh * p->n_slots + p->level_base[lv - 1] + 4 * j) * p->c;
+                in.dst_row = mt;
+              } else {
+                in.src_row = mt;
+                in.dst_row = ((int64_t)bh * p->n_slots + p->level_base[lv] + j) * p->c;
+              }
+              in.bh = (uint32_t)bh;
+              in.round_id = round_merge(lv, j, step);
+              in.pair0 = 0;
+              st.inst.push_back(in);
+            }
+          p->steps.push_back(std::move(st));
+        }
+      }
+    }
+    p->coreset_idx_elems = (uint64_t)p->nodes.rows;
+  }
+  // trace layout and scratch sizes
+  for (auto& st : p->steps) {
+    if (st.copy_only) continue;
+    st.trace_base = p->trace_words;
+    const int nw = st.m_pad / 32;
+    for (size_t i = 0; i < st.inst.size(); ++i) {
+      const HalveInst& in = st.inst[i];
+      p->trace.push_back({in.bh, in.round_id, in.pair0, (uint32_t)st.m, st.trace_base + i * nw});
+    }
+    p->trace_words += (uint64_t)st.inst.size() * nw;
+    p->delta_floats = std::max(p->delta_floats, st.inst.size() * (size_t)st.m_pad * st.m_pad);
+    p->c2_floats = std::max(p->c2_floats, st.inst.size());
+  }
+  build_attn_tables(cf, *p, attention_simt_tile_rows(), p->simt);
+  if (attention_tc_supported(cf.dtype, cf.E, cf.D)) build_attn_tables(cf, *p, attention_tc_tile_rows(), p->tc);
+  // memory layout: tables first, then buffers
+  size_t off = 0;
+  for (auto& st : p->steps) {
+    st.inst_off = off;
+    off = align256(off + st.inst.size() * sizeof(HalveInst));
+  }
+  for (AttnTables* t : {&p->simt, &p->tc}) {
+    t->tiles_off = off;
+    off = align256(off + t->tiles.size() * sizeof(AttnTile));
+    t->segs_off = off;
+    off = align256(off + t->segs.size() * sizeof(AttnSeg));
+  }
+  const size_t es = elt(cf);
+  auto place = [&](BufSpec& b) {
+    b.k_off = off;
+    off = align256(off + (size_t)b.rows * cf.E * es);
+    b.v_off = off;
+    off = align256(off + (size_t)b.rows * cf.D * es);
+    b.idx_off = off;
+    off = align256(off + (size_t)b.rows * 4);
+  };
+  for (auto& b : p->levels) place(b);
+  place(p->nodes);
+  place(p->mtemp);
+  p->delta_off = off;
+  off = align256(off + p->delta_floats * 4);
+  p->c2_off = off;
+  off = align256(off + p->c2_floats * 4);
+  p->bytes = off;
+  *out = p;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status materialise(thin_attn_s* h, Plan* p) {
+  if (!h->d_status) {
+    cudaError_t e = cudaMalloc(&h->d_status, 16);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      h->d_status = nullptr;
+      return fail(THIN_ATTN_ENOMEM, "status word: %s", cudaGetErrorString(e));
+    }
+    e = cudaMemset(h->d_status, 0, 16);
+    if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "status word: %s", cudaGetErrorString(e));
+  }
+  if (p->d_mem) return THIN_ATTN_OK;
+  void* mem = nullptr;
+  cudaError_t e = cudaMalloc(&mem, std::max<size_t>(p->bytes, 256));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(THIN_ATTN_ENOMEM, "workspace of %zu bytes: %s", p->bytes, cudaGetErrorString(e));
+  }
+  // upload tables
+  std::vector<char> host(p->steps.empty() && p->simt.tiles.empty() ? 0 : p->delta_off);
+  size_t tbl_end = 0;
+  for (auto& st : p->steps) {
+    if (!st.inst.empty()) std::memcpy(host.data() + st.inst_off, st.inst.data(), st.inst.size() * sizeof(HalveInst));
+    tbl_end = std::max(tbl_end, st.inst_off + st.inst.size() * sizeof(HalveInst));
+  }
+  for (AttnTables* t : {&p->simt, &p->tc}) {
+    if (!t->tiles.empty()) std::memcpy(host.data() + t->tiles_off, t->tiles.data(), t->tiles.size() * sizeof(AttnTile));
+    if (!t->segs.empty()) std::memcpy(host.data() + t->segs_off, t->segs.data(), t->segs.size() * sizeof(AttnSeg));
+    tbl_end = std::max(tbl_end, t->segs_off + t->segs.size() * sizeof(AttnSeg));
+  }
+  if (tbl_end) {
+    e = cudaMemcpy(mem, host.data(), tbl_end, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+      cudaFree(mem);
+      return fail(THIN_ATTN_ECUDA, "table upload: %s", cudaGetErrorString(e));
+    }
+  }
+  p->d_mem = mem;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status check_cfg(const thin_attn_config* c) {
+  if (!c) return fail(THIN_ATTN_EINVAL, "config is null");
+  if (c->dtype != THIN_ATTN_FP32 && c->dtype != THIN_ATTN_BF16) return fail(THIN_ATTN_EINVAL, "dtype %d", c->dtype);
+  if (c->B < 1 || c->T < 1 || c->H < 1) return fail(THIN_ATTN_EINVAL, "B, T, H must be >= 1");
+  if (c->E < 8 || c->E > 256 || c->E % 8 || c->D < 8 || c->D > 256 || c->D % 8)
+    return fail(THIN_ATTN_EINVAL, "E=%d D=%d: widths must be multiples of 8 in [8, 256]", c->E, c->D);
+  if ((int64_t)c->B * c->T * c->H > ((int64_t)1 << 31) / 4) return fail(THIN_ATTN_EINVAL, "B*T*H too large");
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status get_plan(thin_attn_s* h, int causal, int g, Plan** out) {
+  if (causal != 0 && causal != 1) return fail(THIN_ATTN_EINVAL, "causal must be 0 or 1");
+  if (g < 0 || g > 6) return fail(THIN_ATTN_EINVAL, "g=%d outside 0..6", g);
+  const thin_attn_config& c = h->cfg;
+  if (!causal && (c.S < 1)) return fail(THIN_ATTN_EINVAL, "non-causal attention needs S >= 1");
+  if (causal && (c.batch < 1 || c.n_exact < 0))
+    return fail(THIN_ATTN_EINVAL, "causal attention needs batch >= 1 and n_exact >= 0");
+  auto key = std::make_pair(causal, g);
+  auto it = h->plans.find(key);
+  if (it != h->plans.end()) {
+    *out = it->second;
+    return THIN_ATTN_OK;
+  }
+  Plan* p = nullptr;
+  thin_attn_status s = build_plan(h, causal, g, &p);
+  if (s != THIN_ATTN_OK) return s;
+  for (auto& st : p->steps)
+    if (!st.copy_only && st.m_pad > 2048) {
+      delete p;
+      return fail(THIN_ATTN_EUNSUPPORTED, "halving instance of %d points exceeds 4096", st.n);
+    }
+  h->plans[key] = p;
+  *out = p;
+  return THIN_ATTN_OK;
+}
+
+char* base_of(Plan* p) { return (char*)p->d_mem; }
+
+void buf_ptrs(Plan* p, int id, const void* k, const void* v, const void** K, const void** V,
+              int32_t** idx) {
+  if (id == BUF_TOKENS) {
+    *K = k;
+    *V = v;
+    *idx = nullptr;
+    return;
+  }
+  const BufSpec& b = id == BUF_NODES ? p->nodes : id == BUF_MTEMP ? p->mtemp : p->levels[id];
+  *K = base_of(p) + b.k_off;
+  *V = base_of(p) + b.v_off;
+  *idx = (int32_t*)(base_of(p) + b.idx_off);
+}
+
+thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void* k, const void* v, void* out,
+                             uint64_t seed, float* lse, int32_t* cidx, uint32_t* trace, cudaStream_t st) {
+  const thin_attn_config& cf = h->cfg;
+  const bool use_tc_gram = std::getenv("THIN_ATTN_SIMT_GRAM") == nullptr;
+  for (auto& sp : p->steps) {
+    StepArgs a{};
+    const void *sk, *sv;
+    int32_t* sidx;
+    buf_ptrs(p, sp.src_buf, k, v, &sk, &sv, &sidx);
+    const void *dk, *dv;
+    int32_t* didx;
+    buf_ptrs(p, sp.dst_buf, k, v, &dk, &dv, &didx);
+    a.src_kind = sp.src_buf == BUF_TOKENS ? SRC_TOKENS : SRC_COMPACT;
+    a.srcK = sk;
+    a.srcV = sv;
+    a.srcIdx = sidx;
+    a.H = cf.H;
+    a.S_full = sp.S_full;
+    a.S_sub = sp.S_sub;
+    a.dstK = (void*)dk;
+    a.dstV = (void*)dv;
+    a.dstIdx = didx;
+    a.inst = (const HalveInst*)(base_of(p) + sp.inst_off);
+    a.n_inst = (int)sp.inst.size();
+    a.n = sp.n;
+    a.m = sp.m;
+    a.m_pad = sp.m_pad;
+    a.E = cf.E;
+    a.D = cf.D;
+    a.scale_log2e = (float)((double)h->scale * 1.4426950408889634);
+    a.C = sp.m > 0 ? (float)std::sqrt(2.0 * std::log(4.0 * sp.m)) : 0.f;
+    a.seed = seed;
+    a.c2 = (float*)(base_of(p) + p->c2_off);
+    a.delta = (float*)(base_of(p) + p->delta_off);
+    a.trace = trace;
+    a.trace_base = sp.trace_base;
+    cudaError_t e = sp.copy_only ? launch_copy_step(a, cf.dtype, st)
+                                 : launch_halving_step(a, cf.dtype, use_tc_gram, st);
+    if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "halving step (n=%d): %s", sp.n, cudaGetErrorString(e));
+  }
+  if (cidx) {
+    if (p->final_buf == BUF_TOKENS) {
+      cudaError_t e = launch_iota(cidx, (int64_t)p->coreset_idx_elems, cf.S, st);
+      if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "iota: %s", cudaGetErrorString(e));
+    } else if (p->coreset_idx_elems) {
+      const void *dk, *dv;
+      int32_t* didx;
+      buf_ptrs(p, p->final_buf, k, v, &dk, &dv, &didx);
+      CK(cudaMemcpyAsync(cidx, didx, p->coreset_idx_elems * 4, cudaMemcpyDeviceToDevice, st));
+    }
+  }
+  AttnArgs aa{};
+  aa.q = q;
+  aa.k = k;
+  aa.v = v;
+  if (p->final_buf != BUF_TOKENS) {
+    int32_t* didx;
+    buf_ptrs(p, p->final_buf, k, v, &aa.ck, &aa.cv, &didx);
+  }
+  aa.out = out;
+  aa.lse = lse;
+  aa.B = cf.B;
+  aa.T = cf.T;
+  aa.L = p->causal ? cf.T : cf.S;
+  aa.H = cf.H;
+  aa.E = cf.E;
+  aa.D = cf.D;
+  aa.n_slots = p->att_slots;
+  aa.slot_rows = p->att_slot_rows;
+  aa.scale_log2e = (float)((double)h->scale * 1.4426950408889634);
+  bool done = false;
+  if (!p->tc.tiles.empty() && std::getenv("THIN_ATTN_SIMT_ATTN") == nullptr) {
+    aa.tiles = (const AttnTile*)(base_of(p) + p->tc.tiles_off);
+    aa.segs = (const AttnSeg*)(base_of(p) + p->tc.segs_off);
+    aa.n_tiles = (int)p->tc.tiles.size();
+    cudaError_t e = launch_attention_tc(aa, h->d_status, st, &done);
+    if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "attention (tensor cores): %s", cudaGetErrorString(e));
+  }
+  if (!done) {
+    aa.tiles = (const AttnTile*)(base_of(p) + p->simt.tiles_off);
+    aa.segs = (const AttnSeg*)(base_of(p) + p->simt.segs_off);
+    aa.n_tiles = (int)p->simt.tiles.size();
+    cudaError_t e = launch_attention_simt(aa, cf.dtype, st);
+    if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "attention: %s", cudaGetErrorString(e));
+  }
+  return THIN_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* thin_attn_version(void) { return "thin_attn 0.1 (sm_100a)"; }
+
+const char* thin_attn_last_error(void) { return g_err.c_str(); }
+
+thin_attn_status thin_attn_create(thin_attn_t* out, const thin_attn_config* cfg) {
+  if (!out) return fail(THIN_ATTN_EINVAL, "out is null");
+  *out = nullptr;
+  thin_attn_status s = check_cfg(cfg);
+  if (s != THIN_ATTN_OK) return s;
+  thin_attn_s* h = new thin_attn_s();
+  h->cfg = *cfg;
+  h->scale = cfg->scale > 0.f ? cfg->scale : (float)(1.0 / std::sqrt((double)cfg->E));
+  *out = h;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_destroy(thin_attn_t h) {
+  if (!h) return THIN_ATTN_OK;
+  const bool on_device = h->d_status || h->st_mem;
+  DeviceGuard dg(on_device ? h->cfg.device : -1);
+  for (auto& kv : h->plans) {
+    if (kv.second->d_mem) cudaFree(kv.second->d_mem);
+    delete kv.second;
+  }
+  if (h->d_status) cudaFree(h->d_status);
+  if (h->st_mem) cudaFree(h->st_mem);
+  delete h;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_plan(thin_attn_t h, int causal, int g, thin_attn_plan_info* info) {
+  if (!h || !info) return fail(THIN_ATTN_EINVAL, "null argument");
+  std::lock_guard<std::mutex> lk(h->mu);
+  Plan* p = nullptr;
+  thin_attn_status s = get_plan(h, causal, g, &p);
+  if (s != THIN_ATTN_OK) return s;
+  std::memset(info, 0, sizeof *info);
+  info->levels = p->sz.r;
+  info->leaf = p->sz.L;
+  info->subsampled = p->sz.S_sub;
+  info->coreset_rows = causal ? p->c : (p->sz.r > 0 ? p->sz.C : h->cfg.S);
+  info->n_batches = p->n_b;
+  info->n_nodes = p->n_slots;
+  info->n_halvings = (int)p->trace.size();
+  info->trace_words = p->trace_words;
+  info->coreset_idx_elems = p->coreset_idx_elems;
+  info->workspace_bytes = p->bytes;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_reserve(thin_attn_t h, int causal, int g) {
+  if (!h) return fail(THIN_ATTN_EINVAL, "null handle");
+  std::lock_guard<std::mutex> lk(h->mu);
+  DeviceGuard dg(h->cfg.device);
+  Plan* p = nullptr;
+  thin_attn_status s = get_plan(h, causal, g, &p);
+  if (s != THIN_ATTN_OK) return s;
+  return materialise(h, p);
+}
+
+thin_attn_status thin_attn_trace_layout(thin_attn_t h, int causal, int g, thin_attn_trace_entry* entries,
+                                        size_t capacity, size_t* count) {
+  if (!h || !count) return fail(THIN_ATTN_EINVAL, "null argument");
+  std::lock_guard<std::mutex> lk(h->mu);
+  Plan* p = nullptr;
+  thin_attn_status s = get_plan(h, causal, g, &p);
+  if (s != THIN_ATTN_OK) return s;
+  *count = p->trace.size();
+  if (entries)
+    std::memcpy(entries, p->trace.data(), std::min(capacity, p->trace.size()) * sizeof(thin_attn_trace_entry));
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_forward(thin_attn_t h, const void* q, const void* k, const void* v, void* out,
+                                   int causal, int g, uint64_t seed, float* lse_opt, int32_t* coreset_idx_opt,
+                                   uint32_t* trace_opt, void* stream) {
+  if (!h) return fail(THIN_ATTN_EINVAL, "null handle");
+  if (!q || !k || !v || !out) return fail(THIN_ATTN_EINVAL, "q, k, v and out must be non-null");
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (((uintptr_t)ptr) % 16) return fail(THIN_ATTN_EINVAL, "tensor pointers must be 16-byte aligned");
+  std::lock_guard<std::mutex> lk(h->mu);
+  DeviceGuard dg(h->cfg.device);
+  if (!dg.ok) return fail(THIN_ATTN_ECUDA, "cannot select device %d", h->cfg.device);
+  Plan* p = nullptr;
+  thin_attn_status s = get_plan(h, causal, g, &p);
+  if (s != THIN_ATTN_OK) return s;
+  s = materialise(h, p);
+  if (s != THIN_ATTN_OK) return s;
+  return run_forward(h, p, q, k, v, out, seed, lse_opt, coreset_idx_opt, trace_opt, (cudaStream_t)stream);
+}
+
+thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void* k, const void* v, void* out,
+                                        int causal, int g, uint64_t seed, float* lse_opt, void* stream) {
+  if (!h) return fail(THIN_ATTN_EINVAL, "null handle");
+  if (!q || !k || !v || !out) return fail(THIN_ATTN_EINVAL, "q, k, v and out must be non-null");
+  const thin_attn_config& c = h->cfg;
+  const size_t es = elt(c);
+  const int64_t L = causal ? c.T : c.S;
+  const size_t qb = (size_t)c.B * c.T * c.H * c.E * es, kb = (size_t)c.B * L * c.H * c.E * es,
+               vb = (size_t)c.B * L * c.H * c.D * es, ob = (size_t)c.B * c.T * c.H * c.D * es,
+               lb = (size_t)c.B * c.H * c.T * 4;
+  const size_t need = align256(qb) + align256(kb) + align256(vb) + align256(ob) + align256(lb);
+  cudaStream_t st = (cudaStream_t)stream;
+  {
+    std::lock_guard<std::mutex> lk(h->mu);
+    DeviceGuard dg(c.device);
+    if (h->st_bytes < need) {
+      if (h->st_mem) cudaFree(h->st_mem);
+      h->st_mem = nullptr;
+      h->st_bytes = 0;
+      if (cudaMalloc(&h->st_mem, need) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(THIN_ATTN_ENOMEM, "host-path staging of %zu bytes", need);
+      }
+      h->st_bytes = need;
+    }
+  }
+  char* base = (char*)h->st_mem;
+  char *dq = base, *dk = dq + align256(qb), *dv = dk + align256(kb), *dout = dv + align256(vb),
+       *dl = dout + align256(ob);
+  {
+    DeviceGuard dg(c.device);
+    CK(cudaMemcpyAsync(dq, q, qb, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(dk, k, kb, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(dv, v, vb, cudaMemcpyHostToDevice, st));
+  }
+  thin_attn_status s = thin_attn_forward(h, dq, dk, dv, dout, causal, g, seed, lse_opt ? (float*)dl : nullptr,
+                                         nullptr, nullptr, stream);
+  if (s != THIN_ATTN_OK) return s;
+  DeviceGuard dg(c.device);
+  CK(cudaMemcpyAsync(out, dout, ob, cudaMemcpyDeviceToHost, st));
+  if (lse_opt) CK(cudaMemcpyAsync(lse_opt, dl, lb, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_check(thin_attn_t h, void* stream) {
+  if (!h) return fail(THIN_ATTN_EINVAL, "null handle");
+  DeviceGuard dg(h->cfg.device);
+  CK(cudaStreamSynchronize((cudaStream_t)stream));
+  if (!h->d_status) return THIN_ATTN_OK;
+  int st[4] = {0, 0, 0, 0};
+  CK(cudaMemcpy(st, h->d_status, sizeof st, cudaMemcpyDeviceToHost));
+  if (st[0] != 0) {
+    CK(cudaMemset(h->d_status, 0, 16));
+    return fail(THIN_ATTN_ETIMEOUT, "device wait gave up (code %d, where %d)", st[0], st[1]);
+  }
+  return THIN_ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,293 @@
+// Kernel Halving on the GPU: one "step" halves n_inst independent instances of n points.
+//
+// The walk is the self-balancing walk of Kernel Halving (Dwivedi & Mackey,
+// "Kernel Thinning"), run on the key-value attention kernel kappa_att that the
+// "Express Language Modeling" summary names for Thinformer Express:
+//   kappa((k,v),(k',v')) = exp(s <k,k'>) (<v,v'> + c^2),  c = max |v| of the instance.
+//
+// A step is three launches:
+//   1. c2_kernel        c^2 of every instance
+//   2. pairgram kernel   pair-difference matrix Delta[j][i] = k(x_j,x_i) - k(y_j,x_i)
+//                        - k(x_j,y_i) + k(y_j,y_i) for j <= i (upper triangle, 32x32 pair
+//                        tiles; Delta[i][i] = b_i^2)
+//   3. walk_kernel       the sequential decisions, then the gather of the survivors
+//
+// The decision for pair i keeps its first point iff alpha_i < a_i (1 - 2 u_i), which
+// is u_i < clip((1 - alpha_i/a_i)/2, 0, 1) rearranged (a_i > 0).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace thin {
+
+// ---------------------------------------------------------------------------
+// 1. c^2 = (max |v|)^2 over the instance's points
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) c2_kernel(StepArgs a) {
+  const int inst = blockIdx.x;
+  const HalveInst in = a.inst[inst];
+  __shared__ uint32_t U_s;
+  __shared__ float red[4];
+  if (threadIdx.x == 0) U_s = sub_offset(a, in);
+  __syncthreads();
+  const T* V = (const T*)a.srcV;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float mx = 0.f;
+  for (int p = warp; p < a.n; p += 4) {
+    const PointRef r = point_ref(a, in, p, U_s);
+    for (int d = lane; d < a.D; d += 32) mx = fmaxf(mx, fabsf(to_f(V[r.vrow + d])));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const float v = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    a.c2[inst] = v * v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. pair-difference Gram, CUDA-core version (fp32 inputs, and any bf16 shape)
+//    CTA = one 32x32 tile of Delta = one 64x64 tile of the point Gram.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) pairgram_simt_kernel(StepArgs a) {
+  const int inst = blockIdx.x;
+  const int nb = a.m_pad >> 5;
+  int t = blockIdx.y, tj = 0;
+  while (t >= nb - tj) {
+    t -= nb - tj;
+    ++tj;
+  }
+  const int ti = tj + t;
+  const HalveInst in = a.inst[inst];
+
+  __shared__ float As[64][33];
+  __shared__ float Bs[64][33];
+  __shared__ int64_t rK[64], rV[64], cK[64], cV[64];
+  __shared__ uint32_t U_s;
+  if (threadIdx.x == 0) U_s = sub_offset(a, in);
+  __syncthreads();
+  if (threadIdx.x < 128) {
+    const int which = threadIdx.x >> 6, r = threadIdx.x & 63;
+    const int p = (which ? ti : tj) * 64 + r;
+    int64_t ko = -1, vo = -1;
+    if (p < a.n) {
+      const PointRef pr = point_ref(a, in, p, U_s);
+      ko = pr.krow;
+      vo = pr.vrow;
+    }
+    if (which) { cK[r] = ko; cV[r] = vo; } else { rK[r] = ko; rV[r] = vo; }
+  }
+  __syncthreads();
+
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  float kk[4][4], vv[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) kk[i][j] = vv[i][j] = 0.f;
+
+  for (int part = 0; part < 2; ++part) {
+    const T* X = (const T*)(part ? a.srcV : a.srcK);
+    const int W = part ? a.D : a.E;
+    const int64_t* ro = part ? rV : rK;
+    const int64_t* co = part ? cV : cK;
+    for (int d0 = 0; d0 < W; d0 += 32) {
+      for (int e = threadIdx.x; e < 64 * 32; e += 256) {
+        const int r = e >> 5, c = e & 31;
+        const bool okc = d0 + c < W;
+        As[r][c] = (ro[r] >= 0 && okc) ? to_f(X[ro[r] + d0 + c]) : 0.f;
+        Bs[r][c] = (co[r] >= 0 && okc) ? to_f(X[co[r] + d0 + c]) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int c = 0; c < 32; ++c) {
+        float av[4], bv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) av[i] = As[ty * 4 + i][c];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bv[j] = Bs[tx * 4 + j][c];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (part) vv[i][j] = fmaf(av[i], bv[j], vv[i][j]);
+            else kk[i][j] = fmaf(av[i], bv[j], kk[i][j]);
+          }
+      }
+      __syncthreads();
+    }
+  }
+  const float c2 = a.c2[inst];
+  float kap[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) kap[i][j] = exp2f(kk[i][j] * a.scale_log2e) * (vv[i][j] + c2);
+  float* Dl = a.delta + (size_t)inst * a.m_pad * a.m_pad;
+#pragma unroll
+  for (int pa = 0; pa < 2; ++pa)
+#pragma unroll
+    for (int pb = 0; pb < 2; ++pb) {
+      const int pj = tj * 32 + ty * 2 + pa, pi = ti * 32 + tx * 2 + pb;
+      const float d = kap[2 * pa][2 * pb] - kap[2 * pa + 1][2 * pb] - kap[2 * pa][2 * pb + 1] +
+                      kap[2 * pa + 1][2 * pb + 1];
+      if (pj < a.m && pi < a.m) Dl[(size_t)pj * a.m_pad + pi] = d;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3. the walk and the gather.  CTA = one instance, 128 threads.
+//    Pairs are taken in blocks of 32: warp 0 runs the 32 dependent decisions
+//    of a block from its diagonal Delta tile (lane l holds alpha of pair 32t+l),
+//    then all threads add the block's contribution eta_s Delta[32t+s][k] to the
+//    alpha of every later pair k.  alpha_i therefore accumulates its terms in
+//    pair order j = 0, 1, ..., i-1.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) walk_kernel(StepArgs a) {
+  extern __shared__ float sm[];
+  const int inst = blockIdx.x;
+  const HalveInst in = a.inst[inst];
+  const int m = a.m, mp = a.m_pad, nb = mp >> 5;
+  float* alpha = sm;                              // mp
+  float* ubuf = alpha + mp;                       // mp
+  float* tile = ubuf + mp;                        // 32 x 33
+  uint32_t* bits = (uint32_t*)(tile + 32 * 33);   // nb
+  __shared__ uint32_t U_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* Dl = a.delta + (size_t)inst * mp * mp;
+
+  for (int i = tid; i < mp; i += 128) {
+    alpha[i] = 0.f;
+    ubuf[i] = i < m ? philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)i) : 0.5f;
+  }
+  if (tid == 0) U_s = sub_offset(a, in);
+  float sig2 = 0.f;
+  for (int t = 0; t < nb; ++t) {
+    const int base = t * 32;
+    __syncthreads();
+    for (int e = tid; e < 1024; e += 128) {
+      const int r = e >> 5, c = e & 31;
+      tile[r * 33 + c] = (base + r < m && base + c < m) ? Dl[(size_t)(base + r) * mp + base + c] : 0.f;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      float my = alpha[base + lane];
+      uint32_t kb = 0;
+      const int steps = min(32, m - base);
+      for (int s = 0; s < steps; ++s) {
+        const float ai = __shfl_sync(0xffffffffu, my, s);
+        const float b2 = tile[s * 33 + s];
+        bool keep = true;
+        if (b2 > 0.f) {
+          const float b = sqrtf(b2);
+          const float av = fmaxf(b * sqrtf(sig2) * a.C, b2);
+          keep = ai < av * (1.f - 2.f * ubuf[base + s]);
+          sig2 = sig2 + b2 * fmaxf(0.f, 1.f + (b2 - 2.f * av) * sig2 / (av * av));
+        }
+        if (lane > s) my = fmaf(keep ? 1.f : -1.f, tile[s * 33 + lane], my);
+        kb |= (uint32_t)keep << s;
+      }
+      if (lane == 0) bits[t] = kb;
+    }
+    __syncthreads();
+    const uint32_t kb = bits[t];
+    const int steps = min(32, m - base);
+    for (int k = base + 32 + tid; k < m; k += 128) {
+      float acc = alpha[k];
+      for (int s = 0; s < steps; ++s)
+        acc = fmaf(((kb >> s) & 1u) ? 1.f : -1.f, Dl[(size_t)(base + s) * mp + k], acc);
+      alpha[k] = acc;
+    }
+  }
+  __syncthreads();
+  if (a.trace)
+    for (int w = tid; w < nb; w += 128) a.trace[a.trace_base + (size_t)inst * nb + w] = bits[w];
+
+  // gather the kept point of every pair into row i of the destination
+  const int kw = a.E * (int)sizeof(T) / 16, vw = a.D * (int)sizeof(T) / 16;
+  const uint4* K = (const uint4*)a.srcK;
+  const uint4* V = (const uint4*)a.srcV;
+  uint4* dK = (uint4*)a.dstK;
+  uint4* dV = (uint4*)a.dstV;
+  const int epw = 16 / (int)sizeof(T);
+  for (int i = warp; i < m; i += 4) {
+    const bool keep = (bits[i >> 5] >> (i & 31)) & 1u;
+    const PointRef r = point_ref(a, in, 2 * i + (keep ? 0 : 1), U_s);
+    const int64_t drow = in.dst_row + i;
+    for (int w = lane; w < kw; w += 32) dK[drow * kw + w] = K[r.krow / epw + w];
+    for (int w = lane; w < vw; w += 32) dV[drow * vw + w] = V[r.vrow / epw + w];
+    if (lane == 0) a.dstIdx[drow] = r.idx;
+  }
+}
+
+// Copy runs of tokens unchanged into compact rows (Express batches that need no thinning).
+template <typename T>
+__global__ void copy_tokens_kernel(StepArgs a) {
+  const int inst = blockIdx.x;
+  const HalveInst in = a.inst[inst];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kw = a.E * (int)sizeof(T) / 16, vw = a.D * (int)sizeof(T) / 16;
+  const int epw = 16 / (int)sizeof(T);
+  const uint4* K = (const uint4*)a.srcK;
+  const uint4* V = (const uint4*)a.srcV;
+  uint4* dK = (uint4*)a.dstK;
+  uint4* dV = (uint4*)a.dstV;
+  for (int p = warp; p < a.n; p += blockDim.x / 32) {
+    const PointRef r = point_ref(a, in, p, 0u);
+    const int64_t drow = in.dst_row + p;
+    for (int w = lane; w < kw; w += 32) dK[drow * kw + w] = K[r.krow / epw + w];
+    for (int w = lane; w < vw; w += 32) dV[drow * vw + w] = V[r.vrow / epw + w];
+    if (lane == 0) a.dstIdx[drow] = r.idx;
+  }
+}
+
+__global__ void iota_kernel(int32_t* idx, int64_t rows, int period) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i < rows) idx[i] = (int32_t)(i % period);
+}
+
+size_t walk_smem_bytes(int m_pad) { return (size_t)(2 * m_pad + 32 * 33 + m_pad / 32) * 4; }
+
+template <typename T>
+static cudaError_t launch_step_t(const StepArgs& a, bool use_tc, cudaStream_t st) {
+  if (a.n_inst == 0) return cudaSuccess;
+  c2_kernel<T><<<a.n_inst, 128, 0, st>>>(a);
+  const int nb = a.m_pad / 32;
+  const int ntri = nb * (nb + 1) / 2;
+  bool done = false;
+  if (use_tc) {
+    cudaError_t e = launch_pairgram_tc(a, st, &done);
+    if (e != cudaSuccess) return e;
+  }
+  if (!done) pairgram_simt_kernel<T><<<dim3(a.n_inst, ntri), 256, 0, st>>>(a);
+  const size_t sm = walk_smem_bytes(a.m_pad);
+  if (sm > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(walk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+  }
+  walk_kernel<T><<<a.n_inst, 128, sm, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_halving_step(const StepArgs& a, int dtype, bool use_tc, cudaStream_t st) {
+  return dtype == 0 ? launch_step_t<float>(a, false, st) : launch_step_t<__nv_bfloat16>(a, use_tc, st);
+}
+
+cudaError_t launch_copy_step(const StepArgs& a, int dtype, cudaStream_t st) {
+  if (a.n_inst == 0) return cudaSuccess;
+  if (dtype == 0) copy_tokens_kernel<float><<<a.n_inst, 128, 0, st>>>(a);
+  else copy_tokens_kernel<__nv_bfloat16><<<a.n_inst, 128, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_iota(int32_t* idx, int64_t rows, int period, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  iota_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(idx, rows, period);
+  return cudaGetLastError();
+}
+
+}  // namespace thin

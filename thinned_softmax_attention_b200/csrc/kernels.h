@@ -1,0 +1,28 @@
+// Kernel launchers of the thin_attn library (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace thin {
+
+// Halving step (c^2, pair-difference Gram, walk + gather).  dtype 0 = fp32, 1 = bf16.
+cudaError_t launch_halving_step(const StepArgs& a, int dtype, bool use_tc, cudaStream_t st);
+// Tensor-core pair-difference Gram (bf16, E and D multiples of 64); *done = false when the
+// shape is not covered and the CUDA-core kernel must run instead.
+cudaError_t launch_pairgram_tc(const StepArgs& a, cudaStream_t st, bool* done);
+// Copy of token runs into compact rows (batches that are not thinned).
+cudaError_t launch_copy_step(const StepArgs& a, int dtype, cudaStream_t st);
+cudaError_t launch_iota(int32_t* idx, int64_t rows, int period, cudaStream_t st);
+size_t walk_smem_bytes(int m_pad);
+
+// Attention over key segments.
+cudaError_t launch_attention_simt(const AttnArgs& a, int dtype, cudaStream_t st);
+int attention_simt_tile_rows();
+// Tensor-core attention (bf16, E = D = 128); *done = false when the shape is not covered.
+cudaError_t launch_attention_tc(const AttnArgs& a, int* status_word, cudaStream_t st, bool* done);
+int attention_tc_tile_rows();
+bool attention_tc_supported(int dtype, int E, int D);
+
+}  // namespace thin
