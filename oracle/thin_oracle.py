@@ -406,7 +406,7 @@ def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, head
     trace: Trace = {}
     stats = Stats()
     nodes: Dict[Tuple[int, int], np.ndarray] = {}     # (level, j) -> (n_bh, c) token indices
-    c = compress_sizes(bsz, g)[3] if n_b else 0
+    c = compress_sizes(bsz, g)[3] if bsz > 0 else 0
     # thin phase: every batch compressed independently (batch k depends on its tokens only)
     if n_b:
         Kb = Kall[:, n_e:n_e + n_b * bsz].reshape(n_bh * n_b, bsz, E)
@@ -468,7 +468,7 @@ def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, head
             out[b, sel, h] = o
             lse[b, h, sel] = l
     coreset = (np.stack([nodes[s] for s in slots], axis=1).reshape(B, H, len(slots), c)
-               if slots else np.zeros((B, H, 0, 0), dtype=np.int64))
+               if slots else np.zeros((B, H, 0, c), dtype=np.int64))
     wts = np.array([weight[s] for s in slots]) if slots else np.zeros(0)
     return OracleOut(out, lse, coreset, trace, stats, wts)
 
