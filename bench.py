@@ -1,0 +1,338 @@
+#!/usr/bin/env python
+"""Throughput of Thinformer Express prefill on B200 through the thin_attn C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl thin|reference] [--workload NAME]
+
+One step = one thin_attn_forward of the whole path (batch thinning, HALVE
+merges, attention) over the workload (default: express32k, B=1 H=32 T=32768
+E=D=128 bf16, exact phase 1024, thin batch 1024, g=2) with q, k, v resident in
+HBM.  Prints one JSON line on rank 0.  Multi-GPU (torchrun): every rank runs
+its own independent problem of the same size (weak scaling, no collective on
+the data path); step time is the max over ranks of CUDA-event time.
+
+--impl reference times the fp64 CPU oracle on the host cores (rank 0 only),
+each step one head of the workload.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "attention tokens/s (B·H·T) and ms/layer at S=32K causal; % of roofline"
+UNIT = "tokens/s"
+
+
+def args_():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="thin", choices=["thin", "reference"])
+    p.add_argument("--workload", default="express32k", choices=sorted(W.WORKLOADS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-sdpa", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def digitsum4(k):
+    k = np.asarray(k, dtype=np.int64).copy()
+    s = np.zeros_like(k)
+    while np.any(k):
+        s += k % 4
+        k //= 4
+    return s
+
+
+def attention_work(w, plan):
+    """Algorithmic FLOPs and HBM bytes of one attention launch.
+
+    FLOPs: 2 (E + D) per visible (query, key) pair.  Bytes: q read and out written
+    once, plus every distinct key/value row read once (original tokens and coreset rows)."""
+    BH = w.B * w.H
+    es = 4 if w.dtype == "fp32" else 2
+    if not w.causal:
+        keys = plan["coreset_rows"] if plan["levels"] > 0 else w.S
+        pairs = w.T * keys
+        kv_rows = keys
+    else:
+        t = np.arange(w.T, dtype=np.int64)
+        ne, b, c = min(w.n_exact, w.T), w.batch, plan["coreset_rows"]
+        k = np.maximum(t - ne, 0) // b
+        vis = np.where(t < ne, t + 1, ne + c * digitsum4(k) + (t - (ne + k * b) + 1))
+        pairs = int(vis.sum())
+        kv_rows = w.T + plan["n_nodes"] * c
+    flops = 2.0 * (w.E + w.D) * pairs * BH
+    bytes_ = es * BH * (w.T * (w.E + w.D) + kv_rows * (w.E + w.D))
+    return flops, bytes_, pairs
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons while the timed region runs."""
+
+    def __init__(self, index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        self.p.wait()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows if len(r) >= 9 for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(w, seed_heads, budget_s=12.0, max_heads=8):
+    """The fp64 oracle, as it stands, on a bounded sample: whole heads of the workload."""
+    from oracle import express, thinformer
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    done, t_total = 0, 0.0
+    for h in seed_heads[:max_heads]:
+        q, k, v = W.make_qkv(w.with_(B=1), heads=[h])
+        t0 = time.perf_counter()
+        if w.causal:
+            express(q, k, v, w.n_exact, w.batch, w.g, w.seed, heads=(w.H, [h]))
+        else:
+            thinformer(q, k, v, w.g, w.seed, heads=(w.H, [h]))
+        t_total += time.perf_counter() - t0
+        done += 1
+        if t_total >= budget_s:
+            break
+    return {"value": done * w.T / t_total, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {w.B * w.H} (b,h) slices, all {w.T} queries each: thinning + attention in fp64 numpy",
+            "seconds": round(t_total, 3)}
+
+
+def kernel_traffic(name):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(name)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["sha256"]:
+        return None
+    return d["bytes_per_launch"]
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = W.WORKLOADS[a.workload]
+    from oracle import express, thinformer
+    heads = list(range(w.H)) * (1 + (a.steps + a.warmup) // max(1, w.H))
+    times = []
+    for i in range(a.warmup + a.steps):
+        h = heads[i]
+        q, k, v = W.make_qkv(w.with_(B=1), heads=[h])
+        t0 = time.perf_counter()
+        if w.causal:
+            express(q, k, v, w.n_exact, w.batch, w.g, w.seed, heads=(w.H, [h]))
+        else:
+            thinformer(q, k, v, w.g, w.seed, heads=(w.H, [h]))
+        if i >= a.warmup:
+            times.append(time.perf_counter() - t0)
+    per = sum(times) / len(times)
+    value = w.T / per
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": config_of(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"one (b,h) slice per step ({w.T} queries, thinning + attention)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "S": w.T if w.causal else w.S, "E": w.E, "D": w.D,
+            "causal": w.causal, "g": w.g, "n_exact": w.n_exact, "batch": w.batch, "seed": w.seed,
+            "l2": "inputs larger than L2 (no flush)" if 3 * w.B * w.H * w.T * w.E * 2 > 126e6 else
+            "inputs smaller than L2"}
+
+
+def main():
+    a = args_()
+    if a.impl == "reference":
+        return run_reference(a)
+    import thinned_softmax_attention_b200 as TA
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    w = W.WORKLOADS[a.workload]
+    # each rank an independent problem of the same size (weak scaling)
+    wr = w.with_(data_seed=w.data_seed + 1000 * rank) if rank else w
+    q, k, v = (x.to(dev) for x in W.make_qkv(wr))
+    S = w.T if w.causal else w.S
+    h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch,
+                         device=local)
+    plan = h.plan(w.causal, w.g)
+    h.reserve(w.causal, w.g)
+    out = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype, device=dev)
+
+    def step():
+        h.forward(q, k, v, causal=w.causal, g=w.g, seed=w.seed, out=out)
+
+    for _ in range(max(3, a.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = Clocks(local)
+    h.profile(True)
+    h.profile_read()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(a.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    h.profile(False)
+    ph = h.profile_read()
+    ms = e0.elapsed_time(e1) / a.steps
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = w.B * w.H * w.T
+    value = world * tokens / (ms * 1e-3)
+
+    # dominant kernel roofline: attention
+    pk = peaks()
+    flops, abytes, pairs = attention_work(w, plan)
+    attn_ms = ph["attn_ms"] / max(1, ph["calls"])
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    peak = pk["bf16_tflops_sustained"]
+    roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": kernel_traffic("attention"),
+            "kernel": "attention", "peak_kind": f"bf16 sustained ({pk['source']})",
+            "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
+            "avg_launch_ms": round(attn_ms, 4)}
+    phases = {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
+              "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4),
+              "attn_ms": round(attn_ms, 4)}
+
+    e2e = None
+    if not a.no_e2e:
+        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        oh = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype).pin_memory()
+        for _ in range(2):
+            h.forward_host(qh, kh, vh, oh, causal=w.causal, g=w.g, seed=w.seed)
+        n_e2e = max(2, min(a.steps, 5))
+        if dist:
+            dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(n_e2e):
+            h.forward_host(qh, kh, vh, oh, causal=w.causal, g=w.g, seed=w.seed)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ems = f0.elapsed_time(f1) / n_e2e
+        if dist:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        es = 4 if w.dtype == "fp32" else 2
+        e2e = {"value": world * tokens / (ems * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * es,
+               "d2h_bytes_per_step": out.numel() * es, "ms_per_step": round(ems, 3)}
+
+    sdpa = None
+    if not a.no_sdpa and rank == 0:
+        try:
+            qt, kt, vt = (x.transpose(1, 2) for x in (q, k, v))
+            F = torch.nn.functional.scaled_dot_product_attention
+            for _ in range(2):
+                F(qt, kt, vt, is_causal=w.causal)
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(3):
+                F(qt, kt, vt, is_causal=w.causal)
+            s1.record(stream)
+            torch.cuda.synchronize()
+            sdpa = round(s0.elapsed_time(s1) / 3, 4)
+        except Exception as ex:  # report, do not fail the bench
+            sdpa = f"unavailable: {type(ex).__name__}"
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(w, list(range(w.H)))
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
+            "ms_per_layer": ms, "phases_ms": phases, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": plan["kernel_launches"] * a.steps, "clocks": clk, "exact_sdpa_ms": sdpa,
+            "workspace_bytes": plan["workspace_bytes"]}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -79,7 +79,7 @@ typedef struct {
   int n_batches;               /* causal: completed thin batches n_b */
   int n_nodes;                 /* causal: node slots (level-0 nodes, then level 1, ...) */
   int n_halvings;              /* halving instances (entries of the trace layout) */
-  int reserved;
+  int kernel_launches;         /* kernels one forward launches (without the optional outputs) */
   uint64_t trace_words;        /* uint32 words of the decision trace */
   uint64_t coreset_idx_elems;  /* int32 elements of coreset_idx_opt */
   uint64_t workspace_bytes;    /* device workspace the plan needs */
@@ -144,6 +144,16 @@ THIN_ATTN_API thin_attn_status thin_attn_forward(thin_attn_t h, const void* q, c
 THIN_ATTN_API thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void* k,
                                         const void* v, void* out, int causal, int g,
                                         uint64_t seed, float* lse_opt, void* stream);
+
+/* Per-phase device timing: when enabled, every forward records CUDA events on its
+ * stream between its phases (thinning of sequences or batches, HALVE merges,
+ * attention).  No effect on results. */
+THIN_ATTN_API thin_attn_status thin_attn_profile(thin_attn_t h, int enable);
+
+/* Wait for the recorded forwards and return their summed phase times in
+ * milliseconds: ms[0] thinning, ms[1] merges, ms[2] attention, ms[3] total;
+ * *calls = forwards recorded.  Resets the sums. */
+THIN_ATTN_API thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms, int* calls);
 
 /* Synchronise `stream` and report a device-side failure recorded by the
  * handle's kernels since the last call (THIN_ATTN_ETIMEOUT, ...). */

@@ -42,7 +42,7 @@ class Config(ctypes.Structure):
 class PlanInfo(ctypes.Structure):
     _fields_ = [("levels", ctypes.c_int), ("leaf", ctypes.c_int), ("subsampled", ctypes.c_int),
                 ("coreset_rows", ctypes.c_int), ("n_batches", ctypes.c_int), ("n_nodes", ctypes.c_int),
-                ("n_halvings", ctypes.c_int), ("reserved", ctypes.c_int), ("trace_words", ctypes.c_uint64),
+                ("n_halvings", ctypes.c_int), ("kernel_launches", ctypes.c_int), ("trace_words", ctypes.c_uint64),
                 ("coreset_idx_elems", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64)]
 
 
@@ -54,7 +54,7 @@ class TraceEntry(ctypes.Structure):
 _lib = None
 EXPORTS = ("thin_attn_version", "thin_attn_last_error", "thin_attn_create", "thin_attn_destroy",
            "thin_attn_plan", "thin_attn_reserve", "thin_attn_trace_layout", "thin_attn_forward",
-           "thin_attn_forward_host", "thin_attn_check")
+           "thin_attn_forward_host", "thin_attn_check", "thin_attn_profile", "thin_attn_profile_read")
 
 
 def lib() -> ctypes.CDLL:
@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
     L.thin_attn_forward.argtypes = [vp, vp, vp, vp, vp, i, i, u64, vp, vp, vp, vp]
     L.thin_attn_forward_host.argtypes = [vp, vp, vp, vp, vp, i, i, u64, vp, vp]
     L.thin_attn_check.argtypes = [vp, vp]
+    L.thin_attn_profile.argtypes = [vp, i]
+    L.thin_attn_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
     for f in EXPORTS[2:]:
         getattr(L, f).restype = ctypes.c_int
     _lib = L
@@ -181,6 +183,17 @@ class ThinAttention:
                                             ctypes.c_uint64(seed & (2 ** 64 - 1)), _ptr(lse),
                                             ctypes.c_void_p(stream)))
         return out
+
+    def profile(self, enable: bool = True):
+        """Record per-phase CUDA events on every forward (thinning, merges, attention)."""
+        _check(lib().thin_attn_profile(self._h, int(enable)))
+
+    def profile_read(self):
+        """Summed phase times (ms) of the forwards recorded since the last read, and their count."""
+        ms = (ctypes.c_double * 4)()
+        calls = ctypes.c_int()
+        _check(lib().thin_attn_profile_read(self._h, ms, ctypes.byref(calls)))
+        return {"thin_ms": ms[0], "merge_ms": ms[1], "attn_ms": ms[2], "total_ms": ms[3], "calls": calls.value}
 
     def check(self):
         stream = torch.cuda.current_stream(self.device).cuda_stream

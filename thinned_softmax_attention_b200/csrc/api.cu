@@ -78,6 +78,7 @@ struct BufSpec {
 
 struct StepPlan {
   bool copy_only = false;
+  int phase = 0;   // 0: thinning of sequences / batches, 1: HALVE merges
   int src_buf = BUF_TOKENS, dst_buf = 0;
   int n = 0, m = 0, m_pad = 0;
   int S_full = 0, S_sub = 0;
@@ -123,6 +124,11 @@ struct thin_attn_s {
   // host-buffer staging
   void* st_mem = nullptr;
   size_t st_bytes = 0;
+  // per-phase device timing (thin_attn_profile)
+  bool prof_on = false;
+  std::vector<std::vector<cudaEvent_t>> prof_pending, prof_free;
+  double prof_ms[3] = {0, 0, 0};
+  int prof_calls = 0;
 };
 
 namespace {
@@ -326,6 +332,7 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
         const int nj = p->n_b >> (2 * lv);
         for (int step = 0; step < 2; ++step) {
           StepPlan st;
+          st.phase = 1;
           st.n = (step == 0 ? 4 : 2) * p->c;
           st.m = st.n / 2;
           st.m_pad = (st.m + 31) / 32 * 32;
@@ -499,7 +506,23 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
                              uint64_t seed, float* lse, int32_t* cidx, uint32_t* trace, cudaStream_t st) {
   const thin_attn_config& cf = h->cfg;
   const bool use_tc_gram = std::getenv("THIN_ATTN_SIMT_GRAM") == nullptr;
+  std::vector<cudaEvent_t> ev;
+  if (h->prof_on) {
+    if (!h->prof_free.empty()) {
+      ev = h->prof_free.back();
+      h->prof_free.pop_back();
+    } else {
+      ev.resize(4);
+      for (auto& e : ev) CK(cudaEventCreate(&e));
+    }
+    CK(cudaEventRecord(ev[0], st));
+  }
+  bool merged_mark = false;
   for (auto& sp : p->steps) {
+    if (!ev.empty() && sp.phase == 1 && !merged_mark) {
+      CK(cudaEventRecord(ev[1], st));
+      merged_mark = true;
+    }
     StepArgs a{};
     const void *sk, *sv;
     int32_t* sidx;
@@ -534,6 +557,10 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     cudaError_t e = sp.copy_only ? launch_copy_step(a, cf.dtype, st)
                                  : launch_halving_step(a, cf.dtype, use_tc_gram, st);
     if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "halving step (n=%d): %s", sp.n, cudaGetErrorString(e));
+  }
+  if (!ev.empty()) {
+    if (!merged_mark) CK(cudaEventRecord(ev[1], st));
+    CK(cudaEventRecord(ev[2], st));
   }
   if (cidx) {
     if (p->final_buf == BUF_TOKENS) {
@@ -580,6 +607,10 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     cudaError_t e = launch_attention_simt(aa, cf.dtype, st);
     if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "attention: %s", cudaGetErrorString(e));
   }
+  if (!ev.empty()) {
+    CK(cudaEventRecord(ev[3], st));
+    h->prof_pending.push_back(ev);
+  }
   return THIN_ATTN_OK;
 }
 
@@ -605,7 +636,7 @@ thin_attn_status thin_attn_create(thin_attn_t* out, const thin_attn_config* cfg)
 
 thin_attn_status thin_attn_destroy(thin_attn_t h) {
   if (!h) return THIN_ATTN_OK;
-  const bool on_device = h->d_status || h->st_mem;
+  const bool on_device = h->d_status || h->st_mem || !h->prof_free.empty() || !h->prof_pending.empty();
   DeviceGuard dg(on_device ? h->cfg.device : -1);
   for (auto& kv : h->plans) {
     if (kv.second->d_mem) cudaFree(kv.second->d_mem);
@@ -613,6 +644,9 @@ thin_attn_status thin_attn_destroy(thin_attn_t h) {
   }
   if (h->d_status) cudaFree(h->d_status);
   if (h->st_mem) cudaFree(h->st_mem);
+  for (auto* lst : {&h->prof_pending, &h->prof_free})
+    for (auto& ev : *lst)
+      for (auto e : ev) cudaEventDestroy(e);
   delete h;
   return THIN_ATTN_OK;
 }
@@ -631,6 +665,9 @@ thin_attn_status thin_attn_plan(thin_attn_t h, int causal, int g, thin_attn_plan
   info->n_batches = p->n_b;
   info->n_nodes = p->n_slots;
   info->n_halvings = (int)p->trace.size();
+  int launches = 1;
+  for (auto& st : p->steps) launches += st.inst.empty() ? 0 : (st.copy_only ? 1 : 3);
+  info->kernel_launches = launches;
   info->trace_words = p->trace_words;
   info->coreset_idx_elems = p->coreset_idx_elems;
   info->workspace_bytes = p->bytes;
@@ -723,6 +760,36 @@ thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void
   return THIN_ATTN_OK;
 }
 
+thin_attn_status thin_attn_profile(thin_attn_t h, int enable) {
+  if (!h) return fail(THIN_ATTN_EINVAL, "null handle");
+  std::lock_guard<std::mutex> lk(h->mu);
+  h->prof_on = enable != 0;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms, int* calls) {
+  if (!h || !ms || !calls) return fail(THIN_ATTN_EINVAL, "null argument");
+  std::lock_guard<std::mutex> lk(h->mu);
+  DeviceGuard dg(h->prof_pending.empty() ? -1 : h->cfg.device);
+  for (auto& ev : h->prof_pending) {
+    CK(cudaEventSynchronize(ev[3]));
+    float t[3];
+    for (int i = 0; i < 3; ++i) {
+      CK(cudaEventElapsedTime(&t[i], ev[i], ev[i + 1]));
+      h->prof_ms[i] += t[i];
+    }
+    h->prof_calls += 1;
+    h->prof_free.push_back(ev);
+  }
+  h->prof_pending.clear();
+  for (int i = 0; i < 3; ++i) ms[i] = h->prof_ms[i];
+  ms[3] = h->prof_ms[0] + h->prof_ms[1] + h->prof_ms[2];
+  *calls = h->prof_calls;
+  h->prof_ms[0] = h->prof_ms[1] = h->prof_ms[2] = 0;
+  h->prof_calls = 0;
+  return THIN_ATTN_OK;
+}
+
 thin_attn_status thin_attn_check(thin_attn_t h, void* stream) {
   if (!h) return fail(THIN_ATTN_EINVAL, "null handle");
   DeviceGuard dg(h->cfg.device);
@@ -732,7 +799,8 @@ thin_attn_status thin_attn_check(thin_attn_t h, void* stream) {
   CK(cudaMemcpy(st, h->d_status, sizeof st, cudaMemcpyDeviceToHost));
   if (st[0] != 0) {
     CK(cudaMemset(h->d_status, 0, 16));
-    return fail(THIN_ATTN_ETIMEOUT, "device wait gave up (code %d, where %d)", st[0], st[1]);
+    return fail(THIN_ATTN_ETIMEOUT, "device wait gave up (code %d; query tile %d of (b,h) %d; wait %d at key tile %d)",
+                st[0], st[1] >> 16, st[1] & 0xFFFF, st[2] / 1000, st[2] % 1000);
   }
   return THIN_ATTN_OK;
 }

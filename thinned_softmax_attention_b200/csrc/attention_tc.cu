@@ -1,10 +1,430 @@
-// Tensor-core (tcgen05) attention: placeholder until the sm_100a kernel lands.
+// Weighted softmax attention over key segments on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+//   o_t = sum_j w_j e^{s q_t.k_j} v_j / sum_j w_j e^{s q_t.k_j},  lse_t = ln sum_j w_j e^{s q_t.k_j}
+// for a tile of up to 128 queries of one (b,h) against its key segments (exact prefix, Express
+// nodes with weight 4^l b/c, the causal in-batch keys, or a Thinformer coreset with weight S/|C|),
+// in key tiles of 128 rows.
+//
+// CTA = 6 warps:
+//   warps 0-3  softmax: thread i owns query row i (TMEM lane i); reads S from TMEM, writes
+//              P = exp2(z - m) as bf16 into shared memory (128-byte swizzled, K-major),
+//              rescales O in TMEM when its running max grows by more than 2^8, epilogue
+//   warp 4     TMA producer: Q once, then K and V tiles into a 2-stage ring
+//   warp 5     MMA issuer (one thread): S = Q K^T into a double-buffered TMEM tile (cols 0/128),
+//              O += P V into TMEM cols 256..256+D; also owns the TMEM allocation
+// Every wait on an mbarrier is bounded; a CTA that gives up records the failure in the status
+// word and leaves through the normal exit path (TMEM freed, its TMA copies landed).
+#include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
+
 namespace thin {
-bool attention_tc_supported(int, int, int) { return false; }
-int attention_tc_tile_rows() { return 128; }
-cudaError_t launch_attention_tc(const AttnArgs&, int*, cudaStream_t, bool* done) {
-  *done = false;
-  return cudaSuccess;
+
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128;   // queries per tile
+constexpr int BN = 128;   // keys per tile
+constexpr int NSTAGE = 2;
+
+template <int E, int D>
+struct TcLayout {
+  static constexpr int EC = E / 64, DC = D / 64;
+  static constexpr uint32_t Q_BYTES = BM * E * 2;
+  static constexpr uint32_t K_BYTES = BN * E * 2;
+  static constexpr uint32_t V_BYTES = BN * D * 2;
+  static constexpr uint32_t P_BYTES = BM * BN * 2;
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + NSTAGE * K_BYTES;
+  static constexpr uint32_t OFF_P = OFF_V + NSTAGE * V_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
+  static constexpr uint32_t BYTES = OFF_BAR + 256 + 1024;   // barriers + alignment slack
+};
+
+struct TcMaps {
+  CUtensorMap q, k, v, ck, cv;
+};
+
+__device__ __forceinline__ int count_key_tiles(const AttnArgs& a, const AttnTile& t) {
+  int n = 0;
+  for (int s = 0; s < t.nseg; ++s) n += (a.segs[t.seg0 + s].len + BN - 1) / BN;
+  return n;
 }
+
+template <int E, int D>
+__global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a,
+                                                         int* status) {
+  using Lay = TcLayout<E, D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem + Lay::OFF_Q;
+  uint8_t* sK = smem + Lay::OFF_K;
+  uint8_t* sV = smem + Lay::OFF_V;
+  uint8_t* sP = smem + Lay::OFF_P;
+  uint64_t* bars = (uint64_t*)(smem + Lay::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;     // [NSTAGE]
+  uint64_t* kv_empty = bars + 3;    // [NSTAGE]
+  uint64_t* s_full = bars + 5;      // [2]
+  uint64_t* s_free = bars + 7;      // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* pv_done = bars + 10;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  __shared__ volatile int where_s;   // first wait that gave up: code * 1000 + iteration
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile_id = a.n_tiles - 1 - (int)blockIdx.x;   // heaviest (latest) query tiles first
+  const AttnTile tile = a.tiles[tile_id];
+  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int n_kt = count_key_tiles(a, tile);
+
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    where_s = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full + s, 1);
+      mbar_init(s_free + s, 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) tmem_alloc(&tmem_base_s, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort = &abort_s;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_kt > 0) {
+      mbar_expect_tx(q_full, Lay::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < Lay::EC; ++c) tma_load_3d(sQ + c * 16384, &maps.q, q_full, c * 64, h, b * a.T + tile.q0);
+      int it = 0;
+      int last_fill[NSTAGE] = {-1, -1};
+      bool ok = true;
+      for (int si = 0; si < tile.nseg && ok; ++si) {
+        const AttnSeg sg = a.segs[tile.seg0 + si];
+        for (int j0 = 0; j0 < sg.len && ok; j0 += BN, ++it) {
+          const int st = it % NSTAGE;
+          if (it >= NSTAGE && !mbar_wait(kv_empty + st, ((it / NSTAGE) - 1) & 1, abort)) {
+            ok = false;
+            atomicCAS((int*)&where_s, 0, 1000 + min(it, 999));
+            break;
+          }
+          mbar_expect_tx(kv_full + st, Lay::K_BYTES + Lay::V_BYTES);
+          uint8_t* dK = sK + st * Lay::K_BYTES;
+          uint8_t* dV = sV + st * Lay::V_BYTES;
+          if (sg.kind == SEG_TOKENS) {
+            const int row = b * a.L + sg.first + j0;
+#pragma unroll
+            for (int c = 0; c < Lay::EC; ++c) tma_load_3d(dK + c * 16384, &maps.k, kv_full + st, c * 64, h, row);
+#pragma unroll
+            for (int c = 0; c < Lay::DC; ++c) tma_load_3d(dV + c * 16384, &maps.v, kv_full + st, c * 64, h, row);
+          } else {
+            const int row = (bh * a.n_slots + sg.first) * a.slot_rows + j0;
+#pragma unroll
+            for (int c = 0; c < Lay::EC; ++c) tma_load_2d(dK + c * 16384, &maps.ck, kv_full + st, c * 64, row);
+#pragma unroll
+            for (int c = 0; c < Lay::DC; ++c) tma_load_2d(dV + c * 16384, &maps.cv, kv_full + st, c * 64, row);
+          }
+          last_fill[st] = it;
+        }
+      }
+      // never leave with a copy in flight into this CTA's shared memory
+      for (int st = 0; st < NSTAGE; ++st)
+        if (last_fill[st] >= 0) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(kv_full + st, (last_fill[st] / NSTAGE) & 1) && clock64() - t0 < kWaitCycles) {
+          }
+        }
+      {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(q_full, 0) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_kt > 0) {
+      constexpr uint32_t IQK = idesc_bf16(BM, BN, false);
+      constexpr uint32_t IPV = idesc_bf16(BM, D, true);
+      const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV), pa = smem_u32(sP);
+      bool ok = mbar_wait(q_full, 0, abort);
+      auto issue_s = [&](int it) -> bool {
+        const int st = it % NSTAGE, sb = it & 1;
+        if (!mbar_wait(kv_full + st, (it / NSTAGE) & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 3000 + min(it, 999));
+          return false;
+        }
+        if (it >= 2 && !mbar_wait(s_free + sb, ((it >> 1) - 1) & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 4000 + min(it, 999));
+          return false;
+        }
+        tc_fence_after();
+        const uint32_t kb = ka + st * Lay::K_BYTES;
+#pragma unroll
+        for (int k = 0; k < E / 16; ++k) {
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_bf16(tmem + sb * BN, sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024), IQK, k > 0);
+        }
+        umma_commit(s_full + sb);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int it = 0; it < n_kt && ok; ++it) {
+        if (it + 1 < n_kt && !issue_s(it + 1)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(p_full, it & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 5000 + min(it, 999));
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int st = it % NSTAGE;
+        const uint32_t vb = va + st * Lay::V_BYTES;
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k) {
+          const uint32_t aoff = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_bf16(tmem + 256, sw128_desc(pa + aoff, 16, 1024), sw128_desc(vb + k * 2048, 16384, 1024), IPV,
+                    (it > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(kv_empty + st);
+        umma_commit(pv_done);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroup
+    const int row = warp * 32 + lane;
+    const int tq = tile.q0 + row;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    float m_used = -INFINITY, l = 0.f;
+    int it = 0, where = 0;
+    bool ok = true;
+    for (int si = 0; si < tile.nseg && ok; ++si) {
+      const AttnSeg sg = a.segs[tile.seg0 + si];
+      const float lw2 = sg.logw * 1.4426950408889634f;
+      for (int j0 = 0; j0 < sg.len; j0 += BN, ++it) {
+        const int sb = it & 1;
+        if (!warp_wait(s_full + sb, (it >> 1) & 1, abort)) {
+          ok = false;
+          where = 6;
+          break;
+        }
+        tc_fence_after();
+        float z[BN];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) tmem_ld32(tmem + lane_base + sb * BN + c * 32, z + c * 32);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(s_free + sb);
+        // logits in base 2 with the segment's log-weight; masked keys -> -inf
+        const int nvalid = min(BN, sg.len - j0);
+        const int kt0 = sg.first + j0;
+        const bool causal = sg.kind == SEG_TOKENS && sg.causal;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const bool vis = c < nvalid && (!causal || kt0 + c <= tq);
+          z[c] = vis ? fmaf(z[c], a.scale_log2e, lw2) : -INFINITY;
+          mx = fmaxf(mx, z[c]);
+        }
+        // P of the previous tile must be consumed (PV done) before P and O are touched
+        if (it > 0 && !warp_wait(pv_done, (it - 1) & 1, abort)) {
+          ok = false;
+          where = 7;
+          break;
+        }
+        tc_fence_after();
+        // New running max: rescale the accumulated O and l, lazily (only when the max grows by
+        // more than 2^8).  The TMEM round trip is warp-wide (.sync.aligned): a lane that needs
+        // no rescale multiplies by 1.
+        const bool grow = mx > m_used + 8.f;
+        float corr = 1.f;
+        if (grow) {
+          corr = ex2_approx(m_used - mx);
+          l *= corr;
+          m_used = mx;
+        }
+        if (it > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + 256 + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= corr;
+            tmem_st32(tmem + lane_base + 256 + c * 32, o);
+          }
+          tmem_st_wait();
+        }
+        // P = exp2(z - m) as bf16, summed in the same rounding the MMA sees
+        const float msub = m_used == -INFINITY ? 0.f : m_used;
+        float lsum = 0.f;
+#pragma unroll
+        for (int g = 0; g < BN / 8; ++g) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = ex2_approx(z[g * 8 + 2 * e] - msub);
+            const float p1 = ex2_approx(z[g * 8 + 2 * e + 1] - msub);
+            const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
+            const float2 back = __bfloat1622float2(pp);
+            lsum += back.x + back.y;
+            pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+          }
+          // K-major 128B-swizzled layout: chunk g/8 (64 keys), 16-byte granule g%8 of row `row`
+          const int chunk = g >> 3, gran = g & 7;
+          uint8_t* dst = sP + chunk * 16384 + row * 128 + ((gran ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        l += lsum;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
+      }
+    }
+    // epilogue: O / l to global, lse
+    if (ok && n_kt > 0 && !warp_wait(pv_done, (n_kt - 1) & 1, abort)) where = 8;
+    if (ok && n_kt > 0 && where == 0) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* out = (__nv_bfloat16*)a.out;
+      const bool live = row < tile.qlen;
+      __nv_bfloat16* orow = out + ((int64_t)(b * a.T + tq) * a.H + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + 256 + c * 32, o);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 u;
+            __nv_bfloat162 t0 = __floats2bfloat162_rn(o[i] * inv, o[i + 1] * inv);
+            __nv_bfloat162 t1 = __floats2bfloat162_rn(o[i + 2] * inv, o[i + 3] * inv);
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(o[i + 4] * inv, o[i + 5] * inv);
+            __nv_bfloat162 t3 = __floats2bfloat162_rn(o[i + 6] * inv, o[i + 7] * inv);
+            u.x = *reinterpret_cast<uint32_t*>(&t0);
+            u.y = *reinterpret_cast<uint32_t*>(&t1);
+            u.z = *reinterpret_cast<uint32_t*>(&t2);
+            u.w = *reinterpret_cast<uint32_t*>(&t3);
+            *reinterpret_cast<uint4*>(orow + c * 32 + i) = u;
+          }
+        }
+      }
+      if (live && a.lse) a.lse[(int64_t)bh * a.T + tq] = (m_used + log2f(l)) * 0.6931471805599453f;
+    }
+    if (where && lane == 0) atomicCAS((int*)&where_s, 0, where * 1000 + min(it, 999));
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_s && threadIdx.x == 0 && status) {
+    if (atomicCAS(status, 0, 1) == 0) {
+      status[1] = tile_id * 65536 + bh;
+      status[2] = where_s;
+    }
+  }
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// rows x width bf16 matrix whose rows are `row_stride` elements apart, in (64 x 128) boxes.
+bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows, int width, int64_t row_stride) {
+  cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)base, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// (B*L, H, width) view of a (B, L, H, width) bf16 tensor, boxes of (64, 1 head, 128 rows).
+bool make_map_3d(CUtensorMap* m, const void* base, int64_t BL, int H, int width) {
+  cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)BL};
+  cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)width * H * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t es[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)base, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int E, int D>
+cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
+  TcMaps maps;
+  const int64_t compact_rows = (int64_t)a.B * a.H * a.n_slots * a.slot_rows;
+  bool ok = make_map_3d(&maps.q, a.q, (int64_t)a.B * a.T, a.H, E) &&
+            make_map_3d(&maps.k, a.k, (int64_t)a.B * a.L, a.H, E) &&
+            make_map_3d(&maps.v, a.v, (int64_t)a.B * a.L, a.H, D);
+  if (ok && a.ck && compact_rows > 0) {
+    ok = make_map_2d(&maps.ck, a.ck, compact_rows, E, E) && make_map_2d(&maps.cv, a.cv, compact_rows, D, D);
+  } else if (ok) {
+    maps.ck = maps.k;
+    maps.cv = maps.v;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  const size_t sm = TcLayout<E, D>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<E, D><<<dim3(a.n_tiles, a.B * a.H), 192, sm, st>>>(maps, a, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attention_tc_supported(int dtype, int E, int D) {
+  if (dtype != 1) return false;
+  return (E == 64 && (D == 64 || D == 128 || D == 256)) || (E == 128 && (D == 64 || D == 128));
+}
+
+int attention_tc_tile_rows() { return BM; }
+
+cudaError_t launch_attention_tc(const AttnArgs& a, int* status, cudaStream_t st, bool* done) {
+  *done = false;
+  if (!encode_fn() || a.n_tiles == 0 || a.B * a.H == 0) return cudaSuccess;
+  cudaError_t e = cudaErrorInvalidValue;
+  if (a.E == 64 && a.D == 64) e = launch_tc_t<64, 64>(a, status, st);
+  else if (a.E == 64 && a.D == 128) e = launch_tc_t<64, 128>(a, status, st);
+  else if (a.E == 64 && a.D == 256) e = launch_tc_t<64, 256>(a, status, st);
+  else if (a.E == 128 && a.D == 64) e = launch_tc_t<128, 64>(a, status, st);
+  else if (a.E == 128 && a.D == 128) e = launch_tc_t<128, 128>(a, status, st);
+  else return cudaSuccess;
+  if (e == cudaSuccess) *done = true;
+  return e;
+}
+
 }  // namespace thin
