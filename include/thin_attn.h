@@ -159,6 +159,39 @@ THIN_ATTN_API thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms,
  * handle's kernels since the last call (THIN_ATTN_ETIMEOUT, ...). */
 THIN_ATTN_API thin_attn_status thin_attn_check(thin_attn_t h, void* stream);
 
+/*
+ * Kernel Halving of caller-provided point sets, allocating no device memory.
+ * The pages have no counterpart of this entry point: it exists for callers that
+ * cannot allocate -- an application whose device memory is owned by its own pool
+ * or budgeted up front, or one that cannot accept the device-wide synchronisation
+ * and failure modes that cudaMalloc/cudaFree bring in the middle of a run.
+ *
+ *   K (n_inst, n, E), V (n_inst, n, D)   device, contiguous, fp32 or bf16 (dtype)
+ *   K_out, V_out (n_inst, n/2, E|D)      device: the kept point of every pair, pair order
+ *   idx_out (n_inst, n/2) int32          device: position (0..n-1) of each kept point in its set
+ *   keep_bits_opt                        device uint32[n_inst * ceil(n/64)] or NULL: bit i%32 of
+ *                                        word i/32 of set s (words ceil(n/64) apart) = 1 iff pair i
+ *                                        kept its first point
+ * Set s is halved with the Philox counter (pair, round_id, s, 0) keyed by seed, with the same
+ * kernel-halving walk and kernel as thin_attn_forward; scale <= 0 selects 1/sqrt(E).
+ * n is even, 2 <= n <= 4096; E, D multiples of 8 in [8, 256].
+ *
+ * Scratch is a 16 MiB array in the library's device memory, held by every device that loads
+ * the library until the process exits.  It needs
+ *   n_inst*40 + n_inst*n*4 + n_inst*4 (each rounded up to 256) + n_inst*ceil(n/64)^2*4096
+ * bytes; larger requests fail with THIN_ATTN_EINVAL before anything is enqueued.  All calls
+ * share the array: calls whose work overlaps on the GPU (other streams, other threads) race
+ * on it and must be serialised by the caller.  Every scratch element a call reads is written
+ * earlier in the same call, so nothing needs clearing between calls.
+ * Runs on the current device; the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and should come before any stream capture.
+ */
+THIN_ATTN_API thin_attn_status thin_attn_halve_noalloc(int dtype, const void* K, const void* V, int n_inst,
+                                                      int n, int E, int D, float scale, uint64_t seed,
+                                                      uint32_t round_id, void* K_out, void* V_out,
+                                                      int32_t* idx_out, uint32_t* keep_bits_opt,
+                                                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -115,6 +115,14 @@ struct Plan {
 
 }  // namespace
 
+namespace thin {
+// Record `msg` as the calling thread's last error (read by thin_attn_last_error) and return s.
+int record_error(int s, const char* msg) {
+  g_err = msg;
+  return s;
+}
+}  // namespace thin
+
 struct thin_attn_s {
   thin_attn_config cfg{};
   float scale = 0.f;
