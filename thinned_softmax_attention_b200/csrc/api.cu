@@ -539,6 +539,9 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     int32_t* didx;
     buf_ptrs(p, sp.dst_buf, k, v, &dk, &dv, &didx);
     a.src_kind = sp.src_buf == BUF_TOKENS ? SRC_TOKENS : SRC_COMPACT;
+    a.src_rows = sp.src_buf == BUF_TOKENS ? (int64_t)cf.B * (p->causal ? cf.T : cf.S)
+                 : (sp.src_buf == BUF_NODES ? p->nodes : sp.src_buf == BUF_MTEMP ? p->mtemp : p->levels[sp.src_buf]).rows;
+    a.status = h->d_status;
     a.srcK = sk;
     a.srcV = sv;
     a.srcIdx = sidx;

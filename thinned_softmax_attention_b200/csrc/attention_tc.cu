@@ -230,17 +230,25 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(s_free + sb);
-        // logits in base 2 with the segment's log-weight; masked keys -> -inf
+        // Masked keys -> -inf.  A tile every query of the CTA sees in full (the usual case) skips
+        // the mask; otherwise key c is visible to this row iff c <= lim.
         const int nvalid = min(BN, sg.len - j0);
         const int kt0 = sg.first + j0;
         const bool causal = sg.kind == SEG_TOKENS && sg.causal;
-        float mx = -INFINITY;
+        if (nvalid < BN || (causal && kt0 + BN - 1 > tile.q0)) {
+          const int lim = min(nvalid - 1, causal ? tq - kt0 : BN - 1);
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const bool vis = c < nvalid && (!causal || kt0 + c <= tq);
-          z[c] = vis ? fmaf(z[c], a.scale_log2e, lw2) : -INFINITY;
-          mx = fmaxf(mx, z[c]);
+          for (int c = 0; c < BN; ++c) z[c] = c <= lim ? z[c] : -INFINITY;
         }
+        // row max of the raw scores (scale > 0 keeps the order), 8 independent chains
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = z[i];
+#pragma unroll
+        for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], z[c]);
+        const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float mx = smax == -INFINITY ? -INFINITY : fmaf(smax, a.scale_log2e, lw2);
         // P of the previous tile must be consumed (PV done) before P and O are touched
         if (it > 0 && !warp_wait(pv_done, (it - 1) & 1, abort)) {
           ok = false;
@@ -270,19 +278,19 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           }
           tmem_st_wait();
         }
-        // P = exp2(z - m) as bf16, summed in the same rounding the MMA sees
-        const float msub = m_used == -INFINITY ? 0.f : m_used;
-        float lsum = 0.f;
+        // p = 2^(s * scale * log2e + log2 w - m) in one FMA + EX2; a row that has seen no key yet
+        // (m = -inf) has only -inf scores and gets p = 0.
+        const float off = m_used == -INFINITY ? 0.f : lw2 - m_used;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int g = 0; g < BN / 8; ++g) {
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2_approx(z[g * 8 + 2 * e] - msub);
-            const float p1 = ex2_approx(z[g * 8 + 2 * e + 1] - msub);
+            const float p0 = ex2_approx(fmaf(z[g * 8 + 2 * e], a.scale_log2e, off));
+            const float p1 = ex2_approx(fmaf(z[g * 8 + 2 * e + 1], a.scale_log2e, off));
+            ls[e] += p0 + p1;
             const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
-            const float2 back = __bfloat1622float2(pp);
-            lsum += back.x + back.y;
             pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
           }
           // K-major 128B-swizzled layout: chunk g/8 (64 keys), 16-byte granule g%8 of row `row`
@@ -290,7 +298,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           uint8_t* dst = sP + chunk * 16384 + row * 128 + ((gran ^ (row & 7)) << 4);
           *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        l += lsum;
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(p_full);
@@ -343,55 +351,15 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)p;
-  }
-  return fn;
-}
-
-// rows x width bf16 matrix whose rows are `row_stride` elements apart, in (64 x 128) boxes.
-bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows, int width, int64_t row_stride) {
-  cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t es[2] = {1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)base, dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// (B*L, H, width) view of a (B, L, H, width) bf16 tensor, boxes of (64, 1 head, 128 rows).
-bool make_map_3d(CUtensorMap* m, const void* base, int64_t BL, int H, int width) {
-  cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)BL};
-  cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)width * H * 2};
-  cuuint32_t box[3] = {64, 1, 128};
-  cuuint32_t es[3] = {1, 1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)base, dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int E, int D>
 cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
   TcMaps maps;
   const int64_t compact_rows = (int64_t)a.B * a.H * a.n_slots * a.slot_rows;
-  bool ok = make_map_3d(&maps.q, a.q, (int64_t)a.B * a.T, a.H, E) &&
-            make_map_3d(&maps.k, a.k, (int64_t)a.B * a.L, a.H, E) &&
-            make_map_3d(&maps.v, a.v, (int64_t)a.B * a.L, a.H, D);
+  bool ok = make_map_3d(&maps.q, a.q, (int64_t)a.B * a.T, a.H, E, 128) &&
+            make_map_3d(&maps.k, a.k, (int64_t)a.B * a.L, a.H, E, 128) &&
+            make_map_3d(&maps.v, a.v, (int64_t)a.B * a.L, a.H, D, 128);
   if (ok && a.ck && compact_rows > 0) {
-    ok = make_map_2d(&maps.ck, a.ck, compact_rows, E, E) && make_map_2d(&maps.cv, a.cv, compact_rows, D, D);
+    ok = make_map_2d(&maps.ck, a.ck, compact_rows, E, E, 128) && make_map_2d(&maps.cv, a.cv, compact_rows, D, D, 128);
   } else if (ok) {
     maps.ck = maps.k;
     maps.cv = maps.v;
@@ -406,6 +374,48 @@ cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
 
 }  // namespace
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// rows x width bf16 matrix whose rows are `row_stride` elements apart, in (64 x 128) boxes.
+bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows, int width, int64_t row_stride, int box_rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)base, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// (B*L, H, width) view of a (B, L, H, width) bf16 tensor, boxes of (64, 1 head, 128 rows).
+bool make_map_3d(CUtensorMap* m, const void* base, int64_t BL, int H, int width, int box_rows) {
+  cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)BL};
+  cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)width * H * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)base, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tensor_maps_available() { return encode_fn() != nullptr; }
+
 bool attention_tc_supported(int dtype, int E, int D) {
   if (dtype != 1) return false;
   return (E == 64 && (D == 64 || D == 128 || D == 256)) || (E == 128 && (D == 64 || D == 128));
@@ -415,7 +425,7 @@ int attention_tc_tile_rows() { return BM; }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, int* status, cudaStream_t st, bool* done) {
   *done = false;
-  if (!encode_fn() || a.n_tiles == 0 || a.B * a.H == 0) return cudaSuccess;
+  if (!tensor_maps_available() || a.n_tiles == 0 || a.B * a.H == 0) return cudaSuccess;
   cudaError_t e = cudaErrorInvalidValue;
   if (a.E == 64 && a.D == 64) e = launch_tc_t<64, 64>(a, status, st);
   else if (a.E == 64 && a.D == 128) e = launch_tc_t<64, 128>(a, status, st);

@@ -81,6 +81,7 @@ struct StepArgs {
   const void* srcV;
   const int32_t* srcIdx;   // SRC_COMPACT only
   int H;                   // heads (SRC_TOKENS row addressing)
+  int64_t src_rows;        // rows of the source: B*L (SRC_TOKENS) or compact rows; 0 = unknown
   int S_full, S_sub;       // SRC_TOKENS subsample: token = floor((p*S_full + U)/S_sub)
   // destination
   void* dstK;
@@ -99,6 +100,7 @@ struct StepArgs {
   // scratch
   float* c2;               // (n_inst) squared max |v|
   float* delta;            // (n_inst, m_pad, m_pad)
+  int* status;             // device status word for bounded waits (may be null)
   // trace (may be null)
   uint32_t* trace;
   uint64_t trace_base;     // first word of this step

@@ -1,6 +1,7 @@
 // Kernel launchers of the thin_attn library (internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -24,5 +25,12 @@ int attention_simt_tile_rows();
 cudaError_t launch_attention_tc(const AttnArgs& a, int* status_word, cudaStream_t st, bool* done);
 int attention_tc_tile_rows();
 bool attention_tc_supported(int dtype, int E, int D);
+
+// bf16 TMA tensor maps with 128-byte swizzle and (64 elements x box_rows) boxes:
+// 2D over `rows` rows of `width` elements, rows `row_stride` elements apart;
+// 3D over a (B*L, H, width) view of a (B, L, H, width) tensor, one head per box.
+bool tensor_maps_available();
+bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows, int width, int64_t row_stride, int box_rows);
+bool make_map_3d(CUtensorMap* m, const void* base, int64_t BL, int H, int width, int box_rows);
 
 }  // namespace thin

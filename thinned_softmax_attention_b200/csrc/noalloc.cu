@@ -116,6 +116,7 @@ extern "C" THIN_ATTN_API thin_attn_status thin_attn_halve_noalloc(int dtype, con
   a.srcV = V;
   a.srcIdx = pidx;
   a.H = 1;
+  a.src_rows = (int64_t)n_inst * n;
   a.S_full = a.S_sub = n;
   a.dstK = K_out;
   a.dstV = V_out;
