@@ -19,30 +19,58 @@
 
 namespace thin {
 
+// Approximate square root and reciprocal (MUFU): relative error ~1e-7, far below the 1e-4
+// near-tie margin of the decisions; they sit on the walk's serial chain.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------------------
 // 1. c^2 = (max |v|)^2 over the instance's points
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(128) c2_kernel(StepArgs a) {
+__global__ void __launch_bounds__(256) c2_kernel(StepArgs a) {
   const int inst = blockIdx.x;
   const HalveInst in = a.inst[inst];
   __shared__ uint32_t U_s;
-  __shared__ float red[4];
+  __shared__ float red[8];
   if (threadIdx.x == 0) U_s = sub_offset(a, in);
   __syncthreads();
-  const T* V = (const T*)a.srcV;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int epc = 16 / (int)sizeof(T);            // elements per 16-byte chunk
+  const int cpp = a.D / epc;                       // chunks per point
+  const uint4* V = (const uint4*)a.srcV;
   float mx = 0.f;
-  for (int p = warp; p < a.n; p += 4) {
+  for (int e = threadIdx.x; e < a.n * cpp; e += blockDim.x) {
+    const int p = e / cpp, c = e - p * cpp;
     const PointRef r = point_ref(a, in, p, U_s);
-    for (int d = lane; d < a.D; d += 32) mx = fmaxf(mx, fabsf(to_f(V[r.vrow + d])));
+    const uint4 w = V[r.vrow / epc + c];
+    if (sizeof(T) == 2) {
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(ws[i] << 16), hi = __uint_as_float(ws[i] & 0xFFFF0000u);
+        mx = fmaxf(mx, fmaxf(fabsf(lo), fabsf(hi)));
+      }
+    } else {
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(w.x)), fabsf(__uint_as_float(w.y))),
+                           fmaxf(fabsf(__uint_as_float(w.z)), fabsf(__uint_as_float(w.w)))));
+    }
   }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
   for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if (lane == 0) red[warp] = mx;
   __syncthreads();
   if (threadIdx.x == 0) {
-    const float v = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    float v = red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) v = fmaxf(v, red[w]);
     a.c2[inst] = v * v;
   }
 }
@@ -147,7 +175,7 @@ __global__ void __launch_bounds__(256) pairgram_simt_kernel(StepArgs a) {
 //    pair order j = 0, 1, ..., i-1.
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(128) walk_kernel(StepArgs a) {
+__global__ void __launch_bounds__(128, 8) walk_kernel(StepArgs a) {
   extern __shared__ float sm[];
   const int inst = blockIdx.x;
   const HalveInst in = a.inst[inst];
@@ -174,32 +202,46 @@ __global__ void __launch_bounds__(128) walk_kernel(StepArgs a) {
       tile[r * 33 + c] = (base + r < m && base + c < m) ? Dl[(size_t)(base + r) * mp + base + c] : 0.f;
     }
     __syncthreads();
+    const int steps = min(32, m - base);
     if (warp == 0) {
+      // per-pair values held by lane l (pair base + l): b^2, b, 1 - 2u
+      const float b2l = tile[lane * 33 + lane];
+      const float bl = sqrt_approx(fmaxf(b2l, 0.f));
+      const float ul = 1.f - 2.f * ubuf[base + lane];
       float my = alpha[base + lane];
       uint32_t kb = 0;
-      const int steps = min(32, m - base);
-      for (int s = 0; s < steps; ++s) {
-        const float ai = __shfl_sync(0xffffffffu, my, s);
-        const float b2 = tile[s * 33 + s];
-        bool keep = true;
-        if (b2 > 0.f) {
-          const float b = sqrtf(b2);
-          const float av = fmaxf(b * sqrtf(sig2) * a.C, b2);
-          keep = ai < av * (1.f - 2.f * ubuf[base + s]);
-          sig2 = sig2 + b2 * fmaxf(0.f, 1.f + (b2 - 2.f * av) * sig2 / (av * av));
+#pragma unroll
+      for (int s = 0; s < 32; ++s) {
+        if (s < steps) {
+          const float b2 = __shfl_sync(0xffffffffu, b2l, s);
+          const float b = __shfl_sync(0xffffffffu, bl, s);
+          const float w = __shfl_sync(0xffffffffu, ul, s);
+          const float ai = __shfl_sync(0xffffffffu, my, s);
+          bool keep = true;
+          if (b2 > 0.f) {
+            const float av = fmaxf(b * sqrt_approx(sig2) * a.C, b2);
+            keep = ai < av * w;
+            const float r = rcp_approx(av * av);
+            sig2 = sig2 + b2 * fmaxf(0.f, 1.f + (b2 - 2.f * av) * sig2 * r);
+          }
+          if (lane > s) my = fmaf(keep ? 1.f : -1.f, tile[s * 33 + lane], my);
+          kb |= (uint32_t)keep << s;
         }
-        if (lane > s) my = fmaf(keep ? 1.f : -1.f, tile[s * 33 + lane], my);
-        kb |= (uint32_t)keep << s;
       }
       if (lane == 0) bits[t] = kb;
     }
     __syncthreads();
     const uint32_t kb = bits[t];
-    const int steps = min(32, m - base);
     for (int k = base + 32 + tid; k < m; k += 128) {
       float acc = alpha[k];
-      for (int s = 0; s < steps; ++s)
-        acc = fmaf(((kb >> s) & 1u) ? 1.f : -1.f, Dl[(size_t)(base + s) * mp + k], acc);
+#pragma unroll
+      for (int s0 = 0; s0 < 32; s0 += 8) {
+        float d[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) d[s] = s0 + s < steps ? Dl[(size_t)(base + s0 + s) * mp + k] : 0.f;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) acc = fmaf(((kb >> (s0 + s)) & 1u) ? 1.f : -1.f, d[s], acc);
+      }
       alpha[k] = acc;
     }
   }
@@ -222,6 +264,169 @@ __global__ void __launch_bounds__(128) walk_kernel(StepArgs a) {
     for (int w = lane; w < vw; w += 32) dV[drow * vw + w] = V[r.vrow / epw + w];
     if (lane == 0) a.dstIdx[drow] = r.idx;
   }
+}
+
+// One step of the sigma recursion and the threshold of pair i.  With C = sqrt(2 ln(2/delta_i)) > 1:
+//   b >= sigma C:  a = b^2,          sigma' = b
+//   otherwise:     a = b sigma C,    sigma'^2 = sigma^2 + max(0, b^2 (1 + 1/C^2) - 2 b sigma / C)
+// which is sigma'^2 = sigma^2 + b^2 max(0, 1 + (b^2 - 2a) sigma^2 / a^2) with the two cases of
+// a = max(b sigma C, b^2) written out (in the first, sigma <= b/C < b gives sigma'^2 = b^2).
+// Returns a; sigma is updated in place.  b^2 <= 0 (a repeated point) keeps sigma and returns 0.
+__device__ __forceinline__ float sigma_step(float& sigma, float b2, float b, float C, float q, float r2) {
+  if (!(b2 > 0.f)) return 0.f;
+  const float sc = sigma * C;
+  if (b >= sc) {
+    sigma = b;
+    return b2;
+  }
+  const float a = b * sc;
+  sigma = sqrt_approx(fmaf(sigma, sigma, fmaxf(0.f, fmaf(-r2, sigma, q))));
+  return a;
+}
+
+// Gather the kept point of pair i (keep = first point) into destination row dst_row + i.
+template <typename T>
+__device__ __forceinline__ void gather_row(const StepArgs& a, const HalveInst& in, uint32_t U, int i, bool keep,
+                                           int lane) {
+  const int kw = a.E * (int)sizeof(T) / 16, vw = a.D * (int)sizeof(T) / 16;
+  const int epw = 16 / (int)sizeof(T);
+  const PointRef r = point_ref(a, in, 2 * i + (keep ? 0 : 1), U);
+  const int64_t drow = in.dst_row + i;
+  const uint4* K = (const uint4*)a.srcK;
+  const uint4* V = (const uint4*)a.srcV;
+  uint4* dK = (uint4*)a.dstK;
+  uint4* dV = (uint4*)a.dstV;
+  for (int w = lane; w < kw + vw; w += 32) {
+    if (w < kw) dK[drow * kw + w] = K[r.krow / epw + w];
+    else dV[drow * vw + (w - kw)] = V[r.vrow / epw + (w - kw)];
+  }
+  if (lane == 0) a.dstIdx[drow] = r.idx;
+}
+
+// Walk of instances with m <= 32 pairs: one warp per instance.  Lane l holds column l of the
+// pair-difference matrix (Delta[s][l] for every s) and alpha of pair l.
+template <typename T>
+__global__ void __launch_bounds__(128) walk_small_kernel(StepArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int inst = blockIdx.x * 4 + warp;
+  if (inst >= a.n_inst) return;
+  const HalveInst in = a.inst[inst];
+  const int m = a.m;
+  const float* Dl = a.delta + (size_t)inst * a.m_pad * a.m_pad;
+  float d[32];
+#pragma unroll
+  for (int s = 0; s < 32; ++s) d[s] = (s < m && lane < m) ? Dl[(size_t)s * a.m_pad + lane] : 0.f;
+  const float w_l = lane < m ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)lane) : 0.f;
+  const uint32_t U = sub_offset(a, in);
+  const float C = a.C, cq = 1.f + 1.f / (C * C), c2C = 2.f / C;
+  float my = 0.f, sigma = 0.f;
+  uint32_t kb = 0;
+#pragma unroll
+  for (int s = 0; s < 32; ++s) {
+    if (s < m) {
+      const float b2 = __shfl_sync(0xffffffffu, d[s], s);
+      const float w = __shfl_sync(0xffffffffu, w_l, s);
+      const float b = sqrt_approx(fmaxf(b2, 0.f));
+      const float av = sigma_step(sigma, b2, b, C, b2 * cq, b * c2C);
+      const float ai = __shfl_sync(0xffffffffu, my, s);
+      const bool keep = !(b2 > 0.f) || ai < av * w;
+      if (lane > s) my = fmaf(keep ? 1.f : -1.f, d[s], my);
+      kb |= (uint32_t)keep << s;
+    }
+  }
+  if (a.trace && lane == 0) a.trace[a.trace_base + inst] = kb;
+  for (int i = 0; i < m; ++i) gather_row<T>(a, in, U, i, (kb >> i) & 1u, lane);
+}
+
+// Walk of instances with 32 < m <= 256 pairs: one CTA of 128 threads per instance.  The 32 rows
+// of Delta of pair block t (columns >= 32t) are staged in shared memory with cp.async while
+// block t-1 is walked; warp 0 runs the 32 dependent decisions of a block, then all threads add
+// the block's contribution to the alpha of the later pairs.
+constexpr int kWalkMidMaxPad = 256;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <typename T>
+__global__ void __launch_bounds__(128) walk_mid_kernel(StepArgs a) {
+  extern __shared__ __align__(16) float smf[];
+  const int inst = blockIdx.x;
+  const HalveInst in = a.inst[inst];
+  const int m = a.m, mp = a.m_pad, nb = mp >> 5;
+  float* alpha = smf;                          // mp
+  float* wbuf = alpha + mp;                    // mp: 1 - 2u
+  float* rb = wbuf + mp;                       // 2 x 32 x mp
+  uint32_t* bits = (uint32_t*)(rb + 64 * mp);  // nb
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* Dl = a.delta + (size_t)inst * mp * mp;
+  auto stage = [&](int t) {   // rows [32t, 32t+32), columns [32t, mp) -> rb[t & 1]
+    float* dst = rb + (t & 1) * 32 * mp;
+    const int c0 = 32 * t, nq = (mp - c0) / 4;
+    for (int e = tid; e < 32 * nq; e += 128) {
+      const int r = e / nq, q = e - r * nq;
+      cp_async16(dst + r * mp + c0 + 4 * q, Dl + (size_t)(c0 + r) * mp + c0 + 4 * q);
+    }
+    cp_async_commit();
+  };
+  stage(0);
+  for (int i = tid; i < mp; i += 128) {
+    alpha[i] = 0.f;
+    wbuf[i] = i < m ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)i) : 0.f;
+  }
+  const float C = a.C, cq = 1.f + 1.f / (C * C), c2C = 2.f / C;
+  float sigma = 0.f;
+  for (int t = 0; t < nb; ++t) {
+    const int base = 32 * t;
+    __syncthreads();                 // rb[(t+1)&1] is no longer read (update of block t-1)
+    if (t + 1 < nb) {
+      stage(t + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const float* R = rb + (t & 1) * 32 * mp;
+    const int steps = min(32, m - base);
+    if (warp == 0) {
+      const float dl = lane < steps ? R[lane * mp + base + lane] : 0.f;   // b^2 of pair base+lane
+      const float bl = sqrt_approx(fmaxf(dl, 0.f));
+      const float wl = wbuf[base + lane];
+      float my = alpha[base + lane];
+      uint32_t kb = 0;
+#pragma unroll
+      for (int s = 0; s < 32; ++s) {
+        if (s < steps) {
+          const float b2 = __shfl_sync(0xffffffffu, dl, s);
+          const float b = __shfl_sync(0xffffffffu, bl, s);
+          const float w = __shfl_sync(0xffffffffu, wl, s);
+          const float av = sigma_step(sigma, b2, b, C, b2 * cq, b * c2C);
+          const float ai = __shfl_sync(0xffffffffu, my, s);
+          const bool keep = !(b2 > 0.f) || ai < av * w;
+          if (lane > s) my = fmaf(keep ? 1.f : -1.f, R[s * mp + base + lane], my);
+          kb |= (uint32_t)keep << s;
+        }
+      }
+      if (lane == 0) bits[t] = kb;
+    }
+    __syncthreads();
+    const uint32_t kb = bits[t];
+    for (int k = base + 32 + tid; k < m; k += 128) {
+      float acc = alpha[k];
+#pragma unroll 8
+      for (int s = 0; s < steps; ++s) acc = fmaf(((kb >> s) & 1u) ? 1.f : -1.f, R[s * mp + k], acc);
+      alpha[k] = acc;
+    }
+  }
+  __syncthreads();
+  if (a.trace)
+    for (int w = tid; w < nb; w += 128) a.trace[a.trace_base + (size_t)inst * nb + w] = bits[w];
+  const uint32_t U = sub_offset(a, in);
+  for (int i = warp; i < m; i += 4) gather_row<T>(a, in, U, i, (bits[i >> 5] >> (i & 31)) & 1u, lane);
 }
 
 // Copy runs of tokens unchanged into compact rows (Express batches that need no thinning).
@@ -255,7 +460,7 @@ size_t walk_smem_bytes(int m_pad) { return (size_t)(2 * m_pad + 32 * 33 + m_pad 
 template <typename T>
 static cudaError_t launch_step_t(const StepArgs& a, bool use_tc, cudaStream_t st) {
   if (a.n_inst == 0) return cudaSuccess;
-  c2_kernel<T><<<a.n_inst, 128, 0, st>>>(a);
+  c2_kernel<T><<<a.n_inst, 256, 0, st>>>(a);
   const int nb = a.m_pad / 32;
   const int ntri = nb * (nb + 1) / 2;
   bool done = false;
@@ -264,6 +469,17 @@ static cudaError_t launch_step_t(const StepArgs& a, bool use_tc, cudaStream_t st
     if (e != cudaSuccess) return e;
   }
   if (!done) pairgram_simt_kernel<T><<<dim3(a.n_inst, ntri), 256, 0, st>>>(a);
+  if (a.m <= 32) {
+    walk_small_kernel<T><<<(a.n_inst + 3) / 4, 128, 0, st>>>(a);
+    return cudaGetLastError();
+  }
+  if (a.m_pad <= kWalkMidMaxPad) {
+    const size_t sm = (size_t)(2 * a.m_pad + 64 * a.m_pad + a.m_pad / 32) * 4;
+    cudaError_t e = cudaFuncSetAttribute(walk_mid_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    walk_mid_kernel<T><<<a.n_inst, 128, sm, st>>>(a);
+    return cudaGetLastError();
+  }
   const size_t sm = walk_smem_bytes(a.m_pad);
   if (sm > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(walk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
