@@ -14,6 +14,8 @@
 //              O += P V into TMEM cols 256..256+D; also owns the TMEM allocation
 // Every wait on an mbarrier is bounded; a CTA that gives up records the failure in the status
 // word and leaves through the normal exit path (TMEM freed, its TMA copies landed).
+#include <cstdlib>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -351,6 +353,293 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Two CTAs per SM variant (D <= 128): 96 KB of shared memory and 256 TMEM columns per CTA, so
+// one CTA's MMAs overlap the other's softmax.  S lives in TMEM columns 0..127; the softmax writes
+// P (bf16, two per column) back into columns 0..63 and the PV MMA reads it from there as its A
+// operand; O accumulates in columns 128..128+D.  K and V have one stage each with separate
+// barriers: K(j+1) loads as soon as S(j) is done, V(j+1) as soon as PV(j) is done.  The MMA
+// thread issues S(j+1) only after PV(j) has completed, so P(j) is never overwritten early.
+// The softmax reads S twice (max pass, then exponent pass) to stay within 170 registers.
+template <int E, int D>
+struct Tc2Layout {
+  static constexpr int EC = E / 64, DC = D / 64;
+  static constexpr uint32_t Q_BYTES = BM * E * 2;
+  static constexpr uint32_t K_BYTES = BN * E * 2;
+  static constexpr uint32_t V_BYTES = BN * D * 2;
+  static constexpr uint32_t OFF_K = Q_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + K_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + V_BYTES;
+  static constexpr uint32_t BYTES = OFF_BAR + 128 + 1024;
+};
+
+template <int E, int D>
+__global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a,
+                                                          int* status) {
+  using Lay = Tc2Layout<E, D>;
+  constexpr uint32_t O_COL = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + Lay::OFF_K;
+  uint8_t* sV = smem + Lay::OFF_V;
+  uint64_t* bars = (uint64_t*)(smem + Lay::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 2;
+  uint64_t* v_full = bars + 3;
+  uint64_t* v_empty = bars + 4;
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* pv_done = bars + 7;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  __shared__ volatile int where_s;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile_id = a.n_tiles - 1 - (int)blockIdx.x;
+  const AttnTile tile = a.tiles[tile_id];
+  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int n_kt = count_key_tiles(a, tile);
+
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    where_s = 0;
+    mbar_init(q_full, 1);
+    mbar_init(k_full, 1);
+    mbar_init(k_empty, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) tmem_alloc(&tmem_base_s, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort = &abort_s;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_kt > 0) {
+      mbar_expect_tx(q_full, Lay::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < Lay::EC; ++c) tma_load_3d(sQ + c * 16384, &maps.q, q_full, c * 64, h, b * a.T + tile.q0);
+      int it = 0;
+      bool ok = true;
+      for (int si = 0; si < tile.nseg && ok; ++si) {
+        const AttnSeg sg = a.segs[tile.seg0 + si];
+        const bool tok = sg.kind == SEG_TOKENS;
+        for (int j0 = 0; j0 < sg.len; j0 += BN, ++it) {
+          const int row = tok ? b * a.L + sg.first + j0 : (bh * a.n_slots + sg.first) * a.slot_rows + j0;
+          if (it > 0 && !mbar_wait(k_empty, (it - 1) & 1, abort)) {
+            ok = false;
+            atomicCAS((int*)&where_s, 0, 1000 + min(it, 999));
+            break;
+          }
+          mbar_expect_tx(k_full, Lay::K_BYTES);
+#pragma unroll
+          for (int c = 0; c < Lay::EC; ++c) {
+            if (tok) tma_load_3d(sK + c * 16384, &maps.k, k_full, c * 64, h, row);
+            else tma_load_2d(sK + c * 16384, &maps.ck, k_full, c * 64, row);
+          }
+          if (it > 0 && !mbar_wait(v_empty, (it - 1) & 1, abort)) {
+            ok = false;
+            atomicCAS((int*)&where_s, 0, 2000 + min(it, 999));
+            break;
+          }
+          mbar_expect_tx(v_full, Lay::V_BYTES);
+#pragma unroll
+          for (int c = 0; c < Lay::DC; ++c) {
+            if (tok) tma_load_3d(sV + c * 16384, &maps.v, v_full, c * 64, h, row);
+            else tma_load_2d(sV + c * 16384, &maps.cv, v_full, c * 64, row);
+          }
+        }
+      }
+      // never leave with a copy in flight into this CTA's shared memory
+      if (it > 0) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(k_full, (it - 1) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+        while (!mbar_try_wait(v_full, (it - 1) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+      const long long t0 = clock64();
+      while (!mbar_try_wait(q_full, 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_kt > 0) {
+      constexpr uint32_t IQK = idesc_bf16(BM, BN, false);
+      constexpr uint32_t IPV = idesc_bf16(BM, D, true);
+      const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
+      bool ok = mbar_wait(q_full, 0, abort);
+      for (int it = 0; it < n_kt && ok; ++it) {
+        if (!mbar_wait(k_full, it & 1, abort) || (it > 0 && !mbar_wait(pv_done, (it - 1) & 1, abort))) {
+          atomicCAS((int*)&where_s, 0, 3000 + min(it, 999));
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < E / 16; ++k) {
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_bf16(tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), IQK, k > 0);
+        }
+        umma_commit(s_full);
+        umma_commit(k_empty);
+        if (!mbar_wait(p_full, it & 1, abort) || !mbar_wait(v_full, it & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 5000 + min(it, 999));
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k)
+          umma_bf16_tmem_a(tmem + O_COL, tmem + k * 8, sw128_desc(va + k * 2048, 16384, 1024), IPV,
+                           (it > 0 || k > 0) ? 1u : 0u);
+        umma_commit(pv_done);
+        umma_commit(v_empty);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroup
+    const int row = warp * 32 + lane;
+    const int tq = tile.q0 + row;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    float m_used = -INFINITY, l = 0.f;
+    int it = 0, where = 0;
+    bool ok = true;
+    for (int si = 0; si < tile.nseg && ok; ++si) {
+      const AttnSeg sg = a.segs[tile.seg0 + si];
+      const float lw2 = sg.logw * 1.4426950408889634f;
+      for (int j0 = 0; j0 < sg.len; j0 += BN, ++it) {
+        if (!warp_wait(s_full, it & 1, abort)) {
+          ok = false;
+          where = 6;
+          break;
+        }
+        tc_fence_after();
+        const int nvalid = min(BN, sg.len - j0);
+        const int kt0 = sg.first + j0;
+        const bool causal = sg.kind == SEG_TOKENS && sg.causal;
+        const bool masked = nvalid < BN || (causal && kt0 + BN - 1 > tile.q0);
+        const int lim = min(nvalid - 1, causal ? tq - kt0 : BN - 1);
+        // pass 1: row max of the raw scores
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          float z[32];
+          tmem_ld32(tmem + lane_base + c * 32, z);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float v = (!masked || c * 32 + i <= lim) ? z[i] : -INFINITY;
+            mx8[i & 7] = fmaxf(mx8[i & 7], v);
+          }
+        }
+        const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float mx = smax == -INFINITY ? -INFINITY : fmaf(smax, a.scale_log2e, lw2);
+        // lazy rescale of O and l (PV of the previous tile is complete: S of this tile was
+        // issued after it)
+        const bool grow = mx > m_used + 8.f;
+        float corr = 1.f;
+        if (grow) {
+          corr = ex2_approx(m_used - mx);
+          l *= corr;
+          m_used = mx;
+        }
+        if (it > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= corr;
+            tmem_st32(tmem + lane_base + O_COL + c * 32, o);
+          }
+        }
+        // pass 2: P = 2^(s scale log2e + log2 w - m) as bf16 into TMEM columns 16c..16c+15; they
+        // overlap only S columns already read
+        const float off = m_used == -INFINITY ? 0.f : lw2 - m_used;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          float z[32];
+          tmem_ld32(tmem + lane_base + c * 32, z);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float z0 = (!masked || c * 32 + 2 * e <= lim) ? z[2 * e] : -INFINITY;
+            const float z1 = (!masked || c * 32 + 2 * e + 1 <= lim) ? z[2 * e + 1] : -INFINITY;
+            const float p0 = ex2_approx(fmaf(z0, a.scale_log2e, off));
+            const float p1 = ex2_approx(fmaf(z1, a.scale_log2e, off));
+            ls[e & 3] += p0 + p1;
+            const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+          }
+          tmem_st16(tmem + lane_base + c * 16, pk);
+        }
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full);
+      }
+    }
+    if (ok && n_kt > 0 && !warp_wait(pv_done, (n_kt - 1) & 1, abort)) where = 8;
+    if (ok && n_kt > 0 && where == 0) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* out = (__nv_bfloat16*)a.out;
+      const bool live = row < tile.qlen;
+      __nv_bfloat16* orow = out + ((int64_t)(b * a.T + tq) * a.H + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 u;
+            __nv_bfloat162 t0 = __floats2bfloat162_rn(o[i] * inv, o[i + 1] * inv);
+            __nv_bfloat162 t1 = __floats2bfloat162_rn(o[i + 2] * inv, o[i + 3] * inv);
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(o[i + 4] * inv, o[i + 5] * inv);
+            __nv_bfloat162 t3 = __floats2bfloat162_rn(o[i + 6] * inv, o[i + 7] * inv);
+            u.x = *reinterpret_cast<uint32_t*>(&t0);
+            u.y = *reinterpret_cast<uint32_t*>(&t1);
+            u.z = *reinterpret_cast<uint32_t*>(&t2);
+            u.w = *reinterpret_cast<uint32_t*>(&t3);
+            *reinterpret_cast<uint4*>(orow + c * 32 + i) = u;
+          }
+        }
+      }
+      if (live && a.lse) a.lse[(int64_t)bh * a.T + tq] = (m_used + log2f(l)) * 0.6931471805599453f;
+    }
+    if (where && lane == 0) atomicCAS((int*)&where_s, 0, where * 1000 + min(it, 999));
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_s && threadIdx.x == 0 && status) {
+    if (atomicCAS(status, 0, 1) == 0) {
+      status[1] = tile_id * 65536 + bh;
+      status[2] = where_s;
+    }
+  }
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+
 template <int E, int D>
 cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
   TcMaps maps;
@@ -365,6 +654,15 @@ cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
     maps.cv = maps.v;
   }
   if (!ok) return cudaErrorInvalidValue;
+  if constexpr (D <= 128) {
+    if (std::getenv("THIN_ATTN_TC1") == nullptr) {
+      const size_t sm = Tc2Layout<E, D>::BYTES;
+      cudaError_t e = cudaFuncSetAttribute(attn_tc2_kernel<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if (e != cudaSuccess) return e;
+      attn_tc2_kernel<E, D><<<dim3(a.n_tiles, a.B * a.H), 192, sm, st>>>(maps, a, status);
+      return cudaGetLastError();
+    }
+  }
   const size_t sm = TcLayout<E, D>::BYTES;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
