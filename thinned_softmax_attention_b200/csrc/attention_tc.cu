@@ -373,6 +373,79 @@ struct Tc2Layout {
   static constexpr uint32_t BYTES = OFF_BAR + 128 + 1024;
 };
 
+
+// Softmax of one key tile of the two-CTA kernel for the thread's row: reads S (TMEM columns
+// 0..127) twice -- row max, then P = 2^(s scale log2e + log2 w - m) as bf16 written over the S
+// columns already read (16 columns per 32 read) -- and rescales O lazily (warp-wide TMEM round
+// trip when some row's max grew by more than 2^8).  MASKED: keys c > lim are invisible.
+template <bool MASKED, int D>
+__device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, int lim, float sl2e, float lw2,
+                                             int it, float& m_used, float& l) {
+  constexpr uint32_t O_COL = 128;
+  float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    float z[32];
+    tmem_ld32(tmem + lane_base + c * 32, z);
+    tmem_ld_wait();
+    if (MASKED) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) z[i] = c * 32 + i <= lim ? z[i] : -INFINITY;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      mx4[0] = fmax3(mx4[0], z[i], z[i + 1]);
+      mx4[1] = fmax3(mx4[1], z[i + 2], z[i + 3]);
+      mx4[2] = fmax3(mx4[2], z[i + 4], z[i + 5]);
+      mx4[3] = fmax3(mx4[3], z[i + 6], z[i + 7]);
+    }
+  }
+  const float smax = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+  const float mx = smax == -INFINITY ? -INFINITY : fmaf(smax, sl2e, lw2);
+  const bool grow = mx > m_used + 8.f;
+  float corr = 1.f;
+  if (grow) {
+    corr = ex2_approx(m_used - mx);
+    l *= corr;
+    m_used = mx;
+  }
+  if (it > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] *= corr;
+      tmem_st32(tmem + lane_base + O_COL + c * 32, o);
+    }
+  }
+  const float off = m_used == -INFINITY ? 0.f : lw2 - m_used;
+  float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    float z[32];
+    tmem_ld32(tmem + lane_base + c * 32, z);
+    tmem_ld_wait();
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float z0 = z[2 * e], z1 = z[2 * e + 1];
+      if (MASKED) {
+        z0 = c * 32 + 2 * e <= lim ? z0 : -INFINITY;
+        z1 = c * 32 + 2 * e + 1 <= lim ? z1 : -INFINITY;
+      }
+      const float p0 = ex2_approx(fmaf(z0, sl2e, off));
+      const float p1 = ex2_approx(fmaf(z1, sl2e, off));
+      ls[e & 3] += p0 + p1;
+      const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
+      pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+    }
+    tmem_st16(tmem + lane_base + c * 16, pk);
+  }
+  l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+}
+
 template <int E, int D>
 __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a,
                                                           int* status) {
@@ -527,67 +600,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
         const bool causal = sg.kind == SEG_TOKENS && sg.causal;
         const bool masked = nvalid < BN || (causal && kt0 + BN - 1 > tile.q0);
         const int lim = min(nvalid - 1, causal ? tq - kt0 : BN - 1);
-        // pass 1: row max of the raw scores
-        float mx8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          float z[32];
-          tmem_ld32(tmem + lane_base + c * 32, z);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float v = (!masked || c * 32 + i <= lim) ? z[i] : -INFINITY;
-            mx8[i & 7] = fmaxf(mx8[i & 7], v);
-          }
-        }
-        const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float mx = smax == -INFINITY ? -INFINITY : fmaf(smax, a.scale_log2e, lw2);
-        // lazy rescale of O and l (PV of the previous tile is complete: S of this tile was
-        // issued after it)
-        const bool grow = mx > m_used + 8.f;
-        float corr = 1.f;
-        if (grow) {
-          corr = ex2_approx(m_used - mx);
-          l *= corr;
-          m_used = mx;
-        }
-        if (it > 0 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= corr;
-            tmem_st32(tmem + lane_base + O_COL + c * 32, o);
-          }
-        }
-        // pass 2: P = 2^(s scale log2e + log2 w - m) as bf16 into TMEM columns 16c..16c+15; they
-        // overlap only S columns already read
-        const float off = m_used == -INFINITY ? 0.f : lw2 - m_used;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          float z[32];
-          tmem_ld32(tmem + lane_base + c * 32, z);
-          tmem_ld_wait();
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float z0 = (!masked || c * 32 + 2 * e <= lim) ? z[2 * e] : -INFINITY;
-            const float z1 = (!masked || c * 32 + 2 * e + 1 <= lim) ? z[2 * e + 1] : -INFINITY;
-            const float p0 = ex2_approx(fmaf(z0, a.scale_log2e, off));
-            const float p1 = ex2_approx(fmaf(z1, a.scale_log2e, off));
-            ls[e & 3] += p0 + p1;
-            const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
-          }
-          tmem_st16(tmem + lane_base + c * 16, pk);
-        }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        if (masked) softmax_tile<true, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l);
+        else softmax_tile<false, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);

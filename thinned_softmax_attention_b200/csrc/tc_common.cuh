@@ -54,6 +54,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
+// max(a, b, c) in one instruction (three-input max.f32 of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 2^x with the MUFU.EX2 instruction (ex2.approx.ftz): 2^-inf = +0.
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
