@@ -138,6 +138,21 @@ __device__ __forceinline__ PointRef point_ref(const StepArgs& a, const HalveInst
   return r;
 }
 
+// Element offsets of the K and V rows of point p (no token-index lookup).
+__device__ __forceinline__ void point_rows(const StepArgs& a, const HalveInst& in, int p, uint32_t U, int64_t* krow,
+                                           int64_t* vrow) {
+  int64_t row;
+  if (a.src_kind == SRC_TOKENS) {
+    const int64_t gp = 2 * (int64_t)in.pair0 + p;
+    const int64_t t = (a.S_sub < a.S_full) ? (gp * a.S_full + U) / a.S_sub : gp;
+    row = (in.src_row + t) * a.H + (int)(in.bh % (uint32_t)a.H);
+  } else {
+    row = in.src_row + p;
+  }
+  *krow = row * a.E;
+  *vrow = row * a.D;
+}
+
 // ---------------------------------------------------------------------------
 // Attention over key segments.
 // ---------------------------------------------------------------------------

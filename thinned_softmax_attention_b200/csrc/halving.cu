@@ -49,8 +49,9 @@ __global__ void __launch_bounds__(256) c2_kernel(StepArgs a) {
   float mx = 0.f;
   for (int e = threadIdx.x; e < a.n * cpp; e += blockDim.x) {
     const int p = e / cpp, c = e - p * cpp;
-    const PointRef r = point_ref(a, in, p, U_s);
-    const uint4 w = V[r.vrow / epc + c];
+    int64_t kr, vr;
+    point_rows(a, in, p, U_s, &kr, &vr);
+    const uint4 w = V[vr / epc + c];
     if (sizeof(T) == 2) {
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -284,23 +285,57 @@ __device__ __forceinline__ float sigma_step(float& sigma, float b2, float b, flo
   return a;
 }
 
-// Gather the kept point of pair i (keep = first point) into destination row dst_row + i.
-template <typename T>
-__device__ __forceinline__ void gather_row(const StepArgs& a, const HalveInst& in, uint32_t U, int i, bool keep,
-                                           int lane) {
-  const int kw = a.E * (int)sizeof(T) / 16, vw = a.D * (int)sizeof(T) / 16;
+// Gather the kept point of pairs [i0, i1) (bit i of `bits(i)` set = first point kept) into
+// destination rows dst_row + i, by one warp.  Lane l resolves pair i0 + 32q + l; the warp then
+// copies the rows four at a time with all their 16-byte loads in flight before the stores.
+template <typename T, typename Bits>
+__device__ __forceinline__ void gather_pairs(const StepArgs& a, const HalveInst& in, uint32_t U, int i0, int i1,
+                                             Bits bits, int lane) {
+  const int kw = a.E * (int)sizeof(T) / 16, vw = a.D * (int)sizeof(T) / 16, rw = kw + vw;
   const int epw = 16 / (int)sizeof(T);
-  const PointRef r = point_ref(a, in, 2 * i + (keep ? 0 : 1), U);
-  const int64_t drow = in.dst_row + i;
   const uint4* K = (const uint4*)a.srcK;
   const uint4* V = (const uint4*)a.srcV;
   uint4* dK = (uint4*)a.dstK;
   uint4* dV = (uint4*)a.dstV;
-  for (int w = lane; w < kw + vw; w += 32) {
-    if (w < kw) dK[drow * kw + w] = K[r.krow / epw + w];
-    else dV[drow * vw + (w - kw)] = V[r.vrow / epw + (w - kw)];
+  for (int g = i0; g < i1; g += 32) {
+    const int i = g + lane;
+    int64_t kr = 0, vr = 0;
+    if (i < i1) {
+      const bool keep = bits(i);
+      const int pnt = 2 * i + (keep ? 0 : 1);
+      point_rows(a, in, pnt, U, &kr, &vr);
+      a.dstIdx[in.dst_row + i] =
+          a.src_kind == SRC_TOKENS ? (int32_t)(in.tok0 + (int)(kr / a.E / a.H - in.src_row)) : a.srcIdx[in.src_row + pnt];
+    }
+    kr /= epw;
+    vr /= epw;
+    const int nrows = min(32, i1 - g);
+    for (int j = 0; j < nrows; j += 4) {
+      uint4 buf[4][4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int64_t krj = __shfl_sync(0xffffffffu, kr, (j + jj) & 31);
+        const int64_t vrj = __shfl_sync(0xffffffffu, vr, (j + jj) & 31);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int w = lane + 32 * q;
+          if (j + jj < nrows && w < rw) buf[jj][q] = w < kw ? K[krj + w] : V[vrj + (w - kw)];
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int64_t drow = in.dst_row + g + j + jj;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int w = lane + 32 * q;
+          if (j + jj < nrows && w < rw) {
+            if (w < kw) dK[drow * kw + w] = buf[jj][q];
+            else dV[drow * vw + (w - kw)] = buf[jj][q];
+          }
+        }
+      }
+    }
   }
-  if (lane == 0) a.dstIdx[drow] = r.idx;
 }
 
 // Walk of instances with m <= 32 pairs: one warp per instance.  Lane l holds column l of the
@@ -335,7 +370,7 @@ __global__ void __launch_bounds__(128) walk_small_kernel(StepArgs a) {
     }
   }
   if (a.trace && lane == 0) a.trace[a.trace_base + inst] = kb;
-  for (int i = 0; i < m; ++i) gather_row<T>(a, in, U, i, (kb >> i) & 1u, lane);
+  gather_pairs<T>(a, in, U, 0, m, [kb](int i) { return ((kb >> i) & 1u) != 0; }, lane);
 }
 
 // Walk of instances with 32 < m <= 256 pairs: one CTA of 128 threads per instance.  The 32 rows
@@ -426,7 +461,9 @@ __global__ void __launch_bounds__(128) walk_mid_kernel(StepArgs a) {
   if (a.trace)
     for (int w = tid; w < nb; w += 128) a.trace[a.trace_base + (size_t)inst * nb + w] = bits[w];
   const uint32_t U = sub_offset(a, in);
-  for (int i = warp; i < m; i += 4) gather_row<T>(a, in, U, i, (bits[i >> 5] >> (i & 31)) & 1u, lane);
+  const int per = (m + 3) / 4;
+  gather_pairs<T>(a, in, U, warp * per, min(m, (warp + 1) * per),
+                  [bits](int i) { return ((bits[i >> 5] >> (i & 31)) & 1u) != 0; }, lane);
 }
 
 // Copy runs of tokens unchanged into compact rows (Express batches that need no thinning).
