@@ -274,15 +274,12 @@ __global__ void __launch_bounds__(128, 8) walk_kernel(StepArgs a) {
 // a = max(b sigma C, b^2) written out (in the first, sigma <= b/C < b gives sigma'^2 = b^2).
 // Returns a; sigma is updated in place.  b^2 <= 0 (a repeated point) keeps sigma and returns 0.
 __device__ __forceinline__ float sigma_step(float& sigma, float b2, float b, float C, float q, float r2) {
-  if (!(b2 > 0.f)) return 0.f;
   const float sc = sigma * C;
-  if (b >= sc) {
-    sigma = b;
-    return b2;
-  }
-  const float a = b * sc;
-  sigma = sqrt_approx(fmaf(sigma, sigma, fmaxf(0.f, fmaf(-r2, sigma, q))));
-  return a;
+  const bool first = b >= sc;
+  const float s_else = sqrt_approx(fmaf(sigma, sigma, fmaxf(0.f, fmaf(-r2, sigma, q))));
+  const bool live = b2 > 0.f;
+  sigma = live ? (first ? b : s_else) : sigma;
+  return first ? b2 : b * sc;
 }
 
 // Gather the kept point of pairs [i0, i1) (bit i of `bits(i)` set = first point kept) into
@@ -356,18 +353,18 @@ __global__ void __launch_bounds__(128) walk_small_kernel(StepArgs a) {
   const float C = a.C, cq = 1.f + 1.f / (C * C), c2C = 2.f / C;
   float my = 0.f, sigma = 0.f;
   uint32_t kb = 0;
+  // Pairs s >= m are no-ops: their Delta entries are 0, so b^2 = 0 keeps sigma and alpha as they
+  // are, and their bits are never read.
 #pragma unroll
   for (int s = 0; s < 32; ++s) {
-    if (s < m) {
-      const float b2 = __shfl_sync(0xffffffffu, d[s], s);
-      const float w = __shfl_sync(0xffffffffu, w_l, s);
-      const float b = sqrt_approx(fmaxf(b2, 0.f));
-      const float av = sigma_step(sigma, b2, b, C, b2 * cq, b * c2C);
-      const float ai = __shfl_sync(0xffffffffu, my, s);
-      const bool keep = !(b2 > 0.f) || ai < av * w;
-      if (lane > s) my = fmaf(keep ? 1.f : -1.f, d[s], my);
-      kb |= (uint32_t)keep << s;
-    }
+    const float b2 = __shfl_sync(0xffffffffu, d[s], s);
+    const float w = __shfl_sync(0xffffffffu, w_l, s);
+    const float b = sqrt_approx(fmaxf(b2, 0.f));
+    const float av = sigma_step(sigma, b2, b, C, b2 * cq, b * c2C);
+    const float ai = __shfl_sync(0xffffffffu, my, s);
+    const bool keep = !(b2 > 0.f) || ai < av * w;
+    if (lane > s) my = fmaf(keep ? 1.f : -1.f, d[s], my);
+    kb |= (uint32_t)keep << s;
   }
   if (a.trace && lane == 0) a.trace[a.trace_base + inst] = kb;
   gather_pairs<T>(a, in, U, 0, m, [kb](int i) { return ((kb >> i) & 1u) != 0; }, lane);
@@ -433,18 +430,18 @@ __global__ void __launch_bounds__(128) walk_mid_kernel(StepArgs a) {
       const float wl = wbuf[base + lane];
       float my = alpha[base + lane];
       uint32_t kb = 0;
+      // Pairs s >= steps are no-ops (b^2 = 0 keeps sigma; they only touch alpha of lanes that are
+      // no pair), so the 32 steps run without a guard.
 #pragma unroll
       for (int s = 0; s < 32; ++s) {
-        if (s < steps) {
-          const float b2 = __shfl_sync(0xffffffffu, dl, s);
-          const float b = __shfl_sync(0xffffffffu, bl, s);
-          const float w = __shfl_sync(0xffffffffu, wl, s);
-          const float av = sigma_step(sigma, b2, b, C, b2 * cq, b * c2C);
-          const float ai = __shfl_sync(0xffffffffu, my, s);
-          const bool keep = !(b2 > 0.f) || ai < av * w;
-          if (lane > s) my = fmaf(keep ? 1.f : -1.f, R[s * mp + base + lane], my);
-          kb |= (uint32_t)keep << s;
-        }
+        const float b2 = __shfl_sync(0xffffffffu, dl, s);
+        const float b = __shfl_sync(0xffffffffu, bl, s);
+        const float w = __shfl_sync(0xffffffffu, wl, s);
+        const float av = sigma_step(sigma, b2, b, C, b2 * cq, b * c2C);
+        const float ai = __shfl_sync(0xffffffffu, my, s);
+        const bool keep = !(b2 > 0.f) || ai < av * w;
+        if (lane > s) my = fmaf(keep ? 1.f : -1.f, R[s * mp + base + lane], my);
+        kb |= (uint32_t)keep << s;
       }
       if (lane == 0) bits[t] = kb;
     }
