@@ -218,6 +218,25 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+def rank_workload(w, rank):
+    """Weak scaling: rank r runs its own independent problem of the same size (data seed + 1000 r)."""
+    return w.with_(data_seed=w.data_seed + 1000 * rank) if rank else w
+
+
+def max_over_ranks(x, dist, device):
+    """Max of a per-rank scalar over all ranks (the step time the job is bound by)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, tokens_per_rank, ms):
+    """Whole-job throughput: the tokens every rank processed over the slowest rank's step time."""
+    return world * tokens_per_rank / (ms * 1e-3)
+
+
 def config_of(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "S": w.T if w.causal else w.S, "E": w.E, "D": w.D,
             "causal": w.causal, "g": w.g, "n_exact": w.n_exact, "batch": w.batch, "seed": w.seed,
@@ -241,7 +260,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     w = W.WORKLOADS[a.workload]
     # each rank an independent problem of the same size (weak scaling)
-    wr = w.with_(data_seed=w.data_seed + 1000 * rank) if rank else w
+    wr = rank_workload(w, rank)
     q, k, v = (x.to(dev) for x in W.make_qkv(wr))
     S = w.T if w.causal else w.S
     h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch,
@@ -275,13 +294,9 @@ def main():
     clk = clocks.stop()
     h.profile(False)
     ph = h.profile_read()
-    ms = e0.elapsed_time(e1) / a.steps
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / a.steps, dist, dev)
     tokens = w.B * w.H * w.T
-    value = world * tokens / (ms * 1e-3)
+    value = job_value(world, tokens, ms)
 
     # dominant kernel roofline: attention
     pk = peaks()
@@ -313,13 +328,9 @@ def main():
             h.forward_host(qh, kh, vh, oh, causal=w.causal, g=w.g, seed=w.seed)
         f1.record(stream)
         torch.cuda.synchronize()
-        ems = f0.elapsed_time(f1) / n_e2e
-        if dist:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(f0.elapsed_time(f1) / n_e2e, dist, dev)
         es = 4 if w.dtype == "fp32" else 2
-        e2e = {"value": world * tokens / (ems * 1e-3), "unit": UNIT,
+        e2e = {"value": job_value(world, tokens, ems), "unit": UNIT,
                "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * es,
                "d2h_bytes_per_step": out.numel() * es, "ms_per_step": round(ems, 3)}
 

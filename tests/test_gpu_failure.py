@@ -1,0 +1,36 @@
+"""Failure detection on the GPU without a fault: a bounded wait that runs out.
+
+With THIN_ATTN_INJECT_WAIT_TIMEOUT set, the attention kernel's first CTA withholds its first
+key tile, so its MMA issuer's bounded wait gives up (~0.2 s).  The CTA records the site in the
+handle's status word and exits through its normal path (tensor memory freed, no copy in flight);
+thin_attn_check must report THIN_ATTN_ETIMEOUT, and the next forward on the same context must
+run and match the oracle-checked result.
+"""
+import os
+
+import pytest
+import torch
+
+import thinned_softmax_attention_b200 as TA
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    w = W.WORKLOADS["express32k"].with_(H=2, n_exact=256, batch=256)
+    q, k, v = (x.cuda() for x in W.make_qkv(w, T=1024))
+    h = TA.ThinAttention(w.B, 1024, 1024, w.H, w.E, w.D, w.torch_dtype, n_exact=256, batch=256)
+    good = h.forward(q, k, v, causal=True, g=2, seed=3)["out"].clone()
+    h.check()
+    os.environ["THIN_ATTN_INJECT_WAIT_TIMEOUT"] = "1"
+    try:
+        h.forward(q, k, v, causal=True, g=2, seed=3)
+        with pytest.raises(TA.ThinAttnError, match="ETIMEOUT") as ei:
+            h.check()
+        assert "query tile" in str(ei.value)      # the site of the wait that gave up is reported
+    finally:
+        del os.environ["THIN_ATTN_INJECT_WAIT_TIMEOUT"]
+    again = h.forward(q, k, v, causal=True, g=2, seed=3)["out"]
+    h.check()
+    assert torch.equal(again, good)

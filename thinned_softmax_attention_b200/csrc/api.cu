@@ -603,6 +603,8 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   aa.n_slots = p->att_slots;
   aa.slot_rows = p->att_slot_rows;
   aa.scale_log2e = (float)((double)h->scale * 1.4426950408889634);
+  // Test hook for failure detection: one CTA's bounded wait runs out (no fault, no hang).
+  aa.inject_timeout = std::getenv("THIN_ATTN_INJECT_WAIT_TIMEOUT") != nullptr;
   bool done = false;
   if (!p->tc.tiles.empty() && std::getenv("THIN_ATTN_SIMT_ATTN") == nullptr) {
     aa.tiles = (const AttnTile*)(base_of(p) + p->tc.tiles_off);

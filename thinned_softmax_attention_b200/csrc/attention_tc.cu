@@ -513,11 +513,14 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
             atomicCAS((int*)&where_s, 0, 1000 + min(it, 999));
             break;
           }
-          mbar_expect_tx(k_full, Lay::K_BYTES);
+          const bool withhold = a.inject_timeout && it == 0 && blockIdx.x == 0 && blockIdx.y == 0;
+          if (!withhold) {
+            mbar_expect_tx(k_full, Lay::K_BYTES);
 #pragma unroll
-          for (int c = 0; c < Lay::EC; ++c) {
-            if (tok) tma_load_3d(sK + c * 16384, &maps.k, k_full, c * 64, h, row);
-            else tma_load_2d(sK + c * 16384, &maps.ck, k_full, c * 64, row);
+            for (int c = 0; c < Lay::EC; ++c) {
+              if (tok) tma_load_3d(sK + c * 16384, &maps.k, k_full, c * 64, h, row);
+              else tma_load_2d(sK + c * 16384, &maps.ck, k_full, c * 64, row);
+            }
           }
           if (it > 0 && !mbar_wait(v_empty, (it - 1) & 1, abort)) {
             ok = false;
@@ -534,9 +537,10 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
       }
       // never leave with a copy in flight into this CTA's shared memory
       if (it > 0) {
-        const long long t0 = clock64();
+        long long t0 = clock64();
         while (!mbar_try_wait(k_full, (it - 1) & 1) && clock64() - t0 < kWaitCycles) {
         }
+        t0 = clock64();
         while (!mbar_try_wait(v_full, (it - 1) & 1) && clock64() - t0 < kWaitCycles) {
         }
       }

@@ -189,6 +189,7 @@ struct AttnArgs {
   int B, T, L, H, E, D;
   int n_slots, slot_rows;
   float scale_log2e;
+  int inject_timeout;   // test hook: CTA (0,0) withholds its first key tile so a bounded wait runs out
 };
 
 }  // namespace thin
