@@ -150,9 +150,10 @@ THIN_ATTN_API thin_attn_status thin_attn_forward_host(thin_attn_t h, const void*
  * attention).  No effect on results. */
 THIN_ATTN_API thin_attn_status thin_attn_profile(thin_attn_t h, int enable);
 
-/* Wait for the recorded forwards and return their summed phase times in
- * milliseconds: ms[0] thinning, ms[1] merges, ms[2] attention, ms[3] total;
- * *calls = forwards recorded.  Resets the sums. */
+/* Wait for the recorded forwards and return their summed times in milliseconds:
+ * ms[0] thinning of sequences or batches, ms[1] HALVE merges, ms[2] attention (the
+ * summed durations of its launches, which may overlap the halving steps), ms[3] the
+ * whole forward; *calls = forwards recorded.  Resets the sums. */
 THIN_ATTN_API thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms, int* calls);
 
 /* Synchronise `stream` and report a device-side failure recorded by the

@@ -79,6 +79,7 @@ struct BufSpec {
 struct StepPlan {
   bool copy_only = false;
   int phase = 0;   // 0: thinning of sequences / batches, 1: HALVE merges
+  int merge_level = 0;   // phase 1: target level of the merge
   int src_buf = BUF_TOKENS, dst_buf = 0;
   int n = 0, m = 0, m_pad = 0;
   int S_full = 0, S_sub = 0;
@@ -87,10 +88,17 @@ struct StepPlan {
   uint64_t trace_base = 0;
 };
 
+// A wave: consecutive attention tiles that can run as soon as halving step `after` (and all
+// earlier steps) has run; after = -1: as soon as the forward starts.
+struct AttnWave {
+  int tile0, count, after;
+};
+
 struct AttnTables {
   int rows_per_tile = 0;
   std::vector<AttnTile> tiles;
   std::vector<AttnSeg> segs;
+  std::vector<AttnWave> waves;
   size_t tiles_off = 0, segs_off = 0;
 };
 
@@ -132,10 +140,16 @@ struct thin_attn_s {
   // host-buffer staging
   void* st_mem = nullptr;
   size_t st_bytes = 0;
-  // per-phase device timing (thin_attn_profile)
+  // side stream of the attention waves and its fork/join events
+  cudaStream_t side = nullptr, main = nullptr;
+  cudaEvent_t ev_join = nullptr, ev_join2 = nullptr, ev_fork = nullptr;
+  std::vector<cudaEvent_t> ev_dep;
+  // per-phase device timing (thin_attn_profile): event sets and their wave counts
   bool prof_on = false;
-  std::vector<std::vector<cudaEvent_t>> prof_pending, prof_free;
+  std::vector<std::pair<std::vector<cudaEvent_t>, size_t>> prof_pending;
+  std::vector<std::vector<cudaEvent_t>> prof_free;
   double prof_ms[3] = {0, 0, 0};
+  double prof_total = 0;
   int prof_calls = 0;
 };
 
@@ -157,6 +171,40 @@ struct DeviceGuard {
     if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
   }
 };
+
+// Wave structure of the tiles: a tile of Express batch k reads the nodes present after k
+// completed batches, whose highest level is floor(log4 k); it can run once the batch thinning
+// (k >= 1) and the merges up to that level are done.  Exact-phase tiles and batch 0 read no node.
+void build_waves(const thin_attn_config& cf, const Plan& p, AttnTables& t) {
+  t.waves.clear();
+  const int n_steps = (int)p.steps.size();
+  int last_thin = -1;
+  std::vector<int> last_merge;
+  for (int i = 0; i < n_steps; ++i) {
+    if (p.steps[i].phase == 0) last_thin = i;
+    else {
+      const int lv = p.steps[i].merge_level;
+      if ((int)last_merge.size() <= lv) last_merge.resize(lv + 1, -1);
+      last_merge[lv] = i;
+    }
+  }
+  const int ne = std::min(cf.n_exact, cf.T);
+  for (int i = 0; i < (int)t.tiles.size(); ++i) {
+    int after = n_steps - 1;
+    if (p.causal) {
+      const int q0 = t.tiles[i].q0;
+      const int64_t k = q0 < ne ? -1 : (q0 - ne) / cf.batch;
+      if (k <= 0) after = -1;
+      else {
+        int lv = 0;
+        while (((int64_t)1 << (2 * (lv + 1))) <= k) ++lv;
+        after = lv == 0 ? last_thin : (lv < (int)last_merge.size() ? last_merge[lv] : n_steps - 1);
+      }
+    }
+    if (!t.waves.empty() && t.waves.back().after == after) t.waves.back().count++;
+    else t.waves.push_back({i, 1, after});
+  }
+}
 
 void build_attn_tables(const thin_attn_config& cf, const Plan& p, int QT, AttnTables& t) {
   t.rows_per_tile = QT;
@@ -341,6 +389,7 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
         for (int step = 0; step < 2; ++step) {
           StepPlan st;
           st.phase = 1;
+          st.merge_level = lv;
           st.n = (step == 0 ? 4 : 2) * p->c;
           st.m = st.n / 2;
           st.m_pad = (st.m + 31) / 32 * 32;
@@ -383,7 +432,11 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
     p->c2_floats = std::max(p->c2_floats, st.inst.size());
   }
   build_attn_tables(cf, *p, attention_simt_tile_rows(), p->simt);
-  if (attention_tc_supported(cf.dtype, cf.E, cf.D)) build_attn_tables(cf, *p, attention_tc_tile_rows(), p->tc);
+  build_waves(cf, *p, p->simt);
+  if (attention_tc_supported(cf.dtype, cf.E, cf.D)) {
+    build_attn_tables(cf, *p, attention_tc_tile_rows(), p->tc);
+    build_waves(cf, *p, p->tc);
+  }
   // memory layout: tables first, then buffers
   size_t off = 0;
   for (auto& st : p->steps) {
@@ -514,19 +567,101 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
                              uint64_t seed, float* lse, int32_t* cidx, uint32_t* trace, cudaStream_t st) {
   const thin_attn_config& cf = h->cfg;
   const bool use_tc_gram = std::getenv("THIN_ATTN_SIMT_GRAM") == nullptr;
+  const bool use_tc_attn = !p->tc.tiles.empty() && tensor_maps_available() && std::getenv("THIN_ATTN_SIMT_ATTN") == nullptr;
+  const AttnTables& tab = use_tc_attn ? p->tc : p->simt;
+  // Attention waves run on a side stream, each after the halving step it depends on, so the
+  // tensor cores work while later (latency-bound) halving steps run.  One wave: caller's stream.
+  const bool side = tab.waves.size() > 1 && std::getenv("THIN_ATTN_SERIAL") == nullptr;
+  cudaStream_t sa = st;
+  cudaStream_t caller = st;
+  if (side) {
+    // halving steps on a high-priority stream (their CTAs are dispatched ahead of pending
+    // attention CTAs), attention waves on a low-priority one; both fork from and join back
+    // into the caller's stream
+    if (!h->side) {
+      int lo = 0, hi = 0;
+      CK(cudaDeviceGetStreamPriorityRange(&lo, &hi));
+      CK(cudaStreamCreateWithPriority(&h->side, cudaStreamNonBlocking, lo));
+      CK(cudaStreamCreateWithPriority(&h->main, cudaStreamNonBlocking, hi));
+      CK(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
+      CK(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
+      CK(cudaEventCreateWithFlags(&h->ev_join2, cudaEventDisableTiming));
+    }
+    while (h->ev_dep.size() < tab.waves.size() + 1) {
+      cudaEvent_t e;
+      CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+      h->ev_dep.push_back(e);
+    }
+    CK(cudaEventRecord(h->ev_fork, caller));
+    CK(cudaStreamWaitEvent(h->main, h->ev_fork, 0));
+    CK(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+    st = h->main;
+    sa = h->side;
+  }
+  // profiling events: [0] start, [1] first merge step, [2] all halving steps, [3] end (joined),
+  // then a (start, stop) pair per attention wave on the attention stream
   std::vector<cudaEvent_t> ev;
   if (h->prof_on) {
-    if (!h->prof_free.empty()) {
+    const size_t need = 4 + 2 * tab.waves.size();
+    if (!h->prof_free.empty() && h->prof_free.back().size() >= need) {
       ev = h->prof_free.back();
       h->prof_free.pop_back();
     } else {
-      ev.resize(4);
+      ev.resize(need);
       for (auto& e : ev) CK(cudaEventCreate(&e));
     }
     CK(cudaEventRecord(ev[0], st));
   }
+  AttnArgs aa{};
+  aa.q = q;
+  aa.k = k;
+  aa.v = v;
+  if (p->final_buf != BUF_TOKENS) {
+    int32_t* didx;
+    buf_ptrs(p, p->final_buf, k, v, &aa.ck, &aa.cv, &didx);
+  }
+  aa.out = out;
+  aa.lse = lse;
+  aa.B = cf.B;
+  aa.T = cf.T;
+  aa.L = p->causal ? cf.T : cf.S;
+  aa.H = cf.H;
+  aa.E = cf.E;
+  aa.D = cf.D;
+  aa.n_slots = p->att_slots;
+  aa.slot_rows = p->att_slot_rows;
+  aa.scale_log2e = (float)((double)h->scale * 1.4426950408889634);
+  // Test hook for failure detection: one CTA's bounded wait runs out (no fault, no hang).
+  aa.inject_timeout = std::getenv("THIN_ATTN_INJECT_WAIT_TIMEOUT") != nullptr;
+  aa.tiles = (const AttnTile*)(base_of(p) + tab.tiles_off);
+  aa.segs = (const AttnSeg*)(base_of(p) + tab.segs_off);
+  size_t next_wave = 0, dep_i = 0;
+  auto launch_waves_after = [&](int step) -> thin_attn_status {
+    while (next_wave < tab.waves.size() && tab.waves[next_wave].after <= step) {
+      const AttnWave& w = tab.waves[next_wave];
+      if (side) {
+        CK(cudaEventRecord(h->ev_dep[dep_i], st));
+        CK(cudaStreamWaitEvent(sa, h->ev_dep[dep_i], 0));
+        ++dep_i;
+      }
+      aa.tile0 = w.tile0;
+      aa.n_tiles = w.count;
+      if (!ev.empty()) CK(cudaEventRecord(ev[4 + 2 * next_wave], sa));
+      bool done = false;
+      cudaError_t e = cudaSuccess;
+      if (use_tc_attn) e = launch_attention_tc(aa, h->d_status, sa, &done);
+      if (e == cudaSuccess && !done) e = launch_attention_simt(aa, cf.dtype, sa);
+      if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "attention: %s", cudaGetErrorString(e));
+      if (!ev.empty()) CK(cudaEventRecord(ev[5 + 2 * next_wave], sa));
+      ++next_wave;
+    }
+    return THIN_ATTN_OK;
+  };
+  thin_attn_status ls = launch_waves_after(-1);
+  if (ls != THIN_ATTN_OK) return ls;
   bool merged_mark = false;
-  for (auto& sp : p->steps) {
+  for (size_t si = 0; si < p->steps.size(); ++si) {
+    const StepPlan& sp = p->steps[si];
     if (!ev.empty() && sp.phase == 1 && !merged_mark) {
       CK(cudaEventRecord(ev[1], st));
       merged_mark = true;
@@ -568,11 +703,15 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     cudaError_t e = sp.copy_only ? launch_copy_step(a, cf.dtype, st)
                                  : launch_halving_step(a, cf.dtype, use_tc_gram, st);
     if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "halving step (n=%d): %s", sp.n, cudaGetErrorString(e));
+    ls = launch_waves_after((int)si);
+    if (ls != THIN_ATTN_OK) return ls;
   }
   if (!ev.empty()) {
     if (!merged_mark) CK(cudaEventRecord(ev[1], st));
     CK(cudaEventRecord(ev[2], st));
   }
+  ls = launch_waves_after((int)p->steps.size());
+  if (ls != THIN_ATTN_OK) return ls;
   if (cidx) {
     if (p->final_buf == BUF_TOKENS) {
       cudaError_t e = launch_iota(cidx, (int64_t)p->coreset_idx_elems, cf.S, st);
@@ -584,45 +723,16 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
       CK(cudaMemcpyAsync(cidx, didx, p->coreset_idx_elems * 4, cudaMemcpyDeviceToDevice, st));
     }
   }
-  AttnArgs aa{};
-  aa.q = q;
-  aa.k = k;
-  aa.v = v;
-  if (p->final_buf != BUF_TOKENS) {
-    int32_t* didx;
-    buf_ptrs(p, p->final_buf, k, v, &aa.ck, &aa.cv, &didx);
-  }
-  aa.out = out;
-  aa.lse = lse;
-  aa.B = cf.B;
-  aa.T = cf.T;
-  aa.L = p->causal ? cf.T : cf.S;
-  aa.H = cf.H;
-  aa.E = cf.E;
-  aa.D = cf.D;
-  aa.n_slots = p->att_slots;
-  aa.slot_rows = p->att_slot_rows;
-  aa.scale_log2e = (float)((double)h->scale * 1.4426950408889634);
-  // Test hook for failure detection: one CTA's bounded wait runs out (no fault, no hang).
-  aa.inject_timeout = std::getenv("THIN_ATTN_INJECT_WAIT_TIMEOUT") != nullptr;
-  bool done = false;
-  if (!p->tc.tiles.empty() && std::getenv("THIN_ATTN_SIMT_ATTN") == nullptr) {
-    aa.tiles = (const AttnTile*)(base_of(p) + p->tc.tiles_off);
-    aa.segs = (const AttnSeg*)(base_of(p) + p->tc.segs_off);
-    aa.n_tiles = (int)p->tc.tiles.size();
-    cudaError_t e = launch_attention_tc(aa, h->d_status, st, &done);
-    if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "attention (tensor cores): %s", cudaGetErrorString(e));
-  }
-  if (!done) {
-    aa.tiles = (const AttnTile*)(base_of(p) + p->simt.tiles_off);
-    aa.segs = (const AttnSeg*)(base_of(p) + p->simt.segs_off);
-    aa.n_tiles = (int)p->simt.tiles.size();
-    cudaError_t e = launch_attention_simt(aa, cf.dtype, st);
-    if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "attention: %s", cudaGetErrorString(e));
+  if (side) {
+    CK(cudaEventRecord(h->ev_join, sa));
+    CK(cudaEventRecord(h->ev_join2, st));
+    CK(cudaStreamWaitEvent(caller, h->ev_join, 0));
+    CK(cudaStreamWaitEvent(caller, h->ev_join2, 0));
+    st = caller;
   }
   if (!ev.empty()) {
     CK(cudaEventRecord(ev[3], st));
-    h->prof_pending.push_back(ev);
+    h->prof_pending.push_back({ev, tab.waves.size()});
   }
   return THIN_ATTN_OK;
 }
@@ -649,7 +759,7 @@ thin_attn_status thin_attn_create(thin_attn_t* out, const thin_attn_config* cfg)
 
 thin_attn_status thin_attn_destroy(thin_attn_t h) {
   if (!h) return THIN_ATTN_OK;
-  const bool on_device = h->d_status || h->st_mem || !h->prof_free.empty() || !h->prof_pending.empty();
+  const bool on_device = h->d_status || h->st_mem || h->side || !h->prof_free.empty() || !h->prof_pending.empty();
   DeviceGuard dg(on_device ? h->cfg.device : -1);
   for (auto& kv : h->plans) {
     if (kv.second->d_mem) cudaFree(kv.second->d_mem);
@@ -657,9 +767,15 @@ thin_attn_status thin_attn_destroy(thin_attn_t h) {
   }
   if (h->d_status) cudaFree(h->d_status);
   if (h->st_mem) cudaFree(h->st_mem);
-  for (auto* lst : {&h->prof_pending, &h->prof_free})
-    for (auto& ev : *lst)
-      for (auto e : ev) cudaEventDestroy(e);
+  for (auto& pe : h->prof_pending)
+    for (auto e : pe.first) cudaEventDestroy(e);
+  for (auto& ev : h->prof_free)
+    for (auto e : ev) cudaEventDestroy(e);
+  for (auto e : h->ev_dep) cudaEventDestroy(e);
+  for (auto e : {h->ev_join, h->ev_join2, h->ev_fork})
+    if (e) cudaEventDestroy(e);
+  if (h->side) cudaStreamDestroy(h->side);
+  if (h->main) cudaStreamDestroy(h->main);
   delete h;
   return THIN_ATTN_OK;
 }
@@ -784,21 +900,28 @@ thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms, int* calls) {
   if (!h || !ms || !calls) return fail(THIN_ATTN_EINVAL, "null argument");
   std::lock_guard<std::mutex> lk(h->mu);
   DeviceGuard dg(h->prof_pending.empty() ? -1 : h->cfg.device);
-  for (auto& ev : h->prof_pending) {
+  for (auto& pe : h->prof_pending) {
+    auto& ev = pe.first;
     CK(cudaEventSynchronize(ev[3]));
-    float t[3];
-    for (int i = 0; i < 3; ++i) {
-      CK(cudaEventElapsedTime(&t[i], ev[i], ev[i + 1]));
-      h->prof_ms[i] += t[i];
+    float t;
+    CK(cudaEventElapsedTime(&t, ev[0], ev[1]));
+    h->prof_ms[0] += t;
+    CK(cudaEventElapsedTime(&t, ev[1], ev[2]));
+    h->prof_ms[1] += t;
+    for (size_t w = 0; w < pe.second; ++w) {
+      CK(cudaEventElapsedTime(&t, ev[4 + 2 * w], ev[5 + 2 * w]));
+      h->prof_ms[2] += t;
     }
+    CK(cudaEventElapsedTime(&t, ev[0], ev[3]));
+    h->prof_total += t;
     h->prof_calls += 1;
     h->prof_free.push_back(ev);
   }
   h->prof_pending.clear();
   for (int i = 0; i < 3; ++i) ms[i] = h->prof_ms[i];
-  ms[3] = h->prof_ms[0] + h->prof_ms[1] + h->prof_ms[2];
+  ms[3] = h->prof_total;
   *calls = h->prof_calls;
-  h->prof_ms[0] = h->prof_ms[1] = h->prof_ms[2] = 0;
+  h->prof_ms[0] = h->prof_ms[1] = h->prof_ms[2] = h->prof_total = 0;
   h->prof_calls = 0;
   return THIN_ATTN_OK;
 }

@@ -24,7 +24,7 @@ __global__ void __launch_bounds__(512) attn_simt_kernel(AttnArgs a) {
   float* Ks = sm;                       // SK x (E+1)
   float* Vs = Ks + SK * (E + 1);        // SK x D
   float* Qs = Vs + SK * D;              // SQ x E
-  const AttnTile tile = a.tiles[blockIdx.x];
+  const AttnTile tile = a.tiles[a.tile0 + blockIdx.x];
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const T* q = (const T*)a.q;

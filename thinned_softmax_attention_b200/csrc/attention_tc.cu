@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   __shared__ volatile int where_s;   // first wait that gave up: code * 1000 + iteration
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile_id = a.n_tiles - 1 - (int)blockIdx.x;   // heaviest (latest) query tiles first
+  const int tile_id = a.tile0 + a.n_tiles - 1 - (int)blockIdx.x;   // heaviest (latest) query tiles first
   const AttnTile tile = a.tiles[tile_id];
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int n_kt = count_key_tiles(a, tile);
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
   __shared__ volatile int where_s;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile_id = a.n_tiles - 1 - (int)blockIdx.x;
+  const int tile_id = a.tile0 + a.n_tiles - 1 - (int)blockIdx.x;
   const AttnTile tile = a.tiles[tile_id];
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int n_kt = count_key_tiles(a, tile);
@@ -513,7 +513,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
             atomicCAS((int*)&where_s, 0, 1000 + min(it, 999));
             break;
           }
-          const bool withhold = a.inject_timeout && it == 0 && blockIdx.x == 0 && blockIdx.y == 0;
+          const bool withhold = a.inject_timeout && a.tile0 == 0 && it == 0 && blockIdx.x == 0 && blockIdx.y == 0;
           if (!withhold) {
             mbar_expect_tx(k_full, Lay::K_BYTES);
 #pragma unroll

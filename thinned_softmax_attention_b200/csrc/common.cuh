@@ -185,7 +185,8 @@ struct AttnArgs {
   float* lse;           // (B,H,T) or null
   const AttnTile* tiles;
   const AttnSeg* segs;
-  int n_tiles;
+  int tile0;            // first tile of this launch
+  int n_tiles;          // tiles of this launch
   int B, T, L, H, E, D;
   int n_slots, slot_rows;
   float scale_log2e;

@@ -47,21 +47,35 @@ __global__ void __launch_bounds__(256) c2_kernel(StepArgs a) {
   const int cpp = a.D / epc;                       // chunks per point
   const uint4* V = (const uint4*)a.srcV;
   float mx = 0.f;
-  for (int e = threadIdx.x; e < a.n * cpp; e += blockDim.x) {
-    const int p = e / cpp, c = e - p * cpp;
-    int64_t kr, vr;
-    point_rows(a, in, p, U_s, &kr, &vr);
-    const uint4 w = V[vr / epc + c];
-    if (sizeof(T) == 2) {
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  const int total = a.n * cpp;
+  // 8 independent 16-byte loads in flight per thread
+  for (int e0 = threadIdx.x; e0 < total; e0 += 8 * blockDim.x) {
+    uint4 w[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float lo = __uint_as_float(ws[i] << 16), hi = __uint_as_float(ws[i] & 0xFFFF0000u);
-        mx = fmaxf(mx, fmaxf(fabsf(lo), fabsf(hi)));
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + u * blockDim.x;
+      if (e < total) {
+        const int p = e / cpp, c = e - p * cpp;
+        int64_t kr, vr;
+        point_rows(a, in, p, U_s, &kr, &vr);
+        w[u] = V[vr / epc + c];
+      } else {
+        w[u] = make_uint4(0, 0, 0, 0);
       }
-    } else {
-      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(w.x)), fabsf(__uint_as_float(w.y))),
-                           fmaxf(fabsf(__uint_as_float(w.z)), fabsf(__uint_as_float(w.w)))));
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (sizeof(T) == 2) {
+        const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float lo = __uint_as_float(ws[i] << 16), hi = __uint_as_float(ws[i] & 0xFFFF0000u);
+          mx = fmaxf(mx, fmaxf(fabsf(lo), fabsf(hi)));
+        }
+      } else {
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(w[u].x)), fabsf(__uint_as_float(w[u].y))),
+                             fmaxf(fabsf(__uint_as_float(w[u].z)), fabsf(__uint_as_float(w[u].w)))));
+      }
     }
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,6 +321,27 @@ __device__ __forceinline__ void gather_pairs(const StepArgs& a, const HalveInst&
     kr /= epw;
     vr /= epw;
     const int nrows = min(32, i1 - g);
+    if (rw <= 32) {
+      // one 16-byte chunk per lane per row: 8 rows in flight
+      for (int j = 0; j < nrows; j += 8) {
+        uint4 buf[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int64_t krj = __shfl_sync(0xffffffffu, kr, (j + jj) & 31);
+          const int64_t vrj = __shfl_sync(0xffffffffu, vr, (j + jj) & 31);
+          if (j + jj < nrows && lane < rw) buf[jj] = lane < kw ? K[krj + lane] : V[vrj + (lane - kw)];
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int64_t drow = in.dst_row + g + j + jj;
+          if (j + jj < nrows && lane < rw) {
+            if (lane < kw) dK[drow * kw + lane] = buf[jj];
+            else dV[drow * vw + (lane - kw)] = buf[jj];
+          }
+        }
+      }
+      continue;
+    }
     for (int j = 0; j < nrows; j += 4) {
       uint4 buf[4][4];
 #pragma unroll
