@@ -359,7 +359,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 // P (bf16, two per column) back into columns 0..63 and the PV MMA reads it from there as its A
 // operand; O accumulates in columns 128..128+D.  K and V have one stage each with separate
 // barriers: K(j+1) loads as soon as S(j) is done, V(j+1) as soon as PV(j) is done.  The MMA
-// thread issues S(j+1) only after PV(j) has completed, so P(j) is never overwritten early.
+// thread issues S(j+1) right after PV(j): the tensor-core pipeline runs one thread's MMAs in
+// issue order, so PV(j) reads P(j) before S(j+1) overwrites it.
 // The softmax reads S twice (max pass, then exponent pass) to stay within 170 registers.
 template <int E, int D>
 struct Tc2Layout {
@@ -556,7 +557,10 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
       const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
       bool ok = mbar_wait(q_full, 0, abort);
       for (int it = 0; it < n_kt && ok; ++it) {
-        if (!mbar_wait(k_full, it & 1, abort) || (it > 0 && !mbar_wait(pv_done, (it - 1) & 1, abort))) {
+        // No wait for PV(it-1) before S(it) overwrites the P columns it reads: tcgen05.mma ops
+        // issued by one thread execute in issue order, and the commit after S(it) tracks PV(it-1)
+        // too, so s_full(it) also tells the softmax that O is complete up to tile it-1.
+        if (!mbar_wait(k_full, it & 1, abort)) {
           atomicCAS((int*)&where_s, 0, 3000 + min(it, 999));
           break;
         }

@@ -299,7 +299,7 @@ __device__ __forceinline__ float sigma_step(float& sigma, float b2, float b, flo
 // Gather the kept point of pairs [i0, i1) (bit i of `bits(i)` set = first point kept) into
 // destination rows dst_row + i, by one warp.  Lane l resolves pair i0 + 32q + l; the warp then
 // copies the rows four at a time with all their 16-byte loads in flight before the stores.
-template <typename T, typename Bits>
+template <typename T, bool WIDE, typename Bits>
 __device__ __forceinline__ void gather_pairs(const StepArgs& a, const HalveInst& in, uint32_t U, int i0, int i1,
                                              Bits bits, int lane) {
   const int kw = a.E * (int)sizeof(T) / 16, vw = a.D * (int)sizeof(T) / 16, rw = kw + vw;
@@ -321,7 +321,7 @@ __device__ __forceinline__ void gather_pairs(const StepArgs& a, const HalveInst&
     kr /= epw;
     vr /= epw;
     const int nrows = min(32, i1 - g);
-    if (rw <= 32) {
+    if (WIDE && rw <= 32) {
       // one 16-byte chunk per lane per row: 8 rows in flight
       for (int j = 0; j < nrows; j += 8) {
         uint4 buf[8];
@@ -402,7 +402,7 @@ __global__ void __launch_bounds__(128) walk_small_kernel(StepArgs a) {
     kb |= (uint32_t)keep << s;
   }
   if (a.trace && lane == 0) a.trace[a.trace_base + inst] = kb;
-  gather_pairs<T>(a, in, U, 0, m, [kb](int i) { return ((kb >> i) & 1u) != 0; }, lane);
+  gather_pairs<T, false>(a, in, U, 0, m, [kb](int i) { return ((kb >> i) & 1u) != 0; }, lane);
 }
 
 // Walk of instances with 32 < m <= 256 pairs: one CTA of 128 threads per instance.  The 32 rows
@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(128) walk_mid_kernel(StepArgs a) {
     for (int w = tid; w < nb; w += 128) a.trace[a.trace_base + (size_t)inst * nb + w] = bits[w];
   const uint32_t U = sub_offset(a, in);
   const int per = (m + 3) / 4;
-  gather_pairs<T>(a, in, U, warp * per, min(m, (warp + 1) * per),
+  gather_pairs<T, true>(a, in, U, warp * per, min(m, (warp + 1) * per),
                   [bits](int i) { return ((bits[i >> 5] >> (i & 31)) & 1u) != 0; }, lane);
 }
 
