@@ -315,6 +315,16 @@ def main():
             "kernel": "attention", "peak_kind": peak_kind,
             "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
             "arithmetic_intensity": round(flops / abytes, 1), "avg_launch_ms": round(attn_ms, 4)}
+    # secondary roofline: the halving steps (thinning + merges), HBM-bound by their algorithmic bytes --
+    # every instance's points read once and its survivors written once: 3 m (E+D) elements per instance
+    es = 4 if w.dtype == "fp32" else 2
+    hbytes = sum(3 * m * (w.E + w.D) * es for _, _, _, m, _ in h.trace_layout(w.causal, w.g))
+    hms = (ph["thin_ms"] + ph["merge_ms"]) / max(1, ph["calls"])
+    halving_roof = {"bound": "hbm", "achieved": round(hbytes / (hms * 1e-3) / 1e9, 1) if hms > 0 else None,
+                    "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(hbytes / (hms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if hms > 0 else None,
+                    "algorithmic_bytes_per_step": hbytes, "ms": round(hms, 4),
+                    "note": "all halving steps of a forward (c^2, Gram, walk, gather launches); latency-bound merges included"}
     phases = {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
               "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4),
               "attn_ms": round(attn_ms, 4)}
@@ -369,7 +379,8 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
-            "ms_per_layer": ms, "phases_ms": phases, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "ms_per_layer": ms, "phases_ms": phases, "roofline": roof, "halving_roofline": halving_roof,
+            "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": plan["kernel_launches"] * a.steps, "clocks": clk, "exact_sdpa_ms": sdpa,
             "workspace_bytes": plan["workspace_bytes"]}
     print(json.dumps(line), flush=True)

@@ -161,6 +161,34 @@ THIN_ATTN_API thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms,
 THIN_ATTN_API thin_attn_status thin_attn_check(thin_attn_t h, void* stream);
 
 /*
+ * Express decode cache -- the updatable weighted cache object of "The EXPRESS Meta-Procedure"
+ * (Express Language Modeling).  One token of every (b,h) per call:
+ *   thin_attn_cache_decode appends k_t, v_t, writes out_t = the attention of q_t against the
+ *   cache (exact prefix, the coresets present after the completed batches, the tokens of the
+ *   batch in progress), then -- when the token completes a batch -- KH-Compresses the batch into a
+ *   level-0 coreset and runs the HALVE merges of the 4-ary counter.  Decisions use the same
+ *   Philox rounds and pairs as thin_attn_forward(causal=1), so the coresets and out_t equal the
+ *   prefill's row t (up to the attention kernel's rounding).
+ * cfg: as for thin_attn_create with T = capacity in tokens (S ignored), n_exact, batch >= 1.
+ * q, k, v, out: device (B,1,H,E), (B,1,H,E), (B,1,H,D), (B,1,H,D); lse_opt device (B,H) or NULL.
+ * Raw keys/values are kept only for the exact prefix and the batch in progress; every coreset slot
+ * of the capacity is allocated at creation (no allocation while decoding).
+ */
+typedef struct thin_attn_cache_s* thin_attn_cache_t;
+THIN_ATTN_API thin_attn_status thin_attn_cache_create(thin_attn_cache_t* out, const thin_attn_config* cfg, int g,
+                                                      uint64_t seed);
+THIN_ATTN_API thin_attn_status thin_attn_cache_destroy(thin_attn_cache_t c);
+/* Tokens decoded so far. */
+THIN_ATTN_API thin_attn_status thin_attn_cache_length(thin_attn_cache_t c, int64_t* t);
+THIN_ATTN_API thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, const void* k,
+                                                      const void* v, void* out, float* lse_opt, void* stream);
+/* Device int32 (B,H,n_nodes,c) token indices of every coreset slot (-1 while empty), in the
+ * node order of thin_attn_forward's coreset output. */
+THIN_ATTN_API thin_attn_status thin_attn_cache_nodes(thin_attn_cache_t c, int32_t* idx_out, void* stream);
+/* Synchronise `stream` and report a device-side failure of the cache's kernels. */
+THIN_ATTN_API thin_attn_status thin_attn_cache_check(thin_attn_cache_t c, void* stream);
+
+/*
  * Kernel Halving of caller-provided point sets, allocating no device memory.
  * The pages have no counterpart of this entry point: it exists for callers that
  * cannot allocate -- an application whose device memory is owned by its own pool

@@ -54,7 +54,9 @@ class TraceEntry(ctypes.Structure):
 _lib = None
 EXPORTS = ("thin_attn_version", "thin_attn_last_error", "thin_attn_create", "thin_attn_destroy",
            "thin_attn_plan", "thin_attn_reserve", "thin_attn_trace_layout", "thin_attn_forward",
-           "thin_attn_forward_host", "thin_attn_check", "thin_attn_profile", "thin_attn_profile_read")
+           "thin_attn_forward_host", "thin_attn_check", "thin_attn_profile", "thin_attn_profile_read",
+           "thin_attn_cache_create", "thin_attn_cache_destroy", "thin_attn_cache_length", "thin_attn_cache_decode",
+           "thin_attn_cache_nodes", "thin_attn_cache_check")
 
 
 def lib() -> ctypes.CDLL:
@@ -77,6 +79,12 @@ def lib() -> ctypes.CDLL:
     L.thin_attn_forward.argtypes = [vp, vp, vp, vp, vp, i, i, u64, vp, vp, vp, vp]
     L.thin_attn_forward_host.argtypes = [vp, vp, vp, vp, vp, i, i, u64, vp, vp]
     L.thin_attn_check.argtypes = [vp, vp]
+    L.thin_attn_cache_create.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(Config), i, u64]
+    L.thin_attn_cache_destroy.argtypes = [vp]
+    L.thin_attn_cache_length.argtypes = [vp, ctypes.POINTER(ctypes.c_int64)]
+    L.thin_attn_cache_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+    L.thin_attn_cache_nodes.argtypes = [vp, vp, vp]
+    L.thin_attn_cache_check.argtypes = [vp, vp]
     L.thin_attn_profile.argtypes = [vp, i]
     L.thin_attn_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
     for f in EXPORTS[2:]:
@@ -200,6 +208,69 @@ class ThinAttention:
         _check(lib().thin_attn_check(self._h, ctypes.c_void_p(stream)))
 
 
+class ThinAttentionCache:
+    """Express decode cache: one token per (b,h) and call, attended like query t of the prefill.
+
+    ``decode(q, k, v)`` takes (B,1,H,E), (B,1,H,E), (B,1,H,D) device tensors and returns the
+    (B,1,H,D) attention output of the new token; completed batches are thinned and merged on the
+    fly.  ``capacity`` bounds the number of tokens.
+    """
+
+    def __init__(self, B: int, H: int, E: int, D: int, dtype: torch.dtype, capacity: int, n_exact: int, batch: int,
+                 g: int = 2, seed: int = 0, scale: Optional[float] = None, device: int = 0):
+        self.cfg = Config(FP32 if dtype == torch.float32 else BF16, B, capacity, capacity, H, E, D,
+                          0.0 if scale is None else float(scale), n_exact, batch, device)
+        self.dtype, self.device = dtype, torch.device("cuda", device)
+        self._h = ctypes.c_void_p()
+        _check(lib().thin_attn_cache_create(ctypes.byref(self._h), ctypes.byref(self.cfg), g,
+                                            ctypes.c_uint64(seed & (2 ** 64 - 1))))
+        plan = ThinAttention(B, capacity, capacity, H, E, D, dtype, scale, n_exact, batch, device).plan(True, g)
+        self.n_nodes, self.node_rows = plan["n_nodes"], plan["coreset_rows"]
+
+    def close(self):
+        if self._h:
+            lib().thin_attn_cache_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __len__(self):
+        t = ctypes.c_int64()
+        _check(lib().thin_attn_cache_length(self._h, ctypes.byref(t)))
+        return t.value
+
+    def decode(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
+               lse: Optional[torch.Tensor] = None) -> torch.Tensor:
+        c = self.cfg
+        for name, t, shape in (("q", q, (c.B, 1, c.H, c.E)), ("k", k, (c.B, 1, c.H, c.E)), ("v", v, (c.B, 1, c.H, c.D))):
+            if tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous() or t.device != self.device:
+                raise ValueError(f"{name}: expected contiguous {self.dtype} {shape} on {self.device}")
+        if out is None:
+            out = torch.empty(c.B, 1, c.H, c.D, dtype=self.dtype, device=self.device)
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_cache_decode(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                            ctypes.c_void_p(stream)))
+        return out
+
+    def nodes(self) -> torch.Tensor:
+        """(B,H,n_nodes,c) token indices of every coreset slot (-1 while empty), the node order of
+        ThinAttention.forward(causal=True, return_coreset=True)."""
+        c = self.cfg
+        n = c.B * c.H * self.n_nodes * self.node_rows
+        rows = torch.full((max(1, n),), -1, dtype=torch.int32, device=self.device)
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_cache_nodes(self._h, _ptr(rows), ctypes.c_void_p(stream)))
+        return rows[:n].view(c.B, c.H, self.n_nodes, self.node_rows)
+
+    def check(self):
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_cache_check(self._h, ctypes.c_void_p(stream)))
+
+
 def decode_trace(words, layout) -> Dict[Tuple[int, int], np.ndarray]:
     """Decision bits of every halving, keyed by (b*H+h, round id), over the Philox pair index."""
     w = np.asarray(words.cpu().numpy() if isinstance(words, torch.Tensor) else words).view(np.uint32)
@@ -231,5 +302,5 @@ def thinformer_attention(query: torch.Tensor, key: torch.Tensor, value: torch.Te
     return _cache[k_].forward(query, key, value, causal=causal, g=g, seed=seed)["out"], None
 
 
-__all__ = ["ThinAttention", "ThinAttnError", "thinformer_attention", "decode_trace", "lib", "LIB_PATH",
+__all__ = ["ThinAttention", "ThinAttentionCache", "ThinAttnError", "thinformer_attention", "decode_trace", "lib", "LIB_PATH",
            "EXPORTS"]

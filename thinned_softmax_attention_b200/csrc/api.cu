@@ -707,8 +707,10 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     cudaError_t e = sp.copy_only ? launch_copy_step(a, cf.dtype, st)
                                  : launch_halving_step(a, cf.dtype, use_tc_gram, st);
     if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "halving step (n=%d): %s", sp.n, cudaGetErrorString(e));
-    ls = launch_waves_after((int)si);
-    if (ls != THIN_ATTN_OK) return ls;
+    if (si + 1 < p->steps.size()) {
+      ls = launch_waves_after((int)si);
+      if (ls != THIN_ATTN_OK) return ls;
+    }
   }
   if (!ev.empty()) {
     if (!merged_mark) CK(cudaEventRecord(ev[1], st));
@@ -941,6 +943,416 @@ thin_attn_status thin_attn_check(thin_attn_t h, void* stream) {
     CK(cudaMemset(h->d_status, 0, 16));
     return fail(THIN_ATTN_ETIMEOUT, "device wait gave up (code %d; query tile %d of (b,h) %d; wait %d at key tile %d)",
                 st[0], st[1] >> 16, st[1] & 0xFFFF, st[2] / 1000, st[2] % 1000);
+  }
+  return THIN_ATTN_OK;
+}
+
+}  // extern "C"
+
+// =============================================================================================
+// Express decode cache ("EXPRESS ... operates as an updatable weighted cache object", Express
+// Language Modeling, "The EXPRESS Meta-Procedure").  Token t of each (b,h) is appended, attended
+// exactly as query t of the prefill (exact prefix + snapshot nodes + its own batch), and when a
+// batch completes it is KH-Compressed into a level-0 node and the 4-ary counter's merges run --
+// with the prefill's Philox rounds and pair indices, so the nodes equal the prefill's.  Raw
+// tokens are kept for the exact prefix and the one batch in progress (rows ne .. ne+b-1).
+// =============================================================================================
+namespace {
+
+struct CacheStep {
+  StepPlan sp;
+  int src_level = -1, dst_level = -1;   // intermediate level buffers (or -1)
+};
+
+}  // namespace
+
+struct thin_attn_cache_s {
+  thin_attn_config cf{};
+  int g = 0;
+  uint64_t seed = 0;
+  float scale = 0.f;
+  int ne = 0, bsz = 0, L = 0, c = 0, n_bmax = 0, n_slots = 0;
+  Sizes sz{};
+  std::vector<int> level_base;
+  std::vector<std::vector<CacheStep>> batch_steps;               // [k]
+  std::map<std::pair<int, int>, std::vector<CacheStep>> merges;   // (target level, node) -> 2 steps
+  std::vector<BufSpec> levels;
+  BufSpec raw, nodes, mtemp;
+  AttnTables tab;
+  size_t delta_off = 0, c2_off = 0, delta_floats = 0, c2_floats = 0, bytes = 0;
+  void* d_mem = nullptr;
+  int* d_status = nullptr;
+  int64_t t = 0;
+  bool use_tc = false;
+};
+
+namespace {
+
+void cache_add_step(thin_attn_cache_s* cc, CacheStep& st) {
+  cc->delta_floats = std::max(cc->delta_floats, st.sp.inst.size() * (size_t)st.sp.m_pad * st.sp.m_pad);
+  cc->c2_floats = std::max(cc->c2_floats, st.sp.inst.size());
+}
+
+thin_attn_status cache_build(thin_attn_cache_s* cc) {
+  const thin_attn_config& cf = cc->cf;
+  const int BH = cf.B * cf.H, T = cf.T;
+  cc->ne = std::min(cf.n_exact, T);
+  cc->bsz = cf.batch;
+  cc->L = cc->ne + cc->bsz;
+  cc->n_bmax = T > cc->ne ? (T - cc->ne) / cc->bsz : 0;
+  cc->sz = compress_sizes(cc->bsz, cc->g);
+  cc->c = cc->sz.C;
+  for (int lv = 0; (cc->n_bmax >> (2 * lv)) > 0; ++lv) {
+    cc->level_base.push_back(cc->n_slots);
+    cc->n_slots += cc->n_bmax >> (2 * lv);
+  }
+  const Sizes& sz = cc->sz;
+  // intermediate level buffers of one batch (all (b,h))
+  for (int lv = 1; lv < sz.r; ++lv) {
+    BufSpec b;
+    b.rows = (int64_t)BH * (sz.S_sub >> lv);
+    cc->levels.push_back(b);
+  }
+  cc->raw.rows = (int64_t)cf.B * cc->L * cf.H;
+  cc->nodes.rows = (int64_t)BH * cc->n_slots * cc->c;
+  cc->mtemp.rows = (int64_t)BH * 2 * cc->c;
+  for (int k = 0; k < cc->n_bmax; ++k) {
+    std::vector<CacheStep> steps;
+    if (sz.r == 0) {
+      CacheStep st;
+      st.sp.copy_only = true;
+      st.sp.n = cc->bsz;
+      st.sp.src_buf = BUF_TOKENS;
+      st.sp.dst_buf = BUF_NODES;
+      st.sp.S_full = st.sp.S_sub = cc->bsz;
+      for (int bh = 0; bh < BH; ++bh) {
+        HalveInst in{};
+        in.src_row = (int64_t)(bh / cf.H) * cc->L + cc->ne;
+        in.dst_row = ((int64_t)bh * cc->n_slots + k) * cc->c;
+        in.bh = (uint32_t)bh;
+        in.tok0 = (uint32_t)(cc->ne + k * cc->bsz);
+        st.sp.inst.push_back(in);
+      }
+      steps.push_back(std::move(st));
+    }
+    for (int lv = 1; lv <= sz.r; ++lv) {
+      CacheStep st;
+      st.sp.n = 4 * sz.L * (1 << (lv - 1));
+      st.sp.m = st.sp.n / 2;
+      st.sp.m_pad = (st.sp.m + 31) / 32 * 32;
+      const int in_rows = sz.S_sub >> (lv - 1), G = in_rows / st.sp.n, out_rows = in_rows / 2;
+      st.sp.src_buf = lv == 1 ? BUF_TOKENS : 0;
+      st.src_level = lv == 1 ? -1 : lv - 2;
+      st.sp.dst_buf = lv == sz.r ? BUF_NODES : 0;
+      st.dst_level = lv == sz.r ? -1 : lv - 1;
+      st.sp.S_full = cc->bsz;
+      st.sp.S_sub = sz.S_sub;
+      for (int bh = 0; bh < BH; ++bh)
+        for (int gi = 0; gi < G; ++gi) {
+          HalveInst in{};
+          in.src_row = lv == 1 ? (int64_t)(bh / cf.H) * cc->L + cc->ne : (int64_t)bh * in_rows + (int64_t)gi * st.sp.n;
+          in.dst_row = (lv == sz.r ? ((int64_t)bh * cc->n_slots + k) * cc->c : (int64_t)bh * out_rows) +
+                       (int64_t)gi * st.sp.m;
+          in.bh = (uint32_t)bh;
+          in.round_id = round_batch(k, lv);
+          in.pair0 = (uint32_t)(gi * st.sp.m);
+          in.sub_round = round_subsample(k);
+          in.tok0 = (uint32_t)(cc->ne + k * cc->bsz);
+          st.sp.inst.push_back(in);
+        }
+      cache_add_step(cc, st);
+      steps.push_back(std::move(st));
+    }
+    cc->batch_steps.push_back(std::move(steps));
+  }
+  for (int lv = 1; (cc->n_bmax >> (2 * lv)) > 0; ++lv)
+    for (int j = 0; j < (cc->n_bmax >> (2 * lv)); ++j) {
+      std::vector<CacheStep> two;
+      for (int step = 0; step < 2; ++step) {
+        CacheStep st;
+        st.sp.phase = 1;
+        st.sp.merge_level = lv;
+        st.sp.n = (step == 0 ? 4 : 2) * cc->c;
+        st.sp.m = st.sp.n / 2;
+        st.sp.m_pad = (st.sp.m + 31) / 32 * 32;
+        st.sp.src_buf = step == 0 ? BUF_NODES : BUF_MTEMP;
+        st.sp.dst_buf = step == 0 ? BUF_MTEMP : BUF_NODES;
+        st.sp.S_full = st.sp.S_sub = st.sp.n;
+        for (int bh = 0; bh < BH; ++bh) {
+          HalveInst in{};
+          const int64_t mt = (int64_t)bh * 2 * cc->c;
+          in.src_row = step == 0 ? ((int64_t)bh * cc->n_slots + cc->level_base[lv - 1] + 4 * j) * cc->c : mt;
+          in.dst_row = step == 0 ? mt : ((int64_t)bh * cc->n_slots + cc->level_base[lv] + j) * cc->c;
+          in.bh = (uint32_t)bh;
+          in.round_id = round_merge(lv, j, step);
+          st.sp.inst.push_back(in);
+        }
+        cache_add_step(cc, st);
+        two.push_back(std::move(st));
+      }
+      cc->merges[{lv, j}] = std::move(two);
+    }
+  // attention table: one tile (one query) per position t
+  AttnTables& t = cc->tab;
+  for (int pos = 0; pos < T; ++pos) {
+    const int seg0 = (int)t.segs.size();
+    if (pos < cc->ne) {
+      t.segs.push_back({SEG_TOKENS, 0, pos + 1, 0, 0.f, 0});
+    } else {
+      const int k = (pos - cc->ne) / cc->bsz, tin = (pos - cc->ne) % cc->bsz;
+      if (cc->ne > 0) t.segs.push_back({SEG_TOKENS, 0, cc->ne, 0, 0.f, 0});
+      for (int lv = 0; ((int64_t)1 << (2 * lv)) <= k; ++lv) {
+        const int64_t p4 = (int64_t)1 << (2 * lv);
+        const int d = (int)((k / p4) % 4), base = (int)((k / (p4 * 4)) * 4);
+        const double w = std::ldexp((double)cc->bsz / cc->c, 2 * lv);
+        for (int j = 0; j < d; ++j)
+          t.segs.push_back({SEG_COMPACT, cc->level_base[lv] + base + j, cc->c, 0, (float)std::log(w), 0});
+      }
+      t.segs.push_back({SEG_TOKENS, cc->ne, tin + 1, 0, 0.f, 0});
+    }
+    t.tiles.push_back({0, 1, seg0, (int)t.segs.size() - seg0});
+  }
+  // device layout
+  size_t off = 0;
+  for (auto& steps : cc->batch_steps)
+    for (auto& st : steps) {
+      st.sp.inst_off = off;
+      off = align256(off + st.sp.inst.size() * sizeof(HalveInst));
+    }
+  for (auto& kv : cc->merges)
+    for (auto& st : kv.second) {
+      st.sp.inst_off = off;
+      off = align256(off + st.sp.inst.size() * sizeof(HalveInst));
+    }
+  t.tiles_off = off;
+  off = align256(off + t.tiles.size() * sizeof(AttnTile));
+  t.segs_off = off;
+  off = align256(off + t.segs.size() * sizeof(AttnSeg));
+  const size_t table_end = off;
+  const size_t es = elt(cf);
+  auto place = [&](BufSpec& b) {
+    b.k_off = off;
+    off = align256(off + (size_t)b.rows * cf.E * es);
+    b.v_off = off;
+    off = align256(off + (size_t)b.rows * cf.D * es);
+    b.idx_off = off;
+    off = align256(off + (size_t)b.rows * 4);
+  };
+  for (auto& b : cc->levels) place(b);
+  place(cc->raw);
+  place(cc->nodes);
+  place(cc->mtemp);
+  cc->delta_off = off;
+  off = align256(off + cc->delta_floats * 4);
+  cc->c2_off = off;
+  off = align256(off + std::max<size_t>(cc->c2_floats, 1) * 4);
+  cc->bytes = off;
+  cudaError_t e = cudaMalloc(&cc->d_mem, cc->bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(THIN_ATTN_ENOMEM, "decode cache of %zu bytes: %s", cc->bytes, cudaGetErrorString(e));
+  }
+  std::vector<char> host(table_end);
+  auto put = [&](const std::vector<HalveInst>& v, size_t o) {
+    if (!v.empty()) std::memcpy(host.data() + o, v.data(), v.size() * sizeof(HalveInst));
+  };
+  for (auto& steps : cc->batch_steps)
+    for (auto& st : steps) put(st.sp.inst, st.sp.inst_off);
+  for (auto& kv : cc->merges)
+    for (auto& st : kv.second) put(st.sp.inst, st.sp.inst_off);
+  std::memcpy(host.data() + t.tiles_off, t.tiles.data(), t.tiles.size() * sizeof(AttnTile));
+  std::memcpy(host.data() + t.segs_off, t.segs.data(), t.segs.size() * sizeof(AttnSeg));
+  CK(cudaMemcpy(cc->d_mem, host.data(), table_end, cudaMemcpyHostToDevice));
+  CK(cudaMalloc(&cc->d_status, 16));
+  CK(cudaMemset(cc->d_status, 0, 16));
+  CK(cudaMemset((char*)cc->d_mem + cc->nodes.idx_off, 0xFF, (size_t)cc->nodes.rows * 4));
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status cache_run_step(thin_attn_cache_s* cc, CacheStep& st, cudaStream_t s) {
+  const thin_attn_config& cf = cc->cf;
+  char* base = (char*)cc->d_mem;
+  auto ptrs = [&](int buf, int level, const void** K, const void** V, int32_t** I, int64_t* rows) {
+    const BufSpec& b = buf == BUF_TOKENS ? cc->raw : buf == BUF_NODES ? cc->nodes : buf == BUF_MTEMP ? cc->mtemp
+                                                                                     : cc->levels[level];
+    *K = base + b.k_off;
+    *V = base + b.v_off;
+    *I = (int32_t*)(base + b.idx_off);
+    *rows = buf == BUF_TOKENS ? (int64_t)cf.B * cc->L : b.rows;
+  };
+  StepArgs a{};
+  int64_t rows = 0;
+  const void *sk, *sv, *dk, *dv;
+  int32_t *sidx, *didx;
+  int64_t drows;
+  ptrs(st.sp.src_buf, st.src_level, &sk, &sv, &sidx, &rows);
+  ptrs(st.sp.dst_buf, st.dst_level, &dk, &dv, &didx, &drows);
+  a.src_kind = st.sp.src_buf == BUF_TOKENS ? SRC_TOKENS : SRC_COMPACT;
+  a.srcK = sk;
+  a.srcV = sv;
+  a.srcIdx = st.sp.src_buf == BUF_TOKENS ? nullptr : sidx;
+  a.H = cf.H;
+  a.src_rows = rows;
+  a.S_full = st.sp.S_full;
+  a.S_sub = st.sp.S_sub;
+  a.dstK = (void*)dk;
+  a.dstV = (void*)dv;
+  a.dstIdx = didx;
+  a.inst = (const HalveInst*)(base + st.sp.inst_off);
+  a.n_inst = (int)st.sp.inst.size();
+  a.n = st.sp.n;
+  a.m = st.sp.m;
+  a.m_pad = st.sp.m_pad;
+  a.E = cf.E;
+  a.D = cf.D;
+  a.scale_log2e = (float)((double)cc->scale * 1.4426950408889634);
+  a.C = st.sp.m > 0 ? (float)std::sqrt(2.0 * std::log(4.0 * st.sp.m)) : 0.f;
+  a.seed = cc->seed;
+  a.c2 = (float*)(base + cc->c2_off);
+  a.delta = (float*)(base + cc->delta_off);
+  a.status = cc->d_status;
+  cudaError_t e = st.sp.copy_only ? launch_copy_step(a, cf.dtype, s) : launch_halving_step(a, cf.dtype, true, s);
+  if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "cache halving step (n=%d): %s", st.sp.n, cudaGetErrorString(e));
+  return THIN_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+thin_attn_status thin_attn_cache_create(thin_attn_cache_t* out, const thin_attn_config* cfg, int g, uint64_t seed) {
+  if (!out) return fail(THIN_ATTN_EINVAL, "out is null");
+  *out = nullptr;
+  thin_attn_status s = check_cfg(cfg);
+  if (s != THIN_ATTN_OK) return s;
+  if (g < 0 || g > 6) return fail(THIN_ATTN_EINVAL, "g=%d outside 0..6", g);
+  if (cfg->batch < 1 || cfg->n_exact < 0) return fail(THIN_ATTN_EINVAL, "the cache needs batch >= 1 and n_exact >= 0");
+  DeviceGuard dg(cfg->device);
+  if (!dg.ok) return fail(THIN_ATTN_ECUDA, "cannot select device %d", cfg->device);
+  thin_attn_cache_s* cc = new thin_attn_cache_s();
+  cc->cf = *cfg;
+  cc->cf.S = cfg->T;
+  cc->g = g;
+  cc->seed = seed;
+  cc->scale = cfg->scale > 0.f ? cfg->scale : (float)(1.0 / std::sqrt((double)cfg->E));
+  cc->use_tc = attention_tc_supported(cfg->dtype, cfg->E, cfg->D) && tensor_maps_available();
+  s = cache_build(cc);
+  if (s != THIN_ATTN_OK) {
+    thin_attn_cache_destroy(cc);
+    return s;
+  }
+  for (const auto& steps : cc->batch_steps)
+    for (const auto& st : steps)
+      if (!st.sp.copy_only && st.sp.m_pad > 2048) {
+        thin_attn_cache_destroy(cc);
+        return fail(THIN_ATTN_EUNSUPPORTED, "halving instance of %d points exceeds 4096", st.sp.n);
+      }
+  *out = cc;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_cache_destroy(thin_attn_cache_t c) {
+  if (!c) return THIN_ATTN_OK;
+  DeviceGuard dg(c->d_mem || c->d_status ? c->cf.device : -1);
+  if (c->d_mem) cudaFree(c->d_mem);
+  if (c->d_status) cudaFree(c->d_status);
+  delete c;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_cache_length(thin_attn_cache_t c, int64_t* t) {
+  if (!c || !t) return fail(THIN_ATTN_EINVAL, "null argument");
+  *t = c->t;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, const void* k, const void* v, void* out,
+                                        float* lse_opt, void* stream) {
+  if (!c) return fail(THIN_ATTN_EINVAL, "null cache");
+  if (!q || !k || !v || !out) return fail(THIN_ATTN_EINVAL, "q, k, v and out must be non-null");
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (((uintptr_t)ptr) % 16) return fail(THIN_ATTN_EINVAL, "tensor pointers must be 16-byte aligned");
+  const thin_attn_config& cf = c->cf;
+  if (c->t >= cf.T) return fail(THIN_ATTN_EINVAL, "the cache holds its capacity of %d tokens", cf.T);
+  DeviceGuard dg(cf.device);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t pos = c->t;
+  const size_t es = elt(cf);
+  char* base = (char*)c->d_mem;
+  // 1. the new key/value row: exact prefix row pos, or row ne + (pos - ne) mod b of the batch region
+  const int64_t r = pos < c->ne ? pos : c->ne + (pos - c->ne) % c->bsz;
+  const size_t krow = (size_t)cf.H * cf.E * es, vrow = (size_t)cf.H * cf.D * es;
+  CK(cudaMemcpy2DAsync(base + c->raw.k_off + (size_t)r * krow, (size_t)c->L * krow, k, krow, krow, cf.B,
+                       cudaMemcpyDeviceToDevice, st));
+  CK(cudaMemcpy2DAsync(base + c->raw.v_off + (size_t)r * vrow, (size_t)c->L * vrow, v, vrow, vrow, cf.B,
+                       cudaMemcpyDeviceToDevice, st));
+  // 2. attention of query pos against the cache as it stands (its own token included)
+  AttnArgs aa{};
+  aa.q = q;
+  aa.k = base + c->raw.k_off;
+  aa.v = base + c->raw.v_off;
+  aa.ck = base + c->nodes.k_off;
+  aa.cv = base + c->nodes.v_off;
+  aa.out = out;
+  aa.lse = lse_opt;
+  aa.tiles = (const AttnTile*)(base + c->tab.tiles_off);
+  aa.segs = (const AttnSeg*)(base + c->tab.segs_off);
+  aa.tile0 = (int)pos;
+  aa.n_tiles = 1;
+  aa.B = cf.B;
+  aa.T = 1;
+  aa.L = c->L;
+  aa.H = cf.H;
+  aa.E = cf.E;
+  aa.D = cf.D;
+  aa.n_slots = std::max(1, c->n_slots);
+  aa.slot_rows = c->c;
+  aa.scale_log2e = (float)((double)c->scale * 1.4426950408889634);
+  bool done = false;
+  cudaError_t e = cudaSuccess;
+  if (c->use_tc) e = launch_attention_tc(aa, c->d_status, st, &done);
+  if (e == cudaSuccess && !done) e = launch_attention_simt(aa, cf.dtype, st);
+  if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "cache attention: %s", cudaGetErrorString(e));
+  // 3. a completed batch becomes a level-0 node; the 4-ary counter merges equal levels
+  if (pos >= c->ne && (pos - c->ne + 1) % c->bsz == 0) {
+    const int kb = (int)((pos - c->ne) / c->bsz);
+    for (auto& stp : c->batch_steps[kb]) {
+      thin_attn_status s = cache_run_step(c, stp, st);
+      if (s != THIN_ATTN_OK) return s;
+    }
+    const int64_t done_batches = kb + 1;
+    for (int lv = 1; done_batches % ((int64_t)1 << (2 * lv)) == 0; ++lv) {
+      const int j = (int)(done_batches >> (2 * lv)) - 1;
+      auto it = c->merges.find({lv, j});
+      if (it == c->merges.end()) break;
+      for (auto& stp : it->second) {
+        thin_attn_status s = cache_run_step(c, stp, st);
+        if (s != THIN_ATTN_OK) return s;
+      }
+    }
+  }
+  c->t = pos + 1;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_cache_nodes(thin_attn_cache_t c, int32_t* idx_out, void* stream) {
+  if (!c || !idx_out) return fail(THIN_ATTN_EINVAL, "null argument");
+  DeviceGuard dg(c->cf.device);
+  if (c->nodes.rows)
+    CK(cudaMemcpyAsync(idx_out, (char*)c->d_mem + c->nodes.idx_off, (size_t)c->nodes.rows * 4,
+                       cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_cache_check(thin_attn_cache_t c, void* stream) {
+  if (!c) return fail(THIN_ATTN_EINVAL, "null cache");
+  DeviceGuard dg(c->cf.device);
+  CK(cudaStreamSynchronize((cudaStream_t)stream));
+  int sts[4] = {0, 0, 0, 0};
+  CK(cudaMemcpy(sts, c->d_status, sizeof sts, cudaMemcpyDeviceToHost));
+  if (sts[0] != 0) {
+    CK(cudaMemset(c->d_status, 0, 16));
+    return fail(THIN_ATTN_ETIMEOUT, "device wait gave up (code %d)", sts[0]);
   }
   return THIN_ATTN_OK;
 }
