@@ -5,7 +5,8 @@
 // "Express Language Modeling" summary names for Thinformer Express:
 //   kappa((k,v),(k',v')) = exp(s <k,k'>) (<v,v'> + c^2),  c = max |v| of the instance.
 //
-// A step is three launches:
+// A step is three launches (instances of <= 128 bf16 points whose rows form TMA boxes take the
+// one-launch kernel of halving_fused.cu instead):
 //   1. c2_kernel        c^2 of every instance
 //   2. pairgram kernel   pair-difference matrix Delta[j][i] = k(x_j,x_i) - k(y_j,x_i)
 //                        - k(x_j,y_i) + k(y_j,y_i) for j <= i (upper triangle, 32x32 pair
@@ -16,21 +17,9 @@
 // is u_i < clip((1 - alpha_i/a_i)/2, 0, 1) rearranged (a_i > 0).
 #include "common.cuh"
 #include "kernels.h"
+#include "walk.cuh"
 
 namespace thin {
-
-// Approximate square root and reciprocal (MUFU): relative error ~1e-7, far below the 1e-4
-// near-tie margin of the decisions; they sit on the walk's serial chain.
-__device__ __forceinline__ float sqrt_approx(float x) {
-  float y;
-  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float rcp_approx(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // ---------------------------------------------------------------------------
 // 1. c^2 = (max |v|)^2 over the instance's points
@@ -208,7 +197,7 @@ __global__ void __launch_bounds__(128, 8) walk_kernel(StepArgs a) {
     ubuf[i] = i < m ? philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)i) : 0.5f;
   }
   if (tid == 0) U_s = sub_offset(a, in);
-  float sig2 = 0.f;
+  float sigma = 0.f;
   for (int t = 0; t < nb; ++t) {
     const int base = t * 32;
     __syncthreads();
@@ -219,30 +208,10 @@ __global__ void __launch_bounds__(128, 8) walk_kernel(StepArgs a) {
     __syncthreads();
     const int steps = min(32, m - base);
     if (warp == 0) {
-      // per-pair values held by lane l (pair base + l): b^2, b, 1 - 2u
-      const float b2l = tile[lane * 33 + lane];
-      const float bl = sqrt_approx(fmaxf(b2l, 0.f));
-      const float ul = 1.f - 2.f * ubuf[base + lane];
+      // lane l holds pair base + l; the tile is zero past m, so padded pairs are no-ops
       float my = alpha[base + lane];
-      uint32_t kb = 0;
-#pragma unroll
-      for (int s = 0; s < 32; ++s) {
-        if (s < steps) {
-          const float b2 = __shfl_sync(0xffffffffu, b2l, s);
-          const float b = __shfl_sync(0xffffffffu, bl, s);
-          const float w = __shfl_sync(0xffffffffu, ul, s);
-          const float ai = __shfl_sync(0xffffffffu, my, s);
-          bool keep = true;
-          if (b2 > 0.f) {
-            const float av = fmaxf(b * sqrt_approx(sig2) * a.C, b2);
-            keep = ai < av * w;
-            const float r = rcp_approx(av * av);
-            sig2 = sig2 + b2 * fmaxf(0.f, 1.f + (b2 - 2.f * av) * sig2 * r);
-          }
-          if (lane > s) my = fmaf(keep ? 1.f : -1.f, tile[s * 33 + lane], my);
-          kb |= (uint32_t)keep << s;
-        }
-      }
+      const uint32_t kb = walk_block32(my, sigma, tile[lane * 33 + lane], 1.f - 2.f * ubuf[base + lane], a.C,
+                                       1.f / a.C, lane, [&](int s) { return tile[s * 33 + lane]; });
       if (lane == 0) bits[t] = kb;
     }
     __syncthreads();
@@ -281,20 +250,6 @@ __global__ void __launch_bounds__(128, 8) walk_kernel(StepArgs a) {
   }
 }
 
-// One step of the sigma recursion and the threshold of pair i.  With C = sqrt(2 ln(2/delta_i)) > 1:
-//   b >= sigma C:  a = b^2,          sigma' = b
-//   otherwise:     a = b sigma C,    sigma'^2 = sigma^2 + max(0, b^2 (1 + 1/C^2) - 2 b sigma / C)
-// which is sigma'^2 = sigma^2 + b^2 max(0, 1 + (b^2 - 2a) sigma^2 / a^2) with the two cases of
-// a = max(b sigma C, b^2) written out (in the first, sigma <= b/C < b gives sigma'^2 = b^2).
-// Returns a; sigma is updated in place.  b^2 <= 0 (a repeated point) keeps sigma and returns 0.
-__device__ __forceinline__ float sigma_step(float& sigma, float b2, float b, float C, float q, float r2) {
-  const float sc = sigma * C;
-  const bool first = b >= sc;
-  const float s_else = sqrt_approx(fmaf(sigma, sigma, fmaxf(0.f, fmaf(-r2, sigma, q))));
-  const bool live = b2 > 0.f;
-  sigma = live ? (first ? b : s_else) : sigma;
-  return first ? b2 : b * sc;
-}
 
 // Gather the kept point of pairs [i0, i1) (bit i of `bits(i)` set = first point kept) into
 // destination rows dst_row + i, by one warp.  Lane l resolves pair i0 + 32q + l; the warp then
@@ -385,22 +340,9 @@ __global__ void __launch_bounds__(128) walk_small_kernel(StepArgs a) {
   for (int s = 0; s < 32; ++s) d[s] = (s < m && lane < m) ? Dl[(size_t)s * a.m_pad + lane] : 0.f;
   const float w_l = lane < m ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)lane) : 0.f;
   const uint32_t U = sub_offset(a, in);
-  const float C = a.C, cq = 1.f + 1.f / (C * C), c2C = 2.f / C;
-  float my = 0.f, sigma = 0.f;
-  uint32_t kb = 0;
   // Pairs s >= m are no-ops: their Delta entries are 0, so b^2 = 0 keeps sigma and alpha as they
   // are, and their bits are never read.
-#pragma unroll
-  for (int s = 0; s < 32; ++s) {
-    const float b2 = __shfl_sync(0xffffffffu, d[s], s);
-    const float w = __shfl_sync(0xffffffffu, w_l, s);
-    const float b = sqrt_approx(fmaxf(b2, 0.f));
-    const float av = sigma_step(sigma, b2, b, C, b2 * cq, b * c2C);
-    const float ai = __shfl_sync(0xffffffffu, my, s);
-    const bool keep = !(b2 > 0.f) || ai < av * w;
-    if (lane > s) my = fmaf(keep ? 1.f : -1.f, d[s], my);
-    kb |= (uint32_t)keep << s;
-  }
+  const uint32_t kb = walk_segment<32>(d, w_l, a.C, lane);
   if (a.trace && lane == 0) a.trace[a.trace_base + inst] = kb;
   gather_pairs<T, false>(a, in, U, 0, m, [kb](int i) { return ((kb >> i) & 1u) != 0; }, lane);
 }
@@ -445,7 +387,7 @@ __global__ void __launch_bounds__(128) walk_mid_kernel(StepArgs a) {
     alpha[i] = 0.f;
     wbuf[i] = i < m ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)i) : 0.f;
   }
-  const float C = a.C, cq = 1.f + 1.f / (C * C), c2C = 2.f / C;
+  const float C = a.C, rC = 1.f / C;
   float sigma = 0.f;
   for (int t = 0; t < nb; ++t) {
     const int base = 32 * t;
@@ -461,23 +403,11 @@ __global__ void __launch_bounds__(128) walk_mid_kernel(StepArgs a) {
     const int steps = min(32, m - base);
     if (warp == 0) {
       const float dl = lane < steps ? R[lane * mp + base + lane] : 0.f;   // b^2 of pair base+lane
-      const float bl = sqrt_approx(fmaxf(dl, 0.f));
-      const float wl = wbuf[base + lane];
       float my = alpha[base + lane];
-      uint32_t kb = 0;
       // Pairs s >= steps are no-ops (b^2 = 0 keeps sigma; they only touch alpha of lanes that are
       // no pair), so the 32 steps run without a guard.
-#pragma unroll
-      for (int s = 0; s < 32; ++s) {
-        const float b2 = __shfl_sync(0xffffffffu, dl, s);
-        const float b = __shfl_sync(0xffffffffu, bl, s);
-        const float w = __shfl_sync(0xffffffffu, wl, s);
-        const float av = sigma_step(sigma, b2, b, C, b2 * cq, b * c2C);
-        const float ai = __shfl_sync(0xffffffffu, my, s);
-        const bool keep = !(b2 > 0.f) || ai < av * w;
-        if (lane > s) my = fmaf(keep ? 1.f : -1.f, R[s * mp + base + lane], my);
-        kb |= (uint32_t)keep << s;
-      }
+      const uint32_t kb = walk_block32(my, sigma, dl, wbuf[base + lane], C, rC, lane,
+                                       [&](int s) { return R[s * mp + base + lane]; });
       if (lane == 0) bits[t] = kb;
     }
     __syncthreads();
@@ -529,6 +459,7 @@ size_t walk_smem_bytes(int m_pad) { return (size_t)(2 * m_pad + 32 * 33 + m_pad 
 template <typename T>
 static cudaError_t launch_step_t(const StepArgs& a, bool use_tc, cudaStream_t st) {
   if (a.n_inst == 0) return cudaSuccess;
+  if (sizeof(T) == 2 && use_tc && halving_fused_supported(a)) return launch_halving_fused(a, st);
   c2_kernel<T><<<a.n_inst, 256, 0, st>>>(a);
   const int nb = a.m_pad / 32;
   const int ntri = nb * (nb + 1) / 2;

@@ -1,0 +1,446 @@
+// Kernel Halving of small instances (n <= 128 points) in one persistent kernel.
+//
+// The three-launch step of halving.cu (c^2, pair-difference Gram, walk + gather) reads every
+// point from HBM three times and round-trips the pair-difference matrix through HBM.  For the
+// small instances that dominate the Express batch thinning (groups of 32..128 points) this kernel
+// does the whole step in one pass over the points:
+//
+//   TMA      a unit of 128 point rows lands in one pipeline stage as (E+D)/64 chunks of
+//            128 rows x 64 bf16 (128-byte swizzle); a unit is 4 instances of <= 32 points
+//            (NP = 32), 2 of <= 64 (NP = 64) or 1 of <= 128 (NP = 128)
+//   c^2      max |v| of each instance, read from the stage
+//   tcgen05  kk = K K^T and vv = V V^T of each instance (A = the unit's 128 rows, B = the
+//            instance's NP rows), fp32 accumulators in TMEM
+//   epilogue kappa = 2^(kk s log2 e) (vv + c^2) and the pair differences
+//            Delta[j][i] = kappa[2j][2i] - kappa[2j][2i+1] - kappa[2j+1][2i] + kappa[2j+1][2i+1]
+//            into shared memory (thread = TMEM lane = point row; the row difference is a shuffle)
+//   walk     the sequential decisions of each instance, with the same arithmetic as the walk
+//            kernels of halving.cu, so the decisions are the same
+//   gather   the kept rows, from the stage straight to the destination rows
+//
+// Warp roles (320 threads, one CTA per SM, persistent over units u = blockIdx.x + k gridDim.x):
+//   warp 0     TMA producer (one thread)     warp 1     MMA issuer (one thread), TMEM owner
+//   warps 2,3  walkers of even k             warps 4-7  epilogue (warp w reads TMEM lanes 32(w%4)..)
+//   warps 8,9  walkers of odd k
+// Pipeline: `nst` shared-memory stages, two TMEM accumulator buffers of 256 columns and two
+// Delta buffers (one per walker set).  Every mbarrier wait is bounded; after a time-out the
+// kernel stops, waits (bounded) for the copies and MMAs it started, frees TMEM and reports
+// through the status word (code 3, status[1] = CTA).
+#include <cstdlib>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+#include "walk.cuh"
+
+namespace thin {
+
+namespace {
+
+using namespace tc;
+
+struct FusedMaps {
+  CUtensorMap k, v;
+};
+
+constexpr uint32_t kChunk = 128 * 128;   // 128 rows x 64 bf16 (one feature chunk of a unit)
+constexpr int kThreads = 320;
+constexpr int kMaxChunks = 5;             // (E + D) / 64 <= 5 (the stages must fit in shared memory)
+
+template <int NP>
+struct FusedShape {
+  static constexpr int PAIRS = NP / 2;                     // pairs per instance
+  static constexpr int IPU = 128 / NP;                     // instances per unit
+  static constexpr int LD = PAIRS + 1;                     // Delta row stride (floats): no bank conflicts
+  static constexpr int DELTA_INST = PAIRS * LD;            // floats per instance
+  static constexpr int DELTA_SET = IPU * DELTA_INST;       // floats per walker set
+  static constexpr int SEG = PAIRS < 32 ? PAIRS : 32;      // walk lanes per instance (NP <= 64)
+};
+
+// Copy the kept point of pairs [i0, i1) of one instance from the stage (unit rows row0 + 2i or
+// row0 + 2i + 1) to destination rows dst_row + i, with its token index.  One warp; lane = one
+// 16-byte unit of a row (K units first), four rows in flight.
+template <typename Bit>
+__device__ __forceinline__ void gather_from_stage(const StepArgs& a, int64_t dst_row, int64_t src_row, uint32_t tok_base,
+                                                  const uint8_t* st, int row0, int i0, int i1, Bit bit, int lane,
+                                                  int EC, int NC) {
+  const bool tokens = a.src_kind == SRC_TOKENS;
+  for (int i = i0 + lane; i < i1; i += 32) {
+    const int p = 2 * i + (bit(i) ? 0 : 1);
+    a.dstIdx[dst_row + i] = tokens ? (int32_t)(tok_base + (uint32_t)p) : a.srcIdx[src_row + p];
+  }
+  const int units = NC * 8, kw = a.E / 8, vw = a.D / 8;
+  uint4* dK = (uint4*)a.dstK;
+  uint4* dV = (uint4*)a.dstV;
+  for (int w = lane; w < units; w += 32) {
+    const int c = w >> 3, x = w & 7;
+    uint4* dst = c < EC ? dK + dst_row * kw + c * 8 + x : dV + dst_row * vw + (c - EC) * 8 + x;
+    const int stride = c < EC ? kw : vw;
+    const uint8_t* src = st + c * kChunk;
+    for (int i = i0; i < i1; i += 8) {
+      uint4 buf[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (i + j < i1) {
+          const int R = row0 + 2 * (i + j) + (bit(i + j) ? 0 : 1);
+          buf[j] = *(const uint4*)(src + R * 128 + ((x ^ (R & 7)) << 4));
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (i + j < i1) dst[(int64_t)(i + j) * stride] = buf[j];
+    }
+  }
+}
+
+template <int NP>
+__global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_constant__ FusedMaps maps,
+                                                                  const StepArgs a, int n_units, int nst) {
+  using Sh = FusedShape<NP>;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned, by an offset from the array itself so that the compiler keeps every pointer
+  // derived from it in the shared address space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int EC = a.E / 64, NC = (a.E + a.D) / 64;
+  const uint32_t stage_bytes = (uint32_t)NC * kChunk;
+  float* delta = (float*)(smem + nst * stage_bytes);   // [2 sets][IPU][PAIRS][LD]
+  __shared__ __align__(8) uint64_t bars[24];
+  uint64_t* full = bars;            // [3] stage landed (TMA)
+  uint64_t* empty = bars + 3;       // [3] stage gathered (64 walker lanes)
+  uint64_t* tfull = bars + 6;       // [2] accumulators ready (MMA commit)
+  uint64_t* tempty = bars + 8;      // [2] accumulators read (128 epilogue threads)
+  uint64_t* dfull = bars + 10;      // [2] Delta written (128 epilogue threads)
+  uint64_t* dempty = bars + 12;     // [2] Delta taken by the walkers (64 walker lanes)
+  uint64_t* bitsf = bars + 14;      // [2] decisions of a 128-point instance published (32 lanes)
+  uint64_t* cmax = bars + 16;       // partial max |v| exchanged among the epilogue threads
+  uint64_t* mdone = bars + 17;      // every MMA of this CTA complete
+  __shared__ float red[2][4];
+  __shared__ uint32_t bits_s[2][2];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    for (int s = 0; s < nst; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 64);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 128);
+      mbar_init(dfull + b, 128);
+      mbar_init(dempty + b, 64);
+      mbar_init(bitsf + b, 32);
+    }
+    mbar_init(cmax, 128);
+    mbar_init(mdone, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_s, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort = &abort_s;
+  const int n_local = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    // lane ii < IPU handles instance ii of the unit: its record is read before the stage is free
+    const bool tokens = a.src_kind == SRC_TOKENS;
+    int issued = 0;
+    for (int k = 0; k < n_local; ++k) {
+      const int s = k % nst;
+      const int u = blockIdx.x + k * gridDim.x;
+      const int i0 = u * Sh::IPU, ni = min(Sh::IPU, a.n_inst - i0);
+      int row = 0, h = 0;
+      if (lane < ni) {
+        const HalveInst in = a.inst[i0 + lane];
+        row = (int)(in.src_row + (tokens ? 2 * (int64_t)in.pair0 : 0));
+        h = (int)(in.bh % (uint32_t)a.H);
+      }
+      if (!warp_wait(empty + s, ((k / nst) & 1) ^ 1, abort)) break;
+      if (lane == 0) mbar_expect_tx(full + s, (uint32_t)(ni * NC) * (NP * 128));
+      __syncwarp();
+      if (lane < ni) {
+        uint8_t* st = smem + s * stage_bytes + lane * (NP * 128);
+        for (int c = 0; c < NC; ++c) {
+          const bool isk = c < EC;
+          const CUtensorMap* m = isk ? &maps.k : &maps.v;
+          const int x = (isk ? c : c - EC) * 64;
+          if (tokens) tma_load_3d(st + c * kChunk, m, full + s, x, h, row);
+          else tma_load_2d(st + c * kChunk, m, full + s, x, row);
+        }
+      }
+      issued = k + 1;
+    }
+    // leave no copy in flight: the last fill of every stage has landed
+    if (lane == 0) {
+      for (int k = max(0, issued - nst); k < issued; ++k) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(full + (k % nst), (k / nst) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(128, NP, false);
+      const uint32_t base = smem_u32(smem);
+      for (int k = 0; k < n_local; ++k) {
+        const int s = k % nst, b = k & 1;
+        if (!mbar_wait(full + s, (k / nst) & 1, abort)) break;
+        if (!mbar_wait(tempty + b, ((k >> 1) & 1) ^ 1, abort)) break;
+        tc_fence_after();
+        const uint32_t st = base + s * stage_bytes;
+        const uint32_t d = tmem + (uint32_t)b * 256u;
+        for (int c = 0; c < NC; ++c) {
+          const uint32_t ra = st + c * kChunk;
+          const uint32_t dc = d + (c < EC ? 0u : 128u);
+          const bool first = c == 0 || c == EC;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t adesc = sw128_desc(ra + kk * 32, 16, 1024);
+#pragma unroll
+            for (int ii = 0; ii < Sh::IPU; ++ii)
+              umma_bf16(dc + ii * NP, adesc, sw128_desc(ra + ii * (NP * 128) + kk * 32, 16, 1024), IDESC,
+                        (!first || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(tfull + b);
+      }
+      umma_commit(mdone);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(mdone, 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------------ epilogue
+    const int ew = warp - 4;                 // = warp % 4: TMEM lanes 32 ew .. 32 ew + 31
+    const int r = ew * 32 + lane;            // unit row = TMEM lane
+    const int ii = r / NP, lr = r % NP;      // instance within the unit, row within the instance
+    const uint32_t lane_base = (uint32_t)(ew * 32) << 16;
+    const int m = a.m;
+    for (int k = 0; k < n_local; ++k) {
+      const int s = k % nst, b = k & 1;
+      const int u = blockIdx.x + k * gridDim.x;
+      const bool live = u * Sh::IPU + ii < a.n_inst;
+      if (!warp_wait(full + s, (k / nst) & 1, abort)) break;
+      // c = max |v| over the instance: this row's part, then across the instance's threads
+      float mx = 0.f;
+      if (live && lr < a.n) {
+        const uint8_t* rowp = smem + s * stage_bytes + r * 128;
+        for (int c = EC; c < NC; ++c) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint4 w = *(const uint4*)(rowp + c * kChunk + ((q ^ (r & 7)) << 4));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              mx = fmax3(mx, fabsf(__uint_as_float(ws[e] << 16)), fabsf(__uint_as_float(ws[e] & 0xFFFF0000u)));
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) red[k & 1][ew] = mx;
+      mbar_arrive(cmax);
+      if (!warp_wait(cmax, k & 1, abort)) break;
+      float cm;
+      if (NP == 128) cm = fmaxf(fmaxf(red[k & 1][0], red[k & 1][1]), fmaxf(red[k & 1][2], red[k & 1][3]));
+      else if (NP == 64) cm = fmaxf(red[k & 1][2 * ii], red[k & 1][2 * ii + 1]);
+      else cm = red[k & 1][ii];
+      const float c2 = cm * cm;
+      if (!warp_wait(tfull + b, (k >> 1) & 1, abort)) break;
+      if (!warp_wait(dempty + b, ((k >> 1) & 1) ^ 1, abort)) break;
+      tc_fence_after();
+      float* D = delta + b * Sh::DELTA_SET + ii * Sh::DELTA_INST;
+      const int pj = lr >> 1;
+      const bool writer = (lr & 1) == 0;
+      const uint32_t kcol = tmem + lane_base + (uint32_t)b * 256u + (uint32_t)(ii * NP);
+#pragma unroll 1
+      for (int cc = 0; cc < NP / 32; ++cc) {
+        float kk[32], vv[32];
+        tmem_ld32(kcol + cc * 32, kk);
+        tmem_ld32(kcol + 128 + cc * 32, vv);
+        tmem_ld_wait();
+        float dd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float k0 = exp2f(kk[2 * i] * a.scale_log2e) * (vv[2 * i] + c2);
+          const float k1 = exp2f(kk[2 * i + 1] * a.scale_log2e) * (vv[2 * i + 1] + c2);
+          dd[i] = k0 - k1;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dd[i] -= __shfl_xor_sync(0xffffffffu, dd[i], 1);
+        if (writer) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int pi = cc * 16 + i;
+            D[pj * Sh::LD + pi] = (live && pj < m && pi < m) ? dd[i] : 0.f;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty + b);
+      mbar_arrive(dfull + b);
+    }
+  } else {
+    // ------------------------------------------------------------------ walkers (warps 2, 3, 8, 9)
+    const int set = warp >= 8 ? 1 : 0, wi = warp & 1;
+    const int m = a.m, nb = a.m_pad >> 5;
+    const float C = a.C;
+    for (int k = set; k < n_local; k += 2) {
+      const int s = k % nst;
+      const int u = blockIdx.x + k * gridDim.x;
+      const float* Dset = delta + set * Sh::DELTA_SET;
+      const uint8_t* st = smem + s * stage_bytes;
+      if constexpr (NP <= 64) {
+        // one instance per SEG-lane segment: NP = 64 -> warp wi walks instance wi;
+        // NP = 32 -> warp wi walks instances 2wi (lanes 0-15) and 2wi+1 (lanes 16-31)
+        constexpr int SEG = Sh::SEG;
+        const int seg = lane / SEG, sl = lane % SEG;
+        const int ii = wi * (32 / SEG) + seg;
+        const int inst = u * Sh::IPU + ii;
+        const bool live = inst < a.n_inst;
+        HalveInst in{};
+        if (live) in = a.inst[inst];
+        if (!warp_wait(dfull + set, (k >> 1) & 1, abort)) break;
+        const float* D = Dset + ii * Sh::DELTA_INST;
+        float d[SEG];
+#pragma unroll
+        for (int q = 0; q < SEG; ++q) d[q] = D[q * Sh::LD + sl];
+        __syncwarp();
+        mbar_arrive(dempty + set);
+        const float w_l =
+            (live && sl < m) ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)sl) : 0.f;
+        const uint32_t kb = walk_segment<SEG>(d, w_l, C, lane);
+        if (!warp_wait(full + s, (k / nst) & 1, abort)) break;   // (complete: orders the stage reads)
+#pragma unroll
+        for (int g = 0; g < 32 / SEG; ++g) {
+          const int src = g * SEG;
+          const int gi = u * Sh::IPU + wi * (32 / SEG) + g;
+          const uint32_t kbg = __shfl_sync(0xffffffffu, kb, src);
+          const int64_t dst_row = __shfl_sync(0xffffffffu, in.dst_row, src);
+          const int64_t src_row = __shfl_sync(0xffffffffu, in.src_row, src);
+          const uint32_t tok_base = __shfl_sync(0xffffffffu, in.tok0 + 2u * in.pair0, src);
+          if (gi < a.n_inst) {
+            if (a.trace && lane == 0) a.trace[a.trace_base + (size_t)gi * nb] = kbg;
+            gather_from_stage(a, dst_row, src_row, tok_base, st, (wi * (32 / SEG) + g) * NP, 0, m,
+                              [kbg](int i) { return ((kbg >> i) & 1u) != 0; }, lane, EC, NC);
+          }
+        }
+      } else {
+        // one instance of <= 64 pairs: warp wi = 0 walks it as two blocks of 32 (lane l owns pairs
+        // l and l + 32, Delta read from shared memory as it goes) and publishes the decisions; both
+        // warps gather half of the kept rows
+        const int inst = u;
+        const bool live = inst < a.n_inst;
+        const int half = (m + 1) / 2;
+        HalveInst in{};
+        if (live) in = a.inst[inst];
+        uint32_t kb0 = 0, kb1 = 0;
+        if (wi == 0) {
+          if (!warp_wait(dfull + set, (k >> 1) & 1, abort)) break;
+          const float* D = Dset;
+          const float dg0 = D[lane * Sh::LD + lane], dg1 = D[(32 + lane) * Sh::LD + 32 + lane];
+          float w0 = 0.f, w1 = 0.f;
+          if (live) {
+            if (lane < m) w0 = 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)lane);
+            if (lane + 32 < m)
+              w1 = 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + 32u + (uint32_t)lane);
+          }
+          const float rC = 1.f / C;
+          float my0 = 0.f, my1 = 0.f, sigma = 0.f;
+          kb0 = walk_block32(my0, sigma, dg0, w0, C, rC, lane, [&](int q) { return D[q * Sh::LD + lane]; });
+#pragma unroll
+          for (int q = 0; q < 32; ++q) my1 = fmaf(((kb0 >> q) & 1u) ? 1.f : -1.f, D[q * Sh::LD + 32 + lane], my1);
+          kb1 = walk_block32(my1, sigma, dg1, w1, C, rC, lane, [&](int q) { return D[(32 + q) * Sh::LD + 32 + lane]; });
+          __syncwarp();
+          mbar_arrive(dempty + set);
+          if (lane == 0) {
+            bits_s[set][0] = kb0;
+            bits_s[set][1] = kb1;
+          }
+          __syncwarp();
+          mbar_arrive(bitsf + set);
+        } else {
+          if (!warp_wait(bitsf + set, (k >> 1) & 1, abort)) break;
+          kb0 = bits_s[set][0];
+          kb1 = bits_s[set][1];
+          __syncwarp();
+          mbar_arrive(dempty + set);
+        }
+        if (!warp_wait(full + s, (k / nst) & 1, abort)) break;   // (complete: orders the stage reads)
+        if (live) {
+          if (a.trace && wi == 0 && lane < nb) a.trace[a.trace_base + (size_t)inst * nb + lane] = lane ? kb1 : kb0;
+          auto bit = [kb0, kb1](int i) { return (((i < 32 ? kb0 : kb1) >> (i & 31)) & 1u) != 0; };
+          const uint32_t tok_base = in.tok0 + 2u * in.pair0;
+          if (wi == 0) gather_from_stage(a, in.dst_row, in.src_row, tok_base, st, 0, 0, half, bit, lane, EC, NC);
+          else gather_from_stage(a, in.dst_row, in.src_row, tok_base, st, 0, half, m, bit, lane, EC, NC);
+        }
+      }
+      __syncwarp();
+      mbar_arrive(empty + s);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (abort_s && threadIdx.x == 0 && a.status) {
+    if (atomicCAS(a.status, 0, 3) == 0) a.status[1] = (int)blockIdx.x;
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int NP>
+cudaError_t launch_np(const StepArgs& a, cudaStream_t st) {
+  FusedMaps maps;
+  bool ok;
+  if (a.src_kind == SRC_TOKENS) {
+    ok = make_map_3d(&maps.k, a.srcK, a.src_rows, a.H, a.E, NP) && make_map_3d(&maps.v, a.srcV, a.src_rows, a.H, a.D, NP);
+  } else {
+    ok = make_map_2d(&maps.k, a.srcK, a.src_rows, a.E, a.E, NP) && make_map_2d(&maps.v, a.srcV, a.src_rows, a.D, a.D, NP);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  const int NC = (a.E + a.D) / 64;
+  const size_t delta_bytes = 2 * (size_t)FusedShape<NP>::DELTA_SET * 4;
+  const size_t static_bytes = 512;    // barriers and small arrays declared in the kernel
+  int nst = 3;
+  while (nst > 2 && 1024 + (size_t)nst * NC * kChunk + delta_bytes + static_bytes > 227 * 1024) --nst;
+  size_t sm = 1024 + (size_t)nst * NC * kChunk + delta_bytes;
+  if (sm < 120 * 1024) sm = 120 * 1024;   // one CTA per SM: each holds all 512 TMEM columns
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(halve_fused_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const int n_units = (a.n_inst + FusedShape<NP>::IPU - 1) / FusedShape<NP>::IPU;
+  const int grid = n_units < sms ? n_units : sms;
+  halve_fused_kernel<NP><<<grid, kThreads, sm, st>>>(maps, a, n_units, nst);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool halving_fused_supported(const StepArgs& a) {
+  if (std::getenv("THIN_ATTN_UNFUSED_HALVING") != nullptr) return false;
+  if (a.E % 64 || a.D % 64 || (a.E + a.D) / 64 > kMaxChunks || a.n < 2 || a.n > 128 || a.n % 2) return false;
+  if (a.src_rows <= 0 || !tensor_maps_available()) return false;
+  if (a.src_kind == SRC_TOKENS && a.S_sub < a.S_full) return false;   // subsampled rows do not form boxes
+  return true;
+}
+
+cudaError_t launch_halving_fused(const StepArgs& a, cudaStream_t st) {
+  if (a.n_inst == 0) return cudaSuccess;
+  if (a.n <= 32) return launch_np<32>(a, st);
+  if (a.n <= 64) return launch_np<64>(a, st);
+  return launch_np<128>(a, st);
+}
+
+}  // namespace thin

@@ -13,6 +13,10 @@ cudaError_t launch_halving_step(const StepArgs& a, int dtype, bool use_tc, cudaS
 // Tensor-core pair-difference Gram (bf16, E and D multiples of 64); *done = false when the
 // shape is not covered and the CUDA-core kernel must run instead.
 cudaError_t launch_pairgram_tc(const StepArgs& a, cudaStream_t st, bool* done);
+// One-launch halving of instances of <= 128 points (bf16, E and D multiples of 64, E + D <= 320,
+// rows that form TMA boxes): c^2, Gram, walk and gather fused, the points read once.
+bool halving_fused_supported(const StepArgs& a);
+cudaError_t launch_halving_fused(const StepArgs& a, cudaStream_t st);
 // Copy of token runs into compact rows (batches that are not thinned).
 cudaError_t launch_copy_step(const StepArgs& a, int dtype, cudaStream_t st);
 cudaError_t launch_iota(int32_t* idx, int64_t rows, int period, cudaStream_t st);
