@@ -315,16 +315,31 @@ def main():
             "kernel": "attention", "peak_kind": peak_kind,
             "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
             "arithmetic_intensity": round(flops / abytes, 1), "avg_launch_ms": round(attn_ms, 4)}
-    # secondary roofline: the halving steps (thinning + merges), HBM-bound by their algorithmic bytes --
-    # every instance's points read once and its survivors written once: 3 m (E+D) elements per instance
+    # halving rooflines, HBM-bound by their algorithmic bytes -- every instance's n points read once
+    # and its n/2 survivors written once: 1.5 n (E+D) elements per instance.  Per step from the live
+    # per-step CUDA events; the headline is the step that takes longest (the dominant halving kernel),
+    # beside the whole halving phase (latency-bound merges included).
     es = 4 if w.dtype == "fp32" else 2
-    hbytes = sum(3 * m * (w.E + w.D) * es for _, _, _, m, _ in h.trace_layout(w.causal, w.g))
+    sp = h.profile_steps()
+    steps_tab = []
+    for st in sp["steps"]:
+        sb = st["n_inst"] * 3 * st["n"] // 2 * (w.E + w.D) * es
+        sms = st["ms"] / max(1, sp["calls"])
+        steps_tab.append({"n": st["n"], "n_inst": st["n_inst"], "ms": round(sms, 4), "bytes": sb,
+                          "frac": round(sb / (sms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if sms > 0 else None})
+    hbytes = sum(t["bytes"] for t in steps_tab)
     hms = (ph["thin_ms"] + ph["merge_ms"]) / max(1, ph["calls"])
-    halving_roof = {"bound": "hbm", "achieved": round(hbytes / (hms * 1e-3) / 1e9, 1) if hms > 0 else None,
-                    "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(hbytes / (hms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if hms > 0 else None,
-                    "algorithmic_bytes_per_step": hbytes, "ms": round(hms, 4),
-                    "note": "all halving steps of a forward (c^2, Gram, walk, gather launches); latency-bound merges included"}
+    top = max(steps_tab, key=lambda t: t["ms"]) if steps_tab else None
+    halving_roof = None
+    if top and top["ms"] > 0:
+        halving_roof = {"bound": "hbm", "achieved": round(top["bytes"] / (top["ms"] * 1e-3) / 1e9, 1),
+                        "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": top["frac"],
+                        "kernel": f"halving step n={top['n']} x {top['n_inst']} instances",
+                        "algorithmic_bytes_per_launch": top["bytes"], "avg_launch_ms": top["ms"],
+                        "all_steps": {"achieved": round(hbytes / (hms * 1e-3) / 1e9, 1) if hms > 0 else None,
+                                      "frac": round(hbytes / (hms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if hms > 0 else None,
+                                      "bytes": hbytes, "ms": round(hms, 4)},
+                        "steps": steps_tab}
     phases = {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
               "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4),
               "attn_ms": round(attn_ms, 4)}

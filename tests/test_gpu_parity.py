@@ -204,3 +204,50 @@ def test_dropin_call_returns_output_and_none():
     q, k, v = (x.cuda() for x in W.make_qkv(w))
     out, weights = TA.thinformer_attention(q, k, v, g=2, seed=1)
     assert weights is None and out.shape == (1, 256, 1, 64)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_fused_and_three_launch_halving_agree(causal, monkeypatch):
+    """The one-launch small-instance halving kernel and the c^2 / Gram / walk launches take the same
+    decisions (same arithmetic), so traces, coresets, outputs and LSE are bit-identical."""
+    if causal:
+        w = W.WORKLOADS["express32k"].with_(T=8192, H=4)
+        S = w.T
+    else:
+        w = W.WORKLOADS["express32k"].with_(T=512, H=2, B=2, causal=False, S=1024)
+        S = 1024
+    q, k, v = (x.cuda() for x in W.make_qkv(w, T=w.T, S=S))
+    res = []
+    for unfused in (False, True):
+        if unfused:
+            monkeypatch.setenv("THIN_ATTN_UNFUSED_HALVING", "1")
+        else:
+            monkeypatch.delenv("THIN_ATTN_UNFUSED_HALVING", raising=False)
+        h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
+        r = h.forward(q, k, v, causal=causal, g=w.g, seed=w.seed, return_lse=True, return_coreset=True,
+                      return_trace=True)
+        torch.cuda.synchronize()
+        h.check()
+        res.append(r)
+    for key in ("trace", "coreset", "out", "lse"):
+        assert torch.equal(res[0][key], res[1][key]), key
+
+
+def test_profile_steps_cover_the_halving_phases():
+    w = W.WORKLOADS["express32k"].with_(T=8192, H=4)
+    q, k, v = (x.cuda() for x in W.make_qkv(w))
+    h = TA.ThinAttention(w.B, w.T, w.T, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
+    h.forward(q, k, v, causal=True, g=w.g, seed=w.seed)
+    h.profile(True)
+    for _ in range(2):
+        h.forward(q, k, v, causal=True, g=w.g, seed=w.seed)
+    h.profile(False)
+    ph = h.profile_read()
+    sp = h.profile_steps()
+    assert ph["calls"] == 2 and sp["calls"] == 2
+    steps = sp["steps"]
+    assert len(steps) > 0 and all(s["ms"] > 0 and s["n_inst"] > 0 and s["n"] >= 2 for s in steps)
+    total = sum(s["ms"] for s in steps)
+    assert abs(total - (ph["thin_ms"] + ph["merge_ms"])) <= 0.05 * total + 1e-3
+    again = h.profile_steps()
+    assert again["calls"] == 0 and all(s["ms"] == 0 for s in again["steps"])

@@ -55,6 +55,7 @@ _lib = None
 EXPORTS = ("thin_attn_version", "thin_attn_last_error", "thin_attn_create", "thin_attn_destroy",
            "thin_attn_plan", "thin_attn_reserve", "thin_attn_trace_layout", "thin_attn_forward",
            "thin_attn_forward_host", "thin_attn_check", "thin_attn_profile", "thin_attn_profile_read",
+           "thin_attn_profile_steps",
            "thin_attn_cache_create", "thin_attn_cache_destroy", "thin_attn_cache_length", "thin_attn_cache_decode",
            "thin_attn_cache_nodes", "thin_attn_cache_check")
 
@@ -87,6 +88,8 @@ def lib() -> ctypes.CDLL:
     L.thin_attn_cache_check.argtypes = [vp, vp]
     L.thin_attn_profile.argtypes = [vp, i]
     L.thin_attn_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
+    ip = ctypes.POINTER(ctypes.c_int)
+    L.thin_attn_profile_steps.argtypes = [vp, i, ctypes.POINTER(ctypes.c_double), ip, ip, ip, ip]
     for f in EXPORTS[2:]:
         getattr(L, f).restype = ctypes.c_int
     _lib = L
@@ -202,6 +205,17 @@ class ThinAttention:
         calls = ctypes.c_int()
         _check(lib().thin_attn_profile_read(self._h, ms, ctypes.byref(calls)))
         return {"thin_ms": ms[0], "merge_ms": ms[1], "attn_ms": ms[2], "total_ms": ms[3], "calls": calls.value}
+
+    def profile_steps(self):
+        """Summed device time (ms) of every halving step of the forwards recorded since the last
+        call, in launch order, with each step's instances and points per instance."""
+        cap = 64
+        ms = (ctypes.c_double * cap)()
+        ni, npt = (ctypes.c_int * cap)(), (ctypes.c_int * cap)()
+        ns, calls = ctypes.c_int(), ctypes.c_int()
+        _check(lib().thin_attn_profile_steps(self._h, cap, ms, ni, npt, ctypes.byref(ns), ctypes.byref(calls)))
+        return {"calls": calls.value,
+                "steps": [{"ms": ms[j], "n_inst": ni[j], "n": npt[j]} for j in range(min(ns.value, cap))]}
 
     def check(self):
         stream = torch.cuda.current_stream(self.device).cuda_stream

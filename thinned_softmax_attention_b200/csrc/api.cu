@@ -151,6 +151,10 @@ struct thin_attn_s {
   double prof_ms[3] = {0, 0, 0};
   double prof_total = 0;
   int prof_calls = 0;
+  // per halving step: summed ms and the step's shape (instances, points per instance)
+  std::vector<double> prof_step_ms;
+  std::vector<int> prof_step_inst, prof_step_n;
+  int prof_step_calls = 0;
 };
 
 namespace {
@@ -563,6 +567,28 @@ void buf_ptrs(Plan* p, int id, const void* k, const void* v, const void** K, con
   *idx = (int32_t*)(base_of(p) + b.idx_off);
 }
 
+// Rows of a step's source: the (B*L) token rows, or the rows of its compact buffer.
+int64_t src_rows_of(const thin_attn_config& cf, const Plan* p, const StepPlan& sp) {
+  return sp.src_buf == BUF_TOKENS ? (int64_t)cf.B * (p->causal ? cf.T : cf.S)
+         : (sp.src_buf == BUF_NODES ? p->nodes : sp.src_buf == BUF_MTEMP ? p->mtemp : p->levels[sp.src_buf]).rows;
+}
+
+// Kernels a step launches: 1 (copy, or the fused small-instance kernel) or 3 (c^2, Gram, walk).
+int step_launches(const thin_attn_config& cf, const Plan* p, const StepPlan& sp) {
+  if (sp.inst.empty()) return 0;
+  if (sp.copy_only) return 1;
+  StepArgs a{};
+  a.src_kind = sp.src_buf == BUF_TOKENS ? SRC_TOKENS : SRC_COMPACT;
+  a.src_rows = src_rows_of(cf, p, sp);
+  a.S_full = sp.S_full;
+  a.S_sub = sp.S_sub;
+  a.n = sp.n;
+  a.E = cf.E;
+  a.D = cf.D;
+  const bool tc = cf.dtype == 1 && std::getenv("THIN_ATTN_SIMT_GRAM") == nullptr;
+  return tc && halving_fused_supported(a) ? 1 : 3;
+}
+
 thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void* k, const void* v, void* out,
                              uint64_t seed, float* lse, int32_t* cidx, uint32_t* trace, cudaStream_t st) {
   const thin_attn_config& cf = h->cfg;
@@ -603,10 +629,12 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     sa = h->side;
   }
   // profiling events: [0] start, [1] first merge step, [2] all halving steps, [3] end (joined),
-  // then a (start, stop) pair per attention wave on the attention stream
+  // then a (start, stop) pair per attention wave on the attention stream, then the end of every
+  // halving step on the halving stream
   std::vector<cudaEvent_t> ev;
+  const size_t ev_steps = 4 + 2 * waves.size();
   if (h->prof_on) {
-    const size_t need = 4 + 2 * waves.size();
+    const size_t need = ev_steps + p->steps.size();
     if (!h->prof_free.empty() && h->prof_free.back().size() >= need) {
       ev = h->prof_free.back();
       h->prof_free.pop_back();
@@ -678,8 +706,7 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     int32_t* didx;
     buf_ptrs(p, sp.dst_buf, k, v, &dk, &dv, &didx);
     a.src_kind = sp.src_buf == BUF_TOKENS ? SRC_TOKENS : SRC_COMPACT;
-    a.src_rows = sp.src_buf == BUF_TOKENS ? (int64_t)cf.B * (p->causal ? cf.T : cf.S)
-                 : (sp.src_buf == BUF_NODES ? p->nodes : sp.src_buf == BUF_MTEMP ? p->mtemp : p->levels[sp.src_buf]).rows;
+    a.src_rows = src_rows_of(cf, p, sp);
     a.status = h->d_status;
     a.srcK = sk;
     a.srcV = sv;
@@ -707,6 +734,7 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     cudaError_t e = sp.copy_only ? launch_copy_step(a, cf.dtype, st)
                                  : launch_halving_step(a, cf.dtype, use_tc_gram, st);
     if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "halving step (n=%d): %s", sp.n, cudaGetErrorString(e));
+    if (!ev.empty()) CK(cudaEventRecord(ev[ev_steps + si], st));
     if (si + 1 < p->steps.size()) {
       ls = launch_waves_after((int)si);
       if (ls != THIN_ATTN_OK) return ls;
@@ -739,6 +767,16 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   if (!ev.empty()) {
     CK(cudaEventRecord(ev[3], st));
     h->prof_pending.push_back({ev, waves.size()});
+    if (h->prof_step_ms.size() != p->steps.size()) {
+      h->prof_step_ms.assign(p->steps.size(), 0.0);
+      h->prof_step_inst.resize(p->steps.size());
+      h->prof_step_n.resize(p->steps.size());
+      h->prof_step_calls = 0;
+    }
+    for (size_t si = 0; si < p->steps.size(); ++si) {
+      h->prof_step_inst[si] = (int)p->steps[si].inst.size();
+      h->prof_step_n[si] = p->steps[si].n;
+    }
   }
   return THIN_ATTN_OK;
 }
@@ -801,7 +839,7 @@ thin_attn_status thin_attn_plan(thin_attn_t h, int causal, int g, thin_attn_plan
   info->n_nodes = p->n_slots;
   info->n_halvings = (int)p->trace.size();
   int launches = 1;
-  for (auto& st : p->steps) launches += st.inst.empty() ? 0 : (st.copy_only ? 1 : 3);
+  for (auto& st : p->steps) launches += step_launches(h->cfg, p, st);
   info->kernel_launches = launches;
   info->trace_words = p->trace_words;
   info->coreset_idx_elems = p->coreset_idx_elems;
@@ -902,9 +940,11 @@ thin_attn_status thin_attn_profile(thin_attn_t h, int enable) {
   return THIN_ATTN_OK;
 }
 
-thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms, int* calls) {
-  if (!h || !ms || !calls) return fail(THIN_ATTN_EINVAL, "null argument");
-  std::lock_guard<std::mutex> lk(h->mu);
+}  // extern "C"
+
+namespace {
+// Wait for the recorded forwards and add their times to the phase and step sums (lock held).
+thin_attn_status drain_profile(thin_attn_s* h) {
   DeviceGuard dg(h->prof_pending.empty() ? -1 : h->cfg.device);
   for (auto& pe : h->prof_pending) {
     auto& ev = pe.first;
@@ -914,16 +954,53 @@ thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms, int* calls) {
     h->prof_ms[0] += t;
     CK(cudaEventElapsedTime(&t, ev[1], ev[2]));
     h->prof_ms[1] += t;
+    const size_t first_step = 4 + 2 * pe.second;
     for (size_t w = 0; w < pe.second; ++w) {
       CK(cudaEventElapsedTime(&t, ev[4 + 2 * w], ev[5 + 2 * w]));
       h->prof_ms[2] += t;
     }
+    for (size_t si = 0; si < h->prof_step_ms.size() && first_step + si < ev.size(); ++si) {
+      CK(cudaEventElapsedTime(&t, si ? ev[first_step + si - 1] : ev[0], ev[first_step + si]));
+      h->prof_step_ms[si] += t;
+    }
     CK(cudaEventElapsedTime(&t, ev[0], ev[3]));
     h->prof_total += t;
     h->prof_calls += 1;
+    h->prof_step_calls += 1;
     h->prof_free.push_back(ev);
   }
   h->prof_pending.clear();
+  return THIN_ATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+thin_attn_status thin_attn_profile_steps(thin_attn_t h, int max_steps, double* ms, int* n_inst, int* n_points,
+                                         int* n_steps, int* calls) {
+  if (!h || !n_steps || !calls || max_steps < 0 || (max_steps > 0 && (!ms || !n_inst || !n_points)))
+    return fail(THIN_ATTN_EINVAL, "null argument");
+  std::lock_guard<std::mutex> lk(h->mu);
+  thin_attn_status s = drain_profile(h);
+  if (s != THIN_ATTN_OK) return s;
+  const int ns = (int)h->prof_step_ms.size();
+  for (int i = 0; i < ns && i < max_steps; ++i) {
+    ms[i] = h->prof_step_ms[i];
+    n_inst[i] = h->prof_step_inst[i];
+    n_points[i] = h->prof_step_n[i];
+    h->prof_step_ms[i] = 0;
+  }
+  *n_steps = ns;
+  *calls = h->prof_step_calls;
+  h->prof_step_calls = 0;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms, int* calls) {
+  if (!h || !ms || !calls) return fail(THIN_ATTN_EINVAL, "null argument");
+  std::lock_guard<std::mutex> lk(h->mu);
+  thin_attn_status s = drain_profile(h);
+  if (s != THIN_ATTN_OK) return s;
   for (int i = 0; i < 3; ++i) ms[i] = h->prof_ms[i];
   ms[3] = h->prof_total;
   *calls = h->prof_calls;

@@ -114,8 +114,10 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
   uint64_t* bitsf = bars + 14;      // [2] decisions of a 128-point instance published (32 lanes)
   uint64_t* cmax = bars + 16;       // partial max |v| exchanged among the epilogue threads
   uint64_t* mdone = bars + 17;      // every MMA of this CTA complete
+  uint64_t* thf = bars + 18;        // [2] thresholds of one block of 32 pairs published (32 lanes)
   __shared__ float red[2][4];
   __shared__ uint32_t bits_s[2][2];
+  __shared__ float thr_s[2][64];
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
 
@@ -132,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
       mbar_init(dfull + b, 128);
       mbar_init(dempty + b, 64);
       mbar_init(bitsf + b, 32);
+      mbar_init(thf + b, 32);
     }
     mbar_init(cmax, 128);
     mbar_init(mdone, 1);
@@ -332,31 +335,45 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
           }
         }
       } else {
-        // one instance of <= 64 pairs: warp wi = 0 walks it as two blocks of 32 (lane l owns pairs
-        // l and l + 32, Delta read from shared memory as it goes) and publishes the decisions; both
-        // warps gather half of the kept rows
+        // one instance of <= 64 pairs as two blocks of 32: warp wi = 1 computes the thresholds
+        // (sigma's recursion) of block 0 then block 1, warp wi = 0 walks each block as soon as its
+        // thresholds are published (lane l owns pairs l and l + 32), then publishes the decisions;
+        // both warps gather half of the kept rows
         const int inst = u;
         const bool live = inst < a.n_inst;
         const int half = (m + 1) / 2;
         HalveInst in{};
         if (live) in = a.inst[inst];
+        if (!warp_wait(dfull + set, (k >> 1) & 1, abort)) break;
+        const float* D = Dset;
         uint32_t kb0 = 0, kb1 = 0;
-        if (wi == 0) {
-          if (!warp_wait(dfull + set, (k >> 1) & 1, abort)) break;
-          const float* D = Dset;
-          const float dg0 = D[lane * Sh::LD + lane], dg1 = D[(32 + lane) * Sh::LD + 32 + lane];
-          float w0 = 0.f, w1 = 0.f;
-          if (live) {
-            if (lane < m) w0 = 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)lane);
-            if (lane + 32 < m)
-              w1 = 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + 32u + (uint32_t)lane);
-          }
+        if (wi == 1) {
           const float rC = 1.f / C;
-          float my0 = 0.f, my1 = 0.f, sigma = 0.f;
-          kb0 = walk_block32(my0, sigma, dg0, w0, C, rC, lane, [&](int q) { return D[q * Sh::LD + lane]; });
+          float sigma = 0.f;
+#pragma unroll 1
+          for (int blk = 0; blk < 2; ++blk) {
+            const int p = 32 * blk + lane;
+            const float b2l = D[p * Sh::LD + p];
+            const float wl =
+                (live && p < m) ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)p) : 0.f;
+            thr_s[set][p] = thresholds32(sigma, b2l, wl, C, rC, lane);
+            __syncwarp();
+            mbar_arrive(thf + set);
+          }
+          __syncwarp();
+          mbar_arrive(dempty + set);
+          if (!warp_wait(bitsf + set, (k >> 1) & 1, abort)) break;
+          kb0 = bits_s[set][0];
+          kb1 = bits_s[set][1];
+        } else {
+          float my0 = 0.f, my1 = 0.f;
+          if (!warp_wait(thf + set, 0, abort)) break;
+          kb0 = walk_block32_th(my0, thr_s[set][lane], min(32, m), lane, [&](int q) { return D[q * Sh::LD + lane]; });
 #pragma unroll
           for (int q = 0; q < 32; ++q) my1 = fmaf(((kb0 >> q) & 1u) ? 1.f : -1.f, D[q * Sh::LD + 32 + lane], my1);
-          kb1 = walk_block32(my1, sigma, dg1, w1, C, rC, lane, [&](int q) { return D[(32 + q) * Sh::LD + 32 + lane]; });
+          if (!warp_wait(thf + set, 1, abort)) break;
+          kb1 = walk_block32_th(my1, thr_s[set][32 + lane], m - 32, lane,
+                                [&](int q) { return D[(32 + q) * Sh::LD + 32 + lane]; });
           __syncwarp();
           mbar_arrive(dempty + set);
           if (lane == 0) {
@@ -365,20 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
           }
           __syncwarp();
           mbar_arrive(bitsf + set);
-        } else {
-          if (!warp_wait(bitsf + set, (k >> 1) & 1, abort)) break;
-          kb0 = bits_s[set][0];
-          kb1 = bits_s[set][1];
-          __syncwarp();
-          mbar_arrive(dempty + set);
         }
         if (!warp_wait(full + s, (k / nst) & 1, abort)) break;   // (complete: orders the stage reads)
         if (live) {
           if (a.trace && wi == 0 && lane < nb) a.trace[a.trace_base + (size_t)inst * nb + lane] = lane ? kb1 : kb0;
           auto bit = [kb0, kb1](int i) { return (((i < 32 ? kb0 : kb1) >> (i & 31)) & 1u) != 0; };
           const uint32_t tok_base = in.tok0 + 2u * in.pair0;
-          if (wi == 0) gather_from_stage(a, in.dst_row, in.src_row, tok_base, st, 0, 0, half, bit, lane, EC, NC);
-          else gather_from_stage(a, in.dst_row, in.src_row, tok_base, st, 0, half, m, bit, lane, EC, NC);
+          gather_from_stage(a, in.dst_row, in.src_row, tok_base, st, 0, wi ? half : 0, wi ? m : half, bit, lane, EC, NC);
         }
       }
       __syncwarp();
@@ -409,7 +419,7 @@ cudaError_t launch_np(const StepArgs& a, cudaStream_t st) {
   if (!ok) return cudaErrorInvalidValue;
   const int NC = (a.E + a.D) / 64;
   const size_t delta_bytes = 2 * (size_t)FusedShape<NP>::DELTA_SET * 4;
-  const size_t static_bytes = 512;    // barriers and small arrays declared in the kernel
+  const size_t static_bytes = 1024;   // barriers and small arrays declared in the kernel
   int nst = 3;
   while (nst > 2 && 1024 + (size_t)nst * NC * kChunk + delta_bytes + static_bytes > 227 * 1024) --nst;
   size_t sm = 1024 + (size_t)nst * NC * kChunk + delta_bytes;

@@ -106,4 +106,41 @@ __device__ __forceinline__ uint32_t walk_block32(float& my, float& sigma, float 
   return kb;
 }
 
+// Thresholds of the pairs base..base+31, computed by one warp ahead of the warp that walks them:
+// th = a (1 - 2u) for a pair with b^2 > 0 and +inf otherwise (such a pair keeps its first point).
+// b2l and wl are b^2 and 1 - 2u of pair base + lane (0 for lanes that hold no pair); sigma carries
+// over from block to block.  Lane l returns the threshold of pair base + l.  The sigma recursion,
+// the threshold and their order are those of walk_block32, so the decisions are the same.
+__device__ __forceinline__ float thresholds32(float& sigma, float b2l, float wl, float C, float rC, int lane) {
+  float th_l = __int_as_float(0x7f800000);
+#pragma unroll
+  for (int s = 0; s < 32; ++s) {
+    const float b2 = __shfl_sync(0xffffffffu, b2l, s);
+    const float a = sigma_thr(sigma, b2, C, rC);
+    if (lane == s && b2 > 0.f) th_l = a * wl;
+  }
+  return th_l;
+}
+
+// The decisions of pairs base..base+31 with thresholds from thresholds32 (th_l of pair base+lane):
+// the warp's only serial chain is alpha -> ballot -> alpha.  Pairs s >= steps are padding and keep
+// their first point; their alpha updates touch only lanes that hold no pair.
+template <typename Col>
+__device__ __forceinline__ uint32_t walk_block32_th(float& my, float th_l, int steps, int lane, Col col) {
+  // the column is read into registers first so that no shared-memory load sits on the chain
+  float d[32];
+#pragma unroll
+  for (int s = 0; s < 32; ++s) d[s] = col(s);
+  uint32_t kb = 0;
+#pragma unroll
+  for (int s = 0; s < 32; ++s) {
+    const float th = __shfl_sync(0xffffffffu, th_l, s);
+    const uint32_t bal = __ballot_sync(0xffffffffu, my < th);
+    const bool keep = s >= steps || ((bal >> s) & 1u);
+    if (lane > s) my = fmaf(keep ? 1.f : -1.f, d[s], my);
+    kb |= (uint32_t)keep << s;
+  }
+  return kb;
+}
+
 }  // namespace thin
