@@ -422,7 +422,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, 
     }
   }
   const float off = m_used == -INFINITY ? 0.f : lw2 - m_used;
-  float ls[4] = {0.f, 0.f, 0.f, 0.f};
+  // two scores per instruction: the scale-and-offset FMA and the row-sum add run on packed fp32
+  // pairs (sm_100 FFMA2 / FADD2), which leaves one EX2 per score and one bf16x2 pack per pair
+  const float2 sl2e2 = make_float2(sl2e, sl2e), off2 = make_float2(off, off);
+  float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
     float z[32];
@@ -436,15 +439,16 @@ __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, 
         z0 = c * 32 + 2 * e <= lim ? z0 : -INFINITY;
         z1 = c * 32 + 2 * e + 1 <= lim ? z1 : -INFINITY;
       }
-      const float p0 = ex2_approx(fmaf(z0, sl2e, off));
-      const float p1 = ex2_approx(fmaf(z1, sl2e, off));
-      ls[e & 3] += p0 + p1;
+      const float2 t = __ffma2_rn(make_float2(z0, z1), sl2e2, off2);
+      const float p0 = ex2_approx(t.x);
+      const float p1 = ex2_approx(t.y);
+      ls2[e & 1] = __fadd2_rn(ls2[e & 1], make_float2(p0, p1));
       const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
       pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
     }
     tmem_st16(tmem + lane_base + c * 16, pk);
   }
-  l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+  l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
 }
 
 template <int E, int D>
