@@ -384,21 +384,27 @@ __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, 
                                              int it, float& m_used, float& l) {
   constexpr uint32_t O_COL = 128;
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  // row max: two 32-column loads in flight per wait
 #pragma unroll
-  for (int c = 0; c < BN / 32; ++c) {
-    float z[32];
-    tmem_ld32(tmem + lane_base + c * 32, z);
+  for (int c2 = 0; c2 < BN / 64; ++c2) {
+    float z[2][32];
+    tmem_ld32(tmem + lane_base + c2 * 64, z[0]);
+    tmem_ld32(tmem + lane_base + c2 * 64 + 32, z[1]);
     tmem_ld_wait();
-    if (MASKED) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) z[i] = c * 32 + i <= lim ? z[i] : -INFINITY;
-    }
+    for (int h = 0; h < 2; ++h) {
+      const int c = 2 * c2 + h;
+      if (MASKED) {
 #pragma unroll
-    for (int i = 0; i < 32; i += 8) {
-      mx4[0] = fmax3(mx4[0], z[i], z[i + 1]);
-      mx4[1] = fmax3(mx4[1], z[i + 2], z[i + 3]);
-      mx4[2] = fmax3(mx4[2], z[i + 4], z[i + 5]);
-      mx4[3] = fmax3(mx4[3], z[i + 6], z[i + 7]);
+        for (int i = 0; i < 32; ++i) z[h][i] = c * 32 + i <= lim ? z[h][i] : -INFINITY;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) {
+        mx4[0] = fmax3(mx4[0], z[h][i], z[h][i + 1]);
+        mx4[1] = fmax3(mx4[1], z[h][i + 2], z[h][i + 3]);
+        mx4[2] = fmax3(mx4[2], z[h][i + 4], z[h][i + 5]);
+        mx4[3] = fmax3(mx4[3], z[h][i + 6], z[h][i + 7]);
+      }
     }
   }
   const float smax = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
@@ -426,11 +432,14 @@ __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, 
   // pairs (sm_100 FFMA2 / FADD2), which leaves one EX2 per score and one bf16x2 pack per pair
   const float2 sl2e2 = make_float2(sl2e, sl2e), off2 = make_float2(off, off);
   float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  // 32 columns at a time, the next 32 loading while these are exponentiated
+  float zb[2][32];
+  tmem_ld32(tmem + lane_base, zb[0]);
+  tmem_ld_wait();
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
-    float z[32];
-    tmem_ld32(tmem + lane_base + c * 32, z);
-    tmem_ld_wait();
+    if (c + 1 < BN / 32) tmem_ld32(tmem + lane_base + (c + 1) * 32, zb[(c + 1) & 1]);
+    const float* z = zb[c & 1];
     uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -447,6 +456,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, 
       pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
     }
     tmem_st16(tmem + lane_base + c * 16, pk);
+    if (c + 1 < BN / 32) tmem_ld_wait();
   }
   l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
 }
