@@ -381,7 +381,7 @@ struct Tc2Layout {
 // trip when some row's max grew by more than 2^8).  MASKED: keys c > lim are invisible.
 template <bool MASKED, int D>
 __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, int lim, float sl2e, float lw2,
-                                             int it, float& m_used, float& l) {
+                                             int it, float& m_used, float& l, uint64_t* p_half) {
   constexpr uint32_t O_COL = 128;
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   // row max: two 32-column loads in flight per wait
@@ -456,6 +456,12 @@ __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, 
       pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
     }
     tmem_st16(tmem + lane_base + c * 16, pk);
+    if (c == BN / 64 - 1) {
+      // P of the first half of the keys is in place: the MMA warp starts its half of PV
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_half);
+    }
     if (c + 1 < BN / 32) tmem_ld_wait();
   }
   l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
@@ -478,8 +484,9 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
   uint64_t* v_full = bars + 3;
   uint64_t* v_empty = bars + 4;
   uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
+  uint64_t* p_full = bars + 6;      // P of all keys of the tile written (128 threads)
   uint64_t* pv_done = bars + 7;
+  uint64_t* p_half = bars + 8;      // P of keys 0..BN/2-1 written (128 threads)
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
   __shared__ volatile int where_s;
@@ -501,6 +508,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
     mbar_init(s_full, 1);
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
+    mbar_init(p_half, 128);
     fence_barrier_init();
   }
   if (warp == 5) tmem_alloc(&tmem_base_s, 256);
@@ -586,15 +594,24 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
         }
         umma_commit(s_full);
         umma_commit(k_empty);
-        if (!mbar_wait(p_full, it & 1, abort) || !mbar_wait(v_full, it & 1, abort)) {
+        // PV in two halves over the keys: the first as soon as P of keys 0..BN/2-1 is written
+        if (!mbar_wait(p_half, it & 1, abort) || !mbar_wait(v_full, it & 1, abort)) {
           atomicCAS((int*)&where_s, 0, 5000 + min(it, 999));
           break;
         }
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < BN / 16; ++k)
+        for (int k = 0; k < BN / 32; ++k)
           umma_bf16_tmem_a(tmem + O_COL, tmem + k * 8, sw128_desc(va + k * 2048, 16384, 1024), IPV,
                            (it > 0 || k > 0) ? 1u : 0u);
+        if (!mbar_wait(p_full, it & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 7000 + min(it, 999));
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = BN / 32; k < BN / 16; ++k)
+          umma_bf16_tmem_a(tmem + O_COL, tmem + k * 8, sw128_desc(va + k * 2048, 16384, 1024), IPV, 1u);
         umma_commit(pv_done);
         umma_commit(v_empty);
       }
@@ -622,8 +639,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
         const bool causal = sg.kind == SEG_TOKENS && sg.causal;
         const bool masked = nvalid < BN || (causal && kt0 + BN - 1 > tile.q0);
         const int lim = min(nvalid - 1, causal ? tq - kt0 : BN - 1);
-        if (masked) softmax_tile<true, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l);
-        else softmax_tile<false, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l);
+        if (masked) softmax_tile<true, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
+        else softmax_tile<false, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);
