@@ -336,6 +336,7 @@ def main():
                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": top["frac"],
                         "kernel": f"halving step n={top['n']} x {top['n_inst']} instances",
                         "algorithmic_bytes_per_launch": top["bytes"], "avg_launch_ms": top["ms"],
+                        "traffic": kernel_traffic("halving_fused_n64") if (w.name == "express32k" and top["n"] == 64) else None,
                         "all_steps": {"achieved": round(hbytes / (hms * 1e-3) / 1e9, 1) if hms > 0 else None,
                                       "frac": round(hbytes / (hms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if hms > 0 else None,
                                       "bytes": hbytes, "ms": round(hms, 4)},
