@@ -47,6 +47,9 @@ def args_():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-sdpa", action="store_true")
+    p.add_argument("--decode", action="store_true",
+                   help="time token-by-token decoding of the workload through the Express decode cache "
+                        "(causal workloads; prints its own JSON line)")
     return p.parse_args()
 
 
@@ -244,10 +247,67 @@ def config_of(w):
             "inputs smaller than L2"}
 
 
+def run_decode(a):
+    """Decode the whole workload one token per (b,h) and call through thin_attn_cache_decode.
+
+    Timed with CUDA events from the end of the exact prefix to the last token.  Roofline: HBM, every
+    visible key/value row read once per decoded token (the attention of a single query re-reads its
+    whole key set) plus q read and out written -- the batch thinning and merges on completed batches
+    are included in the time but not in these bytes."""
+    import thinned_softmax_attention_b200 as TA
+    w = W.WORKLOADS[a.workload]
+    if not w.causal:
+        raise SystemExit("--decode needs a causal (Express) workload")
+    dev = torch.device("cuda", 0)
+    q, k, v = (x.to(dev) for x in W.make_qkv(w))
+    h = TA.ThinAttention(w.B, w.T, w.T, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
+    plan = h.plan(True, w.g)
+    cache = TA.ThinAttentionCache(w.B, w.H, w.E, w.D, w.torch_dtype, capacity=w.T, n_exact=w.n_exact,
+                                  batch=w.batch, g=w.g, seed=w.seed)
+    out = torch.empty(w.B, 1, w.H, w.D, dtype=w.torch_dtype, device=dev)
+    ne, T = min(w.n_exact, w.T), w.T
+    tail = min(256, T - ne)
+    stream = torch.cuda.current_stream(dev)
+    ev = {n: torch.cuda.Event(enable_timing=True) for n in ("start", "tail", "end")}
+    clocks = Clocks(0)
+    for t in range(T):
+        if t == ne:
+            ev["start"].record(stream)
+        if t == T - tail:
+            ev["tail"].record(stream)
+        cache.decode(q[:, t:t + 1], k[:, t:t + 1], v[:, t:t + 1], out=out)
+    ev["end"].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    cache.check()
+    ms = ev["start"].elapsed_time(ev["end"])
+    tail_ms = ev["tail"].elapsed_time(ev["end"]) / tail
+    n_tok = T - ne
+    es = 4 if w.dtype == "fp32" else 2
+    tt = np.arange(ne, T, dtype=np.int64)
+    c, b = plan["coreset_rows"], w.batch
+    kk = (tt - ne) // b
+    vis = ne + c * digitsum4(kk) + (tt - (ne + kk * b) + 1)
+    abytes = float(vis.sum() + 2 * n_tok) * (w.E + w.D) * es * w.B * w.H
+    pk = peaks()
+    gbs = abytes / (ms * 1e-3) / 1e9
+    line = {"metric": "decode tokens/s (B*H tokens per decoded position) through the Express decode cache",
+            "value": w.B * w.H * n_tok / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "higher_is_better": True,
+            "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
+            "positions": [ne, T], "ms_per_position": round(ms / n_tok, 5), "tail_ms_per_position": round(tail_ms, 5),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / pk["hbm_gbs"], 4), "algorithmic_bytes": abytes,
+                         "note": "visible keys/values re-read per position; thinning and merges in the time only"},
+            "clocks": clk}
+    print(json.dumps(line))
+
+
 def main():
     a = args_()
     if a.impl == "reference":
         return run_reference(a)
+    if a.decode:
+        return run_decode(a)
     import thinned_softmax_attention_b200 as TA
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

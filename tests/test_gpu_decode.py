@@ -14,12 +14,16 @@ import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("T,n_e,bsz,g,dtype", [
-    (1152, 128, 64, 2, "bf16"),     # 16 batches: level-1 merges and one level-2 merge
-    (700, 100, 96, 2, "bf16"),      # batch not a power of 4 (subsample), trailing partial batch
-    (300, 40, 16, 2, "fp32"),       # batches stored whole (no thinning), fp32 path
+@pytest.mark.parametrize("T,n_e,bsz,g,dtype,tiles", [
+    (1152, 128, 64, 2, "bf16", False),   # 16 batches: level-1 merges and one level-2 merge
+    (1152, 128, 64, 2, "bf16", True),    # the same through the query-tile attention kernels
+    (700, 100, 96, 2, "bf16", False),    # batch not a power of 4 (subsample), trailing partial batch
+    (300, 40, 16, 2, "fp32", False),     # batches stored whole (no thinning), fp32 path
 ])
-def test_decode_matches_prefill(T, n_e, bsz, g, dtype):
+def test_decode_matches_prefill(T, n_e, bsz, g, dtype, tiles, monkeypatch):
+    """Few (b,h) rows take the split-key decode kernels; `tiles` forces the query-tile kernels."""
+    if tiles:
+        monkeypatch.setenv("THIN_ATTN_DECODE_TILES", "1")
     E = D = 128 if dtype == "bf16" else 64
     w = W.Workload("decode", 1, 2, T, T, E, D, dtype, True, g, 9, 6, "rope", n_exact=n_e, batch=bsz)
     q, k, v = (x.cuda() for x in W.make_qkv(w))

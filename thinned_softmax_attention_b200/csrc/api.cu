@@ -1061,6 +1061,11 @@ struct thin_attn_cache_s {
   int* d_status = nullptr;
   int64_t t = 0;
   bool use_tc = false;
+  // split-key decode attention: keys of every position, chunks of the largest, partials buffer
+  bool use_split = false;
+  std::vector<int> pos_keys;
+  int max_splits = 0;
+  size_t part_off = 0;
 };
 
 namespace {
@@ -1189,6 +1194,17 @@ thin_attn_status cache_build(thin_attn_cache_s* cc) {
     }
     t.tiles.push_back({0, 1, seg0, (int)t.segs.size() - seg0});
   }
+  int max_segs = 0;
+  cc->pos_keys.assign(T, 0);
+  for (int pos = 0; pos < T; ++pos) {
+    const AttnTile& tl = t.tiles[pos];
+    max_segs = std::max(max_segs, tl.nseg);
+    for (int q = 0; q < tl.nseg; ++q) cc->pos_keys[pos] += t.segs[tl.seg0 + q].len;
+    cc->max_splits = std::max(cc->max_splits, (cc->pos_keys[pos] + decode_chunk_keys() - 1) / decode_chunk_keys());
+  }
+  // split-key kernels when few (b,h) rows would leave most SMs idle with one CTA per row
+  cc->use_split = decode_attention_supported(cf.E, cf.D, max_segs) && BH <= 64 &&
+                  std::getenv("THIN_ATTN_DECODE_TILES") == nullptr;
   // device layout
   size_t off = 0;
   for (auto& steps : cc->batch_steps)
@@ -1223,6 +1239,8 @@ thin_attn_status cache_build(thin_attn_cache_s* cc) {
   off = align256(off + cc->delta_floats * 4);
   cc->c2_off = off;
   off = align256(off + std::max<size_t>(cc->c2_floats, 1) * 4);
+  cc->part_off = off;
+  if (cc->use_split) off = align256(off + (size_t)cc->max_splits * BH * (cf.D + 2) * 4);
   cc->bytes = off;
   cudaError_t e = cudaMalloc(&cc->d_mem, cc->bytes);
   if (e != cudaSuccess) {
@@ -1358,11 +1376,13 @@ thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, cons
   char* base = (char*)c->d_mem;
   // 1. the new key/value row: exact prefix row pos, or row ne + (pos - ne) mod b of the batch region
   const int64_t r = pos < c->ne ? pos : c->ne + (pos - c->ne) % c->bsz;
-  const size_t krow = (size_t)cf.H * cf.E * es, vrow = (size_t)cf.H * cf.D * es;
-  CK(cudaMemcpy2DAsync(base + c->raw.k_off + (size_t)r * krow, (size_t)c->L * krow, k, krow, krow, cf.B,
-                       cudaMemcpyDeviceToDevice, st));
-  CK(cudaMemcpy2DAsync(base + c->raw.v_off + (size_t)r * vrow, (size_t)c->L * vrow, v, vrow, vrow, cf.B,
-                       cudaMemcpyDeviceToDevice, st));
+  if (!c->use_split) {   // (the split-key kernels read the new row from k, v and append it themselves)
+    const size_t krow = (size_t)cf.H * cf.E * es, vrow = (size_t)cf.H * cf.D * es;
+    CK(cudaMemcpy2DAsync(base + c->raw.k_off + (size_t)r * krow, (size_t)c->L * krow, k, krow, krow, cf.B,
+                         cudaMemcpyDeviceToDevice, st));
+    CK(cudaMemcpy2DAsync(base + c->raw.v_off + (size_t)r * vrow, (size_t)c->L * vrow, v, vrow, vrow, cf.B,
+                         cudaMemcpyDeviceToDevice, st));
+  }
   // 2. attention of query pos against the cache as it stands (its own token included)
   AttnArgs aa{};
   aa.q = q;
@@ -1387,7 +1407,16 @@ thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, cons
   aa.scale_log2e = (float)((double)c->scale * 1.4426950408889634);
   bool done = false;
   cudaError_t e = cudaSuccess;
-  if (c->use_tc) e = launch_attention_tc(aa, c->d_status, st, &done);
+  if (c->use_split) {
+    const int n_splits = (c->pos_keys[pos] + decode_chunk_keys() - 1) / decode_chunk_keys();
+    DecodeAppend ap;
+    ap.new_k = k;
+    ap.new_v = v;
+    ap.row = (int)r;
+    e = launch_decode_attention(aa, cf.dtype, n_splits, (float*)(base + c->part_off), ap, st);
+    done = true;
+  }
+  if (e == cudaSuccess && !done && c->use_tc) e = launch_attention_tc(aa, c->d_status, st, &done);
   if (e == cudaSuccess && !done) e = launch_attention_simt(aa, cf.dtype, st);
   if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "cache attention: %s", cudaGetErrorString(e));
   // 3. a completed batch becomes a level-0 node; the 4-ary counter merges equal levels

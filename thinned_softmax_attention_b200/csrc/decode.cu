@@ -1,0 +1,241 @@
+// Attention of one query per (b,h) against its key segments, split over the keys (decode).
+//
+// A decoded position attends to a few thousand keys (exact prefix, snapshot nodes, the batch in
+// progress) with a single query.  Split kernel: CTA (chunk, b*h) takes 128 consecutive keys of the
+// concatenated segments, one warp per 32 keys, one key per lane:
+//   scores   lane i reads its key's row whole (all 16-byte pieces in flight) and forms
+//            z = s q.k log2e + log2 w (w = the segment's weight) against q held in shared memory
+//   softmax  m = the chunk's max z, p = 2^(z - m), l = sum p (CTA-wide through shared memory)
+//   PV       lane-parallel over D: o += p_i v_i, the p_i broadcast from lane i
+// and writes the partial (m, l, o) of its chunk.  Combine kernel: CTA b*h merges the partials
+//   M = max m,  L = sum l 2^(m - M),  out = sum o 2^(m - M) / L,  lse = (M + log2 L) ln 2.
+// Base 2 throughout, fp32 accumulation, one pass over every key and value row.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace thin {
+
+namespace {
+
+constexpr int kDecodeChunk = 128;     // keys per CTA
+constexpr int kDecodeThreads = 128;   // 4 warps x 32 keys
+
+template <typename T, int EPL>
+__device__ __forceinline__ void load_lane(const T* row, int lane, float (&x)[EPL]) {
+  if constexpr (sizeof(T) == 2) {
+    // EPL bf16 = EPL * 2 bytes per lane
+    if constexpr (EPL == 2) {
+      const uint32_t u = *(const uint32_t*)(row + lane * 2);
+      x[0] = __uint_as_float(u << 16);
+      x[1] = __uint_as_float(u & 0xFFFF0000u);
+    } else if constexpr (EPL == 4) {
+      const uint2 u = *(const uint2*)(row + lane * 4);
+      x[0] = __uint_as_float(u.x << 16);
+      x[1] = __uint_as_float(u.x & 0xFFFF0000u);
+      x[2] = __uint_as_float(u.y << 16);
+      x[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    } else {
+      const uint4 u = *(const uint4*)(row + lane * 8);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) x[i] = to_f(row[lane * EPL + i]);
+  }
+}
+
+template <typename T, int EPL, int DPL>
+__global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(AttnArgs a, float* part, int n_splits,
+                                                                       DecodeAppend ap) {
+  const AttnTile tile = a.tiles[a.tile0];
+  const int split = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int E = EPL * 32, D = DPL * 32;
+  constexpr int KV = E * (int)sizeof(T) / 16;     // 16-byte pieces of a key row
+  __shared__ AttnSeg segs[32];
+  __shared__ int seg_start[33];
+  __shared__ float q_s[E];
+  __shared__ float red_m[4], red_l[4];
+  __shared__ float o_s[4][D];
+  const int nseg = min(tile.nseg, 32);
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int s = 0; s < nseg; ++s) {
+      segs[s] = a.segs[tile.seg0 + s];
+      seg_start[s] = acc;
+      acc += segs[s].len;
+    }
+    seg_start[nseg] = acc;
+  }
+  const T* q = (const T*)a.q + ((int64_t)b * a.T * a.H + h) * E;   // the tile's single query row
+  for (int e = threadIdx.x; e < E; e += kDecodeThreads) q_s[e] = to_f(q[e]) * a.scale_log2e;
+  __syncthreads();
+  // this lane's key: j = chunk start + 32 warp + lane -> K and V rows, log2 weight
+  const int j = split * kDecodeChunk + warp * 32 + lane;
+  const bool valid = j < seg_start[nseg];
+  const T *kr = nullptr, *vr = nullptr;
+  float lw2 = 0.f;
+  if (valid) {
+    int s = 0;
+    while (s + 1 < nseg && seg_start[s + 1] <= j) ++s;
+    const AttnSeg sg = segs[s];
+    const int off = j - seg_start[s];
+    if (sg.kind == SEG_TOKENS) {
+      const int64_t row = ((int64_t)b * a.L + sg.first + off) * a.H + h;
+      kr = (const T*)a.k + row * E;
+      vr = (const T*)a.v + row * D;
+    } else {
+      const int64_t row = ((int64_t)bh * a.n_slots + sg.first) * a.slot_rows + off;
+      kr = (const T*)a.ck + row * E;
+      vr = (const T*)a.cv + row * D;
+    }
+    lw2 = sg.logw * 1.4426950408889634f;
+    if (ap.new_k && j == seg_start[nseg] - 1) {
+      // the last key is the token being decoded: read it from the caller's rows (it is appended to
+      // the cache by the combine launch, after every chunk has been read)
+      kr = (const T*)ap.new_k + ((int64_t)b * a.H + h) * E;
+      vr = (const T*)ap.new_v + ((int64_t)b * a.H + h) * D;
+    }
+  }
+  // score of this lane's key: its whole row in flight, q (pre-scaled by s log2 e) broadcast
+  float z_mine = -INFINITY;
+  if (valid) {
+    uint4 kv[KV];
+#pragma unroll
+    for (int c = 0; c < KV; ++c) kv[c] = ((const uint4*)kr)[c];
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < KV; ++c) {
+      const uint32_t w[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
+      if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc = fmaf(q_s[c * 8 + 2 * i], __uint_as_float(w[i] << 16), acc);
+          acc = fmaf(q_s[c * 8 + 2 * i + 1], __uint_as_float(w[i] & 0xFFFF0000u), acc);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc = fmaf(q_s[c * 4 + i], __uint_as_float(w[i]), acc);
+      }
+    }
+    z_mine = acc + lw2;
+  }
+  // chunk max and 2^(z - m)
+  float wm = z_mine;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+  if (lane == 0) red_m[warp] = wm;
+  __syncthreads();
+  const float m = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+  const float p_mine = (z_mine == -INFINITY || m == -INFINITY) ? 0.f : exp2f(z_mine - m);
+  float wl = p_mine;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
+  if (lane == 0) red_l[warp] = wl;
+  // o = sum p_i v_i over the warp's keys, lane-parallel over D, eight value rows in flight
+  float ov[DPL];
+#pragma unroll
+  for (int d = 0; d < DPL; ++d) ov[d] = 0.f;
+  const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));   // the valid keys are the first ones
+#pragma unroll 1
+  for (int i0 = 0; i0 < nvalid; i0 += 8) {
+    float vv[8][DPL], pp[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const T* r = (const T*)__shfl_sync(0xffffffffu, (unsigned long long)vr, (i0 + u) & 31);
+      pp[u] = __shfl_sync(0xffffffffu, p_mine, (i0 + u) & 31);
+      if (i0 + u < nvalid) load_lane<T, DPL>(r, lane, vv[u]);
+      else pp[u] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (i0 + u < nvalid) {
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) ov[d] = fmaf(pp[u], vv[u][d], ov[d]);
+      }
+  }
+#pragma unroll
+  for (int d = 0; d < DPL; ++d) o_s[warp][lane * DPL + d] = ov[d];
+  __syncthreads();
+  float* out = part + ((size_t)bh * n_splits + split) * (D + 2);
+  for (int d = threadIdx.x; d < D; d += kDecodeThreads) out[d] = o_s[0][d] + o_s[1][d] + o_s[2][d] + o_s[3][d];
+  if (threadIdx.x == 0) {
+    out[D] = m;
+    out[D + 1] = red_l[0] + red_l[1] + red_l[2] + red_l[3];
+  }
+}
+
+template <typename T, int E, int D>
+__global__ void __launch_bounds__(128) decode_combine_kernel(AttnArgs a, const float* part, int n_splits,
+                                                             DecodeAppend ap) {
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+  if (ap.new_k) {
+    // append the decoded token's key and value to the cache row of this position
+    const int64_t src = (int64_t)b * a.H + h, dst = ((int64_t)b * a.L + ap.row) * a.H + h;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) ((T*)a.k)[dst * E + e] = ((const T*)ap.new_k)[src * E + e];
+    for (int d = threadIdx.x; d < D; d += blockDim.x) ((T*)a.v)[dst * D + d] = ((const T*)ap.new_v)[src * D + d];
+  }
+  const float* p = part + (size_t)bh * n_splits * (D + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, p[s * (D + 2) + D]);
+  float L = 0.f;
+  for (int s = 0; s < n_splits; ++s) {
+    const float ms = p[s * (D + 2) + D];
+    if (ms != -INFINITY) L += p[s * (D + 2) + D + 1] * exp2f(ms - M);
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  T* out = (T*)a.out + ((int64_t)b * a.T * a.H + h) * D;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float o = 0.f;
+    for (int s = 0; s < n_splits; ++s) {
+      const float ms = p[s * (D + 2) + D];
+      if (ms != -INFINITY) o += p[s * (D + 2) + d] * exp2f(ms - M);
+    }
+    out[d] = from_f<T>(o * inv);
+  }
+  if (threadIdx.x == 0 && a.lse) a.lse[bh] = (M + log2f(L)) * 0.6931471805599453f;
+}
+
+template <typename T, int EPL, int DPL>
+cudaError_t launch_t(const AttnArgs& a, int n_splits, float* part, const DecodeAppend& ap, cudaStream_t st) {
+  decode_split_kernel<T, EPL, DPL><<<dim3(n_splits, a.B * a.H), kDecodeThreads, 0, st>>>(a, part, n_splits, ap);
+  decode_combine_kernel<T, EPL * 32, DPL * 32><<<a.B * a.H, 128, 0, st>>>(a, part, n_splits, ap);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_dt(const AttnArgs& a, int n_splits, float* part, const DecodeAppend& ap, cudaStream_t st) {
+  const int epl = a.E / 32, dpl = a.D / 32;
+#define THIN_DECODE_CASE(X, Y) \
+  if (epl == X && dpl == Y) return launch_t<T, X, Y>(a, n_splits, part, ap, st);
+  THIN_DECODE_CASE(2, 2)
+  THIN_DECODE_CASE(2, 4)
+  THIN_DECODE_CASE(2, 8)
+  THIN_DECODE_CASE(4, 2)
+  THIN_DECODE_CASE(4, 4)
+  THIN_DECODE_CASE(4, 8)
+#undef THIN_DECODE_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool decode_attention_supported(int E, int D, int max_segments) {
+  const bool ok_e = E == 64 || E == 128, ok_d = D == 64 || D == 128 || D == 256;
+  return ok_e && ok_d && max_segments <= 32;
+}
+
+int decode_chunk_keys() { return kDecodeChunk; }
+
+cudaError_t launch_decode_attention(const AttnArgs& a, int dtype, int n_splits, float* part, const DecodeAppend& ap,
+                                    cudaStream_t st) {
+  if (a.B * a.H == 0 || n_splits <= 0) return cudaSuccess;
+  return dtype == 0 ? launch_dt<float>(a, n_splits, part, ap, st) : launch_dt<__nv_bfloat16>(a, n_splits, part, ap, st);
+}
+
+}  // namespace thin

@@ -30,6 +30,21 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int* status_word, cudaStream_
 int attention_tc_tile_rows();
 bool attention_tc_supported(int dtype, int E, int D);
 
+// Split-key attention of one query per (b,h) (decode): n_splits chunks of decode_chunk_keys() keys
+// of the tile a.tile0, partials (m, l, o) in `part` (n_splits x B*H x (D + 2) floats), then a combine
+// launch writing out and lse.
+// With new_k set, the last key of the tile is the token being decoded: it is read from new_k / new_v
+// ((B,1,H,E), (B,1,H,D)) and then written to row `row` of every (b,h) of a.k / a.v.
+struct DecodeAppend {
+  const void* new_k = nullptr;
+  const void* new_v = nullptr;
+  int row = 0;
+};
+bool decode_attention_supported(int E, int D, int max_segments);
+int decode_chunk_keys();
+cudaError_t launch_decode_attention(const AttnArgs& a, int dtype, int n_splits, float* part, const DecodeAppend& ap,
+                                    cudaStream_t st);
+
 // bf16 TMA tensor maps with 128-byte swizzle and (64 elements x box_rows) boxes:
 // 2D over `rows` rows of `width` elements, rows `row_stride` elements apart;
 // 3D over a (B*L, H, width) view of a (B, L, H, width) tensor, one head per box.
