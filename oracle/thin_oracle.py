@@ -275,10 +275,13 @@ def halve_level(Kall, Vall, idx, n_group, scale, seed, bh, round_ids, trace, fol
 
 
 def kh_compress(Kall, Vall, scale, g, seed, bh, round_of_level: Callable[[int], np.ndarray],
-                sub_round: np.ndarray, trace: Trace, follow: Optional[Trace], stats: Stats):
-    """KH-Compress of I independent point sets of S points each -> (I, |C|) indices into the S points."""
+                sub_round: np.ndarray, trace: Trace, follow: Optional[Trace], stats: Stats,
+                sizes: Optional[Tuple[int, int, int]] = None):
+    """KH-Compress of I independent point sets of S points each -> (I, |C|) indices into the S points.
+
+    ``sizes`` = (r, L, S'): the tree to use instead of compress_sizes(S, g)."""
     I, S, _ = Kall.shape
-    r, L, S_sub, _ = compress_sizes(S, g)
+    r, L, S_sub = sizes if sizes is not None else compress_sizes(S, g)[:3]
     if S_sub < S:
         U = philox_word(seed, bh.astype(np.uint64), sub_round.astype(np.uint64), 0) % np.uint64(S_sub)
         idx = subsample_indices(S, S_sub, U)
@@ -470,6 +473,150 @@ def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, head
     coreset = (np.stack([nodes[s] for s in slots], axis=1).reshape(B, H, len(slots), c)
                if slots else np.zeros((B, H, 0, c), dtype=np.int64))
     wts = np.array([weight[s] for s in slots]) if slots else np.zeros(0)
+    return OracleOut(out, lse, coreset, trace, stats, wts)
+
+
+# --------------------------------------------------------------------------
+# Thinformer Express, page-literal cache ("reading A").
+# --------------------------------------------------------------------------
+def express_a_sizes(N: int, n_out: int, g: int) -> Tuple[int, int, int]:
+    """(r, L, S') thinning a batch of N points to n_out: S' = L 4^r = n_out 2^r points (a uniform
+    subsample when S' < N) through r KH-Compress levels over leaves of L = n_out / 2^r points.
+
+    2^r is the largest power of two with 2^r <= N / n_out and 2^r <= n_out / 4^g, i.e. S' never
+    exceeds N nor the COMPRESS2(g) input size n_out^2 / 4^g (the leaves hold at least 4^g points).
+    """
+    r = 0
+    while 2 ** (r + 1) * n_out <= N and 2 ** (r + 1) * 4 ** g <= n_out and n_out % 2 ** (r + 1) == 0:
+        r += 1
+    L = n_out // 2 ** r
+    return r, L, L * 4 ** r
+
+
+def express_a_layout(T: int, n_out: int):
+    """Batches after the exact phase: (level i, s in 1..3, start, length), batch size 4^i n_out.
+
+    Level 0 covers tokens [n_out, 4 n_out) (inflation 1: three batches of n_out tokens), level i
+    the next 3 4^i n_out tokens; the last batch may be partial.
+    """
+    out, start, i = [], n_out, 0
+    while start < T:
+        for s in range(1, 4):
+            if start >= T:
+                break
+            size = 4 ** i * n_out
+            out.append((i, s, start, min(size, T - start)))
+            start += size
+        i += 1
+    return out
+
+
+def express_a(q, k, v, n_out, g, seed, scale=None, follow=None, rows=None, heads=None, _plant=None):
+    """Thinformer Express prefill with the page-literal cache (reading A).
+
+    The cache holds points of one weight m, the inflation factor (m = 1 at the start):
+      * exact phase: tokens [0, n_out) enter the cache with weight 1;
+      * thin phase: the following tokens come in batches of m n_out; a completed batch is thinned to
+        n_out points (express_a_sizes: a systematic uniform subsample to S' points, then r
+        KH-Compress levels) of weight m and appended to the cache;
+      * HALVE phase: when the cache holds 4 n_out points they are halved twice (4 n_out -> 2 n_out ->
+        n_out, in time order) and m <- 4 m.
+    With m = 1 a batch of n_out tokens is kept whole, so tokens [0, 4 n_out) are attended exactly.
+    Query t in a batch of level i >= 1 attends to the cache at the start of its batch (the HALVE
+    output H_i and the thinned batches of level i before its own, all of weight 4^i) and to tokens
+    [batch start, t] of its own batch (weight 1).
+    Philox rounds: batch number kb (0-based, level 0 included) level l -> round_batch(kb, l),
+    subsample -> round_subsample(kb); HALVE H_j step t -> round_merge(j, 0, t).
+    Coreset slots, in order: for i = 1, 2, ...: H_i, then the thinned batches of level i, each
+    present only if a query uses it (directly or through a later HALVE).
+    ``_plant`` (test hook): "weight" gives the thinned points the weight of the previous level.
+    """
+    q, k_, v = _f64(q), _f64(k), _f64(v)
+    B, T, H, E = q.shape
+    D = v.shape[3]
+    scale = 1.0 / math.sqrt(E) if scale is None else scale
+    hs = np.arange(H) if heads is None else np.asarray(heads[1])
+    Htot = H if heads is None else heads[0]
+    n_bh = B * H
+    bh = (np.arange(B)[:, None] * Htot + hs[None, :]).reshape(-1)
+    Kall = k_.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
+    Vall = v.transpose(0, 2, 1, 3).reshape(n_bh, T, D)
+    Qall = q.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
+    layout = express_a_layout(T, n_out)
+    trace: Trace = {}
+    stats = Stats()
+    levels = sorted({b[0] for b in layout})
+    # which nodes are needed: H_i for every level i >= 1 with a batch; thinned batch (i, s) if batch
+    # (i, s+1) exists (its queries see it) or H_{i+1} is needed
+    have = {(b[0], b[1]): b for b in layout}
+    need_h = {i for i in levels if i >= 1}
+    need_b = set()
+    for (i, s), b in have.items():
+        if i >= 1 and ((i, s + 1) in have or (i + 1) in need_h):
+            need_b.add((i, s))
+    nodes: Dict[Tuple[str, int, int], np.ndarray] = {}
+    for kb, (i, s, start, length) in enumerate(layout):
+        if (i, s) not in need_b:
+            continue
+        r, L, S_sub = express_a_sizes(length, n_out, g)
+        Kb = Kall[:, start:start + length]
+        Vb = Vall[:, start:start + length]
+        loc = kh_compress(Kb, Vb, scale, g, seed, bh,
+                          lambda lv: np.full(n_bh, round_batch(kb, lv), dtype=np.int64),
+                          np.full(n_bh, round_subsample(kb), dtype=np.int64), trace, follow, stats,
+                          sizes=(r, L, S_sub))
+        nodes[("b", i, s)] = loc + start
+    for i in sorted(need_h):
+        if i == 1:
+            idx = np.broadcast_to(np.arange(4 * n_out, dtype=np.int64), (n_bh, 4 * n_out)).copy()
+        else:
+            idx = np.concatenate([nodes[("h", i - 1, 0)]] + [nodes[("b", i - 1, s)] for s in (1, 2, 3)], axis=1)
+        for step in range(2):
+            rid = np.full(n_bh, round_merge(i, 0, step), dtype=np.int64)
+            idx = halve_level(Kall, Vall, idx, idx.shape[1], scale, seed, bh, rid, trace, follow, stats)
+        nodes[("h", i, 0)] = idx
+    slots = []
+    for i in sorted(need_h):
+        slots.append(("h", i, 0))
+        slots += [("b", i, s) for s in (1, 2, 3) if ("b", i, s) in nodes]
+    wlev = (lambda i: 4 ** (i - 1)) if _plant == "weight" else (lambda i: 4 ** i)
+    # attention
+    rsel = np.arange(T) if rows is None else np.sort(np.asarray(rows))
+    out = np.zeros((B, len(rsel), H, D))
+    lse = np.zeros((B, H, len(rsel)))
+    bat = np.full(len(rsel), -1)
+    for kb, (i, s, start, length) in enumerate(layout):
+        if i >= 1:
+            bat[(rsel >= start) & (rsel < start + length)] = kb
+    for grp in np.unique(bat):
+        sel = np.nonzero(bat == grp)[0]
+        tq = rsel[sel]
+        for n in range(n_bh):
+            b, h = divmod(n, H)
+            if grp < 0:
+                hi = int(tq.max()) + 1
+                key = np.arange(hi)
+                logw = np.zeros(hi)
+                mask = key[None, :] <= tq[:, None]
+            else:
+                i, s, start, length = layout[grp]
+                parts = [nodes[("h", i, 0)][n]] + [nodes[("b", i, s2)][n] for s2 in range(1, s)]
+                n_fixed = sum(len(p) for p in parts)
+                w_i = wlev(i)
+                h_w = 4 ** i
+                lw = [np.full(n_out, math.log(h_w))] + [np.full(n_out, math.log(w_i)) for _ in range(1, s)]
+                parts.append(np.arange(start, start + length))
+                lw.append(np.zeros(length))
+                key = np.concatenate(parts)
+                logw = np.concatenate(lw)
+                mask = np.ones((len(tq), len(key)), dtype=bool)
+                mask[:, n_fixed:] = np.arange(start, start + length)[None, :] <= tq[:, None]
+            o, l = weighted_attention(Qall[n, tq], Kall[n, key], Vall[n, key], scale, logw, mask)
+            out[b, sel, h] = o
+            lse[b, h, sel] = l
+    coreset = (np.stack([nodes[sl] for sl in slots], axis=1).reshape(B, H, len(slots), n_out)
+               if slots else np.zeros((B, H, 0, n_out), dtype=np.int64))
+    wts = np.array([float(4 ** sl[1]) for sl in slots]) if slots else np.zeros(0)
     return OracleOut(out, lse, coreset, trace, stats, wts)
 
 

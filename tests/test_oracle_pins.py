@@ -16,7 +16,8 @@ import pytest
 import torch
 
 import workloads as W
-from oracle import (compress_sizes, exact_attention, express, express_layout, kappa_att,
+from oracle import (compress_sizes, exact_attention, express, express_a, express_a_layout, express_a_sizes,
+                    express_layout, kappa_att,
                     kernel_halving, philox4x32_10, philox_uniform, round_batch, round_merge,
                     snapshot_nodes, subsample_indices, thinformer, weighted_attention)
 from tests.plain_kh import plain_kernel_halving
@@ -383,3 +384,74 @@ def test_express_merges_only_equal_levels():
         assert covered[0][0] == 0 and covered[-1][1] == kb
         assert all(a[1] == b[0] for a, b in zip(covered, covered[1:]))
         assert all(sum(1 for x in nodes if x[0] == lv) <= 3 for lv, _ in nodes)
+
+
+# ---------------------------------------------------------------- Express, page-literal cache (reading A)
+def test_express_a_sizes():
+    """Thinning N = m n_out tokens to n_out: S' = L 4^r = n_out 2^r, capped by N and by the COMPRESS2(g)
+    input size n_out^2 / 4^g (leaves of at least 4^g points)."""
+    assert express_a_sizes(128, 128, 2) == (0, 128, 128)       # inflation 1: kept whole
+    assert express_a_sizes(512, 128, 2) == (2, 32, 512)        # 512 -> 256 -> 128, no subsample
+    assert express_a_sizes(2048, 128, 2) == (3, 16, 1024)      # subsample to 1024 = 128^2 / 16
+    assert express_a_sizes(8192, 128, 2) == (3, 16, 1024)
+    for n_out in (16, 64, 128, 512):
+        for g in (0, 1, 2):
+            for i in range(5):
+                N = 4 ** i * n_out
+                r, L, S = express_a_sizes(N, n_out, g)
+                assert S == L * 4 ** r == n_out * 2 ** r and S <= N and L * 2 ** r == n_out
+                assert S <= max(n_out, n_out * n_out // 4 ** g)
+
+
+def test_express_a_layout():
+    L = express_a_layout(32768, 128)
+    assert [b[3] for b in L] == [128] * 3 + [512] * 3 + [2048] * 3 + [8192] * 3
+    assert all(b[2] == 128 + sum(x[3] for x in L[:j]) for j, b in enumerate(L))
+    Lp = express_a_layout(5000, 128)    # last batch partial
+    assert Lp[-1][2] + Lp[-1][3] == 5000 and Lp[-1][3] < 4 ** Lp[-1][0] * 128
+
+
+def _small_express_a(T=16 * 64 + 100, zero_q=False, plant=None):
+    w = W.WORKLOADS["express32k"].with_(E=16, D=16)
+    q, k, v = W.make_qkv(w, T=T, heads=[0, 1])
+    if zero_q:
+        q = torch.zeros_like(q)
+    return (q, k, v), express_a(q, k, v, 16, 1, 5, heads=(w.H, [0, 1]), _plant=plant)
+
+
+def test_express_a_is_exact_until_the_first_halve():
+    """With inflation 1 a batch of n_out tokens is kept whole: tokens [0, 4 n_out) are attended exactly."""
+    (q, k, v), o = _small_express_a()
+    ex, _ = exact_attention(q, k, v, causal=True)
+    np.testing.assert_allclose(o.out[:, :64], ex[:, :64], rtol=1e-11, atol=1e-13)
+    assert np.abs(o.out[:, 64:] - ex[:, 64:]).max() > 1e-6
+
+
+def test_express_a_mass_is_token_count():
+    """q = 0: lse_t = ln(total weight seen by t) = ln(t+1): the HALVE outputs and the thinned batches
+    of level i weigh 4^i each, the raw tokens of the batch in progress 1."""
+    (q, k, v), o = _small_express_a(zero_q=True)
+    np.testing.assert_allclose(o.lse[0, 0], np.log(np.arange(q.shape[1]) + 1.0), rtol=1e-12)
+    np.testing.assert_allclose(o.lse[0, 1], np.log(np.arange(q.shape[1]) + 1.0), rtol=1e-12)
+
+
+def test_express_a_mass_pin_catches_a_wrong_weight():
+    (q, k, v), o = _small_express_a(zero_q=True, plant="weight")
+    assert np.abs(o.lse[0, 0] - np.log(np.arange(q.shape[1]) + 1.0)).max() > 0.1
+
+
+def test_express_a_node_structure():
+    """T = 1124, n_out = 16: levels 1 and 2 complete, level 3 a partial batch -> slots H_1, B(1,1..3),
+    H_2, B(2,1..3), H_3; every node n_out distinct tokens in time order, inside its batch (thinned
+    batches) or inside the tokens its HALVE consumed (H_i: tokens [0, 4^i n_out))."""
+    T = 16 * 64 + 100
+    (q, k, v), o = _small_express_a(T=T)
+    L = express_a_layout(T, 16)
+    assert o.coreset.shape == (1, 2, 9, 16)
+    np.testing.assert_array_equal(o.weights, [4, 4, 4, 4, 16, 16, 16, 16, 64])
+    ranges = ([(0, 64)] + [(b[2], b[2] + b[3]) for b in L if b[0] == 1] + [(0, 256)] +
+              [(b[2], b[2] + b[3]) for b in L if b[0] == 2] + [(0, 1024)])
+    for sl, (lo, hi) in enumerate(ranges):
+        for h in range(2):
+            node = o.coreset[0, h, sl]
+            assert len(node) == 16 and np.all(np.diff(node) > 0) and node[0] >= lo and node[-1] < hi
