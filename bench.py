@@ -82,6 +82,23 @@ def attention_work(w, plan):
         keys = plan["coreset_rows"] if plan["levels"] > 0 else w.S
         pairs = w.T * keys
         kv_rows = keys
+    elif w.cache == "A":
+        # tokens [0, 4 n_out) exactly; batch (i, s): H_i and s - 1 thinned batches (n_out points each)
+        # and its own tokens causally
+        n_out = min(w.n_exact, w.T)
+        ex = min(4 * n_out, w.T)
+        vis = [np.arange(1, ex + 1, dtype=np.int64)]
+        start, i = n_out * 4, 1
+        while start < w.T:
+            for s_ in range(1, 4):
+                if start >= w.T:
+                    break
+                size = min(4 ** i * n_out, w.T - start)
+                vis.append(s_ * n_out + np.arange(1, size + 1, dtype=np.int64))
+                start += size
+            i += 1
+        pairs = int(np.concatenate(vis).sum())
+        kv_rows = w.T + plan["n_nodes"] * plan["coreset_rows"]
     else:
         t = np.arange(w.T, dtype=np.int64)
         ne, b, c = min(w.n_exact, w.T), w.batch, plan["coreset_rows"]
@@ -149,7 +166,7 @@ class Clocks:
 
 def cpu_baseline(w, seed_heads, budget_s=12.0, max_heads=8):
     """The fp64 oracle, as it stands, on a bounded sample: whole heads of the workload."""
-    from oracle import express, thinformer
+    from oracle import express, express_a, thinformer
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -160,7 +177,10 @@ def cpu_baseline(w, seed_heads, budget_s=12.0, max_heads=8):
         q, k, v = W.make_qkv(w.with_(B=1), heads=[h])
         t0 = time.perf_counter()
         if w.causal:
-            express(q, k, v, w.n_exact, w.batch, w.g, w.seed, heads=(w.H, [h]))
+            if w.cache == "A":
+                express_a(q, k, v, w.n_exact, w.g, w.seed, heads=(w.H, [h]))
+            else:
+                express(q, k, v, w.n_exact, w.batch, w.g, w.seed, heads=(w.H, [h]))
         else:
             thinformer(q, k, v, w.g, w.seed, heads=(w.H, [h]))
         t_total += time.perf_counter() - t0
@@ -191,7 +211,7 @@ def run_reference(a):
     if rank != 0:
         return
     w = W.WORKLOADS[a.workload]
-    from oracle import express, thinformer
+    from oracle import express, express_a, thinformer
     heads = list(range(w.H)) * (1 + (a.steps + a.warmup) // max(1, w.H))
     times = []
     for i in range(a.warmup + a.steps):
@@ -199,7 +219,10 @@ def run_reference(a):
         q, k, v = W.make_qkv(w.with_(B=1), heads=[h])
         t0 = time.perf_counter()
         if w.causal:
-            express(q, k, v, w.n_exact, w.batch, w.g, w.seed, heads=(w.H, [h]))
+            if w.cache == "A":
+                express_a(q, k, v, w.n_exact, w.g, w.seed, heads=(w.H, [h]))
+            else:
+                express(q, k, v, w.n_exact, w.batch, w.g, w.seed, heads=(w.H, [h]))
         else:
             thinformer(q, k, v, w.g, w.seed, heads=(w.H, [h]))
         if i >= a.warmup:
@@ -242,7 +265,8 @@ def job_value(world, tokens_per_rank, ms):
 
 def config_of(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "S": w.T if w.causal else w.S, "E": w.E, "D": w.D,
-            "causal": w.causal, "g": w.g, "n_exact": w.n_exact, "batch": w.batch, "seed": w.seed,
+            "causal": w.causal, "cache": w.cache if w.causal else None, "g": w.g, "n_exact": w.n_exact,
+            "batch": w.batch, "seed": w.seed,
             "l2": "inputs larger than L2 (no flush)" if 3 * w.B * w.H * w.T * w.E * 2 > 126e6 else
             "inputs smaller than L2"}
 
@@ -256,8 +280,8 @@ def run_decode(a):
     are included in the time but not in these bytes."""
     import thinned_softmax_attention_b200 as TA
     w = W.WORKLOADS[a.workload]
-    if not w.causal:
-        raise SystemExit("--decode needs a causal (Express) workload")
+    if not w.causal or w.cache != "B":
+        raise SystemExit("--decode needs an Express workload with the 4-ary node cache")
     dev = torch.device("cuda", 0)
     q, k, v = (x.to(dev) for x in W.make_qkv(w))
     h = TA.ThinAttention(w.B, w.T, w.T, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
@@ -325,12 +349,12 @@ def main():
     S = w.T if w.causal else w.S
     h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch,
                          device=local)
-    plan = h.plan(w.causal, w.g)
-    h.reserve(w.causal, w.g)
+    plan = h.plan(w.mode, w.g)
+    h.reserve(w.mode, w.g)
     out = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype, device=dev)
 
     def step():
-        h.forward(q, k, v, causal=w.causal, g=w.g, seed=w.seed, out=out)
+        h.forward(q, k, v, causal=w.mode, g=w.g, seed=w.seed, out=out)
 
     for _ in range(max(3, a.warmup)):
         step()
@@ -410,14 +434,14 @@ def main():
         qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
         oh = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype).pin_memory()
         for _ in range(2):
-            h.forward_host(qh, kh, vh, oh, causal=w.causal, g=w.g, seed=w.seed)
+            h.forward_host(qh, kh, vh, oh, causal=w.mode, g=w.g, seed=w.seed)
         n_e2e = max(2, min(a.steps, 5))
         if dist:
             dist.barrier()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
         for _ in range(n_e2e):
-            h.forward_host(qh, kh, vh, oh, causal=w.causal, g=w.g, seed=w.seed)
+            h.forward_host(qh, kh, vh, oh, causal=w.mode, g=w.g, seed=w.seed)
         f1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(f0.elapsed_time(f1) / n_e2e, dist, dev)

@@ -121,7 +121,11 @@ THIN_ATTN_API thin_attn_status thin_attn_trace_layout(thin_attn_t h, int causal,
 /*
  * Forward pass on device memory.
  *   q, k, v, out      device pointers in the layouts above
- *   causal            0: Thinformer; 1: Thinformer Express prefill
+ *   causal            0: Thinformer; 1: Thinformer Express prefill (exact prefix of n_exact tokens,
+ *                     batches of `batch` tokens, 4-ary counter of HALVE merges); 2: Thinformer
+ *                     Express with the cache of "The EXPRESS Meta-Procedure" read literally: an exact
+ *                     phase of n_out = n_exact tokens, batches of m n_out tokens thinned to n_out points
+ *                     of weight m, the whole cache halved twice at 4 n_out with m <- 4m (`batch` unused)
  *   g                 oversampling parameter of KH-Compress, 0..6 (coreset ~ 2^g sqrt(S))
  *   seed              Philox key of the thinning decisions
  *   lse_opt           device (B,H,T) fp32 log-sum-exp ln sum_j w_j e^{s q.k_j}, or NULL

@@ -15,7 +15,7 @@ import torch
 
 import thinned_softmax_attention_b200 as TA
 import workloads as W
-from oracle import express, thinformer
+from oracle import express, express_a, thinformer
 
 pytestmark = pytest.mark.gpu
 
@@ -39,15 +39,17 @@ def run_case(w, T=None, S=None, heads=None, rows=None, g=None, seed=None, check_
     q, k, v = W.make_qkv(w, T=T, S=S)
     dev = torch.device("cuda", 0)
     h = TA.ThinAttention(w.B, T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
-    r = h.forward(q.to(dev), k.to(dev), v.to(dev), causal=w.causal, g=g, seed=seed, return_lse=True,
+    r = h.forward(q.to(dev), k.to(dev), v.to(dev), causal=w.mode, g=g, seed=seed, return_lse=True,
                   return_coreset=True, return_trace=True)
     torch.cuda.synchronize()
     h.check()
-    follow = TA.decode_trace(r["trace"], h.trace_layout(w.causal, g))
+    follow = TA.decode_trace(r["trace"], h.trace_layout(w.mode, g))
     hs = list(range(w.H)) if check_heads is None else list(check_heads)
     rsel = np.arange(T) if rows is None else np.sort(np.asarray(rows))
     qh, kh, vh = q[:, :, hs], k[:, :, hs], v[:, :, hs]
-    if w.causal:
+    if w.causal and w.cache == "A":
+        ref = express_a(qh, kh, vh, w.n_exact, g, seed, follow=follow, rows=rsel, heads=(w.H, hs))
+    elif w.causal:
         ref = express(qh, kh, vh, w.n_exact, w.batch, g, seed, follow=follow, rows=rsel, heads=(w.H, hs))
     else:
         ref = thinformer(qh, kh, vh, g, seed, follow=follow, rows=rsel, heads=(w.H, hs))
@@ -251,3 +253,25 @@ def test_profile_steps_cover_the_halving_phases():
     assert abs(total - (ph["thin_ms"] + ph["merge_ms"])) <= 0.05 * total + 1e-3
     again = h.profile_steps()
     assert again["calls"] == 0 and all(s["ms"] == 0 for s in again["steps"])
+
+
+
+# ---------------------------------------------------------------- Express with the page-literal cache
+@pytest.mark.parametrize("T,n_out,g,dtype", [
+    (2048, 32, 1, "bf16"),     # levels 0..2 (batches of 32, 128, 512 -> subsampled to 256), H_1, H_2
+    (1500, 64, 2, "bf16"),     # level 2 a partial batch: H_2 over the three thinned level-1 batches
+    (700, 16, 0, "fp32"),      # fp32 path, g = 0 (leaves of one point)
+    (200, 64, 2, "bf16"),      # shorter than 4 n_out: exact attention throughout
+])
+def test_express_a_reduced(T, n_out, g, dtype):
+    w = W.WORKLOADS["express32k_a"].with_(T=T, H=2, n_exact=n_out, g=g, dtype=dtype,
+                                          E=128 if dtype == "bf16" else 64, D=128 if dtype == "bf16" else 64)
+    res = run_case(w)
+    assert_parity(res, dtype)
+
+
+def test_express_a_32k_sampled_rows():
+    w = W.WORKLOADS["express32k_a"]
+    rows = np.sort(np.random.default_rng(3).choice(w.T, 128, replace=False))
+    res = run_case(w, rows=rows, check_heads=[0, 17])
+    assert_parity(res, "bf16")

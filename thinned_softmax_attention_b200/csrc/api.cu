@@ -10,6 +10,10 @@
 //   points (weight b/c); a 4-ary counter merges four level-l nodes by two
 //   halvings (4c -> 2c -> c, weight x4); a query of batch k attends to the exact
 //   prefix, the nodes present after k completed batches, and its batch causally.
+// Plan of the causal path with the page-literal cache (causal = 2, "The EXPRESS Meta-Procedure"
+// read literally): exact phase [0, n_out); batches of m n_out tokens thinned to n_out points of
+// weight m; the whole cache halved twice when it holds 4 n_out points, m <- 4m.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -62,6 +66,35 @@ Sizes compress_sizes(int64_t S, int g) {
   return {r, (int)L, (int)(L * p4(r)), (int)(L << r)};
 }
 
+// Reading A of Express: thinning a batch of N points to n_out: S' = L 4^r = n_out 2^r (a systematic
+// uniform subsample when S' < N) through r KH-Compress levels over leaves of L = n_out / 2^r; 2^r is
+// the largest power of two with 2^r <= N / n_out and 2^r <= n_out / 4^g (S' <= n_out^2 / 4^g).
+Sizes express_a_sizes(int64_t N, int n_out, int g) {
+  int r = 0;
+  while (((int64_t)n_out << (r + 1)) <= N && ((int64_t)1 << (r + 1 + 2 * g)) <= n_out && n_out % (1 << (r + 1)) == 0)
+    ++r;
+  const int L = n_out >> r;
+  return {r, L, L << (2 * r), n_out};
+}
+
+// Batches of reading A after the exact phase [0, n_out): level i holds three batches of 4^i n_out
+// tokens (the last batch may be partial).
+struct ABatch {
+  int level, s;
+  int64_t start, len;
+};
+std::vector<ABatch> express_a_layout(int64_t T, int n_out) {
+  std::vector<ABatch> out;
+  int64_t start = n_out;
+  for (int i = 0; start < T; ++i)
+    for (int s = 1; s <= 3 && start < T; ++s) {
+      const int64_t size = ((int64_t)n_out) << (2 * i);
+      out.push_back({i, s, start, std::min(size, T - start)});
+      start += size;
+    }
+  return out;
+}
+
 uint32_t round_noncausal(int level) { return (uint32_t)level; }
 uint32_t round_batch(int k, int level) { return 0x40000000u | ((uint32_t)k << 4) | (uint32_t)level; }
 uint32_t round_merge(int level, int node, int step) {
@@ -107,6 +140,10 @@ struct Plan {
   Sizes sz{};
   int n_b = 0, n_slots = 0, c = 0;
   std::vector<int> level_base;   // causal: first slot of each node level
+  // causal == 2 (Express, page-literal cache): batches, slot of H_i, slot of thinned batch (i, s)
+  std::vector<ABatch> a_batches;
+  std::map<int, int> a_slot_h;
+  std::map<std::pair<int, int>, int> a_slot_b;
   std::vector<StepPlan> steps;
   std::vector<BufSpec> levels;   // intermediate halving outputs
   BufSpec nodes, mtemp;
@@ -195,7 +232,9 @@ void build_waves(const thin_attn_config& cf, const Plan& p, AttnTables& t) {
   const int ne = std::min(cf.n_exact, cf.T);
   for (int i = 0; i < (int)t.tiles.size(); ++i) {
     int after = n_steps - 1;
-    if (p.causal) {
+    if (p.causal == 2) {
+      if (t.tiles[i].q0 < 4 * p.c) after = -1;   // the exact tiles need no halving step
+    } else if (p.causal) {
       const int q0 = t.tiles[i].q0;
       const int64_t k = q0 < ne ? -1 : (q0 - ne) / cf.batch;
       if (k <= 0) after = -1;
@@ -229,6 +268,30 @@ void build_attn_tables(const thin_attn_config& cf, const Plan& p, int QT, AttnTa
     }
     t.segs.push_back(s);
     for (int q0 = 0; q0 < cf.T; q0 += QT) t.tiles.push_back({q0, std::min(QT, cf.T - q0), 0, 1});
+    return;
+  }
+  if (p.causal == 2) {
+    // tokens [0, 4 n_out) exactly; a query of batch (i, s), i >= 1: H_i and the thinned batches
+    // (i, 1..s-1), all of weight 4^i, and its batch causally
+    const int T = cf.T, n_out = p.c;
+    const int ex = (int)std::min<int64_t>((int64_t)4 * n_out, T);
+    for (int q0 = 0; q0 < ex; q0 += QT) {
+      const int ql = std::min(QT, ex - q0);
+      t.tiles.push_back({q0, ql, (int)t.segs.size(), 1});
+      t.segs.push_back({SEG_TOKENS, 0, q0 + ql, 1, 0.f, 0});
+    }
+    for (const ABatch& b : p.a_batches) {
+      if (b.level < 1) continue;
+      const float lw = (float)std::log(std::ldexp(1.0, 2 * b.level));
+      for (int64_t q0 = b.start; q0 < b.start + b.len; q0 += QT) {
+        const int ql = (int)std::min<int64_t>(QT, b.start + b.len - q0);
+        const int seg0 = (int)t.segs.size();
+        t.segs.push_back({SEG_COMPACT, p.a_slot_h.at(b.level), n_out, 0, lw, 0});
+        for (int s2 = 1; s2 < b.s; ++s2) t.segs.push_back({SEG_COMPACT, p.a_slot_b.at({b.level, s2}), n_out, 0, lw, 0});
+        t.segs.push_back({SEG_TOKENS, (int)b.start, (int)(q0 + ql - b.start), 1, 0.f, 0});
+        t.tiles.push_back({(int)q0, ql, seg0, (int)t.segs.size() - seg0});
+      }
+    }
     return;
   }
   const int T = cf.T, ne = std::min(cf.n_exact, T), bsz = cf.batch;
@@ -274,8 +337,8 @@ struct RunDesc {
 };
 
 void add_compress_steps(Plan& p, const std::vector<RunDesc>& runs, int S_run, int final_buf,
-                        std::vector<int64_t>& level_rows_per_run) {
-  const Sizes sz = compress_sizes(S_run, p.g);
+                        std::vector<int64_t>& level_rows_per_run, const Sizes* sizes = nullptr) {
+  const Sizes sz = sizes ? *sizes : compress_sizes(S_run, p.g);
   level_rows_per_run.clear();
   const int nr = (int)runs.size();
   for (int lv = 1; lv <= sz.r; ++lv) {
@@ -343,6 +406,85 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
       p->att_slot_rows = p->sz.C;
     }
     p->coreset_idx_elems = (uint64_t)BH * (p->sz.r > 0 ? p->sz.C : cf.S);
+  } else if (causal == 2) {
+    // Express with the page-literal cache: thinned batches (independent of the cache), then the
+    // HALVEs H_1, H_2, ... in order (H_i consumes H_{i-1} and the three thinned batches of level
+    // i-1, or the raw tokens [0, 4 n_out) for H_1)
+    const int T = cf.T, n_out = std::min(cf.n_exact, T);
+    p->c = n_out;
+    p->a_batches = express_a_layout(T, n_out);
+    const auto& L = p->a_batches;
+    std::map<std::pair<int, int>, size_t> have;
+    for (size_t j = 0; j < L.size(); ++j) have[{L[j].level, L[j].s}] = j;
+    std::vector<int> need_h;
+    for (const auto& b : L)
+      if (b.level >= 1 && (need_h.empty() || need_h.back() != b.level)) need_h.push_back(b.level);
+    auto needs_h = [&](int i) { return std::find(need_h.begin(), need_h.end(), i) != need_h.end(); };
+    std::vector<std::pair<int, int>> need_b;
+    for (const auto& b : L)
+      if (b.level >= 1 && (have.count({b.level, b.s + 1}) || needs_h(b.level + 1))) need_b.push_back({b.level, b.s});
+    for (int i : need_h) {
+      p->a_slot_h[i] = p->n_slots++;
+      for (int s2 = 1; s2 <= 3; ++s2)
+        if (std::find(need_b.begin(), need_b.end(), std::make_pair(i, s2)) != need_b.end()) p->a_slot_b[{i, s2}] = p->n_slots++;
+    }
+    p->n_b = (int)need_b.size();
+    p->nodes.rows = (int64_t)BH * p->n_slots * n_out;
+    p->final_buf = BUF_NODES;
+    p->att_slots = std::max(1, p->n_slots);
+    p->att_slot_rows = n_out;
+    // thinned batches, level by level (one set of steps per batch size)
+    for (int i : need_h) {
+      std::vector<RunDesc> runs;
+      int64_t len = 0;
+      for (int bh = 0; bh < BH; ++bh)
+        for (int s2 = 1; s2 <= 3; ++s2) {
+          auto it = p->a_slot_b.find({i, s2});
+          if (it == p->a_slot_b.end()) continue;
+          const ABatch& b = L[have[{i, s2}]];
+          len = b.len;
+          const int kb = (int)have[{i, s2}];
+          runs.push_back({(uint32_t)bh, (int64_t)(bh / cf.H) * T + b.start, (uint32_t)b.start, kb,
+                          ((int64_t)bh * p->n_slots + it->second) * n_out});
+        }
+      if (runs.empty()) continue;
+      const Sizes sz = express_a_sizes(len, n_out, g);
+      std::vector<int64_t> lr;
+      if (sz.r > 0) add_compress_steps(*p, runs, (int)len, BUF_NODES, lr, &sz);
+    }
+    // HALVEs: 4 n_out points -> 2 n_out (MTEMP) -> n_out (slot H_i)
+    p->mtemp.rows = (int64_t)BH * 2 * n_out;
+    for (int i : need_h) {
+      for (int step = 0; step < 2; ++step) {
+        StepPlan st;
+        st.phase = 1;
+        st.merge_level = i;
+        st.n = (step == 0 ? 4 : 2) * n_out;
+        st.m = st.n / 2;
+        st.m_pad = (st.m + 31) / 32 * 32;
+        st.src_buf = step == 0 ? (i == 1 ? BUF_TOKENS : BUF_NODES) : BUF_MTEMP;
+        st.dst_buf = step == 0 ? BUF_MTEMP : BUF_NODES;
+        st.S_full = st.S_sub = st.n;
+        for (int bh = 0; bh < BH; ++bh) {
+          HalveInst in{};
+          const int64_t mt = (int64_t)bh * 2 * n_out;
+          if (step == 0) {
+            in.src_row = i == 1 ? (int64_t)(bh / cf.H) * T : ((int64_t)bh * p->n_slots + p->a_slot_h[i - 1]) * n_out;
+            in.dst_row = mt;
+          } else {
+            in.src_row = mt;
+            in.dst_row = ((int64_t)bh * p->n_slots + p->a_slot_h[i]) * n_out;
+          }
+          in.bh = (uint32_t)bh;
+          in.round_id = round_merge(i, 0, step);
+          in.pair0 = 0;
+          in.tok0 = 0;
+          st.inst.push_back(in);
+        }
+        p->steps.push_back(std::move(st));
+      }
+    }
+    p->coreset_idx_elems = (uint64_t)p->nodes.rows;
   } else {
     const int T = cf.T, ne = std::min(cf.n_exact, T), bsz = cf.batch;
     p->n_b = T > ne ? (T - ne) / bsz : 0;
@@ -526,12 +668,14 @@ thin_attn_status check_cfg(const thin_attn_config* c) {
 }
 
 thin_attn_status get_plan(thin_attn_s* h, int causal, int g, Plan** out) {
-  if (causal != 0 && causal != 1) return fail(THIN_ATTN_EINVAL, "causal must be 0 or 1");
+  if (causal < 0 || causal > 2) return fail(THIN_ATTN_EINVAL, "causal must be 0, 1 or 2");
   if (g < 0 || g > 6) return fail(THIN_ATTN_EINVAL, "g=%d outside 0..6", g);
   const thin_attn_config& c = h->cfg;
   if (!causal && (c.S < 1)) return fail(THIN_ATTN_EINVAL, "non-causal attention needs S >= 1");
-  if (causal && (c.batch < 1 || c.n_exact < 0))
+  if (causal == 1 && (c.batch < 1 || c.n_exact < 0))
     return fail(THIN_ATTN_EINVAL, "causal attention needs batch >= 1 and n_exact >= 0");
+  if (causal == 2 && c.n_exact < 2)
+    return fail(THIN_ATTN_EINVAL, "Express with the page-literal cache needs n_exact (the cache size n_out) >= 2");
   auto key = std::make_pair(causal, g);
   auto it = h->plans.find(key);
   if (it != h->plans.end()) {

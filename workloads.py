@@ -22,6 +22,7 @@ Started": query (B,T,H,E), key (B,S,H,E), value (B,S,H,D)):
   express32k   B=1 H=32 T=32768  E=D=128 bf16 causal; q,k = E^-1/4 N(0,1) then
                RoPE (base 10000, pairs (2i,2i+1), angle t*10000^(-2i/E)); v ~ N(0,1)
   express128k  B=1 H=32 T=131072 E=D=128 bf16 causal; same generator, seed 3
+  express32k_a the express32k tensors through the page-literal cache (n_out = 128)
 """
 from __future__ import annotations
 
@@ -47,8 +48,14 @@ class Workload:
     seed: int             # Philox seed of the thinning decisions
     data_seed: int        # seed of the synthetic tensors
     kind: str             # "iid" | "rank8" | "rope"
-    n_exact: int = 0      # Express exact phase (causal only)
-    batch: int = 0        # Express thin batch (causal only)
+    n_exact: int = 0      # Express exact phase (causal only); the cache size n_out for cache "A"
+    batch: int = 0        # Express thin batch (causal only, cache "B")
+    cache: str = "B"      # causal only: "B" nodes of a 4-ary counter, "A" the page-literal cache
+
+    @property
+    def mode(self) -> int:
+        """The library's `causal` argument: 0 Thinformer, 1 Express, 2 Express with the page-literal cache."""
+        return 0 if not self.causal else (2 if self.cache == "A" else 1)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -70,6 +77,8 @@ WORKLOADS = {
                            "rope", n_exact=1024, batch=1024),
     "express128k": Workload("express128k", 1, 32, 131072, 131072, 128, 128, "bf16", True, 2, 4, 3,
                             "rope", n_exact=2048, batch=2048),
+    "express32k_a": Workload("express32k_a", 1, 32, 32768, 32768, 128, 128, "bf16", True, 2, 1, 0,
+                             "rope", n_exact=128, cache="A"),
 }
 
 
