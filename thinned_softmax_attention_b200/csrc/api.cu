@@ -116,10 +116,20 @@ struct StepPlan {
   int src_buf = BUF_TOKENS, dst_buf = 0;
   int n = 0, m = 0, m_pad = 0;
   int S_full = 0, S_sub = 0;
+  int sub_stride = 0;    // see StepArgs::sub_stride
   std::vector<HalveInst> inst;
   size_t inst_off = 0;
   uint64_t trace_base = 0;
 };
+
+// Subsample stride of a token-source step (StepArgs::sub_stride).
+int sub_stride_of(const StepPlan& sp) {
+  if (sp.src_buf != BUF_TOKENS || sp.S_sub <= 0 || sp.S_sub >= sp.S_full || sp.S_full % sp.S_sub) return 0;
+  const int k = sp.S_full / sp.S_sub;
+  for (const HalveInst& in : sp.inst)
+    if (in.src_row % k) return 0;
+  return k;
+}
 
 // A wave: consecutive attention tiles that can run as soon as halving step `after` (and all
 // earlier steps) has run; after = -1: as soon as the forward starts.
@@ -566,6 +576,7 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
   }
   // trace layout and scratch sizes
   for (auto& st : p->steps) {
+    st.sub_stride = sub_stride_of(st);
     if (st.copy_only) continue;
     st.trace_base = p->trace_words;
     const int nw = st.m_pad / 32;
@@ -726,6 +737,7 @@ int step_launches(const thin_attn_config& cf, const Plan* p, const StepPlan& sp)
   a.src_rows = src_rows_of(cf, p, sp);
   a.S_full = sp.S_full;
   a.S_sub = sp.S_sub;
+  a.sub_stride = sp.sub_stride;
   a.n = sp.n;
   a.E = cf.E;
   a.D = cf.D;
@@ -858,6 +870,7 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     a.H = cf.H;
     a.S_full = sp.S_full;
     a.S_sub = sp.S_sub;
+    a.sub_stride = sp.sub_stride;
     a.dstK = (void*)dk;
     a.dstV = (void*)dv;
     a.dstIdx = didx;
@@ -1215,6 +1228,7 @@ struct thin_attn_cache_s {
 namespace {
 
 void cache_add_step(thin_attn_cache_s* cc, CacheStep& st) {
+  st.sp.sub_stride = sub_stride_of(st.sp);
   cc->delta_floats = std::max(cc->delta_floats, st.sp.inst.size() * (size_t)st.sp.m_pad * st.sp.m_pad);
   cc->c2_floats = std::max(cc->c2_floats, st.sp.inst.size());
 }
@@ -1434,6 +1448,7 @@ thin_attn_status cache_run_step(thin_attn_cache_s* cc, CacheStep& st, cudaStream
   a.src_rows = rows;
   a.S_full = st.sp.S_full;
   a.S_sub = st.sp.S_sub;
+  a.sub_stride = st.sp.sub_stride;
   a.dstK = (void*)dk;
   a.dstV = (void*)dv;
   a.dstIdx = didx;

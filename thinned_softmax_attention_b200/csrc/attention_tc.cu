@@ -765,6 +765,19 @@ bool make_map_3d(CUtensorMap* m, const void* base, int64_t BL, int H, int width,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// (B*L/k, k, H, width) view of a (B, L, H, width) bf16 tensor, boxes of (64, 1 head, 1, box_rows):
+// a box starting at (x, h, 0, R) holds rows R k, (R+1) k, ... -- every k-th row.
+bool make_map_4d_strided(CUtensorMap* m, const void* base, int64_t BL, int H, int width, int k, int box_rows) {
+  if (k < 1 || BL / k < 1) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)k, (cuuint64_t)(BL / k)};
+  cuuint64_t strides[3] = {(cuuint64_t)width * 2, (cuuint64_t)width * H * 2, (cuuint64_t)width * H * k * 2};
+  cuuint32_t box[4] = {64, 1, 1, (cuuint32_t)box_rows};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, (void*)base, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tensor_maps_available() { return encode_fn() != nullptr; }
 
 bool attention_tc_supported(int dtype, int E, int D) {

@@ -83,6 +83,9 @@ struct StepArgs {
   int H;                   // heads (SRC_TOKENS row addressing)
   int64_t src_rows;        // rows of the source: B*L (SRC_TOKENS) or compact rows; 0 = unknown
   int S_full, S_sub;       // SRC_TOKENS subsample: token = floor((p*S_full + U)/S_sub)
+  int sub_stride;          // k = S_full / S_sub when that is an integer and every run starts on a multiple
+                           // of k: the subsample is then tokens 0, k, 2k, ... (U < S_sub drops out), a
+                           // strided box for TMA; 0 otherwise
   // destination
   void* dstK;
   void* dstV;

@@ -64,10 +64,12 @@ template <typename Bit>
 __device__ __forceinline__ void gather_from_stage(const StepArgs& a, int64_t dst_row, int64_t src_row, uint32_t tok_base,
                                                   const uint8_t* st, int row0, int i0, int i1, Bit bit, int lane,
                                                   int EC, int NC) {
+  // token index of point p of the instance: tok_base + p k (k = subsample stride, 1 without subsample)
   const bool tokens = a.src_kind == SRC_TOKENS;
+  const uint32_t k = a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u;
   for (int i = i0 + lane; i < i1; i += 32) {
     const int p = 2 * i + (bit(i) ? 0 : 1);
-    a.dstIdx[dst_row + i] = tokens ? (int32_t)(tok_base + (uint32_t)p) : a.srcIdx[src_row + p];
+    a.dstIdx[dst_row + i] = tokens ? (int32_t)(tok_base + (uint32_t)p * k) : a.srcIdx[src_row + p];
   }
   const int units = NC * 8, kw = a.E / 8, vw = a.D / 8;
   uint4* dK = (uint4*)a.dstK;
@@ -160,7 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
       int row = 0, h = 0;
       if (lane < ni) {
         const HalveInst in = a.inst[i0 + lane];
-        row = (int)(in.src_row + (tokens ? 2 * (int64_t)in.pair0 : 0));
+        // token runs: first row of the instance, in units of the subsample stride k for strided runs
+        row = (int)(tokens ? (a.sub_stride > 1 ? in.src_row / a.sub_stride : in.src_row) + 2 * (int64_t)in.pair0
+                           : in.src_row);
         h = (int)(in.bh % (uint32_t)a.H);
       }
       if (!warp_wait(empty + s, ((k / nst) & 1) ^ 1, abort)) break;
@@ -172,8 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
           const bool isk = c < EC;
           const CUtensorMap* m = isk ? &maps.k : &maps.v;
           const int x = (isk ? c : c - EC) * 64;
-          if (tokens) tma_load_3d(st + c * kChunk, m, full + s, x, h, row);
-          else tma_load_2d(st + c * kChunk, m, full + s, x, row);
+          if (!tokens) tma_load_2d(st + c * kChunk, m, full + s, x, row);
+          else if (a.sub_stride > 1) tma_load_4d(st + c * kChunk, m, full + s, x, h, 0, row);
+          else tma_load_3d(st + c * kChunk, m, full + s, x, h, row);
         }
       }
       issued = k + 1;
@@ -327,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
           const uint32_t kbg = __shfl_sync(0xffffffffu, kb, src);
           const int64_t dst_row = __shfl_sync(0xffffffffu, in.dst_row, src);
           const int64_t src_row = __shfl_sync(0xffffffffu, in.src_row, src);
-          const uint32_t tok_base = __shfl_sync(0xffffffffu, in.tok0 + 2u * in.pair0, src);
+          const uint32_t tok_base = __shfl_sync(0xffffffffu, in.tok0 + 2u * in.pair0 * (a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u), src);
           if (gi < a.n_inst) {
             if (a.trace && lane == 0) a.trace[a.trace_base + (size_t)gi * nb] = kbg;
             gather_from_stage(a, dst_row, src_row, tok_base, st, (wi * (32 / SEG) + g) * NP, 0, m,
@@ -387,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
         if (live) {
           if (a.trace && wi == 0 && lane < nb) a.trace[a.trace_base + (size_t)inst * nb + lane] = lane ? kb1 : kb0;
           auto bit = [kb0, kb1](int i) { return (((i < 32 ? kb0 : kb1) >> (i & 31)) & 1u) != 0; };
-          const uint32_t tok_base = in.tok0 + 2u * in.pair0;
+          const uint32_t tok_base = in.tok0 + 2u * in.pair0 * (a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u);
           gather_from_stage(a, in.dst_row, in.src_row, tok_base, st, 0, wi ? half : 0, wi ? m : half, bit, lane, EC, NC);
         }
       }
@@ -411,7 +416,10 @@ template <int NP>
 cudaError_t launch_np(const StepArgs& a, cudaStream_t st) {
   FusedMaps maps;
   bool ok;
-  if (a.src_kind == SRC_TOKENS) {
+  if (a.src_kind == SRC_TOKENS && a.sub_stride > 1) {
+    ok = make_map_4d_strided(&maps.k, a.srcK, a.src_rows, a.H, a.E, a.sub_stride, NP) &&
+         make_map_4d_strided(&maps.v, a.srcV, a.src_rows, a.H, a.D, a.sub_stride, NP);
+  } else if (a.src_kind == SRC_TOKENS) {
     ok = make_map_3d(&maps.k, a.srcK, a.src_rows, a.H, a.E, NP) && make_map_3d(&maps.v, a.srcV, a.src_rows, a.H, a.D, NP);
   } else {
     ok = make_map_2d(&maps.k, a.srcK, a.src_rows, a.E, a.E, NP) && make_map_2d(&maps.v, a.srcV, a.src_rows, a.D, a.D, NP);
@@ -442,7 +450,8 @@ bool halving_fused_supported(const StepArgs& a) {
   if (std::getenv("THIN_ATTN_UNFUSED_HALVING") != nullptr) return false;
   if (a.E % 64 || a.D % 64 || (a.E + a.D) / 64 > kMaxChunks || a.n < 2 || a.n > 128 || a.n % 2) return false;
   if (a.src_rows <= 0 || !tensor_maps_available()) return false;
-  if (a.src_kind == SRC_TOKENS && a.S_sub < a.S_full) return false;   // subsampled rows do not form boxes
+  // subsampled rows form boxes only as a strided view (integer ratio, runs on multiples of it)
+  if (a.src_kind == SRC_TOKENS && a.S_sub < a.S_full && a.sub_stride < 2) return false;
   return true;
 }
 

@@ -51,5 +51,8 @@ cudaError_t launch_decode_attention(const AttnArgs& a, int dtype, int n_splits, 
 bool tensor_maps_available();
 bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows, int width, int64_t row_stride, int box_rows);
 bool make_map_3d(CUtensorMap* m, const void* base, int64_t BL, int H, int width, int box_rows);
+// 4D view over every k-th row (a systematic subsample with integer ratio k): box (64, 1, 1, box_rows)
+// at (x, h, 0, R) holds rows R k, (R+1) k, ...
+bool make_map_4d_strided(CUtensorMap* m, const void* base, int64_t BL, int H, int width, int k, int box_rows);
 
 }  // namespace thin

@@ -81,7 +81,8 @@ __global__ void __launch_bounds__(128) pairgram_tc_kernel(const __grid_constant_
     const bool tokens = a.src_kind == SRC_TOKENS;
     const int h = (int)(in.bh % (uint32_t)a.H);
     // first source row of the instance: a token run starts 2*pair0 points into its (b,h) run
-    const int64_t base_row = in.src_row + (tokens ? 2 * (int64_t)in.pair0 : 0);
+    const int64_t base_row = tokens ? (a.sub_stride > 1 ? in.src_row / a.sub_stride : in.src_row) + 2 * (int64_t)in.pair0
+                                    : in.src_row;
     const int row_r = (int)(base_row + (int64_t)tj * P), row_c = (int)(base_row + (int64_t)ti * P);
     auto load = [&](int c) {
       const int st = c & 1;
@@ -90,7 +91,10 @@ __global__ void __launch_bounds__(128) pairgram_tc_kernel(const __grid_constant_
       const bool isk = c < EC;
       const CUtensorMap* m = isk ? &maps.k : &maps.v;
       const int x = (isk ? c : c - EC) * 64;
-      if (tokens) {
+      if (tokens && a.sub_stride > 1) {
+        tma_load_4d(dst, m, full + st, x, h, 0, row_r);
+        if (!diag) tma_load_4d(dst + Lay::CHUNK, m, full + st, x, h, 0, row_c);
+      } else if (tokens) {
         tma_load_3d(dst, m, full + st, x, h, row_r);
         if (!diag) tma_load_3d(dst + Lay::CHUNK, m, full + st, x, h, row_c);
       } else {
@@ -191,7 +195,10 @@ template <int P>
 cudaError_t launch_p(const StepArgs& a, int* status, cudaStream_t st) {
   GramMaps maps;
   bool ok;
-  if (a.src_kind == SRC_TOKENS) {
+  if (a.src_kind == SRC_TOKENS && a.sub_stride > 1) {
+    ok = make_map_4d_strided(&maps.k, a.srcK, a.src_rows, a.H, a.E, a.sub_stride, P) &&
+         make_map_4d_strided(&maps.v, a.srcV, a.src_rows, a.H, a.D, a.sub_stride, P);
+  } else if (a.src_kind == SRC_TOKENS) {
     ok = make_map_3d(&maps.k, a.srcK, a.src_rows, a.H, a.E, P) && make_map_3d(&maps.v, a.srcV, a.src_rows, a.H, a.D, P);
   } else {
     ok = make_map_2d(&maps.k, a.srcK, a.src_rows, a.E, a.E, P) && make_map_2d(&maps.v, a.srcV, a.src_rows, a.D, a.D, P);
@@ -210,7 +217,8 @@ cudaError_t launch_p(const StepArgs& a, int* status, cudaStream_t st) {
 cudaError_t launch_pairgram_tc(const StepArgs& a, cudaStream_t st, bool* done) {
   *done = false;
   if (a.E % 64 || a.D % 64 || a.src_rows <= 0 || !tensor_maps_available()) return cudaSuccess;
-  if (a.src_kind == SRC_TOKENS && a.S_sub < a.S_full) return cudaSuccess;   // subsampled rows: not a box
+  // subsampled rows are a box only as a strided view (integer ratio, runs on multiples of it)
+  if (a.src_kind == SRC_TOKENS && a.S_sub < a.S_full && a.sub_stride < 2) return cudaSuccess;
   cudaError_t e;
   if (a.n <= 32) e = launch_p<32>(a, a.status, st);
   else if (a.n <= 64) e = launch_p<64>(a, a.status, st);
