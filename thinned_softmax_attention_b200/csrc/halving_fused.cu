@@ -63,7 +63,7 @@ struct FusedShape {
 template <typename Bit>
 __device__ __forceinline__ void gather_from_stage(const StepArgs& a, int64_t dst_row, int64_t src_row, uint32_t tok_base,
                                                   const uint8_t* st, int row0, int i0, int i1, Bit bit, int lane,
-                                                  int EC, int NC) {
+                                                  int EC, int NC, uint32_t chunk_bytes = kChunk) {
   // token index of point p of the instance: tok_base + p k (k = subsample stride, 1 without subsample)
   const bool tokens = a.src_kind == SRC_TOKENS;
   const uint32_t k = a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u;
@@ -78,7 +78,7 @@ __device__ __forceinline__ void gather_from_stage(const StepArgs& a, int64_t dst
     const int c = w >> 3, x = w & 7;
     uint4* dst = c < EC ? dK + dst_row * kw + c * 8 + x : dV + dst_row * vw + (c - EC) * 8 + x;
     const int stride = c < EC ? kw : vw;
-    const uint8_t* src = st + c * kChunk;
+    const uint8_t* src = st + c * chunk_bytes;
     for (int i = i0; i < i1; i += 8) {
       uint4 buf[8];
 #pragma unroll
@@ -444,11 +444,316 @@ cudaError_t launch_np(const StepArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------------------------------
+// Instances of 129..256 points: one CTA per instance (its 256 rows, 32 KB per feature chunk, and the
+// 128 x 128 pair differences take the shared memory of an SM).  Warps: 0 TMA, 1 MMA (TMEM owner),
+// 2-5 epilogue (warp w reads TMEM lanes 32 (w % 4)..), 6 sigma's recursion, 7 the walk; all eight
+// gather.  The Gram takes two rounds through the 512 TMEM columns: rows 0..127 against all 256 rows
+// (kk in columns 0..255, vv in 256..511), then rows 128..255 against themselves (columns 0..127 and
+// 256..383), so Delta rows 0..63 are written while the second round runs.  Every barrier is used
+// once (phase 0) and every wait is bounded.
+__global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant__ FusedMaps maps, const StepArgs a) {
+  constexpr int LD = 129;                       // Delta row stride (floats)
+  constexpr uint32_t CB = 2 * kChunk;           // one feature chunk: 256 rows x 64 bf16
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int EC = a.E / 64, NC = (a.E + a.D) / 64;
+  float* D = (float*)(smem + NC * CB);          // [128][LD]
+  __shared__ __align__(8) uint64_t bars[16];
+  uint64_t* full = bars;          // rows landed
+  uint64_t* tfull0 = bars + 1;    // round 1 accumulators ready
+  uint64_t* tempty0 = bars + 2;   // round 1 accumulators read (128)
+  uint64_t* tfull1 = bars + 3;    // round 2 accumulators ready
+  uint64_t* cmax = bars + 4;      // c exchanged among the epilogue threads (128)
+  uint64_t* dhalf = bars + 5;     // Delta rows 0..63 written (128)
+  uint64_t* dfull = bars + 6;     // Delta rows 64..127 written (128)
+  uint64_t* bitsf = bars + 7;     // decisions published (32)
+  uint64_t* mdone = bars + 8;     // every MMA complete
+  uint64_t* thf = bars + 9;       // [4] thresholds of pair block b published (32)
+  __shared__ float red[4];
+  __shared__ float thr_s[128];
+  __shared__ uint32_t bits_s[4];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int inst = blockIdx.x;
+  const int m = a.m, n = a.n;
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    mbar_init(full, 1);
+    mbar_init(tfull0, 1);
+    mbar_init(tempty0, 128);
+    mbar_init(tfull1, 1);
+    mbar_init(cmax, 128);
+    mbar_init(dhalf, 128);
+    mbar_init(dfull, 128);
+    mbar_init(bitsf, 32);
+    mbar_init(mdone, 1);
+    for (int b = 0; b < 4; ++b) mbar_init(thf + b, 32);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_s, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort = &abort_s;
+  const HalveInst in = a.inst[inst];
+  const bool tokens = a.src_kind == SRC_TOKENS;
+  const int ks = a.sub_stride > 1 ? a.sub_stride : 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int row = (int)(tokens ? in.src_row / ks + 2 * (int64_t)in.pair0 : in.src_row);
+      const int h = (int)(in.bh % (uint32_t)a.H);
+      mbar_expect_tx(full, (uint32_t)NC * CB);
+      for (int c = 0; c < NC; ++c) {
+        const bool isk = c < EC;
+        const CUtensorMap* mp = isk ? &maps.k : &maps.v;
+        const int x = (isk ? c : c - EC) * 64;
+        for (int blk = 0; blk < 2; ++blk) {
+          uint8_t* dst = smem + c * CB + blk * kChunk;
+          if (!tokens) tma_load_2d(dst, mp, full, x, row + 128 * blk);
+          else if (ks > 1) tma_load_4d(dst, mp, full, x, h, 0, row + 128 * blk);
+          else tma_load_3d(dst, mp, full, x, h, row + 128 * blk);
+        }
+      }
+      const long long t0 = clock64();
+      while (!mbar_try_wait(full, 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t base = smem_u32(smem);
+      bool ok = mbar_wait(full, 0, abort);
+      if (ok) {
+        tc_fence_after();
+        constexpr uint32_t I256 = idesc_bf16(128, 256, false), I128 = idesc_bf16(128, 128, false);
+        for (int c = 0; c < NC; ++c) {
+          const uint32_t ra = base + c * CB;
+          const uint32_t dc = tmem + (c < EC ? 0u : 256u);
+          const bool first = c == 0 || c == EC;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(dc, sw128_desc(ra + kk * 32, 16, 1024), sw128_desc(ra + kk * 32, 16, 1024), I256,
+                      (!first || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(tfull0);
+        ok = mbar_wait(tempty0, 0, abort);
+        if (ok) {
+          tc_fence_after();
+          for (int c = 0; c < NC; ++c) {
+            const uint32_t rb = base + c * CB + kChunk;
+            const uint32_t dc = tmem + (c < EC ? 0u : 256u);
+            const bool first = c == 0 || c == EC;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(dc, sw128_desc(rb + kk * 32, 16, 1024), sw128_desc(rb + kk * 32, 16, 1024), I128,
+                        (!first || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(tfull1);
+        }
+      }
+      umma_commit(mdone);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(mdone, 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else if (warp >= 2 && warp < 6) {
+    // ------------------------------------------------------------------ epilogue
+    const int q4 = warp & 3;                    // TMEM lane quarter of this warp
+    const int r = q4 * 32 + lane;               // row r of round 1 (row 128 + r of round 2)
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    bool ok = warp_wait(full, 0, abort);
+    float c2 = 0.f;
+    if (ok) {
+      float mx = 0.f;
+#pragma unroll
+      for (int blk = 0; blk < 2; ++blk) {
+        const int R = r + 128 * blk;
+        if (R < n) {
+          const uint8_t* rowp = smem + blk * kChunk + r * 128;
+          for (int c = EC; c < NC; ++c) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint4 w = *(const uint4*)(rowp + c * CB + ((q ^ (r & 7)) << 4));
+              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                mx = fmax3(mx, fabsf(__uint_as_float(ws[e] << 16)), fabsf(__uint_as_float(ws[e] & 0xFFFF0000u)));
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) red[q4] = mx;
+      mbar_arrive(cmax);
+      ok = warp_wait(cmax, 0, abort);
+      const float cm = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+      c2 = cm * cm;
+    }
+    // round 1: pair rows 0..63 against pair columns 0..127
+    if (ok) ok = warp_wait(tfull0, 0, abort);
+    if (ok) {
+      tc_fence_after();
+      const int pj = r >> 1;
+      const bool writer = (r & 1) == 0;
+#pragma unroll 1
+      for (int cc = 0; cc < 8; ++cc) {
+        float kk[32], vv[32];
+        tmem_ld32(tmem + lane_base + cc * 32, kk);
+        tmem_ld32(tmem + lane_base + 256 + cc * 32, vv);
+        tmem_ld_wait();
+        float dd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float k0 = exp2f(kk[2 * i] * a.scale_log2e) * (vv[2 * i] + c2);
+          const float k1 = exp2f(kk[2 * i + 1] * a.scale_log2e) * (vv[2 * i + 1] + c2);
+          dd[i] = k0 - k1;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dd[i] -= __shfl_xor_sync(0xffffffffu, dd[i], 1);
+        if (writer) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int pi = cc * 16 + i;
+            D[pj * LD + pi] = (pj < m && pi < m) ? dd[i] : 0.f;
+          }
+        }
+      }
+      tc_fence_before();
+    }
+    mbar_arrive(tempty0);
+    mbar_arrive(dhalf);
+    // round 2: pair rows 64..127 against pair columns 64..127
+    if (ok) ok = warp_wait(tfull1, 0, abort);
+    if (ok) {
+      tc_fence_after();
+      const int pj = 64 + (r >> 1);
+      const bool writer = (r & 1) == 0;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float kk[32], vv[32];
+        tmem_ld32(tmem + lane_base + cc * 32, kk);
+        tmem_ld32(tmem + lane_base + 256 + cc * 32, vv);
+        tmem_ld_wait();
+        float dd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float k0 = exp2f(kk[2 * i] * a.scale_log2e) * (vv[2 * i] + c2);
+          const float k1 = exp2f(kk[2 * i + 1] * a.scale_log2e) * (vv[2 * i + 1] + c2);
+          dd[i] = k0 - k1;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dd[i] -= __shfl_xor_sync(0xffffffffu, dd[i], 1);
+        if (writer) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int pi = 64 + cc * 16 + i;
+            D[pj * LD + pi] = (pj < m && pi < m) ? dd[i] : 0.f;
+          }
+        }
+      }
+      tc_fence_before();
+    }
+    mbar_arrive(dfull);
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ sigma's recursion
+    const float C = a.C, rC = 1.f / C;
+    float sigma = 0.f;
+#pragma unroll 1
+    for (int blk = 0; blk < 4; ++blk) {
+      if (!warp_wait(blk < 2 ? dhalf : dfull, 0, abort)) break;
+      const int p = 32 * blk + lane;
+      const float wl = p < m ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)p) : 0.f;
+      thr_s[p] = thresholds32(sigma, D[p * LD + p], wl, C, rC, lane);
+      __syncwarp();
+      mbar_arrive(thf + blk);
+    }
+  } else {
+    // ------------------------------------------------------------------ the walk (warp 7)
+    float my[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t kb[4] = {0u, 0u, 0u, 0u};
+    bool ok = true;
+#pragma unroll 1
+    for (int blk = 0; blk < 4 && ok; ++blk) {
+      ok = warp_wait(thf + blk, 0, abort);
+      if (!ok) break;
+      const int base = 32 * blk;
+      float cur = blk == 0 ? my[0] : blk == 1 ? my[1] : blk == 2 ? my[2] : my[3];
+      const uint32_t bb = walk_block32_th(cur, thr_s[base + lane], m - base, lane,
+                                          [&](int q) { return D[(base + q) * LD + base + lane]; });
+      kb[blk] = bb;
+      // this block's contribution to the alpha of every later pair, in pair order
+#pragma unroll 1
+      for (int b2 = blk + 1; b2 < 4; ++b2) {
+        float acc = b2 == 1 ? my[1] : b2 == 2 ? my[2] : my[3];
+#pragma unroll 8
+        for (int q = 0; q < 32; ++q) acc = fmaf(((bb >> q) & 1u) ? 1.f : -1.f, D[(base + q) * LD + 32 * b2 + lane], acc);
+        if (b2 == 1) my[1] = acc;
+        else if (b2 == 2) my[2] = acc;
+        else my[3] = acc;
+      }
+    }
+    if (lane == 0)
+      for (int b = 0; b < 4; ++b) bits_s[b] = kb[b];
+    __syncwarp();
+    mbar_arrive(bitsf);
+  }
+  // ------------------------------------------------------------------ gather (all warps)
+  __syncwarp();
+  if (warp_wait(bitsf, 0, abort)) {
+    const uint32_t b0 = bits_s[0], b1 = bits_s[1], b2 = bits_s[2], b3 = bits_s[3];
+    auto bit = [b0, b1, b2, b3](int i) {
+      const uint32_t w = i < 64 ? (i < 32 ? b0 : b1) : (i < 96 ? b2 : b3);
+      return ((w >> (i & 31)) & 1u) != 0;
+    };
+    const int per = (m + 7) / 8;
+    const uint32_t tok_base = in.tok0 + 2u * in.pair0 * (uint32_t)ks;
+    gather_from_stage(a, in.dst_row, in.src_row, tok_base, smem, 0, min(m, warp * per), min(m, (warp + 1) * per),
+                      bit, lane, EC, NC, CB);
+    if (a.trace && warp == 0 && lane < 4) {
+      const int nb = a.m_pad >> 5;
+      if (lane < nb) a.trace[a.trace_base + (size_t)inst * nb + lane] = lane == 0 ? b0 : lane == 1 ? b1 : lane == 2 ? b2 : b3;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_s && threadIdx.x == 0 && a.status) {
+    if (atomicCAS(a.status, 0, 5) == 0) a.status[1] = inst;
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_256(const StepArgs& a, cudaStream_t st) {
+  FusedMaps maps;
+  bool ok;
+  if (a.src_kind == SRC_TOKENS && a.sub_stride > 1) {
+    ok = make_map_4d_strided(&maps.k, a.srcK, a.src_rows, a.H, a.E, a.sub_stride, 128) &&
+         make_map_4d_strided(&maps.v, a.srcV, a.src_rows, a.H, a.D, a.sub_stride, 128);
+  } else if (a.src_kind == SRC_TOKENS) {
+    ok = make_map_3d(&maps.k, a.srcK, a.src_rows, a.H, a.E, 128) && make_map_3d(&maps.v, a.srcV, a.src_rows, a.H, a.D, 128);
+  } else {
+    ok = make_map_2d(&maps.k, a.srcK, a.src_rows, a.E, a.E, 128) && make_map_2d(&maps.v, a.srcV, a.src_rows, a.D, a.D, 128);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  const int NC = (a.E + a.D) / 64;
+  const size_t sm = 1024 + (size_t)NC * 2 * kChunk + (size_t)128 * 129 * 4;
+  cudaError_t e = cudaFuncSetAttribute(halve256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  halve256_kernel<<<a.n_inst, 256, sm, st>>>(maps, a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool halving_fused_supported(const StepArgs& a) {
   if (std::getenv("THIN_ATTN_UNFUSED_HALVING") != nullptr) return false;
-  if (a.E % 64 || a.D % 64 || (a.E + a.D) / 64 > kMaxChunks || a.n < 2 || a.n > 128 || a.n % 2) return false;
+  if (a.E % 64 || a.D % 64 || (a.E + a.D) / 64 > kMaxChunks || a.n < 2 || a.n > 256 || a.n % 2) return false;
   if (a.src_rows <= 0 || !tensor_maps_available()) return false;
   // subsampled rows form boxes only as a strided view (integer ratio, runs on multiples of it)
   if (a.src_kind == SRC_TOKENS && a.S_sub < a.S_full && a.sub_stride < 2) return false;
@@ -459,7 +764,8 @@ cudaError_t launch_halving_fused(const StepArgs& a, cudaStream_t st) {
   if (a.n_inst == 0) return cudaSuccess;
   if (a.n <= 32) return launch_np<32>(a, st);
   if (a.n <= 64) return launch_np<64>(a, st);
-  return launch_np<128>(a, st);
+  if (a.n <= 128) return launch_np<128>(a, st);
+  return launch_256(a, st);
 }
 
 }  // namespace thin
