@@ -6,9 +6,12 @@
 One step = one thin_attn_forward of the whole path (batch thinning, HALVE
 merges, attention) over the workload (default: express32k, B=1 H=32 T=32768
 E=D=128 bf16, exact phase 1024, thin batch 1024, g=2) with q, k, v resident in
-HBM.  Prints one JSON line on rank 0.  Multi-GPU (torchrun): every rank runs
-its own independent problem of the same size (weak scaling, no collective on
-the data path); step time is the max over ranks of CUDA-event time.
+HBM.  Prints one JSON line on rank 0.  Multi-GPU (torchrun): the ranks hold
+parts of one problem whose (b,h) slices are independent -- `--shard batch`
+(default, weak scaling): rank r holds batch rows [rB, (r+1)B) of a problem with
+N*B rows; `--shard heads` (strong scaling): rank r holds H/N heads of the
+workload.  No collective on the data path; the random decisions are keyed on the
+whole problem's (b,h); step time is the max over ranks of CUDA-event time.
 
 --impl reference times the fp64 CPU oracle on the host cores (rank 0 only),
 each step one head of the workload.
@@ -44,6 +47,8 @@ def args_():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="thin", choices=["thin", "reference"])
     p.add_argument("--workload", default="express32k", choices=sorted(W.WORKLOADS))
+    p.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                   help="N>1: batch rows of one larger problem per rank (weak) or the heads of one problem (strong)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-sdpa", action="store_true")
@@ -244,9 +249,39 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
-def rank_workload(w, rank):
-    """Weak scaling: rank r runs its own independent problem of the same size (data seed + 1000 r)."""
-    return w.with_(data_seed=w.data_seed + 1000 * rank) if rank else w
+class Shard:
+    """This rank's part of the whole problem.
+
+    ``batch`` (weak scaling): the whole problem has world * B batch rows and rank r holds rows
+    [r B, (r+1) B) -- per-rank work fixed as the job grows.  ``heads`` (strong scaling): the whole
+    problem is the workload itself and rank r holds heads [r H/N, (r+1) H/N).  Either way the
+    handle's Philox counters are keyed on the whole problem's (b,h), so every rank computes exactly
+    what a single run of the whole problem computes for its rows; no data crosses between ranks."""
+
+    def __init__(self, w, world, rank, mode="batch"):
+        if mode not in ("batch", "heads"):
+            raise ValueError(mode)
+        if mode == "heads" and w.H % world:
+            raise ValueError(f"--shard heads needs H={w.H} divisible by the {world} ranks")
+        self.mode, self.world, self.rank = mode, world, rank
+        hl = w.H // world if mode == "heads" else w.H
+        self.b0 = rank * w.B if mode == "batch" else 0
+        self.h0 = rank * hl if mode == "heads" else 0
+        self.local = w.with_(H=hl)                      # the shape this rank's handle holds
+        self.heads = list(range(self.h0, self.h0 + hl))
+        self.H_total = w.H
+        self.global_batch = world * w.B if mode == "batch" else w.B
+        self.whole_tokens = self.global_batch * w.H * w.T
+        self.scaling = "weak" if mode == "batch" else "strong"
+        self.parallelism = f"{'dp' if mode == 'batch' else 'hp'}{world}"
+
+    @property
+    def abi(self):
+        """(b0, h0, H_total) of the handle's config."""
+        return (self.b0, self.h0, self.H_total)
+
+    def inputs(self, w):
+        return W.make_qkv(w, heads=self.heads, b0=self.b0)
 
 
 def max_over_ranks(x, dist, device):
@@ -256,11 +291,6 @@ def max_over_ranks(x, dist, device):
     t = torch.tensor([float(x)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
-
-
-def job_value(world, tokens_per_rank, ms):
-    """Whole-job throughput: the tokens every rank processed over the slowest rank's step time."""
-    return world * tokens_per_rank / (ms * 1e-3)
 
 
 def config_of(w):
@@ -342,13 +372,12 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    w = W.WORKLOADS[a.workload]
-    # each rank an independent problem of the same size (weak scaling)
-    wr = rank_workload(w, rank)
-    q, k, v = (x.to(dev) for x in W.make_qkv(wr))
+    shard = Shard(W.WORKLOADS[a.workload], world, rank, a.shard)
+    w = shard.local
+    q, k, v = (x.to(dev) for x in shard.inputs(w))
     S = w.T if w.causal else w.S
     h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch,
-                         device=local)
+                         device=local, shard=shard.abi)
     plan = h.plan(w.mode, w.g)
     h.reserve(w.mode, w.g)
     out = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype, device=dev)
@@ -380,7 +409,7 @@ def main():
     ph = h.profile_read()
     ms = max_over_ranks(e0.elapsed_time(e1) / a.steps, dist, dev)
     tokens = w.B * w.H * w.T
-    value = job_value(world, tokens, ms)
+    value = shard.whole_tokens / (ms * 1e-3)
 
     # dominant kernel roofline: attention.  Bound by arithmetic intensity against the measured ridge
     # (sustained bf16 FLOP/s over HBM bytes/s): tensor cores above it, HBM below it.
@@ -446,7 +475,7 @@ def main():
         torch.cuda.synchronize()
         ems = max_over_ranks(f0.elapsed_time(f1) / n_e2e, dist, dev)
         es = 4 if w.dtype == "fp32" else 2
-        e2e = {"value": job_value(world, tokens, ems), "unit": UNIT,
+        e2e = {"value": shard.whole_tokens / (ems * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * es,
                "d2h_bytes_per_step": out.numel() * es, "ms_per_step": round(ems, 3)}
 
@@ -477,8 +506,10 @@ def main():
     if rank != 0:
         return
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
-            "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
+            "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": shard.scaling,
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {**config_of(W.WORKLOADS[a.workload]), "global_batch": shard.global_batch,
+                       "parallelism": shard.parallelism, "heads_per_gpu": w.H},
             "ms_per_layer": ms, "phases_ms": phases, "roofline": roof, "halving_roofline": halving_roof,
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": plan["kernel_launches"] * a.steps, "clocks": clk, "exact_sdpa_ms": sdpa,

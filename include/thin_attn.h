@@ -68,6 +68,14 @@ typedef struct {
   int n_exact;     /* Express exact phase length (causal only) */
   int batch;       /* Express thin batch length (causal only; > 0) */
   int device;      /* CUDA device ordinal the handle's memory lives on */
+  /* Shard of a larger problem (batch- or head-parallel runs, one handle per GPU).  The Philox
+   * counter of (b,h) is keyed on the whole problem's (b0 + b) * H_total + h0 + h, so the decisions,
+   * coresets and outputs of a shard equal those of the whole problem's run for its (b,h).  Zero
+   * gives the unsharded problem.  EINVAL when b0 < 0, h0 < 0, h0 + H > H_total or
+   * (b0 + B) * H_total >= 2^32. */
+  int b0;          /* whole-problem index of this handle's batch row 0 */
+  int h0;          /* whole-problem index of this handle's head 0 */
+  int H_total;     /* heads of the whole problem; <= 0 selects H */
 } thin_attn_config;
 
 /* Sizes of one (causal, g) plan. */

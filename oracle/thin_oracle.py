@@ -314,13 +314,14 @@ class OracleOut:
     weights: Optional[np.ndarray] = None   # causal: (n_nodes,) node weights
 
 
-def thinformer(q, k, v, g, seed, scale=None, follow=None, rows=None, heads=None):
+def thinformer(q, k, v, g, seed, scale=None, follow=None, rows=None, heads=None, b0=0):
     """Non-causal Thinformer: per (b,h), KH-Compress the S keys/values to a coreset C,
     then weighted attention of every query against C with weight S/|C| per point.
 
     q (B,T,H,E), k (B,S,H,E), v (B,S,H,D) (torch or numpy; read as fp64).
     ``rows``: optional query rows to evaluate (all by default). ``heads``: global
-    head ids of the H axis when the tensors hold a subset (bh = b*H_total + h).
+    head ids of the H axis when the tensors hold a subset, ``b0``: the whole problem's
+    index of batch row 0 (Philox (b,h) word = (b0 + b)*H_total + h).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, T, H, E = q.shape
@@ -328,7 +329,7 @@ def thinformer(q, k, v, g, seed, scale=None, follow=None, rows=None, heads=None)
     scale = 1.0 / math.sqrt(E) if scale is None else scale
     hs = np.arange(H) if heads is None else np.asarray(heads[1])
     Htot = H if heads is None else heads[0]
-    bh = (np.arange(B)[:, None] * Htot + hs[None, :]).reshape(-1)
+    bh = ((b0 + np.arange(B))[:, None] * Htot + hs[None, :]).reshape(-1)
     Kall = k.transpose(0, 2, 1, 3).reshape(B * H, S, E)
     Vall = v.transpose(0, 2, 1, 3).reshape(B * H, S, -1)
     trace: Trace = {}
@@ -381,7 +382,7 @@ def snapshot_nodes(k: int):
     return nodes
 
 
-def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, heads=None):
+def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, heads=None, b0=0):
     """Thinformer Express prefill (causal).
 
     * tokens [0, n_e): kept exactly (weight 1) -- exact phase;
@@ -401,7 +402,7 @@ def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, head
     hs = np.arange(H) if heads is None else np.asarray(heads[1])
     Htot = H if heads is None else heads[0]
     n_bh = B * H
-    bh = (np.arange(B)[:, None] * Htot + hs[None, :]).reshape(-1)
+    bh = ((b0 + np.arange(B))[:, None] * Htot + hs[None, :]).reshape(-1)
     Kall = k_.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
     Vall = v.transpose(0, 2, 1, 3).reshape(n_bh, T, D)
     Qall = q.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
@@ -511,7 +512,7 @@ def express_a_layout(T: int, n_out: int):
     return out
 
 
-def express_a(q, k, v, n_out, g, seed, scale=None, follow=None, rows=None, heads=None, _plant=None):
+def express_a(q, k, v, n_out, g, seed, scale=None, follow=None, rows=None, heads=None, b0=0, _plant=None):
     """Thinformer Express prefill with the page-literal cache (reading A).
 
     The cache holds points of one weight m, the inflation factor (m = 1 at the start):
@@ -538,7 +539,7 @@ def express_a(q, k, v, n_out, g, seed, scale=None, follow=None, rows=None, heads
     hs = np.arange(H) if heads is None else np.asarray(heads[1])
     Htot = H if heads is None else heads[0]
     n_bh = B * H
-    bh = (np.arange(B)[:, None] * Htot + hs[None, :]).reshape(-1)
+    bh = ((b0 + np.arange(B))[:, None] * Htot + hs[None, :]).reshape(-1)
     Kall = k_.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
     Vall = v.transpose(0, 2, 1, 3).reshape(n_bh, T, D)
     Qall = q.transpose(0, 2, 1, 3).reshape(n_bh, T, E)

@@ -108,6 +108,17 @@ def test_bad_arguments_are_rejected_on_the_host():
     assert T.lib().thin_attn_destroy(None) == 0
 
 
+def test_shard_offsets_are_checked_on_the_host():
+    w = W.WORKLOADS["express32k"]
+    mk = lambda shard: T.ThinAttention(1, 4096, 4096, 4, w.E, w.D, w.torch_dtype, n_exact=1024, batch=1024,
+                                       shard=shard)
+    for bad in [(0, 2, 4), (-1, 0, 0), (0, -1, 8), (0, 0, 2), (1 << 30, 0, 8)]:
+        with pytest.raises(T.ThinAttnError, match="EINVAL"):
+            mk(bad)
+    h = mk((3, 4, 8))                    # batch row 3, heads 4..7 of an 8-head problem
+    assert h.trace_layout(True, 2) == mk((0, 0, 0)).trace_layout(True, 2)   # same instances, local (b,h)
+
+
 def test_decode_trace_bit_order():
     lay = [(3, 7, 0, 40, 0), (3, 7, 40, 40, 2)]
     words = np.array([0b101, 1 << 7, 1, 0], dtype=np.uint32)

@@ -1,0 +1,116 @@
+"""Batch- and head-parallel shards on one GPU, through the C ABI.
+
+A shard is a handle over batch rows [b0, b0 + B) and heads [h0, h0 + H) of a larger problem
+(config fields b0, h0, H_total): its Philox counters are keyed on the whole problem's (b,h), so its
+decisions, coresets, outputs and log-sum-exps must equal the whole problem's run on the same GPU
+bit for bit -- the shards of a multi-GPU run compute exactly what one GPU would.  The shards run one
+after the other here (no kernel waits on another); the oracle of the whole problem checks one shard
+on its own as well.
+"""
+import numpy as np
+import pytest
+import torch
+
+import thinned_softmax_attention_b200 as TA
+import workloads as W
+from oracle import express, express_a, thinformer
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda", 0)
+
+
+def _run(w, q, k, v, shard=(0, 0, 0)):
+    B, T, H = q.shape[0], q.shape[1], q.shape[2]
+    S = k.shape[1]
+    h = TA.ThinAttention(B, T, S, H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch, shard=shard)
+    r = h.forward(q.to(DEV), k.to(DEV), v.to(DEV), causal=w.mode, g=w.g, seed=w.seed, return_lse=True,
+                  return_coreset=True, return_trace=True)
+    torch.cuda.synchronize()
+    h.check()
+    r["decisions"] = TA.decode_trace(r["trace"], h.trace_layout(w.mode, w.g))
+    r["H"] = H
+    return r
+
+
+def _assert_shard_equals_whole(whole, part, bsel, hsel, b0, h0):
+    assert torch.equal(part["out"], whole["out"][bsel][:, :, hsel])
+    assert torch.equal(part["lse"], whole["lse"][bsel][:, hsel])
+    assert torch.equal(part["coreset"], whole["coreset"][bsel][:, hsel])
+    Hw, Hp = whole["H"], part["H"]
+    n = 0
+    for (bh, rid), bits in part["decisions"].items():
+        g_bh = (b0 + bh // Hp) * Hw + h0 + bh % Hp
+        np.testing.assert_array_equal(bits, whole["decisions"][(g_bh, rid)])
+        n += 1
+    assert n > 0
+
+
+CASES = {
+    "vit": W.WORKLOADS["vit"].with_(B=4),
+    "biggan": W.WORKLOADS["biggan"].with_(B=2, T=1024),
+    "express": W.WORKLOADS["express32k"].with_(H=4, T=12 * 1024),
+    "express_a": W.WORKLOADS["express32k_a"].with_(H=4, T=12 * 1024),
+}
+
+
+@pytest.mark.parametrize("name", ["vit", "biggan"])
+def test_batch_shards_equal_the_whole_problem(name):
+    w = CASES[name]
+    q, k, v = W.make_qkv(w)
+    whole = _run(w, q, k, v)
+    for b0, b1 in [(0, 1), (1, w.B)]:
+        part = _run(w, q[b0:b1].contiguous(), k[b0:b1].contiguous(), v[b0:b1].contiguous(), shard=(b0, 0, 0))
+        _assert_shard_equals_whole(whole, part, slice(b0, b1), slice(0, w.H), b0, 0)
+
+
+@pytest.mark.parametrize("name", ["express", "express_a"])
+def test_head_shards_equal_the_whole_problem(name):
+    w = CASES[name]
+    q, k, v = W.make_qkv(w)
+    whole = _run(w, q, k, v)
+    for h0, h1 in [(0, 1), (1, 4)]:
+        sl = (slice(None), slice(None), slice(h0, h1))
+        part = _run(w, q[sl].contiguous(), k[sl].contiguous(), v[sl].contiguous(), shard=(0, h0, w.H))
+        _assert_shard_equals_whole(whole, part, slice(0, w.B), slice(h0, h1), 0, h0)
+
+
+def test_unsharded_stream_differs():
+    """Without its offsets a shard draws the stream of (b,h) = (0,0): its decisions differ."""
+    w = CASES["express"]
+    q, k, v = W.make_qkv(w, heads=[2])
+    right = _run(w, q, k, v, shard=(0, 2, w.H))
+    wrong = _run(w, q, k, v)
+    assert not torch.equal(right["coreset"], wrong["coreset"])
+
+
+@pytest.mark.parametrize("name", ["vit", "express", "express_a"])
+def test_shard_matches_the_oracle(name):
+    """One shard (batch row 1, or heads 2..3) against the oracle run with the shard's offsets."""
+    w = CASES[name]
+    if w.causal:
+        b0, hs = 0, [2, 3]
+        q, k, v = W.make_qkv(w.with_(B=1), heads=hs)
+        shard = (0, hs[0], w.H)
+    else:
+        b0, hs = 1, list(range(w.H))
+        q, k, v = W.make_qkv(w.with_(B=1), b0=b0)
+        shard = (b0, 0, w.H)
+    r = _run(w, q, k, v, shard=shard)
+    Hp = len(hs)
+    follow = {((b0 + bh // Hp) * w.H + hs[bh % Hp], rid): bits for (bh, rid), bits in r["decisions"].items()}
+    rows = np.sort(np.random.default_rng(3).choice(w.T, 256, replace=False))
+    kw = dict(follow=follow, rows=rows, heads=(w.H, hs), b0=b0)
+    if w.mode == 2:
+        ref = express_a(q, k, v, w.n_exact, w.g, w.seed, **kw)
+    elif w.mode == 1:
+        ref = express(q, k, v, w.n_exact, w.batch, w.g, w.seed, **kw)
+    else:
+        ref = thinformer(q, k, v, w.g, w.seed, **kw)
+    assert ref.stats.mismatches == 0
+    assert np.array_equal(r["coreset"].cpu().numpy(), ref.coreset)
+    o = r["out"].float().cpu().numpy()[:, rows]
+    err = np.abs(o - ref.out).max(axis=(1, 3)) / np.abs(ref.out).max(axis=(1, 3))
+    assert float(err.max()) <= 1e-2
+    lse = r["lse"].cpu().numpy()[:, :, rows]
+    assert float(np.abs(lse - ref.lse).max()) <= 2e-3

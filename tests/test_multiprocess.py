@@ -1,12 +1,15 @@
 """The multi-GPU host logic of bench.py on two gloo ranks (CPU, no GPU).
 
-Each rank runs its own problem (weak scaling, no collective on the data path); the only
-collective is the max of the per-rank step times, from which the whole-job throughput is
-computed.
+The ranks hold parts of one problem: batch rows (weak scaling) or heads (strong scaling).  No data
+crosses between ranks; the only collective is the max of the per-rank step times.  Each rank
+computes its part with the oracle under the shard's Philox offsets, the parts are gathered here
+(test-only), and the whole must equal the oracle run of the whole problem: sharding changes no
+decision and no output.
 """
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -23,41 +26,94 @@ def _free_port():
     return port
 
 
-def _rank(rank, world, port, q):
+# the whole problems: tiny fp32 Thinformer with 2 batch rows x 2 heads, and a short Express one
+_WHOLE = {
+    "thin": W.WORKLOADS["tiny"].with_(B=2, H=2),
+    "express": W.Workload("xs", 1, 2, 700, 700, 32, 32, "fp32", True, 1, 7, 5, "rope", n_exact=64, batch=128),
+}
+
+
+def _oracle_part(w, shard):
+    from oracle import express, thinformer
+    q, k, v = shard.inputs(w)
+    kw = dict(heads=(shard.H_total, shard.heads), b0=shard.b0)
+    if w.causal:
+        return express(q, k, v, w.n_exact, w.batch, w.g, w.seed, **kw)
+    return thinformer(q, k, v, w.g, w.seed, **kw)
+
+
+def _rank(rank, world, port, q, name, mode):
     import datetime
     import bench
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        w = bench.rank_workload(W.WORKLOADS["express32k"], rank)
-        step_ms = [2.0, 3.5][rank]
-        ms = bench.max_over_ranks(step_ms, dist, torch.device("cpu"))
-        val = bench.job_value(world, w.B * w.H * w.T, ms)
-        q.put((rank, w.data_seed, ms, val))
+        whole = _WHOLE[name]
+        whole = whole.with_(B=whole.B // world) if mode == "batch" else whole
+        sh = bench.Shard(whole, world, rank, mode)
+        part = _oracle_part(sh.local, sh)
+        out = torch.from_numpy(np.ascontiguousarray(part.out))
+        parts = [torch.empty_like(out) for _ in range(world)]
+        dist.all_gather(parts, out)                      # test-only: compare the whole on rank 0
+        ms = bench.max_over_ranks([2.0, 3.5][rank], dist, torch.device("cpu"))
+        q.put((rank, sh.b0, sh.h0, sh.local.B, sh.local.H, sh.scaling, sh.whole_tokens, ms,
+               [p.numpy() for p in parts] if rank == 0 else None))
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-def test_two_rank_weak_scaling_host_logic():
+def _run(name, mode):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q, name, mode)) for r in range(2)]
     for p in procs:
         p.start()
+    res = sorted((q.get(timeout=300) for _ in range(2)), key=lambda r: r[0])
     for p in procs:
-        p.join(120)
+        p.join(60)
     assert all(p.exitcode == 0 for p in procs)
-    res = sorted(q.get(timeout=5) for _ in range(2))
-    seeds = {r[1] for r in res}
-    assert len(seeds) == 2                                 # independent problems per rank
-    assert all(r[2] == 3.5 for r in res)                   # the slowest rank bounds the job
-    tokens = 32 * 32768
-    assert all(abs(r[3] - 2 * tokens / 3.5e-3) < 1e-6 * r[3] for r in res)
+    return res
+
+
+@pytest.mark.parametrize("name,mode", [("thin", "batch"), ("thin", "heads"), ("express", "heads")])
+def test_two_rank_shards_reproduce_the_whole_problem(name, mode):
+    from oracle import express, thinformer
+    res = _run(name, mode)
+    whole = _WHOLE[name]
+    assert all(r[7] == 3.5 for r in res)                 # the slowest rank bounds the job
+    if mode == "batch":
+        assert [(r[1], r[2], r[3], r[4]) for r in res] == [(0, 0, 1, 2), (1, 0, 1, 2)]
+        assert {r[5] for r in res} == {"weak"}
+        assert all(r[6] == whole.B * whole.H * whole.T for r in res)
+    else:
+        assert [(r[1], r[2], r[3], r[4]) for r in res] == [(0, 0, whole.B, 1), (0, 1, whole.B, 1)]
+        assert {r[5] for r in res} == {"strong"}
+    q, k, v = W.make_qkv(whole)
+    ref = (express(q, k, v, whole.n_exact, whole.batch, whole.g, whole.seed) if whole.causal
+           else thinformer(q, k, v, whole.g, whole.seed))
+    got = np.concatenate(res[0][8], axis=0 if mode == "batch" else 2)
+    np.testing.assert_array_equal(got, ref.out)
+
+
+def test_philox_offsets_matter():
+    """A shard that forgot its offset draws another stream: some decision differs."""
+    from oracle import thinformer
+    w = _WHOLE["thin"]
+    q, k, v = W.make_qkv(w)
+    whole = thinformer(q, k, v, w.g, w.seed)
+    q1, k1, v1 = q[1:], k[1:], v[1:]
+    right = thinformer(q1, k1, v1, w.g, w.seed, heads=(w.H, [0, 1]), b0=1)
+    wrong = thinformer(q1, k1, v1, w.g, w.seed)
+    np.testing.assert_array_equal(right.coreset, whole.coreset[1:])
+    assert not np.array_equal(wrong.coreset, whole.coreset[1:])
 
 
 def test_single_process_needs_no_collective():
     import bench
     assert bench.max_over_ranks(4.25, None, torch.device("cpu")) == 4.25
-    assert bench.rank_workload(W.WORKLOADS["tiny"], 0) == W.WORKLOADS["tiny"]
+    sh = bench.Shard(W.WORKLOADS["express32k"], 1, 0)
+    assert sh.abi == (0, 0, 32) and sh.local == W.WORKLOADS["express32k"] and sh.scaling == "weak"
+    with pytest.raises(ValueError):
+        bench.Shard(W.WORKLOADS["express32k"], 3, 0, "heads")

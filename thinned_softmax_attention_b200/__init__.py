@@ -36,7 +36,8 @@ class ThinAttnError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("B", ctypes.c_int), ("T", ctypes.c_int), ("S", ctypes.c_int),
                 ("H", ctypes.c_int), ("E", ctypes.c_int), ("D", ctypes.c_int), ("scale", ctypes.c_float),
-                ("n_exact", ctypes.c_int), ("batch", ctypes.c_int), ("device", ctypes.c_int)]
+                ("n_exact", ctypes.c_int), ("batch", ctypes.c_int), ("device", ctypes.c_int),
+                ("b0", ctypes.c_int), ("h0", ctypes.c_int), ("H_total", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -111,12 +112,18 @@ class ThinAttention:
     ``forward(q, k, v, causal, g, seed)`` returns ``(attn_output, None)``: the dense
     attention weights are never formed; pass ``return_lse=True`` for the
     log-sum-exp ln sum_j w_j e^{s q.k_j} instead.
+
+    ``shard=(b0, h0, H_total)``: the tensors hold batch rows [b0, b0 + B) and heads
+    [h0, h0 + H) of a larger problem with H_total heads (one handle per GPU of a batch- or
+    head-parallel run); the random decisions, and so every output, equal the whole
+    problem's for those (b,h).
     """
 
     def __init__(self, B: int, T: int, S: int, H: int, E: int, D: int, dtype: torch.dtype,
-                 scale: Optional[float] = None, n_exact: int = 0, batch: int = 0, device: int = 0):
+                 scale: Optional[float] = None, n_exact: int = 0, batch: int = 0, device: int = 0,
+                 shard: Tuple[int, int, int] = (0, 0, 0)):
         self.cfg = Config(FP32 if dtype == torch.float32 else BF16, B, T, S, H, E, D,
-                          0.0 if scale is None else float(scale), n_exact, batch, device)
+                          0.0 if scale is None else float(scale), n_exact, batch, device, *shard)
         self.dtype = dtype
         self.device = torch.device("cuda", device)
         self._h = ctypes.c_void_p()
@@ -231,9 +238,10 @@ class ThinAttentionCache:
     """
 
     def __init__(self, B: int, H: int, E: int, D: int, dtype: torch.dtype, capacity: int, n_exact: int, batch: int,
-                 g: int = 2, seed: int = 0, scale: Optional[float] = None, device: int = 0):
+                 g: int = 2, seed: int = 0, scale: Optional[float] = None, device: int = 0,
+                 shard: Tuple[int, int, int] = (0, 0, 0)):
         self.cfg = Config(FP32 if dtype == torch.float32 else BF16, B, capacity, capacity, H, E, D,
-                          0.0 if scale is None else float(scale), n_exact, batch, device)
+                          0.0 if scale is None else float(scale), n_exact, batch, device, *shard)
         self.dtype, self.device = dtype, torch.device("cuda", device)
         self._h = ctypes.c_void_p()
         _check(lib().thin_attn_cache_create(ctypes.byref(self._h), ctypes.byref(self.cfg), g,

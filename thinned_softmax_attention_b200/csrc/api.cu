@@ -207,6 +207,11 @@ struct thin_attn_s {
 namespace {
 
 size_t elt(const thin_attn_config& c) { return c.dtype == THIN_ATTN_FP32 ? 4 : 2; }
+// Philox (b,h) word of the handle's local b * H + h: its index in the whole problem.
+uint32_t ctr_bh_of(const thin_attn_config& c, uint32_t bh) {
+  const uint32_t Ht = (uint32_t)(c.H_total > 0 ? c.H_total : c.H);
+  return ((uint32_t)c.b0 + bh / (uint32_t)c.H) * Ht + (uint32_t)c.h0 + bh % (uint32_t)c.H;
+}
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct DeviceGuard {
@@ -577,6 +582,7 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
   // trace layout and scratch sizes
   for (auto& st : p->steps) {
     st.sub_stride = sub_stride_of(st);
+    for (auto& in : st.inst) in.ctr_bh = ctr_bh_of(cf, in.bh);
     if (st.copy_only) continue;
     st.trace_base = p->trace_words;
     const int nw = st.m_pad / 32;
@@ -675,8 +681,15 @@ thin_attn_status check_cfg(const thin_attn_config* c) {
   if (c->E < 8 || c->E > 256 || c->E % 8 || c->D < 8 || c->D > 256 || c->D % 8)
     return fail(THIN_ATTN_EINVAL, "E=%d D=%d: widths must be multiples of 8 in [8, 256]", c->E, c->D);
   if ((int64_t)c->B * c->T * c->H > ((int64_t)1 << 31) / 4) return fail(THIN_ATTN_EINVAL, "B*T*H too large");
+  const int64_t Ht = c->H_total > 0 ? c->H_total : c->H;
+  if (c->b0 < 0 || c->h0 < 0 || c->h0 + (int64_t)c->H > Ht)
+    return fail(THIN_ATTN_EINVAL, "shard b0=%d h0=%d H=%d outside the whole problem's H_total=%lld", c->b0, c->h0, c->H,
+                (long long)Ht);
+  if (((int64_t)c->b0 + c->B) * Ht > (int64_t)UINT32_MAX)
+    return fail(THIN_ATTN_EINVAL, "(b0 + B) * H_total exceeds the 32-bit Philox (b,h) word");
   return THIN_ATTN_OK;
 }
+
 
 thin_attn_status get_plan(thin_attn_s* h, int causal, int g, Plan** out) {
   if (causal < 0 || causal > 2) return fail(THIN_ATTN_EINVAL, "causal must be 0, 1 or 2");
@@ -1229,6 +1242,7 @@ namespace {
 
 void cache_add_step(thin_attn_cache_s* cc, CacheStep& st) {
   st.sp.sub_stride = sub_stride_of(st.sp);
+  for (auto& in : st.sp.inst) in.ctr_bh = ctr_bh_of(cc->cf, in.bh);
   cc->delta_floats = std::max(cc->delta_floats, st.sp.inst.size() * (size_t)st.sp.m_pad * st.sp.m_pad);
   cc->c2_floats = std::max(cc->c2_floats, st.sp.inst.size());
 }

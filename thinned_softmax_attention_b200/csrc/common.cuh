@@ -71,7 +71,7 @@ struct HalveInst {
   uint32_t pair0;      // Philox pair index of pair 0
   uint32_t sub_round;  // Philox round of the subsample word (SRC_TOKENS with S_sub < S_full)
   uint32_t tok0;       // SRC_TOKENS: token index of the run start (stored in idx)
-  uint32_t pad;
+  uint32_t ctr_bh;     // (b,h) word of the Philox counter: (b0 + b) * H_total + h0 + h of the whole problem
 };
 
 struct StepArgs {
@@ -112,7 +112,7 @@ struct StepArgs {
 // Subsample word U of an instance (0 when no subsample).
 __device__ __forceinline__ uint32_t sub_offset(const StepArgs& a, const HalveInst& in) {
   if (a.src_kind != SRC_TOKENS || a.S_sub >= a.S_full) return 0u;
-  return philox_x0(a.seed, in.bh, in.sub_round, 0u) % (uint32_t)a.S_sub;
+  return philox_x0(a.seed, in.ctr_bh, in.sub_round, 0u) % (uint32_t)a.S_sub;
 }
 
 // Row of point p (0..n-1) of an instance: element offset of its K row, V row, and its token index.

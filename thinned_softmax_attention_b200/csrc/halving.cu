@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(128, 8) walk_kernel(StepArgs a) {
 
   for (int i = tid; i < mp; i += 128) {
     alpha[i] = 0.f;
-    ubuf[i] = i < m ? philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)i) : 0.5f;
+    ubuf[i] = i < m ? philox_uniform(a.seed, in.ctr_bh, in.round_id, in.pair0 + (uint32_t)i) : 0.5f;
   }
   if (tid == 0) U_s = sub_offset(a, in);
   float sigma = 0.f;
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(128) walk_small_kernel(StepArgs a) {
   float d[32];
 #pragma unroll
   for (int s = 0; s < 32; ++s) d[s] = (s < m && lane < m) ? Dl[(size_t)s * a.m_pad + lane] : 0.f;
-  const float w_l = lane < m ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)lane) : 0.f;
+  const float w_l = lane < m ? 1.f - 2.f * philox_uniform(a.seed, in.ctr_bh, in.round_id, in.pair0 + (uint32_t)lane) : 0.f;
   const uint32_t U = sub_offset(a, in);
   // Pairs s >= m are no-ops: their Delta entries are 0, so b^2 = 0 keeps sigma and alpha as they
   // are, and their bits are never read.
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(128) walk_mid_kernel(StepArgs a) {
   stage(0);
   for (int i = tid; i < mp; i += 128) {
     alpha[i] = 0.f;
-    wbuf[i] = i < m ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)i) : 0.f;
+    wbuf[i] = i < m ? 1.f - 2.f * philox_uniform(a.seed, in.ctr_bh, in.round_id, in.pair0 + (uint32_t)i) : 0.f;
   }
   const float C = a.C, rC = 1.f / C;
   float sigma = 0.f;

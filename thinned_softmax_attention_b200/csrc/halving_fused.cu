@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
         __syncwarp();
         mbar_arrive(dempty + set);
         const float w_l =
-            (live && sl < m) ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)sl) : 0.f;
+            (live && sl < m) ? 1.f - 2.f * philox_uniform(a.seed, in.ctr_bh, in.round_id, in.pair0 + (uint32_t)sl) : 0.f;
         const uint32_t kb = walk_segment<SEG>(d, w_l, C, lane);
         if (!warp_wait(full + s, (k / nst) & 1, abort)) break;   // (complete: orders the stage reads)
 #pragma unroll
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
             const int p = 32 * blk + lane;
             const float b2l = D[p * Sh::LD + p];
             const float wl =
-                (live && p < m) ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)p) : 0.f;
+                (live && p < m) ? 1.f - 2.f * philox_uniform(a.seed, in.ctr_bh, in.round_id, in.pair0 + (uint32_t)p) : 0.f;
             thr_s[set][p] = thresholds32(sigma, b2l, wl, C, rC, lane);
             __syncwarp();
             mbar_arrive(thf + set);
@@ -666,7 +666,7 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
     for (int blk = 0; blk < 4; ++blk) {
       if (!warp_wait(blk < 2 ? dhalf : dfull, 0, abort)) break;
       const int p = 32 * blk + lane;
-      const float wl = p < m ? 1.f - 2.f * philox_uniform(a.seed, in.bh, in.round_id, in.pair0 + (uint32_t)p) : 0.f;
+      const float wl = p < m ? 1.f - 2.f * philox_uniform(a.seed, in.ctr_bh, in.round_id, in.pair0 + (uint32_t)p) : 0.f;
       thr_s[p] = thresholds32(sigma, D[p * LD + p], wl, C, rC, lane);
       __syncwarp();
       mbar_arrive(thf + blk);

@@ -69,6 +69,7 @@ __global__ void fill_noalloc_tables(HalveInst* inst, int32_t* pidx, int n_inst, 
     h.src_row = i * n;
     h.dst_row = i * m;
     h.bh = (uint32_t)i;
+    h.ctr_bh = (uint32_t)i;
     h.round_id = round_id;
     inst[i] = h;
   }

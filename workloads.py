@@ -131,10 +131,11 @@ def slice_qkv(w: Workload, b: int, h: int, T: int | None = None, S: int | None =
 
 
 def make_qkv(w: Workload, T: int | None = None, S: int | None = None,
-             heads: Iterable[int] | None = None):
+             heads: Iterable[int] | None = None, b0: int = 0):
     """Full (B,T,H,E), (B,S,H,E), (B,S,H,D) tensors on the CPU.
 
-    ``heads`` restricts to a subset of heads (the H axis then has len(heads)).
+    ``heads`` restricts to a subset of heads (the H axis then has len(heads)); ``b0`` is the
+    index of batch row 0 in a larger problem (rows b0 .. b0+B-1 of it are drawn).
     """
     T = w.T if T is None else T
     S = (T if w.causal else w.S) if S is None else S
@@ -145,6 +146,6 @@ def make_qkv(w: Workload, T: int | None = None, S: int | None = None,
     v = torch.empty(w.B, S, len(hs), w.D, dtype=dt)
     for b in range(w.B):
         for j, h in enumerate(hs):
-            qs, ks, vs = slice_qkv(w, b, h, T, S)
+            qs, ks, vs = slice_qkv(w, b0 + b, h, T, S)
             q[b, :, j], k[b, :, j], v[b, :, j] = qs, ks, vs
     return q, k, v
