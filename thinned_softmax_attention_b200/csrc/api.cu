@@ -635,13 +635,13 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
 
 thin_attn_status materialise(thin_attn_s* h, Plan* p) {
   if (!h->d_status) {
-    cudaError_t e = cudaMalloc(&h->d_status, 16);
+    cudaError_t e = cudaMalloc(&h->d_status, kStatusBytes);
     if (e != cudaSuccess) {
       cudaGetLastError();
       h->d_status = nullptr;
       return fail(THIN_ATTN_ENOMEM, "status word: %s", cudaGetErrorString(e));
     }
-    e = cudaMemset(h->d_status, 0, 16);
+    e = cudaMemset(h->d_status, 0, kStatusBytes);
     if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "status word: %s", cudaGetErrorString(e));
   }
   if (p->d_mem) return THIN_ATTN_OK;
@@ -1430,8 +1430,8 @@ thin_attn_status cache_build(thin_attn_cache_s* cc) {
   std::memcpy(host.data() + t.tiles_off, t.tiles.data(), t.tiles.size() * sizeof(AttnTile));
   std::memcpy(host.data() + t.segs_off, t.segs.data(), t.segs.size() * sizeof(AttnSeg));
   CK(cudaMemcpy(cc->d_mem, host.data(), table_end, cudaMemcpyHostToDevice));
-  CK(cudaMalloc(&cc->d_status, 16));
-  CK(cudaMemset(cc->d_status, 0, 16));
+  CK(cudaMalloc(&cc->d_status, kStatusBytes));
+  CK(cudaMemset(cc->d_status, 0, kStatusBytes));
   CK(cudaMemset((char*)cc->d_mem + cc->nodes.idx_off, 0xFF, (size_t)cc->nodes.rows * 4));
   return THIN_ATTN_OK;
 }

@@ -693,6 +693,313 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
 }
 
 
+// Persistent form of attn_tc2_kernel: two CTAs per SM, each looping over work items (query tile,
+// (b,h)).  Items are handed out dynamically in the order the per-tile grid runs -- (b,h) by
+// (b,h), the last (heaviest) tiles first: item j = tile n_tiles-1 - j % n_tiles of (b,h)
+// j / n_tiles -- so the CTAs running at one time read the keys of one or two heads (they stay in
+// L2) and the load balances like the hardware's own block scheduling.  The producer takes the next
+// item from a counter in global memory (sched[0]) and passes it to the MMA and softmax roles
+// through a two-slot ring in shared memory; the last CTA to leave resets the counter (sched[1]
+// counts the CTAs that left).  Per item the roles run the same key-tile pipeline as attn_tc2_kernel; what persistence
+// adds is the overlap between items: the producer loads the next item's Q as soon as the last S
+// MMA of the current item has read Q (q_empty), and the next item's first S MMA runs while the
+// softmax warps write the current item's O (the first PV of an item waits for that: o_empty).
+// Barrier parities follow a key-tile count and an item count that run across items.
+template <int E, int D>
+__global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a,
+                                                           int* status) {
+  using Lay = Tc2Layout<E, D>;
+  constexpr uint32_t O_COL = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + Lay::OFF_K;
+  uint8_t* sV = smem + Lay::OFF_V;
+  uint64_t* bars = (uint64_t*)(smem + Lay::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 2;
+  uint64_t* v_full = bars + 3;
+  uint64_t* v_empty = bars + 4;
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;      // P of all keys of the tile written (128 threads)
+  uint64_t* pv_done = bars + 7;
+  uint64_t* p_half = bars + 8;      // P of keys 0..BN/2-1 written (128 threads)
+  uint64_t* q_empty = bars + 9;     // the item's last S MMA has read Q (commit)
+  uint64_t* o_empty = bars + 10;    // the item's O has been read out of TMEM (128 threads)
+  uint64_t* item_full = bars + 11;  // [2] next item index published (producer)
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  __shared__ volatile int where_s;
+  __shared__ int item_s;
+  __shared__ int item_ring[2];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = a.n_tiles * a.B * a.H;
+  int* sched = status + 4;
+
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    where_s = 0;
+    item_s = -1;
+    mbar_init(q_full, 1);
+    mbar_init(k_full, 1);
+    mbar_init(k_empty, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(p_half, 128);
+    mbar_init(q_empty, 1);
+    mbar_init(o_empty, 128);
+    mbar_init(item_full, 1);
+    mbar_init(item_full + 1, 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) tmem_alloc(&tmem_base_s, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort = &abort_s;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int git = 0, r = 0;
+      bool ok = true;
+      for (;; ++r) {
+        // the ring slot of item r was last read at the start of item r-2, before q_empty(r-1)
+        if (r > 0 && !mbar_wait(q_empty, (r - 1) & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 9000 + min(r, 999));
+          ok = false;
+        }
+        const int j = ok ? atomicAdd(sched, 1) : n_items;
+        item_ring[r & 1] = j < n_items ? j : -1;
+        mbar_arrive(item_full + (r & 1));
+        if (j >= n_items) break;
+        const AttnTile tile = a.tiles[a.tile0 + a.n_tiles - 1 - j % a.n_tiles];
+        const int bh = j / a.n_tiles, b = bh / a.H, h = bh % a.H;
+        mbar_expect_tx(q_full, Lay::Q_BYTES);
+#pragma unroll
+        for (int c = 0; c < Lay::EC; ++c) tma_load_3d(sQ + c * 16384, &maps.q, q_full, c * 64, h, b * a.T + tile.q0);
+        for (int si = 0; si < tile.nseg && ok; ++si) {
+          const AttnSeg sg = a.segs[tile.seg0 + si];
+          const bool tok = sg.kind == SEG_TOKENS;
+          for (int j0 = 0; j0 < sg.len; j0 += BN, ++git) {
+            const int row = tok ? b * a.L + sg.first + j0 : (bh * a.n_slots + sg.first) * a.slot_rows + j0;
+            if (git > 0 && !mbar_wait(k_empty, (git - 1) & 1, abort)) {
+              ok = false;
+              atomicCAS((int*)&where_s, 0, 1000 + min(git, 999));
+              break;
+            }
+            const bool withhold = a.inject_timeout && a.tile0 == 0 && git == 0 && blockIdx.x == 0;
+            if (!withhold) {
+              mbar_expect_tx(k_full, Lay::K_BYTES);
+#pragma unroll
+              for (int c = 0; c < Lay::EC; ++c) {
+                if (tok) tma_load_3d(sK + c * 16384, &maps.k, k_full, c * 64, h, row);
+                else tma_load_2d(sK + c * 16384, &maps.ck, k_full, c * 64, row);
+              }
+            }
+            if (git > 0 && !mbar_wait(v_empty, (git - 1) & 1, abort)) {
+              ok = false;
+              atomicCAS((int*)&where_s, 0, 2000 + min(git, 999));
+              break;
+            }
+            mbar_expect_tx(v_full, Lay::V_BYTES);
+#pragma unroll
+            for (int c = 0; c < Lay::DC; ++c) {
+              if (tok) tma_load_3d(sV + c * 16384, &maps.v, v_full, c * 64, h, row);
+              else tma_load_2d(sV + c * 16384, &maps.cv, v_full, c * 64, row);
+            }
+          }
+        }
+        if (!ok) break;   // abort is set: every other role's next wait returns at once
+      }
+      // never leave with a copy in flight into this CTA's shared memory
+      if (git > 0) {
+        long long t0 = clock64();
+        while (!mbar_try_wait(k_full, (git - 1) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+        t0 = clock64();
+        while (!mbar_try_wait(v_full, (git - 1) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+      if (r > 0) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(q_full, (r - 1) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IQK = idesc_bf16(BM, BN, false);
+      constexpr uint32_t IPV = idesc_bf16(BM, D, true);
+      const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
+      int git = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        if (!mbar_wait(item_full + (r & 1), (r >> 1) & 1, abort)) break;
+        const int j = item_ring[r & 1];
+        if (j < 0) break;
+        const AttnTile tile = a.tiles[a.tile0 + a.n_tiles - 1 - j % a.n_tiles];
+        const int n_kt = count_key_tiles(a, tile);
+        if (!mbar_wait(q_full, r & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 4000 + min(r, 999));
+          break;
+        }
+        for (int it = 0; it < n_kt; ++it, ++git) {
+          // S(it) may overwrite the P columns PV(it-1) reads: tcgen05.mma ops issued by one thread
+          // execute in issue order, and the commit after S(it) tracks PV(it-1) too
+          if (!mbar_wait(k_full, git & 1, abort)) {
+            ok = false;
+            atomicCAS((int*)&where_s, 0, 3000 + min(git, 999));
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < E / 16; ++k) {
+            const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+            umma_bf16(tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), IQK, k > 0);
+          }
+          umma_commit(s_full);
+          umma_commit(k_empty);
+          if (it == n_kt - 1) umma_commit(q_empty);
+          if (!mbar_wait(p_half, git & 1, abort) || !mbar_wait(v_full, git & 1, abort) ||
+              (it == 0 && r > 0 && !mbar_wait(o_empty, (r - 1) & 1, abort))) {
+            ok = false;
+            atomicCAS((int*)&where_s, 0, 5000 + min(git, 999));
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < BN / 32; ++k)
+            umma_bf16_tmem_a(tmem + O_COL, tmem + k * 8, sw128_desc(va + k * 2048, 16384, 1024), IPV,
+                             (it > 0 || k > 0) ? 1u : 0u);
+          if (!mbar_wait(p_full, git & 1, abort)) {
+            ok = false;
+            atomicCAS((int*)&where_s, 0, 7000 + min(git, 999));
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = BN / 32; k < BN / 16; ++k)
+            umma_bf16_tmem_a(tmem + O_COL, tmem + k * 8, sw128_desc(va + k * 2048, 16384, 1024), IPV, 1u);
+          umma_commit(pv_done);
+          umma_commit(v_empty);
+        }
+        if (n_kt == 0) umma_commit(q_empty);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroup
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    int git = 0, where = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      if (!warp_wait(item_full + (r & 1), (r >> 1) & 1, abort)) {
+        where = 10;
+        break;
+      }
+      const int j = item_ring[r & 1];
+      if (j < 0) break;
+      const int tile_id = a.tile0 + a.n_tiles - 1 - j % a.n_tiles;
+      const AttnTile tile = a.tiles[tile_id];
+      const int bh = j / a.n_tiles, b = bh / a.H, h = bh % a.H;
+      if (count_key_tiles(a, tile) == 0) {
+        mbar_arrive(o_empty);
+        continue;
+      }
+      if (threadIdx.x == 0) item_s = tile_id * 65536 + bh;
+      const int tq = tile.q0 + row;
+      float m_used = -INFINITY, l = 0.f;
+      int it = 0;
+      for (int si = 0; si < tile.nseg && ok; ++si) {
+        const AttnSeg sg = a.segs[tile.seg0 + si];
+        const float lw2 = sg.logw * 1.4426950408889634f;
+        for (int j0 = 0; j0 < sg.len; j0 += BN, ++it, ++git) {
+          if (!warp_wait(s_full, git & 1, abort)) {
+            ok = false;
+            where = 6;
+            break;
+          }
+          tc_fence_after();
+          const int nvalid = min(BN, sg.len - j0);
+          const int kt0 = sg.first + j0;
+          const bool causal = sg.kind == SEG_TOKENS && sg.causal;
+          const bool masked = nvalid < BN || (causal && kt0 + BN - 1 > tile.q0);
+          const int lim = min(nvalid - 1, causal ? tq - kt0 : BN - 1);
+          if (masked) softmax_tile<true, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
+          else softmax_tile<false, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(p_full);
+        }
+      }
+      if (!ok) break;
+      if (!warp_wait(pv_done, (git - 1) & 1, abort)) {
+        where = 8;
+        break;
+      }
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* out = (__nv_bfloat16*)a.out;
+      const bool live = row < tile.qlen;
+      __nv_bfloat16* orow = out + ((int64_t)(b * a.T + tq) * a.H + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 u;
+            __nv_bfloat162 t0 = __floats2bfloat162_rn(o[i] * inv, o[i + 1] * inv);
+            __nv_bfloat162 t1 = __floats2bfloat162_rn(o[i + 2] * inv, o[i + 3] * inv);
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(o[i + 4] * inv, o[i + 5] * inv);
+            __nv_bfloat162 t3 = __floats2bfloat162_rn(o[i + 6] * inv, o[i + 7] * inv);
+            u.x = *reinterpret_cast<uint32_t*>(&t0);
+            u.y = *reinterpret_cast<uint32_t*>(&t1);
+            u.z = *reinterpret_cast<uint32_t*>(&t2);
+            u.w = *reinterpret_cast<uint32_t*>(&t3);
+            *reinterpret_cast<uint4*>(orow + c * 32 + i) = u;
+          }
+        }
+      }
+      // O is in registers: the next item's first PV may overwrite it
+      tc_fence_before();
+      mbar_arrive(o_empty);
+      if (live && a.lse) a.lse[(int64_t)bh * a.T + tq] = (m_used + log2f(l)) * 0.6931471805599453f;
+    }
+    if (where && lane == 0) atomicCAS((int*)&where_s, 0, where * 1000 + min(git, 999));
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_s && threadIdx.x == 0) {
+    if (atomicCAS(status, 0, 1) == 0) {
+      status[1] = item_s;
+      status[2] = where_s;
+    }
+  }
+  if (threadIdx.x == 0) {
+    // every CTA has taken its last item before it counts itself out: the last one resets
+    __threadfence();
+    if (atomicAdd(sched + 1, 1) == (int)gridDim.x - 1) {
+      atomicExch(sched, 0);
+      atomicExch(sched + 1, 0);
+    }
+  }
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 template <int E, int D>
 cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
   TcMaps maps;
@@ -710,9 +1017,20 @@ cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
   if constexpr (D <= 128) {
     if (std::getenv("THIN_ATTN_TC1") == nullptr) {
       const size_t sm = Tc2Layout<E, D>::BYTES;
-      cudaError_t e = cudaFuncSetAttribute(attn_tc2_kernel<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if (std::getenv("THIN_ATTN_TC2_PER_TILE") != nullptr || status == nullptr) {
+        cudaError_t e = cudaFuncSetAttribute(attn_tc2_kernel<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        attn_tc2_kernel<E, D><<<dim3(a.n_tiles, a.B * a.H), 192, sm, st>>>(maps, a, status);
+        return cudaGetLastError();
+      }
+      int dev = 0, sms = 0;
+      cudaError_t e = cudaGetDevice(&dev);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_tc2p_kernel<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
       if (e != cudaSuccess) return e;
-      attn_tc2_kernel<E, D><<<dim3(a.n_tiles, a.B * a.H), 192, sm, st>>>(maps, a, status);
+      const int64_t items = (int64_t)a.n_tiles * a.B * a.H;
+      const int grid = (int)std::min<int64_t>(items, 2 * (int64_t)sms);
+      attn_tc2p_kernel<E, D><<<grid, 192, sm, st>>>(maps, a, status);
       return cudaGetLastError();
     }
   }

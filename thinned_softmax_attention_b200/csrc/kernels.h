@@ -26,6 +26,11 @@ size_t walk_smem_bytes(int m_pad);
 cudaError_t launch_attention_simt(const AttnArgs& a, int dtype, cudaStream_t st);
 int attention_simt_tile_rows();
 // Tensor-core attention (bf16, E = D = 128); *done = false when the shape is not covered.
+// Device status buffer of a handle (zeroed at creation): ints [0..3] the status word (code and
+// detail of a bounded wait that gave up), [4..5] the work counter of the persistent attention
+// kernel (left at zero by every launch).
+constexpr size_t kStatusBytes = 32;
+
 cudaError_t launch_attention_tc(const AttnArgs& a, int* status_word, cudaStream_t st, bool* done);
 int attention_tc_tile_rows();
 bool attention_tc_supported(int dtype, int E, int D);
