@@ -950,30 +950,30 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
       __nv_bfloat16* out = (__nv_bfloat16*)a.out;
       const bool live = row < tile.qlen;
       __nv_bfloat16* orow = out + ((int64_t)(b * a.T + tq) * a.H + h) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
-        tmem_ld_wait();
-        if (live) {
+      // the row of O, normalised and packed to bf16 pairs in registers (64 columns per TMEM wait),
+      // then O is released to the next item's first PV before the stores go out
+      uint32_t pk[D / 2];
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 u;
-            __nv_bfloat162 t0 = __floats2bfloat162_rn(o[i] * inv, o[i + 1] * inv);
-            __nv_bfloat162 t1 = __floats2bfloat162_rn(o[i + 2] * inv, o[i + 3] * inv);
-            __nv_bfloat162 t2 = __floats2bfloat162_rn(o[i + 4] * inv, o[i + 5] * inv);
-            __nv_bfloat162 t3 = __floats2bfloat162_rn(o[i + 6] * inv, o[i + 7] * inv);
-            u.x = *reinterpret_cast<uint32_t*>(&t0);
-            u.y = *reinterpret_cast<uint32_t*>(&t1);
-            u.z = *reinterpret_cast<uint32_t*>(&t2);
-            u.w = *reinterpret_cast<uint32_t*>(&t3);
-            *reinterpret_cast<uint4*>(orow + c * 32 + i) = u;
+      for (int c2 = 0; c2 < D / 64; ++c2) {
+        float o[2][32];
+        tmem_ld32(tmem + lane_base + O_COL + c2 * 64, o[0]);
+        tmem_ld32(tmem + lane_base + O_COL + c2 * 64 + 32, o[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const __nv_bfloat162 t = __floats2bfloat162_rn(o[hh][i] * inv, o[hh][i + 1] * inv);
+            pk[(c2 * 64 + hh * 32 + i) / 2] = *reinterpret_cast<const uint32_t*>(&t);
           }
-        }
       }
-      // O is in registers: the next item's first PV may overwrite it
       tc_fence_before();
       mbar_arrive(o_empty);
+      if (live) {
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i)
+          *reinterpret_cast<uint4*>(orow + 8 * i) = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      }
       if (live && a.lse) a.lse[(int64_t)bh * a.T + tq] = (m_used + log2f(l)) * 0.6931471805599453f;
     }
     if (where && lane == 0) atomicCAS((int*)&where_s, 0, where * 1000 + min(git, 999));
