@@ -235,6 +235,38 @@ def test_fused_and_three_launch_halving_agree(causal, monkeypatch):
         assert torch.equal(res[0][key], res[1][key]), key
 
 
+@pytest.mark.parametrize("name", ["vit", "express", "express_a"])
+def test_attention_launch_forms_agree(name, monkeypatch):
+    """The persistent attention kernel (items from a work counter), its one-CTA-per-tile form, and
+    the persistent kernel launched as several dependent waves on a side stream (each launch takes
+    and resets the same counter) run the same per-tile arithmetic: outputs and LSE are bit-identical."""
+    w = {"vit": W.WORKLOADS["vit"].with_(B=8),
+         "express": W.WORKLOADS["express32k"].with_(T=8192, H=4),
+         "express_a": W.WORKLOADS["express32k_a"].with_(T=8192, H=4)}[name]
+    S = w.T if w.causal else w.S
+    q, k, v = (x.cuda() for x in W.make_qkv(w))
+    forms = [{}, {"THIN_ATTN_TC2_PER_TILE": "1"}, {"THIN_ATTN_OVERLAP": "1"}]
+    res = []
+    for env in forms:
+        for key in ("THIN_ATTN_TC2_PER_TILE", "THIN_ATTN_OVERLAP"):
+            if key in env:
+                monkeypatch.setenv(key, env[key])
+            else:
+                monkeypatch.delenv(key, raising=False)
+        h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
+        outs = []
+        for _ in range(2):   # a second forward on the same handle starts from a reset counter
+            r = h.forward(q, k, v, causal=w.mode, g=w.g, seed=w.seed, return_lse=True)
+            torch.cuda.synchronize()
+            h.check()
+            outs.append(r)
+        assert torch.equal(outs[0]["out"], outs[1]["out"])
+        res.append(outs[0])
+    for r in res[1:]:
+        assert torch.equal(res[0]["out"], r["out"])
+        assert torch.equal(res[0]["lse"], r["lse"])
+
+
 def test_profile_steps_cover_the_halving_phases():
     w = W.WORKLOADS["express32k"].with_(T=8192, H=4)
     q, k, v = (x.cuda() for x in W.make_qkv(w))
