@@ -729,6 +729,385 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Instances of 257..512 points (the first step of a HALVE merge of four 128-point nodes): one CTA per
+// instance.  The 256 x 256 pair differences are kept as the packed upper triangle (row j holds
+// columns j..255, 131.6 KB) in shared memory (before the first Delta is written, that area holds the
+// instance's V rows, loaded by TMA for c = max |v|); the 512 point rows do not fit beside it, so the Gram
+// runs over the 10 upper-triangle pairs (bi <= bj) of 128-row blocks in row-block order, each a
+// (128 x 128) kk and vv product streamed through a two-stage ring of 64-column chunks (A = rows of
+// block bi, B = rows of block bj), accumulators double-buffered in TMEM.  The kept rows are gathered
+// from global memory
+// (still in L2: the ring read them moments before).  Warps: 0 TMA, 1 MMA (TMEM owner), 2-5 epilogue
+// (warp w reads TMEM lanes 32 (w % 4)..), 6 sigma's recursion, 7 the walk; all eight gather.  The
+// walk of pair block t starts once Delta rows 32t..32t+31 (row block t/2) are complete.  Every wait
+// is bounded.
+constexpr int kH512Pairs = 256;
+
+__device__ __forceinline__ int tri_offset(int j) { return j * kH512Pairs - (j * (j - 1)) / 2; }
+
+// Copy the kept point of pairs [i0, i1) of one instance from its source rows in global memory to
+// destination rows dst_row + i, with its token index.  One warp; lane = one 16-byte unit of a row
+// (K units first), ROWS rows in flight.  Token runs: point p is token tok0 + (2 pair0 + p) k of
+// the (b,h) run (k = subsample stride, 1 without subsample).
+template <int ROWS, typename Bit>
+__device__ __forceinline__ void gather_global(const StepArgs& a, const HalveInst& in, int i0, int i1, Bit bit, int lane) {
+  const bool tokens = a.src_kind == SRC_TOKENS;
+  const int64_t k = a.sub_stride > 1 ? a.sub_stride : 1;
+  const int h = (int)(in.bh % (uint32_t)a.H);
+  const int kw = a.E / 8, vw = a.D / 8, units = kw + vw;
+  const uint4* K = (const uint4*)a.srcK;
+  const uint4* V = (const uint4*)a.srcV;
+  uint4* dK = (uint4*)a.dstK;
+  uint4* dV = (uint4*)a.dstV;
+  for (int g = i0; g < i1; g += 32) {
+    const int i = g + lane;
+    int64_t row = 0;
+    if (i < i1) {
+      const int p = 2 * i + (bit(i) ? 0 : 1);
+      if (tokens) {
+        const int64_t t = (2 * (int64_t)in.pair0 + p) * k;
+        row = (in.src_row + t) * a.H + h;
+        a.dstIdx[in.dst_row + i] = (int32_t)(in.tok0 + t);
+      } else {
+        row = in.src_row + p;
+        a.dstIdx[in.dst_row + i] = a.srcIdx[row];
+      }
+    }
+    const int nrows = min(32, i1 - g);
+    for (int w0 = 0; w0 < units; w0 += 32) {
+      const int w = w0 + lane;
+      const bool act = w < units, isk = w < kw;
+      for (int j = 0; j < nrows; j += ROWS) {
+        uint4 buf[ROWS];
+#pragma unroll
+        for (int jj = 0; jj < ROWS; ++jj) {
+          const int64_t r = __shfl_sync(0xffffffffu, row, (j + jj) & 31);
+          if (act && j + jj < nrows) buf[jj] = isk ? K[r * kw + w] : V[r * vw + (w - kw)];
+        }
+#pragma unroll
+        for (int jj = 0; jj < ROWS; ++jj) {
+          const int64_t d = in.dst_row + g + j + jj;
+          if (act && j + jj < nrows) {
+            if (isk) dK[d * kw + w] = buf[jj];
+            else dV[d * vw + (w - kw)] = buf[jj];
+          }
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant__ FusedMaps maps, const StepArgs a) {
+  constexpr int NBP = 10;                       // block pairs (bi <= bj) of four 128-row blocks
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int EC = a.E / 64, NC = (a.E + a.D) / 64;
+  float* D = (float*)(smem + 4 * kChunk);       // packed upper triangle, row j at tri_offset(j)
+  __shared__ __align__(8) uint64_t bars[24];
+  uint64_t* full = bars;          // [2] ring stage landed
+  uint64_t* empty = bars + 2;     // [2] ring stage read by its MMAs (commit)
+  uint64_t* tfull = bars + 4;     // [2] accumulators ready (commit)
+  uint64_t* tempty = bars + 6;    // [2] accumulators read (128)
+  uint64_t* cmax = bars + 8;      // c exchanged among the epilogue threads (128)
+  uint64_t* drow = bars + 9;      // [4] Delta rows of row block b complete (128)
+  uint64_t* mdone = bars + 14;    // every MMA complete
+  uint64_t* vfull = bars + 15;    // the instance's V rows landed in the Delta area
+  __shared__ __align__(8) uint64_t thf[8];   // thresholds of pair block t published (32)
+  __shared__ __align__(8) uint64_t bitsb[8]; // decisions of pair block t published (32; blocks in order)
+  __shared__ float red[4];
+  __shared__ float thr_s[kH512Pairs];
+  __shared__ float alpha_s[kH512Pairs];
+  __shared__ uint32_t bits_s[8];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int inst = blockIdx.x;
+  const int m = a.m, n = a.n;
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(full + b, 1);
+      mbar_init(empty + b, 1);
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 128);
+    }
+    mbar_init(cmax, 128);
+    for (int b = 0; b < 4; ++b) mbar_init(drow + b, 128);
+    mbar_init(mdone, 1);
+    mbar_init(vfull, 1);
+    for (int t = 0; t < 8; ++t) {
+      mbar_init(thf + t, 32);
+      mbar_init(bitsb + t, 32);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_s, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort = &abort_s;
+  const HalveInst in = a.inst[inst];
+  const bool tokens = a.src_kind == SRC_TOKENS;
+  const int ks = a.sub_stride > 1 ? a.sub_stride : 1;
+  // block pair q -> (bi, bj), row-block order: (0,0) (0,1) (0,2) (0,3) (1,1) (1,2) (1,3) (2,2) (2,3) (3,3)
+  auto pair_of = [](int q, int& bi, int& bj) {
+    bi = q < 4 ? 0 : q < 7 ? 1 : q < 9 ? 2 : 3;
+    const int first = bi == 0 ? 0 : bi == 1 ? 4 : bi == 2 ? 7 : 9;
+    bj = bi + (q - first);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const int row = (int)(tokens ? in.src_row / ks + 2 * (int64_t)in.pair0 : in.src_row);
+      const int h = (int)(in.bh % (uint32_t)a.H);
+      // V rows of the four blocks into the Delta area (DC chunks of 128 rows x 64 columns per block)
+      const int DCn = NC - EC;
+      mbar_expect_tx(vfull, (uint32_t)(4 * DCn) * kChunk);
+      for (int blk = 0; blk < 4; ++blk)
+        for (int c = 0; c < DCn; ++c) {
+          uint8_t* dst = (uint8_t*)D + (blk * DCn + c) * kChunk;
+          if (!tokens) tma_load_2d(dst, &maps.v, vfull, c * 64, row + 128 * blk);
+          else if (ks > 1) tma_load_4d(dst, &maps.v, vfull, c * 64, h, 0, row + 128 * blk);
+          else tma_load_3d(dst, &maps.v, vfull, c * 64, h, row + 128 * blk);
+        }
+      int g = 0;
+      bool ok = true;
+      for (int q = 0; q < NBP && ok; ++q) {
+        int bi, bj;
+        pair_of(q, bi, bj);
+        for (int c = 0; c < NC; ++c, ++g) {
+          const int s = g & 1;
+          if (g >= 2 && !mbar_wait(empty + s, ((g >> 1) & 1) ^ 1, abort)) {
+            ok = false;
+            break;
+          }
+          const bool isk = c < EC;
+          const CUtensorMap* mp = isk ? &maps.k : &maps.v;
+          const int x = (isk ? c : c - EC) * 64;
+          mbar_expect_tx(full + s, (bi == bj ? 1u : 2u) * kChunk);
+          for (int side = 0; side < (bi == bj ? 1 : 2); ++side) {
+            uint8_t* dst = smem + s * 2 * kChunk + side * kChunk;
+            const int r0 = row + 128 * (side ? bj : bi);
+            if (!tokens) tma_load_2d(dst, mp, full + s, x, r0);
+            else if (ks > 1) tma_load_4d(dst, mp, full + s, x, h, 0, r0);
+            else tma_load_3d(dst, mp, full + s, x, h, r0);
+          }
+        }
+      }
+      // leave no copy in flight: the last fill of each stage has landed
+      for (int gg = max(0, g - 2); gg < g; ++gg) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(full + (gg & 1), (gg >> 1) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+      const long long t0 = clock64();
+      while (!mbar_try_wait(vfull, 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t I128 = idesc_bf16(128, 128, false);
+      const uint32_t base = smem_u32(smem);
+      int g = 0;
+      bool ok = true;
+      for (int q = 0; q < NBP && ok; ++q) {
+        int bi, bj;
+        pair_of(q, bi, bj);
+        const int tb = q & 1;
+        if (q >= 2 && !mbar_wait(tempty + tb, ((q >> 1) & 1) ^ 1, abort)) break;
+        for (int c = 0; c < NC; ++c, ++g) {
+          const int s = g & 1;
+          if (!mbar_wait(full + s, (g >> 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ra = base + s * 2 * kChunk;
+          const uint32_t rb = bi == bj ? ra : ra + kChunk;
+          const uint32_t dc = tmem + tb * 256u + (c < EC ? 0u : 128u);
+          const bool first = c == 0 || c == EC;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(dc, sw128_desc(ra + kk * 32, 16, 1024), sw128_desc(rb + kk * 32, 16, 1024), I128,
+                      (!first || kk > 0) ? 1u : 0u);
+          umma_commit(empty + s);
+        }
+        if (ok) umma_commit(tfull + tb);
+      }
+      umma_commit(mdone);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(mdone, 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else if (warp >= 2 && warp < 6) {
+    // ------------------------------------------------------------------ epilogue
+    const int q4 = warp & 3;                    // TMEM lane quarter of this warp
+    const int r = q4 * 32 + lane;               // row within a 128-row block = TMEM lane
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    // c = max |v| over the instance's rows, from the V rows staged in the Delta area (row R of
+    // block blk: 128 bytes per chunk, 16-byte units swizzled by R & 7)
+    bool ok = warp_wait(vfull, 0, abort);
+    float mx = 0.f;
+    if (ok) {
+      const int DCn = NC - EC;
+      for (int blk = 0; blk < 4; ++blk) {
+        if (128 * blk + r >= n) break;
+        for (int c = 0; c < DCn; ++c) {
+          const uint8_t* rowp = (const uint8_t*)D + (blk * DCn + c) * kChunk + r * 128;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint4 w = *(const uint4*)(rowp + ((q ^ (r & 7)) << 4));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              mx = fmax3(mx, fabsf(__uint_as_float(ws[e] << 16)), fabsf(__uint_as_float(ws[e] & 0xFFFF0000u)));
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[q4] = mx;
+    mbar_arrive(cmax);   // every epilogue thread has read its V rows: the area may take Delta now
+    if (ok) ok = warp_wait(cmax, 0, abort);
+    const float cm = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const float c2 = cm * cm;
+    for (int q = 0; q < NBP; ++q) {
+      int bi, bj;
+      pair_of(q, bi, bj);
+      const int tb = q & 1;
+      if (ok) ok = warp_wait(tfull + tb, (q >> 1) & 1, abort);
+      if (ok) {
+        tc_fence_after();
+        const int pj = bi * 64 + (r >> 1);
+        const bool writer = (r & 1) == 0;
+        // on a diagonal block the chunks left of this warp's 16 pair rows hold no upper-triangle entry
+#pragma unroll 1
+        for (int cc = (bi == bj ? q4 : 0); cc < 4; ++cc) {
+          float kk[32], vv[32];
+          tmem_ld32(tmem + lane_base + tb * 256u + cc * 32, kk);
+          tmem_ld32(tmem + lane_base + tb * 256u + 128 + cc * 32, vv);
+          tmem_ld_wait();
+          float dd[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float k0 = exp2f(kk[2 * i] * a.scale_log2e) * (vv[2 * i] + c2);
+            const float k1 = exp2f(kk[2 * i + 1] * a.scale_log2e) * (vv[2 * i + 1] + c2);
+            dd[i] = k0 - k1;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) dd[i] -= __shfl_xor_sync(0xffffffffu, dd[i], 1);
+          if (writer) {
+            float* Drow = D + tri_offset(pj) - pj;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int pi = bj * 64 + cc * 16 + i;
+              if (pi >= pj) Drow[pi] = (pj < m && pi < m) ? dd[i] : 0.f;
+            }
+          }
+        }
+        tc_fence_before();
+      }
+      mbar_arrive(tempty + tb);
+      if (bj == 3) mbar_arrive(drow + bi);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ sigma's recursion
+    const float C = a.C, rC = 1.f / C;
+    float sigma = 0.f;
+#pragma unroll 1
+    for (int t = 0; t < 8; ++t) {
+      if (!warp_wait(drow + (t >> 1), 0, abort)) break;
+      const int p = 32 * t + lane;
+      const float wl = p < m ? 1.f - 2.f * philox_uniform(a.seed, in.ctr_bh, in.round_id, in.pair0 + (uint32_t)p) : 0.f;
+      thr_s[p] = thresholds32(sigma, D[tri_offset(p)], wl, C, rC, lane);
+      __syncwarp();
+      mbar_arrive(thf + t);
+    }
+  } else {
+    // ------------------------------------------------------------------ the walk (warp 7)
+    // alpha of pair 32 t2 + lane lives in alpha_s (no register array indexed by block); each block's
+    // terms are added to every later pair's alpha in row order, as the walk kernels do
+    for (int i = lane; i < kH512Pairs; i += 32) alpha_s[i] = 0.f;
+    __syncwarp();
+    bool ok = true;
+#pragma unroll 1
+    for (int t = 0; t < 8; ++t) {
+      uint32_t bb = 0u;
+      if (ok) ok = warp_wait(thf + t, 0, abort);
+      if (ok) {
+        const int base = 32 * t;
+        float my = alpha_s[base + lane];
+        bb = walk_block32_th(my, thr_s[base + lane], m - base, lane,
+                             [&](int q) { return D[tri_offset(base + q) - (base + q) + base + lane]; });
+        // the later blocks' sums run side by side (seven independent chains, each in row order)
+        float acc[7];
+#pragma unroll
+        for (int j = 0; j < 7; ++j) acc[j] = t + 1 + j < 8 ? alpha_s[32 * (t + 1 + j) + lane] : 0.f;
+#pragma unroll 4
+        for (int q = 0; q < 32; ++q) {
+          const float* Dq = D + tri_offset(base + q) - (base + q) + lane;
+          const float sg = ((bb >> q) & 1u) ? 1.f : -1.f;
+#pragma unroll
+          for (int j = 0; j < 7; ++j)
+            if (t + 1 + j < 8) acc[j] = fmaf(sg, Dq[32 * (t + 1 + j)], acc[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 7; ++j)
+          if (t + 1 + j < 8) alpha_s[32 * (t + 1 + j) + lane] = acc[j];
+      }
+      if (lane == 0) bits_s[t] = bb;
+      __syncwarp();
+      mbar_arrive(bitsb + t);
+    }
+  }
+  // ------------------------------------------------------------------ gather (all warps)
+  __syncwarp();
+  if (warp_wait(bitsb + 7, 0, abort)) {
+    auto bit = [&](int i) { return ((bits_s[i >> 5] >> (i & 31)) & 1u) != 0; };
+    const int per = (m + 7) / 8;
+    gather_global<8>(a, in, min(m, warp * per), min(m, (warp + 1) * per), bit, lane);
+    if (a.trace && warp == 0) {
+      const int nb = a.m_pad >> 5;
+      if (lane < nb) a.trace[a.trace_base + (size_t)inst * nb + lane] = bits_s[lane];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_s && threadIdx.x == 0 && a.status) {
+    if (atomicCAS(a.status, 0, 6) == 0) a.status[1] = inst;
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_512(const StepArgs& a, cudaStream_t st) {
+  FusedMaps maps;
+  bool ok;
+  if (a.src_kind == SRC_TOKENS && a.sub_stride > 1) {
+    ok = make_map_4d_strided(&maps.k, a.srcK, a.src_rows, a.H, a.E, a.sub_stride, 128) &&
+         make_map_4d_strided(&maps.v, a.srcV, a.src_rows, a.H, a.D, a.sub_stride, 128);
+  } else if (a.src_kind == SRC_TOKENS) {
+    ok = make_map_3d(&maps.k, a.srcK, a.src_rows, a.H, a.E, 128) && make_map_3d(&maps.v, a.srcV, a.src_rows, a.H, a.D, 128);
+  } else {
+    ok = make_map_2d(&maps.k, a.srcK, a.src_rows, a.E, a.E, 128) && make_map_2d(&maps.v, a.srcV, a.src_rows, a.D, a.D, 128);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  const size_t delta_bytes = (size_t)(kH512Pairs * (kH512Pairs + 1) / 2) * 4;
+  if ((size_t)4 * (a.D / 64) * kChunk > delta_bytes) return cudaErrorInvalidValue;   // V staging must fit
+  const size_t sm = 1024 + 4 * (size_t)kChunk + delta_bytes;
+  cudaError_t e = cudaFuncSetAttribute(halve512_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  halve512_kernel<<<a.n_inst, 256, sm, st>>>(maps, a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_256(const StepArgs& a, cudaStream_t st) {
   FusedMaps maps;
   bool ok;
@@ -753,8 +1132,11 @@ cudaError_t launch_256(const StepArgs& a, cudaStream_t st) {
 
 bool halving_fused_supported(const StepArgs& a) {
   if (std::getenv("THIN_ATTN_UNFUSED_HALVING") != nullptr) return false;
-  if (a.E % 64 || a.D % 64 || (a.E + a.D) / 64 > kMaxChunks || a.n < 2 || a.n > 256 || a.n % 2) return false;
+  if (a.E % 64 || a.D % 64 || (a.E + a.D) / 64 > kMaxChunks || a.n < 2 || a.n > 512 || a.n % 2) return false;
   if (a.src_rows <= 0 || !tensor_maps_available()) return false;
+  // 257..512 points: the V rows (4 blocks x D/64 chunks of 16 KB) are staged in the 131.6 KB Delta
+  // area for c, so D <= 128
+  if (a.n > 256 && a.D > 128) return false;
   // subsampled rows form boxes only as a strided view (integer ratio, runs on multiples of it)
   if (a.src_kind == SRC_TOKENS && a.S_sub < a.S_full && a.sub_stride < 2) return false;
   return true;
@@ -765,7 +1147,8 @@ cudaError_t launch_halving_fused(const StepArgs& a, cudaStream_t st) {
   if (a.n <= 32) return launch_np<32>(a, st);
   if (a.n <= 64) return launch_np<64>(a, st);
   if (a.n <= 128) return launch_np<128>(a, st);
-  return launch_256(a, st);
+  if (a.n <= 256) return launch_256(a, st);
+  return launch_512(a, st);
 }
 
 }  // namespace thin
