@@ -108,6 +108,8 @@ def test_full_workload_sampled_rows(name):
     (1, 1, 40, 64, 64, 64, 3, "fp32"),       # S <= 4^g: coreset = all keys, exact attention
     (2, 2, 300, 513, 128, 128, 1, "fp32"),   # odd S, fp32
     (1, 1, 1, 4096, 64, 64, 2, "bf16"),      # a single query
+    (1, 2, 64, 2000, 128, 128, 2, "bf16"),   # last level 224 points: partial second 128-row block
+    (1, 2, 64, 3000, 256, 64, 2, "bf16"),    # last level 352 points (257..512), E = 256, D = 64
 ])
 def test_noncausal_edge_cases(B, H, T, S, E, D, g, dtype):
     w = W.Workload("edge", B, H, T, S, E, D, dtype, False, g, 11, 5, "iid")
@@ -208,16 +210,21 @@ def test_dropin_call_returns_output_and_none():
     assert weights is None and out.shape == (1, 256, 1, 64)
 
 
-@pytest.mark.parametrize("causal", [True, False])
-def test_fused_and_three_launch_halving_agree(causal, monkeypatch):
-    """The one-launch small-instance halving kernel and the c^2 / Gram / walk launches take the same
-    decisions (same arithmetic), so traces, coresets, outputs and LSE are bit-identical."""
+@pytest.mark.parametrize("case", ["causal", "noncausal", "ragged224", "ragged352"])
+def test_fused_and_three_launch_halving_agree(case, monkeypatch):
+    """The one-launch halving kernels (up to 512 points) and the c^2 / Gram / walk launches take the
+    same decisions (same arithmetic), so traces, coresets, outputs and LSE are bit-identical."""
+    causal = case == "causal"
     if causal:
         w = W.WORKLOADS["express32k"].with_(T=8192, H=4)
         S = w.T
-    else:
+    elif case == "noncausal":
         w = W.WORKLOADS["express32k"].with_(T=512, H=2, B=2, causal=False, S=1024)
         S = 1024
+    else:
+        S = 2000 if case == "ragged224" else 3000
+        w = W.WORKLOADS["express32k"].with_(T=256, H=3, B=1, causal=False, S=S, E=128 if S == 2000 else 256,
+                                            D=128 if S == 2000 else 64)
     q, k, v = (x.cuda() for x in W.make_qkv(w, T=w.T, S=S))
     res = []
     for unfused in (False, True):
