@@ -267,8 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
       const int pj = lr >> 1;
       const bool writer = (lr & 1) == 0;
       const uint32_t kcol = tmem + lane_base + (uint32_t)b * 256u + (uint32_t)(ii * NP);
+      // the walk reads Delta[j][i] for j <= i only: a chunk of columns left of this warp's 16 pair
+      // rows (of its instance) holds none of those and is skipped
 #pragma unroll 1
-      for (int cc = 0; cc < NP / 32; ++cc) {
+      for (int cc = ew % (NP / 32); cc < NP / 32; ++cc) {
         float kk[32], vv[32];
         tmem_ld32(kcol + cc * 32, kk);
         tmem_ld32(kcol + 128 + cc * 32, vv);
@@ -599,8 +601,9 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
       tc_fence_after();
       const int pj = r >> 1;
       const bool writer = (r & 1) == 0;
+      // chunks of columns left of this warp's 16 pair rows hold no entry the walk reads (j <= i)
 #pragma unroll 1
-      for (int cc = 0; cc < 8; ++cc) {
+      for (int cc = q4; cc < 8; ++cc) {
         float kk[32], vv[32];
         tmem_ld32(tmem + lane_base + cc * 32, kk);
         tmem_ld32(tmem + lane_base + 256 + cc * 32, vv);
@@ -633,7 +636,7 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
       const int pj = 64 + (r >> 1);
       const bool writer = (r & 1) == 0;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = q4; cc < 4; ++cc) {
         float kk[32], vv[32];
         tmem_ld32(tmem + lane_base + cc * 32, kk);
         tmem_ld32(tmem + lane_base + 256 + cc * 32, vv);
