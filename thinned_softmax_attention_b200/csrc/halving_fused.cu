@@ -1,9 +1,14 @@
-// Kernel Halving of small instances (n <= 128 points) in one persistent kernel.
+// Kernel Halving steps of up to 512 points per instance in one launch each.
 //
 // The three-launch step of halving.cu (c^2, pair-difference Gram, walk + gather) reads every
-// point from HBM three times and round-trips the pair-difference matrix through HBM.  For the
-// small instances that dominate the Express batch thinning (groups of 32..128 points) this kernel
-// does the whole step in one pass over the points:
+// point from HBM three times and round-trips the pair-difference matrix through HBM.  This file
+// does a whole step in one pass over the points, in three kernels:
+//   halve_fused_kernel<NP>  instances of <= 128 points (the bulk of the Express batch thinning),
+//                           persistent, units of 128 rows -- described below;
+//   halve256_kernel         129..256 points, one CTA per instance (further down);
+//   halve512_kernel         257..512 points with D <= 128, one CTA per instance, the pair
+//                           differences as a packed upper triangle (further down).
+// The persistent kernel's steps per unit:
 //
 //   TMA      a unit of 128 point rows lands in one pipeline stage as (E+D)/64 chunks of
 //            128 rows x 64 bf16 (128-byte swizzle); a unit is 4 instances of <= 32 points
