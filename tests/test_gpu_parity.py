@@ -210,6 +210,29 @@ def test_dropin_call_returns_output_and_none():
     assert weights is None and out.shape == (1, 256, 1, 64)
 
 
+@pytest.mark.parametrize("name,mode", [("express", 1), ("express_a", 2), ("vit", 0)])
+def test_pipelined_host_path_equals_device_path(name, mode):
+    """Inputs of 64 MB and more go through the host path in four shards (heads, or batch rows when H
+    does not divide), copies overlapping the other shards' compute; outputs and LSE equal the
+    device-resident forward's bit for bit."""
+    w = {"express": W.WORKLOADS["express32k"].with_(T=16384, H=8),
+         "express_a": W.WORKLOADS["express32k_a"].with_(T=16384, H=8),
+         "vit": W.WORKLOADS["vit"].with_(B=64)}[name]
+    S = w.T if w.causal else w.S
+    q, k, v = W.make_qkv(w)
+    assert (q.numel() + k.numel() + v.numel()) * 2 >= 64 << 20
+    h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
+    dev = h.forward(q.cuda(), k.cuda(), v.cuda(), causal=mode, g=w.g, seed=w.seed, return_lse=True)
+    torch.cuda.synchronize()
+    out = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype).pin_memory()
+    lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32).pin_memory()
+    for _ in range(2):   # the second call reuses the shards, streams and staging
+        out.zero_()
+        h.forward_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), out, causal=mode, g=w.g, seed=w.seed, lse=lse)
+        assert torch.equal(out, dev["out"].cpu())
+        assert torch.equal(lse, dev["lse"].cpu())
+
+
 @pytest.mark.parametrize("case", ["causal", "noncausal", "ragged224", "ragged352"])
 def test_fused_and_three_launch_halving_agree(case, monkeypatch):
     """The one-launch halving kernels (up to 512 points) and the c^2 / Gram / walk launches take the

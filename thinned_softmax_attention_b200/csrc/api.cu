@@ -187,6 +187,12 @@ struct thin_attn_s {
   // host-buffer staging
   void* st_mem = nullptr;
   size_t st_bytes = 0;
+  // pipelined host path: one handle per group of heads (or batch rows), copy-in / compute / copy-out
+  // streams and their events (one set per group)
+  std::vector<thin_attn_s*> hp_sub;
+  bool hp_by_heads = true;
+  cudaStream_t hp_in = nullptr, hp_comp = nullptr, hp_out = nullptr;
+  std::vector<cudaEvent_t> hp_ev;   // [3 * groups + 1]: in_done, comp_done, out_done per group; start
   // side stream of the attention waves and its fork/join events
   cudaStream_t side = nullptr, main = nullptr;
   cudaEvent_t ev_join = nullptr, ev_join2 = nullptr, ev_fork = nullptr;
@@ -990,6 +996,10 @@ thin_attn_status thin_attn_destroy(thin_attn_t h) {
     if (e) cudaEventDestroy(e);
   if (h->side) cudaStreamDestroy(h->side);
   if (h->main) cudaStreamDestroy(h->main);
+  for (auto sub : h->hp_sub) thin_attn_destroy(sub);
+  for (auto e : h->hp_ev) cudaEventDestroy(e);
+  for (auto st : {h->hp_in, h->hp_comp, h->hp_out})
+    if (st) cudaStreamDestroy(st);
   delete h;
   return THIN_ATTN_OK;
 }
@@ -1058,6 +1068,48 @@ thin_attn_status thin_attn_forward(thin_attn_t h, const void* q, const void* k, 
   return run_forward(h, p, q, k, v, out, seed, lse_opt, coreset_idx_opt, trace_opt, (cudaStream_t)stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+constexpr int kHostGroups = 4;                  // groups of the pipelined host path
+constexpr size_t kHostPipelineMin = 64u << 20;  // input bytes from which it pipelines
+
+// Set up the pipelined host path once: kHostGroups handles, each a shard (b0, h0, H_total) of this
+// handle's problem -- whole heads when H divides, else whole batch rows -- so their random streams,
+// and so every output, are this handle's; three non-blocking streams and their events.
+thin_attn_status host_pipeline_setup(thin_attn_s* h) {
+  if (!h->hp_sub.empty()) return THIN_ATTN_OK;
+  const thin_attn_config& c = h->cfg;
+  h->hp_by_heads = c.H % kHostGroups == 0;
+  const int Ht = c.H_total > 0 ? c.H_total : c.H;
+  for (int gi = 0; gi < kHostGroups; ++gi) {
+    thin_attn_config sc = c;
+    if (h->hp_by_heads) {
+      sc.H = c.H / kHostGroups;
+      sc.h0 = c.h0 + gi * sc.H;
+      sc.H_total = Ht;
+    } else {
+      sc.B = c.B / kHostGroups;
+      sc.b0 = c.b0 + gi * sc.B;
+      sc.H_total = Ht;
+    }
+    thin_attn_t sub = nullptr;
+    thin_attn_status s = thin_attn_create(&sub, &sc);
+    if (s != THIN_ATTN_OK) return s;
+    h->hp_sub.push_back(sub);
+  }
+  DeviceGuard dg(c.device);
+  for (cudaStream_t* st : {&h->hp_in, &h->hp_comp, &h->hp_out}) CK(cudaStreamCreateWithFlags(st, cudaStreamNonBlocking));
+  h->hp_ev.resize(3 * kHostGroups + 1);
+  for (auto& e : h->hp_ev) CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  return THIN_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void* k, const void* v, void* out,
                                         int causal, int g, uint64_t seed, float* lse_opt, void* stream) {
   if (!h) return fail(THIN_ATTN_EINVAL, "null handle");
@@ -1068,8 +1120,14 @@ thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void
   const size_t qb = (size_t)c.B * c.T * c.H * c.E * es, kb = (size_t)c.B * L * c.H * c.E * es,
                vb = (size_t)c.B * L * c.H * c.D * es, ob = (size_t)c.B * c.T * c.H * c.D * es,
                lb = (size_t)c.B * c.H * c.T * 4;
-  const size_t need = align256(qb) + align256(kb) + align256(vb) + align256(ob) + align256(lb);
   cudaStream_t st = (cudaStream_t)stream;
+  // Large problems run as kHostGroups shards in a pipeline: the copy-in of group i+1 and the
+  // copy-out of group i-1 overlap the compute of group i (double-buffered staging).
+  const bool pipeline = qb + kb + vb >= kHostPipelineMin && (c.H % kHostGroups == 0 || c.B % kHostGroups == 0);
+  const int NG = pipeline ? kHostGroups : 1;
+  const size_t gq = qb / NG, gk = kb / NG, gv = vb / NG, go = ob / NG, gl = lb / NG;
+  const size_t slot = align256(gq) + align256(gk) + align256(gv) + align256(go) + align256(gl);
+  const size_t need = (pipeline ? 2 : 1) * slot;
   {
     std::lock_guard<std::mutex> lk(h->mu);
     DeviceGuard dg(c.device);
@@ -1083,23 +1141,90 @@ thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void
       }
       h->st_bytes = need;
     }
+    if (pipeline) {
+      thin_attn_status s = host_pipeline_setup(h);
+      if (s != THIN_ATTN_OK) return s;
+    }
   }
-  char* base = (char*)h->st_mem;
-  char *dq = base, *dk = dq + align256(qb), *dv = dk + align256(kb), *dout = dv + align256(vb),
-       *dl = dout + align256(ob);
-  {
-    DeviceGuard dg(c.device);
+  auto slot_ptrs = [&](int sl, char** dq, char** dk, char** dv, char** dout, char** dl) {
+    char* base = (char*)h->st_mem + sl * slot;
+    *dq = base;
+    *dk = *dq + align256(gq);
+    *dv = *dk + align256(gk);
+    *dout = *dv + align256(gv);
+    *dl = *dout + align256(go);
+  };
+  DeviceGuard dg(c.device);
+  if (!pipeline) {
+    char *dq, *dk, *dv, *dout, *dl;
+    slot_ptrs(0, &dq, &dk, &dv, &dout, &dl);
     CK(cudaMemcpyAsync(dq, q, qb, cudaMemcpyHostToDevice, st));
     CK(cudaMemcpyAsync(dk, k, kb, cudaMemcpyHostToDevice, st));
     CK(cudaMemcpyAsync(dv, v, vb, cudaMemcpyHostToDevice, st));
+    thin_attn_status s = thin_attn_forward(h, dq, dk, dv, dout, causal, g, seed, lse_opt ? (float*)dl : nullptr,
+                                           nullptr, nullptr, stream);
+    if (s != THIN_ATTN_OK) return s;
+    CK(cudaMemcpyAsync(out, dout, ob, cudaMemcpyDeviceToHost, st));
+    if (lse_opt) CK(cudaMemcpyAsync(lse_opt, dl, lb, cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
+    return THIN_ATTN_OK;
   }
-  thin_attn_status s = thin_attn_forward(h, dq, dk, dv, dout, causal, g, seed, lse_opt ? (float*)dl : nullptr,
-                                         nullptr, nullptr, stream);
-  if (s != THIN_ATTN_OK) return s;
-  DeviceGuard dg(c.device);
-  CK(cudaMemcpyAsync(out, dout, ob, cudaMemcpyDeviceToHost, st));
-  if (lse_opt) CK(cudaMemcpyAsync(lse_opt, dl, lb, cudaMemcpyDeviceToHost, st));
+  // group gi: heads [gi G, (gi+1) G) of every (b, t) row -- a 2-D copy with the row pitch of the
+  // whole tensor -- or batch rows [gi B', (gi+1) B') -- a contiguous range
+  const int Gh = c.H / NG, Gb = c.B / NG;
+  auto copy = [&](void* dst, const void* src, size_t row_elems, int64_t rows, int gi, bool to_dev, cudaStream_t s2) {
+    const size_t full = row_elems * es;   // bytes of one (b, t) row of the whole tensor
+    if (h->hp_by_heads) {
+      const size_t w = full / NG, off = (size_t)gi * w;
+      return to_dev ? cudaMemcpy2DAsync(dst, w, (const char*)src + off, full, w, rows, cudaMemcpyHostToDevice, s2)
+                    : cudaMemcpy2DAsync((char*)dst + off, full, src, w, w, rows, cudaMemcpyDeviceToHost, s2);
+    }
+    const size_t bytes = full * rows / NG, off = (size_t)gi * bytes;
+    return to_dev ? cudaMemcpyAsync(dst, (const char*)src + off, bytes, cudaMemcpyHostToDevice, s2)
+                  : cudaMemcpyAsync((char*)dst + off, src, bytes, cudaMemcpyDeviceToHost, s2);
+  };
+  cudaEvent_t* ev = h->hp_ev.data();
+  cudaEvent_t ev_start = ev[3 * NG];
+  CK(cudaEventRecord(ev_start, st));
+  for (cudaStream_t s2 : {h->hp_in, h->hp_comp, h->hp_out}) CK(cudaStreamWaitEvent(s2, ev_start, 0));
+  for (int gi = 0; gi < NG; ++gi) {
+    char *dq, *dk, *dv, *dout, *dl;
+    slot_ptrs(gi & 1, &dq, &dk, &dv, &dout, &dl);
+    cudaEvent_t in_done = ev[3 * gi], comp_done = ev[3 * gi + 1], out_done = ev[3 * gi + 2];
+    // the slot's inputs are free once group gi-2 has computed
+    if (gi >= 2) CK(cudaStreamWaitEvent(h->hp_in, ev[3 * (gi - 2) + 1], 0));
+    const int64_t rows_q = (int64_t)c.B * c.T;
+    const int64_t rows_kv = (int64_t)c.B * L;
+    CK(copy(dq, q, (size_t)c.H * c.E, rows_q, gi, true, h->hp_in));
+    CK(copy(dk, k, (size_t)c.H * c.E, rows_kv, gi, true, h->hp_in));
+    CK(copy(dv, v, (size_t)c.H * c.D, rows_kv, gi, true, h->hp_in));
+    CK(cudaEventRecord(in_done, h->hp_in));
+    // compute once the inputs are in and the slot's outputs of group gi-2 are out
+    CK(cudaStreamWaitEvent(h->hp_comp, in_done, 0));
+    if (gi >= 2) CK(cudaStreamWaitEvent(h->hp_comp, ev[3 * (gi - 2) + 2], 0));
+    thin_attn_status s = thin_attn_forward(h->hp_sub[gi], dq, dk, dv, dout, causal, g, seed,
+                                           lse_opt ? (float*)dl : nullptr, nullptr, nullptr, h->hp_comp);
+    if (s != THIN_ATTN_OK) return s;
+    CK(cudaEventRecord(comp_done, h->hp_comp));
+    CK(cudaStreamWaitEvent(h->hp_out, comp_done, 0));
+    CK(copy(out, dout, (size_t)c.H * c.D, (int64_t)c.B * c.T, gi, false, h->hp_out));
+    if (lse_opt) {
+      // lse (B, H, T): group gi holds heads [gi G, (gi+1) G) of every b, or batch rows of it
+      if (h->hp_by_heads)
+        CK(cudaMemcpy2DAsync(lse_opt + (size_t)gi * Gh * c.T, (size_t)c.H * c.T * 4, dl, (size_t)Gh * c.T * 4,
+                             (size_t)Gh * c.T * 4, c.B, cudaMemcpyDeviceToHost, h->hp_out));
+      else
+        CK(cudaMemcpyAsync(lse_opt + (size_t)gi * Gb * c.H * c.T, dl, gl, cudaMemcpyDeviceToHost, h->hp_out));
+    }
+    CK(cudaEventRecord(out_done, h->hp_out));
+  }
+  CK(cudaStreamWaitEvent(st, ev[3 * (NG - 1) + 2], 0));
   CK(cudaStreamSynchronize(st));
+  // a bounded wait that gave up in a group's kernels is reported here, like thin_attn_check would
+  for (auto sub : h->hp_sub) {
+    thin_attn_status s = thin_attn_check(sub, st);
+    if (s != THIN_ATTN_OK) return s;
+  }
   return THIN_ATTN_OK;
 }
 
