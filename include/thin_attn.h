@@ -152,8 +152,9 @@ THIN_ATTN_API thin_attn_status thin_attn_forward(thin_attn_t h, const void* q, c
  * handle, runs the forward, copies out (and lse when lse_opt is not NULL) back,
  * and synchronises `stream`.  Page-locked host buffers give asynchronous
  * copies; pageable ones work too.  When q, k and v hold 64 MB or more and H (or
- * else B) is a multiple of 4, the problem runs as four shards of its heads (or
- * batch rows), each a handle with this one's random stream (config b0/h0/H_total),
+ * else B) is a multiple of 4, the problem runs as eight (H or B a multiple of 8) or
+ * four shards of its heads (or batch rows), each a handle with this one's random
+ * stream (config b0/h0/H_total),
  * in a pipeline on internal streams ordered after `stream`: the copy-in of one
  * shard and the copy-out of another overlap the compute of a third.  Results
  * are those of one thin_attn_forward of the whole problem, bit for bit.

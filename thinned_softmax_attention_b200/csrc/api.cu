@@ -191,6 +191,7 @@ struct thin_attn_s {
   // streams and their events (one set per group)
   std::vector<thin_attn_s*> hp_sub;
   bool hp_by_heads = true;
+  int hp_groups = 0;
   cudaStream_t hp_in = nullptr, hp_comp = nullptr, hp_out = nullptr;
   std::vector<cudaEvent_t> hp_ev;   // [3 * groups + 1]: in_done, comp_done, out_done per group; start
   // side stream of the attention waves and its fork/join events
@@ -1072,25 +1073,44 @@ thin_attn_status thin_attn_forward(thin_attn_t h, const void* q, const void* k, 
 
 namespace {
 
-constexpr int kHostGroups = 4;                  // groups of the pipelined host path
-constexpr size_t kHostPipelineMin = 64u << 20;  // input bytes from which it pipelines
+constexpr size_t kHostPipelineMin = 64u << 20;  // input bytes from which the host path pipelines
 
-// Set up the pipelined host path once: kHostGroups handles, each a shard (b0, h0, H_total) of this
-// handle's problem -- whole heads when H divides, else whole batch rows -- so their random streams,
-// and so every output, are this handle's; three non-blocking streams and their events.
+// Shards of the pipelined host path: 8 or 4 groups of heads, else of batch rows (0: no pipeline).
+// The copy-in bounds the pipeline; more shards shorten the tail (the last shard's compute and
+// copy-out).
+void host_groups(const thin_attn_config& c, int* groups, bool* by_heads) {
+  *groups = 0;
+  *by_heads = true;
+  for (int ng : {8, 4})
+    if (c.H % ng == 0) {
+      *groups = ng;
+      return;
+    }
+  *by_heads = false;
+  for (int ng : {8, 4})
+    if (c.B % ng == 0) {
+      *groups = ng;
+      return;
+    }
+}
+
+// Set up the pipelined host path once: one handle per group, each a shard (b0, h0, H_total) of this
+// handle's problem, so their random streams, and so every output, are this handle's; three
+// non-blocking streams and their events.
 thin_attn_status host_pipeline_setup(thin_attn_s* h) {
   if (!h->hp_sub.empty()) return THIN_ATTN_OK;
   const thin_attn_config& c = h->cfg;
-  h->hp_by_heads = c.H % kHostGroups == 0;
+  host_groups(c, &h->hp_groups, &h->hp_by_heads);
+  const int NG = h->hp_groups;
   const int Ht = c.H_total > 0 ? c.H_total : c.H;
-  for (int gi = 0; gi < kHostGroups; ++gi) {
+  for (int gi = 0; gi < NG; ++gi) {
     thin_attn_config sc = c;
     if (h->hp_by_heads) {
-      sc.H = c.H / kHostGroups;
+      sc.H = c.H / NG;
       sc.h0 = c.h0 + gi * sc.H;
       sc.H_total = Ht;
     } else {
-      sc.B = c.B / kHostGroups;
+      sc.B = c.B / NG;
       sc.b0 = c.b0 + gi * sc.B;
       sc.H_total = Ht;
     }
@@ -1101,7 +1121,7 @@ thin_attn_status host_pipeline_setup(thin_attn_s* h) {
   }
   DeviceGuard dg(c.device);
   for (cudaStream_t* st : {&h->hp_in, &h->hp_comp, &h->hp_out}) CK(cudaStreamCreateWithFlags(st, cudaStreamNonBlocking));
-  h->hp_ev.resize(3 * kHostGroups + 1);
+  h->hp_ev.resize(3 * NG + 1);
   for (auto& e : h->hp_ev) CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
   return THIN_ATTN_OK;
 }
@@ -1121,10 +1141,13 @@ thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void
                vb = (size_t)c.B * L * c.H * c.D * es, ob = (size_t)c.B * c.T * c.H * c.D * es,
                lb = (size_t)c.B * c.H * c.T * 4;
   cudaStream_t st = (cudaStream_t)stream;
-  // Large problems run as kHostGroups shards in a pipeline: the copy-in of group i+1 and the
-  // copy-out of group i-1 overlap the compute of group i (double-buffered staging).
-  const bool pipeline = qb + kb + vb >= kHostPipelineMin && (c.H % kHostGroups == 0 || c.B % kHostGroups == 0);
-  const int NG = pipeline ? kHostGroups : 1;
+  // Large problems run as shards in a pipeline: the copy-in of group i+1 and the copy-out of group
+  // i-1 overlap the compute of group i (double-buffered staging).
+  int groups;
+  bool by_heads;
+  host_groups(c, &groups, &by_heads);
+  const bool pipeline = qb + kb + vb >= kHostPipelineMin && groups > 0;
+  const int NG = pipeline ? groups : 1;
   const size_t gq = qb / NG, gk = kb / NG, gv = vb / NG, go = ob / NG, gl = lb / NG;
   const size_t slot = align256(gq) + align256(gk) + align256(gv) + align256(go) + align256(gl);
   const size_t need = (pipeline ? 2 : 1) * slot;
