@@ -68,13 +68,20 @@ struct FusedShape {
 template <typename Bit>
 __device__ __forceinline__ void gather_from_stage(const StepArgs& a, int64_t dst_row, int64_t src_row, uint32_t tok_base,
                                                   const uint8_t* st, int row0, int i0, int i1, Bit bit, int lane,
-                                                  int EC, int NC, uint32_t chunk_bytes = kChunk) {
-  // token index of point p of the instance: tok_base + p k (k = subsample stride, 1 without subsample)
+                                                  int EC, int NC, uint32_t chunk_bytes = kChunk, uint32_t gap_u = 0,
+                                                  uint32_t gp0 = 0) {
+  // token index of point p of the instance: tok_base + p k (k = subsample stride, 1 without
+  // subsample); for a subsample of another ratio tok_base + floor(((gp0 + p) S + U) / S') with
+  // gp0 = 2 pair0 and U = gap_u, the subsample's own formula
   const bool tokens = a.src_kind == SRC_TOKENS;
+  const bool gapped = tokens && a.S_sub < a.S_full && a.sub_stride < 2;
   const uint32_t k = a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u;
   for (int i = i0 + lane; i < i1; i += 32) {
     const int p = 2 * i + (bit(i) ? 0 : 1);
-    a.dstIdx[dst_row + i] = tokens ? (int32_t)(tok_base + (uint32_t)p * k) : a.srcIdx[src_row + p];
+    a.dstIdx[dst_row + i] =
+        !tokens ? a.srcIdx[src_row + p]
+                : gapped ? (int32_t)(tok_base + (uint32_t)(((uint64_t)(gp0 + p) * (uint64_t)a.S_full + gap_u) / (uint64_t)a.S_sub))
+                         : (int32_t)(tok_base + (uint32_t)p * k);
   }
   const int units = NC * 8, kw = a.E / 8, vw = a.D / 8;
   uint4* dK = (uint4*)a.dstK;
@@ -122,6 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
   uint64_t* cmax = bars + 16;       // partial max |v| exchanged among the epilogue threads
   uint64_t* mdone = bars + 17;      // every MMA of this CTA complete
   uint64_t* thf = bars + 18;        // [2] thresholds of one block of 32 pairs published (32 lanes)
+  uint64_t* fixed = bars + 20;      // [3] stage compacted (subsample of a non-integer ratio; 128 threads)
+  uint64_t* cfix = bars + 23;       // the compaction's loads of one chunk done / its stores done (128)
   __shared__ float red[2][4];
   __shared__ uint32_t bits_s[2][2];
   __shared__ float thr_s[2][64];
@@ -134,7 +143,9 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
     for (int s = 0; s < nst; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 64);
+      mbar_init(fixed + s, 128);
     }
+    mbar_init(cfix, 128);
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
       mbar_init(tempty + b, 128);
@@ -154,6 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
   const uint32_t tmem = tmem_base_s;
   volatile int* abort = &abort_s;
   const int n_local = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  // token runs subsampled with a non-integer ratio: an instance's n points are n of the tokens
+  // [t(2 pair0), t(2 pair0 + n - 1)] (t = the subsample's index formula), at most NP of them, so
+  // the box of NP rows from the first holds them all; the epilogue warps move the selected rows
+  // up to rows 0..n-1 before the MMAs read the stage
+  const bool gapped = a.src_kind == SRC_TOKENS && a.S_sub < a.S_full && a.sub_stride < 2;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -168,8 +184,13 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
       if (lane < ni) {
         const HalveInst in = a.inst[i0 + lane];
         // token runs: first row of the instance, in units of the subsample stride k for strided runs
-        row = (int)(tokens ? (a.sub_stride > 1 ? in.src_row / a.sub_stride : in.src_row) + 2 * (int64_t)in.pair0
-                           : in.src_row);
+        if (gapped) {
+          const uint32_t U = sub_offset(a, in);
+          row = (int)(in.src_row + (int64_t)(((uint64_t)(2 * in.pair0) * (uint64_t)a.S_full + U) / (uint64_t)a.S_sub));
+        } else {
+          row = (int)(tokens ? (a.sub_stride > 1 ? in.src_row / a.sub_stride : in.src_row) + 2 * (int64_t)in.pair0
+                             : in.src_row);
+        }
         h = (int)(in.bh % (uint32_t)a.H);
       }
       if (!warp_wait(empty + s, ((k / nst) & 1) ^ 1, abort)) break;
@@ -203,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
       const uint32_t base = smem_u32(smem);
       for (int k = 0; k < n_local; ++k) {
         const int s = k % nst, b = k & 1;
-        if (!mbar_wait(full + s, (k / nst) & 1, abort)) break;
+        if (!mbar_wait((gapped ? fixed : full) + s, (k / nst) & 1, abort)) break;
         if (!mbar_wait(tempty + b, ((k >> 1) & 1) ^ 1, abort)) break;
         tc_fence_after();
         const uint32_t st = base + s * stage_bytes;
@@ -235,11 +256,54 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
     const int ii = r / NP, lr = r % NP;      // instance within the unit, row within the instance
     const uint32_t lane_base = (uint32_t)(ew * 32) << 16;
     const int m = a.m;
+    int cfix_uses = 0;   // completions of cfix so far (its parity)
     for (int k = 0; k < n_local; ++k) {
       const int s = k % nst, b = k & 1;
       const int u = blockIdx.x + k * gridDim.x;
       const bool live = u * Sh::IPU + ii < a.n_inst;
       if (!warp_wait(full + s, (k / nst) & 1, abort)) break;
+      if (gapped) {
+        // move the selected rows of each instance to rows 0..n-1 of its slot: thread item j is
+        // unit row R = t/8 + 16 j (instance R / NP, point p = R % NP) and 16-byte unit x = t % 8;
+        // all loads of a chunk, then all stores (a bounded wait on cfix between)
+        const int t = ew * 32 + lane, x = t & 7;
+        int srow[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int R = (t >> 3) + 16 * j, ii = R / NP, p = R % NP;
+          srow[j] = R;
+          const int inst = u * Sh::IPU + ii;
+          if (p < a.n && inst < a.n_inst) {
+            const HalveInst gi = a.inst[inst];
+            const uint32_t U = sub_offset(a, gi);
+            const uint64_t g0 = 2ull * gi.pair0;
+            const int64_t t0 = (int64_t)((g0 * (uint64_t)a.S_full + U) / (uint64_t)a.S_sub);
+            const int64_t tp = (int64_t)(((g0 + p) * (uint64_t)a.S_full + U) / (uint64_t)a.S_sub);
+            srow[j] = ii * NP + (int)(tp - t0);
+          }
+        }
+        uint8_t* stg = smem + s * stage_bytes;
+        bool fok = true;
+        for (int c = 0; c < NC && fok; ++c) {
+          uint8_t* ch = stg + c * kChunk;
+          uint4 buf[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) buf[j] = *(const uint4*)(ch + srow[j] * 128 + ((x ^ (srow[j] & 7)) << 4));
+          mbar_arrive(cfix);
+          fok = warp_wait(cfix, cfix_uses++ & 1, abort);
+          if (!fok) break;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int R = (t >> 3) + 16 * j;
+            if (srow[j] != R) *(uint4*)(ch + R * 128 + ((x ^ (R & 7)) << 4)) = buf[j];
+          }
+          mbar_arrive(cfix);
+          fok = warp_wait(cfix, cfix_uses++ & 1, abort);
+        }
+        if (!fok) break;
+        fence_proxy_async_smem();   // the MMAs read the stage through the async proxy
+        mbar_arrive(fixed + s);
+      }
       // c = max |v| over the instance: this row's part, then across the instance's threads
       float mx = 0.f;
       if (live && lr < a.n) {
@@ -339,11 +403,14 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
           const uint32_t kbg = __shfl_sync(0xffffffffu, kb, src);
           const int64_t dst_row = __shfl_sync(0xffffffffu, in.dst_row, src);
           const int64_t src_row = __shfl_sync(0xffffffffu, in.src_row, src);
-          const uint32_t tok_base = __shfl_sync(0xffffffffu, in.tok0 + 2u * in.pair0 * (a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u), src);
+          const uint32_t tok_base = __shfl_sync(
+              0xffffffffu, gapped ? in.tok0 : in.tok0 + 2u * in.pair0 * (a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u), src);
+          const uint32_t gap_u = __shfl_sync(0xffffffffu, gapped && live ? sub_offset(a, in) : 0u, src);
+          const uint32_t gp0 = __shfl_sync(0xffffffffu, 2u * in.pair0, src);
           if (gi < a.n_inst) {
             if (a.trace && lane == 0) a.trace[a.trace_base + (size_t)gi * nb] = kbg;
             gather_from_stage(a, dst_row, src_row, tok_base, st, (wi * (32 / SEG) + g) * NP, 0, m,
-                              [kbg](int i) { return ((kbg >> i) & 1u) != 0; }, lane, EC, NC);
+                              [kbg](int i) { return ((kbg >> i) & 1u) != 0; }, lane, EC, NC, kChunk, gap_u, gp0);
           }
         }
       } else {
@@ -399,8 +466,9 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
         if (live) {
           if (a.trace && wi == 0 && lane < nb) a.trace[a.trace_base + (size_t)inst * nb + lane] = lane ? kb1 : kb0;
           auto bit = [kb0, kb1](int i) { return (((i < 32 ? kb0 : kb1) >> (i & 31)) & 1u) != 0; };
-          const uint32_t tok_base = in.tok0 + 2u * in.pair0 * (a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u);
-          gather_from_stage(a, in.dst_row, in.src_row, tok_base, st, 0, wi ? half : 0, wi ? m : half, bit, lane, EC, NC);
+          const uint32_t tok_base = gapped ? in.tok0 : in.tok0 + 2u * in.pair0 * (a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u);
+          gather_from_stage(a, in.dst_row, in.src_row, tok_base, st, 0, wi ? half : 0, wi ? m : half, bit, lane, EC, NC,
+                            kChunk, gapped ? sub_offset(a, in) : 0u, 2u * in.pair0);
         }
       }
       __syncwarp();
@@ -1145,8 +1213,15 @@ bool halving_fused_supported(const StepArgs& a) {
   // 257..512 points: the V rows (4 blocks x D/64 chunks of 16 KB) are staged in the 131.6 KB Delta
   // area for c, so D <= 128
   if (a.n > 256 && a.D > 128) return false;
-  // subsampled rows form boxes only as a strided view (integer ratio, runs on multiples of it)
-  if (a.src_kind == SRC_TOKENS && a.S_sub < a.S_full && a.sub_stride < 2) return false;
+  // subsampled rows: an integer ratio is a strided view (runs on multiples of it); another ratio
+  // needs the tokens spanned by an instance's n points, at most ceil((n-1) S / S') + 1, to fit the
+  // box of NP rows of the persistent kernel
+  if (a.src_kind == SRC_TOKENS && a.S_sub < a.S_full && a.sub_stride < 2) {
+    if (a.n > 128) return false;
+    const int NP = a.n <= 32 ? 32 : a.n <= 64 ? 64 : 128;
+    const int64_t span = ((int64_t)(a.n - 1) * a.S_full + a.S_sub - 1) / a.S_sub + 1;
+    if (span > NP) return false;
+  }
   return true;
 }
 
