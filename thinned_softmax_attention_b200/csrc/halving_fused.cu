@@ -65,7 +65,7 @@ struct FusedShape {
 // Copy the kept point of pairs [i0, i1) of one instance from the stage (unit rows row0 + 2i or
 // row0 + 2i + 1) to destination rows dst_row + i, with its token index.  One warp; lane = one
 // 16-byte unit of a row (K units first), four rows in flight.
-template <typename Bit>
+template <bool GAP = false, typename Bit>
 __device__ __forceinline__ void gather_from_stage(const StepArgs& a, int64_t dst_row, int64_t src_row, uint32_t tok_base,
                                                   const uint8_t* st, int row0, int i0, int i1, Bit bit, int lane,
                                                   int EC, int NC, uint32_t chunk_bytes = kChunk, uint32_t gap_u = 0,
@@ -74,7 +74,7 @@ __device__ __forceinline__ void gather_from_stage(const StepArgs& a, int64_t dst
   // subsample); for a subsample of another ratio tok_base + floor(((gp0 + p) S + U) / S') with
   // gp0 = 2 pair0 and U = gap_u, the subsample's own formula
   const bool tokens = a.src_kind == SRC_TOKENS;
-  const bool gapped = tokens && a.S_sub < a.S_full && a.sub_stride < 2;
+  constexpr bool gapped = GAP;   // (the caller's: tokens subsampled with a non-integer ratio)
   const uint32_t k = a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u;
   for (int i = i0 + lane; i < i1; i += 32) {
     const int p = 2 * i + (bit(i) ? 0 : 1);
@@ -107,7 +107,9 @@ __device__ __forceinline__ void gather_from_stage(const StepArgs& a, int64_t dst
   }
 }
 
-template <int NP>
+// GAP: token runs subsampled with a non-integer ratio (a separate instance of the kernel, so that
+// the others carry none of its code).
+template <int NP, bool GAP>
 __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_constant__ FusedMaps maps,
                                                                   const StepArgs a, int n_units, int nst) {
   using Sh = FusedShape<NP>;
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
   // [t(2 pair0), t(2 pair0 + n - 1)] (t = the subsample's index formula), at most NP of them, so
   // the box of NP rows from the first holds them all; the epilogue warps move the selected rows
   // up to rows 0..n-1 before the MMAs read the stage
-  const bool gapped = a.src_kind == SRC_TOKENS && a.S_sub < a.S_full && a.sub_stride < 2;
+  constexpr bool gapped = GAP;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -409,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
           const uint32_t gp0 = __shfl_sync(0xffffffffu, 2u * in.pair0, src);
           if (gi < a.n_inst) {
             if (a.trace && lane == 0) a.trace[a.trace_base + (size_t)gi * nb] = kbg;
-            gather_from_stage(a, dst_row, src_row, tok_base, st, (wi * (32 / SEG) + g) * NP, 0, m,
+            gather_from_stage<GAP>(a, dst_row, src_row, tok_base, st, (wi * (32 / SEG) + g) * NP, 0, m,
                               [kbg](int i) { return ((kbg >> i) & 1u) != 0; }, lane, EC, NC, kChunk, gap_u, gp0);
           }
         }
@@ -467,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
           if (a.trace && wi == 0 && lane < nb) a.trace[a.trace_base + (size_t)inst * nb + lane] = lane ? kb1 : kb0;
           auto bit = [kb0, kb1](int i) { return (((i < 32 ? kb0 : kb1) >> (i & 31)) & 1u) != 0; };
           const uint32_t tok_base = gapped ? in.tok0 : in.tok0 + 2u * in.pair0 * (a.sub_stride > 1 ? (uint32_t)a.sub_stride : 1u);
-          gather_from_stage(a, in.dst_row, in.src_row, tok_base, st, 0, wi ? half : 0, wi ? m : half, bit, lane, EC, NC,
+          gather_from_stage<GAP>(a, in.dst_row, in.src_row, tok_base, st, 0, wi ? half : 0, wi ? m : half, bit, lane, EC, NC,
                             kChunk, gapped ? sub_offset(a, in) : 0u, 2u * in.pair0);
         }
       }
@@ -511,11 +513,13 @@ cudaError_t launch_np(const StepArgs& a, cudaStream_t st) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(halve_fused_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  const bool gap = a.src_kind == SRC_TOKENS && a.S_sub < a.S_full && a.sub_stride < 2;
+  auto kern = gap ? halve_fused_kernel<NP, true> : halve_fused_kernel<NP, false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const int n_units = (a.n_inst + FusedShape<NP>::IPU - 1) / FusedShape<NP>::IPU;
   const int grid = n_units < sms ? n_units : sms;
-  halve_fused_kernel<NP><<<grid, kThreads, sm, st>>>(maps, a, n_units, nst);
+  kern<<<grid, kThreads, sm, st>>>(maps, a, n_units, nst);
   return cudaGetLastError();
 }
 
@@ -809,7 +813,8 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
 // Instances of 257..512 points (the first step of a HALVE merge of four 128-point nodes): one CTA per
 // instance.  The 256 x 256 pair differences are kept as the packed upper triangle (row j holds
 // columns j..255, 131.6 KB) in shared memory (before the first Delta is written, that area holds the
-// instance's V rows, loaded by TMA for c = max |v|); the 512 point rows do not fit beside it, so the Gram
+// instance's V rows, loaded by TMA for c = max |v| in one round for D <= 128, two for D <= 256); the
+// 512 point rows do not fit beside it, so the Gram
 // runs over the 10 upper-triangle pairs (bi <= bj) of 128-row blocks in row-block order, each a
 // (128 x 128) kk and vv product streamed through a two-stage ring of 64-column chunks (A = rows of
 // block bi, B = rows of block bj), accumulators double-buffered in TMEM.  The kept rows are gathered
@@ -819,6 +824,10 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
 // walk of pair block t starts once Delta rows 32t..32t+31 (row block t/2) are complete.  Every wait
 // is bounded.
 constexpr int kH512Pairs = 256;
+
+// Blocks of 128 V rows staged per round in the 131.6 KB Delta area: all four for D <= 128 (at most
+// 8 chunks of 16 KB), two for D <= 256.
+__host__ __device__ __forceinline__ int v_blocks_per_round(int DCn) { return DCn <= 2 ? 4 : 2; }
 
 __device__ __forceinline__ int tri_offset(int j) { return j * kH512Pairs - (j * (j - 1)) / 2; }
 
@@ -888,7 +897,8 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
   uint64_t* cmax = bars + 8;      // c exchanged among the epilogue threads (128)
   uint64_t* drow = bars + 9;      // [4] Delta rows of row block b complete (128)
   uint64_t* mdone = bars + 14;    // every MMA complete
-  uint64_t* vfull = bars + 15;    // the instance's V rows landed in the Delta area
+  uint64_t* vfull = bars + 15;    // a round of the instance's V rows landed in the Delta area
+  uint64_t* vread = bars + 16;    // a round of V rows read by every epilogue thread (128)
   __shared__ __align__(8) uint64_t thf[8];   // thresholds of pair block t published (32)
   __shared__ __align__(8) uint64_t bitsb[8]; // decisions of pair block t published (32; blocks in order)
   __shared__ float red[4];
@@ -912,6 +922,7 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
     for (int b = 0; b < 4; ++b) mbar_init(drow + b, 128);
     mbar_init(mdone, 1);
     mbar_init(vfull, 1);
+    mbar_init(vread, 128);
     for (int t = 0; t < 8; ++t) {
       mbar_init(thf + t, 32);
       mbar_init(bitsb + t, 32);
@@ -936,19 +947,29 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const int row = (int)(tokens ? in.src_row / ks + 2 * (int64_t)in.pair0 : in.src_row);
-      const int h = (int)(in.bh % (uint32_t)a.H);
-      // V rows of the four blocks into the Delta area (DC chunks of 128 rows x 64 columns per block)
-      const int DCn = NC - EC;
-      mbar_expect_tx(vfull, (uint32_t)(4 * DCn) * kChunk);
-      for (int blk = 0; blk < 4; ++blk)
-        for (int c = 0; c < DCn; ++c) {
-          uint8_t* dst = (uint8_t*)D + (blk * DCn + c) * kChunk;
-          if (!tokens) tma_load_2d(dst, &maps.v, vfull, c * 64, row + 128 * blk);
-          else if (ks > 1) tma_load_4d(dst, &maps.v, vfull, c * 64, h, 0, row + 128 * blk);
-          else tma_load_3d(dst, &maps.v, vfull, c * 64, h, row + 128 * blk);
+    const int row = (int)(tokens ? in.src_row / ks + 2 * (int64_t)in.pair0 : in.src_row);
+    const int h = (int)(in.bh % (uint32_t)a.H);
+    if (lane == 1) {
+      // V rows into the Delta area for c, in rounds of bpr blocks (DC chunks of 128 rows x 64
+      // columns per block); a round overwrites the area once every epilogue thread read the last
+      const int DCn = NC - EC, bpr = v_blocks_per_round(DCn);
+      for (int r0 = 0; r0 < 4; r0 += bpr) {
+        if (r0 > 0 && !mbar_wait(vread, (r0 / bpr - 1) & 1, abort)) break;
+        mbar_expect_tx(vfull, (uint32_t)(bpr * DCn) * kChunk);
+        for (int blk = r0; blk < r0 + bpr; ++blk)
+          for (int c = 0; c < DCn; ++c) {
+            uint8_t* dst = (uint8_t*)D + ((blk - r0) * DCn + c) * kChunk;
+            if (!tokens) tma_load_2d(dst, &maps.v, vfull, c * 64, row + 128 * blk);
+            else if (ks > 1) tma_load_4d(dst, &maps.v, vfull, c * 64, h, 0, row + 128 * blk);
+            else tma_load_3d(dst, &maps.v, vfull, c * 64, h, row + 128 * blk);
+          }
+        // leave no copy in flight
+        const long long t0 = clock64();
+        while (!mbar_try_wait(vfull, (r0 / bpr) & 1) && clock64() - t0 < kWaitCycles) {
         }
+      }
+    }
+    if (lane == 0) {
       int g = 0;
       bool ok = true;
       for (int q = 0; q < NBP && ok; ++q) {
@@ -978,9 +999,6 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
         const long long t0 = clock64();
         while (!mbar_try_wait(full + (gg & 1), (gg >> 1) & 1) && clock64() - t0 < kWaitCycles) {
         }
-      }
-      const long long t0 = clock64();
-      while (!mbar_try_wait(vfull, 0) && clock64() - t0 < kWaitCycles) {
       }
     }
   } else if (warp == 1) {
@@ -1024,25 +1042,30 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
     const int q4 = warp & 3;                    // TMEM lane quarter of this warp
     const int r = q4 * 32 + lane;               // row within a 128-row block = TMEM lane
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    // c = max |v| over the instance's rows, from the V rows staged in the Delta area (row R of
-    // block blk: 128 bytes per chunk, 16-byte units swizzled by R & 7)
-    bool ok = warp_wait(vfull, 0, abort);
+    // c = max |v| over the instance's rows, from the V rows staged in the Delta area round by
+    // round (row R of a block: 128 bytes per chunk, 16-byte units swizzled by R & 7)
+    bool ok = true;
     float mx = 0.f;
-    if (ok) {
-      const int DCn = NC - EC;
-      for (int blk = 0; blk < 4; ++blk) {
-        if (128 * blk + r >= n) break;
-        for (int c = 0; c < DCn; ++c) {
-          const uint8_t* rowp = (const uint8_t*)D + (blk * DCn + c) * kChunk + r * 128;
+    {
+      const int DCn = NC - EC, bpr = v_blocks_per_round(DCn);
+      for (int r0 = 0; r0 < 4 && ok; r0 += bpr) {
+        ok = warp_wait(vfull, (r0 / bpr) & 1, abort);
+        if (!ok) break;
+        for (int blk = r0; blk < r0 + bpr; ++blk) {
+          if (128 * blk + r >= n) break;
+          for (int c = 0; c < DCn; ++c) {
+            const uint8_t* rowp = (const uint8_t*)D + ((blk - r0) * DCn + c) * kChunk + r * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 w = *(const uint4*)(rowp + ((q ^ (r & 7)) << 4));
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            for (int q = 0; q < 8; ++q) {
+              const uint4 w = *(const uint4*)(rowp + ((q ^ (r & 7)) << 4));
+              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              mx = fmax3(mx, fabsf(__uint_as_float(ws[e] << 16)), fabsf(__uint_as_float(ws[e] & 0xFFFF0000u)));
+              for (int e = 0; e < 4; ++e)
+                mx = fmax3(mx, fabsf(__uint_as_float(ws[e] << 16)), fabsf(__uint_as_float(ws[e] & 0xFFFF0000u)));
+            }
           }
         }
+        mbar_arrive(vread);   // this thread's reads of the round are done
       }
     }
 #pragma unroll
@@ -1176,7 +1199,7 @@ cudaError_t launch_512(const StepArgs& a, cudaStream_t st) {
   }
   if (!ok) return cudaErrorInvalidValue;
   const size_t delta_bytes = (size_t)(kH512Pairs * (kH512Pairs + 1) / 2) * 4;
-  if ((size_t)4 * (a.D / 64) * kChunk > delta_bytes) return cudaErrorInvalidValue;   // V staging must fit
+  if ((size_t)v_blocks_per_round(a.D / 64) * (a.D / 64) * kChunk > delta_bytes) return cudaErrorInvalidValue;
   const size_t sm = 1024 + 4 * (size_t)kChunk + delta_bytes;
   cudaError_t e = cudaFuncSetAttribute(halve512_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
@@ -1210,9 +1233,6 @@ bool halving_fused_supported(const StepArgs& a) {
   if (std::getenv("THIN_ATTN_UNFUSED_HALVING") != nullptr) return false;
   if (a.E % 64 || a.D % 64 || (a.E + a.D) / 64 > kMaxChunks || a.n < 2 || a.n > 512 || a.n % 2) return false;
   if (a.src_rows <= 0 || !tensor_maps_available()) return false;
-  // 257..512 points: the V rows (4 blocks x D/64 chunks of 16 KB) are staged in the 131.6 KB Delta
-  // area for c, so D <= 128
-  if (a.n > 256 && a.D > 128) return false;
   // subsampled rows: an integer ratio is a strided view (runs on multiples of it); another ratio
   // needs the tokens spanned by an instance's n points, at most ceil((n-1) S / S') + 1, to fit the
   // box of NP rows of the persistent kernel
