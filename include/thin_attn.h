@@ -55,7 +55,7 @@ typedef enum {
   THIN_ATTN_ENOMEM = 2,        /* device or host allocation failed */
   THIN_ATTN_ECUDA = 3,         /* a CUDA call failed (message holds the CUDA error) */
   THIN_ATTN_ETIMEOUT = 4,      /* a bounded device-side wait gave up */
-  THIN_ATTN_EUNSUPPORTED = 5   /* valid request outside what this build implements */
+  THIN_ATTN_EUNSUPPORTED = 5   /* valid request outside what this library implements */
 } thin_attn_status;
 
 typedef enum { THIN_ATTN_FP32 = 0, THIN_ATTN_BF16 = 1 } thin_attn_dtype;

@@ -50,7 +50,7 @@ def _call(Ks, Vs, seed, round_id):
                                            (128, 3, 64, 64, "fp32")])
 def test_noalloc_matches_forward_twice(S, g, E, D, dtype):
     # S with 4^g < S <= 4^(g+1) and S = 4L: KH-Compress is a single halving of all S keys of each
-    # (b,h) with Philox round 1 and counter word b*H+h -- the instance index below.
+    # (b,h) with Philox round id 1 and counter word b*H+h -- the instance index below.
     w = W.Workload("noalloc", 2, 3, 16, S, E, D, dtype, False, g, 5, 8, "iid")
     q, k, v = (x.cuda() for x in W.make_qkv(w))
     h = TA.ThinAttention(w.B, w.T, S, w.H, E, D, w.torch_dtype)

@@ -527,9 +527,9 @@ cudaError_t launch_np(const StepArgs& a, cudaStream_t st) {
 // Instances of 129..256 points: one CTA per instance (its 256 rows, 32 KB per feature chunk, and the
 // 128 x 128 pair differences take the shared memory of an SM).  Warps: 0 TMA, 1 MMA (TMEM owner),
 // 2-5 epilogue (warp w reads TMEM lanes 32 (w % 4)..), 6 sigma's recursion, 7 the walk; all eight
-// gather.  The Gram takes two rounds through the 512 TMEM columns: rows 0..127 against all 256 rows
+// gather.  The Gram takes two passes through the 512 TMEM columns: rows 0..127 against all 256 rows
 // (kk in columns 0..255, vv in 256..511), then rows 128..255 against themselves (columns 0..127 and
-// 256..383), so Delta rows 0..63 are written while the second round runs.  Every barrier is used
+// 256..383), so Delta rows 0..63 are written while the second pass runs.  Every barrier is used
 // once (phase 0) and every wait is bounded.
 __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant__ FusedMaps maps, const StepArgs a) {
   constexpr int LD = 129;                       // Delta row stride (floats)
@@ -540,9 +540,9 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
   float* D = (float*)(smem + NC * CB);          // [128][LD]
   __shared__ __align__(8) uint64_t bars[16];
   uint64_t* full = bars;          // rows landed
-  uint64_t* tfull0 = bars + 1;    // round 1 accumulators ready
-  uint64_t* tempty0 = bars + 2;   // round 1 accumulators read (128)
-  uint64_t* tfull1 = bars + 3;    // round 2 accumulators ready
+  uint64_t* tfull0 = bars + 1;    // first-pass accumulators ready
+  uint64_t* tempty0 = bars + 2;   // first-pass accumulators read (128)
+  uint64_t* tfull1 = bars + 3;    // second-pass accumulators ready
   uint64_t* cmax = bars + 4;      // c exchanged among the epilogue threads (128)
   uint64_t* dhalf = bars + 5;     // Delta rows 0..63 written (128)
   uint64_t* dfull = bars + 6;     // Delta rows 64..127 written (128)
@@ -641,7 +641,7 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
   } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------------ epilogue
     const int q4 = warp & 3;                    // TMEM lane quarter of this warp
-    const int r = q4 * 32 + lane;               // row r of round 1 (row 128 + r of round 2)
+    const int r = q4 * 32 + lane;               // row r of the first pass (row 128 + r of the second)
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     bool ok = warp_wait(full, 0, abort);
     float c2 = 0.f;
@@ -672,7 +672,7 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
       const float cm = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
       c2 = cm * cm;
     }
-    // round 1: pair rows 0..63 against pair columns 0..127
+    // first pass: pair rows 0..63 against pair columns 0..127
     if (ok) ok = warp_wait(tfull0, 0, abort);
     if (ok) {
       tc_fence_after();
@@ -706,7 +706,7 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
     }
     mbar_arrive(tempty0);
     mbar_arrive(dhalf);
-    // round 2: pair rows 64..127 against pair columns 64..127
+    // second pass: pair rows 64..127 against pair columns 64..127
     if (ok) ok = warp_wait(tfull1, 0, abort);
     if (ok) {
       tc_fence_after();
@@ -813,7 +813,7 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
 // Instances of 257..512 points (the first step of a HALVE merge of four 128-point nodes): one CTA per
 // instance.  The 256 x 256 pair differences are kept as the packed upper triangle (row j holds
 // columns j..255, 131.6 KB) in shared memory (before the first Delta is written, that area holds the
-// instance's V rows, loaded by TMA for c = max |v| in one round for D <= 128, two for D <= 256); the
+// instance's V rows, loaded by TMA for c = max |v| in one pass for D <= 128, two for D <= 256); the
 // 512 point rows do not fit beside it, so the Gram
 // runs over the 10 upper-triangle pairs (bi <= bj) of 128-row blocks in row-block order, each a
 // (128 x 128) kk and vv product streamed through a two-stage ring of 64-column chunks (A = rows of
@@ -825,7 +825,7 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
 // is bounded.
 constexpr int kH512Pairs = 256;
 
-// Blocks of 128 V rows staged per round in the 131.6 KB Delta area: all four for D <= 128 (at most
+// Blocks of 128 V rows staged per pass in the 131.6 KB Delta area: all four for D <= 128 (at most
 // 8 chunks of 16 KB), two for D <= 256.
 __host__ __device__ __forceinline__ int v_blocks_per_round(int DCn) { return DCn <= 2 ? 4 : 2; }
 
@@ -897,8 +897,8 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
   uint64_t* cmax = bars + 8;      // c exchanged among the epilogue threads (128)
   uint64_t* drow = bars + 9;      // [4] Delta rows of row block b complete (128)
   uint64_t* mdone = bars + 14;    // every MMA complete
-  uint64_t* vfull = bars + 15;    // a round of the instance's V rows landed in the Delta area
-  uint64_t* vread = bars + 16;    // a round of V rows read by every epilogue thread (128)
+  uint64_t* vfull = bars + 15;    // a pass of the instance's V rows landed in the Delta area
+  uint64_t* vread = bars + 16;    // a pass of V rows read by every epilogue thread (128)
   __shared__ __align__(8) uint64_t thf[8];   // thresholds of pair block t published (32)
   __shared__ __align__(8) uint64_t bitsb[8]; // decisions of pair block t published (32; blocks in order)
   __shared__ float red[4];
@@ -950,8 +950,8 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
     const int row = (int)(tokens ? in.src_row / ks + 2 * (int64_t)in.pair0 : in.src_row);
     const int h = (int)(in.bh % (uint32_t)a.H);
     if (lane == 1) {
-      // V rows into the Delta area for c, in rounds of bpr blocks (DC chunks of 128 rows x 64
-      // columns per block); a round overwrites the area once every epilogue thread read the last
+      // V rows into the Delta area for c, in passes of bpr blocks (DC chunks of 128 rows x 64
+      // columns per block); a pass overwrites the area once every epilogue thread read the last
       const int DCn = NC - EC, bpr = v_blocks_per_round(DCn);
       for (int r0 = 0; r0 < 4; r0 += bpr) {
         if (r0 > 0 && !mbar_wait(vread, (r0 / bpr - 1) & 1, abort)) break;
@@ -1042,8 +1042,8 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
     const int q4 = warp & 3;                    // TMEM lane quarter of this warp
     const int r = q4 * 32 + lane;               // row within a 128-row block = TMEM lane
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    // c = max |v| over the instance's rows, from the V rows staged in the Delta area round by
-    // round (row R of a block: 128 bytes per chunk, 16-byte units swizzled by R & 7)
+    // c = max |v| over the instance's rows, from the V rows staged in the Delta area pass by
+    // pass (row R of a block: 128 bytes per chunk, 16-byte units swizzled by R & 7)
     bool ok = true;
     float mx = 0.f;
     {
@@ -1065,7 +1065,7 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
             }
           }
         }
-        mbar_arrive(vread);   // this thread's reads of the round are done
+        mbar_arrive(vread);   // this thread's reads of the pass are done
       }
     }
 #pragma unroll
