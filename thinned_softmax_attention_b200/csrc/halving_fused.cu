@@ -827,7 +827,7 @@ constexpr int kH512Pairs = 256;
 
 // Blocks of 128 V rows staged per pass in the 131.6 KB Delta area: all four for D <= 128 (at most
 // 8 chunks of 16 KB), two for D <= 256.
-__host__ __device__ __forceinline__ int v_blocks_per_round(int DCn) { return DCn <= 2 ? 4 : 2; }
+__host__ __device__ __forceinline__ int v_blocks_per_pass(int DCn) { return DCn <= 2 ? 4 : 2; }
 
 __device__ __forceinline__ int tri_offset(int j) { return j * kH512Pairs - (j * (j - 1)) / 2; }
 
@@ -952,7 +952,7 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
     if (lane == 1) {
       // V rows into the Delta area for c, in passes of bpr blocks (DC chunks of 128 rows x 64
       // columns per block); a pass overwrites the area once every epilogue thread read the last
-      const int DCn = NC - EC, bpr = v_blocks_per_round(DCn);
+      const int DCn = NC - EC, bpr = v_blocks_per_pass(DCn);
       for (int r0 = 0; r0 < 4; r0 += bpr) {
         if (r0 > 0 && !mbar_wait(vread, (r0 / bpr - 1) & 1, abort)) break;
         mbar_expect_tx(vfull, (uint32_t)(bpr * DCn) * kChunk);
@@ -1047,7 +1047,7 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
     bool ok = true;
     float mx = 0.f;
     {
-      const int DCn = NC - EC, bpr = v_blocks_per_round(DCn);
+      const int DCn = NC - EC, bpr = v_blocks_per_pass(DCn);
       for (int r0 = 0; r0 < 4 && ok; r0 += bpr) {
         ok = warp_wait(vfull, (r0 / bpr) & 1, abort);
         if (!ok) break;
@@ -1199,7 +1199,7 @@ cudaError_t launch_512(const StepArgs& a, cudaStream_t st) {
   }
   if (!ok) return cudaErrorInvalidValue;
   const size_t delta_bytes = (size_t)(kH512Pairs * (kH512Pairs + 1) / 2) * 4;
-  if ((size_t)v_blocks_per_round(a.D / 64) * (a.D / 64) * kChunk > delta_bytes) return cudaErrorInvalidValue;
+  if ((size_t)v_blocks_per_pass(a.D / 64) * (a.D / 64) * kChunk > delta_bytes) return cudaErrorInvalidValue;
   const size_t sm = 1024 + 4 * (size_t)kChunk + delta_bytes;
   cudaError_t e = cudaFuncSetAttribute(halve512_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
