@@ -646,7 +646,8 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
     bool ok = warp_wait(full, 0, abort);
     float c2 = 0.f;
     if (ok) {
-      float mx = 0.f;
+      // four independent max chains (one per 32-bit word of a 16-byte unit)
+      float m4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk) {
         const int R = r + 128 * blk;
@@ -659,11 +660,12 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
               const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                mx = fmax3(mx, fabsf(__uint_as_float(ws[e] << 16)), fabsf(__uint_as_float(ws[e] & 0xFFFF0000u)));
+                m4[e] = fmax3(m4[e], fabsf(__uint_as_float(ws[e] << 16)), fabsf(__uint_as_float(ws[e] & 0xFFFF0000u)));
             }
           }
         }
       }
+      float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 #pragma unroll
       for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       if (lane == 0) red[q4] = mx;
@@ -742,11 +744,18 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
     // ------------------------------------------------------------------ sigma's recursion
     const float C = a.C, rC = 1.f / C;
     float sigma = 0.f;
+    // the random numbers of all four blocks first, while Delta is still being formed
+    float wls[4];
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      const int p = 32 * blk + lane;
+      wls[blk] = p < m ? 1.f - 2.f * philox_uniform(a.seed, in.ctr_bh, in.round_id, in.pair0 + (uint32_t)p) : 0.f;
+    }
 #pragma unroll 1
     for (int blk = 0; blk < 4; ++blk) {
       if (!warp_wait(blk < 2 ? dhalf : dfull, 0, abort)) break;
       const int p = 32 * blk + lane;
-      const float wl = p < m ? 1.f - 2.f * philox_uniform(a.seed, in.ctr_bh, in.round_id, in.pair0 + (uint32_t)p) : 0.f;
+      const float wl = blk == 0 ? wls[0] : blk == 1 ? wls[1] : blk == 2 ? wls[2] : wls[3];
       thr_s[p] = thresholds32(sigma, D[p * LD + p], wl, C, rC, lane);
       __syncwarp();
       mbar_arrive(thf + blk);
