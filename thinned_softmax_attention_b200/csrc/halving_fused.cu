@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int EC = a.E / 64, NC = (a.E + a.D) / 64;
   float* D = (float*)(smem + NC * CB);          // [128][LD]
-  __shared__ __align__(8) uint64_t bars[16];
+  __shared__ __align__(8) uint64_t bars[20];
   uint64_t* full = bars;          // rows landed
   uint64_t* tfull0 = bars + 1;    // first-pass accumulators ready
   uint64_t* tempty0 = bars + 2;   // first-pass accumulators read (128)
@@ -546,9 +546,9 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
   uint64_t* cmax = bars + 4;      // c exchanged among the epilogue threads (128)
   uint64_t* dhalf = bars + 5;     // Delta rows 0..63 written (128)
   uint64_t* dfull = bars + 6;     // Delta rows 64..127 written (128)
-  uint64_t* bitsf = bars + 7;     // decisions published (32)
   uint64_t* mdone = bars + 8;     // every MMA complete
   uint64_t* thf = bars + 9;       // [4] thresholds of pair block b published (32)
+  uint64_t* bitsb = bars + 13;    // [4] decisions of pair block b published (32; blocks in order)
   __shared__ float red[4];
   __shared__ float thr_s[128];
   __shared__ uint32_t bits_s[4];
@@ -566,9 +566,11 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
     mbar_init(cmax, 128);
     mbar_init(dhalf, 128);
     mbar_init(dfull, 128);
-    mbar_init(bitsf, 32);
     mbar_init(mdone, 1);
-    for (int b = 0; b < 4; ++b) mbar_init(thf + b, 32);
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(thf + b, 32);
+      mbar_init(bitsb + b, 32);
+    }
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(&tmem_base_s, 512);
@@ -774,6 +776,9 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
       const uint32_t bb = walk_block32_th(cur, thr_s[base + lane], m - base, lane,
                                           [&](int q) { return D[(base + q) * LD + base + lane]; });
       kb[blk] = bb;
+      if (lane == 0) bits_s[blk] = bb;
+      __syncwarp();
+      mbar_arrive(bitsb + blk);   // the gatherers of this block may start
       // this block's contribution to the alpha of every later pair, in pair order
 #pragma unroll 1
       for (int b2 = blk + 1; b2 < 4; ++b2) {
@@ -785,22 +790,27 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
         else my[3] = acc;
       }
     }
-    if (lane == 0)
-      for (int b = 0; b < 4; ++b) bits_s[b] = kb[b];
-    __syncwarp();
-    mbar_arrive(bitsf);
   }
-  // ------------------------------------------------------------------ gather (all warps)
+  // ------------------------------------------------------------------ gather
+  // pair block t's kept rows from the stage as soon as its decisions are out: blocks 0..2 by warp
+  // pairs (0,1), (2,3), (4,5) -- idle by then -- while the walk goes on, block 3 by all eight warps
   __syncwarp();
-  if (warp_wait(bitsf, 0, abort)) {
+  {
+    auto bit = [&](int i) { return ((bits_s[i >> 5] >> (i & 31)) & 1u) != 0; };
+    const uint32_t tok_base = in.tok0 + 2u * in.pair0 * (uint32_t)ks;
+    if (warp < 6 && warp_wait(bitsb + (warp >> 1), 0, abort)) {
+      const int i0 = 32 * (warp >> 1) + 16 * (warp & 1);
+      gather_from_stage(a, in.dst_row, in.src_row, tok_base, smem, 0, min(m, i0), min(m, i0 + 16), bit, lane, EC, NC, CB);
+    }
+  }
+  if (warp_wait(bitsb + 3, 0, abort)) {
     const uint32_t b0 = bits_s[0], b1 = bits_s[1], b2 = bits_s[2], b3 = bits_s[3];
     auto bit = [b0, b1, b2, b3](int i) {
       const uint32_t w = i < 64 ? (i < 32 ? b0 : b1) : (i < 96 ? b2 : b3);
       return ((w >> (i & 31)) & 1u) != 0;
     };
-    const int per = (m + 7) / 8;
     const uint32_t tok_base = in.tok0 + 2u * in.pair0 * (uint32_t)ks;
-    gather_from_stage(a, in.dst_row, in.src_row, tok_base, smem, 0, min(m, warp * per), min(m, (warp + 1) * per),
+    gather_from_stage(a, in.dst_row, in.src_row, tok_base, smem, 0, min(m, 96 + 4 * warp), min(m, 100 + 4 * warp),
                       bit, lane, EC, NC, CB);
     if (a.trace && warp == 0 && lane < 4) {
       const int nb = a.m_pad >> 5;
