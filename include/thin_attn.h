@@ -26,6 +26,9 @@
  *
  * Execution: device entry points enqueue kernels on the caller's stream and
  * return without synchronising.  The host-buffer entry point synchronises.
+ * A handle's forwards share its workspace (and the work counter of its
+ * attention kernel), so they must not overlap on the GPU: issue them on one
+ * stream, or order the streams; use one handle per concurrent stream.
  *
  * Errors: every entry point returns a thin_attn_status; on failure the
  * calling thread's message is available from thin_attn_last_error().  Invalid
