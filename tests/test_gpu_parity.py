@@ -208,6 +208,16 @@ def test_dropin_call_returns_output_and_none():
     q, k, v = (x.cuda() for x in W.make_qkv(w))
     out, weights = TA.thinformer_attention(q, k, v, g=2, seed=1)
     assert weights is None and out.shape == (1, 256, 1, 64)
+    # the README's layer object: the same call, non-causal and causal
+    layer = TA.ThinformerAttention(g=2, seed=1)
+    out2, weights2 = layer(q, k, v)
+    assert weights2 is None and torch.equal(out, out2)
+    we = W.WORKLOADS["express32k"].with_(H=2)
+    qe, ke, ve = (x.cuda() for x in W.make_qkv(we, T=4096))
+    h = TA.ThinAttention(1, 4096, 4096, 2, we.E, we.D, we.torch_dtype, n_exact=1024, batch=1024)
+    ref = h.forward(qe, ke, ve, causal=True, g=2, seed=1)["out"]
+    out3, weights3 = layer(qe, ke, ve, causal=True)
+    assert weights3 is None and torch.equal(out3, ref)
 
 
 @pytest.mark.parametrize("name,mode", [("express", 1), ("express_a", 2), ("vit", 0)])

@@ -324,5 +324,22 @@ def thinformer_attention(query: torch.Tensor, key: torch.Tensor, value: torch.Te
     return _cache[k_].forward(query, key, value, causal=causal, g=g, seed=seed)["out"], None
 
 
-__all__ = ["ThinAttention", "ThinAttentionCache", "ThinAttnError", "thinformer_attention", "decode_trace", "lib", "LIB_PATH",
-           "EXPORTS"]
+class ThinformerAttention:
+    """The README's layer: ``layer = ThinformerAttention(); out, weights = layer(query, key, value)``
+    (query (B,T,H,E), key (B,S,H,E), value (B,S,H,D)) or ``layer(query, key, value, causal=True)``
+    (S = T, Thinformer Express with an exact phase of ``n_exact`` tokens and thin batches of
+    ``batch``).  ``weights`` is always None: the dense attention weights are never formed.  Every
+    call with the same shapes reuses one handle (and its workspace) per device.
+    """
+
+    def __init__(self, g: int = 2, seed: int = 0, n_exact: int = 1024, batch: int = 1024,
+                 scale: Optional[float] = None):
+        self.g, self.seed, self.n_exact, self.batch, self.scale = g, seed, n_exact, batch, scale
+
+    def __call__(self, query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, causal: bool = False):
+        return thinformer_attention(query, key, value, causal=causal, g=self.g, seed=self.seed,
+                                    n_exact=self.n_exact, batch=self.batch, scale=self.scale)
+
+
+__all__ = ["ThinAttention", "ThinAttentionCache", "ThinAttnError", "ThinformerAttention", "thinformer_attention",
+           "decode_trace", "lib", "LIB_PATH", "EXPORTS"]
