@@ -1100,29 +1100,60 @@ void host_groups(const thin_attn_config& c, int* groups, bool* by_heads) {
 thin_attn_status host_pipeline_setup(thin_attn_s* h) {
   if (!h->hp_sub.empty()) return THIN_ATTN_OK;
   const thin_attn_config& c = h->cfg;
-  host_groups(c, &h->hp_groups, &h->hp_by_heads);
-  const int NG = h->hp_groups;
+  int NG;
+  bool by_heads;
+  host_groups(c, &NG, &by_heads);
   const int Ht = c.H_total > 0 ? c.H_total : c.H;
+  // all or nothing: everything is made first and kept only if every piece was made
+  std::vector<thin_attn_s*> subs;
+  std::vector<cudaEvent_t> evs;
+  cudaStream_t sts[3] = {nullptr, nullptr, nullptr};
+  auto undo = [&]() {
+    for (auto sub : subs) thin_attn_destroy(sub);
+    for (auto e : evs) cudaEventDestroy(e);
+    for (auto st : sts)
+      if (st) cudaStreamDestroy(st);
+  };
   for (int gi = 0; gi < NG; ++gi) {
     thin_attn_config sc = c;
-    if (h->hp_by_heads) {
+    if (by_heads) {
       sc.H = c.H / NG;
       sc.h0 = c.h0 + gi * sc.H;
-      sc.H_total = Ht;
     } else {
       sc.B = c.B / NG;
       sc.b0 = c.b0 + gi * sc.B;
-      sc.H_total = Ht;
     }
+    sc.H_total = Ht;
     thin_attn_t sub = nullptr;
     thin_attn_status s = thin_attn_create(&sub, &sc);
-    if (s != THIN_ATTN_OK) return s;
-    h->hp_sub.push_back(sub);
+    if (s != THIN_ATTN_OK) {
+      undo();
+      return s;
+    }
+    subs.push_back(sub);
   }
   DeviceGuard dg(c.device);
-  for (cudaStream_t* st : {&h->hp_in, &h->hp_comp, &h->hp_out}) CK(cudaStreamCreateWithFlags(st, cudaStreamNonBlocking));
-  h->hp_ev.resize(3 * NG + 1);
-  for (auto& e : h->hp_ev) CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  for (auto& st : sts)
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) {
+      st = nullptr;
+      undo();
+      return fail(THIN_ATTN_ECUDA, "host pipeline: %s", cudaGetErrorString(cudaGetLastError()));
+    }
+  for (int i = 0; i < 3 * NG + 1; ++i) {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      undo();
+      return fail(THIN_ATTN_ECUDA, "host pipeline: %s", cudaGetErrorString(cudaGetLastError()));
+    }
+    evs.push_back(e);
+  }
+  h->hp_sub = subs;
+  h->hp_ev = evs;
+  h->hp_in = sts[0];
+  h->hp_comp = sts[1];
+  h->hp_out = sts[2];
+  h->hp_groups = NG;
+  h->hp_by_heads = by_heads;
   return THIN_ATTN_OK;
 }
 
