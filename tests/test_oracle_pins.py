@@ -193,6 +193,37 @@ def test_kh_first_pair_is_a_fair_coin():
         assert np.all(kernel_halving(K, V, 0.5, u).keep_first[:, 0] == want)
 
 
+def test_kh_follow_mode_replays_only_near_ties():
+    """Near-tie follow mode. Pair 0 has alpha = 0 and a = b^2, so u = 1/2 puts its decision exactly on
+    the swap boundary (margin 0). Following "keep x" there must give the walk that u = 1/4 gives
+    (only pair 0's decision differs between the two, and it feeds alpha of every later pair);
+    a followed decision that disagrees away from a near tie is flagged and not taken."""
+    K, V, _ = _rand_instances(8, 32, 4, 4, 11)
+    rng = np.random.default_rng(12)
+    u = rng.uniform(0.05, 0.95, size=(8, 16))
+    for first, u0 in ((True, 0.25), (False, 0.75)):
+        ua, ub = u.copy(), u.copy()
+        ua[:, 0], ub[:, 0] = u0, 0.5
+        ref = kernel_halving(K, V, 0.5, ua)
+        assert not ref.near[:, 0].any() and np.all(ref.keep_first[:, 0] == first)
+        own = kernel_halving(K, V, 0.5, ub)
+        assert own.near[:, 0].all()
+        fol = kernel_halving(K, V, 0.5, ub, follow=ref.keep_first)
+        assert np.array_equal(fol.keep_first, ref.keep_first)
+        assert not fol.mismatch.any()
+        assert np.array_equal(fol.near[:, 1:], ref.near[:, 1:])
+    # a disagreement away from a near tie: flagged, and the walk keeps its own decision
+    ref = kernel_halving(K, V, 0.5, u)
+    bad = ref.keep_first.copy()
+    far = ~ref.near
+    far[:, :5] = False
+    i, j = np.argwhere(far)[0]
+    bad[i, j] = ~bad[i, j]
+    fol = kernel_halving(K, V, 0.5, u, follow=bad)
+    assert fol.mismatch.sum() == 1 and fol.mismatch[i, j]
+    assert np.array_equal(fol.keep_first, ref.keep_first)
+
+
 def _mmd2(G, sel):
     n = G.shape[0]
     w = -np.ones(n) / n
