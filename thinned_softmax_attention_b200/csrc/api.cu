@@ -649,7 +649,11 @@ thin_attn_status materialise(thin_attn_s* h, Plan* p) {
       return fail(THIN_ATTN_ENOMEM, "status word: %s", cudaGetErrorString(e));
     }
     e = cudaMemset(h->d_status, 0, kStatusBytes);
-    if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "status word: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess) {  // a status word that is not zero is never kept
+      cudaFree(h->d_status);
+      h->d_status = nullptr;
+      return fail(THIN_ATTN_ECUDA, "status word: %s", cudaGetErrorString(e));
+    }
   }
   if (p->d_mem) return THIN_ATTN_OK;
   void* mem = nullptr;
@@ -980,7 +984,8 @@ thin_attn_status thin_attn_create(thin_attn_t* out, const thin_attn_config* cfg)
 
 thin_attn_status thin_attn_destroy(thin_attn_t h) {
   if (!h) return THIN_ATTN_OK;
-  const bool on_device = h->d_status || h->st_mem || h->side || !h->prof_free.empty() || !h->prof_pending.empty();
+  const bool on_device = h->d_status || h->st_mem || h->side || h->main || h->hp_in || !h->prof_free.empty() ||
+                         !h->prof_pending.empty();
   DeviceGuard dg(on_device ? h->cfg.device : -1);
   for (auto& kv : h->plans) {
     if (kv.second->d_mem) cudaFree(kv.second->d_mem);
