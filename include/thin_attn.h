@@ -161,6 +161,11 @@ THIN_ATTN_API thin_attn_status thin_attn_forward(thin_attn_t h, const void* q, c
  * in a pipeline on internal streams ordered after `stream`: the copy-in of one
  * shard and the copy-out of another overlap the compute of a third.  Results
  * are those of one thin_attn_forward of the whole problem, bit for bit.
+ * The staging belongs to the handle: run one host-buffer forward per handle at
+ * a time (one handle per host thread).  Errors: THIN_ATTN_ENOMEM when the
+ * staging cannot be allocated, the creation error of a shard handle, or
+ * THIN_ATTN_ECUDA when a stream or event cannot be made; none of the pieces is
+ * kept then, so a later call starts over.
  */
 THIN_ATTN_API thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void* k,
                                         const void* v, void* out, int causal, int g,
