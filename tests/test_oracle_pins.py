@@ -314,6 +314,21 @@ def test_subsample_indices_are_distinct_increasing():
             assert len(idx) == Ss and idx[0] >= 0 and idx[-1] < S and np.all(np.diff(idx) >= 1)
 
 
+@pytest.mark.parametrize("S,Ss", [(17, 16), (100, 64), (150, 64), (3136, 3072)])
+def test_subsample_is_evenly_spread(S, Ss):
+    """Systematic sampling with start U in [0, S'): every gap between kept indices is floor(S/S') or
+    ceil(S/S'), index 0 is always kept, and over all U a token is kept between max(0, 2S' - S) and S'
+    times (a window of S' starts can overlap at most one skipped run of S - S'), S'^2 times in all."""
+    U = np.arange(Ss)
+    idx = subsample_indices(S, Ss, U)
+    gaps = np.unique(np.diff(idx, axis=1))
+    assert set(gaps.tolist()) <= {S // Ss, -(-S // Ss)}
+    assert np.all(idx[:, 0] == 0) and np.all(idx[:, -1] < S)
+    counts = np.bincount(idx.ravel(), minlength=S)
+    assert counts.sum() == Ss * Ss
+    assert counts.min() >= max(0, 2 * Ss - S) and counts.max() <= Ss
+
+
 @pytest.mark.parametrize("S,g", [(16, 2), (60, 3), (64, 3)])
 def test_coreset_equal_full_set_is_exact_attention(S, g):
     """S <= 4^g: the coreset is every point (weight 1), so Thinformer is exact attention."""
