@@ -220,14 +220,6 @@ THIN_ATTN_API thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const
 /* Device int32 (B,H,n_nodes,c) token indices of every coreset slot (-1 while empty), in the
  * node order of thin_attn_forward's coreset output. */
 THIN_ATTN_API thin_attn_status thin_attn_cache_nodes(thin_attn_cache_t c, int32_t* idx_out, void* stream);
-/* The same recordings per halving step, in launch order: ms[i] the summed device time of step i
- * (from the end of the previous step, or the start of the forward, to its end), n_inst[i] its
- * instances and n_points[i] the points of each.  Up to max_steps entries are written;
- * *n_steps = steps of the most recently profiled plan (the sums restart when a forward of another
- * plan is recorded), *calls = forwards summed.  Resets the step sums.  Both readers wait for the
- * recorded forwards; each returns and resets only its own sums, so each sees every forward. */
-THIN_ATTN_API thin_attn_status thin_attn_profile_steps(thin_attn_t h, int max_steps, double* ms, int* n_inst,
-                                                       int* n_points, int* n_steps, int* calls);
 
 /* Synchronise `stream` and report a device-side failure of the cache's kernels. */
 THIN_ATTN_API thin_attn_status thin_attn_cache_check(thin_attn_cache_t c, void* stream);

@@ -109,9 +109,12 @@ def _ptr(t: Optional[torch.Tensor]):
 class ThinAttention:
     """One problem shape on one device: Thinformer (non-causal) and Thinformer Express (causal).
 
-    ``forward(q, k, v, causal, g, seed)`` returns ``(attn_output, None)``: the dense
-    attention weights are never formed; pass ``return_lse=True`` for the
-    log-sum-exp ln sum_j w_j e^{s q.k_j} instead.
+    ``forward(q, k, v, causal, g, seed)`` returns a dict: ``out`` (B,T,H,D) and, on request,
+    ``lse`` (B,H,T) fp32, the log-sum-exp ln sum_j w_j e^{s q.k_j} (``return_lse=True``),
+    ``coreset`` int32 token indices (``return_coreset=True``: (B,H,|C|), or (B,H,n_nodes,c) when
+    causal) and ``trace``, one bit per halving decision (``return_trace=True``).  The dense
+    attention weights are never formed; the layer call ``thinformer_attention`` returns
+    ``(attn_output, None)``.
 
     ``shard=(b0, h0, H_total)``: the tensors hold batch rows [b0, b0 + B) and heads
     [h0, h0 + H) of a larger problem with H_total heads (one handle per GPU of a batch- or
