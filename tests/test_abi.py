@@ -126,3 +126,47 @@ def test_decode_trace_bit_order():
     bits = d[(3, 7)]
     assert bits.shape == (80,)
     assert list(np.nonzero(bits)[0]) == [0, 2, 39, 40]
+
+
+def _plan_pairs(h, causal, g):
+    """(b*H+h, round id) -> pairs, from the plan's trace layout; each key's pair ranges tile 0..m."""
+    parts = {}
+    for bh, rid, pair0, m, _ in h.trace_layout(causal, g):
+        parts.setdefault((bh, rid), []).append((pair0, m))
+    out = {}
+    for key, ps in parts.items():
+        ps.sort()
+        assert ps[0][0] == 0 and all(a[0] + a[1] == b[0] for a, b in zip(ps, ps[1:])), key
+        out[key] = ps[-1][0] + ps[-1][1]
+    return out
+
+
+# (mode, B, H, T, S, g, n_exact, batch): mode 0 Thinformer, 1 Express, 2 Express with the page-literal cache
+_PLAN_SWEEP = [
+    (0, 1, 2, 4, 1, 2, 0, 0), (0, 1, 1, 4, 17, 0, 0, 0), (0, 2, 1, 4, 100, 1, 0, 0), (0, 1, 1, 4, 300, 2, 0, 0),
+    (0, 1, 2, 4, 1000, 2, 0, 0), (0, 1, 1, 4, 3136, 2, 0, 0), (0, 1, 1, 4, 1024, 3, 0, 0), (0, 1, 1, 4, 4097, 5, 0, 0),
+    (1, 1, 2, 700, 700, 2, 100, 64), (1, 1, 1, 1000, 1000, 1, 0, 64), (1, 1, 1, 2048, 2048, 2, 256, 96),
+    (1, 1, 1, 300, 300, 2, 512, 256), (1, 1, 1, 700, 700, 2, 100, 16), (1, 1, 1, 5000, 5000, 2, 64, 64),
+    (2, 1, 1, 700, 700, 2, 16, 0), (2, 1, 2, 2000, 2000, 1, 32, 0), (2, 1, 1, 3000, 3000, 2, 64, 0),
+    (2, 1, 1, 100, 100, 2, 128, 0),
+]
+
+
+@pytest.mark.parametrize("mode,B,H,T_,S,g,n_e,bsz", _PLAN_SWEEP)
+def test_plan_halvings_are_the_oracles(mode, B, H, T_, S, g, n_e, bsz):
+    """The planner's halvings -- every (b,h, Philox round) and its pair count -- are exactly those the
+    oracle's run of the same problem takes, in all three modes."""
+    from oracle import express, express_a, thinformer
+    rng = np.random.default_rng(mode * 1000 + S + g)
+    L = S if mode == 0 else T_
+    q = rng.normal(size=(B, T_, H, 8))
+    k = rng.normal(size=(B, L, H, 8))
+    v = rng.normal(size=(B, L, H, 8))
+    if mode == 0:
+        ref = thinformer(q, k, v, g, 3, rows=[0])
+    elif mode == 1:
+        ref = express(q, k, v, n_e, bsz, g, 3, rows=[0])
+    else:
+        ref = express_a(q, k, v, n_e, g, 3, rows=[0])
+    h = T.ThinAttention(B, T_, L, H, 8, 8, W.WORKLOADS["tiny"].torch_dtype, n_exact=n_e, batch=bsz)
+    assert _plan_pairs(h, mode, g) == {key: len(bits) for key, bits in ref.trace.items()}
