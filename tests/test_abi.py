@@ -170,3 +170,11 @@ def test_plan_halvings_are_the_oracles(mode, B, H, T_, S, g, n_e, bsz):
         ref = express_a(q, k, v, n_e, g, 3, rows=[0])
     h = T.ThinAttention(B, T_, L, H, 8, 8, W.WORKLOADS["tiny"].torch_dtype, n_exact=n_e, batch=bsz)
     assert _plan_pairs(h, mode, g) == {key: len(bits) for key, bits in ref.trace.items()}
+    # and the coreset index output has the oracle's layout: (B,H,|C|), or (B,H,n_nodes,c) when causal
+    p = h.plan(mode, g)
+    assert p["coreset_idx_elems"] == ref.coreset.size
+    if mode == 0:
+        assert ref.coreset.shape == (B, H, p["coreset_rows"])
+    else:
+        assert ref.coreset.shape[:3] == (B, H, p["n_nodes"])
+        assert p["n_nodes"] == 0 or ref.coreset.shape[3] == p["coreset_rows"]
