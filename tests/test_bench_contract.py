@@ -1,11 +1,13 @@
-"""bench.py's reference arm (the fp64 oracle on the host cores) keeps the one-JSON-line contract.
-
-Runs on the CPU: the reference arm never touches a GPU.
+"""bench.py on the CPU: the reference arm (the fp64 oracle on the host cores) keeps the one-JSON-line
+contract, and the attention roofline counts the (query, key) pairs the method attends to.
 """
 import json
 import os
 import subprocess
 import sys
+
+import numpy as np
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
@@ -40,3 +42,42 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run({"RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+@pytest.mark.parametrize("mode,T,S,g,n_e,bsz", [
+    (0, 40, 1000, 2, 0, 0), (0, 30, 60, 3, 0, 0),
+    (1, 700, 700, 2, 100, 64), (1, 1000, 1000, 1, 0, 64), (1, 300, 300, 2, 512, 256), (1, 2048, 2048, 2, 256, 96),
+    (2, 700, 700, 2, 16, 0), (2, 3000, 3000, 2, 64, 0), (2, 100, 100, 2, 128, 0),
+])
+def test_roofline_pair_count_is_what_the_oracle_attends(mode, T, S, g, n_e, bsz, monkeypatch):
+    """The (query, key) pairs behind the attention roofline's FLOPs equal the pairs the oracle's
+    attention actually weighs: its weighted-softmax calls are counted (visible entries of each mask)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle.thin_oracle as O
+    import thinned_softmax_attention_b200 as TA
+    import workloads as W
+
+    seen = [0]
+    real = O.weighted_attention
+
+    def counting(q, K, V, scale, logw=None, mask=None):
+        seen[0] += int(mask.sum()) if mask is not None else q.shape[0] * K.shape[0]
+        return real(q, K, V, scale, logw, mask)
+
+    monkeypatch.setattr(O, "weighted_attention", counting)
+    w = W.Workload("count", 1, 1, T, S if mode == 0 else T, 8, 8, "fp32", mode > 0, g, 3, 1, "iid",
+                   n_exact=n_e, batch=bsz, cache="A" if mode == 2 else "B")
+    rng = np.random.default_rng(T + S)
+    L = w.S
+    q, k, v = rng.normal(size=(1, T, 1, 8)), rng.normal(size=(1, L, 1, 8)), rng.normal(size=(1, L, 1, 8))
+    if mode == 0:
+        O.thinformer(q, k, v, g, 3)
+    elif mode == 1:
+        O.express(q, k, v, n_e, bsz, g, 3)
+    else:
+        O.express_a(q, k, v, n_e, g, 3)
+    plan = TA.ThinAttention(1, T, L, 1, 8, 8, w.torch_dtype, n_exact=n_e, batch=bsz).plan(w.mode, g)
+    flops, _, pairs = bench.attention_work(w, plan)
+    assert pairs == seen[0] > 0
+    assert flops == 2.0 * (w.E + w.D) * pairs
