@@ -107,6 +107,24 @@ def test_weighted_attention_matches_sdpa(T, S, E, D, causal):
     np.testing.assert_allclose(lse, torch.logsumexp(z, dim=1).numpy(), rtol=1e-12)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_attention_matches_sdpa_per_batch_and_head(causal):
+    """The (B,T,H,E) wrapper: every (b,h) slice and any subset of query rows equals torch's SDPA in
+    fp64 on the (B,H,T,E) layout, with LSE from logsumexp."""
+    rng = np.random.default_rng(21 + causal)
+    B, T, H, E, D = 2, 19, 3, 8, 5
+    q, k, v = rng.normal(size=(B, T, H, E)), rng.normal(size=(B, T, H, E)), rng.normal(size=(B, T, H, D))
+    rows = np.array([0, 4, 11, 18])
+    out, lse = exact_attention(q, k, v, causal=causal, rows=rows)
+    qt, kt, vt = (torch.as_tensor(x).transpose(1, 2) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal).transpose(1, 2)
+    np.testing.assert_allclose(out, ref.numpy()[:, rows], rtol=1e-12, atol=1e-12)
+    z = qt @ kt.transpose(-1, -2) / math.sqrt(E)
+    if causal:
+        z = z.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), 1), -math.inf)
+    np.testing.assert_allclose(lse, torch.logsumexp(z, dim=-1).numpy()[:, :, rows], rtol=1e-12)
+
+
 def test_weight_is_multiplicity():
     """A key of weight 2 is the same as that key listed twice (weights multiply exp(s q.k))."""
     rng = np.random.default_rng(1)
