@@ -145,6 +145,8 @@ THIN_ATTN_API thin_attn_status thin_attn_trace_layout(thin_attn_t h, int causal,
  *   trace_opt         device uint32[trace_words] decision bits (thin_attn_trace_layout), or NULL
  *   stream            cudaStream_t to enqueue on (NULL = legacy default stream)
  * Allocates the plan's workspace on first use (not inside stream capture).
+ * THIN_ATTN_EUNSUPPORTED when a halving instance would hold more than 4096 points: the last
+ * KH-Compress level halves 2|C| points (2c per Express batch) and a HALVE merge 4c points.
  */
 THIN_ATTN_API thin_attn_status thin_attn_forward(thin_attn_t h, const void* q, const void* k, const void* v,
                                    void* out, int causal, int g, uint64_t seed, float* lse_opt,

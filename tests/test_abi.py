@@ -178,3 +178,23 @@ def test_plan_halvings_are_the_oracles(mode, B, H, T_, S, g, n_e, bsz):
     else:
         assert ref.coreset.shape[:3] == (B, H, p["n_nodes"])
         assert p["n_nodes"] == 0 or ref.coreset.shape[3] == p["coreset_rows"]
+
+
+def test_empty_inputs_and_the_largest_instance():
+    """B, T, H = 0 or S = 0 are rejected on the host; the largest halving instance is 4096 points
+    (the last level halves 2|C| points), one level beyond it is EUNSUPPORTED."""
+    bf16 = W.WORKLOADS["vit"].torch_dtype
+    for B_, T_, H_ in [(0, 4, 1), (1, 0, 1), (1, 4, 0)]:
+        with pytest.raises(T.ThinAttnError, match="EINVAL"):
+            T.ThinAttention(B_, T_, 4, H_, 64, 64, bf16)
+    with pytest.raises(T.ThinAttnError, match="EINVAL"):
+        T.ThinAttention(1, 4, 0, 1, 64, 64, bf16).plan(False, 2)
+    for S, g, ok in [(16384, 4, True), (65536, 4, False), (16384, 5, False), (4096, 6, True)]:
+        C = compress_sizes(S, g)[3]
+        h = T.ThinAttention(1, 4, S, 1, 64, 64, bf16)
+        assert ok == (compress_sizes(S, g)[0] == 0 or 2 * C <= 4096)
+        if ok:
+            assert h.plan(False, g)["coreset_rows"] == C
+        else:
+            with pytest.raises(T.ThinAttnError, match="EUNSUPPORTED"):
+                h.plan(False, g)
