@@ -198,3 +198,14 @@ def test_empty_inputs_and_the_largest_instance():
         else:
             with pytest.raises(T.ThinAttnError, match="EUNSUPPORTED"):
                 h.plan(False, g)
+
+
+def test_decode_cache_arguments_are_checked_on_the_host():
+    bf16 = W.WORKLOADS["vit"].torch_dtype
+    for kw in (dict(g=7), dict(g=-1), dict(batch=0), dict(n_exact=-1)):
+        args = dict(capacity=4096, n_exact=1024, batch=1024, g=2)
+        args.update(kw)
+        with pytest.raises(T.ThinAttnError, match="EINVAL"):
+            T.ThinAttentionCache(1, 4, 64, 64, bf16, **args)
+    with pytest.raises(T.ThinAttnError, match="EINVAL"):
+        T.ThinAttentionCache(1, 4, 12, 64, bf16, capacity=4096, n_exact=1024, batch=1024)   # E % 8
