@@ -29,10 +29,11 @@ algorithm, so each step below states the reading it takes:
   c points of weight b/c; a 4-ary counter merges four equal-level coresets
   by two halvings into one of 4x the weight ("HALVE" phase)      -- reading
 
-Parity is pinned by the tests in ``tests/test_oracle_*.py`` (library
-routines, closed forms, invariants, statistics).  The exact sequence of KH
-decisions has no printed value to check against: it is pinned only by the
-invariants and by an independent plain-loop implementation in the tests.
+The oracle is pinned by ``tests/test_oracle_pins.py`` (library routines,
+closed forms, invariants, statistics, an independent plain-loop walk) and
+``tests/test_golden.py`` (the cache relations the Express summary prints).
+The exact sequence of KH decisions has no printed value to check against: it
+is pinned only by the invariants and by the independent plain-loop walk.
 """
 from __future__ import annotations
 
