@@ -52,6 +52,8 @@ def args_():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-sdpa", action="store_true")
+    p.add_argument("--no-per-workload", action="store_true",
+                   help="N=1: skip the GPU-timed records of the other workloads")
     p.add_argument("--decode", action="store_true",
                    help="time token-by-token decoding of the workload through the Express decode cache "
                         "(causal workloads; prints its own JSON line)")
@@ -356,6 +358,157 @@ def run_decode(a):
     print(json.dumps(line))
 
 
+def exact_reference_error(w, q, k, v, out, n_rows=128, max_b=4, max_h=4):
+    """Approximation error of the computed output against exact softmax attention.
+
+    Exact attention in fp64 by torch's SDPA on the host, on a seeded sample of query rows of up to
+    ``max_b`` batch rows x ``max_h`` heads (outside any timed region).  Reported per (b,h) slice as
+    max|o - o_exact| / max|o_exact| (worst slice), and per query row as max_d |o - o_exact| /
+    max_d |o_exact| (worst row), with the mean over rows."""
+    rng = np.random.default_rng(0)
+    bs = list(range(min(w.B, max_b)))
+    hs = sorted(set(np.linspace(0, w.H - 1, min(w.H, max_h)).round().astype(int).tolist()))
+    rows = np.sort(rng.choice(w.T, min(n_rows, w.T), replace=False))
+    S = k.shape[1]
+    nb = len(bs)
+    o = out[:nb, rows][:, :, hs].double().cpu()                        # (b, rows, h, D)
+    qs = q[:nb, rows][:, :, hs].double().transpose(1, 2)               # (b, h, rows, E)
+    ks = k[:nb, :, hs].double().transpose(1, 2)
+    vs = v[:nb, :, hs].double().transpose(1, 2)
+    mask = None
+    if w.causal:
+        mask = torch.as_tensor(np.arange(S)[None, :] <= rows[:, None])
+    ex = torch.nn.functional.scaled_dot_product_attention(qs, ks, vs, attn_mask=mask, scale=w.scale)
+    ex = ex.transpose(1, 2)                                            # (b, rows, h, D)
+    d = (o - ex).abs()
+    slice_err = (d.amax(dim=(1, 3)) / ex.abs().amax(dim=(1, 3))).max().item()
+    row = d.amax(dim=3) / ex.abs().amax(dim=3)
+    return {"vs": "exact softmax attention, fp64 (torch SDPA on the host)", "rows": len(rows),
+            "batch_rows": bs, "heads": hs, "max_rel_per_slice": round(slice_err, 5),
+            "max_rel_per_row": round(row.max().item(), 5), "mean_rel_per_row": round(row.mean().item(), 5)}
+
+
+def attention_roofline(w, plan, attn_ms, pk):
+    """Roofline of the attention launch: bound by its arithmetic intensity against the ridge of the
+    burst bf16 peak over HBM copy bandwidth.  The launch is timed alone, sub-second, at full clocks,
+    so the burst peak is the denominator; the fraction of the sustained (power-capped) peak is
+    reported beside it."""
+    flops, abytes, pairs = attention_work(w, plan)
+    ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+    if w.dtype != "fp32" and flops / abytes >= ridge:
+        achieved = flops / (attn_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops"], 4),
+                "frac_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
+                "peak_kind": f"bf16 dense burst ({pk['source']}); sustained {pk['bf16_tflops_sustained']}"}
+    else:
+        achieved = abytes / (attn_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 2), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "peak_kind": f"HBM copy ({pk['source']})"}
+    roof.update({"kernel": "attention", "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
+                 "arithmetic_intensity": round(flops / abytes, 1), "ridge": round(ridge, 1),
+                 "avg_launch_ms": round(attn_ms, 4)})
+    return roof
+
+
+def halving_roofline(w, h, ph, pk):
+    """Halving steps, HBM-bound by their algorithmic bytes: every instance's n points read once and its
+    n/2 survivors written once, 1.5 n (E+D) elements per instance.  Per step from the live per-step
+    CUDA events; the headline is the step that takes longest, beside the whole halving phase."""
+    es = 4 if w.dtype == "fp32" else 2
+    sp = h.profile_steps()
+    steps_tab = []
+    for st in sp["steps"]:
+        sb = st["n_inst"] * 3 * st["n"] // 2 * (w.E + w.D) * es
+        sms = st["ms"] / max(1, sp["calls"])
+        steps_tab.append({"n": st["n"], "n_inst": st["n_inst"], "ms": round(sms, 4), "bytes": sb,
+                          "frac": round(sb / (sms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if sms > 0 else None})
+    hbytes = sum(t["bytes"] for t in steps_tab)
+    hms = (ph["thin_ms"] + ph["merge_ms"]) / max(1, ph["calls"])
+    top = max(steps_tab, key=lambda t: t["ms"]) if steps_tab else None
+    if not top or top["ms"] <= 0:
+        return None
+    return {"bound": "hbm", "achieved": round(top["bytes"] / (top["ms"] * 1e-3) / 1e9, 1),
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": top["frac"],
+            "kernel": f"halving step n={top['n']} x {top['n_inst']} instances",
+            "algorithmic_bytes_per_launch": top["bytes"], "avg_launch_ms": top["ms"],
+            "traffic": kernel_traffic("halving_fused_n64") if (w.name == "express32k" and top["n"] == 64) else None,
+            "all_steps": {"achieved": round(hbytes / (hms * 1e-3) / 1e9, 1) if hms > 0 else None,
+                          "frac": round(hbytes / (hms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if hms > 0 else None,
+                          "bytes": hbytes, "ms": round(hms, 4)},
+            "steps": steps_tab}
+
+
+L2_BYTES = 126e6
+
+
+def timed_steps(step, steps, stream, flush):
+    """CUDA-event time per step (ms).  With ``flush`` (a device buffer larger than L2) the buffer is
+    rewritten before every step and each step is timed alone; otherwise the steps run back to back."""
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+    evs = []
+    for _ in range(steps):
+        flush.add_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / steps
+
+
+def measure_workload(TA, name, dev, steps, warmup):
+    """One workload on this GPU alone: ms per layer (CUDA events, inputs resident in HBM), phases,
+    the attention and halving rooflines and the approximation error against exact attention."""
+    w = W.WORKLOADS[name]
+    qc, kc, vc = W.make_qkv(w)
+    q, k, v = (x.to(dev) for x in (qc, kc, vc))
+    S = w.T if w.causal else w.S
+    h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch, device=dev.index)
+    plan = h.plan(w.mode, w.g)
+    h.reserve(w.mode, w.g)
+    out = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype, device=dev)
+    es = 4 if w.dtype == "fp32" else 2
+    in_bytes = (q.numel() + k.numel() + v.numel()) * es
+    flush = torch.empty(int(2 * L2_BYTES) // 4, dtype=torch.float32, device=dev) if in_bytes < L2_BYTES else None
+
+    def step():
+        h.forward(q, k, v, causal=w.mode, g=w.g, seed=w.seed, out=out)
+
+    for _ in range(max(3, warmup)):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    h.profile(True)
+    h.profile_read()
+    ms = timed_steps(step, steps, stream, flush)
+    h.profile(False)
+    ph = h.profile_read()
+    pk = peaks()
+    attn_ms = ph["attn_ms"] / max(1, ph["calls"])
+    rec = {"workload": name, "ms_per_layer": round(ms, 5), "tokens_per_s": w.B * w.H * w.T / (ms * 1e-3),
+           "steps": steps, "l2": "flushed before every step (inputs smaller than L2)" if flush is not None else
+           "inputs larger than L2 (no flush)",
+           "phases_ms": {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
+                         "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4), "attn_ms": round(attn_ms, 4)},
+           "roofline": attention_roofline(w, plan, attn_ms, pk),
+           "halving_roofline": halving_roofline(w, h, ph, pk),
+           "gpu_launches_per_step": plan["kernel_launches"]}
+    rec["approx_error"] = exact_reference_error(w, qc, kc, vc, out)
+    h.close()
+    del q, k, v, out, flush
+    torch.cuda.empty_cache()
+    return rec
+
+
 def main():
     a = args_()
     if a.impl == "reference":
@@ -374,13 +527,17 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     shard = Shard(W.WORKLOADS[a.workload], world, rank, a.shard)
     w = shard.local
-    q, k, v = (x.to(dev) for x in shard.inputs(w))
+    qc, kc, vc = shard.inputs(w)
+    q, k, v = (x.to(dev) for x in (qc, kc, vc))
     S = w.T if w.causal else w.S
     h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch,
                          device=local, shard=shard.abi)
     plan = h.plan(w.mode, w.g)
     h.reserve(w.mode, w.g)
     out = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype, device=dev)
+    es = 4 if w.dtype == "fp32" else 2
+    in_bytes = (q.numel() + k.numel() + v.numel()) * es
+    flush = torch.empty(int(2 * L2_BYTES) // 4, dtype=torch.float32, device=dev) if in_bytes < L2_BYTES else None
 
     def step():
         h.forward(q, k, v, causal=w.mode, g=w.g, seed=w.seed, out=out)
@@ -395,72 +552,28 @@ def main():
     h.profile(True)
     h.profile_read()
     stream = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(a.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    step_ms = timed_steps(step, a.steps, stream, flush)
     if dist:
         dist.barrier()
     clk = clocks.stop()
     h.profile(False)
     ph = h.profile_read()
-    ms = max_over_ranks(e0.elapsed_time(e1) / a.steps, dist, dev)
-    tokens = w.B * w.H * w.T
+    ms = max_over_ranks(step_ms, dist, dev)
     value = shard.whole_tokens / (ms * 1e-3)
 
-    # dominant kernel roofline: attention.  Bound by arithmetic intensity against the measured ridge
-    # (sustained bf16 FLOP/s over HBM bytes/s): tensor cores above it, HBM below it.
     pk = peaks()
-    flops, abytes, pairs = attention_work(w, plan)
     attn_ms = ph["attn_ms"] / max(1, ph["calls"])
-    ridge = pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
-    if flops / abytes >= ridge:
-        achieved, peak, unit, bound = flops / (attn_ms * 1e-3) / 1e12, pk["bf16_tflops_sustained"], "TFLOP/s", "tensor"
-        peak_kind = f"bf16 sustained ({pk['source']})"
-    else:
-        achieved, peak, unit, bound = abytes / (attn_ms * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm"
-        peak_kind = f"HBM copy ({pk['source']})"
-    roof = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-            "frac": round(achieved / peak, 4), "traffic": kernel_traffic("attention") if w.name == "express32k" else None,
-            "kernel": "attention", "peak_kind": peak_kind,
-            "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
-            "arithmetic_intensity": round(flops / abytes, 1), "avg_launch_ms": round(attn_ms, 4)}
-    # halving rooflines, HBM-bound by their algorithmic bytes -- every instance's n points read once
-    # and its n/2 survivors written once: 1.5 n (E+D) elements per instance.  Per step from the live
-    # per-step CUDA events; the headline is the step that takes longest (the dominant halving kernel),
-    # beside the whole halving phase (latency-bound merges included).
-    es = 4 if w.dtype == "fp32" else 2
-    sp = h.profile_steps()
-    steps_tab = []
-    for st in sp["steps"]:
-        sb = st["n_inst"] * 3 * st["n"] // 2 * (w.E + w.D) * es
-        sms = st["ms"] / max(1, sp["calls"])
-        steps_tab.append({"n": st["n"], "n_inst": st["n_inst"], "ms": round(sms, 4), "bytes": sb,
-                          "frac": round(sb / (sms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if sms > 0 else None})
-    hbytes = sum(t["bytes"] for t in steps_tab)
-    hms = (ph["thin_ms"] + ph["merge_ms"]) / max(1, ph["calls"])
-    top = max(steps_tab, key=lambda t: t["ms"]) if steps_tab else None
-    halving_roof = None
-    if top and top["ms"] > 0:
-        halving_roof = {"bound": "hbm", "achieved": round(top["bytes"] / (top["ms"] * 1e-3) / 1e9, 1),
-                        "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": top["frac"],
-                        "kernel": f"halving step n={top['n']} x {top['n_inst']} instances",
-                        "algorithmic_bytes_per_launch": top["bytes"], "avg_launch_ms": top["ms"],
-                        "traffic": kernel_traffic("halving_fused_n64") if (w.name == "express32k" and top["n"] == 64) else None,
-                        "all_steps": {"achieved": round(hbytes / (hms * 1e-3) / 1e9, 1) if hms > 0 else None,
-                                      "frac": round(hbytes / (hms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if hms > 0 else None,
-                                      "bytes": hbytes, "ms": round(hms, 4)},
-                        "steps": steps_tab}
+    roof = attention_roofline(w, plan, attn_ms, pk)
+    roof["traffic"] = kernel_traffic("attention") if w.name == "express32k" else None
+    halving_roof = halving_roofline(w, h, ph, pk)
     phases = {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
               "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4),
               "attn_ms": round(attn_ms, 4)}
 
     e2e = None
     if not a.no_e2e:
-        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        qh, kh, vh = (x.pin_memory() for x in (qc, kc, vc))
         oh = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype).pin_memory()
         for _ in range(2):
             h.forward_host(qh, kh, vh, oh, causal=w.mode, g=w.g, seed=w.seed)
@@ -474,7 +587,6 @@ def main():
         f1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(f0.elapsed_time(f1) / n_e2e, dist, dev)
-        es = 4 if w.dtype == "fp32" else 2
         e2e = {"value": shard.whole_tokens / (ems * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * es,
                "d2h_bytes_per_step": out.numel() * es, "ms_per_step": round(ems, 3)}
@@ -496,6 +608,20 @@ def main():
         except Exception as ex:  # report, do not fail the bench
             sdpa = f"unavailable: {type(ex).__name__}"
 
+    approx = None
+    per_workload = None
+    if rank == 0 and world == 1:
+        approx = exact_reference_error(w, qc, kc, vc, out)
+        if not a.no_per_workload:
+            h.close()
+            del q, k, v, out, flush
+            torch.cuda.empty_cache()
+            per_workload = {}
+            for name in ("tiny", "vit", "biggan", "express128k"):
+                if name != a.workload:
+                    per_workload[name] = measure_workload(TA, name, dev, 10 if name == "express128k" else 20,
+                                                          a.warmup)
+
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         cpu = cpu_baseline(w, list(range(w.H)))
@@ -511,9 +637,9 @@ def main():
             "config": {**config_of(W.WORKLOADS[a.workload]), "global_batch": shard.global_batch,
                        "parallelism": shard.parallelism, "heads_per_gpu": w.H},
             "ms_per_layer": ms, "phases_ms": phases, "roofline": roof, "halving_roofline": halving_roof,
-            "cpu_baseline": cpu, "e2e": e2e,
+            "approx_error": approx, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": plan["kernel_launches"] * a.steps, "clocks": clk, "exact_sdpa_ms": sdpa,
-            "workspace_bytes": plan["workspace_bytes"]}
+            "workspace_bytes": plan["workspace_bytes"], "per_workload": per_workload}
     print(json.dumps(line), flush=True)
 
 

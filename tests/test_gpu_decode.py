@@ -1,17 +1,27 @@
-"""Express decode cache (the pages' updatable weighted cache object) against the prefill.
+"""Express decode cache (the pages' updatable weighted cache object) against the fp64 oracle.
 
-Decoding the tokens of a sequence one at a time must reproduce the prefill: the same coresets
-(token indices, bit for bit: same Philox rounds, same points, same kernels) and, for every token t,
-the prefill's output row t within the bf16 / fp32 tolerance, since query t of the prefill attends
-to exactly the cache the decoder holds after token t.
+Decoding the tokens of a sequence one at a time must reproduce the oracle's Express prefill: token t
+attends to the cache held after token t (exact prefix, the nodes of the completed batches, its own
+batch), which is exactly what query t of the prefill sees.  Checked directly against
+``oracle.express``: every node of the cache (token indices, bit for bit), every decoded row within
+the bf16 / fp32 tolerance per (b,h) slice and per row, and every LSE.  The oracle replays the
+thinning in follow mode on the decision trace of a prefill of the same tokens (taken only where a
+decision is a near tie; any other disagreement fails).  The cache must also equal the library's
+prefill bit for bit (same Philox rounds, same points, same halving kernels).
 """
+import numpy as np
 import pytest
 import torch
 
 import thinned_softmax_attention_b200 as TA
 import workloads as W
+from oracle import express
 
 pytestmark = pytest.mark.gpu
+
+TOL = {"fp32": 1e-5, "bf16": 1e-2}
+ROW_TOL = {"fp32": 1e-4, "bf16": 2e-2}
+LSE_TOL = {"fp32": 1e-5, "bf16": 2e-3}
 
 
 @pytest.mark.parametrize("T,n_e,bsz,g,dtype,tiles", [
@@ -20,15 +30,20 @@ pytestmark = pytest.mark.gpu
     (700, 100, 96, 2, "bf16", False),    # batch not a power of 4 (subsample), trailing partial batch
     (300, 40, 16, 2, "fp32", False),     # batches stored whole (no thinning), fp32 path
 ])
-def test_decode_matches_prefill(T, n_e, bsz, g, dtype, tiles, monkeypatch):
+def test_decode_matches_oracle(T, n_e, bsz, g, dtype, tiles, monkeypatch):
     """Few (b,h) rows take the split-key decode kernels; `tiles` forces the query-tile kernels."""
     if tiles:
         monkeypatch.setenv("THIN_ATTN_DECODE_TILES", "1")
     E = D = 128 if dtype == "bf16" else 64
     w = W.Workload("decode", 1, 2, T, T, E, D, dtype, True, g, 9, 6, "rope", n_exact=n_e, batch=bsz)
-    q, k, v = (x.cuda() for x in W.make_qkv(w))
+    qc, kc, vc = W.make_qkv(w)
+    q, k, v = (x.cuda() for x in (qc, kc, vc))
     pre = TA.ThinAttention(w.B, T, T, w.H, E, D, w.torch_dtype, n_exact=n_e, batch=bsz)
-    ref = pre.forward(q, k, v, causal=True, g=g, seed=w.seed, return_coreset=True, return_lse=True)
+    pf = pre.forward(q, k, v, causal=True, g=g, seed=w.seed, return_coreset=True, return_trace=True)
+    torch.cuda.synchronize()
+    follow = TA.decode_trace(pf["trace"], pre.trace_layout(True, g))
+    ref = express(qc, kc, vc, n_e, bsz, g, w.seed, follow=follow, heads=(w.H, [0, 1]))
+    assert ref.stats.mismatches == 0
     cache = TA.ThinAttentionCache(w.B, w.H, E, D, w.torch_dtype, capacity=T, n_exact=n_e, batch=bsz, g=g, seed=w.seed)
     outs, lses = [], []
     for t in range(T):
@@ -38,13 +53,17 @@ def test_decode_matches_prefill(T, n_e, bsz, g, dtype, tiles, monkeypatch):
         lses.append(lse)
     cache.check()
     assert len(cache) == T
-    assert torch.equal(cache.nodes(), ref["coreset"])
-    o = torch.cat(outs, dim=1).float()
-    r = ref["out"].float()
-    err = ((o - r).abs().amax(dim=(1, 3)) / r.abs().amax(dim=(1, 3))).max().item()
-    assert err <= (1e-2 if dtype == "bf16" else 1e-5), err
-    lse = torch.stack(lses, dim=2)
-    assert (lse - ref["lse"]).abs().max().item() <= (2e-3 if dtype == "bf16" else 1e-5)
+    nodes = cache.nodes().cpu().numpy()
+    assert np.array_equal(nodes, ref.coreset)
+    assert torch.equal(cache.nodes(), pf["coreset"])
+    o = torch.cat(outs, dim=1).float().cpu().numpy()
+    d = np.abs(o - ref.out)
+    slice_err = (d.max(axis=(1, 3)) / np.abs(ref.out).max(axis=(1, 3))).max()
+    row_err = (d.max(axis=3) / np.abs(ref.out).max(axis=3)).max()
+    assert slice_err <= TOL[dtype], slice_err
+    assert row_err <= ROW_TOL[dtype], row_err
+    lse = torch.stack(lses, dim=2).cpu().numpy()
+    assert np.abs(lse - ref.lse).max() <= LSE_TOL[dtype]
 
 
 def test_cache_refuses_tokens_beyond_capacity():

@@ -46,12 +46,15 @@ def _call(Ks, Vs, seed, round_id):
     return Ko, Vo, idx, bits
 
 
-@pytest.mark.parametrize("S,g,E,D,dtype", [(64, 2, 64, 128, "bf16"), (256, 3, 128, 128, "bf16"),
-                                           (128, 3, 64, 64, "fp32")])
-def test_noalloc_matches_forward_twice(S, g, E, D, dtype):
+@pytest.mark.parametrize("S,g,E,D,dtype,B,H", [
+    (64, 2, 64, 128, "bf16", 2, 3), (256, 3, 128, 128, "bf16", 2, 3), (128, 3, 64, 64, "fp32", 2, 3),
+    (1024, 4, 64, 64, "bf16", 2, 3),     # 6 sets of 1024 points: 6 MiB of pair differences
+    (2048, 5, 64, 128, "bf16", 1, 3),    # 3 sets of 2048 points: 12 MiB, near the scratch's limit
+])
+def test_noalloc_matches_forward_twice(S, g, E, D, dtype, B, H):
     # S with 4^g < S <= 4^(g+1) and S = 4L: KH-Compress is a single halving of all S keys of each
     # (b,h) with Philox round id 1 and counter word b*H+h -- the instance index below.
-    w = W.Workload("noalloc", 2, 3, 16, S, E, D, dtype, False, g, 5, 8, "iid")
+    w = W.Workload("noalloc", B, H, 16, S, E, D, dtype, False, g, 5, 8, "iid")
     q, k, v = (x.cuda() for x in W.make_qkv(w))
     h = TA.ThinAttention(w.B, w.T, S, w.H, E, D, w.torch_dtype)
     plan = h.plan(False, g)
