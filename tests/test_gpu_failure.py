@@ -17,7 +17,12 @@ import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_reports_timeout_and_context_survives():
+@pytest.mark.parametrize("kernel", ["two_cta", "ping_pong"])
+def test_bounded_wait_reports_timeout_and_context_survives(kernel, monkeypatch):
+    """Both persistent attention kernels: the two-CTA one (this shape's default) and the ping-pong
+    one (forced), whose withheld key tile is the first of the K ring."""
+    if kernel == "ping_pong":
+        monkeypatch.setenv("THIN_ATTN_PP", "1")
     w = W.WORKLOADS["express32k"].with_(H=2, n_exact=256, batch=256)
     q, k, v = (x.cuda() for x in W.make_qkv(w, T=1024))
     h = TA.ThinAttention(w.B, 1024, 1024, w.H, w.E, w.D, w.torch_dtype, n_exact=256, batch=256)

@@ -300,20 +300,24 @@ def test_fused_and_three_launch_halving_agree(case, monkeypatch):
         assert torch.equal(res[0][key], res[1][key]), key
 
 
-@pytest.mark.parametrize("name", ["vit", "express", "express_a"])
+@pytest.mark.parametrize("name", ["vit", "express", "express_a", "express_ragged"])
 def test_attention_launch_forms_agree(name, monkeypatch):
-    """The persistent attention kernel (items from a work counter), its one-CTA-per-tile form, and
-    the persistent kernel launched as several dependent waves on a side stream (each launch takes
-    and resets the same counter) run the same per-tile arithmetic: outputs and LSE are bit-identical."""
+    """The ping-pong kernel (two query tiles of a head against one K/V stream, one CTA per SM), the
+    two-CTA persistent kernel (items from a work counter), its one-CTA-per-tile form, and the
+    persistent kernel launched as several dependent waves on a side stream (each launch takes and
+    resets the same counter) run the same per-tile arithmetic: outputs and LSE are bit-identical.
+    ViT's 25 query tiles per head leave one tile unpaired; the ragged Express shape has batches of
+    three tiles, so pairs cross from the exact phase into batches and some tiles run alone."""
     w = {"vit": W.WORKLOADS["vit"].with_(B=8),
          "express": W.WORKLOADS["express32k"].with_(T=8192, H=4),
-         "express_a": W.WORKLOADS["express32k_a"].with_(T=8192, H=4)}[name]
+         "express_a": W.WORKLOADS["express32k_a"].with_(T=8192, H=4),
+         "express_ragged": W.WORKLOADS["express32k"].with_(T=3000, H=3, n_exact=200, batch=300)}[name]
     S = w.T if w.causal else w.S
     q, k, v = (x.cuda() for x in W.make_qkv(w))
-    forms = [{}, {"THIN_ATTN_TC2_PER_TILE": "1"}, {"THIN_ATTN_OVERLAP": "1"}]
+    forms = [{"THIN_ATTN_PP": "1"}, {"THIN_ATTN_TC2P": "1"}, {"THIN_ATTN_TC2_PER_TILE": "1"}, {"THIN_ATTN_OVERLAP": "1"}]
     res = []
     for env in forms:
-        for key in ("THIN_ATTN_TC2_PER_TILE", "THIN_ATTN_OVERLAP"):
+        for key in ("THIN_ATTN_PP", "THIN_ATTN_TC2P", "THIN_ATTN_TC2_PER_TILE", "THIN_ATTN_OVERLAP"):
             if key in env:
                 monkeypatch.setenv(key, env[key])
             else:

@@ -142,7 +142,9 @@ struct AttnTables {
   std::vector<AttnTile> tiles;
   std::vector<AttnSeg> segs;
   std::vector<AttnWave> waves;
-  size_t tiles_off = 0, segs_off = 0;
+  std::vector<int2> pairs;   // tile pairs of the ping-pong attention kernel (AttnArgs::pairs)
+  double key_tiles_per_tile = 0;   // mean 128-key tiles a query tile attends to
+  size_t tiles_off = 0, segs_off = 0, pairs_off = 0;
 };
 
 struct Plan {
@@ -344,6 +346,42 @@ void build_attn_tables(const thin_attn_config& cf, const Plan& p, int QT, AttnTa
       }
       t.segs.push_back({SEG_TOKENS, (int)start, q0 + ql - (int)start, 1, 0.f, 0});
       t.tiles.push_back({q0, ql, seg0, (int)t.segs.size() - seg0});
+    }
+  }
+}
+
+// Whether tile A's key tiles are the first key tiles of tile B's: the same segments, except that
+// A's last one may stop earlier in B's segment of the same place (the causal in-batch keys of two
+// neighbouring query tiles).  Such a pair shares one stream of K/V tiles.
+bool key_tiles_nest(const AttnTables& t, const AttnTile& A, const AttnTile& B) {
+  if (A.nseg < 1 || A.nseg > B.nseg) return false;
+  for (int i = 0; i < A.nseg; ++i) {
+    const AttnSeg& x = t.segs[A.seg0 + i];
+    const AttnSeg& y = t.segs[B.seg0 + i];
+    if (x.kind != y.kind || x.first != y.first || x.causal != y.causal || x.logw != y.logw) return false;
+    if (i + 1 < A.nseg ? x.len != y.len : x.len > y.len) return false;
+  }
+  return true;
+}
+
+// Pair neighbouring tiles (i, i+1) whose key lists nest, in either order; a tile left over runs alone.
+void build_pairs(AttnTables& t) {
+  t.pairs.clear();
+  const int n = (int)t.tiles.size();
+  int64_t kt = 0;
+  for (const AttnTile& tl : t.tiles)
+    for (int s = 0; s < tl.nseg; ++s) kt += (t.segs[tl.seg0 + s].len + 127) / 128;
+  t.key_tiles_per_tile = n ? (double)kt / n : 0.0;
+  for (int i = 0; i < n;) {
+    if (i + 1 < n && key_tiles_nest(t, t.tiles[i], t.tiles[i + 1])) {
+      t.pairs.push_back(make_int2(i, i + 1));
+      i += 2;
+    } else if (i + 1 < n && key_tiles_nest(t, t.tiles[i + 1], t.tiles[i])) {
+      t.pairs.push_back(make_int2(i + 1, i));
+      i += 2;
+    } else {
+      t.pairs.push_back(make_int2(-1, i));
+      i += 1;
     }
   }
 }
@@ -606,6 +644,7 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
   if (attention_tc_supported(cf.dtype, cf.E, cf.D)) {
     build_attn_tables(cf, *p, attention_tc_tile_rows(), p->tc);
     build_waves(cf, *p, p->tc);
+    build_pairs(p->tc);
   }
   // memory layout: tables first, then buffers
   size_t off = 0;
@@ -618,6 +657,8 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
     off = align256(off + t->tiles.size() * sizeof(AttnTile));
     t->segs_off = off;
     off = align256(off + t->segs.size() * sizeof(AttnSeg));
+    t->pairs_off = off;
+    off = align256(off + t->pairs.size() * sizeof(int2));
   }
   const size_t es = elt(cf);
   auto place = [&](BufSpec& b) {
@@ -672,7 +713,8 @@ thin_attn_status materialise(thin_attn_s* h, Plan* p) {
   for (AttnTables* t : {&p->simt, &p->tc}) {
     if (!t->tiles.empty()) std::memcpy(host.data() + t->tiles_off, t->tiles.data(), t->tiles.size() * sizeof(AttnTile));
     if (!t->segs.empty()) std::memcpy(host.data() + t->segs_off, t->segs.data(), t->segs.size() * sizeof(AttnSeg));
-    tbl_end = std::max(tbl_end, t->segs_off + t->segs.size() * sizeof(AttnSeg));
+    if (!t->pairs.empty()) std::memcpy(host.data() + t->pairs_off, t->pairs.data(), t->pairs.size() * sizeof(int2));
+    tbl_end = std::max(tbl_end, t->pairs_off + t->pairs.size() * sizeof(int2));
   }
   if (tbl_end) {
     e = cudaMemcpy(mem, host.data(), tbl_end, cudaMemcpyHostToDevice);
@@ -847,6 +889,19 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   aa.inject_timeout = std::getenv("THIN_ATTN_INJECT_WAIT_TIMEOUT") != nullptr;
   aa.tiles = (const AttnTile*)(base_of(p) + tab.tiles_off);
   aa.segs = (const AttnSeg*)(base_of(p) + tab.segs_off);
+  // The ping-pong kernel (tile pairs sharing one K/V stream) pays a Q reload and a pipeline refill
+  // at every pair it starts and gains in every key tile after that, so it runs where a query tile
+  // attends to kPpMinKeyTiles key tiles or more on average (Express 128K: 28; Express 32K: 15, ViT
+  // 2 stay on the two-CTA kernel, measured faster there).  THIN_ATTN_PP / THIN_ATTN_TC2P force
+  // one form or the other.
+  constexpr double kPpMinKeyTiles = 24.0;
+  const bool want_pp = std::getenv("THIN_ATTN_TC2P") == nullptr &&
+                       (std::getenv("THIN_ATTN_PP") != nullptr || tab.key_tiles_per_tile >= kPpMinKeyTiles);
+  if (!side && use_tc_attn && want_pp && !tab.pairs.empty()) {
+    aa.pairs = (const int2*)(base_of(p) + tab.pairs_off);
+    aa.pair0 = 0;
+    aa.n_pairs = (int)tab.pairs.size();
+  }
   size_t next_wave = 0, dep_i = 0;
   auto launch_waves_after = [&](int step) -> thin_attn_status {
     while (next_wave < waves.size() && waves[next_wave].after <= step) {

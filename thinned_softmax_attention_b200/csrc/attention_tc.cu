@@ -14,11 +14,13 @@
 //              O += P V into TMEM cols 256..256+D; also owns the TMEM allocation
 // Every wait on an mbarrier is bounded; a CTA that gives up records the failure in the status
 // word and leaves through the normal exit path (TMEM freed, its TMA copies landed).
+#include <algorithm>
 #include <cstdlib>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
+#include "thin_attn.h"
 
 namespace thin {
 
@@ -375,21 +377,20 @@ struct Tc2Layout {
 };
 
 
-// Softmax of one key tile of the two-CTA kernel for the thread's row: reads S (TMEM columns
-// 0..127) twice -- row max, then P = 2^(s scale log2e + log2 w - m) as bf16 written over the S
-// columns already read (16 columns per 32 read) -- and rescales O lazily (warp-wide TMEM round
-// trip when some row's max grew by more than 2^8).  MASKED: keys c > lim are invisible.
+// Softmax of one key tile for the thread's row (TMEM address ts of its 128 S columns, to of its O
+// columns): reads S twice -- row max, then P = 2^(s scale log2e + log2 w - m) as bf16 written over
+// the S columns already read (16 columns per 32 read) -- and rescales O lazily (warp-wide TMEM
+// round trip when some row's max grew by more than 2^8).  MASKED: keys c > lim are invisible.
 template <bool MASKED, int D>
-__device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, int lim, float sl2e, float lw2,
-                                             int it, float& m_used, float& l, uint64_t* p_half) {
-  constexpr uint32_t O_COL = 128;
+__device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int lim, float sl2e, float lw2, int it,
+                                             float& m_used, float& l, uint64_t* p_half) {
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   // row max: two 32-column loads in flight per wait
 #pragma unroll
   for (int c2 = 0; c2 < BN / 64; ++c2) {
     float z[2][32];
-    tmem_ld32(tmem + lane_base + c2 * 64, z[0]);
-    tmem_ld32(tmem + lane_base + c2 * 64 + 32, z[1]);
+    tmem_ld32(ts + c2 * 64, z[0]);
+    tmem_ld32(ts + c2 * 64 + 32, z[1]);
     tmem_ld_wait();
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -420,11 +421,11 @@ __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, 
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       float o[32];
-      tmem_ld32(tmem + lane_base + O_COL + c * 32, o);
+      tmem_ld32(to + c * 32, o);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i) o[i] *= corr;
-      tmem_st32(tmem + lane_base + O_COL + c * 32, o);
+      tmem_st32(to + c * 32, o);
     }
   }
   const float off = m_used == -INFINITY ? 0.f : lw2 - m_used;
@@ -434,11 +435,11 @@ __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, 
   float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   // 32 columns at a time, the next 32 loading while these are exponentiated
   float zb[2][32];
-  tmem_ld32(tmem + lane_base, zb[0]);
+  tmem_ld32(ts, zb[0]);
   tmem_ld_wait();
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
-    if (c + 1 < BN / 32) tmem_ld32(tmem + lane_base + (c + 1) * 32, zb[(c + 1) & 1]);
+    if (c + 1 < BN / 32) tmem_ld32(ts + (c + 1) * 32, zb[(c + 1) & 1]);
     const float* z = zb[c & 1];
     uint32_t pk[16];
 #pragma unroll
@@ -455,7 +456,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t tmem, uint32_t lane_base, 
       const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
       pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
     }
-    tmem_st16(tmem + lane_base + c * 16, pk);
+    tmem_st16(ts + c * 16, pk);
     if (c == BN / 64 - 1) {
       // P of the first half of the keys is in place: the MMA warp starts its half of PV
       tmem_st_wait();
@@ -639,8 +640,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
         const bool causal = sg.kind == SEG_TOKENS && sg.causal;
         const bool masked = nvalid < BN || (causal && kt0 + BN - 1 > tile.q0);
         const int lim = min(nvalid - 1, causal ? tq - kt0 : BN - 1);
-        if (masked) softmax_tile<true, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
-        else softmax_tile<false, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
+        if (masked) softmax_tile<true, D>(tmem + lane_base, tmem + lane_base + 128, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
+        else softmax_tile<false, D>(tmem + lane_base, tmem + lane_base + 128, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);
@@ -933,8 +934,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
           const bool causal = sg.kind == SEG_TOKENS && sg.causal;
           const bool masked = nvalid < BN || (causal && kt0 + BN - 1 > tile.q0);
           const int lim = min(nvalid - 1, causal ? tq - kt0 : BN - 1);
-          if (masked) softmax_tile<true, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
-          else softmax_tile<false, D>(tmem, lane_base, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
+          if (masked) softmax_tile<true, D>(tmem + lane_base, tmem + lane_base + 128, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
+          else softmax_tile<false, D>(tmem + lane_base, tmem + lane_base + 128, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(p_full);
@@ -1000,6 +1001,545 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Ping-pong form (E, D <= 128): one persistent CTA per SM runs two query tiles of one (b,h) at a
+// time, tile A and tile B, against a single stream of K/V tiles.  The host pairs tiles whose key
+// lists nest: A's key tiles are the first n_A key tiles of B's (two neighbouring tiles of one
+// Express batch, the exact phase, or any two tiles of a Thinformer head), so every K/V tile is
+// loaded once for both; the K and V rings fill the shared memory beside the two Q tiles.
+//   TMEM (512 columns): S_A / P_A 0..127, S_B / P_B 128..255, O_A 256..383, O_B 384..511.
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B (thread = query row = TMEM lane)
+//   warp 8     TMA producer: work items, Q_A and Q_B per item, K per key tile into the K ring
+//   warp 10    TMA producer: V per key tile into the V ring; warp 11 idle
+// After set-up the softmax warpgroups take 208 registers per thread and warps 8-11 give theirs down
+// to 88, so a softmax thread holds its row of S and reads it from TMEM once per key tile.
+//   warp 9     MMA issuer: per key tile j, PV_A(j), S_A(j+1), PV_B(j), S_B(j+1) -- while one
+//              softmax warpgroup turns its S into P, the tensor pipe runs the other tile's PV and S
+// The per-row arithmetic is softmax_tile's, as in the two-CTA kernels, so outputs equal theirs bit
+// for bit.
+// Items (tile pair, (b,h)) come from the work counter in the handle's status buffer, heaviest
+// pairs first, through a two-slot ring whose slots are released by every reader (item_empty).
+template <int E, int D>
+struct PpLayout {
+  static constexpr int EC = E / 64, DC = D / 64;
+  static constexpr uint32_t Q_BYTES = BM * E * 2;
+  static constexpr uint32_t K_BYTES = BN * E * 2;
+  static constexpr uint32_t V_BYTES = BN * D * 2;
+  // K and V rings as deep as the shared memory beside the two Q tiles allows (227 KB per CTA, less
+  // barriers and alignment slack), at most 4 stages each: E = D = 128 gives 3 K and 2 V stages
+  static constexpr uint32_t AVAIL = 232448 - 2048 - 2 * Q_BYTES;
+  static constexpr int NK = (AVAIL - 2 * V_BYTES) / K_BYTES < 4 ? (int)((AVAIL - 2 * V_BYTES) / K_BYTES) : 4;
+  static constexpr int NV = (AVAIL - NK * K_BYTES) / V_BYTES < 4 ? (int)((AVAIL - NK * K_BYTES) / V_BYTES) : 4;
+  static_assert(NK >= 2 && NV >= 2, "two stages of K and V at least");
+  static constexpr uint32_t OFF_QB = Q_BYTES;
+  static constexpr uint32_t OFF_K = 2 * Q_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + NK * K_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + NV * V_BYTES;
+  static constexpr uint32_t BYTES = OFF_BAR + 256 + 1024;
+  static_assert(BYTES <= 232448, "shared memory per CTA");
+};
+
+// softmax_tile with the thread's whole row of S in registers (one TMEM read per tile; the
+// ping-pong kernel's softmax threads hold 208 registers): the same arithmetic in the same order,
+// so the same P, row sum and rescale decisions.
+template <bool MASKED, int D>
+__device__ __forceinline__ void softmax_tile_reg(uint32_t ts, uint32_t to, int lim, float sl2e, float lw2, int it,
+                                                 float& m_used, float& l, uint64_t* p_half) {
+  float z[BN];
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) tmem_ld32(ts + c * 32, z + c * 32);
+  tmem_ld_wait();
+  if (MASKED) {
+#pragma unroll
+    for (int i = 0; i < BN; ++i) z[i] = i <= lim ? z[i] : -INFINITY;
+  }
+  float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int i = 0; i < BN; i += 8) {
+    mx4[0] = fmax3(mx4[0], z[i], z[i + 1]);
+    mx4[1] = fmax3(mx4[1], z[i + 2], z[i + 3]);
+    mx4[2] = fmax3(mx4[2], z[i + 4], z[i + 5]);
+    mx4[3] = fmax3(mx4[3], z[i + 6], z[i + 7]);
+  }
+  const float smax = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+  const float mx = smax == -INFINITY ? -INFINITY : fmaf(smax, sl2e, lw2);
+  const bool grow = mx > m_used + 8.f;
+  float corr = 1.f;
+  if (grow) {
+    corr = ex2_approx(m_used - mx);
+    l *= corr;
+    m_used = mx;
+  }
+  if (it > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      tmem_ld32(to + c * 32, o);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] *= corr;
+      tmem_st32(to + c * 32, o);
+    }
+  }
+  const float off = m_used == -INFINITY ? 0.f : lw2 - m_used;
+  const float2 sl2e2 = make_float2(sl2e, sl2e), off2 = make_float2(off, off);
+  float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float2 t = __ffma2_rn(make_float2(z[c * 32 + 2 * e], z[c * 32 + 2 * e + 1]), sl2e2, off2);
+      const float p0 = ex2_approx(t.x);
+      const float p1 = ex2_approx(t.y);
+      ls2[e & 1] = __fadd2_rn(ls2[e & 1], make_float2(p0, p1));
+      const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
+      pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+    }
+    tmem_st16(ts + c * 16, pk);
+    if (c == BN / 64 - 1) {
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_half);
+    }
+  }
+  l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
+}
+
+// Registers per thread of the ping-pong kernel after its reallocation: the two softmax warpgroups
+// take kPpSoftmaxRegs, the producer / MMA warpgroup keeps kPpOtherRegs; the sum fits the launch's
+// 384 x kPpLaunchRegs (checked on the host before every launch).
+constexpr int kPpLaunchRegs = 168, kPpSoftmaxRegs = 208, kPpOtherRegs = 88;
+static_assert(256 * kPpSoftmaxRegs + 128 * kPpOtherRegs <= 384 * kPpLaunchRegs, "register split");
+
+template <int E, int D>
+__global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a,
+                                                         int* status) {
+  using Lay = PpLayout<E, D>;
+  constexpr int NK = Lay::NK, NV = Lay::NV;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQA = smem;
+  uint8_t* sQB = smem + Lay::OFF_QB;
+  uint8_t* sK = smem + Lay::OFF_K;
+  uint8_t* sV = smem + Lay::OFF_V;
+  uint64_t* bars = (uint64_t*)(smem + Lay::OFF_BAR);
+  uint64_t* q_full = bars + 0;       // Q_A (if used) and Q_B of the item landed
+  uint64_t* q_empty = bars + 1;      // the item's last S MMA has read Q (commit)
+  uint64_t* k_full = bars + 2;            // [NK]
+  uint64_t* k_empty = k_full + NK;        // [NK] S_A and S_B of the tile have read K (commit)
+  uint64_t* v_full = k_empty + NK;        // [NV]
+  uint64_t* v_empty = v_full + NV;        // [NV] PV_A and PV_B of the tile have read V (commit)
+  uint64_t* s_full = v_empty + NV;        // [2] S_x ready (commit after S_x)
+  uint64_t* p_half = s_full + 2;          // [2] P_x of keys 0..63 written (128 threads)
+  uint64_t* p_full = p_half + 2;          // [2] P_x of all keys written (128 threads)
+  uint64_t* pv_done = p_full + 2;         // [2] the item's last PV_x done (commit)
+  uint64_t* o_empty = pv_done + 2;        // [2] O_x read out of TMEM (128 threads)
+  uint64_t* item_full = o_empty + 2;      // [2] ring slot written (K producer)
+  uint64_t* item_empty = item_full + 2;   // [2] ring slot read by the V producer, the MMA thread and
+                                          //     all 256 softmax threads
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  __shared__ volatile int where_s;
+  __shared__ int item_s;
+  __shared__ int item_ring[2];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = a.n_pairs * a.B * a.H;
+  int* sched = status + 4;
+
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    where_s = 0;
+    item_s = -1;
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full + x, 1);
+      mbar_init(p_half + x, 128);
+      mbar_init(p_full + x, 128);
+      mbar_init(pv_done + x, 1);
+      mbar_init(o_empty + x, 128);
+      mbar_init(item_full + x, 1);
+      mbar_init(item_empty + x, 258);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 9) tmem_alloc(&tmem_base_s, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort = &abort_s;
+  // item j: pair n_pairs - 1 - j % n_pairs (the heaviest first) of (b,h) j / n_pairs
+  auto pair_of = [&](int j) { return a.pairs[a.pair0 + a.n_pairs - 1 - j % a.n_pairs]; };
+  auto tiles_of = [&](int t) { return t < 0 ? 0 : count_key_tiles(a, a.tiles[t]); };
+
+  if (warp >= 8) {
+  regs_dec<kPpOtherRegs>();   // the whole warpgroup 8-11
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer: work items, Q and K
+    if (lane == 0) {
+      int g = 0, r = 0;
+      bool ok = true;
+      // the CTA's next item is taken one item ahead, and its Q tiles and first key tile are
+      // prefetched into L2 while the current item runs: Q rows are read once, from HBM, and
+      // their load would otherwise stall the tensor pipe at every item boundary
+      auto prefetch = [&](int jn) {
+        const int2 pn = pair_of(jn);
+        const int bhn = jn / a.n_pairs, bn = bhn / a.H, hn = bhn % a.H;
+        const AttnTile tn = a.tiles[pn.y];
+        for (int c = 0; c < Lay::EC; ++c) {
+          tma_prefetch_3d(&maps.q, c * 64, hn, bn * a.T + tn.q0);
+          if (pn.x >= 0) tma_prefetch_3d(&maps.q, c * 64, hn, bn * a.T + a.tiles[pn.x].q0);
+        }
+        if (tn.nseg > 0) {
+          const AttnSeg sg = a.segs[tn.seg0];
+          if (sg.kind == SEG_TOKENS) {
+            for (int c = 0; c < Lay::EC; ++c) tma_prefetch_3d(&maps.k, c * 64, hn, bn * a.L + sg.first);
+            for (int c = 0; c < Lay::DC; ++c) tma_prefetch_3d(&maps.v, c * 64, hn, bn * a.L + sg.first);
+          } else {
+            const int row = (bhn * a.n_slots + sg.first) * a.slot_rows;
+            for (int c = 0; c < Lay::EC; ++c) tma_prefetch_2d(&maps.ck, c * 64, row);
+            for (int c = 0; c < Lay::DC; ++c) tma_prefetch_2d(&maps.cv, c * 64, row);
+          }
+        }
+      };
+      int j_next = atomicAdd(sched, 1);
+      for (;; ++r) {
+        const int slot = r & 1;
+        if (r >= 2 && !mbar_wait(item_empty + slot, ((r >> 1) - 1) & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 11000 + min(r, 999));
+          ok = false;
+        }
+        if (ok && r > 0 && !mbar_wait(q_empty, (r - 1) & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 9000 + min(r, 999));
+          ok = false;
+        }
+        const int j = ok ? j_next : n_items;
+        item_ring[slot] = j < n_items ? j : -1;
+        mbar_arrive(item_full + slot);
+        if (j >= n_items) break;
+        j_next = atomicAdd(sched, 1);
+        if (j_next < n_items) prefetch(j_next);
+        const int2 pr = pair_of(j);
+        const int bh = j / a.n_pairs, b = bh / a.H, h = bh % a.H;
+        const AttnTile tB = a.tiles[pr.y];
+        const bool useA = tiles_of(pr.x) > 0;
+        mbar_expect_tx(q_full, (useA ? 2u : 1u) * Lay::Q_BYTES);
+        if (useA) {
+          const int q0 = a.tiles[pr.x].q0;
+#pragma unroll
+          for (int c = 0; c < Lay::EC; ++c) tma_load_3d(sQA + c * 16384, &maps.q, q_full, c * 64, h, b * a.T + q0);
+        }
+#pragma unroll
+        for (int c = 0; c < Lay::EC; ++c) tma_load_3d(sQB + c * 16384, &maps.q, q_full, c * 64, h, b * a.T + tB.q0);
+        for (int si = 0; si < tB.nseg && ok; ++si) {
+          const AttnSeg sg = a.segs[tB.seg0 + si];
+          const bool tok = sg.kind == SEG_TOKENS;
+          for (int j0 = 0; j0 < sg.len; j0 += BN, ++g) {
+            const int row = tok ? b * a.L + sg.first + j0 : (bh * a.n_slots + sg.first) * a.slot_rows + j0;
+            const int st = g % NK;
+            if (g >= NK && !mbar_wait(k_empty + st, ((g / NK) - 1) & 1, abort)) {
+              ok = false;
+              atomicCAS((int*)&where_s, 0, 1000 + min(g, 999));
+              break;
+            }
+            if (a.inject_timeout && g == 0 && blockIdx.x == 0) continue;   // test hook: K(0) withheld
+            mbar_expect_tx(k_full + st, Lay::K_BYTES);
+#pragma unroll
+            for (int c = 0; c < Lay::EC; ++c) {
+              if (tok) tma_load_3d(sK + st * Lay::K_BYTES + c * 16384, &maps.k, k_full + st, c * 64, h, row);
+              else tma_load_2d(sK + st * Lay::K_BYTES + c * 16384, &maps.ck, k_full + st, c * 64, row);
+            }
+          }
+        }
+        if (!ok) break;   // abort is set: every other role's next wait returns at once
+      }
+      // never leave with a copy in flight into this CTA's shared memory: wait (bounded) for the
+      // last fill of every K stage and for the last Q load
+      for (int st = 0; st < NK; ++st) {
+        const int last = g - 1 - ((g - 1 - st) % NK + NK) % NK;   // largest g' < g with g' % NK == st
+        if (last < 0) continue;
+        const long long t0 = clock64();
+        while (!mbar_try_wait(k_full + st, (last / NK) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+      if (r > 0) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(q_full, (r - 1) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ TMA producer: V, on its own so that
+    // a K load never waits for a V stage to drain
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int slot = r & 1;
+        if (!mbar_wait(item_full + slot, (r >> 1) & 1, abort)) break;
+        const int j = item_ring[slot];
+        mbar_arrive(item_empty + slot);
+        if (j < 0) break;
+        const int2 pr = pair_of(j);
+        const int bh = j / a.n_pairs, b = bh / a.H, h = bh % a.H;
+        const AttnTile tB = a.tiles[pr.y];
+        for (int si = 0; si < tB.nseg && ok; ++si) {
+          const AttnSeg sg = a.segs[tB.seg0 + si];
+          const bool tok = sg.kind == SEG_TOKENS;
+          for (int j0 = 0; j0 < sg.len; j0 += BN, ++g) {
+            const int row = tok ? b * a.L + sg.first + j0 : (bh * a.n_slots + sg.first) * a.slot_rows + j0;
+            const int st = g % NV;
+            if (g >= NV && !mbar_wait(v_empty + st, ((g / NV) - 1) & 1, abort)) {
+              ok = false;
+              atomicCAS((int*)&where_s, 0, 2000 + min(g, 999));
+              break;
+            }
+            mbar_expect_tx(v_full + st, Lay::V_BYTES);
+#pragma unroll
+            for (int c = 0; c < Lay::DC; ++c) {
+              if (tok) tma_load_3d(sV + st * Lay::V_BYTES + c * 16384, &maps.v, v_full + st, c * 64, h, row);
+              else tma_load_2d(sV + st * Lay::V_BYTES + c * 16384, &maps.cv, v_full + st, c * 64, row);
+            }
+          }
+        }
+      }
+      for (int st = 0; st < NV; ++st) {
+        const int last = g - 1 - ((g - 1 - st) % NV + NV) % NV;
+        if (last < 0) continue;
+        const long long t0 = clock64();
+        while (!mbar_try_wait(v_full + st, (last / NV) & 1) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IQK = idesc_bf16(BM, BN, false);
+      constexpr uint32_t IPV = idesc_bf16(BM, D, true);
+      const uint32_t qa = smem_u32(sQA), qb = smem_u32(sQB), ka = smem_u32(sK), va = smem_u32(sV);
+      int g = 0, gx[2] = {0, 0}, ix[2] = {0, 0};
+      bool ok = true;
+      auto fail = [&](int code, int at) {
+        ok = false;
+        atomicCAS((int*)&where_s, 0, code + min(at, 999));
+      };
+      // S_x = Q_x K^T of ring position gg into TMEM columns 128 x
+      auto issue_s = [&](int x, int gg) {
+        const uint32_t q = x ? qb : qa;
+        const uint32_t kb = ka + (gg % NK) * Lay::K_BYTES;
+#pragma unroll
+        for (int k = 0; k < E / 16; ++k) {
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_bf16(tmem + 128 * x, sw128_desc(q + off, 16, 1024), sw128_desc(kb + off, 16, 1024), IQK, k > 0);
+        }
+        umma_commit(s_full + x);
+      };
+      // O_x += P_x V of ring position gg, in two halves over the keys (the first once P of keys 0..63
+      // is written); the first of an item waits for the previous item's O_x to be read out
+      auto issue_pv = [&](int x, int gg, bool first) -> bool {
+        const int st = gg % NV;
+        if (!mbar_wait(p_half + x, gx[x] & 1, abort) || !mbar_wait(v_full + st, (gg / NV) & 1, abort) ||
+            (first && ix[x] > 0 && !mbar_wait(o_empty + x, (ix[x] - 1) & 1, abort))) {
+          fail(5000, gg);
+          return false;
+        }
+        tc_fence_after();
+        const uint32_t vb = va + st * Lay::V_BYTES;
+#pragma unroll
+        for (int k = 0; k < BN / 32; ++k)
+          umma_bf16_tmem_a(tmem + 256 + 128 * x, tmem + 128 * x + k * 8, sw128_desc(vb + k * 2048, 16384, 1024), IPV,
+                           (!first || k > 0) ? 1u : 0u);
+        if (!mbar_wait(p_full + x, gx[x] & 1, abort)) {
+          fail(7000, gg);
+          return false;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = BN / 32; k < BN / 16; ++k)
+          umma_bf16_tmem_a(tmem + 256 + 128 * x, tmem + 128 * x + k * 8, sw128_desc(vb + k * 2048, 16384, 1024), IPV,
+                           1u);
+        ++gx[x];
+        return true;
+      };
+      auto wait_k = [&](int gg) -> bool {
+        if (!mbar_wait(k_full + gg % NK, (gg / NK) & 1, abort)) {
+          fail(3000, gg);
+          return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      for (int r = 0; ok; ++r) {
+        const int slot = r & 1;
+        if (!mbar_wait(item_full + slot, (r >> 1) & 1, abort)) break;
+        const int j = item_ring[slot];
+        mbar_arrive(item_empty + slot);
+        if (j < 0) break;
+        const int2 pr = pair_of(j);
+        const int n_a = tiles_of(pr.x), n_b = tiles_of(pr.y);
+        if (!mbar_wait(q_full, r & 1, abort)) {
+          fail(4000, r);
+          break;
+        }
+        if (n_b == 0) {
+          umma_commit(q_empty);
+          continue;
+        }
+        if (!wait_k(g)) break;
+        if (n_a > 0) issue_s(0, g);
+        issue_s(1, g);
+        umma_commit(k_empty + g % NK);
+        if (n_b == 1) umma_commit(q_empty);
+        for (int jj = 0; jj < n_b && ok; ++jj) {
+          const int gg = g + jj;
+          // S_x(jj + 1) overwrites the columns PV_x(jj) reads P_x from: tcgen05.mma ops issued by one
+          // thread execute in issue order, and the commit after S_x(jj + 1) tracks PV_x(jj) too
+          if (jj < n_a) {
+            if (!issue_pv(0, gg, jj == 0)) break;
+            if (jj == n_a - 1) {
+              umma_commit(pv_done + 0);
+              ++ix[0];
+            }
+            if (jj + 1 < n_a) {
+              if (!wait_k(gg + 1)) break;
+              issue_s(0, gg + 1);
+            }
+          }
+          if (!issue_pv(1, gg, jj == 0)) break;
+          umma_commit(v_empty + gg % NV);
+          if (jj == n_b - 1) {
+            umma_commit(pv_done + 1);
+            ++ix[1];
+          } else {
+            if (!wait_k(gg + 1)) break;
+            issue_s(1, gg + 1);
+            umma_commit(k_empty + (gg + 1) % NK);
+            if (jj + 1 == n_b - 1) umma_commit(q_empty);
+          }
+        }
+        g += n_b;
+      }
+    }
+  }
+  } else {
+    regs_inc<kPpSoftmaxRegs>();
+    // ------------------------------------------------------------ softmax warpgroups A (warps 0-3), B (4-7)
+    const int x = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t ts = tmem + lane_base + 128 * x, to = tmem + lane_base + 256 + 128 * x;
+    int gx = 0, ix = 0, where = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int slot = r & 1;
+      if (!warp_wait(item_full + slot, (r >> 1) & 1, abort)) {
+        where = 10;
+        break;
+      }
+      const int j = item_ring[slot];
+      mbar_arrive(item_empty + slot);
+      if (j < 0) break;
+      const int2 pr = pair_of(j);
+      const int tile_id = x ? pr.y : pr.x;
+      if (tiles_of(tile_id) == 0) continue;
+      const AttnTile tile = a.tiles[tile_id];
+      const int bh = j / a.n_pairs, b = bh / a.H, h = bh % a.H;
+      if (row == 0) item_s = tile_id * 65536 + bh;
+      const int tq = tile.q0 + row;
+      float m_used = -INFINITY, l = 0.f;
+      int it = 0;
+      for (int si = 0; si < tile.nseg && ok; ++si) {
+        const AttnSeg sg = a.segs[tile.seg0 + si];
+        const float lw2 = sg.logw * 1.4426950408889634f;
+        for (int j0 = 0; j0 < sg.len; j0 += BN, ++it, ++gx) {
+          if (!warp_wait(s_full + x, gx & 1, abort)) {
+            ok = false;
+            where = 6;
+            break;
+          }
+          tc_fence_after();
+          const int nvalid = min(BN, sg.len - j0);
+          const int kt0 = sg.first + j0;
+          const bool causal = sg.kind == SEG_TOKENS && sg.causal;
+          const bool masked = nvalid < BN || (causal && kt0 + BN - 1 > tile.q0);
+          const int lim = min(nvalid - 1, causal ? tq - kt0 : BN - 1);
+          if (masked) softmax_tile_reg<true, D>(ts, to, lim, a.scale_log2e, lw2, it, m_used, l, p_half + x);
+          else softmax_tile_reg<false, D>(ts, to, lim, a.scale_log2e, lw2, it, m_used, l, p_half + x);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(p_full + x);
+        }
+      }
+      if (!ok) break;
+      if (!warp_wait(pv_done + x, ix & 1, abort)) {
+        where = 8;
+        break;
+      }
+      ++ix;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* out = (__nv_bfloat16*)a.out;
+      const bool live = row < tile.qlen;
+      __nv_bfloat16* orow = out + ((int64_t)(b * a.T + tq) * a.H + h) * D;
+      uint32_t pk[D / 2];
+#pragma unroll
+      for (int c2 = 0; c2 < D / 64; ++c2) {
+        float o[2][32];
+        tmem_ld32(to + c2 * 64, o[0]);
+        tmem_ld32(to + c2 * 64 + 32, o[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const __nv_bfloat162 t = __floats2bfloat162_rn(o[hh][i] * inv, o[hh][i + 1] * inv);
+            pk[(c2 * 64 + hh * 32 + i) / 2] = *reinterpret_cast<const uint32_t*>(&t);
+          }
+      }
+      tc_fence_before();
+      mbar_arrive(o_empty + x);
+      if (live) {
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i)
+          *reinterpret_cast<uint4*>(orow + 8 * i) = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      }
+      if (live && a.lse) a.lse[(int64_t)bh * a.T + tq] = (m_used + log2f(l)) * 0.6931471805599453f;
+    }
+    if (where && lane == 0) atomicCAS((int*)&where_s, 0, where * 1000 + min(gx, 999));
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_s && threadIdx.x == 0) {
+    if (atomicCAS(status, 0, 1) == 0) {
+      status[1] = item_s;
+      status[2] = where_s;
+    }
+  }
+  if (threadIdx.x == 0) {
+    // every CTA has taken its last item before it counts itself out: the last one resets
+    __threadfence();
+    if (atomicAdd(sched + 1, 1) == (int)gridDim.x - 1) {
+      atomicExch(sched, 0);
+      atomicExch(sched + 1, 0);
+    }
+  }
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 template <int E, int D>
 cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
   TcMaps maps;
@@ -1014,6 +1554,30 @@ cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
     maps.cv = maps.v;
   }
   if (!ok) return cudaErrorInvalidValue;
+  if constexpr (D <= 128 && E <= 128) {
+    if (a.pairs && a.n_pairs > 0 && status && std::getenv("THIN_ATTN_TC1") == nullptr &&
+        std::getenv("THIN_ATTN_TC2_PER_TILE") == nullptr) {
+      int dev = 0, sms = 0;
+      cudaError_t e = cudaGetDevice(&dev);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      const size_t sm = PpLayout<E, D>::BYTES;
+      auto kern = attn_pp_kernel<E, D>;
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      int per_sm = 0;
+      if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 384, sm);
+      cudaFuncAttributes fa{};
+      if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return e;
+      // the register reallocation inside the kernel is sized for a launch of exactly kPpLaunchRegs per
+      // thread: with any other count the two-CTA kernel below runs instead
+      if (per_sm >= 1 && fa.numRegs == kPpLaunchRegs) {
+        const int64_t items = (int64_t)a.n_pairs * a.B * a.H;
+        const int grid = (int)std::min<int64_t>(items, (int64_t)sms);
+        kern<<<grid, 384, sm, st>>>(maps, a, status);
+        return cudaGetLastError();
+      }
+    }
+  }
   if constexpr (D <= 128) {
     if (std::getenv("THIN_ATTN_TC1") == nullptr) {
       const size_t sm = Tc2Layout<E, D>::BYTES;

@@ -194,6 +194,10 @@ struct AttnArgs {
   int n_slots, slot_rows;
   float scale_log2e;
   int inject_timeout;   // test hook: CTA (0,0) withholds its first key tile so a bounded wait runs out
+  // tile pairs of the ping-pong kernel: (x, y) = tiles A and B, A's key tiles the first ones of B's
+  // (x = -1: B alone); pairs [pair0, pair0 + n_pairs) of the table.  Null: no pairs.
+  const int2* pairs;
+  int pair0, n_pairs;
 };
 
 }  // namespace thin
