@@ -412,31 +412,40 @@ def attention_roofline(w, plan, attn_ms, pk):
 
 
 def halving_roofline(w, h, ph, pk):
-    """Halving steps, HBM-bound by their algorithmic bytes: every instance's n points read once and its
-    n/2 survivors written once, 1.5 n (E+D) elements per instance.  Per step from the live per-step
-    CUDA events; the headline is the step that takes longest, beside the whole halving phase."""
+    """Halving launches, HBM-bound by their algorithmic bytes: every instance's n points read once and
+    its n/2 survivors written once, 1.5 n (E+D) elements per instance.  Per launch from the live
+    per-step CUDA events: the steps that ran in the persistent halving launch report its time on the
+    first of them and 0 on the others, so they form one entry.  The headline is the launch that takes
+    longest, beside the whole halving phase."""
     es = 4 if w.dtype == "fp32" else 2
     sp = h.profile_steps()
-    steps_tab = []
+    tab = []
     for st in sp["steps"]:
         sb = st["n_inst"] * 3 * st["n"] // 2 * (w.E + w.D) * es
         sms = st["ms"] / max(1, sp["calls"])
-        steps_tab.append({"n": st["n"], "n_inst": st["n_inst"], "ms": round(sms, 4), "bytes": sb,
-                          "frac": round(sb / (sms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if sms > 0 else None})
-    hbytes = sum(t["bytes"] for t in steps_tab)
+        if sms == 0 and tab:
+            tab[-1]["steps"].append({"n": st["n"], "n_inst": st["n_inst"]})
+            tab[-1]["bytes"] += sb
+            continue
+        tab.append({"steps": [{"n": st["n"], "n_inst": st["n_inst"]}], "ms": round(sms, 4), "bytes": sb})
+    for t in tab:
+        t["frac"] = round(t["bytes"] / (t["ms"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if t["ms"] > 0 else None
+        t["kernel"] = (f"halving step n={t['steps'][0]['n']} x {t['steps'][0]['n_inst']} instances" if len(t["steps"]) == 1
+                       else "persistent halving launch of " + " + ".join(f"{x['n_inst']} x {x['n']}" for x in t["steps"]))
+    hbytes = sum(t["bytes"] for t in tab)
     hms = (ph["thin_ms"] + ph["merge_ms"]) / max(1, ph["calls"])
-    top = max(steps_tab, key=lambda t: t["ms"]) if steps_tab else None
+    top = max(tab, key=lambda t: t["ms"]) if tab else None
     if not top or top["ms"] <= 0:
         return None
     return {"bound": "hbm", "achieved": round(top["bytes"] / (top["ms"] * 1e-3) / 1e9, 1),
-            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": top["frac"],
-            "kernel": f"halving step n={top['n']} x {top['n_inst']} instances",
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": top["frac"], "kernel": top["kernel"],
             "algorithmic_bytes_per_launch": top["bytes"], "avg_launch_ms": top["ms"],
-            "traffic": kernel_traffic("halving_fused_n64") if (w.name == "express32k" and top["n"] == 64) else None,
+            "traffic": (kernel_traffic("halving_fused_n64") if (w.name == "express32k" and len(top["steps"]) == 1
+                                                                and top["steps"][0]["n"] == 64) else None),
             "all_steps": {"achieved": round(hbytes / (hms * 1e-3) / 1e9, 1) if hms > 0 else None,
                           "frac": round(hbytes / (hms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if hms > 0 else None,
                           "bytes": hbytes, "ms": round(hms, 4)},
-            "steps": steps_tab}
+            "launches": tab}
 
 
 L2_BYTES = 126e6

@@ -188,10 +188,23 @@ THIN_ATTN_API thin_attn_status thin_attn_profile_read(thin_attn_t h, double* ms,
  * (from the end of the previous step, or the start of the forward, to its end), n_inst[i] its
  * instances and n_points[i] the points of each.  Up to max_steps entries are written;
  * *n_steps = steps of the most recently profiled plan (the sums restart when a forward of another
- * plan is recorded), *calls = forwards summed.  Resets the step sums.  Both readers wait for the
+ * plan is recorded), *calls = forwards summed.  Steps that ran together in the persistent halving
+ * launch (thin_attn_sched_layout) report its time on the first of them and 0 on the others.
+ * Resets the step sums.  Both readers wait for the
  * recorded forwards; each returns and resets only its own sums, so each sees every forward. */
 THIN_ATTN_API thin_attn_status thin_attn_profile_steps(thin_attn_t h, int max_steps, double* ms, int* n_inst,
                                                        int* n_points, int* n_steps, int* calls);
+
+/* The halving steps of a plan that run as one persistent launch (the last thinning level of the
+ * Express batches and the HALVE merges, or the last levels of a Thinformer compress): work item i
+ * runs the halving of trace entry entry[i] (thin_attn_trace_layout's order) once the items
+ * preds[pred_off[i] .. pred_off[i+1]) have finished (items are numbered in queue order; every
+ * predecessor comes earlier).  Call with max_items = max_preds = 0 for the sizes (*n_items,
+ * *n_preds); the arrays then need n_items, n_items + 1 and n_preds elements.  n_items = 0: the
+ * plan runs every step as its own launch.  Host arrays; nothing is enqueued. */
+THIN_ATTN_API thin_attn_status thin_attn_sched_layout(thin_attn_t h, int causal, int g, int32_t* entry,
+                                                     int32_t* pred_off, int32_t* preds, size_t max_items,
+                                                     size_t max_preds, size_t* n_items, size_t* n_preds);
 
 /* Synchronise `stream` and report a device-side failure recorded by the
  * handle's kernels since the last call (THIN_ATTN_ETIMEOUT, ...). */

@@ -209,3 +209,57 @@ def test_decode_cache_arguments_are_checked_on_the_host():
             T.ThinAttentionCache(1, 4, 64, 64, bf16, **args)
     with pytest.raises(T.ThinAttnError, match="EINVAL"):
         T.ThinAttentionCache(1, 4, 12, 64, bf16, capacity=4096, n_exact=1024, batch=1024)   # E % 8
+
+
+def _round_kind(rid):
+    """(kind, fields) of a Philox round id: ('batch', k, level) / ('merge', level, node, step) / ('level', l)."""
+    if rid & 0xC0000000 == 0x40000000:
+        return ("batch", (rid >> 4) & 0x3FFFFFF, rid & 0xF)
+    if rid & 0xC0000000 == 0x80000000:
+        return ("merge", (rid >> 24) & 0x3F, (rid >> 1) & 0x7FFFFF, rid & 1)
+    return ("level", rid)
+
+
+@pytest.mark.parametrize("T,n_e,bsz,H", [(32768, 1024, 1024, 32), (8192, 1024, 1024, 4), (22000, 100, 600, 2)])
+def test_sched_layout_merges_wait_for_their_children(T, n_e, bsz, H):
+    """The persistent halving launch of an Express plan: the last level of every batch and both steps
+    of every HALVE merge; the queue order is topological; the first step of merge (l, j) waits for
+    exactly the four items that write its children (the last level of batches 4j..4j+3, or the second
+    steps of merges (l-1, 4j..4j+3)) of the same (b,h), its second step for exactly its first."""
+    w = W.WORKLOADS["express32k"].with_(T=T, H=H, n_exact=n_e, batch=bsz)
+    h = _handle(w)
+    ent, preds = h.sched_layout(True, w.g)
+    lay = h.trace_layout(True, w.g)
+    assert len(ent) > 0
+    assert all(q < i for i, ps in enumerate(preds) for q in ps)
+    last = h.plan(True, w.g)["levels"]
+    keys = [(lay[e][0],) + _round_kind(lay[e][1]) for e in ent]
+    where = {k: i for i, k in enumerate(keys)}
+    assert len(where) == len(keys)
+    n_merge = 0
+    for i, k in enumerate(keys):
+        bh, kind = k[0], k[1]
+        if kind == "batch":
+            assert k[3] == last and preds[i] == []
+            continue
+        assert kind == "merge"
+        lv, j, step = k[2], k[3], k[4]
+        if step == 1:
+            assert preds[i] == [where[(bh, "merge", lv, j, 0)]]
+            continue
+        n_merge += 1
+        if lv == 1:
+            want = {where[(bh, "batch", 4 * j + c, last)] for c in range(4)}
+        else:
+            want = {where[(bh, "merge", lv - 1, 4 * j + c, 1)] for c in range(4)}
+        assert set(preds[i]) == want
+    n_b = (T - n_e) // bsz
+    assert n_merge == H * sum(n_b >> (2 * lv) for lv in range(1, 8))
+
+
+def test_sched_layout_noncausal_has_none():
+    """The persistent halving launch is planned only where HALVE merges follow the last thinning level:
+    a Thinformer compress (ViT's 192- and 384-point levels, BigGAN's) runs one launch per level."""
+    for name in ("vit", "biggan"):
+        w = W.WORKLOADS[name]
+        assert _handle(w).sched_layout(False, w.g) == ([], [])

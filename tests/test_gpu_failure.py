@@ -39,3 +39,29 @@ def test_bounded_wait_reports_timeout_and_context_survives(kernel, monkeypatch):
     again = h.forward(q, k, v, causal=True, g=2, seed=3)["out"]
     h.check()
     assert torch.equal(again, good)
+
+
+def test_scheduler_dependency_wait_reports_timeout_and_context_survives():
+    """The persistent halving launch: with THIN_ATTN_INJECT_SCHED_TIMEOUT set, one work item waits on a
+    completion flag that nothing sets; its bounded wait gives up (~0.2 s), the status word stops every
+    other CTA at its next item, and thin_attn_check reports THIN_ATTN_ETIMEOUT naming the scheduler.
+    The next forward on the same context (a new epoch for the flags, counters reset by the last CTA)
+    is exact."""
+    w = W.WORKLOADS["express32k"].with_(H=2)
+    q, k, v = (x.cuda() for x in W.make_qkv(w, T=8192))
+    h = TA.ThinAttention(w.B, 8192, 8192, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
+    assert len(h.sched_layout(True, 2)[0]) > 0
+    good = h.forward(q, k, v, causal=True, g=2, seed=3, return_coreset=True)
+    good = {key: t.clone() for key, t in good.items()}
+    h.check()
+    os.environ["THIN_ATTN_INJECT_SCHED_TIMEOUT"] = "1"
+    try:
+        h.forward(q, k, v, causal=True, g=2, seed=3)
+        with pytest.raises(TA.ThinAttnError, match="ETIMEOUT") as ei:
+            h.check()
+        assert "scheduler" in str(ei.value)
+    finally:
+        del os.environ["THIN_ATTN_INJECT_SCHED_TIMEOUT"]
+    again = h.forward(q, k, v, causal=True, g=2, seed=3, return_coreset=True)
+    h.check()
+    assert torch.equal(again["out"], good["out"]) and torch.equal(again["coreset"], good["coreset"])

@@ -300,6 +300,38 @@ def test_fused_and_three_launch_halving_agree(case, monkeypatch):
         assert torch.equal(res[0][key], res[1][key]), key
 
 
+@pytest.mark.parametrize("name", ["express", "express_long", "express_ragged", "express_a"])
+def test_scheduled_and_levelwise_halving_agree(name, monkeypatch):
+    """The persistent halving launch (the last batch level and every HALVE merge as work items waiting
+    on their inputs) and one launch per step run the
+    same instance kernels: traces, coresets, outputs and LSE are bit-identical, on two forwards in a
+    row (the completion flags of the first must not satisfy the second's waits)."""
+    w = {"express": W.WORKLOADS["express32k"].with_(T=8192, H=4),
+         "express_long": W.WORKLOADS["express128k"].with_(T=40960, H=2),
+         "express_ragged": W.WORKLOADS["express32k"].with_(T=22000, H=2, n_exact=100, batch=600),
+         "express_a": W.WORKLOADS["express32k_a"].with_(T=16384, H=2)}[name]
+    S = w.T if w.causal else w.S
+    q, k, v = (x.cuda() for x in W.make_qkv(w))
+    res = []
+    for levelwise in (False, True):
+        if levelwise:
+            monkeypatch.setenv("THIN_ATTN_LEVELWISE", "1")
+        else:
+            monkeypatch.delenv("THIN_ATTN_LEVELWISE", raising=False)
+        h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch)
+        if not levelwise:
+            assert len(h.sched_layout(w.mode, w.g)[0]) > 0
+        for _ in range(2):
+            r = h.forward(q, k, v, causal=w.mode, g=w.g, seed=w.seed, return_lse=True, return_coreset=True,
+                          return_trace=True)
+            torch.cuda.synchronize()
+            h.check()
+            res.append(r)
+    for r in res[1:]:
+        for key in ("trace", "coreset", "out", "lse"):
+            assert torch.equal(res[0][key], r[key]), key
+
+
 @pytest.mark.parametrize("name", ["vit", "express", "express_a", "express_ragged"])
 def test_attention_launch_forms_agree(name, monkeypatch):
     """The ping-pong kernel (two query tiles of a head against one K/V stream, one CTA per SM), the
@@ -349,7 +381,17 @@ def test_profile_steps_cover_the_halving_phases():
     sp = h.profile_steps()
     assert ph["calls"] == 2 and sp["calls"] == 2
     steps = sp["steps"]
-    assert len(steps) > 0 and all(s["ms"] > 0 and s["n_inst"] > 0 and s["n"] >= 2 for s in steps)
+    # steps that ran in the persistent halving launch report its time on the first of them, 0 after
+    grouped = set()
+    ent, _ = h.sched_layout(True, w.g)
+    if ent:
+        lay = h.trace_layout(True, w.g)
+        rounds = {(lay[e][0], lay[e][1]) for e in ent}
+        grouped = {i for i, s in enumerate(steps) if s["n"] > 128}
+        assert len(rounds) > 0
+    assert len(steps) > 0 and all(s["n_inst"] > 0 and s["n"] >= 2 for s in steps)
+    assert all(s["ms"] > 0 for i, s in enumerate(steps) if i not in grouped or i == min(grouped))
+    assert all(s["ms"] == 0 for i, s in enumerate(steps) if i in grouped and i != min(grouped))
     total = sum(s["ms"] for s in steps)
     assert abs(total - (ph["thin_ms"] + ph["merge_ms"])) <= 0.05 * total + 1e-3
     again = h.profile_steps()

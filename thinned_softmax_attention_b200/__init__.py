@@ -58,7 +58,7 @@ EXPORTS = ("thin_attn_version", "thin_attn_last_error", "thin_attn_create", "thi
            "thin_attn_forward_host", "thin_attn_check", "thin_attn_profile", "thin_attn_profile_read",
            "thin_attn_profile_steps",
            "thin_attn_cache_create", "thin_attn_cache_destroy", "thin_attn_cache_length", "thin_attn_cache_decode",
-           "thin_attn_cache_nodes", "thin_attn_cache_check")
+           "thin_attn_cache_nodes", "thin_attn_cache_check", "thin_attn_sched_layout")
 
 
 def lib() -> ctypes.CDLL:
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
     L.thin_attn_cache_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     L.thin_attn_cache_nodes.argtypes = [vp, vp, vp]
     L.thin_attn_cache_check.argtypes = [vp, vp]
+    sz = ctypes.c_size_t
+    L.thin_attn_sched_layout.argtypes = [vp, i, i, vp, vp, vp, sz, sz, ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.thin_attn_profile.argtypes = [vp, i]
     L.thin_attn_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
     ip = ctypes.POINTER(ctypes.c_int)
@@ -147,6 +149,19 @@ class ThinAttention:
         info = PlanInfo()
         _check(lib().thin_attn_plan(self._h, int(causal), g, ctypes.byref(info)))
         return {f: getattr(info, f) for f, _ in PlanInfo._fields_}
+
+    def sched_layout(self, causal: bool, g: int):
+        """Work items of the persistent halving launch: (trace entry of each item in queue order,
+        list of predecessor item indices per item); empty when every step runs on its own."""
+        ni, npr = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().thin_attn_sched_layout(self._h, int(causal), g, None, None, None, 0, 0, ctypes.byref(ni),
+                                            ctypes.byref(npr)))
+        ent = (ctypes.c_int32 * max(1, ni.value))()
+        off = (ctypes.c_int32 * (ni.value + 1))()
+        prd = (ctypes.c_int32 * max(1, npr.value))()
+        _check(lib().thin_attn_sched_layout(self._h, int(causal), g, ent, off, prd, ni.value, npr.value,
+                                            ctypes.byref(ni), ctypes.byref(npr)))
+        return list(ent[:ni.value]), [list(prd[off[i]:off[i + 1]]) for i in range(ni.value)]
 
     def reserve(self, causal: bool, g: int):
         _check(lib().thin_attn_reserve(self._h, int(causal), g))

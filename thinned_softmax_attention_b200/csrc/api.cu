@@ -20,6 +20,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <queue>
 #include <mutex>
 #include <string>
 #include <utility>
@@ -165,6 +166,12 @@ struct Plan {
   int final_buf = BUF_TOKENS;    // compact buffer holding the coreset / nodes
   int att_slots = 1, att_slot_rows = 0;
   AttnTables simt, tc;
+  // steps [sched_s0, sched_s1) run as one persistent launch (launch_halving_sched); s0 == s1: none
+  int sched_s0 = 0, sched_s1 = 0;
+  std::vector<int2> sched_items;            // (step - sched_s0, instance) in queue order
+  std::vector<int> sched_pred_off, sched_preds;
+  size_t sched_items_off = 0, sched_pred_off_off = 0, sched_preds_off = 0, sched_done_off = 0;
+  int sched_epoch = 0;
   size_t delta_off = 0, c2_off = 0, delta_floats = 0, c2_floats = 0;
   size_t bytes = 0;
   void* d_mem = nullptr;
@@ -202,7 +209,12 @@ struct thin_attn_s {
   std::vector<cudaEvent_t> ev_dep;
   // per-phase device timing (thin_attn_profile): event sets and their wave counts
   bool prof_on = false;
-  std::vector<std::pair<std::vector<cudaEvent_t>, size_t>> prof_pending;
+  struct ProfPending {
+    std::vector<cudaEvent_t> ev;
+    size_t waves;
+    int group0, group1;   // steps [group0, group1) ran as one launch (none when equal)
+  };
+  std::vector<ProfPending> prof_pending;
   std::vector<std::vector<cudaEvent_t>> prof_free;
   double prof_ms[3] = {0, 0, 0};
   double prof_total = 0;
@@ -438,6 +450,170 @@ void add_compress_steps(Plan& p, const std::vector<RunDesc>& runs, int S_run, in
   }
 }
 
+int64_t src_rows_of(const thin_attn_config& cf, const Plan* p, const StepPlan& sp);
+
+// Whether the persistent halving scheduler can run this step (instances of 129..512 points that the
+// one-launch kernels take).
+bool sched_step_ok(const thin_attn_config& cf, const Plan* p, const StepPlan& sp) {
+  if (sp.copy_only || sp.inst.empty() || sp.n <= 128 || sp.n > 512 || cf.dtype != THIN_ATTN_BF16) return false;
+  StepArgs a{};
+  a.src_kind = sp.src_buf == BUF_TOKENS ? SRC_TOKENS : SRC_COMPACT;
+  a.src_rows = src_rows_of(cf, p, sp);
+  a.S_full = sp.S_full;
+  a.S_sub = sp.S_sub;
+  a.sub_stride = sp.sub_stride;
+  a.n = sp.n;
+  a.E = cf.E;
+  a.D = cf.D;
+  return halving_sched_shape_ok(a);
+}
+
+// The scheduled group -- the longest run of two or more consecutive steps the scheduler can run, when
+// it holds HALVE merges --
+// its work items, their dependencies and the queue order.  Item X of a later step depends on item Y
+// of an earlier one when X reads rows Y writes, writes rows Y reads, or writes rows Y writes (same
+// buffer, overlapping row ranges).  The queue order comes from a list schedule of the items on the
+// SMs with durations proportional to the measured instance times (a 512-point instance ~2.4 times a
+// 256-point one), taking among the ready items the one with the longest chain of work after it; so
+// the order is topological and puts the instances that feed the deepest merges first.
+void build_sched(const thin_attn_config& cf, Plan* p, int n_sms) {
+  p->sched_s0 = p->sched_s1 = 0;
+  p->sched_items.clear();
+  p->sched_pred_off.clear();
+  p->sched_preds.clear();
+  const int ns = (int)p->steps.size(), cap = halving_sched_max_steps();
+  int best0 = 0, best1 = 0;
+  for (int i = 0; i < ns;) {
+    if (!sched_step_ok(cf, p, p->steps[i])) {
+      ++i;
+      continue;
+    }
+    int j = i;
+    while (j < ns && j - i < cap && sched_step_ok(cf, p, p->steps[j])) ++j;
+    if (j - i > best1 - best0) best0 = i, best1 = j;
+    i = j;
+  }
+  // only where HALVE merges follow the last thinning level: a Thinformer compress's last two levels
+  // (ViT) ran slower as one launch than as two (15 us of 240)
+  bool merges = false;
+  for (int si = best0; si < best1; ++si) merges = merges || p->steps[si].phase == 1;
+  if (best1 - best0 < 2 || !merges) return;
+  struct It {
+    int step, inst;
+  };
+  std::vector<It> items;
+  std::vector<int> first(best1 - best0 + 1, 0);
+  for (int si = best0; si < best1; ++si) {
+    first[si - best0] = (int)items.size();
+    for (int i = 0; i < (int)p->steps[si].inst.size(); ++i) items.push_back({si, i});
+  }
+  first[best1 - best0] = (int)items.size();
+  const int n = (int)items.size();
+  auto src_range = [&](const It& x, int64_t* lo, int64_t* hi) {
+    const StepPlan& sp = p->steps[x.step];
+    *lo = sp.inst[x.inst].src_row;
+    *hi = *lo + sp.n;
+  };
+  auto dst_range = [&](const It& x, int64_t* lo, int64_t* hi) {
+    const StepPlan& sp = p->steps[x.step];
+    *lo = sp.inst[x.inst].dst_row;
+    *hi = *lo + sp.m;
+  };
+  // per earlier step: its items' source and destination ranges, each sorted by start
+  struct Rg {
+    int64_t lo, hi;
+    int item;
+  };
+  std::vector<std::vector<Rg>> by_src(best1 - best0), by_dst(best1 - best0);
+  for (int x = 0; x < n; ++x) {
+    Rg r{0, 0, x};
+    const int k = items[x].step - best0;
+    src_range(items[x], &r.lo, &r.hi);
+    by_src[k].push_back(r);
+    dst_range(items[x], &r.lo, &r.hi);
+    by_dst[k].push_back(r);
+  }
+  for (auto* v : {&by_src, &by_dst})
+    for (auto& l : *v) std::sort(l.begin(), l.end(), [](const Rg& a, const Rg& b) { return a.lo < b.lo; });
+  auto overlapping = [](const std::vector<Rg>& l, int64_t lo, int64_t hi, std::vector<int>& out) {
+    // ranges of one step do not overlap each other, so their ends are sorted too
+    auto it = std::lower_bound(l.begin(), l.end(), lo, [](const Rg& r, int64_t v) { return r.hi <= v; });
+    for (; it != l.end() && it->lo < hi; ++it) out.push_back(it->item);
+  };
+  std::vector<std::vector<int>> preds(n), succs(n);
+  for (int x = 0; x < n; ++x) {
+    const StepPlan& sx = p->steps[items[x].step];
+    int64_t slo, shi, dlo, dhi;
+    src_range(items[x], &slo, &shi);
+    dst_range(items[x], &dlo, &dhi);
+    std::vector<int> c;
+    for (int sy = best0; sy < items[x].step; ++sy) {
+      const StepPlan& so = p->steps[sy];
+      if (sx.src_buf != BUF_TOKENS && sx.src_buf == so.dst_buf) overlapping(by_dst[sy - best0], slo, shi, c);
+      if (sx.dst_buf == so.src_buf) overlapping(by_src[sy - best0], dlo, dhi, c);
+      if (sx.dst_buf == so.dst_buf) overlapping(by_dst[sy - best0], dlo, dhi, c);
+    }
+    std::sort(c.begin(), c.end());
+    c.erase(std::unique(c.begin(), c.end()), c.end());
+    preds[x] = c;
+    for (int y : c) succs[y].push_back(x);
+  }
+  // list schedule: longest chain of (estimated) work after each item first
+  std::vector<double> dur(n), chain(n, 0.0);
+  for (int x = 0; x < n; ++x) dur[x] = p->steps[items[x].step].n > 256 ? 2.4 : 1.0;
+  for (int x = n - 1; x >= 0; --x) {   // successors always come later in step order
+    double mx = 0.0;
+    for (int y : succs[x]) mx = std::max(mx, chain[y]);
+    chain[x] = dur[x] + mx;
+  }
+  auto worse = [&](int a, int b) { return chain[a] < chain[b] || (chain[a] == chain[b] && a > b); };
+  std::priority_queue<int, std::vector<int>, decltype(worse)> ready(worse);
+  std::vector<int> left(n);
+  for (int x = 0; x < n; ++x)
+    if ((left[x] = (int)preds[x].size()) == 0) ready.push(x);
+  using Ev = std::pair<double, int>;
+  std::priority_queue<Ev, std::vector<Ev>, std::greater<Ev>> running;
+  std::vector<int> order;
+  order.reserve(n);
+  int free_sms = std::max(1, n_sms);
+  while ((int)order.size() < n) {
+    while (free_sms > 0 && !ready.empty()) {
+      const int x = ready.top();
+      ready.pop();
+      order.push_back(x);
+      running.push({dur[x], x});   // times of running items are relative to the current time
+      --free_sms;
+    }
+    if (running.empty()) break;   // cannot happen: the dependencies point forward in step order
+    const double t = running.top().first;
+    while (!running.empty() && running.top().first <= t) {
+      const int x = running.top().second;
+      running.pop();
+      ++free_sms;
+      for (int y : succs[x])
+        if (--left[y] == 0) ready.push(y);
+    }
+    // items started later start at t: shift the clock of what is still running
+    std::vector<Ev> keep;
+    while (!running.empty()) {
+      keep.push_back({running.top().first - t, running.top().second});
+      running.pop();
+    }
+    for (auto& e : keep) running.push(e);
+  }
+  std::vector<int> pos(n);
+  for (int i = 0; i < n; ++i) pos[order[i]] = i;
+  p->sched_s0 = best0;
+  p->sched_s1 = best1;
+  p->sched_pred_off.push_back(0);
+  for (int i = 0; i < n; ++i) {
+    const int x = order[i];
+    p->sched_items.push_back(make_int2(items[x].step - best0, items[x].inst));
+    for (int y : preds[x]) p->sched_preds.push_back(pos[y]);
+    p->sched_pred_off.push_back((int)p->sched_preds.size());
+  }
+}
+
 thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
   const thin_attn_config& cf = h->cfg;
   Plan* p = new Plan();
@@ -587,10 +763,14 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
         std::vector<int64_t> lr;
         add_compress_steps(*p, runs, bsz, BUF_NODES, lr);
       }
-      // HALVE merges: target level L' takes level L'-1 slots 4j'..4j'+3
-      const int nj1 = p->n_b / 4;
-      p->mtemp.rows = (int64_t)BH * nj1 * 2 * p->c;
-      for (int lv = 1; (p->n_b >> (2 * lv)) > 0; ++lv) {
+      // HALVE merges: target level L' takes level L'-1 slots 4j'..4j'+3.  The first step's output
+      // goes to rows of the merge buffer of its own (level, b, h, node), so merges of different
+      // levels never share rows (the halving scheduler runs them concurrently)
+      int64_t merges = 0;
+      for (int lv = 1; (p->n_b >> (2 * lv)) > 0; ++lv) merges += (int64_t)BH * (p->n_b >> (2 * lv));
+      p->mtemp.rows = merges * 2 * p->c;
+      int64_t level_first = 0;
+      for (int lv = 1; (p->n_b >> (2 * lv)) > 0; level_first += (int64_t)BH * (p->n_b >> (2 * lv)), ++lv) {
         const int nj = p->n_b >> (2 * lv);
         for (int step = 0; step < 2; ++step) {
           StepPlan st;
@@ -605,7 +785,7 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
           for (int bh = 0; bh < BH; ++bh)
             for (int j = 0; j < nj; ++j) {
               HalveInst in{};
-              const int64_t mt = ((int64_t)bh * nj + j) * 2 * p->c;
+              const int64_t mt = (level_first + (int64_t)bh * nj + j) * 2 * p->c;
               if (step == 0) {
                 in.src_row = ((int64_t)bh * p->n_slots + p->level_base[lv - 1] + 4 * j) * p->c;
                 in.dst_row = mt;
@@ -646,12 +826,26 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
     build_waves(cf, *p, p->tc);
     build_pairs(p->tc);
   }
+  {
+    int sms = 148;
+    if (cf.device >= 0) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, cf.device);
+    cudaGetLastError();
+    build_sched(cf, p, sms);
+  }
   // memory layout: tables first, then buffers
   size_t off = 0;
   for (auto& st : p->steps) {
     st.inst_off = off;
     off = align256(off + st.inst.size() * sizeof(HalveInst));
   }
+  p->sched_items_off = off;
+  off = align256(off + p->sched_items.size() * sizeof(int2));
+  p->sched_pred_off_off = off;
+  off = align256(off + p->sched_pred_off.size() * sizeof(int));
+  p->sched_preds_off = off;
+  off = align256(off + p->sched_preds.size() * sizeof(int));
+  p->sched_done_off = off;   // zeros, uploaded with the tables
+  off = align256(off + p->sched_items.size() * sizeof(int));
   for (AttnTables* t : {&p->simt, &p->tc}) {
     t->tiles_off = off;
     off = align256(off + t->tiles.size() * sizeof(AttnTile));
@@ -709,6 +903,13 @@ thin_attn_status materialise(thin_attn_s* h, Plan* p) {
   for (auto& st : p->steps) {
     if (!st.inst.empty()) std::memcpy(host.data() + st.inst_off, st.inst.data(), st.inst.size() * sizeof(HalveInst));
     tbl_end = std::max(tbl_end, st.inst_off + st.inst.size() * sizeof(HalveInst));
+  }
+  if (!p->sched_items.empty()) {
+    std::memcpy(host.data() + p->sched_items_off, p->sched_items.data(), p->sched_items.size() * sizeof(int2));
+    std::memcpy(host.data() + p->sched_pred_off_off, p->sched_pred_off.data(), p->sched_pred_off.size() * sizeof(int));
+    if (!p->sched_preds.empty())
+      std::memcpy(host.data() + p->sched_preds_off, p->sched_preds.data(), p->sched_preds.size() * sizeof(int));
+    tbl_end = std::max(tbl_end, p->sched_done_off + p->sched_items.size() * sizeof(int));
   }
   for (AttnTables* t : {&p->simt, &p->tc}) {
     if (!t->tiles.empty()) std::memcpy(host.data() + t->tiles_off, t->tiles.data(), t->tiles.size() * sizeof(AttnTile));
@@ -927,11 +1128,21 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   thin_attn_status ls = launch_waves_after(-1);
   if (ls != THIN_ATTN_OK) return ls;
   bool merged_mark = false;
+  // the scheduled group runs as one launch unless THIN_ATTN_LEVELWISE asks for a launch per step
+  const bool sched = p->sched_s1 > p->sched_s0 && use_tc_gram && std::getenv("THIN_ATTN_LEVELWISE") == nullptr;
+  std::vector<StepArgs> group;
   for (size_t si = 0; si < p->steps.size(); ++si) {
     const StepPlan& sp = p->steps[si];
-    if (!ev.empty() && sp.phase == 1 && !merged_mark) {
-      CK(cudaEventRecord(ev[1], st));
-      merged_mark = true;
+    const bool in_group = sched && (int)si >= p->sched_s0 && (int)si < p->sched_s1;
+    if (!ev.empty() && !merged_mark) {
+      // the first merge step; a scheduled group that holds merges counts as merging from its start
+      bool merges = sp.phase == 1;
+      if (in_group && (int)si == p->sched_s0)
+        for (int sj = p->sched_s0; sj < p->sched_s1; ++sj) merges = merges || p->steps[sj].phase == 1;
+      if (merges && (!in_group || (int)si == p->sched_s0)) {
+        CK(cudaEventRecord(ev[1], st));
+        merged_mark = true;
+      }
     }
     StepArgs a{};
     const void *sk, *sv;
@@ -967,10 +1178,40 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     a.delta = (float*)(base_of(p) + p->delta_off);
     a.trace = trace;
     a.trace_base = sp.trace_base;
-    cudaError_t e = sp.copy_only ? launch_copy_step(a, cf.dtype, st)
-                                 : launch_halving_step(a, cf.dtype, use_tc_gram, st);
-    if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "halving step (n=%d): %s", sp.n, cudaGetErrorString(e));
-    if (!ev.empty()) CK(cudaEventRecord(ev[ev_steps + si], st));
+    if (in_group) {
+      group.push_back(a);
+      if ((int)si + 1 < p->sched_s1) continue;
+      bool ok = true;
+      for (const StepArgs& ga : group) ok = ok && halving_sched_step_supported(ga);
+      if (ok) {
+        SchedTables t{};
+        t.items = (const int2*)(base_of(p) + p->sched_items_off);
+        t.pred_off = (const int*)(base_of(p) + p->sched_pred_off_off);
+        t.preds = (const int*)(base_of(p) + p->sched_preds_off);
+        t.n_items = (int)p->sched_items.size();
+        t.done = (int*)(base_of(p) + p->sched_done_off);
+        if (++p->sched_epoch <= 0) p->sched_epoch = 1;
+        t.epoch = p->sched_epoch;
+        t.sched = h->d_status + 6;
+        t.status = h->d_status;
+        // test hook: the middle item's dependency wait runs out (failure detection without a fault)
+        t.inject_item = std::getenv("THIN_ATTN_INJECT_SCHED_TIMEOUT") ? t.n_items / 2 : -1;
+        cudaError_t e = launch_halving_sched(group.data(), (int)group.size(), t, st);
+        if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "halving scheduler: %s", cudaGetErrorString(e));
+      } else {
+        for (const StepArgs& ga : group) {
+          cudaError_t e = launch_halving_step(ga, cf.dtype, use_tc_gram, st);
+          if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "halving step (n=%d): %s", ga.n, cudaGetErrorString(e));
+        }
+      }
+      // per-step profile: one event after the group (drain_profile puts its time on the first step)
+      if (!ev.empty()) CK(cudaEventRecord(ev[ev_steps + p->sched_s1 - 1], st));
+    } else {
+      cudaError_t e = sp.copy_only ? launch_copy_step(a, cf.dtype, st)
+                                   : launch_halving_step(a, cf.dtype, use_tc_gram, st);
+      if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "halving step (n=%d): %s", sp.n, cudaGetErrorString(e));
+      if (!ev.empty()) CK(cudaEventRecord(ev[ev_steps + si], st));
+    }
     if (si + 1 < p->steps.size()) {
       ls = launch_waves_after((int)si);
       if (ls != THIN_ATTN_OK) return ls;
@@ -1002,7 +1243,7 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   }
   if (!ev.empty()) {
     CK(cudaEventRecord(ev[3], st));
-    h->prof_pending.push_back({ev, waves.size()});
+    h->prof_pending.push_back({ev, waves.size(), sched ? p->sched_s0 : 0, sched ? p->sched_s1 : 0});
     if (h->prof_step_ms.size() != p->steps.size()) {
       h->prof_step_ms.assign(p->steps.size(), 0.0);
       h->prof_step_inst.resize(p->steps.size());
@@ -1049,7 +1290,7 @@ thin_attn_status thin_attn_destroy(thin_attn_t h) {
   if (h->d_status) cudaFree(h->d_status);
   if (h->st_mem) cudaFree(h->st_mem);
   for (auto& pe : h->prof_pending)
-    for (auto e : pe.first) cudaEventDestroy(e);
+    for (auto e : pe.ev) cudaEventDestroy(e);
   for (auto& ev : h->prof_free)
     for (auto e : ev) cudaEventDestroy(e);
   for (auto e : h->ev_dep) cudaEventDestroy(e);
@@ -1062,6 +1303,37 @@ thin_attn_status thin_attn_destroy(thin_attn_t h) {
   for (auto st : {h->hp_in, h->hp_comp, h->hp_out})
     if (st) cudaStreamDestroy(st);
   delete h;
+  return THIN_ATTN_OK;
+}
+
+thin_attn_status thin_attn_sched_layout(thin_attn_t h, int causal, int g, int32_t* entry, int32_t* pred_off,
+                                       int32_t* preds, size_t max_items, size_t max_preds, size_t* n_items,
+                                       size_t* n_preds) {
+  if (!h || !n_items || !n_preds) return fail(THIN_ATTN_EINVAL, "null argument");
+  std::lock_guard<std::mutex> lk(h->mu);
+  Plan* p = nullptr;
+  thin_attn_status s = get_plan(h, causal, g, &p);
+  if (s != THIN_ATTN_OK) return s;
+  const size_t ni = p->sched_items.size(), np = p->sched_preds.size();
+  *n_items = ni;
+  *n_preds = np;
+  if (max_items < ni || max_preds < np) return THIN_ATTN_OK;   // sizes only
+  if ((ni && (!entry || !pred_off)) || (np && !preds)) return fail(THIN_ATTN_EINVAL, "null array");
+  // first trace entry of every step (copy steps have none)
+  std::vector<int64_t> first(p->steps.size(), -1);
+  int64_t e = 0;
+  for (size_t si = 0; si < p->steps.size(); ++si) {
+    if (p->steps[si].copy_only) continue;
+    first[si] = e;
+    e += (int64_t)p->steps[si].inst.size();
+  }
+  for (size_t i = 0; i < ni; ++i) {
+    const int2 it = p->sched_items[i];
+    entry[i] = (int32_t)(first[p->sched_s0 + it.x] + it.y);
+    pred_off[i] = p->sched_pred_off[i];
+  }
+  if (ni) pred_off[ni] = p->sched_pred_off[ni];
+  for (size_t i = 0; i < np; ++i) preds[i] = p->sched_preds[i];
   return THIN_ATTN_OK;
 }
 
@@ -1080,7 +1352,11 @@ thin_attn_status thin_attn_plan(thin_attn_t h, int causal, int g, thin_attn_plan
   info->n_nodes = p->n_slots;
   info->n_halvings = (int)p->trace.size();
   int launches = 1;
-  for (auto& st : p->steps) launches += step_launches(h->cfg, p, st);
+  const bool sched = p->sched_s1 > p->sched_s0 && std::getenv("THIN_ATTN_SIMT_GRAM") == nullptr &&
+                     std::getenv("THIN_ATTN_LEVELWISE") == nullptr;
+  for (int si = 0; si < (int)p->steps.size(); ++si)
+    if (!sched || si < p->sched_s0 || si >= p->sched_s1) launches += step_launches(h->cfg, p, p->steps[si]);
+  if (sched) launches += 1;
   info->kernel_launches = launches;
   info->trace_words = p->trace_words;
   info->coreset_idx_elems = p->coreset_idx_elems;
@@ -1356,20 +1632,23 @@ namespace {
 thin_attn_status drain_profile(thin_attn_s* h) {
   DeviceGuard dg(h->prof_pending.empty() ? -1 : h->cfg.device);
   for (auto& pe : h->prof_pending) {
-    auto& ev = pe.first;
+    auto& ev = pe.ev;
     CK(cudaEventSynchronize(ev[3]));
     float t;
     CK(cudaEventElapsedTime(&t, ev[0], ev[1]));
     h->prof_ms[0] += t;
     CK(cudaEventElapsedTime(&t, ev[1], ev[2]));
     h->prof_ms[1] += t;
-    const size_t first_step = 4 + 2 * pe.second;
-    for (size_t w = 0; w < pe.second; ++w) {
+    const size_t first_step = 4 + 2 * pe.waves;
+    for (size_t w = 0; w < pe.waves; ++w) {
       CK(cudaEventElapsedTime(&t, ev[4 + 2 * w], ev[5 + 2 * w]));
       h->prof_ms[2] += t;
     }
     for (size_t si = 0; si < h->prof_step_ms.size() && first_step + si < ev.size(); ++si) {
-      CK(cudaEventElapsedTime(&t, si ? ev[first_step + si - 1] : ev[0], ev[first_step + si]));
+      // a group's steps share the event recorded after it: its whole time goes on its first step
+      if ((int)si > pe.group0 && (int)si < pe.group1) continue;
+      const size_t end = (int)si == pe.group0 && pe.group1 > pe.group0 ? (size_t)pe.group1 - 1 : si;
+      CK(cudaEventElapsedTime(&t, si ? ev[first_step + si - 1] : ev[0], ev[first_step + end]));
       h->prof_step_ms[si] += t;
     }
     CK(cudaEventElapsedTime(&t, ev[0], ev[3]));
@@ -1427,6 +1706,11 @@ thin_attn_status thin_attn_check(thin_attn_t h, void* stream) {
   CK(cudaMemcpy(st, h->d_status, sizeof st, cudaMemcpyDeviceToHost));
   if (st[0] != 0) {
     CK(cudaMemset(h->d_status, 0, 16));
+    if (st[0] == 7)
+      return fail(THIN_ATTN_ETIMEOUT, "device wait gave up (code 7: halving scheduler, work item %d waited for its inputs)",
+                  st[1]);
+    if (st[0] != 1)
+      return fail(THIN_ATTN_ETIMEOUT, "device wait gave up (code %d: halving kernel, instance or CTA %d)", st[0], st[1]);
     return fail(THIN_ATTN_ETIMEOUT, "device wait gave up (code %d; query tile %d of (b,h) %d; wait %d at key tile %d)",
                 st[0], st[1] >> 16, st[1] & 0xFFFF, st[2] / 1000, st[2] % 1000);
   }

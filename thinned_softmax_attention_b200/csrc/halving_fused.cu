@@ -31,6 +31,7 @@
 // Delta buffers (one per walker set).  Every mbarrier wait is bounded; after a time-out the
 // kernel stops, waits (bounded) for the copies and MMAs it started, frees TMEM and reports
 // through the status word (code 3, status[1] = CTA).
+#include <algorithm>
 #include <cstdlib>
 
 #include "common.cuh"
@@ -531,11 +532,14 @@ cudaError_t launch_np(const StepArgs& a, cudaStream_t st) {
 // (kk in columns 0..255, vv in 256..511), then rows 128..255 against themselves (columns 0..127 and
 // 256..383), so Delta rows 0..63 are written while the second pass runs.  Every barrier is used
 // once (phase 0) and every wait is bounded.
-__global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant__ FusedMaps maps, const StepArgs a) {
+// One instance (`inst` of step `a`) with the CTA's 256 threads; `smem` is the 1024-byte aligned
+// dynamic shared memory, `tmem` 512 allocated TMEM columns.  The barriers are initialised here and
+// invalidated before returning, so a persistent caller can run one instance after another.
+// Returns false when a bounded wait gave up (reported in a.status).
+__device__ __forceinline__ bool halve256_body(const FusedMaps& maps, const StepArgs& a, const int inst, uint8_t* smem,
+                                              const uint32_t tmem) {
   constexpr int LD = 129;                       // Delta row stride (floats)
   constexpr uint32_t CB = 2 * kChunk;           // one feature chunk: 256 rows x 64 bf16
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int EC = a.E / 64, NC = (a.E + a.D) / 64;
   float* D = (float*)(smem + NC * CB);          // [128][LD]
   __shared__ __align__(8) uint64_t bars[20];
@@ -552,10 +556,8 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
   __shared__ float red[4];
   __shared__ float thr_s[128];
   __shared__ uint32_t bits_s[4];
-  __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int inst = blockIdx.x;
   const int m = a.m, n = a.n;
   if (threadIdx.x == 0) {
     abort_s = 0;
@@ -573,11 +575,9 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
     }
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(&tmem_base_s, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_base_s;
   volatile int* abort = &abort_s;
   const HalveInst in = a.inst[inst];
   const bool tokens = a.src_kind == SRC_TOKENS;
@@ -822,9 +822,27 @@ __global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant_
   if (abort_s && threadIdx.x == 0 && a.status) {
     if (atomicCAS(a.status, 0, 5) == 0) a.status[1] = inst;
   }
-  if (warp == 1) {
+  const bool ok = !abort_s;
+  __syncthreads();
+  if (threadIdx.x == 0 && ok) {   // after a time-out the CTA stops; nothing re-initialises them
+    for (int i = 0; i < 17; ++i)
+      if (i != 7) mbar_inval(bars + i);
+  }
+  return ok;
+}
+
+__global__ void __launch_bounds__(256, 1) halve256_kernel(const __grid_constant__ FusedMaps maps, const StepArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint32_t tmem_base_s;
+  if (threadIdx.x >> 5 == 1) tmem_alloc(&tmem_base_s, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  halve256_body(maps, a, blockIdx.x, smem, tmem_base_s);
+  if (threadIdx.x >> 5 == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem_base_s, 512);
   }
 }
 
@@ -902,10 +920,11 @@ __device__ __forceinline__ void gather_global(const StepArgs& a, const HalveInst
   }
 }
 
-__global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant__ FusedMaps maps, const StepArgs a) {
+// One instance with the CTA's 256 threads, as halve256_body (barriers initialised here and
+// invalidated before returning; false when a bounded wait gave up).
+__device__ __forceinline__ bool halve512_body(const FusedMaps& maps, const StepArgs& a, const int inst, uint8_t* smem,
+                                              const uint32_t tmem) {
   constexpr int NBP = 10;                       // block pairs (bi <= bj) of four 128-row blocks
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int EC = a.E / 64, NC = (a.E + a.D) / 64;
   float* D = (float*)(smem + 4 * kChunk);       // packed upper triangle, row j at tri_offset(j)
   __shared__ __align__(8) uint64_t bars[24];
@@ -924,10 +943,8 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
   __shared__ float thr_s[kH512Pairs];
   __shared__ float alpha_s[kH512Pairs];
   __shared__ uint32_t bits_s[8];
-  __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int inst = blockIdx.x;
   const int m = a.m, n = a.n;
   if (threadIdx.x == 0) {
     abort_s = 0;
@@ -948,11 +965,9 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
     }
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(&tmem_base_s, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_base_s;
   volatile int* abort = &abort_s;
   const HalveInst in = a.inst[inst];
   const bool tokens = a.src_kind == SRC_TOKENS;
@@ -1199,27 +1214,53 @@ __global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant_
   if (abort_s && threadIdx.x == 0 && a.status) {
     if (atomicCAS(a.status, 0, 6) == 0) a.status[1] = inst;
   }
-  if (warp == 1) {
+  const bool ok = !abort_s;
+  __syncthreads();
+  if (threadIdx.x == 0 && ok) {   // after a time-out the CTA stops; nothing re-initialises them
+    for (int i = 0; i < 17; ++i)
+      if (i != 13) mbar_inval(bars + i);
+    for (int t = 0; t < 8; ++t) {
+      mbar_inval(thf + t);
+      mbar_inval(bitsb + t);
+    }
+  }
+  return ok;
+}
+
+__global__ void __launch_bounds__(256, 1) halve512_kernel(const __grid_constant__ FusedMaps maps, const StepArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint32_t tmem_base_s;
+  if (threadIdx.x >> 5 == 1) tmem_alloc(&tmem_base_s, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  halve512_body(maps, a, blockIdx.x, smem, tmem_base_s);
+  if (threadIdx.x >> 5 == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem_base_s, 512);
   }
 }
 
+// TMA maps of a step's source rows (128-row boxes): tokens, every k-th token, or compact rows.
+bool make_step_maps(const StepArgs& a, FusedMaps* maps) {
+  if (a.src_kind == SRC_TOKENS && a.sub_stride > 1)
+    return make_map_4d_strided(&maps->k, a.srcK, a.src_rows, a.H, a.E, a.sub_stride, 128) &&
+           make_map_4d_strided(&maps->v, a.srcV, a.src_rows, a.H, a.D, a.sub_stride, 128);
+  if (a.src_kind == SRC_TOKENS)
+    return make_map_3d(&maps->k, a.srcK, a.src_rows, a.H, a.E, 128) && make_map_3d(&maps->v, a.srcV, a.src_rows, a.H, a.D, 128);
+  return make_map_2d(&maps->k, a.srcK, a.src_rows, a.E, a.E, 128) && make_map_2d(&maps->v, a.srcV, a.src_rows, a.D, a.D, 128);
+}
+
+constexpr size_t kDelta512Bytes = (size_t)(kH512Pairs * (kH512Pairs + 1) / 2) * 4;
+size_t smem_512() { return 1024 + 4 * (size_t)kChunk + kDelta512Bytes; }
+size_t smem_256(const StepArgs& a) { return 1024 + (size_t)((a.E + a.D) / 64) * 2 * kChunk + (size_t)128 * 129 * 4; }
+
 cudaError_t launch_512(const StepArgs& a, cudaStream_t st) {
   FusedMaps maps;
-  bool ok;
-  if (a.src_kind == SRC_TOKENS && a.sub_stride > 1) {
-    ok = make_map_4d_strided(&maps.k, a.srcK, a.src_rows, a.H, a.E, a.sub_stride, 128) &&
-         make_map_4d_strided(&maps.v, a.srcV, a.src_rows, a.H, a.D, a.sub_stride, 128);
-  } else if (a.src_kind == SRC_TOKENS) {
-    ok = make_map_3d(&maps.k, a.srcK, a.src_rows, a.H, a.E, 128) && make_map_3d(&maps.v, a.srcV, a.src_rows, a.H, a.D, 128);
-  } else {
-    ok = make_map_2d(&maps.k, a.srcK, a.src_rows, a.E, a.E, 128) && make_map_2d(&maps.v, a.srcV, a.src_rows, a.D, a.D, 128);
-  }
-  if (!ok) return cudaErrorInvalidValue;
-  const size_t delta_bytes = (size_t)(kH512Pairs * (kH512Pairs + 1) / 2) * 4;
-  if ((size_t)v_blocks_per_pass(a.D / 64) * (a.D / 64) * kChunk > delta_bytes) return cudaErrorInvalidValue;
-  const size_t sm = 1024 + 4 * (size_t)kChunk + delta_bytes;
+  if (!make_step_maps(a, &maps)) return cudaErrorInvalidValue;
+  if ((size_t)v_blocks_per_pass(a.D / 64) * (a.D / 64) * kChunk > kDelta512Bytes) return cudaErrorInvalidValue;
+  const size_t sm = smem_512();
   cudaError_t e = cudaFuncSetAttribute(halve512_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   halve512_kernel<<<a.n_inst, 256, sm, st>>>(maps, a);
@@ -1228,30 +1269,123 @@ cudaError_t launch_512(const StepArgs& a, cudaStream_t st) {
 
 cudaError_t launch_256(const StepArgs& a, cudaStream_t st) {
   FusedMaps maps;
-  bool ok;
-  if (a.src_kind == SRC_TOKENS && a.sub_stride > 1) {
-    ok = make_map_4d_strided(&maps.k, a.srcK, a.src_rows, a.H, a.E, a.sub_stride, 128) &&
-         make_map_4d_strided(&maps.v, a.srcV, a.src_rows, a.H, a.D, a.sub_stride, 128);
-  } else if (a.src_kind == SRC_TOKENS) {
-    ok = make_map_3d(&maps.k, a.srcK, a.src_rows, a.H, a.E, 128) && make_map_3d(&maps.v, a.srcV, a.src_rows, a.H, a.D, 128);
-  } else {
-    ok = make_map_2d(&maps.k, a.srcK, a.src_rows, a.E, a.E, 128) && make_map_2d(&maps.v, a.srcV, a.src_rows, a.D, a.D, 128);
-  }
-  if (!ok) return cudaErrorInvalidValue;
-  const int NC = (a.E + a.D) / 64;
-  const size_t sm = 1024 + (size_t)NC * 2 * kChunk + (size_t)128 * 129 * 4;
+  if (!make_step_maps(a, &maps)) return cudaErrorInvalidValue;
+  const size_t sm = smem_256(a);
   cudaError_t e = cudaFuncSetAttribute(halve256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   halve256_kernel<<<a.n_inst, 256, sm, st>>>(maps, a);
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------------------------------
+// Several steps of 129..512-point instances in one persistent launch (the last thinning level of the
+// Express batches and both steps of every HALVE merge): one CTA per SM takes work items (step,
+// instance) from a counter in the host-built queue order, waits until the items that write its
+// source rows -- or read or write its destination rows -- have finished, runs the instance with the
+// body of halve256_kernel or halve512_kernel, and publishes its completion.  A merge thus starts as
+// soon as its four child coresets exist, and the SMs that one level leaves idle at its tail take the
+// next level's ready instances.  The queue order is a topological order of those dependencies (the
+// host simulates a list schedule of the items on the SMs), so an item only ever waits for items that
+// CTAs already hold, and every wait is bounded: a wait that gives up (or any failure reported in the
+// status word) stops every CTA at its next item.
+constexpr int kSchedMaxSteps = 12;
+
+struct SchedParams {
+  FusedMaps maps[kSchedMaxSteps];
+  StepArgs steps[kSchedMaxSteps];
+  const int2* items;      // (step, instance) in queue order
+  const int* pred_off;    // predecessors of item i: preds[pred_off[i] .. pred_off[i + 1])
+  const int* preds;
+  int n_items;
+  int* done;              // per item: `epoch` once its outputs are written
+  int epoch;
+  int* sched;             // [0] next item, [1] CTAs that have left (the last one resets both)
+  int* status;
+  int inject_item;        // test hook: this item's wait never succeeds (-1: none)
+};
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__global__ void __launch_bounds__(256, 1) halve_sched_kernel(const __grid_constant__ SchedParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int item_s;
+  if (threadIdx.x >> 5 == 1) tmem_alloc(&tmem_base_s, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* status = P.status;
+  for (;;) {
+    if (threadIdx.x == 0) {
+      int it = status[0] == 0 ? atomicAdd(P.sched, 1) : P.n_items;
+      if (it >= P.n_items) it = -1;
+      if (it >= 0) {
+        bool ok = true;
+        const long long t0 = clock64();
+        for (int q = P.pred_off[it]; q < P.pred_off[it + 1] && ok; ++q) {
+          const int* flag = P.done + P.preds[q];
+          while (ld_acquire(flag) != P.epoch) {
+            if (status[0] != 0 || clock64() - t0 > kWaitCycles) {
+              ok = false;
+              break;
+            }
+          }
+        }
+        if (ok && it == P.inject_item) {   // a flag that nothing sets: the wait runs out
+          while (status[0] == 0 && clock64() - t0 <= kWaitCycles) {
+          }
+          ok = false;
+        }
+        if (!ok) {
+          if (atomicCAS(P.status, 0, 7) == 0) P.status[1] = it;
+          it = -1;
+        }
+      }
+      item_s = it;
+    }
+    __syncthreads();
+    const int it = item_s;
+    if (it < 0) break;
+    // the predecessors' outputs were written by other CTAs' ordinary stores: make them visible to
+    // this CTA's tensor-memory-access loads
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    const int2 w = P.items[it];
+    const bool ok = P.steps[w.x].n > 256 ? halve512_body(P.maps[w.x], P.steps[w.x], w.y, smem, tmem)
+                                         : halve256_body(P.maps[w.x], P.steps[w.x], w.y, smem, tmem);
+    __threadfence();
+    __syncthreads();
+    if (!ok) break;
+    if (threadIdx.x == 0) st_release(P.done + it, P.epoch);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(P.sched + 1, 1) == (int)gridDim.x - 1) {
+      atomicExch(P.sched, 0);
+      atomicExch(P.sched + 1, 0);
+    }
+  }
+  if (threadIdx.x >> 5 == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
-bool halving_fused_supported(const StepArgs& a) {
-  if (std::getenv("THIN_ATTN_UNFUSED_HALVING") != nullptr) return false;
+// The shapes the one-launch kernels take (independent of the driver and the environment).
+bool halving_fused_shape_ok(const StepArgs& a) {
   if (a.E % 64 || a.D % 64 || (a.E + a.D) / 64 > kMaxChunks || a.n < 2 || a.n > 512 || a.n % 2) return false;
-  if (a.src_rows <= 0 || !tensor_maps_available()) return false;
+  if (a.src_rows <= 0) return false;
   // subsampled rows: an integer ratio is a strided view (runs on multiples of it); another ratio
   // needs the tokens spanned by an instance's n points, at most ceil((n-1) S / S') + 1, to fit the
   // box of NP rows of the persistent kernel
@@ -1262,6 +1396,56 @@ bool halving_fused_supported(const StepArgs& a) {
     if (span > NP) return false;
   }
   return true;
+}
+
+bool halving_fused_supported(const StepArgs& a) {
+  return std::getenv("THIN_ATTN_UNFUSED_HALVING") == nullptr && halving_fused_shape_ok(a) && tensor_maps_available();
+}
+
+// Dynamic shared memory the scheduler can give an instance: 227 KB per CTA less the static arrays of
+// both instance bodies (about 3.1 KB), with room to spare.
+constexpr size_t kSchedDynSmemMax = 232448 - 4096;
+
+bool halving_sched_shape_ok(const StepArgs& a) {
+  if (!halving_fused_shape_ok(a) || a.n <= 128) return false;
+  if (a.n <= 256) return smem_256(a) <= kSchedDynSmemMax;
+  return smem_512() <= kSchedDynSmemMax && (size_t)v_blocks_per_pass(a.D / 64) * (a.D / 64) * kChunk <= kDelta512Bytes;
+}
+
+bool halving_sched_step_supported(const StepArgs& a) { return halving_fused_supported(a) && halving_sched_shape_ok(a); }
+
+int halving_sched_max_steps() { return kSchedMaxSteps; }
+
+cudaError_t launch_halving_sched(const StepArgs* steps, int n_steps, const SchedTables& t, cudaStream_t st) {
+  if (n_steps < 1 || n_steps > kSchedMaxSteps || t.n_items == 0) return cudaErrorInvalidValue;
+  SchedParams P{};
+  size_t sm = 0;
+  for (int i = 0; i < n_steps; ++i) {
+    if (!halving_sched_step_supported(steps[i]) || !make_step_maps(steps[i], &P.maps[i])) return cudaErrorInvalidValue;
+    P.steps[i] = steps[i];
+    sm = std::max(sm, steps[i].n > 256 ? smem_512() : smem_256(steps[i]));
+  }
+  P.items = t.items;
+  P.pred_off = t.pred_off;
+  P.preds = t.preds;
+  P.n_items = t.n_items;
+  P.done = t.done;
+  P.epoch = t.epoch;
+  P.sched = t.sched;
+  P.status = t.status;
+  P.inject_item = t.inject_item;
+  int dev = 0, sms = 0, optin = 0;
+  cudaFuncAttributes fa{};
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, halve_sched_kernel);
+  if (e != cudaSuccess) return e;
+  if (sm + fa.sharedSizeBytes > (size_t)optin) return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(halve_sched_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  halve_sched_kernel<<<std::min(t.n_items, sms), 256, sm, st>>>(P);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_halving_fused(const StepArgs& a, cudaStream_t st) {

@@ -17,6 +17,23 @@ cudaError_t launch_pairgram_tc(const StepArgs& a, cudaStream_t st, bool* done);
 // rows that form TMA boxes): c^2, Gram, walk and gather fused, the points read once.
 bool halving_fused_supported(const StepArgs& a);
 cudaError_t launch_halving_fused(const StepArgs& a, cudaStream_t st);
+// Several halving steps of 129..512-point instances in one persistent launch, each work item (step,
+// instance) waiting for the items it depends on.  Tables in device memory, built by the host:
+struct SchedTables {
+  const int2* items;      // (step, instance) in queue order (a topological order of the dependencies)
+  const int* pred_off;    // predecessors of item i: preds[pred_off[i] .. pred_off[i + 1]) (item indices)
+  const int* preds;
+  int n_items;
+  int* done;              // per item: completion epoch (zeroed once; never equal to a live epoch before)
+  int epoch;              // this launch's epoch (>= 1, different from every earlier launch's)
+  int* sched;             // two ints: work counter and exit count, zero between launches
+  int* status;            // the handle's status word (code 7: a dependency wait gave up, [1] = item)
+  int inject_item;        // test hook: item whose wait runs out (-1: none)
+};
+bool halving_sched_shape_ok(const StepArgs& a);         // the plan's choice (shapes only)
+bool halving_sched_step_supported(const StepArgs& a);   // the launch's (and the driver's TMA, the environment)
+int halving_sched_max_steps();
+cudaError_t launch_halving_sched(const StepArgs* steps, int n_steps, const SchedTables& t, cudaStream_t st);
 // Copy of token runs into compact rows (batches that are not thinned).
 cudaError_t launch_copy_step(const StepArgs& a, int dtype, cudaStream_t st);
 cudaError_t launch_iota(int32_t* idx, int64_t rows, int period, cudaStream_t st);
@@ -28,7 +45,7 @@ int attention_simt_tile_rows();
 // Tensor-core attention (bf16, E = D = 128); *done = false when the shape is not covered.
 // Device status buffer of a handle (zeroed at creation): ints [0..3] the status word (code and
 // detail of a bounded wait that gave up), [4..5] the work counter of the persistent attention
-// kernel (left at zero by every launch).
+// kernels, [6..7] that of the halving scheduler (each left at zero by every launch).
 constexpr size_t kStatusBytes = 32;
 
 cudaError_t launch_attention_tc(const AttnArgs& a, int* status_word, cudaStream_t st, bool* done);
