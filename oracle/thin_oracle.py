@@ -315,16 +315,25 @@ class OracleOut:
     weights: Optional[np.ndarray] = None   # causal: (n_nodes,) node weights
 
 
-def thinformer(q, k, v, g, seed, scale=None, follow=None, rows=None, heads=None, b0=0):
+def _attn_operands(q, k, attn_q, attn_k):
+    """The q and k the attention step uses: by default the inputs themselves; the e4m3 QK^T path of
+    the library attends with e4m3-rounded copies (passed here, dequantised) while the thinning keeps
+    the original keys."""
+    return (q if attn_q is None else _f64(attn_q)), (k if attn_k is None else _f64(attn_k))
+
+
+def thinformer(q, k, v, g, seed, scale=None, follow=None, rows=None, heads=None, b0=0, attn_q=None, attn_k=None):
     """Non-causal Thinformer: per (b,h), KH-Compress the S keys/values to a coreset C,
     then weighted attention of every query against C with weight S/|C| per point.
 
     q (B,T,H,E), k (B,S,H,E), v (B,S,H,D) (torch or numpy; read as fp64).
     ``rows``: optional query rows to evaluate (all by default). ``heads``: global
     head ids of the H axis when the tensors hold a subset, ``b0``: the whole problem's
-    index of batch row 0 (Philox (b,h) word = (b0 + b)*H_total + h).
+    index of batch row 0 (Philox (b,h) word = (b0 + b)*H_total + h).  ``attn_q``, ``attn_k``:
+    the query and key tensors of the attention step when they differ from q, k (same shapes).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
+    qa, ka = _attn_operands(q, k, attn_q, attn_k)
     B, T, H, E = q.shape
     S = k.shape[1]
     scale = 1.0 / math.sqrt(E) if scale is None else scale
@@ -347,8 +356,8 @@ def thinformer(q, k, v, g, seed, scale=None, follow=None, rows=None, heads=None,
     logw = np.full(C, math.log(S / C)) if C > 0 else None
     for i in range(n_bh):
         b, h = divmod(i, H)
-        Kc, Vc = Kall[i, cidx[i]], Vall[i, cidx[i]]
-        o, l = weighted_attention(q[b, rsel, h], Kc, Vc, scale, logw)
+        Kc, Vc = ka[b, :, h][cidx[i]], Vall[i, cidx[i]]
+        o, l = weighted_attention(qa[b, rsel, h], Kc, Vc, scale, logw)
         out[b, :, h], lse[b, h] = o, l
     return OracleOut(out, lse, cidx.reshape(B, H, C), trace, stats)
 
@@ -383,7 +392,8 @@ def snapshot_nodes(k: int):
     return nodes
 
 
-def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, heads=None, b0=0):
+def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, heads=None, b0=0, attn_q=None,
+            attn_k=None):
     """Thinformer Express prefill (causal).
 
     * tokens [0, n_e): kept exactly (weight 1) -- exact phase;
@@ -395,8 +405,10 @@ def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, head
     * query t < n_e: exact causal attention; query t in batch k (k may be n_b for
       a trailing partial batch): the exact prefix, the nodes after k completed
       batches, and tokens [n_e + k b, t] of its own batch (weight 1).
+    ``attn_q``, ``attn_k``: as for thinformer.
     """
     q, k_, v = _f64(q), _f64(k), _f64(v)
+    qa, ka = _attn_operands(q, k_, attn_q, attn_k)
     B, T, H, E = q.shape
     D = v.shape[3]
     scale = 1.0 / math.sqrt(E) if scale is None else scale
@@ -406,7 +418,8 @@ def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, head
     bh = ((b0 + np.arange(B))[:, None] * Htot + hs[None, :]).reshape(-1)
     Kall = k_.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
     Vall = v.transpose(0, 2, 1, 3).reshape(n_bh, T, D)
-    Qall = q.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
+    Qall = qa.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
+    Kattn = ka.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
     n_b, slots = express_layout(T, n_e, bsz)
     trace: Trace = {}
     stats = Stats()
@@ -469,7 +482,7 @@ def express(q, k, v, n_e, bsz, g, seed, scale=None, follow=None, rows=None, head
                 logw = np.concatenate(lw)
                 mask = np.ones((len(tq), len(key)), dtype=bool)
                 mask[:, n_fixed:] = np.arange(start, end)[None, :] <= tq[:, None]
-            o, l = weighted_attention(Qall[i, tq], Kall[i, key], Vall[i, key], scale, logw, mask)
+            o, l = weighted_attention(Qall[i, tq], Kattn[i, key], Vall[i, key], scale, logw, mask)
             out[b, sel, h] = o
             lse[b, h, sel] = l
     coreset = (np.stack([nodes[s] for s in slots], axis=1).reshape(B, H, len(slots), c)
@@ -513,7 +526,8 @@ def express_a_layout(T: int, n_out: int):
     return out
 
 
-def express_a(q, k, v, n_out, g, seed, scale=None, follow=None, rows=None, heads=None, b0=0, _plant=None):
+def express_a(q, k, v, n_out, g, seed, scale=None, follow=None, rows=None, heads=None, b0=0, _plant=None,
+              attn_q=None, attn_k=None):
     """Thinformer Express prefill with the page-literal cache (reading A).
 
     The cache holds points of one weight m, the inflation factor (m = 1 at the start):
@@ -532,8 +546,10 @@ def express_a(q, k, v, n_out, g, seed, scale=None, follow=None, rows=None, heads
     Coreset slots, in order: for i = 1, 2, ...: H_i, then the thinned batches of level i, each
     present only if a query uses it (directly or through a later HALVE).
     ``_plant`` (test hook): "weight" gives the thinned points the weight of the previous level.
+    ``attn_q``, ``attn_k``: as for thinformer.
     """
     q, k_, v = _f64(q), _f64(k), _f64(v)
+    qa, ka = _attn_operands(q, k_, attn_q, attn_k)
     B, T, H, E = q.shape
     D = v.shape[3]
     scale = 1.0 / math.sqrt(E) if scale is None else scale
@@ -543,7 +559,8 @@ def express_a(q, k, v, n_out, g, seed, scale=None, follow=None, rows=None, heads
     bh = ((b0 + np.arange(B))[:, None] * Htot + hs[None, :]).reshape(-1)
     Kall = k_.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
     Vall = v.transpose(0, 2, 1, 3).reshape(n_bh, T, D)
-    Qall = q.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
+    Qall = qa.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
+    Kattn = ka.transpose(0, 2, 1, 3).reshape(n_bh, T, E)
     layout = express_a_layout(T, n_out)
     trace: Trace = {}
     stats = Stats()
@@ -613,7 +630,7 @@ def express_a(q, k, v, n_out, g, seed, scale=None, follow=None, rows=None, heads
                 logw = np.concatenate(lw)
                 mask = np.ones((len(tq), len(key)), dtype=bool)
                 mask[:, n_fixed:] = np.arange(start, start + length)[None, :] <= tq[:, None]
-            o, l = weighted_attention(Qall[n, tq], Kall[n, key], Vall[n, key], scale, logw, mask)
+            o, l = weighted_attention(Qall[n, tq], Kattn[n, key], Vall[n, key], scale, logw, mask)
             out[b, sel, h] = o
             lse[b, h, sel] = l
     coreset = (np.stack([nodes[sl] for sl in slots], axis=1).reshape(B, H, len(slots), n_out)

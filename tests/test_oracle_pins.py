@@ -519,3 +519,30 @@ def test_express_a_node_structure():
         for h in range(2):
             node = o.coreset[0, h, sl]
             assert len(node) == 16 and np.all(np.diff(node) > 0) and node[0] >= lo and node[-1] < hi
+
+
+def test_attention_operands_leave_the_thinning_alone():
+    """Attention with separately given q and k (the e4m3 QK^T path attends with rounded copies) keeps
+    the coresets and the decisions of the original keys; given the inputs themselves it is the default
+    run bit for bit; and its outputs are the weighted attention of those operands over the same keys."""
+    w = W.WORKLOADS["express32k"].with_(T=1280, H=2, n_exact=128, batch=128)
+    q, k, v = W.make_qkv(w)
+    rows = np.arange(0, 1280, 53)
+    base = express(q, k, v, 128, 128, 2, 4, rows=rows)
+    same = express(q, k, v, 128, 128, 2, 4, rows=rows, attn_q=q, attn_k=k)
+    assert np.array_equal(base.out, same.out) and np.array_equal(base.lse, same.lse)
+    qa, ka = q.double() * 1.5, k.double().flip(-1)
+    alt = express(q, k, v, 128, 128, 2, 4, rows=rows, attn_q=qa, attn_k=ka)
+    assert np.array_equal(alt.coreset, base.coreset) and alt.trace.keys() == base.trace.keys()
+    assert all(np.array_equal(alt.trace[key], base.trace[key]) for key in base.trace)
+    # exact-phase rows (t < n_e): plain causal attention of the given operands
+    t = rows[rows < 128]
+    o, _ = weighted_attention(qa[0, t, 1].numpy(), ka[0, :128, 1].numpy(), v[0, :128, 1].double().numpy(), w.scale,
+                              None, np.arange(128)[None, :] <= t[:, None])
+    np.testing.assert_allclose(alt.out[0, :len(t), 1], o, rtol=1e-12, atol=1e-14)
+    # Thinformer likewise
+    wt = W.WORKLOADS["tiny"]
+    qt, kt, vt = W.make_qkv(wt)
+    b0 = thinformer(qt, kt, vt, 2, 1)
+    b1 = thinformer(qt, kt, vt, 2, 1, attn_q=qt * 2.0, attn_k=kt)
+    assert np.array_equal(b0.coreset, b1.coreset) and not np.allclose(b0.out, b1.out)
