@@ -79,6 +79,12 @@ typedef struct {
   int b0;          /* whole-problem index of this handle's batch row 0 */
   int h0;          /* whole-problem index of this handle's head 0 */
   int H_total;     /* heads of the whole problem; <= 0 selects H */
+  /* QK^T in e4m3 (FP8; "Express Language Modeling", Limitations, lists FP8 as unexploited): 0 keeps
+   * bf16.  1: after the thinning, q, k and the coreset keys are copied to e4m3 with one scale per
+   * (b,h) and tensor (its largest |x| maps to 448), S = q8 k8^T on the tensor cores' e4m3 path and
+   * the scales undone in the softmax; P V stays bf16.  The thinning always uses the bf16 keys.  bf16
+   * handles with E = 128, D <= 128, H <= 128; EUNSUPPORTED otherwise.  The decode cache ignores it. */
+  int qk_fp8;
 } thin_attn_config;
 
 /* Sizes of one (causal, g) plan. */

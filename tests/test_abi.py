@@ -263,3 +263,12 @@ def test_sched_layout_noncausal_has_none():
     for name in ("vit", "biggan"):
         w = W.WORKLOADS[name]
         assert _handle(w).sched_layout(False, w.g) == ([], [])
+
+
+@pytest.mark.parametrize("kw", [dict(E=64), dict(D=256), dict(dtype="fp32", E=128, D=128), dict(H=129)])
+def test_fp8_qk_refuses_unsupported_shapes(kw):
+    """e4m3 QK^T is built for bf16 handles with E = 128 and D = 64 or 128: anything else is refused at
+    creation, before any device work."""
+    w = W.WORKLOADS["express32k"].with_(**kw)
+    with pytest.raises(T.ThinAttnError, match="EUNSUPPORTED"):
+        T.ThinAttention(w.B, w.T, w.T, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch, qk_fp8=True)

@@ -37,7 +37,7 @@ class Config(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("B", ctypes.c_int), ("T", ctypes.c_int), ("S", ctypes.c_int),
                 ("H", ctypes.c_int), ("E", ctypes.c_int), ("D", ctypes.c_int), ("scale", ctypes.c_float),
                 ("n_exact", ctypes.c_int), ("batch", ctypes.c_int), ("device", ctypes.c_int),
-                ("b0", ctypes.c_int), ("h0", ctypes.c_int), ("H_total", ctypes.c_int)]
+                ("b0", ctypes.c_int), ("h0", ctypes.c_int), ("H_total", ctypes.c_int), ("qk_fp8", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -118,6 +118,9 @@ class ThinAttention:
     attention weights are never formed; the layer call ``thinformer_attention`` returns
     ``(attn_output, None)``.
 
+    ``qk_fp8=True``: QK^T in e4m3 with one scale per (b,h) for q and for k (E = 128, bf16); the
+    thinning keeps the bf16 keys.
+
     ``shard=(b0, h0, H_total)``: the tensors hold batch rows [b0, b0 + B) and heads
     [h0, h0 + H) of a larger problem with H_total heads (one handle per GPU of a batch- or
     head-parallel run); the random decisions, and so every output, equal the whole
@@ -126,9 +129,9 @@ class ThinAttention:
 
     def __init__(self, B: int, T: int, S: int, H: int, E: int, D: int, dtype: torch.dtype,
                  scale: Optional[float] = None, n_exact: int = 0, batch: int = 0, device: int = 0,
-                 shard: Tuple[int, int, int] = (0, 0, 0)):
+                 shard: Tuple[int, int, int] = (0, 0, 0), qk_fp8: bool = False):
         self.cfg = Config(FP32 if dtype == torch.float32 else BF16, B, T, S, H, E, D,
-                          0.0 if scale is None else float(scale), n_exact, batch, device, *shard)
+                          0.0 if scale is None else float(scale), n_exact, batch, device, *shard, int(qk_fp8))
         self.dtype = dtype
         self.device = torch.device("cuda", device)
         self._h = ctypes.c_void_p()

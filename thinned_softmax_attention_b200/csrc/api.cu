@@ -173,6 +173,9 @@ struct Plan {
   size_t sched_items_off = 0, sched_pred_off_off = 0, sched_preds_off = 0, sched_done_off = 0;
   int sched_epoch = 0;
   size_t delta_off = 0, c2_off = 0, delta_floats = 0, c2_floats = 0;
+  // e4m3 QK^T (thin_attn_config::qk_fp8): q8, k8, ck8 copies, the amax words, scales and 1/(sq sk)
+  size_t fp8_q_off = 0, fp8_k_off = 0, fp8_ck_off = 0, fp8_amax_off = 0, fp8_scales_off = 0, fp8_inv_off = 0;
+  int64_t fp8_ck_rows = 0;
   size_t bytes = 0;
   void* d_mem = nullptr;
 };
@@ -870,6 +873,22 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
   off = align256(off + p->delta_floats * 4);
   p->c2_off = off;
   off = align256(off + p->c2_floats * 4);
+  if (cf.qk_fp8) {
+    const int64_t BH = (int64_t)cf.B * cf.H, L = causal ? cf.T : cf.S;
+    p->fp8_ck_rows = p->final_buf != BUF_TOKENS ? BH * p->att_slots * p->att_slot_rows : 0;
+    p->fp8_q_off = off;
+    off = align256(off + (size_t)cf.B * cf.T * cf.H * cf.E);
+    p->fp8_k_off = off;
+    off = align256(off + (size_t)cf.B * L * cf.H * cf.E);
+    p->fp8_ck_off = off;
+    off = align256(off + (size_t)p->fp8_ck_rows * cf.E);
+    p->fp8_amax_off = off;
+    off = align256(off + (size_t)2 * BH * 4);
+    p->fp8_scales_off = off;
+    off = align256(off + (size_t)2 * BH * 4);
+    p->fp8_inv_off = off;
+    off = align256(off + (size_t)BH * 4);
+  }
   p->bytes = off;
   *out = p;
   return THIN_ATTN_OK;
@@ -941,6 +960,10 @@ thin_attn_status check_cfg(const thin_attn_config* c) {
                 (long long)Ht);
   if (((int64_t)c->b0 + c->B) * Ht > (int64_t)UINT32_MAX)
     return fail(THIN_ATTN_EINVAL, "(b0 + B) * H_total exceeds the 32-bit Philox (b,h) word");
+  if (c->qk_fp8 != 0 && c->qk_fp8 != 1) return fail(THIN_ATTN_EINVAL, "qk_fp8 must be 0 or 1");
+  if (c->qk_fp8 && (c->dtype != THIN_ATTN_BF16 || c->E != 128 || c->D > 128 || c->D % 64 || !qk_fp8_supported(c->H, c->E)))
+    return fail(THIN_ATTN_EUNSUPPORTED, "qk_fp8 needs bf16 with E = 128, D = 64 or 128 and H <= 128 (E=%d D=%d H=%d)", c->E,
+                c->D, c->H);
   return THIN_ATTN_OK;
 }
 
@@ -1022,7 +1045,8 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   // step it depends on, so the tensor cores work while later (latency-bound) halving steps run.
   // By default one attention launch follows all halving steps on the caller's stream: the waves
   // save ~3 % of an Express step but share SMs with the halving kernels.
-  const bool side = tab.waves.size() > 1 && std::getenv("THIN_ATTN_OVERLAP") != nullptr;
+  const bool fp8 = cf.qk_fp8 && use_tc_attn;
+  const bool side = tab.waves.size() > 1 && std::getenv("THIN_ATTN_OVERLAP") != nullptr && !fp8;
   const std::vector<AttnWave> one_wave = {{0, (int)tab.tiles.size(), (int)p->steps.size() - 1}};
   const std::vector<AttnWave>& waves = side ? tab.waves : one_wave;
   cudaStream_t sa = st;
@@ -1114,7 +1138,8 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
       }
       aa.tile0 = w.tile0;
       aa.n_tiles = w.count;
-      if (!ev.empty()) CK(cudaEventRecord(ev[4 + 2 * next_wave], sa));
+      // (with e4m3 QK^T the attention phase starts before the copies of q and k, recorded there)
+      if (!ev.empty() && !(fp8 && next_wave == 0)) CK(cudaEventRecord(ev[4 + 2 * next_wave], sa));
       bool done = false;
       cudaError_t e = cudaSuccess;
       if (use_tc_attn) e = launch_attention_tc(aa, h->d_status, sa, &done);
@@ -1220,6 +1245,35 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   if (!ev.empty()) {
     if (!merged_mark) CK(cudaEventRecord(ev[1], st));
     CK(cudaEventRecord(ev[2], st));
+  }
+  if (fp8) {
+    // e4m3 copies of q, k and the coreset keys for the attention's QK^T (timed with the attention)
+    QkFp8Args fa{};
+    fa.q = q;
+    fa.k = k;
+    fa.ck = p->fp8_ck_rows > 0 ? aa.ck : nullptr;
+    fa.B = cf.B;
+    fa.T = cf.T;
+    fa.L = p->causal ? cf.T : cf.S;
+    fa.H = cf.H;
+    fa.E = cf.E;
+    fa.ck_rows = p->fp8_ck_rows;
+    fa.rows_per_bh = (int64_t)p->att_slots * p->att_slot_rows;
+    fa.q8 = (uint8_t*)(base_of(p) + p->fp8_q_off);
+    fa.k8 = (uint8_t*)(base_of(p) + p->fp8_k_off);
+    fa.ck8 = (uint8_t*)(base_of(p) + p->fp8_ck_off);
+    fa.amax = (unsigned*)(base_of(p) + p->fp8_amax_off);
+    fa.scales = (float*)(base_of(p) + p->fp8_scales_off);
+    fa.qk_inv = (float*)(base_of(p) + p->fp8_inv_off);
+    if (!ev.empty()) CK(cudaEventRecord(ev[4], sa));
+    cudaError_t e = launch_qk_fp8(fa, st);
+    if (e != cudaSuccess) return fail(THIN_ATTN_ECUDA, "e4m3 copies of q and k: %s", cudaGetErrorString(e));
+    aa.q8 = fa.q8;
+    aa.k8 = fa.k8;
+    aa.ck8 = p->fp8_ck_rows > 0 ? fa.ck8 : nullptr;
+    aa.qk_inv = fa.qk_inv;
+    aa.pairs = nullptr;   // the e4m3 S MMAs are in the two-CTA kernel
+    aa.n_pairs = 0;
   }
   ls = launch_waves_after((int)p->steps.size());
   if (ls != THIN_ATTN_OK) return ls;

@@ -364,11 +364,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 // thread issues S(j+1) right after PV(j): the tensor-core pipeline runs one thread's MMAs in
 // issue order, so PV(j) reads P(j) before S(j+1) overwrites it.
 // The softmax reads S twice (max pass, then exponent pass) to stay within 170 registers.
-template <int E, int D>
+template <int E, int D, bool FP8 = false>
 struct Tc2Layout {
-  static constexpr int EC = E / 64, DC = D / 64;
-  static constexpr uint32_t Q_BYTES = BM * E * 2;
-  static constexpr uint32_t K_BYTES = BN * E * 2;
+  // Q and K in 128-byte rows of chunks: 64 bf16 or 128 e4m3 elements each
+  static constexpr int CW = FP8 ? 128 : 64;
+  static constexpr int EC = E / CW, DC = D / 64;
+  static constexpr uint32_t Q_BYTES = BM * E * (FP8 ? 1 : 2);
+  static constexpr uint32_t K_BYTES = BN * E * (FP8 ? 1 : 2);
   static constexpr uint32_t V_BYTES = BN * D * 2;
   static constexpr uint32_t OFF_K = Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + K_BYTES;
@@ -706,10 +708,10 @@ __global__ void __launch_bounds__(192, 2) attn_tc2_kernel(const __grid_constant_
 // MMA of the current item has read Q (q_empty), and the next item's first S MMA runs while the
 // softmax warps write the current item's O (the first PV of an item waits for that: o_empty).
 // Barrier parities follow a key-tile count and an item count that run across items.
-template <int E, int D>
+template <int E, int D, bool FP8 = false>
 __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a,
                                                            int* status) {
-  using Lay = Tc2Layout<E, D>;
+  using Lay = Tc2Layout<E, D, FP8>;
   constexpr uint32_t O_COL = 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -784,7 +786,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
         const int bh = j / a.n_tiles, b = bh / a.H, h = bh % a.H;
         mbar_expect_tx(q_full, Lay::Q_BYTES);
 #pragma unroll
-        for (int c = 0; c < Lay::EC; ++c) tma_load_3d(sQ + c * 16384, &maps.q, q_full, c * 64, h, b * a.T + tile.q0);
+        for (int c = 0; c < Lay::EC; ++c) tma_load_3d(sQ + c * 16384, &maps.q, q_full, c * Lay::CW, h, b * a.T + tile.q0);
         for (int si = 0; si < tile.nseg && ok; ++si) {
           const AttnSeg sg = a.segs[tile.seg0 + si];
           const bool tok = sg.kind == SEG_TOKENS;
@@ -800,8 +802,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
               mbar_expect_tx(k_full, Lay::K_BYTES);
 #pragma unroll
               for (int c = 0; c < Lay::EC; ++c) {
-                if (tok) tma_load_3d(sK + c * 16384, &maps.k, k_full, c * 64, h, row);
-                else tma_load_2d(sK + c * 16384, &maps.ck, k_full, c * 64, row);
+                if (tok) tma_load_3d(sK + c * 16384, &maps.k, k_full, c * Lay::CW, h, row);
+                else tma_load_2d(sK + c * 16384, &maps.ck, k_full, c * Lay::CW, row);
               }
             }
             if (git > 0 && !mbar_wait(v_empty, (git - 1) & 1, abort)) {
@@ -837,7 +839,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IQK = idesc_bf16(BM, BN, false);
+      constexpr uint32_t IQK = FP8 ? idesc_e4m3(BM, BN) : idesc_bf16(BM, BN, false);
       constexpr uint32_t IPV = idesc_bf16(BM, D, true);
       const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
       int git = 0;
@@ -862,9 +864,11 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
           }
           tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < E / 16; ++k) {
+          // 32 bytes of K per instruction: 16 bf16 or 32 e4m3 elements
+          for (int k = 0; k < E / (FP8 ? 32 : 16); ++k) {
             const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-            umma_bf16(tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), IQK, k > 0);
+            if (FP8) umma_e4m3(tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), IQK, k > 0);
+            else umma_bf16(tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), IQK, k > 0);
           }
           umma_commit(s_full);
           umma_commit(k_empty);
@@ -917,6 +921,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
       }
       if (threadIdx.x == 0) item_s = tile_id * 65536 + bh;
       const int tq = tile.q0 + row;
+      // e4m3 scores are q k^T times scale_q scale_k: the (b,h) factor that undoes it joins s log2 e
+      const float sl2e = FP8 ? a.scale_log2e * a.qk_inv[bh] : a.scale_log2e;
       float m_used = -INFINITY, l = 0.f;
       int it = 0;
       for (int si = 0; si < tile.nseg && ok; ++si) {
@@ -934,8 +940,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
           const bool causal = sg.kind == SEG_TOKENS && sg.causal;
           const bool masked = nvalid < BN || (causal && kt0 + BN - 1 > tile.q0);
           const int lim = min(nvalid - 1, causal ? tq - kt0 : BN - 1);
-          if (masked) softmax_tile<true, D>(tmem + lane_base, tmem + lane_base + 128, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
-          else softmax_tile<false, D>(tmem + lane_base, tmem + lane_base + 128, lim, a.scale_log2e, lw2, it, m_used, l, p_half);
+          if (masked) softmax_tile<true, D>(tmem + lane_base, tmem + lane_base + 128, lim, sl2e, lw2, it, m_used, l, p_half);
+          else softmax_tile<false, D>(tmem + lane_base, tmem + lane_base + 128, lim, sl2e, lw2, it, m_used, l, p_half);
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(p_full);
@@ -1554,6 +1560,27 @@ cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
     maps.cv = maps.v;
   }
   if (!ok) return cudaErrorInvalidValue;
+  if constexpr (E == 128 && D <= 128) {
+    if (a.q8) {
+      // e4m3 QK^T: the persistent two-CTA kernel with its S MMAs on e4m3 copies of q and the keys
+      TcMaps m8 = maps;
+      bool ok8 = status && make_map_3d_u8(&m8.q, a.q8, (int64_t)a.B * a.T, a.H, E, 128) &&
+                 make_map_3d_u8(&m8.k, a.k8, (int64_t)a.B * a.L, a.H, E, 128);
+      if (ok8 && a.ck8 && compact_rows > 0) ok8 = make_map_2d_u8(&m8.ck, a.ck8, compact_rows, E, E, 128);
+      else m8.ck = m8.k;
+      if (!ok8) return cudaErrorInvalidValue;
+      int dev = 0, sms = 0;
+      cudaError_t e = cudaGetDevice(&dev);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      const size_t sm = Tc2Layout<E, D, true>::BYTES;
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(attn_tc2p_kernel<E, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if (e != cudaSuccess) return e;
+      const int64_t items = (int64_t)a.n_tiles * a.B * a.H;
+      attn_tc2p_kernel<E, D, true><<<(int)std::min<int64_t>(items, 2 * (int64_t)sms), 192, sm, st>>>(m8, a, status);
+      return cudaGetLastError();
+    }
+  }
   if constexpr (D <= 128 && E <= 128) {
     if (a.pairs && a.n_pairs > 0 && status && std::getenv("THIN_ATTN_TC1") == nullptr &&
         std::getenv("THIN_ATTN_TC2_PER_TILE") == nullptr) {
@@ -1656,6 +1683,26 @@ bool make_map_4d_strided(CUtensorMap* m, const void* base, int64_t BL, int H, in
   cuuint32_t box[4] = {64, 1, 1, (cuuint32_t)box_rows};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, (void*)base, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// e4m3 (one byte per element) forms of make_map_2d / make_map_3d: boxes of 128 elements (128 bytes).
+bool make_map_2d_u8(CUtensorMap* m, const void* base, int64_t rows, int width, int64_t row_stride, int box_rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride};
+  cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)base, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool make_map_3d_u8(CUtensorMap* m, const void* base, int64_t BL, int H, int width, int box_rows) {
+  cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)BL};
+  cuuint64_t strides[2] = {(cuuint64_t)width, (cuuint64_t)width * H};
+  cuuint32_t box[3] = {128, 1, (cuuint32_t)box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)base, dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -198,6 +198,12 @@ struct AttnArgs {
   // (x = -1: B alone); pairs [pair0, pair0 + n_pairs) of the table.  Null: no pairs.
   const int2* pairs;
   int pair0, n_pairs;
+  // e4m3 QK^T (null: bf16): q8, k8 and ck8 hold q, k and the compact keys times the (b,h) scales,
+  // rounded to e4m3 (same layouts, one byte per element); qk_inv[bh] = 1 / (scale_q * scale_k)
+  const void* q8;
+  const void* k8;
+  const void* ck8;
+  const float* qk_inv;
 };
 
 }  // namespace thin

@@ -76,5 +76,29 @@ bool make_map_3d(CUtensorMap* m, const void* base, int64_t BL, int H, int width,
 // 4D view over every k-th row (a systematic subsample with integer ratio k): box (64, 1, 1, box_rows)
 // at (x, h, 0, R) holds rows R k, (R+1) k, ...
 bool make_map_4d_strided(CUtensorMap* m, const void* base, int64_t BL, int H, int width, int k, int box_rows);
+// The same 2D / 3D maps over one-byte (e4m3) elements, boxes of 128 elements.
+bool make_map_2d_u8(CUtensorMap* m, const void* base, int64_t rows, int width, int64_t row_stride, int box_rows);
+bool make_map_3d_u8(CUtensorMap* m, const void* base, int64_t BL, int H, int width, int box_rows);
+
+// e4m3 copies for QK^T (thin_attn_config::qk_fp8).  Per (b,h): scale_q = 448 / max|q| over its T
+// rows, scale_k = 448 / max|k| over its L token rows (1 when the maximum is 0); q8 = e4m3(q scale_q),
+// k8 = e4m3(k scale_k), ck8 = e4m3(ck scale_k) for the compact key rows (rows_per_bh rows per (b,h));
+// qk_inv[bh] = 1 / (scale_q scale_k).  `amax` (2 B H words) is cleared here.  bf16 inputs, E a
+// multiple of 8 and H E / 8 <= 2048.
+struct QkFp8Args {
+  const void* q;
+  const void* k;
+  const void* ck;          // may be null (no compact rows)
+  int B, T, L, H, E;
+  int64_t ck_rows, rows_per_bh;
+  uint8_t* q8;
+  uint8_t* k8;
+  uint8_t* ck8;
+  unsigned* amax;          // [2][B H] scratch
+  float* scales;           // [2][B H]: scale_q, scale_k
+  float* qk_inv;           // [B H]
+};
+bool qk_fp8_supported(int H, int E);
+cudaError_t launch_qk_fp8(const QkFp8Args& a, cudaStream_t st);
 
 }  // namespace thin
