@@ -54,6 +54,8 @@ def args_():
     p.add_argument("--no-sdpa", action="store_true")
     p.add_argument("--no-per-workload", action="store_true",
                    help="N=1: skip the GPU-timed records of the other workloads")
+    p.add_argument("--heads", type=int, default=0,
+                   help="run the workload with this many heads instead of its own (small cases for profilers)")
     p.add_argument("--decode", action="store_true",
                    help="time token-by-token decoding of the workload through the Express decode cache "
                         "(causal workloads; prints its own JSON line)")
@@ -440,8 +442,9 @@ def halving_roofline(w, h, ph, pk):
     return {"bound": "hbm", "achieved": round(top["bytes"] / (top["ms"] * 1e-3) / 1e9, 1),
             "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": top["frac"], "kernel": top["kernel"],
             "algorithmic_bytes_per_launch": top["bytes"], "avg_launch_ms": top["ms"],
-            "traffic": (kernel_traffic("halving_fused_n64") if (w.name == "express32k" and len(top["steps"]) == 1
-                                                                and top["steps"][0]["n"] == 64) else None),
+            "traffic": (None if w.name != "express32k" or w.H != 32 else
+                        kernel_traffic("halving_sched") if len(top["steps"]) > 1 else
+                        kernel_traffic("halving_fused_n64") if top["steps"][0]["n"] == 64 else None),
             "all_steps": {"achieved": round(hbytes / (hms * 1e-3) / 1e9, 1) if hms > 0 else None,
                           "frac": round(hbytes / (hms * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if hms > 0 else None,
                           "bytes": hbytes, "ms": round(hms, 4)},
@@ -534,7 +537,8 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    shard = Shard(W.WORKLOADS[a.workload], world, rank, a.shard)
+    wl = W.WORKLOADS[a.workload] if a.heads <= 0 else W.WORKLOADS[a.workload].with_(H=a.heads)
+    shard = Shard(wl, world, rank, a.shard)
     w = shard.local
     qc, kc, vc = shard.inputs(w)
     q, k, v = (x.to(dev) for x in (qc, kc, vc))
@@ -574,7 +578,7 @@ def main():
     pk = peaks()
     attn_ms = ph["attn_ms"] / max(1, ph["calls"])
     roof = attention_roofline(w, plan, attn_ms, pk)
-    roof["traffic"] = kernel_traffic("attention") if w.name == "express32k" else None
+    roof["traffic"] = kernel_traffic("attention") if (w.name == "express32k" and w.H == 32) else None
     halving_roof = halving_roofline(w, h, ph, pk)
     phases = {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
               "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4),
@@ -643,7 +647,7 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": shard.scaling,
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {**config_of(W.WORKLOADS[a.workload]), "global_batch": shard.global_batch,
+            "config": {**config_of(wl), "global_batch": shard.global_batch,
                        "parallelism": shard.parallelism, "heads_per_gpu": w.H},
             "ms_per_layer": ms, "phases_ms": phases, "roofline": roof, "halving_roofline": halving_roof,
             "approx_error": approx, "cpu_baseline": cpu, "e2e": e2e,
