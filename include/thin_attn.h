@@ -238,6 +238,14 @@ THIN_ATTN_API thin_attn_status thin_attn_cache_destroy(thin_attn_cache_t c);
 THIN_ATTN_API thin_attn_status thin_attn_cache_length(thin_attn_cache_t c, int64_t* t);
 THIN_ATTN_API thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, const void* k,
                                                       const void* v, void* out, float* lse_opt, void* stream);
+/* n consecutive tokens of every (b,h) in one call: q, k (B,n,H,E), v, out (B,n,H,D) device, lse_opt
+ * (B,H,n) or NULL.  Token i attends to the cache after tokens 0..i-1 of the call, exactly as n calls
+ * of thin_attn_cache_decode would (same kernels, bit-identical results), without a host round trip
+ * per token.  EINVAL if the capacity would be exceeded; EUNSUPPORTED for n > 1 when B*H > 64 (the
+ * query-tile decode path). */
+THIN_ATTN_API thin_attn_status thin_attn_cache_decode_n(thin_attn_cache_t c, const void* q, const void* k,
+                                                       const void* v, void* out, float* lse_opt, int n,
+                                                       void* stream);
 /* Device int32 (B,H,n_nodes,c) token indices of every coreset slot (-1 while empty), in the
  * node order of thin_attn_forward's coreset output. */
 THIN_ATTN_API thin_attn_status thin_attn_cache_nodes(thin_attn_cache_t c, int32_t* idx_out, void* stream);

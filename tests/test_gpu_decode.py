@@ -66,6 +66,37 @@ def test_decode_matches_oracle(T, n_e, bsz, g, dtype, tiles, monkeypatch):
     assert np.abs(lse - ref.lse).max() <= LSE_TOL[dtype]
 
 
+@pytest.mark.parametrize("chunks", [[1, 7, 64, 200, 500, 380], [1152]])
+def test_decode_n_equals_token_by_token(chunks):
+    """Several tokens per call (batch boundaries, merges and the exact phase crossed inside a call):
+    outputs, LSE and coresets bit-identical to one call per token."""
+    T, n_e, bsz, g = 1152, 128, 64, 2
+    w = W.Workload("decode", 1, 2, T, T, 128, 128, "bf16", True, g, 9, 6, "rope", n_exact=n_e, batch=bsz)
+    q, k, v = (x.cuda() for x in W.make_qkv(w))
+    one = TA.ThinAttentionCache(1, 2, 128, 128, w.torch_dtype, capacity=T, n_exact=n_e, batch=bsz, g=g, seed=w.seed)
+    outs, lses = [], []
+    for t in range(T):
+        lse = torch.empty(1, 2, dtype=torch.float32, device="cuda")
+        outs.append(one.decode(q[:, t:t + 1].contiguous(), k[:, t:t + 1].contiguous(), v[:, t:t + 1].contiguous(),
+                               lse=lse))
+        lses.append(lse)
+    many = TA.ThinAttentionCache(1, 2, 128, 128, w.torch_dtype, capacity=T, n_exact=n_e, batch=bsz, g=g, seed=w.seed)
+    got, got_lse, t0 = [], [], 0
+    for n in chunks:
+        lse = torch.empty(1, 2, n, dtype=torch.float32, device="cuda")
+        got.append(many.decode_n(q[:, t0:t0 + n].contiguous(), k[:, t0:t0 + n].contiguous(),
+                                 v[:, t0:t0 + n].contiguous(), lse=lse))
+        got_lse.append(lse)
+        t0 += n
+    torch.cuda.synchronize()
+    one.check()
+    many.check()
+    assert t0 == T and len(many) == T
+    assert torch.equal(torch.cat(outs, dim=1), torch.cat(got, dim=1))
+    assert torch.equal(torch.stack(lses, dim=2), torch.cat(got_lse, dim=2))
+    assert torch.equal(one.nodes(), many.nodes())
+
+
 def test_cache_refuses_tokens_beyond_capacity():
     w = W.WORKLOADS["express32k"].with_(H=1)
     cache = TA.ThinAttentionCache(1, 1, w.E, w.D, w.torch_dtype, capacity=2, n_exact=1, batch=1, g=0, seed=1)

@@ -58,7 +58,7 @@ EXPORTS = ("thin_attn_version", "thin_attn_last_error", "thin_attn_create", "thi
            "thin_attn_forward_host", "thin_attn_check", "thin_attn_profile", "thin_attn_profile_read",
            "thin_attn_profile_steps",
            "thin_attn_cache_create", "thin_attn_cache_destroy", "thin_attn_cache_length", "thin_attn_cache_decode",
-           "thin_attn_cache_nodes", "thin_attn_cache_check", "thin_attn_sched_layout")
+           "thin_attn_cache_nodes", "thin_attn_cache_check", "thin_attn_sched_layout", "thin_attn_cache_decode_n")
 
 
 def lib() -> ctypes.CDLL:
@@ -85,6 +85,7 @@ def lib() -> ctypes.CDLL:
     L.thin_attn_cache_destroy.argtypes = [vp]
     L.thin_attn_cache_length.argtypes = [vp, ctypes.POINTER(ctypes.c_int64)]
     L.thin_attn_cache_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+    L.thin_attn_cache_decode_n.argtypes = [vp, vp, vp, vp, vp, vp, i, vp]
     L.thin_attn_cache_nodes.argtypes = [vp, vp, vp]
     L.thin_attn_cache_check.argtypes = [vp, vp]
     sz = ctypes.c_size_t
@@ -269,6 +270,7 @@ class ThinAttentionCache:
                                             ctypes.c_uint64(seed & (2 ** 64 - 1))))
         plan = ThinAttention(B, capacity, capacity, H, E, D, dtype, scale, n_exact, batch, device).plan(True, g)
         self.n_nodes, self.node_rows = plan["n_nodes"], plan["coreset_rows"]
+        self._shapes = None
 
     def close(self):
         if self._h:
@@ -289,14 +291,33 @@ class ThinAttentionCache:
     def decode(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
                lse: Optional[torch.Tensor] = None) -> torch.Tensor:
         c = self.cfg
-        for name, t, shape in (("q", q, (c.B, 1, c.H, c.E)), ("k", k, (c.B, 1, c.H, c.E)), ("v", v, (c.B, 1, c.H, c.D))):
-            if tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous() or t.device != self.device:
+        if self._shapes is None:
+            self._shapes = ((c.B, 1, c.H, c.E), (c.B, 1, c.H, c.E), (c.B, 1, c.H, c.D))
+            self._decode_fn = lib().thin_attn_cache_decode
+        for name, t, shape in zip("qkv", (q, k, v), self._shapes):
+            if t.shape != shape or t.dtype != self.dtype or not t.is_contiguous() or t.device != self.device:
                 raise ValueError(f"{name}: expected contiguous {self.dtype} {shape} on {self.device}")
         if out is None:
             out = torch.empty(c.B, 1, c.H, c.D, dtype=self.dtype, device=self.device)
         stream = torch.cuda.current_stream(self.device).cuda_stream
-        _check(lib().thin_attn_cache_decode(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
-                                            ctypes.c_void_p(stream)))
+        _check(self._decode_fn(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               None if lse is None else lse.data_ptr(), stream))
+        return out
+
+    def decode_n(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """n consecutive tokens in one call: (B,n,H,E), (B,n,H,E), (B,n,H,D) -> (B,n,H,D); the same
+        results as n calls of decode, without a host round trip per token.  ``lse``: (B,H,n) fp32."""
+        c = self.cfg
+        n = q.shape[1]
+        for name, t, shape in (("q", q, (c.B, n, c.H, c.E)), ("k", k, (c.B, n, c.H, c.E)), ("v", v, (c.B, n, c.H, c.D))):
+            if tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous() or t.device != self.device:
+                raise ValueError(f"{name}: expected contiguous {self.dtype} {shape} on {self.device}")
+        if out is None:
+            out = torch.empty(c.B, n, c.H, c.D, dtype=self.dtype, device=self.device)
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_cache_decode_n(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                              None if lse is None else lse.data_ptr(), n, stream))
         return out
 
     def nodes(self) -> torch.Tensor:

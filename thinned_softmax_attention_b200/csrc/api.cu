@@ -1812,7 +1812,7 @@ struct thin_attn_cache_s {
   bool use_split = false;
   std::vector<int> pos_keys;
   int max_splits = 0;
-  size_t part_off = 0;
+  size_t part_off = 0, arrive_off = 0;
 };
 
 namespace {
@@ -1990,6 +1990,8 @@ thin_attn_status cache_build(thin_attn_cache_s* cc) {
   off = align256(off + std::max<size_t>(cc->c2_floats, 1) * 4);
   cc->part_off = off;
   if (cc->use_split) off = align256(off + (size_t)cc->max_splits * BH * (cf.D + 2) * 4);
+  cc->arrive_off = off;
+  if (cc->use_split) off = align256(off + (size_t)BH * 4);
   cc->bytes = off;
   cudaError_t e = cudaMalloc(&cc->d_mem, cc->bytes);
   if (e != cudaSuccess) {
@@ -2010,6 +2012,7 @@ thin_attn_status cache_build(thin_attn_cache_s* cc) {
   CK(cudaMalloc(&cc->d_status, kStatusBytes));
   CK(cudaMemset(cc->d_status, 0, kStatusBytes));
   CK(cudaMemset((char*)cc->d_mem + cc->nodes.idx_off, 0xFF, (size_t)cc->nodes.rows * 4));
+  if (cc->use_split) CK(cudaMemset((char*)cc->d_mem + cc->arrive_off, 0, (size_t)BH * 4));
   return THIN_ATTN_OK;
 }
 
@@ -2111,26 +2114,26 @@ thin_attn_status thin_attn_cache_length(thin_attn_cache_t c, int64_t* t) {
   return THIN_ATTN_OK;
 }
 
-thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, const void* k, const void* v, void* out,
-                                        float* lse_opt, void* stream) {
-  if (!c) return fail(THIN_ATTN_EINVAL, "null cache");
-  if (!q || !k || !v || !out) return fail(THIN_ATTN_EINVAL, "q, k, v and out must be non-null");
-  for (const void* ptr : {q, k, v, (const void*)out})
-    if (((uintptr_t)ptr) % 16) return fail(THIN_ATTN_EINVAL, "tensor pointers must be 16-byte aligned");
+}  // extern "C"
+
+namespace {
+// One decoded token of every (b,h).  q, k, v, out point at the token's row of batch entry 0; entry b
+// is `bstride` token rows further on (1 for (B,1,H,.) tensors, n for (B,n,H,.) ones); lse, if given,
+// at the token's column of (b,h) 0, (b,h) i at lse + i * bstride.
+thin_attn_status cache_decode_one(thin_attn_cache_s* c, const void* q, const void* k, const void* v, void* out,
+                                  float* lse_opt, int64_t bstride, cudaStream_t st) {
   const thin_attn_config& cf = c->cf;
   if (c->t >= cf.T) return fail(THIN_ATTN_EINVAL, "the cache holds its capacity of %d tokens", cf.T);
-  DeviceGuard dg(cf.device);
-  cudaStream_t st = (cudaStream_t)stream;
   const int64_t pos = c->t;
   const size_t es = elt(cf);
   char* base = (char*)c->d_mem;
   // 1. the new key/value row: exact prefix row pos, or row ne + (pos - ne) mod b of the batch region
   const int64_t r = pos < c->ne ? pos : c->ne + (pos - c->ne) % c->bsz;
-  if (!c->use_split) {   // (the split-key kernels read the new row from k, v and append it themselves)
+  if (!c->use_split) {   // (the split-key kernel reads the new row from k, v and appends it itself)
     const size_t krow = (size_t)cf.H * cf.E * es, vrow = (size_t)cf.H * cf.D * es;
-    CK(cudaMemcpy2DAsync(base + c->raw.k_off + (size_t)r * krow, (size_t)c->L * krow, k, krow, krow, cf.B,
+    CK(cudaMemcpy2DAsync(base + c->raw.k_off + (size_t)r * krow, (size_t)c->L * krow, k, krow * bstride, krow, cf.B,
                          cudaMemcpyDeviceToDevice, st));
-    CK(cudaMemcpy2DAsync(base + c->raw.v_off + (size_t)r * vrow, (size_t)c->L * vrow, v, vrow, vrow, cf.B,
+    CK(cudaMemcpy2DAsync(base + c->raw.v_off + (size_t)r * vrow, (size_t)c->L * vrow, v, vrow * bstride, vrow, cf.B,
                          cudaMemcpyDeviceToDevice, st));
   }
   // 2. attention of query pos against the cache as it stands (its own token included)
@@ -2147,7 +2150,7 @@ thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, cons
   aa.tile0 = (int)pos;
   aa.n_tiles = 1;
   aa.B = cf.B;
-  aa.T = 1;
+  aa.T = (int)bstride;   // the query (and output) rows of batch entries b are bstride rows apart
   aa.L = c->L;
   aa.H = cf.H;
   aa.E = cf.E;
@@ -2163,8 +2166,16 @@ thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, cons
     ap.new_k = k;
     ap.new_v = v;
     ap.row = (int)r;
+    ap.arrive = (int*)(base + c->arrive_off);
+    const AttnTile& tl = c->tab.tiles[pos];
+    if (tl.nseg <= 32) {
+      ap.nseg = tl.nseg;
+      for (int s2 = 0; s2 < tl.nseg; ++s2) ap.segs[s2] = c->tab.segs[tl.seg0 + s2];
+    }
     e = launch_decode_attention(aa, cf.dtype, n_splits, (float*)(base + c->part_off), ap, st);
     done = true;
+  } else if (bstride != 1) {
+    return fail(THIN_ATTN_EUNSUPPORTED, "several tokens per call need the split-key decode (B*H <= 64)");
   }
   if (e == cudaSuccess && !done && c->use_tc) e = launch_attention_tc(aa, c->d_status, st, &done);
   if (e == cudaSuccess && !done) e = launch_attention_simt(aa, cf.dtype, st);
@@ -2188,6 +2199,43 @@ thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, cons
     }
   }
   c->t = pos + 1;
+  return THIN_ATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+thin_attn_status thin_attn_cache_decode(thin_attn_cache_t c, const void* q, const void* k, const void* v, void* out,
+                                        float* lse_opt, void* stream) {
+  if (!c) return fail(THIN_ATTN_EINVAL, "null cache");
+  if (!q || !k || !v || !out) return fail(THIN_ATTN_EINVAL, "q, k, v and out must be non-null");
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (((uintptr_t)ptr) % 16) return fail(THIN_ATTN_EINVAL, "tensor pointers must be 16-byte aligned");
+  DeviceGuard dg(c->cf.device);
+  return cache_decode_one(c, q, k, v, out, lse_opt, 1, (cudaStream_t)stream);
+}
+
+thin_attn_status thin_attn_cache_decode_n(thin_attn_cache_t c, const void* q, const void* k, const void* v, void* out,
+                                          float* lse_opt, int n, void* stream) {
+  if (!c) return fail(THIN_ATTN_EINVAL, "null cache");
+  if (n < 0) return fail(THIN_ATTN_EINVAL, "n = %d", n);
+  if (n == 0) return THIN_ATTN_OK;
+  if (!q || !k || !v || !out) return fail(THIN_ATTN_EINVAL, "q, k, v and out must be non-null");
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (((uintptr_t)ptr) % 16) return fail(THIN_ATTN_EINVAL, "tensor pointers must be 16-byte aligned");
+  const thin_attn_config& cf = c->cf;
+  if (c->t + n > cf.T) return fail(THIN_ATTN_EINVAL, "%d tokens would exceed the capacity of %d (holds %lld)", n, cf.T,
+                                   (long long)c->t);
+  if (n > 1 && !c->use_split)
+    return fail(THIN_ATTN_EUNSUPPORTED, "several tokens per call need the split-key decode (B*H <= 64)");
+  DeviceGuard dg(cf.device);
+  const size_t es = elt(cf), krow = (size_t)cf.H * cf.E * es, vrow = (size_t)cf.H * cf.D * es;
+  for (int i = 0; i < n; ++i) {
+    thin_attn_status s = cache_decode_one(c, (const char*)q + i * krow, (const char*)k + i * krow,
+                                          (const char*)v + i * vrow, (char*)out + i * vrow,
+                                          lse_opt ? lse_opt + i : nullptr, n, (cudaStream_t)stream);
+    if (s != THIN_ATTN_OK) return s;
+  }
   return THIN_ATTN_OK;
 }
 

@@ -7,9 +7,11 @@
 //            z = s q.k log2e + log2 w (w = the segment's weight) against q held in shared memory
 //   softmax  m = the chunk's max z, p = 2^(z - m), l = sum p (CTA-wide through shared memory)
 //   PV       lane-parallel over D: o += p_i v_i, the p_i broadcast from lane i
-// and writes the partial (m, l, o) of its chunk.  Combine kernel: CTA b*h merges the partials
-//   M = max m,  L = sum l 2^(m - M),  out = sum o 2^(m - M) / L,  lse = (M + log2 L) ln 2.
-// Base 2 throughout, fp32 accumulation, one pass over every key and value row.
+// and writes the partial (m, l, o) of its chunk.  The last CTA of a (b,h) to finish (an arrival
+// counter per (b,h)) merges the partials
+//   M = max m,  L = sum l 2^(m - M),  out = sum o 2^(m - M) / L,  lse = (M + log2 L) ln 2,
+// appends the decoded token's key and value to the cache and clears the counter: one launch per
+// token.  Base 2 throughout, fp32 accumulation, one pass over every key and value row.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -49,10 +51,13 @@ __device__ __forceinline__ void load_lane(const T* row, int lane, float (&x)[EPL
   }
 }
 
+template <typename T, int E, int D>
+__device__ __forceinline__ void decode_combine(const AttnArgs& a, const float* part, int n_splits,
+                                               const DecodeAppend& ap, int bh);
+
 template <typename T, int EPL, int DPL>
 __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(AttnArgs a, float* part, int n_splits,
                                                                        DecodeAppend ap) {
-  const AttnTile tile = a.tiles[a.tile0];
   const int split = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int E = EPL * 32, D = DPL * 32;
@@ -62,15 +67,25 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(AttnArgs a
   __shared__ float q_s[E];
   __shared__ float red_m[4], red_l[4];
   __shared__ float o_s[4][D];
+  const bool own = ap.nseg >= 0;   // segments passed in the launch
+  const AttnTile tile = own ? AttnTile{0, 1, 0, ap.nseg} : a.tiles[a.tile0];
   const int nseg = min(tile.nseg, 32);
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int s = 0; s < nseg; ++s) {
-      segs[s] = a.segs[tile.seg0 + s];
-      seg_start[s] = acc;
-      acc += segs[s].len;
+  if (warp == 0) {
+    // one segment per lane (all in flight at once), start offsets by a warp prefix sum
+    int len = 0;
+    if (lane < nseg) {
+      segs[lane] = own ? ap.segs[lane] : a.segs[tile.seg0 + lane];
+      len = segs[lane].len;
     }
-    seg_start[nseg] = acc;
+    int incl = len;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane < nseg) seg_start[lane] = incl - len;
+    if (lane == nseg - 1) seg_start[nseg] = incl;
+    if (nseg == 0 && lane == 0) seg_start[0] = 0;
   }
   const T* q = (const T*)a.q + ((int64_t)b * a.T * a.H + h) * E;   // the tile's single query row
   for (int e = threadIdx.x; e < E; e += kDecodeThreads) q_s[e] = to_f(q[e]) * a.scale_log2e;
@@ -98,8 +113,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(AttnArgs a
     if (ap.new_k && j == seg_start[nseg] - 1) {
       // the last key is the token being decoded: read it from the caller's rows (it is appended to
       // the cache by the combine launch, after every chunk has been read)
-      kr = (const T*)ap.new_k + ((int64_t)b * a.H + h) * E;
-      vr = (const T*)ap.new_v + ((int64_t)b * a.H + h) * D;
+      kr = (const T*)ap.new_k + ((int64_t)b * a.T * a.H + h) * E;
+      vr = (const T*)ap.new_v + ((int64_t)b * a.T * a.H + h) * D;
     }
   }
   // score of this lane's key: its whole row in flight, q (pre-scaled by s log2 e) broadcast
@@ -137,23 +152,25 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(AttnArgs a
 #pragma unroll
   for (int o = 16; o; o >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
   if (lane == 0) red_l[warp] = wl;
-  // o = sum p_i v_i over the warp's keys, lane-parallel over D, eight value rows in flight
+  // o = sum p_i v_i over the warp's keys, lane-parallel over D, sixteen value rows in flight (the
+  // decode of a token is a chain of dependent memory latencies: the fewer rounds the better)
+  constexpr int RV = 16;
   float ov[DPL];
 #pragma unroll
   for (int d = 0; d < DPL; ++d) ov[d] = 0.f;
   const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));   // the valid keys are the first ones
 #pragma unroll 1
-  for (int i0 = 0; i0 < nvalid; i0 += 8) {
-    float vv[8][DPL], pp[8];
+  for (int i0 = 0; i0 < nvalid; i0 += RV) {
+    float vv[RV][DPL], pp[RV];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < RV; ++u) {
       const T* r = (const T*)__shfl_sync(0xffffffffu, (unsigned long long)vr, (i0 + u) & 31);
       pp[u] = __shfl_sync(0xffffffffu, p_mine, (i0 + u) & 31);
       if (i0 + u < nvalid) load_lane<T, DPL>(r, lane, vv[u]);
       else pp[u] = 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < RV; ++u)
       if (i0 + u < nvalid) {
 #pragma unroll
         for (int d = 0; d < DPL; ++d) ov[d] = fmaf(pp[u], vv[u][d], ov[d]);
@@ -168,43 +185,54 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(AttnArgs a
     out[D] = m;
     out[D + 1] = red_l[0] + red_l[1] + red_l[2] + red_l[3];
   }
+  // the last chunk of this (b,h) to finish merges them all
+  __shared__ int last_s;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last_s = atomicAdd(ap.arrive + bh, 1) == n_splits - 1;
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  decode_combine<T, E, D>(a, part, n_splits, ap, bh);
+  if (threadIdx.x == 0) ap.arrive[bh] = 0;   // ready for the next token (a later launch)
 }
 
+// Merge of the chunks' partials of (b,h) `bh` by one CTA (partials written by other CTAs of this
+// launch: read through L2), append of the decoded token.
 template <typename T, int E, int D>
-__global__ void __launch_bounds__(128) decode_combine_kernel(AttnArgs a, const float* part, int n_splits,
-                                                             DecodeAppend ap) {
-  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+__device__ __forceinline__ void decode_combine(const AttnArgs& a, const float* part, int n_splits,
+                                               const DecodeAppend& ap, int bh) {
+  const int b = bh / a.H, h = bh % a.H;
   if (ap.new_k) {
     // append the decoded token's key and value to the cache row of this position
-    const int64_t src = (int64_t)b * a.H + h, dst = ((int64_t)b * a.L + ap.row) * a.H + h;
+    const int64_t src = (int64_t)b * a.T * a.H + h, dst = ((int64_t)b * a.L + ap.row) * a.H + h;
     for (int e = threadIdx.x; e < E; e += blockDim.x) ((T*)a.k)[dst * E + e] = ((const T*)ap.new_k)[src * E + e];
     for (int d = threadIdx.x; d < D; d += blockDim.x) ((T*)a.v)[dst * D + d] = ((const T*)ap.new_v)[src * D + d];
   }
   const float* p = part + (size_t)bh * n_splits * (D + 2);
   float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, p[s * (D + 2) + D]);
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, __ldcg(p + s * (D + 2) + D));
   float L = 0.f;
   for (int s = 0; s < n_splits; ++s) {
-    const float ms = p[s * (D + 2) + D];
-    if (ms != -INFINITY) L += p[s * (D + 2) + D + 1] * exp2f(ms - M);
+    const float ms = __ldcg(p + s * (D + 2) + D);
+    if (ms != -INFINITY) L += __ldcg(p + s * (D + 2) + D + 1) * exp2f(ms - M);
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   T* out = (T*)a.out + ((int64_t)b * a.T * a.H + h) * D;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float o = 0.f;
     for (int s = 0; s < n_splits; ++s) {
-      const float ms = p[s * (D + 2) + D];
-      if (ms != -INFINITY) o += p[s * (D + 2) + d] * exp2f(ms - M);
+      const float ms = __ldcg(p + s * (D + 2) + D);
+      if (ms != -INFINITY) o += __ldcg(p + s * (D + 2) + d) * exp2f(ms - M);
     }
     out[d] = from_f<T>(o * inv);
   }
-  if (threadIdx.x == 0 && a.lse) a.lse[bh] = (M + log2f(L)) * 0.6931471805599453f;
+  if (threadIdx.x == 0 && a.lse) a.lse[(int64_t)bh * a.T] = (M + log2f(L)) * 0.6931471805599453f;
 }
 
 template <typename T, int EPL, int DPL>
 cudaError_t launch_t(const AttnArgs& a, int n_splits, float* part, const DecodeAppend& ap, cudaStream_t st) {
   decode_split_kernel<T, EPL, DPL><<<dim3(n_splits, a.B * a.H), kDecodeThreads, 0, st>>>(a, part, n_splits, ap);
-  decode_combine_kernel<T, EPL * 32, DPL * 32><<<a.B * a.H, 128, 0, st>>>(a, part, n_splits, ap);
   return cudaGetLastError();
 }
 

@@ -53,14 +53,20 @@ int attention_tc_tile_rows();
 bool attention_tc_supported(int dtype, int E, int D);
 
 // Split-key attention of one query per (b,h) (decode): n_splits chunks of decode_chunk_keys() keys
-// of the tile a.tile0, partials (m, l, o) in `part` (n_splits x B*H x (D + 2) floats), then a combine
-// launch writing out and lse.
+// of the tile a.tile0, partials (m, l, o) in `part` (n_splits x B*H x (D + 2) floats), merged into
+// out and lse by the last chunk of each (b,h) to finish (one launch).
 // With new_k set, the last key of the tile is the token being decoded: it is read from new_k / new_v
-// ((B,1,H,E), (B,1,H,D)) and then written to row `row` of every (b,h) of a.k / a.v.
+// (batch entry b a.T token rows after entry 0, like q and out; lse of (b,h) i at a.lse[i a.T]) and
+// then written to row `row` of every (b,h) of a.k / a.v.
 struct DecodeAppend {
   const void* new_k = nullptr;
   const void* new_v = nullptr;
   int row = 0;
+  int* arrive = nullptr;   // B*H arrival counters of the chunks, zero between launches (required)
+  // the tile's segments, copied from the host's tables into the launch (saves two dependent loads at
+  // the head of a token's latency chain); nseg = -1: read a.tiles / a.segs instead
+  int nseg = -1;
+  AttnSeg segs[32];
 };
 bool decode_attention_supported(int E, int D, int max_segments);
 int decode_chunk_keys();
