@@ -713,6 +713,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
                                                            int* status) {
   using Lay = Tc2Layout<E, D, FP8>;
   constexpr uint32_t O_COL = 128;
+  // S/P and O: 256 TMEM columns for D <= 128 (two CTAs per SM), 512 for D = 256 (one CTA per SM)
+  constexpr uint32_t TCOLS = D <= 128 ? 256 : 512;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
@@ -760,7 +762,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
     mbar_init(item_full + 1, 1);
     fence_barrier_init();
   }
-  if (warp == 5) tmem_alloc(&tmem_base_s, 256);
+  if (warp == 5) tmem_alloc(&tmem_base_s, TCOLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -957,29 +959,57 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
       __nv_bfloat16* out = (__nv_bfloat16*)a.out;
       const bool live = row < tile.qlen;
       __nv_bfloat16* orow = out + ((int64_t)(b * a.T + tq) * a.H + h) * D;
-      // the row of O, normalised and packed to bf16 pairs in registers (64 columns per TMEM wait),
-      // then O is released to the next item's first PV before the stores go out
-      uint32_t pk[D / 2];
+      if constexpr (D <= 128) {
+        // the row of O, normalised and packed to bf16 pairs in registers (64 columns per TMEM wait),
+        // then O is released to the next item's first PV before the stores go out
+        uint32_t pk[D / 2];
 #pragma unroll
-      for (int c2 = 0; c2 < D / 64; ++c2) {
-        float o[2][32];
-        tmem_ld32(tmem + lane_base + O_COL + c2 * 64, o[0]);
-        tmem_ld32(tmem + lane_base + O_COL + c2 * 64 + 32, o[1]);
-        tmem_ld_wait();
+        for (int c2 = 0; c2 < D / 64; ++c2) {
+          float o[2][32];
+          tmem_ld32(tmem + lane_base + O_COL + c2 * 64, o[0]);
+          tmem_ld32(tmem + lane_base + O_COL + c2 * 64 + 32, o[1]);
+          tmem_ld_wait();
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
+          for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const __nv_bfloat162 t = __floats2bfloat162_rn(o[hh][i] * inv, o[hh][i + 1] * inv);
-            pk[(c2 * 64 + hh * 32 + i) / 2] = *reinterpret_cast<const uint32_t*>(&t);
+            for (int i = 0; i < 32; i += 2) {
+              const __nv_bfloat162 t = __floats2bfloat162_rn(o[hh][i] * inv, o[hh][i + 1] * inv);
+              pk[(c2 * 64 + hh * 32 + i) / 2] = *reinterpret_cast<const uint32_t*>(&t);
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(o_empty);
+        if (live) {
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i)
+            *reinterpret_cast<uint4*>(orow + 8 * i) = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      } else {
+        // D = 256: a packed row would not fit in registers; every 64 columns go out as they are
+        // packed, and O is released after the last of them
+#pragma unroll 1
+        for (int c2 = 0; c2 < D / 64; ++c2) {
+          float o[2][32];
+          tmem_ld32(tmem + lane_base + O_COL + c2 * 64, o[0]);
+          tmem_ld32(tmem + lane_base + O_COL + c2 * 64 + 32, o[1]);
+          tmem_ld_wait();
+          uint32_t pk[32];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const __nv_bfloat162 t = __floats2bfloat162_rn(o[hh][i] * inv, o[hh][i + 1] * inv);
+              pk[(hh * 32 + i) / 2] = *reinterpret_cast<const uint32_t*>(&t);
+            }
+          if (live) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              *reinterpret_cast<uint4*>(orow + c2 * 64 + 8 * i) =
+                  make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
-      }
-      tc_fence_before();
-      mbar_arrive(o_empty);
-      if (live) {
-#pragma unroll
-        for (int i = 0; i < D / 8; ++i)
-          *reinterpret_cast<uint4*>(orow + 8 * i) = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+        tc_fence_before();
+        mbar_arrive(o_empty);
       }
       if (live && a.lse) a.lse[(int64_t)bh * a.T + tq] = (m_used + log2f(l)) * 0.6931471805599453f;
     }
@@ -1003,7 +1033,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
   }
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, TCOLS);
   }
 }
 
@@ -1603,6 +1633,21 @@ cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
         kern<<<grid, 384, sm, st>>>(maps, a, status);
         return cudaGetLastError();
       }
+    }
+  }
+  if constexpr (D == 256 && E == 64) {
+    // D = 256 (BigGAN): the persistent kernel, one CTA per SM (S and O take 384 TMEM columns)
+    if (std::getenv("THIN_ATTN_TC1") == nullptr && status != nullptr) {
+      int dev = 0, sms = 0;
+      cudaError_t e = cudaGetDevice(&dev);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      // more shared memory than half an SM's, so that no second CTA lands on an SM and waits for TMEM
+      const size_t sm = std::max<size_t>(Tc2Layout<E, D>::BYTES, 120 * 1024);
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_tc2p_kernel<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if (e != cudaSuccess) return e;
+      const int64_t items = (int64_t)a.n_tiles * a.B * a.H;
+      attn_tc2p_kernel<E, D><<<(int)std::min<int64_t>(items, sms), 192, sm, st>>>(maps, a, status);
+      return cudaGetLastError();
     }
   }
   if constexpr (D <= 128) {
