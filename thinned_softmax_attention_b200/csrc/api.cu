@@ -365,6 +365,14 @@ void build_attn_tables(const thin_attn_config& cf, const Plan& p, int QT, AttnTa
   }
 }
 
+// Each tile's count of 128-key tiles (AttnTile::nkt), which the attention kernels read.
+void set_key_tile_counts(AttnTables& t) {
+  for (AttnTile& tl : t.tiles) {
+    tl.nkt = 0;
+    for (int s = 0; s < tl.nseg; ++s) tl.nkt += (t.segs[tl.seg0 + s].len + 127) / 128;
+  }
+}
+
 // Whether tile A's key tiles are the first key tiles of tile B's: the same segments, except that
 // A's last one may stop earlier in B's segment of the same place (the causal in-batch keys of two
 // neighbouring query tiles).  Such a pair shares one stream of K/V tiles.
@@ -931,6 +939,7 @@ thin_attn_status materialise(thin_attn_s* h, Plan* p) {
     tbl_end = std::max(tbl_end, p->sched_done_off + p->sched_items.size() * sizeof(int));
   }
   for (AttnTables* t : {&p->simt, &p->tc}) {
+    set_key_tile_counts(*t);
     if (!t->tiles.empty()) std::memcpy(host.data() + t->tiles_off, t->tiles.data(), t->tiles.size() * sizeof(AttnTile));
     if (!t->segs.empty()) std::memcpy(host.data() + t->segs_off, t->segs.data(), t->segs.size() * sizeof(AttnSeg));
     if (!t->pairs.empty()) std::memcpy(host.data() + t->pairs_off, t->pairs.data(), t->pairs.size() * sizeof(int2));
@@ -2006,6 +2015,7 @@ thin_attn_status cache_build(thin_attn_cache_s* cc) {
     for (auto& st : steps) put(st.sp.inst, st.sp.inst_off);
   for (auto& kv : cc->merges)
     for (auto& st : kv.second) put(st.sp.inst, st.sp.inst_off);
+  set_key_tile_counts(t);
   std::memcpy(host.data() + t.tiles_off, t.tiles.data(), t.tiles.size() * sizeof(AttnTile));
   std::memcpy(host.data() + t.segs_off, t.segs.data(), t.segs.size() * sizeof(AttnSeg));
   CK(cudaMemcpy(cc->d_mem, host.data(), table_end, cudaMemcpyHostToDevice));

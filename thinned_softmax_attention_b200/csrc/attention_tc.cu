@@ -51,11 +51,9 @@ struct TcMaps {
   CUtensorMap q, k, v, ck, cv;
 };
 
-__device__ __forceinline__ int count_key_tiles(const AttnArgs& a, const AttnTile& t) {
-  int n = 0;
-  for (int s = 0; s < t.nseg; ++s) n += (a.segs[t.seg0 + s].len + BN - 1) / BN;
-  return n;
-}
+// 128-key tiles of a query tile (counted by the host, so that a kernel learns an item's length from
+// the tile record alone instead of walking its segments in global memory)
+__device__ __forceinline__ int count_key_tiles(const AttnArgs&, const AttnTile& t) { return t.nkt; }
 
 template <int E, int D>
 __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a,
@@ -917,10 +915,12 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
       const int tile_id = a.tile0 + a.n_tiles - 1 - j % a.n_tiles;
       const AttnTile tile = a.tiles[tile_id];
       const int bh = j / a.n_tiles, b = bh / a.H, h = bh % a.H;
-      if (count_key_tiles(a, tile) == 0) {
+      if (tile.nkt == 0) {
         mbar_arrive(o_empty);
         continue;
       }
+      // the tile's segment records into L1: the loads at the segment boundaries below then hit there
+      if (lane == 0) prefetch_l1(a.segs + tile.seg0, tile.nseg * (int)sizeof(AttnSeg));
       if (threadIdx.x == 0) item_s = tile_id * 65536 + bh;
       const int tq = tile.q0 + row;
       // e4m3 scores are q k^T times scale_q scale_k: the (b,h) factor that undoes it joins s log2 e
@@ -1042,41 +1042,48 @@ __global__ void __launch_bounds__(192, 2) attn_tc2p_kernel(const __grid_constant
 // time, tile A and tile B, against a single stream of K/V tiles.  The host pairs tiles whose key
 // lists nest: A's key tiles are the first n_A key tiles of B's (two neighbouring tiles of one
 // Express batch, the exact phase, or any two tiles of a Thinformer head), so every K/V tile is
-// loaded once for both; the K and V rings fill the shared memory beside the two Q tiles.
+// loaded once for both; the K and V rings fill the shared memory beside the Q buffers.
 //   TMEM (512 columns): S_A / P_A 0..127, S_B / P_B 128..255, O_A 256..383, O_B 384..511.
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B (thread = query row = TMEM lane)
-//   warp 8     TMA producer: work items, Q_A and Q_B per item, K per key tile into the K ring
-//   warp 10    TMA producer: V per key tile into the V ring; warp 11 idle
-// After set-up the softmax warpgroups take 208 registers per thread and warps 8-11 give theirs down
-// to 88, so a softmax thread holds its row of S and reads it from TMEM once per key tile.
+//   warp 8     TMA producer: work items (published one item ahead), K per key tile into the K ring
+//   warp 10    TMA producer: V per key tile into the V ring
+//   warp 11    TMA producer: Q_A and Q_B of every item into a ring of NQ Q buffers (item r takes
+//              fills 2r and 2r + 1), each refilled once the last S MMA reading it has completed, so
+//              that the next item's Q_A loads while the current item's B tile still runs
+// After set-up the softmax warpgroups take 192 registers per thread and warps 8-11 keep 120, so a
+// softmax thread holds its row of S and reads it from TMEM once per key tile.
 //   warp 9     MMA issuer: per key tile j, PV_A(j), S_A(j+1), PV_B(j), S_B(j+1) -- while one
-//              softmax warpgroup turns its S into P, the tensor pipe runs the other tile's PV and S
+//              softmax warpgroup turns its S into P, the tensor pipe runs the other tile's PV and S.
+//              A's key list ends no later than B's, so in an item's last step the A slot is free:
+//              the next item's S_A(0) is issued there, ahead of the last PV_B, and the A softmax
+//              starts the next item while B finishes this one.
 // The per-row arithmetic is softmax_tile's, as in the two-CTA kernels, so outputs equal theirs bit
 // for bit.
 // Items (tile pair, (b,h)) come from the work counter in the handle's status buffer, heaviest
 // pairs first, through a two-slot ring whose slots are released by every reader (item_empty).
-template <int E, int D>
+template <int E, int D, int NQ>
 struct PpLayout {
   static constexpr int EC = E / 64, DC = D / 64;
   static constexpr uint32_t Q_BYTES = BM * E * 2;
   static constexpr uint32_t K_BYTES = BN * E * 2;
   static constexpr uint32_t V_BYTES = BN * D * 2;
-  // K and V rings as deep as the shared memory beside the two Q tiles allows (227 KB per CTA, less
+  // K and V rings as deep as the shared memory beside the Q buffers allows (227 KB per CTA, less
   // barriers and alignment slack), at most 4 stages each: E = D = 128 gives 3 K and 2 V stages
-  static constexpr uint32_t AVAIL = 232448 - 2048 - 2 * Q_BYTES;
+  // beside two Q buffers, 2 and 2 beside three
+  static constexpr uint32_t AVAIL = 232448 - 2048 - NQ * Q_BYTES;
   static constexpr int NK = (AVAIL - 2 * V_BYTES) / K_BYTES < 4 ? (int)((AVAIL - 2 * V_BYTES) / K_BYTES) : 4;
   static constexpr int NV = (AVAIL - NK * K_BYTES) / V_BYTES < 4 ? (int)((AVAIL - NK * K_BYTES) / V_BYTES) : 4;
-  static_assert(NK >= 2 && NV >= 2, "two stages of K and V at least");
-  static constexpr uint32_t OFF_QB = Q_BYTES;
-  static constexpr uint32_t OFF_K = 2 * Q_BYTES;
+  static_assert(NQ >= 2 && NK >= 2 && NV >= 2, "two Q buffers and two stages of K and V at least");
+  static constexpr uint32_t OFF_K = NQ * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + NK * K_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + NV * V_BYTES;
-  static constexpr uint32_t BYTES = OFF_BAR + 256 + 1024;
+  static constexpr int N_BARS = 2 * NQ + 2 * NK + 2 * NV + 14;
+  static constexpr uint32_t BYTES = OFF_BAR + ((N_BARS * 8 + 127) / 128) * 128 + 1024;
   static_assert(BYTES <= 232448, "shared memory per CTA");
 };
 
 // softmax_tile with the thread's whole row of S in registers (one TMEM read per tile; the
-// ping-pong kernel's softmax threads hold 208 registers): the same arithmetic in the same order,
+// ping-pong kernel's softmax threads hold 192 registers): the same arithmetic in the same order,
 // so the same P, row sum and rescale decisions.
 template <bool MASKED, int D>
 __device__ __forceinline__ void softmax_tile_reg(uint32_t ts, uint32_t to, int lim, float sl2e, float lw2, int it,
@@ -1145,24 +1152,23 @@ __device__ __forceinline__ void softmax_tile_reg(uint32_t ts, uint32_t to, int l
 // Registers per thread of the ping-pong kernel after its reallocation: the two softmax warpgroups
 // take kPpSoftmaxRegs, the producer / MMA warpgroup keeps kPpOtherRegs; the sum fits the launch's
 // 384 x kPpLaunchRegs (checked on the host before every launch).
-constexpr int kPpLaunchRegs = 168, kPpSoftmaxRegs = 208, kPpOtherRegs = 88;
+constexpr int kPpLaunchRegs = 168, kPpSoftmaxRegs = 192, kPpOtherRegs = 120;
 static_assert(256 * kPpSoftmaxRegs + 128 * kPpOtherRegs <= 384 * kPpLaunchRegs, "register split");
 
-template <int E, int D>
+template <int E, int D, int NQ>
 __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a,
                                                          int* status) {
-  using Lay = PpLayout<E, D>;
+  using Lay = PpLayout<E, D, NQ>;
   constexpr int NK = Lay::NK, NV = Lay::NV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQA = smem;
-  uint8_t* sQB = smem + Lay::OFF_QB;
+  uint8_t* sQ = smem;
   uint8_t* sK = smem + Lay::OFF_K;
   uint8_t* sV = smem + Lay::OFF_V;
   uint64_t* bars = (uint64_t*)(smem + Lay::OFF_BAR);
-  uint64_t* q_full = bars + 0;       // Q_A (if used) and Q_B of the item landed
-  uint64_t* q_empty = bars + 1;      // the item's last S MMA has read Q (commit)
-  uint64_t* k_full = bars + 2;            // [NK]
+  uint64_t* q_full = bars;                // [NQ] the Q buffer's fill landed (or, for an absent A tile, was skipped)
+  uint64_t* q_empty = q_full + NQ;        // [NQ] the last S MMA reading the buffer has completed (commit)
+  uint64_t* k_full = q_empty + NQ;        // [NK]
   uint64_t* k_empty = k_full + NK;        // [NK] S_A and S_B of the tile have read K (commit)
   uint64_t* v_full = k_empty + NK;        // [NV]
   uint64_t* v_empty = v_full + NV;        // [NV] PV_A and PV_B of the tile have read V (commit)
@@ -1172,8 +1178,8 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
   uint64_t* pv_done = p_full + 2;         // [2] the item's last PV_x done (commit)
   uint64_t* o_empty = pv_done + 2;        // [2] O_x read out of TMEM (128 threads)
   uint64_t* item_full = o_empty + 2;      // [2] ring slot written (K producer)
-  uint64_t* item_empty = item_full + 2;   // [2] ring slot read by the V producer, the MMA thread and
-                                          //     all 256 softmax threads
+  uint64_t* item_empty = item_full + 2;   // [2] ring slot read by the V and Q producers, the MMA thread
+                                          //     and all 256 softmax threads
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
   __shared__ volatile int where_s;
@@ -1188,8 +1194,10 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
     abort_s = 0;
     where_s = 0;
     item_s = -1;
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(q_full + s, 1);
+      mbar_init(q_empty + s, 1);
+    }
     for (int s = 0; s < NK; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
@@ -1205,7 +1213,7 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
       mbar_init(pv_done + x, 1);
       mbar_init(o_empty + x, 128);
       mbar_init(item_full + x, 1);
-      mbar_init(item_empty + x, 258);
+      mbar_init(item_empty + x, 259);
     }
     fence_barrier_init();
   }
@@ -1222,21 +1230,16 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
   if (warp >= 8) {
   regs_dec<kPpOtherRegs>();   // the whole warpgroup 8-11
   if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer: work items, Q and K
+    // ------------------------------------------------------------ TMA producer: work items and K
     if (lane == 0) {
       int g = 0, r = 0;
       bool ok = true;
-      // the CTA's next item is taken one item ahead, and its Q tiles and first key tile are
-      // prefetched into L2 while the current item runs: Q rows are read once, from HBM, and
-      // their load would otherwise stall the tensor pipe at every item boundary
+      // item r + 1 is taken and published when item r's K loads start, so that the Q producer loads
+      // its Q tiles a whole item ahead; its first key tile is prefetched into L2 meanwhile
       auto prefetch = [&](int jn) {
         const int2 pn = pair_of(jn);
         const int bhn = jn / a.n_pairs, bn = bhn / a.H, hn = bhn % a.H;
         const AttnTile tn = a.tiles[pn.y];
-        for (int c = 0; c < Lay::EC; ++c) {
-          tma_prefetch_3d(&maps.q, c * 64, hn, bn * a.T + tn.q0);
-          if (pn.x >= 0) tma_prefetch_3d(&maps.q, c * 64, hn, bn * a.T + a.tiles[pn.x].q0);
-        }
         if (tn.nseg > 0) {
           const AttnSeg sg = a.segs[tn.seg0];
           if (sg.kind == SEG_TOKENS) {
@@ -1249,35 +1252,28 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
           }
         }
       };
-      int j_next = atomicAdd(sched, 1);
-      for (;; ++r) {
-        const int slot = r & 1;
-        if (r >= 2 && !mbar_wait(item_empty + slot, ((r >> 1) - 1) & 1, abort)) {
-          atomicCAS((int*)&where_s, 0, 11000 + min(r, 999));
-          ok = false;
+      // ring slot rr & 1 holds item rr; it is rewritten once all readers have taken item rr - 2
+      auto publish = [&](int rr, int jv) -> bool {
+        if (rr >= 2 && !mbar_wait(item_empty + (rr & 1), ((rr >> 1) - 1) & 1, abort)) {
+          atomicCAS((int*)&where_s, 0, 11000 + min(rr, 999));
+          return false;
         }
-        if (ok && r > 0 && !mbar_wait(q_empty, (r - 1) & 1, abort)) {
-          atomicCAS((int*)&where_s, 0, 9000 + min(r, 999));
+        item_ring[rr & 1] = jv < n_items ? jv : -1;
+        mbar_arrive(item_full + (rr & 1));
+        return true;
+      };
+      int j = atomicAdd(sched, 1);
+      ok = publish(0, j);
+      for (; ok && j < n_items; ++r) {
+        const int j_next = atomicAdd(sched, 1);
+        if (!publish(r + 1, j_next)) {
           ok = false;
+          break;
         }
-        const int j = ok ? j_next : n_items;
-        item_ring[slot] = j < n_items ? j : -1;
-        mbar_arrive(item_full + slot);
-        if (j >= n_items) break;
-        j_next = atomicAdd(sched, 1);
         if (j_next < n_items) prefetch(j_next);
         const int2 pr = pair_of(j);
         const int bh = j / a.n_pairs, b = bh / a.H, h = bh % a.H;
         const AttnTile tB = a.tiles[pr.y];
-        const bool useA = tiles_of(pr.x) > 0;
-        mbar_expect_tx(q_full, (useA ? 2u : 1u) * Lay::Q_BYTES);
-        if (useA) {
-          const int q0 = a.tiles[pr.x].q0;
-#pragma unroll
-          for (int c = 0; c < Lay::EC; ++c) tma_load_3d(sQA + c * 16384, &maps.q, q_full, c * 64, h, b * a.T + q0);
-        }
-#pragma unroll
-        for (int c = 0; c < Lay::EC; ++c) tma_load_3d(sQB + c * 16384, &maps.q, q_full, c * 64, h, b * a.T + tB.q0);
         for (int si = 0; si < tB.nseg && ok; ++si) {
           const AttnSeg sg = a.segs[tB.seg0 + si];
           const bool tok = sg.kind == SEG_TOKENS;
@@ -1298,10 +1294,10 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
             }
           }
         }
-        if (!ok) break;   // abort is set: every other role's next wait returns at once
+        j = j_next;
       }
       // never leave with a copy in flight into this CTA's shared memory: wait (bounded) for the
-      // last fill of every K stage and for the last Q load
+      // last fill of every K stage
       for (int st = 0; st < NK; ++st) {
         const int last = g - 1 - ((g - 1 - st) % NK + NK) % NK;   // largest g' < g with g' % NK == st
         if (last < 0) continue;
@@ -1309,9 +1305,45 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
         while (!mbar_try_wait(k_full + st, (last / NK) & 1) && clock64() - t0 < kWaitCycles) {
         }
       }
-      if (r > 0) {
+    }
+  } else if (warp == 11) {
+    // ------------------------------------------------------------ TMA producer: Q
+    if (lane == 0) {
+      int nq = 0;   // fills issued
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int slot = r & 1;
+        if (!mbar_wait(item_full + slot, (r >> 1) & 1, abort)) break;
+        const int j = item_ring[slot];
+        mbar_arrive(item_empty + slot);
+        if (j < 0) break;
+        const int2 pr = pair_of(j);
+        const int bh = j / a.n_pairs, b = bh / a.H, h = bh % a.H;
+        for (int x = 0; x < 2; ++x) {
+          const int n = 2 * r + x, buf = n % NQ;
+          if (n >= NQ && !mbar_wait(q_empty + buf, ((n / NQ) - 1) & 1, abort)) {
+            atomicCAS((int*)&where_s, 0, 9000 + min(n, 999));
+            ok = false;
+            break;
+          }
+          ++nq;
+          const int t = x ? pr.y : pr.x;
+          if (x == 0 && tiles_of(t) == 0) {
+            mbar_arrive(q_full + buf);   // no A tile: the fill is empty
+            continue;
+          }
+          mbar_expect_tx(q_full + buf, Lay::Q_BYTES);
+          const int q0 = a.tiles[t].q0;
+#pragma unroll
+          for (int c = 0; c < Lay::EC; ++c)
+            tma_load_3d(sQ + buf * Lay::Q_BYTES + c * 16384, &maps.q, q_full + buf, c * 64, h, b * a.T + q0);
+        }
+      }
+      for (int buf = 0; buf < NQ; ++buf) {
+        const int last = nq - 1 - ((nq - 1 - buf) % NQ + NQ) % NQ;
+        if (last < 0) continue;
         const long long t0 = clock64();
-        while (!mbar_try_wait(q_full, (r - 1) & 1) && clock64() - t0 < kWaitCycles) {
+        while (!mbar_try_wait(q_full + buf, (last / NQ) & 1) && clock64() - t0 < kWaitCycles) {
         }
       }
     }
@@ -1363,16 +1395,16 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
     if (lane == 0) {
       constexpr uint32_t IQK = idesc_bf16(BM, BN, false);
       constexpr uint32_t IPV = idesc_bf16(BM, D, true);
-      const uint32_t qa = smem_u32(sQA), qb = smem_u32(sQB), ka = smem_u32(sK), va = smem_u32(sV);
+      const uint32_t q0 = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
       int g = 0, gx[2] = {0, 0}, ix[2] = {0, 0};
       bool ok = true;
       auto fail = [&](int code, int at) {
         ok = false;
         atomicCAS((int*)&where_s, 0, code + min(at, 999));
       };
-      // S_x = Q_x K^T of ring position gg into TMEM columns 128 x
-      auto issue_s = [&](int x, int gg) {
-        const uint32_t q = x ? qb : qa;
+      // S_x = Q (fill n) K^T of ring position gg into TMEM columns 128 x
+      auto issue_s = [&](int x, int gg, int n) {
+        const uint32_t q = q0 + (n % NQ) * Lay::Q_BYTES;
         const uint32_t kb = ka + (gg % NK) * Lay::K_BYTES;
 #pragma unroll
         for (int k = 0; k < E / 16; ++k) {
@@ -1380,6 +1412,16 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
           umma_bf16(tmem + 128 * x, sw128_desc(q + off, 16, 1024), sw128_desc(kb + off, 16, 1024), IQK, k > 0);
         }
         umma_commit(s_full + x);
+      };
+      // the Q buffer of fill n is free again once every MMA issued so far has completed
+      auto q_release = [&](int n) { umma_commit(q_empty + n % NQ); };
+      auto q_wait = [&](int n) -> bool {
+        if (!mbar_wait(q_full + n % NQ, (n / NQ) & 1, abort)) {
+          fail(4000, n);
+          return false;
+        }
+        tc_fence_after();
+        return true;
       };
       // O_x += P_x V of ring position gg, in two halves over the keys (the first once P of keys 0..63
       // is written); the first of an item waits for the previous item's O_x to be read out
@@ -1416,27 +1458,52 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
         tc_fence_after();
         return true;
       };
-      for (int r = 0; ok; ++r) {
-        const int slot = r & 1;
-        if (!mbar_wait(item_full + slot, (r >> 1) & 1, abort)) break;
-        const int j = item_ring[slot];
-        mbar_arrive(item_empty + slot);
-        if (j < 0) break;
-        const int2 pr = pair_of(j);
-        const int n_a = tiles_of(pr.x), n_b = tiles_of(pr.y);
-        if (!mbar_wait(q_full, r & 1, abort)) {
-          fail(4000, r);
-          break;
+      auto fetch = [&](int rr) -> int {
+        if (!mbar_wait(item_full + (rr & 1), (rr >> 1) & 1, abort)) {
+          fail(12000, rr);
+          return -1;
         }
+        const int jv = item_ring[rr & 1];
+        mbar_arrive(item_empty + (rr & 1));
+        return jv;
+      };
+      // an item's key-tile counts, read from its tile records
+      auto lengths = [&](int jv, int& na, int& nb) {
+        na = nb = 0;
+        if (jv >= 0) {
+          const int2 pv = pair_of(jv);
+          na = tiles_of(pv.x);
+          nb = tiles_of(pv.y);
+        }
+      };
+      int j = fetch(0), n_a = 0, n_b = 0;
+      lengths(j, n_a, n_b);
+      bool pre = false;   // S_A(0) of item r was issued in item r - 1's last step
+      for (int r = 0; ok && j >= 0; ++r) {
+        const int fa = 2 * r, fb = 2 * r + 1;   // the item's Q fills
+        if ((!pre && !q_wait(fa)) || !q_wait(fb)) break;
         if (n_b == 0) {
-          umma_commit(q_empty);
+          q_release(fa);
+          q_release(fb);
+          j = fetch(r + 1);
+          lengths(j, n_a, n_b);
           continue;
         }
-        if (!wait_k(g)) break;
-        if (n_a > 0) issue_s(0, g);
-        issue_s(1, g);
+        if (!pre) {
+          if (!wait_k(g)) break;
+          if (n_a > 0) issue_s(0, g, fa);
+          if (n_a <= 1) q_release(fa);
+        }
+        issue_s(1, g, fb);
         umma_commit(k_empty + g % NK);
-        if (n_b == 1) umma_commit(q_empty);
+        if (n_b == 1) q_release(fb);
+        // the next item is taken now (it is published an item ahead), so that reading its tile
+        // records overlaps this item instead of stalling the tensor pipe at the boundary
+        const int jn = fetch(r + 1);
+        if (!ok) break;
+        int n_a_next = 0, n_b_next = 0;
+        lengths(jn, n_a_next, n_b_next);
+        bool pre_next = false;
         for (int jj = 0; jj < n_b && ok; ++jj) {
           const int gg = g + jj;
           // S_x(jj + 1) overwrites the columns PV_x(jj) reads P_x from: tcgen05.mma ops issued by one
@@ -1449,7 +1516,29 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
             }
             if (jj + 1 < n_a) {
               if (!wait_k(gg + 1)) break;
-              issue_s(0, gg + 1);
+              issue_s(0, gg + 1, fa);
+              if (jj + 1 == n_a - 1) q_release(fa);
+            }
+          }
+          if (jj == n_b - 1) {
+            // the A slot is done with this item: the next item's S_A(0) goes ahead of the last PV_B
+            // if its Q fill and first key tile land before B's last P is half written (neither
+            // depends on anything issued from here on); otherwise it waits for the next item's start
+            if (jn >= 0) {
+              const int fn = fa + 2, kn = g + n_b;
+              const long long t0 = clock64();
+              while (n_a_next > 0) {
+                if (mbar_test(q_full + fn % NQ, (fn / NQ) & 1) && mbar_test(k_full + kn % NK, (kn / NK) & 1)) {
+                  pre_next = true;
+                  break;
+                }
+                if (mbar_test(p_half + 1, gx[1] & 1) || *abort || clock64() - t0 > kWaitCycles) break;
+              }
+              if (pre_next) {
+                tc_fence_after();
+                issue_s(0, kn, fn);
+                if (n_a_next == 1) q_release(fn);
+              }
             }
           }
           if (!issue_pv(1, gg, jj == 0)) break;
@@ -1459,12 +1548,17 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
             ++ix[1];
           } else {
             if (!wait_k(gg + 1)) break;
-            issue_s(1, gg + 1);
+            issue_s(1, gg + 1, fb);
             umma_commit(k_empty + (gg + 1) % NK);
-            if (jj + 1 == n_b - 1) umma_commit(q_empty);
+            if (jj + 1 == n_b - 1) q_release(fb);
           }
         }
+        if (!ok) break;
         g += n_b;
+        j = jn;
+        n_a = n_a_next;
+        n_b = n_b_next;
+        pre = pre_next;
       }
     }
   }
@@ -1477,20 +1571,39 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
     const uint32_t ts = tmem + lane_base + 128 * x, to = tmem + lane_base + 256 + 128 * x;
     int gx = 0, ix = 0, where = 0;
     bool ok = true;
-    for (int r = 0; ok; ++r) {
-      const int slot = r & 1;
-      if (!warp_wait(item_full + slot, (r >> 1) & 1, abort)) {
+    // item rr of the ring: its index and this warpgroup's tile, read ahead of the previous item's
+    // epilogue, and the tile's segment records pulled into L1, so that none of these loads sits on
+    // the slot's critical path
+    struct Next {
+      int j, tile_id;
+      AttnTile tile;
+    };
+    auto take = [&](int rr, Next& nx) -> bool {
+      if (!warp_wait(item_full + (rr & 1), (rr >> 1) & 1, abort)) {
         where = 10;
-        break;
+        return false;
       }
-      const int j = item_ring[slot];
-      mbar_arrive(item_empty + slot);
-      if (j < 0) break;
-      const int2 pr = pair_of(j);
-      const int tile_id = x ? pr.y : pr.x;
-      if (tiles_of(tile_id) == 0) continue;
-      const AttnTile tile = a.tiles[tile_id];
-      const int bh = j / a.n_pairs, b = bh / a.H, h = bh % a.H;
+      nx.j = item_ring[rr & 1];
+      mbar_arrive(item_empty + (rr & 1));
+      nx.tile_id = -1;
+      nx.tile = AttnTile{0, 0, 0, 0};
+      if (nx.j < 0) return true;
+      const int2 pr = pair_of(nx.j);
+      nx.tile_id = x ? pr.y : pr.x;
+      if (nx.tile_id >= 0) nx.tile = a.tiles[nx.tile_id];
+      if (nx.tile.nkt > 0 && lane == 0) prefetch_l1(a.segs + nx.tile.seg0, nx.tile.nseg * (int)sizeof(AttnSeg));
+      return true;
+    };
+    Next cur;
+    if (!take(0, cur)) ok = false;
+    for (int r = 0; ok && cur.j >= 0; ++r) {
+      if (cur.tile.nkt == 0) {
+        if (!take(r + 1, cur)) break;
+        continue;
+      }
+      const int tile_id = cur.tile_id;
+      const AttnTile tile = cur.tile;
+      const int bh = cur.j / a.n_pairs, b = bh / a.H, h = bh % a.H;
       if (row == 0) item_s = tile_id * 65536 + bh;
       const int tq = tile.q0 + row;
       float m_used = -INFINITY, l = 0.f;
@@ -1518,6 +1631,7 @@ __global__ void __launch_bounds__(384, 1) attn_pp_kernel(const __grid_constant__
         }
       }
       if (!ok) break;
+      if (!take(r + 1, cur)) break;
       if (!warp_wait(pv_done + x, ix & 1, abort)) {
         where = 8;
         break;
@@ -1617,8 +1731,9 @@ cudaError_t launch_tc_t(const AttnArgs& a, int* status, cudaStream_t st) {
       int dev = 0, sms = 0;
       cudaError_t e = cudaGetDevice(&dev);
       if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-      const size_t sm = PpLayout<E, D>::BYTES;
-      auto kern = attn_pp_kernel<E, D>;
+      // two Q buffers: a third costs a K stage (E = D = 128) and measured no faster
+      const size_t sm = PpLayout<E, D, 2>::BYTES;
+      auto kern = attn_pp_kernel<E, D, 2>;
       if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
       int per_sm = 0;
       if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 384, sm);

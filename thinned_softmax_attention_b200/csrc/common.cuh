@@ -176,6 +176,7 @@ struct AttnTile {
   int qlen;      // queries in the tile
   int seg0;      // first segment in the segment table
   int nseg;
+  int nkt = 0;   // 128-key tiles over its segments (sum of ceil(len / 128)), filled by the host before upload
 };
 
 struct AttnArgs {

@@ -35,6 +35,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Pull the 128-byte lines covering [p, p + bytes) into this SM's L1 (no registers held).
+__device__ __forceinline__ void prefetch_l1(const void* p, int bytes) {
+  const uintptr_t b = (uintptr_t)p & ~(uintptr_t)127, e = (uintptr_t)p + bytes;
+  for (uintptr_t x = b; x < e; x += 128) asm volatile("prefetch.global.L1 [%0];" ::"l"(x));
+}
+// Non-blocking test: has the phase of `parity` completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase of `parity` to complete.  Gives up (returns false) when *abort is set by
 // another thread or after kWaitCycles, in which case it sets *abort itself.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
