@@ -215,6 +215,20 @@ def kernel_traffic(name):
     return d["bytes_per_launch"]
 
 
+KERNEL_SWITCHES = ("THIN_ATTN_PP", "THIN_ATTN_TC2P", "THIN_ATTN_TC1", "THIN_ATTN_TC2_PER_TILE", "THIN_ATTN_SIMT_ATTN",
+                   "THIN_ATTN_OVERLAP")
+
+
+def attention_traffic(w):
+    """DRAM bytes per launch of the attention kernel the library picks for this workload, from the
+    committed ncu summaries (Express 32K: the two-CTA kernel; Express 128K: the ping-pong kernel);
+    None when another kernel is forced or the workload differs from the captured one."""
+    if w.H != 32 or any(os.environ.get(k) for k in KERNEL_SWITCHES):
+        return None
+    return {"express32k": kernel_traffic("attention"),
+            "express128k": kernel_traffic("attention_pp_express128k")}.get(w.name)
+
+
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -533,7 +547,7 @@ def measure_workload(TA, name, dev, steps, warmup):
            "inputs larger than L2 (no flush)",
            "phases_ms": {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
                          "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4), "attn_ms": round(attn_ms, 4)},
-           "roofline": attention_roofline(w, plan, attn_ms, pk),
+           "roofline": dict(attention_roofline(w, plan, attn_ms, pk), traffic=attention_traffic(w)),
            "halving_roofline": halving_roofline(w, h, ph, pk),
            "gpu_launches_per_step": plan["kernel_launches"]}
     rec["approx_error"] = exact_reference_error(w, qc, kc, vc, out)
@@ -600,7 +614,7 @@ def main():
     pk = peaks()
     attn_ms = ph["attn_ms"] / max(1, ph["calls"])
     roof = attention_roofline(w, plan, attn_ms, pk)
-    roof["traffic"] = kernel_traffic("attention") if (w.name == "express32k" and w.H == 32) else None
+    roof["traffic"] = attention_traffic(w)
     halving_roof = halving_roofline(w, h, ph, pk)
     phases = {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
               "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4),
