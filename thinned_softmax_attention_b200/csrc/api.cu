@@ -1961,7 +1961,7 @@ thin_attn_status cache_build(thin_attn_cache_s* cc) {
     cc->max_splits = std::max(cc->max_splits, (cc->pos_keys[pos] + decode_chunk_keys() - 1) / decode_chunk_keys());
   }
   // split-key kernels when few (b,h) rows would leave most SMs idle with one CTA per row
-  cc->use_split = decode_attention_supported(cf.E, cf.D, max_segs) && BH <= 64 &&
+  cc->use_split = decode_attention_supported(cf.E, cf.D, max_segs, cc->max_splits) && BH <= 64 &&
                   std::getenv("THIN_ATTN_DECODE_TILES") == nullptr;
   // device layout
   size_t off = 0;

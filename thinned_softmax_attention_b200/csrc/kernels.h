@@ -68,7 +68,7 @@ struct DecodeAppend {
   int nseg = -1;
   AttnSeg segs[32];
 };
-bool decode_attention_supported(int E, int D, int max_segments);
+bool decode_attention_supported(int E, int D, int max_segments, int max_splits);
 int decode_chunk_keys();
 cudaError_t launch_decode_attention(const AttnArgs& a, int dtype, int n_splits, float* part, const DecodeAppend& ap,
                                     cudaStream_t st);
