@@ -332,15 +332,18 @@ def test_scheduled_and_levelwise_halving_agree(name, monkeypatch):
             assert torch.equal(res[0][key], r[key]), key
 
 
-@pytest.mark.parametrize("name", ["vit", "express", "express_a", "express_ragged"])
+@pytest.mark.parametrize("name", ["vit", "express", "express_a", "express_ragged", "vit_e64_d128", "vit_e128_d64"])
 def test_attention_launch_forms_agree(name, monkeypatch):
     """The ping-pong kernel (two query tiles of a head against one K/V stream, one CTA per SM), the
     two-CTA persistent kernel (items from a work counter), its one-CTA-per-tile form, and the
     persistent kernel launched as several dependent waves on a side stream (each launch takes and
     resets the same counter) run the same per-tile arithmetic: outputs and LSE are bit-identical.
     ViT's 25 query tiles per head leave one tile unpaired; the ragged Express shape has batches of
-    three tiles, so pairs cross from the exact phase into batches and some tiles run alone."""
+    three tiles, so pairs cross from the exact phase into batches and some tiles run alone.  The two
+    ViT variants with unequal head dims take the ping-pong kernel's other ring layouts (4 K stages)."""
     w = {"vit": W.WORKLOADS["vit"].with_(B=8),
+         "vit_e64_d128": W.WORKLOADS["vit"].with_(B=4, D=128),
+         "vit_e128_d64": W.WORKLOADS["vit"].with_(B=4, E=128),
          "express": W.WORKLOADS["express32k"].with_(T=8192, H=4),
          "express_a": W.WORKLOADS["express32k_a"].with_(T=8192, H=4),
          "express_ragged": W.WORKLOADS["express32k"].with_(T=3000, H=3, n_exact=200, batch=300)}[name]
