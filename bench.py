@@ -10,8 +10,10 @@ HBM.  Prints one JSON line on rank 0.  Multi-GPU (torchrun): the ranks hold
 parts of one problem whose (b,h) slices are independent -- `--shard batch`
 (default, weak scaling): rank r holds batch rows [rB, (r+1)B) of a problem with
 N*B rows; `--shard heads` (strong scaling): rank r holds H/N heads of the
-workload.  No collective on the data path; the random decisions are keyed on the
-whole problem's (b,h); step time is the max over ranks of CUDA-event time.
+workload; `--shard seq` (strong scaling): rank r attends query rows
+[r T/N, (r+1) T/N) (128-aligned) of every (b,h), each rank thinning all keys.
+No collective on the data path; the random decisions are keyed on the whole
+problem's (b,h); step time is the max over ranks of CUDA-event time.
 
 --impl reference times the fp64 CPU oracle on the host cores (rank 0 only),
 each step one head of the workload.
@@ -47,7 +49,7 @@ def args_():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="thin", choices=["thin", "reference"])
     p.add_argument("--workload", default="express32k", choices=sorted(W.WORKLOADS))
-    p.add_argument("--shard", default="batch", choices=["batch", "heads"],
+    p.add_argument("--shard", default="batch", choices=["batch", "heads", "seq"],
                    help="N>1: batch rows of one larger problem per rank (weak) or the heads of one problem (strong)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -80,43 +82,46 @@ def digitsum4(k):
     return s
 
 
-def attention_work(w, plan):
+def attention_work(w, plan, rows=None):
     """Algorithmic FLOPs and HBM bytes of one attention launch.
 
     FLOPs: 2 (E + D) per visible (query, key) pair.  Bytes: q read and out written
-    once, plus every distinct key/value row read once (original tokens and coreset rows)."""
+    once, plus every distinct key/value row read once (original tokens and coreset rows).
+    ``rows=(q0, q1)``: a query-row shard's launch (its rows' pairs, q and out; the key/value rows
+    are counted whole, an upper bound)."""
     BH = w.B * w.H
     es = 4 if w.dtype == "fp32" else 2
     if not w.causal:
         keys = plan["coreset_rows"] if plan["levels"] > 0 else w.S
-        pairs = w.T * keys
+        vis = np.full(w.T, keys, dtype=np.int64)
         kv_rows = keys
     elif w.cache == "A":
         # tokens [0, 4 n_out) exactly; batch (i, s): H_i and s - 1 thinned batches (n_out points each)
         # and its own tokens causally
         n_out = min(w.n_exact, w.T)
         ex = min(4 * n_out, w.T)
-        vis = [np.arange(1, ex + 1, dtype=np.int64)]
+        parts = [np.arange(1, ex + 1, dtype=np.int64)]
         start, i = n_out * 4, 1
         while start < w.T:
             for s_ in range(1, 4):
                 if start >= w.T:
                     break
                 size = min(4 ** i * n_out, w.T - start)
-                vis.append(s_ * n_out + np.arange(1, size + 1, dtype=np.int64))
+                parts.append(s_ * n_out + np.arange(1, size + 1, dtype=np.int64))
                 start += size
             i += 1
-        pairs = int(np.concatenate(vis).sum())
+        vis = np.concatenate(parts)
         kv_rows = w.T + plan["n_nodes"] * plan["coreset_rows"]
     else:
         t = np.arange(w.T, dtype=np.int64)
         ne, b, c = min(w.n_exact, w.T), w.batch, plan["coreset_rows"]
         k = np.maximum(t - ne, 0) // b
         vis = np.where(t < ne, t + 1, ne + c * digitsum4(k) + (t - (ne + k * b) + 1))
-        pairs = int(vis.sum())
         kv_rows = w.T + plan["n_nodes"] * c
+    q0, q1 = rows if rows else (0, w.T)
+    pairs = int(vis[q0:q1].sum())
     flops = 2.0 * (w.E + w.D) * pairs * BH
-    bytes_ = es * BH * (w.T * (w.E + w.D) + kv_rows * (w.E + w.D))
+    bytes_ = es * BH * ((q1 - q0) * (w.E + w.D) + kv_rows * (w.E + w.D))
     return flops, bytes_, pairs
 
 
@@ -277,7 +282,7 @@ class Shard:
     what a single run of the whole problem computes for its rows; no data crosses between ranks."""
 
     def __init__(self, w, world, rank, mode="batch"):
-        if mode not in ("batch", "heads"):
+        if mode not in ("batch", "heads", "seq"):
             raise ValueError(mode)
         if mode == "heads" and w.H % world:
             raise ValueError(f"--shard heads needs H={w.H} divisible by the {world} ranks")
@@ -291,7 +296,20 @@ class Shard:
         self.global_batch = world * w.B if mode == "batch" else w.B
         self.whole_tokens = self.global_batch * w.H * w.T
         self.scaling = "weak" if mode == "batch" else "strong"
-        self.parallelism = f"{'dp' if mode == 'batch' else 'hp'}{world}"
+        self.parallelism = {"batch": "dp", "heads": "hp", "seq": "sp"}[mode] + str(world)
+        self.q_range = (0, 0)
+        if mode == "seq":
+            # equal 128-aligned slices of the query rows, the last one ending at T
+            step = -(-w.T // world // 128) * 128 if w.T >= 128 * world else 0
+            q0, q1 = rank * step, (w.T if rank == world - 1 else (rank + 1) * step)
+            if step == 0 or q0 >= q1 or q1 > w.T:
+                raise ValueError(f"--shard seq needs T={w.T} >= 128 rows per rank")
+            self.q_range = (q0, q1)
+
+    @property
+    def rows(self):
+        """Query rows this rank attends (all of them unless --shard seq)."""
+        return self.q_range if self.mode == "seq" else None
 
     @property
     def abi(self):
@@ -426,12 +444,12 @@ def exact_reference_error(w, q, k, v, out, n_rows=128, max_b=4, max_h=4):
             "max_rel_per_row": round(row.max().item(), 5), "mean_rel_per_row": round(row.mean().item(), 5)}
 
 
-def attention_roofline(w, plan, attn_ms, pk):
+def attention_roofline(w, plan, attn_ms, pk, rows=None):
     """Roofline of the attention launch: bound by its arithmetic intensity against the ridge of the
     burst bf16 peak over HBM copy bandwidth.  The launch is timed alone, sub-second, at full clocks,
     so the burst peak is the denominator; the fraction of the sustained (power-capped) peak is
     reported beside it."""
-    flops, abytes, pairs = attention_work(w, plan)
+    flops, abytes, pairs = attention_work(w, plan, rows)
     ridge = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
     if w.dtype != "fp32" and flops / abytes >= ridge:
         achieved = flops / (attn_ms * 1e-3) / 1e12
@@ -580,7 +598,7 @@ def main():
     q, k, v = (x.to(dev) for x in (qc, kc, vc))
     S = w.T if w.causal else w.S
     h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch,
-                         device=local, shard=shard.abi)
+                         device=local, shard=shard.abi, q_range=shard.q_range)
     plan = h.plan(w.mode, w.g)
     h.reserve(w.mode, w.g)
     out = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype, device=dev)
@@ -613,15 +631,43 @@ def main():
 
     pk = peaks()
     attn_ms = ph["attn_ms"] / max(1, ph["calls"])
-    roof = attention_roofline(w, plan, attn_ms, pk)
-    roof["traffic"] = attention_traffic(w)
+    roof = attention_roofline(w, plan, attn_ms, pk, shard.rows)
+    roof["traffic"] = attention_traffic(w) if shard.rows is None else None
     halving_roof = halving_roofline(w, h, ph, pk)
     phases = {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
               "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4),
               "attn_ms": round(attn_ms, 4)}
 
     e2e = None
-    if not a.no_e2e:
+    if not a.no_e2e and shard.rows is not None:
+        # the host-buffer entry takes no query-row range: the inputs go in by pinned copies, this
+        # rank's rows of out come back the same way, all on the timed stream
+        q0, q1 = shard.rows
+        qh, kh, vh = (x.pin_memory() for x in (qc, kc, vc))
+        oh = torch.empty(w.B, q1 - q0, w.H, w.D, dtype=w.torch_dtype).pin_memory()
+
+        def e2e_step():
+            for dst, src in ((q, qh), (k, kh), (v, vh)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            oh.copy_(out[:, q0:q1], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        n_e2e = max(2, min(a.steps, 5))
+        if dist:
+            dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(f0.elapsed_time(f1) / n_e2e, dist, dev)
+        e2e = {"value": shard.whole_tokens / (ems * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * es,
+               "d2h_bytes_per_step": oh.numel() * es, "ms_per_step": round(ems, 3)}
+    elif not a.no_e2e:
         qh, kh, vh = (x.pin_memory() for x in (qc, kc, vc))
         oh = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype).pin_memory()
         for _ in range(2):

@@ -85,6 +85,14 @@ typedef struct {
    * the scales undone in the softmax; P V stays bf16.  The thinning always uses the bf16 keys.  bf16
    * handles with E = 128, D <= 128, H <= 128; EUNSUPPORTED otherwise.  The decode cache ignores it. */
   int qk_fp8;
+  /* Query-row shard: attend only the query rows [q_begin, q_end) of every (b,h).  The thinning still
+   * runs over all keys, so these rows come out bit-identical to the whole run's, and the rows of out
+   * and lse outside the range are not written: ranks holding disjoint ranges of one sequence need
+   * no communication (sequence parallelism when B*H is below the GPU count).  Both zero: every row.
+   * EINVAL unless 0 <= q_begin < q_end <= T, q_begin a multiple of 128 and q_end a multiple of 128
+   * or T.  thin_attn_forward_host and the decode cache take no range (EUNSUPPORTED / EINVAL). */
+  int q_begin;
+  int q_end;
 } thin_attn_config;
 
 /* Sizes of one (causal, g) plan. */
@@ -100,6 +108,7 @@ typedef struct {
   uint64_t trace_words;        /* uint32 words of the decision trace */
   uint64_t coreset_idx_elems;  /* int32 elements of coreset_idx_opt */
   uint64_t workspace_bytes;    /* device workspace the plan needs */
+  int attn_rows;               /* query rows of each (b,h) the attention writes (T, or q_end - q_begin) */
 } thin_attn_plan_info;
 
 /* Where the decisions of one halving instance sit in the trace. */

@@ -9,6 +9,7 @@ import re
 import subprocess
 
 import numpy as np
+import torch
 import pytest
 
 import thinned_softmax_attention_b200 as T
@@ -272,3 +273,45 @@ def test_fp8_qk_refuses_unsupported_shapes(kw):
     w = W.WORKLOADS["express32k"].with_(**kw)
     with pytest.raises(T.ThinAttnError, match="EUNSUPPORTED"):
         T.ThinAttention(w.B, w.T, w.T, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch, qk_fp8=True)
+
+
+@pytest.mark.parametrize("mode,T_,S,ne,bsz", [(1, 3000, 3000, 200, 300), (1, 8192, 8192, 1024, 1024),
+                                             (0, 3136, 3136, 0, 0), (2, 8192, 8192, 128, 0)])
+def test_query_ranges_cover_every_row_once(mode, T_, S, ne, bsz):
+    """Query-row shards (sequence parallelism): each range's plan attends exactly its rows, and ranges
+    that partition [0, T) cover every row once -- also where the tiles do not start on multiples of
+    128 (200 exact tokens, batches of 300), so tiles are clipped at the range ends."""
+    dt = W.WORKLOADS["express32k"].torch_dtype
+    full = T.ThinAttention(1, T_, S, 2, 128, 128, dt, n_exact=ne, batch=bsz).plan(mode, 2)
+    assert full["attn_rows"] == T_
+    cuts = [0, 1024, 1152, 2048, T_]
+    total = 0
+    for r in zip(cuts[:-1], cuts[1:]):
+        h = T.ThinAttention(1, T_, S, 2, 128, 128, dt, n_exact=ne, batch=bsz, q_range=r)
+        p = h.plan(mode, 2)
+        assert p["attn_rows"] == r[1] - r[0]
+        # the thinning is the whole run's: same halvings, same coreset layout
+        assert p["n_halvings"] == full["n_halvings"] and p["coreset_idx_elems"] == full["coreset_idx_elems"]
+        total += p["attn_rows"]
+    assert total == T_
+
+
+@pytest.mark.parametrize("r", [(100, 384), (0, 100), (256, 128), (-128, 128), (0, 3128), (128, 128)])
+def test_query_range_must_be_aligned_and_inside(r):
+    with pytest.raises(T.ThinAttnError, match="EINVAL"):
+        T.ThinAttention(1, 3000, 3000, 2, 128, 128, W.WORKLOADS["express32k"].torch_dtype, n_exact=200, batch=300,
+                        q_range=r)
+
+
+def test_query_range_is_refused_by_the_host_path_and_the_cache():
+    dt = W.WORKLOADS["express32k"].torch_dtype
+    h = T.ThinAttention(1, 3000, 3000, 1, 128, 128, dt, n_exact=200, batch=300, q_range=(0, 1024))
+    x = torch.zeros(1, 3000, 1, 128, dtype=dt)
+    o = torch.zeros_like(x)
+    p = ctypes.c_void_p
+    st = T.lib().thin_attn_forward_host(h._h, p(x.data_ptr()), p(x.data_ptr()), p(x.data_ptr()), p(o.data_ptr()), 1, 2,
+                                        ctypes.c_uint64(1), None, None)
+    assert st == 5, st   # THIN_ATTN_EUNSUPPORTED, refused before any copy
+    cfg = T.Config(T.BF16, 1, 64, 64, 1, 128, 128, 0.0, 16, 16, 0, 0, 0, 0, 0, 0, 64)
+    c = ctypes.c_void_p()
+    assert T.lib().thin_attn_cache_create(ctypes.byref(c), ctypes.byref(cfg), 2, ctypes.c_uint64(1)) != 0

@@ -1,4 +1,4 @@
-"""Batch- and head-parallel shards on one GPU, through the C ABI.
+"""Batch-, head- and sequence-parallel shards on one GPU, through the C ABI.
 
 A shard is a handle over batch rows [b0, b0 + B) and heads [h0, h0 + H) of a larger problem
 (config fields b0, h0, H_total): its Philox counters are keyed on the whole problem's (b,h), so its
@@ -114,3 +114,41 @@ def test_shard_matches_the_oracle(name):
     assert float(err.max()) <= 1e-2
     lse = r["lse"].cpu().numpy()[:, :, rows]
     assert float(np.abs(lse - ref.lse).max()) <= 2e-3
+
+
+SEQ_CASES = {
+    "express": (W.WORKLOADS["express32k"].with_(H=4, T=12 * 1024), [0, 1024, 4096, 4224, 12 * 1024]),
+    "express_ragged": (W.WORKLOADS["express32k"].with_(T=3000, H=3, n_exact=200, batch=300), [0, 128, 1152, 2048, 3000]),
+    "express_a": (W.WORKLOADS["express32k_a"].with_(H=4, T=8192), [0, 512, 2048, 8192]),
+    "vit": (W.WORKLOADS["vit"].with_(B=4), [0, 1024, 1152, 3136]),
+}
+
+
+@pytest.mark.parametrize("form", ["default", "ping_pong"])
+@pytest.mark.parametrize("name", sorted(SEQ_CASES))
+def test_query_row_shards_equal_the_whole_problem(name, form, monkeypatch):
+    """Sequence-parallel shards (config q_begin, q_end): every shard thins all keys and attends only
+    its query rows; its rows of out and lse equal the whole run's bit for bit, its coreset and
+    decisions are the whole run's, and the rows outside its range keep what the buffers held (a
+    sentinel).  Range ends fall inside tiles where the exact phase and the batches are not multiples
+    of 128 rows (the ragged shape), so clipped tiles are covered; the ping-pong form rebuilds its tile
+    pairs inside each range."""
+    if form == "ping_pong":
+        monkeypatch.setenv("THIN_ATTN_PP", "1")
+    w, cuts = SEQ_CASES[name]
+    q, k, v = (x.to(DEV) for x in W.make_qkv(w))
+    S = w.T if w.causal else w.S
+    whole = _run(w, q, k, v)
+    for q0, q1 in zip(cuts[:-1], cuts[1:]):
+        h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch,
+                             q_range=(q0, q1))
+        out = torch.full((w.B, w.T, w.H, w.D), 7.0, dtype=w.torch_dtype, device=DEV)
+        lse = torch.full((w.B, w.H, w.T), -3.0, dtype=torch.float32, device=DEV)
+        r = h.forward(q, k, v, causal=w.mode, g=w.g, seed=w.seed, out=out, lse=lse, return_coreset=True)
+        torch.cuda.synchronize()
+        h.check()
+        assert torch.equal(out[:, q0:q1], whole["out"][:, q0:q1])
+        assert torch.equal(lse[:, :, q0:q1], whole["lse"][:, :, q0:q1])
+        assert bool((out[:, :q0] == 7.0).all()) and bool((out[:, q1:] == 7.0).all())
+        assert bool((lse[:, :, :q0] == -3.0).all()) and bool((lse[:, :, q1:] == -3.0).all())
+        assert torch.equal(r["coreset"], whole["coreset"])

@@ -117,3 +117,61 @@ def test_single_process_needs_no_collective():
     assert sh.abi == (0, 0, 32) and sh.local == W.WORKLOADS["express32k"] and sh.scaling == "weak"
     with pytest.raises(ValueError):
         bench.Shard(W.WORKLOADS["express32k"], 3, 0, "heads")
+
+
+def _rank_seq(rank, world, port, q, name):
+    import datetime
+    import bench
+    from oracle import express, thinformer
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = _WHOLE[name]
+        sh = bench.Shard(w, world, rank, "seq")
+        q0, q1 = sh.q_range
+        qq, kk, vv = sh.inputs(sh.local)
+        rows = list(range(q0, q1))
+        part = (express(qq, kk, vv, w.n_exact, w.batch, w.g, w.seed, rows=rows) if w.causal
+                else thinformer(qq, kk, vv, w.g, w.seed, rows=rows))
+        ms = bench.max_over_ranks([2.0, 3.5][rank], dist, torch.device("cpu"))
+        q.put((rank, sh.q_range, sh.abi, sh.local.H, sh.scaling, sh.parallelism, sh.whole_tokens, ms, part.out))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name", ["thin", "express"])
+def test_two_rank_sequence_shards_reproduce_the_whole_problem(name):
+    """--shard seq: each rank holds every head and attends a 128-aligned slice of the query rows
+    (the last ending at T); the slices partition [0, T) and the stacked rows equal the whole run's
+    (the oracle evaluates a subset of rows with other BLAS blocking: equal to 1e-12)."""
+    from oracle import express, thinformer
+    ctx = mp.get_context("spawn")
+    qu = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_seq, args=(r, 2, port, qu, name)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((qu.get(timeout=300) for _ in range(2)), key=lambda r: r[0])
+    for p in procs:
+        p.join(60)
+    assert all(p.exitcode == 0 for p in procs)
+    whole = _WHOLE[name]
+    ranges = [r[1] for r in res]
+    assert ranges[0][0] == 0 and ranges[0][1] == ranges[1][0] and ranges[1][1] == whole.T
+    assert ranges[0][1] % 128 == 0
+    assert all(r[2] == (0, 0, whole.H) and r[3] == whole.H for r in res)
+    assert {r[4] for r in res} == {"strong"} and {r[5] for r in res} == {"sp2"}
+    assert all(r[6] == whole.B * whole.H * whole.T and r[7] == 3.5 for r in res)
+    q, k, v = W.make_qkv(whole)
+    ref = (express(q, k, v, whole.n_exact, whole.batch, whole.g, whole.seed) if whole.causal
+           else thinformer(q, k, v, whole.g, whole.seed))
+    np.testing.assert_allclose(np.concatenate([r[8] for r in res], axis=1), ref.out, rtol=0, atol=1e-12)
+
+
+def test_sequence_shard_needs_rows_for_every_rank():
+    import bench
+    with pytest.raises(ValueError):
+        bench.Shard(W.WORKLOADS["tiny"], 3, 0, "seq")        # T = 256 < 3 x 128
+    sh = bench.Shard(W.WORKLOADS["express32k"], 8, 7, "seq")
+    assert sh.q_range == (28672, 32768) and sh.rows == (28672, 32768)

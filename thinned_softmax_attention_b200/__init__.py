@@ -37,14 +37,15 @@ class Config(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("B", ctypes.c_int), ("T", ctypes.c_int), ("S", ctypes.c_int),
                 ("H", ctypes.c_int), ("E", ctypes.c_int), ("D", ctypes.c_int), ("scale", ctypes.c_float),
                 ("n_exact", ctypes.c_int), ("batch", ctypes.c_int), ("device", ctypes.c_int),
-                ("b0", ctypes.c_int), ("h0", ctypes.c_int), ("H_total", ctypes.c_int), ("qk_fp8", ctypes.c_int)]
+                ("b0", ctypes.c_int), ("h0", ctypes.c_int), ("H_total", ctypes.c_int), ("qk_fp8", ctypes.c_int),
+                ("q_begin", ctypes.c_int), ("q_end", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
     _fields_ = [("levels", ctypes.c_int), ("leaf", ctypes.c_int), ("subsampled", ctypes.c_int),
                 ("coreset_rows", ctypes.c_int), ("n_batches", ctypes.c_int), ("n_nodes", ctypes.c_int),
                 ("n_halvings", ctypes.c_int), ("kernel_launches", ctypes.c_int), ("trace_words", ctypes.c_uint64),
-                ("coreset_idx_elems", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64)]
+                ("coreset_idx_elems", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64), ("attn_rows", ctypes.c_int)]
 
 
 class TraceEntry(ctypes.Structure):
@@ -126,13 +127,20 @@ class ThinAttention:
     [h0, h0 + H) of a larger problem with H_total heads (one handle per GPU of a batch- or
     head-parallel run); the random decisions, and so every output, equal the whole
     problem's for those (b,h).
+
+    ``q_range=(q_begin, q_end)``: attend only query rows [q_begin, q_end) (multiples of 128; the
+    end may be T) of every (b,h); the thinning runs over all keys, so those rows equal the whole
+    run's and the other rows of ``out`` and ``lse`` are left as they were (sequence-parallel
+    shards of one long sequence, one per GPU, with no communication).
     """
 
     def __init__(self, B: int, T: int, S: int, H: int, E: int, D: int, dtype: torch.dtype,
                  scale: Optional[float] = None, n_exact: int = 0, batch: int = 0, device: int = 0,
-                 shard: Tuple[int, int, int] = (0, 0, 0), qk_fp8: bool = False):
+                 shard: Tuple[int, int, int] = (0, 0, 0), qk_fp8: bool = False,
+                 q_range: Tuple[int, int] = (0, 0)):
         self.cfg = Config(FP32 if dtype == torch.float32 else BF16, B, T, S, H, E, D,
-                          0.0 if scale is None else float(scale), n_exact, batch, device, *shard, int(qk_fp8))
+                          0.0 if scale is None else float(scale), n_exact, batch, device, *shard, int(qk_fp8),
+                          *q_range)
         self.dtype = dtype
         self.device = torch.device("cuda", device)
         self._h = ctypes.c_void_p()
@@ -179,7 +187,9 @@ class ThinAttention:
 
     def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, g: int = 2,
                 seed: int = 0, return_lse: bool = False, return_coreset: bool = False,
-                return_trace: bool = False, out: Optional[torch.Tensor] = None):
+                return_trace: bool = False, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+        """``out`` and ``lse`` (B,H,T fp32) may be the caller's buffers (a query-row shard writes only its
+        rows of them); ``lse`` given implies ``return_lse``."""
         c = self.cfg
         L = c.T if causal else c.S
         for name, t, shape in (("q", q, (c.B, c.T, c.H, c.E)), ("k", k, (c.B, L, c.H, c.E)),
@@ -190,7 +200,12 @@ class ThinAttention:
         if out is None:
             out = torch.empty(c.B, c.T, c.H, c.D, dtype=self.dtype, device=self.device)
         info = self.plan(causal, g)
-        lse = torch.empty(c.B, c.H, c.T, dtype=torch.float32, device=self.device) if return_lse else None
+        if lse is not None:
+            if tuple(lse.shape) != (c.B, c.H, c.T) or lse.dtype != torch.float32 or not lse.is_contiguous():
+                raise ValueError(f"lse: expected contiguous float32 {(c.B, c.H, c.T)}, got {lse.dtype} {tuple(lse.shape)}")
+            return_lse = True
+        elif return_lse:
+            lse = torch.empty(c.B, c.H, c.T, dtype=torch.float32, device=self.device)
         cidx = (torch.empty(max(1, info["coreset_idx_elems"]), dtype=torch.int32, device=self.device)
                 if return_coreset else None)
         trace = (torch.zeros(max(1, info["trace_words"]), dtype=torch.int32, device=self.device)

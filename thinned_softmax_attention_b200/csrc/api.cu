@@ -365,6 +365,22 @@ void build_attn_tables(const thin_attn_config& cf, const Plan& p, int QT, AttnTa
   }
 }
 
+// A query-row shard (config q_begin, q_end): keep the tiles that hold rows of the range, each clipped
+// to it.  A clipped tile keeps its key segments; a row's arithmetic depends on its own position only
+// (the causal mask is per row), so its output is the whole run's.
+void restrict_rows(const thin_attn_config& cf, AttnTables& t) {
+  if (cf.q_begin == 0 && cf.q_end == 0) return;
+  std::vector<AttnTile> kept;
+  for (AttnTile tl : t.tiles) {
+    const int a = std::max(tl.q0, cf.q_begin), b = std::min(tl.q0 + tl.qlen, cf.q_end);
+    if (a >= b) continue;
+    tl.q0 = a;
+    tl.qlen = b - a;
+    kept.push_back(tl);
+  }
+  t.tiles.swap(kept);
+}
+
 // Each tile's count of 128-key tiles (AttnTile::nkt), which the attention kernels read.
 void set_key_tile_counts(AttnTables& t) {
   for (AttnTile& tl : t.tiles) {
@@ -831,9 +847,11 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
     p->c2_floats = std::max(p->c2_floats, st.inst.size());
   }
   build_attn_tables(cf, *p, attention_simt_tile_rows(), p->simt);
+  restrict_rows(cf, p->simt);
   build_waves(cf, *p, p->simt);
   if (attention_tc_supported(cf.dtype, cf.E, cf.D)) {
     build_attn_tables(cf, *p, attention_tc_tile_rows(), p->tc);
+    restrict_rows(cf, p->tc);
     build_waves(cf, *p, p->tc);
     build_pairs(p->tc);
   }
@@ -969,6 +987,13 @@ thin_attn_status check_cfg(const thin_attn_config* c) {
                 (long long)Ht);
   if (((int64_t)c->b0 + c->B) * Ht > (int64_t)UINT32_MAX)
     return fail(THIN_ATTN_EINVAL, "(b0 + B) * H_total exceeds the 32-bit Philox (b,h) word");
+  if (c->q_begin != 0 || c->q_end != 0) {
+    if (c->q_begin < 0 || c->q_end <= c->q_begin || c->q_end > c->T)
+      return fail(THIN_ATTN_EINVAL, "query rows [%d, %d) are not a range inside [0, T=%d)", c->q_begin, c->q_end, c->T);
+    if (c->q_begin % 128 || (c->q_end % 128 && c->q_end != c->T))
+      return fail(THIN_ATTN_EINVAL, "query rows [%d, %d): both ends must be multiples of 128 (the end may be T)",
+                  c->q_begin, c->q_end);
+  }
   if (c->qk_fp8 != 0 && c->qk_fp8 != 1) return fail(THIN_ATTN_EINVAL, "qk_fp8 must be 0 or 1");
   if (c->qk_fp8 && (c->dtype != THIN_ATTN_BF16 || c->E != 128 || c->D > 128 || c->D % 64 || !qk_fp8_supported(c->H, c->E)))
     return fail(THIN_ATTN_EUNSUPPORTED, "qk_fp8 needs bf16 with E = 128, D = 64 or 128 and H <= 128 (E=%d D=%d H=%d)", c->E,
@@ -1421,6 +1446,12 @@ thin_attn_status thin_attn_plan(thin_attn_t h, int causal, int g, thin_attn_plan
     if (!sched || si < p->sched_s0 || si >= p->sched_s1) launches += step_launches(h->cfg, p, p->steps[si]);
   if (sched) launches += 1;
   info->kernel_launches = launches;
+  {
+    const AttnTables& at = !p->tc.tiles.empty() ? p->tc : p->simt;
+    int rows = 0;
+    for (const AttnTile& tl : at.tiles) rows += tl.qlen;
+    info->attn_rows = rows;
+  }
   info->trace_words = p->trace_words;
   info->coreset_idx_elems = p->coreset_idx_elems;
   info->workspace_bytes = p->bytes;
@@ -1565,6 +1596,8 @@ thin_attn_status thin_attn_forward_host(thin_attn_t h, const void* q, const void
   if (!h) return fail(THIN_ATTN_EINVAL, "null handle");
   if (!q || !k || !v || !out) return fail(THIN_ATTN_EINVAL, "q, k, v and out must be non-null");
   const thin_attn_config& c = h->cfg;
+  if (c.q_begin != 0 || c.q_end != 0)
+    return fail(THIN_ATTN_EUNSUPPORTED, "the host-buffer forward takes no query-row range (q_begin, q_end)");
   const size_t es = elt(c);
   const int64_t L = causal ? c.T : c.S;
   const size_t qb = (size_t)c.B * c.T * c.H * c.E * es, kb = (size_t)c.B * L * c.H * c.E * es,
@@ -2085,6 +2118,7 @@ thin_attn_status thin_attn_cache_create(thin_attn_cache_t* out, const thin_attn_
   if (s != THIN_ATTN_OK) return s;
   if (g < 0 || g > 6) return fail(THIN_ATTN_EINVAL, "g=%d outside 0..6", g);
   if (cfg->batch < 1 || cfg->n_exact < 0) return fail(THIN_ATTN_EINVAL, "the cache needs batch >= 1 and n_exact >= 0");
+  if (cfg->q_begin != 0 || cfg->q_end != 0) return fail(THIN_ATTN_EINVAL, "the decode cache takes no query-row range");
   DeviceGuard dg(cfg->device);
   if (!dg.ok) return fail(THIN_ATTN_ECUDA, "cannot select device %d", cfg->device);
   thin_attn_cache_s* cc = new thin_attn_cache_s();
