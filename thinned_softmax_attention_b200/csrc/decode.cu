@@ -279,11 +279,18 @@ __device__ __forceinline__ void decode_combine(const AttnArgs& a, const float* p
     for (int d = threadIdx.x; d < D; d += blockDim.x) ((T*)a.v)[dst * D + d] = ((const T*)ap.new_v)[src * D + d];
   }
   // the chunks' (m, l) in one round of loads, one chunk per thread, then M, the chunks' factors
-  // 2^(m - M) and L through shared memory; o in rounds of sixteen chunks' loads
+  // 2^(m - M) and L through shared memory; o in rounds of sixteen chunks' loads, the first of
+  // them issued with (m, l)
   __shared__ float m_s[kDecodeMaxSplits], f_s[kDecodeMaxSplits], l_s[kDecodeMaxSplits];
   __shared__ float red[4];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* p = part + (size_t)bh * n_splits * (D + 2);
+  // this thread's first column of o for the first sixteen chunks, loaded in the same round as (m, l)
+  constexpr int RO = 16;
+  float x0[RO];
+#pragma unroll
+  for (int u = 0; u < RO; ++u)
+    x0[u] = (u < n_splits && (int)threadIdx.x < D) ? __ldcg(p + (size_t)u * (D + 2) + threadIdx.x) : 0.f;
   float mloc = -INFINITY;
   for (int s = threadIdx.x; s < n_splits; s += blockDim.x) {
     const float ms = __ldcg(p + (size_t)s * (D + 2) + D), ls = __ldcg(p + (size_t)s * (D + 2) + D + 1);
@@ -312,12 +319,17 @@ __device__ __forceinline__ void decode_combine(const AttnArgs& a, const float* p
   T* out = (T*)a.out + ((int64_t)b * a.T * a.H + h) * D;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float o = 0.f;
-    for (int s0 = 0; s0 < n_splits; s0 += 16) {
-      float x[16];
+    for (int s0 = 0; s0 < n_splits; s0 += RO) {
+      float x[RO];
+      if (s0 == 0 && d == (int)threadIdx.x) {
 #pragma unroll
-      for (int u = 0; u < 16; ++u) x[u] = s0 + u < n_splits ? __ldcg(p + (size_t)(s0 + u) * (D + 2) + d) : 0.f;
+        for (int u = 0; u < RO; ++u) x[u] = x0[u];
+      } else {
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
+        for (int u = 0; u < RO; ++u) x[u] = s0 + u < n_splits ? __ldcg(p + (size_t)(s0 + u) * (D + 2) + d) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < RO; ++u)
         if (s0 + u < n_splits) o = fmaf(x[u], f_s[s0 + u], o);
     }
     out[d] = from_f<T>(o * inv);
