@@ -81,3 +81,24 @@ def test_roofline_pair_count_is_what_the_oracle_attends(mode, T, S, g, n_e, bsz,
     flops, _, pairs = bench.attention_work(w, plan)
     assert pairs == seen[0] > 0
     assert flops == 2.0 * (w.E + w.D) * pairs
+
+
+@pytest.mark.parametrize("name", ["express32k", "express32k_a", "vit"])
+def test_attention_work_of_row_shards_adds_up(name):
+    """bench.attention_work over the query-row ranges of --shard seq: the shards' pairs and FLOPs sum
+    to the whole launch's, and each shard's q/out bytes are its rows'."""
+    import bench
+    import thinned_softmax_attention_b200 as T
+    import workloads as W
+    w = W.WORKLOADS[name]
+    plan = T.ThinAttention(w.B, w.T, w.T if w.causal else w.S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact,
+                           batch=w.batch).plan(w.mode, w.g)
+    full_f, full_b, full_p = bench.attention_work(w, plan)
+    fs, ps = 0.0, 0
+    for r in range(4):
+        rows = bench.Shard(w, 4, r, "seq").rows
+        f, b, p = bench.attention_work(w, plan, rows)
+        fs += f
+        ps += p
+        assert b < full_b
+    assert ps == full_p and fs == full_f
