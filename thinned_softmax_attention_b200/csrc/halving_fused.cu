@@ -271,17 +271,25 @@ __global__ void __launch_bounds__(kThreads, 1) halve_fused_kernel(const __grid_c
         // all loads of a chunk, then all stores (a bounded wait on cfix between)
         const int t = ew * 32 + lane, x = t & 7;
         int srow[8];
+        // the subsample offset U and first point of each instance of the unit, once per instance
+        // (a thread's rows span at most a few instances; U costs a Philox evaluation)
+        int cur_ii = -1;
+        uint32_t cur_u = 0;
+        uint64_t cur_g0 = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int R = (t >> 3) + 16 * j, ii = R / NP, p = R % NP;
           srow[j] = R;
           const int inst = u * Sh::IPU + ii;
           if (p < a.n && inst < a.n_inst) {
-            const HalveInst gi = a.inst[inst];
-            const uint32_t U = sub_offset(a, gi);
-            const uint64_t g0 = 2ull * gi.pair0;
-            const int64_t t0 = (int64_t)((g0 * (uint64_t)a.S_full + U) / (uint64_t)a.S_sub);
-            const int64_t tp = (int64_t)(((g0 + p) * (uint64_t)a.S_full + U) / (uint64_t)a.S_sub);
+            if (ii != cur_ii) {
+              const HalveInst gi = a.inst[inst];
+              cur_ii = ii;
+              cur_u = sub_offset(a, gi);
+              cur_g0 = 2ull * gi.pair0;
+            }
+            const int64_t t0 = (int64_t)((cur_g0 * (uint64_t)a.S_full + cur_u) / (uint64_t)a.S_sub);
+            const int64_t tp = (int64_t)(((cur_g0 + p) * (uint64_t)a.S_full + cur_u) / (uint64_t)a.S_sub);
             srow[j] = ii * NP + (int)(tp - t0);
           }
         }
