@@ -69,7 +69,8 @@ def peaks():
     if os.path.exists(path):
         d = json.load(open(path))
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
@@ -478,13 +479,24 @@ def halving_roofline(w, h, ph, pk):
     tab = []
     for st in sp["steps"]:
         sb = st["n_inst"] * 3 * st["n"] // 2 * (w.E + w.D) * es
+        kappa = st["n_inst"] * st["n"] * st["n"] // 2          # kernel evaluations of the instances' Grams
         sms = st["ms"] / max(1, sp["calls"])
         if sms == 0 and tab:
             tab[-1]["steps"].append({"n": st["n"], "n_inst": st["n_inst"]})
             tab[-1]["bytes"] += sb
+            tab[-1]["kappa"] += kappa
             continue
-        tab.append({"steps": [{"n": st["n"], "n_inst": st["n_inst"]}], "ms": round(sms, 4), "bytes": sb})
+        tab.append({"steps": [{"n": st["n"], "n_inst": st["n_inst"]}], "ms": round(sms, 4), "bytes": sb, "kappa": kappa})
+    # The three floors of a halving launch: its Gram on the tensor cores (2 (E+D) flops per kernel
+    # evaluation, at the burst bf16 peak), one exponential per evaluation on the MUFU pipes (16 per SM
+    # per clock at the maximum SM clock, 148 SMs) and its algorithmic HBM bytes; the largest is the
+    # launch's bound (HBM at every workload here).
+    mufu_per_s = 148 * 16 * pk.get("sm_max_mhz", 1965.0) * 1e6
     for t in tab:
+        terms = {"tensor_ms": t["kappa"] * 2 * (w.E + w.D) / (pk["bf16_tflops"] * 1e12) * 1e3,
+                 "mufu_ms": t["kappa"] / mufu_per_s * 1e3,
+                 "hbm_ms": t["bytes"] / (pk["hbm_gbs"] * 1e9) * 1e3}
+        t["floors_ms"] = {k: round(v, 5) for k, v in terms.items()}
         t["frac"] = round(t["bytes"] / (t["ms"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4) if t["ms"] > 0 else None
         t["kernel"] = (f"halving step n={t['steps'][0]['n']} x {t['steps'][0]['n_inst']} instances" if len(t["steps"]) == 1
                        else "persistent halving launch of " + " + ".join(f"{x['n_inst']} x {x['n']}" for x in t["steps"]))
@@ -493,7 +505,9 @@ def halving_roofline(w, h, ph, pk):
     top = max(tab, key=lambda t: t["ms"]) if tab else None
     if not top or top["ms"] <= 0:
         return None
-    return {"bound": "hbm", "achieved": round(top["bytes"] / (top["ms"] * 1e-3) / 1e9, 1),
+    floors = top["floors_ms"]
+    return {"bound": max(floors, key=floors.get)[:-3], "floors_ms": floors,
+            "achieved": round(top["bytes"] / (top["ms"] * 1e-3) / 1e9, 1),
             "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": top["frac"], "kernel": top["kernel"],
             "algorithmic_bytes_per_launch": top["bytes"], "avg_launch_ms": top["ms"],
             "traffic": (None if w.name != "express32k" or w.H != 32 else

@@ -102,3 +102,25 @@ def test_attention_work_of_row_shards_adds_up(name):
         ps += p
         assert b < full_b
     assert ps == full_p and fs == full_f
+
+
+def test_halving_floors_put_hbm_on_top_at_express32k():
+    """The halving launches' three floors (Gram on the tensor cores, one exponential per kernel
+    evaluation on MUFU, algorithmic HBM bytes): at Express 32K's level-1 step HBM is the largest, so
+    the reported fraction is against the binding one."""
+    import bench
+    import workloads as W
+
+    class FakeHandle:
+        def profile_steps(self):
+            return {"calls": 1, "steps": [{"n": 64, "n_inst": 15872, "ms": 0.195}, {"n": 128, "n_inst": 3968, "ms": 0.183},
+                                          {"n": 256, "n_inst": 992, "ms": 0.297}, {"n": 512, "n_inst": 224, "ms": 0.0}]}
+
+    w = W.WORKLOADS["express32k"]
+    r = bench.halving_roofline(w, FakeHandle(), {"thin_ms": 0.6, "merge_ms": 0.08, "calls": 1}, bench.peaks())
+    assert r["bound"] == "hbm"
+    for t in r["launches"]:
+        f = t["floors_ms"]
+        assert f["hbm_ms"] > f["tensor_ms"] and f["hbm_ms"] > f["mufu_ms"]
+    lv1 = r["launches"][0]["floors_ms"]
+    assert abs(lv1["hbm_ms"] - 780140544 / 6553e9 * 1e3) < 1e-4
