@@ -545,6 +545,24 @@ def timed_steps(step, steps, stream, flush):
     return sum(a.elapsed_time(b) for a, b in evs) / steps
 
 
+def sdpa_ms(w, q, k, v, stream):
+    """Exact attention at the same shape (PyTorch SDPA, the tensors' dtype), CUDA events, 3 runs."""
+    try:
+        qt, kt, vt = (x.transpose(1, 2) for x in (q, k, v))
+        F = torch.nn.functional.scaled_dot_product_attention
+        for _ in range(2):
+            F(qt, kt, vt, is_causal=w.causal)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(3):
+            F(qt, kt, vt, is_causal=w.causal)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        return round(s0.elapsed_time(s1) / 3, 4)
+    except Exception as ex:  # report, do not fail the bench
+        return f"unavailable: {type(ex).__name__}"
+
+
 def measure_workload(TA, name, dev, steps, warmup):
     """One workload on this GPU alone: ms per layer (CUDA events, inputs resident in HBM), phases,
     the attention and halving rooflines and the approximation error against exact attention."""
@@ -583,6 +601,7 @@ def measure_workload(TA, name, dev, steps, warmup):
            "halving_roofline": halving_roofline(w, h, ph, pk),
            "gpu_launches_per_step": plan["kernel_launches"]}
     rec["approx_error"] = exact_reference_error(w, qc, kc, vc, out)
+    rec["exact_sdpa_ms"] = sdpa_ms(w, q, k, v, stream)
     h.close()
     del q, k, v, out, flush
     torch.cuda.empty_cache()
@@ -702,20 +721,7 @@ def main():
 
     sdpa = None
     if not a.no_sdpa and rank == 0:
-        try:
-            qt, kt, vt = (x.transpose(1, 2) for x in (q, k, v))
-            F = torch.nn.functional.scaled_dot_product_attention
-            for _ in range(2):
-                F(qt, kt, vt, is_causal=w.causal)
-            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s0.record(stream)
-            for _ in range(3):
-                F(qt, kt, vt, is_causal=w.causal)
-            s1.record(stream)
-            torch.cuda.synchronize()
-            sdpa = round(s0.elapsed_time(s1) / 3, 4)
-        except Exception as ex:  # report, do not fail the bench
-            sdpa = f"unavailable: {type(ex).__name__}"
+        sdpa = sdpa_ms(w, q, k, v, stream)
 
     approx = None
     per_workload = None
