@@ -11,7 +11,9 @@ parts of one problem whose (b,h) slices are independent -- `--shard batch`
 (default, weak scaling): rank r holds batch rows [rB, (r+1)B) of a problem with
 N*B rows; `--shard heads` (strong scaling): rank r holds H/N heads of the
 workload; `--shard seq` (strong scaling): rank r attends query rows
-[r T/N, (r+1) T/N) (128-aligned) of every (b,h), each rank thinning all keys.
+[r T/N, (r+1) T/N) (128-aligned) of every (b,h), each rank thinning all keys;
+`--shard seqx`: the same ranges, each rank thinning only its own Express batches,
+then one all-gather of the batch coresets (NCCL) before the merges and attention.
 No collective on the data path; the random decisions are keyed on the whole
 problem's (b,h); step time is the max over ranks of CUDA-event time.
 
@@ -49,7 +51,7 @@ def args_():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="thin", choices=["thin", "reference"])
     p.add_argument("--workload", default="express32k", choices=sorted(W.WORKLOADS))
-    p.add_argument("--shard", default="batch", choices=["batch", "heads", "seq"],
+    p.add_argument("--shard", default="batch", choices=["batch", "heads", "seq", "seqx"],
                    help="N>1: batch rows of one larger problem per rank (weak) or the heads of one problem (strong)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -283,8 +285,12 @@ class Shard:
     what a single run of the whole problem computes for its rows; no data crosses between ranks."""
 
     def __init__(self, w, world, rank, mode="batch"):
-        if mode not in ("batch", "heads", "seq"):
+        if mode not in ("batch", "heads", "seq", "seqx"):
             raise ValueError(mode)
+        if mode == "seqx" and w.mode != 1:
+            raise ValueError("--shard seqx splits Express batch thinning: causal workloads with the batch cache only")
+        self.split = mode == "seqx"
+        mode = "seq" if mode == "seqx" else mode
         if mode == "heads" and w.H % world:
             raise ValueError(f"--shard heads needs H={w.H} divisible by the {world} ranks")
         self.mode, self.world, self.rank = mode, world, rank
@@ -297,7 +303,7 @@ class Shard:
         self.global_batch = world * w.B if mode == "batch" else w.B
         self.whole_tokens = self.global_batch * w.H * w.T
         self.scaling = "weak" if mode == "batch" else "strong"
-        self.parallelism = {"batch": "dp", "heads": "hp", "seq": "sp"}[mode] + str(world)
+        self.parallelism = {"batch": "dp", "heads": "hp", "seq": "sp"}[mode] + ("x" if self.split else "") + str(world)
         self.q_range = (0, 0)
         if mode == "seq":
             # equal 128-aligned slices of the query rows, the last one ending at T
@@ -631,7 +637,7 @@ def main():
     q, k, v = (x.to(dev) for x in (qc, kc, vc))
     S = w.T if w.causal else w.S
     h = TA.ThinAttention(w.B, w.T, S, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch,
-                         device=local, shard=shard.abi, q_range=shard.q_range)
+                         device=local, shard=shard.abi, q_range=shard.q_range, thin_split=shard.split)
     plan = h.plan(w.mode, w.g)
     h.reserve(w.mode, w.g)
     out = torch.empty(w.B, w.T, w.H, w.D, dtype=w.torch_dtype, device=dev)
@@ -640,7 +646,14 @@ def main():
     flush = torch.empty(int(2 * L2_BYTES) // 4, dtype=torch.float32, device=dev) if in_bytes < L2_BYTES else None
 
     def step():
-        h.forward(q, k, v, causal=w.mode, g=w.g, seed=w.seed, out=out)
+        if shard.split:
+            # own batches, the coreset exchange (one all-gather over the ranks), merges + attention
+            h.forward_phase(q, k, v, phase=1, g=w.g, seed=w.seed)
+            if dist:
+                TA.exchange_batch_coresets(h, w.g, dist)
+            h.forward_phase(q, k, v, phase=2, g=w.g, seed=w.seed, out=out)
+        else:
+            h.forward(q, k, v, causal=w.mode, g=w.g, seed=w.seed, out=out)
 
     for _ in range(max(3, a.warmup)):
         step()
@@ -663,13 +676,19 @@ def main():
     value = shard.whole_tokens / (ms * 1e-3)
 
     pk = peaks()
-    attn_ms = ph["attn_ms"] / max(1, ph["calls"])
-    roof = attention_roofline(w, plan, attn_ms, pk, shard.rows)
-    roof["traffic"] = attention_traffic(w) if shard.rows is None else None
-    halving_roof = halving_roofline(w, h, ph, pk)
-    phases = {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
-              "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4),
-              "attn_ms": round(attn_ms, 4)}
+    if shard.split:
+        # a phased forward records no per-phase events: the step time is the measurement
+        roof = {"unavailable": "per-phase times are not recorded for split-thinning forwards"}
+        halving_roof = None
+        phases = None
+    else:
+        attn_ms = ph["attn_ms"] / max(1, ph["calls"])
+        roof = attention_roofline(w, plan, attn_ms, pk, shard.rows)
+        roof["traffic"] = attention_traffic(w) if shard.rows is None else None
+        halving_roof = halving_roofline(w, h, ph, pk)
+        phases = {"thin_ms": round(ph["thin_ms"] / max(1, ph["calls"]), 4),
+                  "merge_ms": round(ph["merge_ms"] / max(1, ph["calls"]), 4),
+                  "attn_ms": round(attn_ms, 4)}
 
     e2e = None
     if not a.no_e2e and shard.rows is not None:

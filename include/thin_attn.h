@@ -93,6 +93,15 @@ typedef struct {
    * or T.  thin_attn_forward_host and the decode cache take no range (EUNSUPPORTED / EINVAL). */
   int q_begin;
   int q_end;
+  /* Express sequence shards with the thinning split too (causal = 1 only): with thin_split = 1 the
+   * handle thins only the batches it owns -- batch k is owned by the range [q_begin, q_end) that
+   * holds its last token ("Express Language Modeling", The EXPRESS Meta-Procedure: batches are
+   * thinned independently) -- and the other batches' coresets come from the ranks that own them.
+   * A forward then runs in two calls of thin_attn_forward_phase: phase 1 thins the owned batches;
+   * the caller exchanges the batch coresets (thin_attn_nodes_export on every rank, an all-gather,
+   * thin_attn_nodes_import of the others' batches); phase 2 runs every HALVE merge and the
+   * attention of the range.  Outputs equal the whole run's bit for bit.  0: thin every batch. */
+  int thin_split;
 } thin_attn_config;
 
 /* Sizes of one (causal, g) plan. */
@@ -134,6 +143,31 @@ THIN_ATTN_API thin_attn_status thin_attn_destroy(thin_attn_t h);
 
 /* Sizes of the (causal, g) plan; 0 <= g <= 6. */
 THIN_ATTN_API thin_attn_status thin_attn_plan(thin_attn_t h, int causal, int g, thin_attn_plan_info* info);
+
+/* One phase of a forward of a thin_split handle (see thin_attn_config::thin_split): phase 1 thins
+ * the owned batches into their level-0 nodes; phase 2 runs the merges and the attention of the
+ * query-row range and writes out, lse_opt, coreset_idx_opt (every node; valid once the other
+ * ranks' batches have been imported) and trace_opt (this handle's halvings).  Arguments as for
+ * thin_attn_forward.  EINVAL unless the handle has thin_split = 1, causal = 1 and phase is 1 or 2;
+ * thin_attn_forward on such a handle is EINVAL. */
+THIN_ATTN_API thin_attn_status thin_attn_forward_phase(thin_attn_t h, const void* q, const void* k, const void* v,
+                                                       void* out, int causal, int g, uint64_t seed, float* lse_opt,
+                                                       int32_t* coreset_idx_opt, uint32_t* trace_opt, int phase,
+                                                       void* stream);
+
+/* The batch coresets of a causal (Express, causal = 1) plan, for the exchange between thin_split
+ * ranks.  *own_begin, *own_end: the batches this handle thins; *n_batches: all completed batches;
+ * *bytes_per_batch: bytes of one batch's exchange block -- its level-0 node of every (b,h): keys
+ * (B*H*c*E elements), values (B*H*c*D elements), then token indices (B*H*c int32), each (b,h)-major. */
+THIN_ATTN_API thin_attn_status thin_attn_nodes_layout(thin_attn_t h, int causal, int g, int* own_begin, int* own_end,
+                                                      int* n_batches, uint64_t* bytes_per_batch);
+/* Copy the owned batches' blocks, in batch order, into dst (device memory, (own_end - own_begin) *
+ * bytes_per_batch bytes, 16-byte aligned), on stream after the phase-1 work queued there. */
+THIN_ATTN_API thin_attn_status thin_attn_nodes_export(thin_attn_t h, int causal, int g, void* dst, void* stream);
+/* Write the blocks of batches [batch_begin, batch_end) from src (device memory, in batch order) into
+ * this handle's level-0 nodes, on stream, before phase 2.  EINVAL for batches outside [0, n_batches). */
+THIN_ATTN_API thin_attn_status thin_attn_nodes_import(thin_attn_t h, int causal, int g, const void* src,
+                                                      int batch_begin, int batch_end, void* stream);
 
 /* Allocate the workspace of the (causal, g) plan now (so the first forward allocates nothing). */
 THIN_ATTN_API thin_attn_status thin_attn_reserve(thin_attn_t h, int causal, int g);

@@ -315,3 +315,32 @@ def test_query_range_is_refused_by_the_host_path_and_the_cache():
     cfg = T.Config(T.BF16, 1, 64, 64, 1, 128, 128, 0.0, 16, 16, 0, 0, 0, 0, 0, 0, 64)
     c = ctypes.c_void_p()
     assert T.lib().thin_attn_cache_create(ctypes.byref(c), ctypes.byref(cfg), 2, ctypes.c_uint64(1)) != 0
+
+
+@pytest.mark.parametrize("T_,ne,bsz,cuts", [(8192, 1024, 1024, [0, 2048, 4224, 8192]),
+                                            (3000, 200, 300, [0, 128, 1152, 2048, 3000])])
+def test_split_thinning_ranges_own_every_batch_once(T_, ne, bsz, cuts):
+    """thin_split: batch k belongs to the range holding its last token; the ranges' batches partition
+    the completed batches, and each plan holds its batches' halvings plus every merge."""
+    dt = W.WORKLOADS["express32k"].torch_dtype
+    full = T.ThinAttention(1, T_, T_, 2, 128, 128, dt, n_exact=ne, batch=bsz)
+    n_full = full.plan(True, 2)["n_halvings"]
+    hs = [T.ThinAttention(1, T_, T_, 2, 128, 128, dt, n_exact=ne, batch=bsz, q_range=r, thin_split=True)
+          for r in zip(cuts[:-1], cuts[1:])]
+    lays = [h.nodes_layout(2) for h in hs]
+    n_b = (T_ - ne) // bsz
+    assert [lay[2] for lay in lays] == [n_b] * len(hs)
+    assert lays[0][0] == 0 and lays[-1][1] == n_b and all(a[1] == b[0] for a, b in zip(lays[:-1], lays[1:]))
+    for (q0, q1), (k0, k1, _, _) in zip(zip(cuts[:-1], cuts[1:]), lays):
+        assert all(q0 <= ne + (kk + 1) * bsz - 1 < q1 for kk in range(k0, k1))
+    # a plan holds owned x P batch halvings plus every merge's M: solve P, M from two plans, then the
+    # plans together hold the whole run's halvings with the merges counted once per plan
+    counts = [h.plan(True, 2)["n_halvings"] for h in hs]
+    owned = [k1 - k0 for k0, k1, _, _ in lays]
+    i, j = min(range(len(hs)), key=owned.__getitem__), max(range(len(hs)), key=owned.__getitem__)
+    P = (counts[j] - counts[i]) // (owned[j] - owned[i])
+    M = counts[i] - owned[i] * P
+    assert all(c == o * P + M for c, o in zip(counts, owned))
+    assert sum(counts) - (len(hs) - 1) * M == n_full
+    with pytest.raises(T.ThinAttnError, match="EUNSUPPORTED"):
+        T.ThinAttention(1, T_, T_, 2, 128, 128, dt, n_exact=ne, batch=bsz, q_range=(0, 1024), thin_split=True).plan(2, 2)

@@ -152,3 +152,49 @@ def test_query_row_shards_equal_the_whole_problem(name, form, monkeypatch):
         assert bool((out[:, :q0] == 7.0).all()) and bool((out[:, q1:] == 7.0).all())
         assert bool((lse[:, :, :q0] == -3.0).all()) and bool((lse[:, :, q1:] == -3.0).all())
         assert torch.equal(r["coreset"], whole["coreset"])
+
+
+@pytest.mark.parametrize("name", ["express", "express_ragged"])
+def test_split_thinning_sequence_shards_equal_the_whole_problem(name):
+    """Sequence shards that split the thinning too (thin_split): each emulated rank thins only the
+    batches whose last token lies in its range (phase 1), the batch coresets are exchanged between the
+    ranks (export, import), and each rank runs every merge and its rows' attention (phase 2).  Every
+    rank's rows, the full node coresets and every halving decision equal the whole run's bit for
+    bit; the ragged shape gives one range that owns no batch."""
+    w, cuts = SEQ_CASES[name]
+    q, k, v = (x.to(DEV) for x in W.make_qkv(w))
+    whole = _run(w, q, k, v)
+    ranges = list(zip(cuts[:-1], cuts[1:]))
+    hs = [TA.ThinAttention(w.B, w.T, w.T, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch, q_range=r,
+                           thin_split=True) for r in ranges]
+    owned = [h.nodes_layout(w.g)[:2] for h in hs]
+    n_b = hs[0].nodes_layout(w.g)[2]
+    assert owned[0][0] == 0 and owned[-1][1] == n_b and n_b > 0        # the ranges' batches partition them
+    assert all(a[1] == b[0] for a, b in zip(owned[:-1], owned[1:]))
+    traces1 = [h.forward_phase(q, k, v, phase=1, g=w.g, seed=w.seed, return_trace=True)["trace"] for h in hs]
+    TA.exchange_batch_coresets(hs, w.g)
+    for h, (q0, q1), tr1 in zip(hs, ranges, traces1):
+        out = torch.full((w.B, w.T, w.H, w.D), 7.0, dtype=w.torch_dtype, device=DEV)
+        lse = torch.full((w.B, w.H, w.T), -3.0, dtype=torch.float32, device=DEV)
+        r = h.forward_phase(q, k, v, phase=2, g=w.g, seed=w.seed, out=out, lse=lse, return_coreset=True,
+                            return_trace=True)
+        torch.cuda.synchronize()
+        h.check()
+        assert torch.equal(out[:, q0:q1], whole["out"][:, q0:q1])
+        assert torch.equal(lse[:, :, q0:q1], whole["lse"][:, :, q0:q1])
+        assert bool((out[:, :q0] == 7.0).all()) and bool((out[:, q1:] == 7.0).all())
+        assert torch.equal(r["coreset"], whole["coreset"])
+        # phase 1 recorded the batches' decisions, phase 2 the merges' (disjoint words of the trace)
+        mine = TA.decode_trace(r["trace"] | tr1, h.trace_layout(w.mode, w.g))
+        assert len(mine) > 0 or h.nodes_layout(w.g)[0] == h.nodes_layout(w.g)[1]
+        for key, bits in mine.items():
+            np.testing.assert_array_equal(bits, whole["decisions"][key])
+
+
+def test_split_thinning_refuses_the_one_call_forward():
+    w, _ = SEQ_CASES["express"]
+    h = TA.ThinAttention(w.B, w.T, w.T, w.H, w.E, w.D, w.torch_dtype, n_exact=w.n_exact, batch=w.batch, q_range=(0, 1024),
+                         thin_split=True)
+    x = torch.zeros(w.B, w.T, w.H, w.E, dtype=w.torch_dtype, device=DEV)
+    with pytest.raises(TA.ThinAttnError, match="EINVAL"):
+        h.forward(x, x, x, causal=True, g=w.g, seed=w.seed)

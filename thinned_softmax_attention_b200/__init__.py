@@ -38,7 +38,7 @@ class Config(ctypes.Structure):
                 ("H", ctypes.c_int), ("E", ctypes.c_int), ("D", ctypes.c_int), ("scale", ctypes.c_float),
                 ("n_exact", ctypes.c_int), ("batch", ctypes.c_int), ("device", ctypes.c_int),
                 ("b0", ctypes.c_int), ("h0", ctypes.c_int), ("H_total", ctypes.c_int), ("qk_fp8", ctypes.c_int),
-                ("q_begin", ctypes.c_int), ("q_end", ctypes.c_int)]
+                ("q_begin", ctypes.c_int), ("q_end", ctypes.c_int), ("thin_split", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -59,7 +59,8 @@ EXPORTS = ("thin_attn_version", "thin_attn_last_error", "thin_attn_create", "thi
            "thin_attn_forward_host", "thin_attn_check", "thin_attn_profile", "thin_attn_profile_read",
            "thin_attn_profile_steps",
            "thin_attn_cache_create", "thin_attn_cache_destroy", "thin_attn_cache_length", "thin_attn_cache_decode",
-           "thin_attn_cache_nodes", "thin_attn_cache_check", "thin_attn_sched_layout", "thin_attn_cache_decode_n")
+           "thin_attn_cache_nodes", "thin_attn_cache_check", "thin_attn_sched_layout", "thin_attn_cache_decode_n",
+           "thin_attn_forward_phase", "thin_attn_nodes_layout", "thin_attn_nodes_export", "thin_attn_nodes_import")
 
 
 def lib() -> ctypes.CDLL:
@@ -132,15 +133,20 @@ class ThinAttention:
     end may be T) of every (b,h); the thinning runs over all keys, so those rows equal the whole
     run's and the other rows of ``out`` and ``lse`` are left as they were (sequence-parallel
     shards of one long sequence, one per GPU, with no communication).
+
+    ``thin_split=True`` (Express, with ``q_range``): the handle thins only the batches whose last
+    token lies in its range; a forward is ``forward_phase(..., phase=1)``, an exchange of the batch
+    coresets (``nodes_export`` on every rank, an all-gather, ``nodes_import`` of the others'), then
+    ``forward_phase(..., phase=2)`` (see ``exchange_batch_coresets``).
     """
 
     def __init__(self, B: int, T: int, S: int, H: int, E: int, D: int, dtype: torch.dtype,
                  scale: Optional[float] = None, n_exact: int = 0, batch: int = 0, device: int = 0,
                  shard: Tuple[int, int, int] = (0, 0, 0), qk_fp8: bool = False,
-                 q_range: Tuple[int, int] = (0, 0)):
+                 q_range: Tuple[int, int] = (0, 0), thin_split: bool = False):
         self.cfg = Config(FP32 if dtype == torch.float32 else BF16, B, T, S, H, E, D,
                           0.0 if scale is None else float(scale), n_exact, batch, device, *shard, int(qk_fp8),
-                          *q_range)
+                          *q_range, int(thin_split))
         self.dtype = dtype
         self.device = torch.device("cuda", device)
         self._h = ctypes.c_void_p()
@@ -226,6 +232,61 @@ class ThinAttention:
         if return_trace:
             res["trace"] = trace
         return res
+
+    def forward_phase(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, phase: int, g: int = 2, seed: int = 0,
+                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      return_coreset: bool = False, return_trace: bool = False):
+        """One phase of a thin_split handle's Express forward: 1 thins the owned batches, 2 runs the
+        merges and the attention of the query-row range (after the batch coresets are exchanged)."""
+        c = self.cfg
+        for name, t, shape in (("q", q, (c.B, c.T, c.H, c.E)), ("k", k, (c.B, c.T, c.H, c.E)),
+                               ("v", v, (c.B, c.T, c.H, c.D))):
+            if tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous() or t.device != self.device:
+                raise ValueError(f"{name}: expected contiguous {self.dtype} {shape} on {self.device}")
+        if out is None:
+            out = torch.empty(c.B, c.T, c.H, c.D, dtype=self.dtype, device=self.device)
+        info = self.plan(True, g)
+        cidx = (torch.empty(max(1, info["coreset_idx_elems"]), dtype=torch.int32, device=self.device)
+                if return_coreset else None)
+        trace = (torch.zeros(max(1, info["trace_words"]), dtype=torch.int32, device=self.device)
+                 if return_trace else None)
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_forward_phase(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), 1, g,
+                                             ctypes.c_uint64(seed & (2 ** 64 - 1)), _ptr(lse), _ptr(cidx), _ptr(trace),
+                                             int(phase), ctypes.c_void_p(stream)))
+        res = {"out": out}
+        if lse is not None:
+            res["lse"] = lse
+        if return_coreset:
+            n = info["coreset_idx_elems"]
+            res["coreset"] = cidx[:n].view(c.B, c.H, info["n_nodes"], info["coreset_rows"])
+        if return_trace:
+            res["trace"] = trace
+        return res
+
+    def nodes_layout(self, g: int = 2):
+        """(own_begin, own_end, n_batches, bytes_per_batch) of the Express batch coresets."""
+        k0, k1, nb, bpb = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_uint64()
+        _check(lib().thin_attn_nodes_layout(self._h, 1, g, ctypes.byref(k0), ctypes.byref(k1), ctypes.byref(nb),
+                                            ctypes.byref(bpb)))
+        return k0.value, k1.value, nb.value, bpb.value
+
+    def nodes_export(self, dst: torch.Tensor, g: int = 2):
+        """The owned batches' coreset blocks into ``dst`` (uint8 on this device)."""
+        k0, k1, _, bpb = self.nodes_layout(g)
+        if dst.device != self.device or dst.dtype != torch.uint8 or dst.numel() < (k1 - k0) * bpb:
+            raise ValueError("dst: uint8 on the handle's device, (own_end - own_begin) * bytes_per_batch bytes")
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_nodes_export(self._h, 1, g, _ptr(dst), ctypes.c_void_p(stream)))
+
+    def nodes_import(self, src: torch.Tensor, batch_begin: int, batch_end: int, g: int = 2):
+        """Write batches [batch_begin, batch_end)'s coreset blocks from ``src`` into this handle."""
+        _, _, _, bpb = self.nodes_layout(g)
+        if src.device != self.device or src.dtype != torch.uint8 or src.numel() < (batch_end - batch_begin) * bpb:
+            raise ValueError("src: uint8 on the handle's device, one block per batch")
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        _check(lib().thin_attn_nodes_import(self._h, 1, g, _ptr(src), int(batch_begin), int(batch_end),
+                                            ctypes.c_void_p(stream)))
 
     def forward_host(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                      causal: bool = False, g: int = 2, seed: int = 0, lse: Optional[torch.Tensor] = None):
@@ -399,4 +460,42 @@ class ThinformerAttention:
 
 
 __all__ = ["ThinAttention", "ThinAttentionCache", "ThinAttnError", "ThinformerAttention", "thinformer_attention",
-           "decode_trace", "lib", "LIB_PATH", "EXPORTS"]
+           "decode_trace", "exchange_batch_coresets", "lib", "LIB_PATH", "EXPORTS"]
+
+
+def exchange_batch_coresets(h: "ThinAttention", g: int = 2, dist=None):
+    """Between phase 1 and phase 2 of thin_split handles: every rank's owned batch coresets reach
+    every other rank.  With ``dist`` (torch.distributed, one handle per rank): one all-gather of the
+    padded blocks over the process group.  ``h`` may also be a list of handles on this device (ranks
+    emulated in one process), whose blocks are copied directly."""
+    if isinstance(h, (list, tuple)):
+        lays = [x.nodes_layout(g) for x in h]
+        bufs = []
+        for x, (k0, k1, _, bpb) in zip(h, lays):
+            buf = torch.empty(max(1, (k1 - k0) * bpb), dtype=torch.uint8, device=x.device)
+            if k1 > k0:
+                x.nodes_export(buf, g)
+            bufs.append(buf)
+        for i, x in enumerate(h):
+            for j, (k0, k1, _, bpb) in enumerate(lays):
+                if j != i and k1 > k0:
+                    x.nodes_import(bufs[j].to(x.device), k0, k1, g)
+        return
+    k0, k1, nb, bpb = h.nodes_layout(g)
+    world = dist.get_world_size()
+    rng = torch.tensor([k0, k1], dtype=torch.int64, device=h.device)
+    ranges = [torch.empty_like(rng) for _ in range(world)]
+    dist.all_gather(ranges, rng)
+    ranges = [tuple(int(x) for x in r.tolist()) for r in ranges]
+    kmax = max(b - a for a, b in ranges)
+    if kmax == 0:
+        return
+    send = torch.zeros(kmax * bpb, dtype=torch.uint8, device=h.device)
+    if k1 > k0:
+        h.nodes_export(send, g)
+    recv = [torch.empty_like(send) for _ in range(world)]
+    dist.all_gather(recv, send)
+    me = dist.get_rank()
+    for r, (a, b) in enumerate(ranges):
+        if r != me and b > a:
+            h.nodes_import(recv[r], a, b, g)

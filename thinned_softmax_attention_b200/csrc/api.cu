@@ -152,6 +152,7 @@ struct Plan {
   int causal = 0, g = 0;
   Sizes sz{};
   int n_b = 0, n_slots = 0, c = 0;
+  int own_k0 = 0, own_k1 = 0;    // causal: the batches this handle thins (all unless thin_split)
   std::vector<int> level_base;   // causal: first slot of each node level
   // causal == 2 (Express, page-literal cache): batches, slot of H_i, slot of thinned batch (i, s)
   std::vector<ABatch> a_batches;
@@ -508,6 +509,7 @@ void build_sched(const thin_attn_config& cf, Plan* p, int n_sms) {
   p->sched_items.clear();
   p->sched_pred_off.clear();
   p->sched_preds.clear();
+  if (cf.thin_split) return;   // the batch steps and the merges run in different phases
   const int ns = (int)p->steps.size(), cap = halving_sched_max_steps();
   int best0 = 0, best1 = 0;
   for (int i = 0; i < ns;) {
@@ -751,6 +753,21 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
   } else {
     const int T = cf.T, ne = std::min(cf.n_exact, T), bsz = cf.batch;
     p->n_b = T > ne ? (T - ne) / bsz : 0;
+    p->own_k0 = 0;
+    p->own_k1 = p->n_b;
+    if (cf.thin_split) {
+      // batch k belongs to the query-row range holding its last token ne + (k + 1) b - 1
+      // (the batches whose last token lies before q_begin, and before q_end: a range owning no batch
+      // gets an empty range in place)
+      const int qb = cf.q_begin, qe = (cf.q_begin == 0 && cf.q_end == 0) ? T : cf.q_end;
+      auto before = [&](int64_t t) {
+        int n = 0;
+        while (n < p->n_b && (int64_t)ne + (int64_t)(n + 1) * bsz - 1 < t) ++n;
+        return n;
+      };
+      p->own_k0 = before(qb);
+      p->own_k1 = before(qe);
+    }
     p->sz = compress_sizes(bsz, g);
     p->c = p->sz.C;
     for (int lv = 0; (p->n_b >> (2 * lv)) > 0; ++lv) {
@@ -764,7 +781,7 @@ thin_attn_status build_plan(thin_attn_s* h, int causal, int g, Plan** out) {
     if (p->n_b > 0) {
       std::vector<RunDesc> runs;
       for (int bh = 0; bh < BH; ++bh)
-        for (int k = 0; k < p->n_b; ++k) {
+        for (int k = p->own_k0; k < p->own_k1; ++k) {
           const int b = bh / cf.H;
           const uint32_t tok0 = (uint32_t)(ne + k * bsz);
           runs.push_back({(uint32_t)bh, (int64_t)b * T + tok0, tok0, k,
@@ -994,6 +1011,8 @@ thin_attn_status check_cfg(const thin_attn_config* c) {
       return fail(THIN_ATTN_EINVAL, "query rows [%d, %d): both ends must be multiples of 128 (the end may be T)",
                   c->q_begin, c->q_end);
   }
+  if (c->thin_split != 0 && c->thin_split != 1) return fail(THIN_ATTN_EINVAL, "thin_split must be 0 or 1");
+  if (c->thin_split && c->qk_fp8) return fail(THIN_ATTN_EUNSUPPORTED, "thin_split takes no qk_fp8");
   if (c->qk_fp8 != 0 && c->qk_fp8 != 1) return fail(THIN_ATTN_EINVAL, "qk_fp8 must be 0 or 1");
   if (c->qk_fp8 && (c->dtype != THIN_ATTN_BF16 || c->E != 128 || c->D > 128 || c->D % 64 || !qk_fp8_supported(c->H, c->E)))
     return fail(THIN_ATTN_EUNSUPPORTED, "qk_fp8 needs bf16 with E = 128, D = 64 or 128 and H <= 128 (E=%d D=%d H=%d)", c->E,
@@ -1011,6 +1030,8 @@ thin_attn_status get_plan(thin_attn_s* h, int causal, int g, Plan** out) {
     return fail(THIN_ATTN_EINVAL, "causal attention needs batch >= 1 and n_exact >= 0");
   if (causal == 2 && c.n_exact < 2)
     return fail(THIN_ATTN_EINVAL, "Express with the page-literal cache needs n_exact (the cache size n_out) >= 2");
+  if (c.thin_split && causal != 1)
+    return fail(THIN_ATTN_EUNSUPPORTED, "thin_split runs Express (causal = 1) with its batch cache only");
   auto key = std::make_pair(causal, g);
   auto it = h->plans.find(key);
   if (it != h->plans.end()) {
@@ -1069,8 +1090,12 @@ int step_launches(const thin_attn_config& cf, const Plan* p, const StepPlan& sp)
   return tc && halving_fused_supported(a) ? 1 : 3;
 }
 
+// phase 0: the whole forward.  Sequence shards with split thinning (thin_split) run it in two calls:
+// phase 1 the batch-thinning steps only, phase 2 the merge steps, the attention and the coreset
+// output (the other ranks' batch coresets imported in between).
 thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void* k, const void* v, void* out,
-                             uint64_t seed, float* lse, int32_t* cidx, uint32_t* trace, cudaStream_t st) {
+                             uint64_t seed, float* lse, int32_t* cidx, uint32_t* trace, cudaStream_t st,
+                             int phase = 0) {
   const thin_attn_config& cf = h->cfg;
   const bool use_tc_gram = std::getenv("THIN_ATTN_SIMT_GRAM") == nullptr;
   const bool use_tc_attn = !p->tc.tiles.empty() && tensor_maps_available() && std::getenv("THIN_ATTN_SIMT_ATTN") == nullptr;
@@ -1080,7 +1105,7 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   // By default one attention launch follows all halving steps on the caller's stream: the waves
   // save ~3 % of an Express step but share SMs with the halving kernels.
   const bool fp8 = cf.qk_fp8 && use_tc_attn;
-  const bool side = tab.waves.size() > 1 && std::getenv("THIN_ATTN_OVERLAP") != nullptr && !fp8;
+  const bool side = phase == 0 && tab.waves.size() > 1 && std::getenv("THIN_ATTN_OVERLAP") != nullptr && !fp8;
   const std::vector<AttnWave> one_wave = {{0, (int)tab.tiles.size(), (int)p->steps.size() - 1}};
   const std::vector<AttnWave>& waves = side ? tab.waves : one_wave;
   cudaStream_t sa = st;
@@ -1114,7 +1139,7 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   // halving step on the halving stream
   std::vector<cudaEvent_t> ev;
   const size_t ev_steps = 4 + 2 * waves.size();
-  if (h->prof_on) {
+  if (h->prof_on && phase == 0) {
     const size_t need = ev_steps + p->steps.size();
     if (!h->prof_free.empty() && h->prof_free.back().size() >= need) {
       ev = h->prof_free.back();
@@ -1163,6 +1188,7 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   }
   size_t next_wave = 0, dep_i = 0;
   auto launch_waves_after = [&](int step) -> thin_attn_status {
+    if (phase == 1) return THIN_ATTN_OK;   // no attention in the thinning phase
     while (next_wave < waves.size() && waves[next_wave].after <= step) {
       const AttnWave& w = waves[next_wave];
       if (side) {
@@ -1192,6 +1218,7 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
   std::vector<StepArgs> group;
   for (size_t si = 0; si < p->steps.size(); ++si) {
     const StepPlan& sp = p->steps[si];
+    if ((phase == 1 && sp.phase != 0) || (phase == 2 && sp.phase == 0)) continue;
     const bool in_group = sched && (int)si >= p->sched_s0 && (int)si < p->sched_s1;
     if (!ev.empty() && !merged_mark) {
       // the first merge step; a scheduled group that holds merges counts as merging from its start
@@ -1280,6 +1307,7 @@ thin_attn_status run_forward(thin_attn_s* h, Plan* p, const void* q, const void*
     if (!merged_mark) CK(cudaEventRecord(ev[1], st));
     CK(cudaEventRecord(ev[2], st));
   }
+  if (phase == 1) return THIN_ATTN_OK;
   if (fp8) {
     // e4m3 copies of q, k and the coreset keys for the attention's QK^T (timed with the attention)
     QkFp8Args fa{};
@@ -1496,7 +1524,108 @@ thin_attn_status thin_attn_forward(thin_attn_t h, const void* q, const void* k, 
   if (s != THIN_ATTN_OK) return s;
   s = materialise(h, p);
   if (s != THIN_ATTN_OK) return s;
+  if (h->cfg.thin_split)
+    return fail(THIN_ATTN_EINVAL, "a thin_split handle forwards in two phases (thin_attn_forward_phase)");
   return run_forward(h, p, q, k, v, out, seed, lse_opt, coreset_idx_opt, trace_opt, (cudaStream_t)stream);
+}
+
+thin_attn_status thin_attn_forward_phase(thin_attn_t h, const void* q, const void* k, const void* v, void* out,
+                                         int causal, int g, uint64_t seed, float* lse_opt, int32_t* coreset_idx_opt,
+                                         uint32_t* trace_opt, int phase, void* stream) {
+  if (!h) return fail(THIN_ATTN_EINVAL, "null handle");
+  if (!h->cfg.thin_split || causal != 1) return fail(THIN_ATTN_EINVAL, "phases need a thin_split handle and causal = 1");
+  if (phase != 1 && phase != 2) return fail(THIN_ATTN_EINVAL, "phase %d: 1 (thinning) or 2 (merges and attention)", phase);
+  if (!q || !k || !v || !out) return fail(THIN_ATTN_EINVAL, "q, k, v and out must be non-null");
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (((uintptr_t)ptr) % 16) return fail(THIN_ATTN_EINVAL, "tensor pointers must be 16-byte aligned");
+  std::lock_guard<std::mutex> lk(h->mu);
+  DeviceGuard dg(h->cfg.device);
+  if (!dg.ok) return fail(THIN_ATTN_ECUDA, "cannot select device %d", h->cfg.device);
+  Plan* p = nullptr;
+  thin_attn_status s = get_plan(h, causal, g, &p);
+  if (s != THIN_ATTN_OK) return s;
+  s = materialise(h, p);
+  if (s != THIN_ATTN_OK) return s;
+  return run_forward(h, p, q, k, v, out, seed, lse_opt, coreset_idx_opt, trace_opt, (cudaStream_t)stream, phase);
+}
+
+thin_attn_status thin_attn_nodes_layout(thin_attn_t h, int causal, int g, int* own_begin, int* own_end, int* n_batches,
+                                        uint64_t* bytes_per_batch) {
+  if (!h || !own_begin || !own_end || !n_batches || !bytes_per_batch) return fail(THIN_ATTN_EINVAL, "null argument");
+  if (causal != 1) return fail(THIN_ATTN_EINVAL, "batch coresets exist for causal = 1 only");
+  std::lock_guard<std::mutex> lk(h->mu);
+  Plan* p = nullptr;
+  thin_attn_status s = get_plan(h, causal, g, &p);
+  if (s != THIN_ATTN_OK) return s;
+  const thin_attn_config& cf = h->cfg;
+  *own_begin = p->own_k0;
+  *own_end = p->own_k1;
+  *n_batches = p->n_b;
+  *bytes_per_batch = (uint64_t)cf.B * cf.H * p->c * ((uint64_t)(cf.E + cf.D) * elt(cf) + 4);
+  return THIN_ATTN_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// The level-0 nodes of batches [k0, k1) to or from exchange blocks (see thin_attn_nodes_layout): per
+// batch, keys, values and token indices of every (b,h), each section (b,h)-major.
+thin_attn_status nodes_copy(thin_attn_s* h, int causal, int g, void* blocks, int k0, int k1, bool to_blocks,
+                            cudaStream_t st) {
+  std::lock_guard<std::mutex> lk(h->mu);
+  DeviceGuard dg(h->cfg.device);
+  if (!dg.ok) return fail(THIN_ATTN_ECUDA, "cannot select device %d", h->cfg.device);
+  Plan* p = nullptr;
+  thin_attn_status s = get_plan(h, causal, g, &p);
+  if (s != THIN_ATTN_OK) return s;
+  s = materialise(h, p);
+  if (s != THIN_ATTN_OK) return s;
+  if (k0 < 0 || k1 > p->n_b || k0 > k1) return fail(THIN_ATTN_EINVAL, "batches [%d, %d) outside [0, %d)", k0, k1, p->n_b);
+  if (((uintptr_t)blocks) % 16) return fail(THIN_ATTN_EINVAL, "the exchange buffer must be 16-byte aligned");
+  const thin_attn_config& cf = h->cfg;
+  const size_t es = elt(cf), BH = (size_t)cf.B * cf.H, c = p->c;
+  const void *nk, *nv;
+  int32_t* nidx;
+  buf_ptrs(p, BUF_NODES, nullptr, nullptr, &nk, &nv, &nidx);
+  const size_t kw = c * cf.E * es, vw = c * cf.D * es, iw = c * 4;   // bytes of one (b,h)'s node
+  const size_t block = BH * (kw + vw + iw);
+  const size_t slots = (size_t)p->n_slots;
+  for (int kb = k0; kb < k1; ++kb) {
+    char* blk = (char*)blocks + (size_t)(kb - k0) * block;
+    struct Sec { char* node; size_t w; char* b; } secs[3] = {
+        {(char*)nk + (size_t)kb * kw, kw, blk}, {(char*)nv + (size_t)kb * vw, vw, blk + BH * kw},
+        {(char*)nidx + (size_t)kb * iw, iw, blk + BH * (kw + vw)}};
+    for (const Sec& x : secs) {
+      // node rows of batch kb for every (b,h): pitch = one (b,h)'s node slots
+      if (to_blocks)
+        CK(cudaMemcpy2DAsync(x.b, x.w, x.node, slots * x.w, x.w, BH, cudaMemcpyDeviceToDevice, st));
+      else
+        CK(cudaMemcpy2DAsync(x.node, slots * x.w, x.b, x.w, x.w, BH, cudaMemcpyDeviceToDevice, st));
+    }
+  }
+  return THIN_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+thin_attn_status thin_attn_nodes_export(thin_attn_t h, int causal, int g, void* dst, void* stream) {
+  if (!h || !dst) return fail(THIN_ATTN_EINVAL, "null argument");
+  if (causal != 1) return fail(THIN_ATTN_EINVAL, "batch coresets exist for causal = 1 only");
+  int k0 = 0, k1 = 0, nb = 0;
+  uint64_t bpb = 0;
+  thin_attn_status s = thin_attn_nodes_layout(h, causal, g, &k0, &k1, &nb, &bpb);
+  if (s != THIN_ATTN_OK) return s;
+  return nodes_copy(h, causal, g, dst, k0, k1, true, (cudaStream_t)stream);
+}
+
+thin_attn_status thin_attn_nodes_import(thin_attn_t h, int causal, int g, const void* src, int batch_begin,
+                                        int batch_end, void* stream) {
+  if (!h || !src) return fail(THIN_ATTN_EINVAL, "null argument");
+  if (causal != 1) return fail(THIN_ATTN_EINVAL, "batch coresets exist for causal = 1 only");
+  return nodes_copy(h, causal, g, (void*)src, batch_begin, batch_end, false, (cudaStream_t)stream);
 }
 
 }  // extern "C"
