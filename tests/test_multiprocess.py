@@ -175,3 +175,61 @@ def test_sequence_shard_needs_rows_for_every_rank():
         bench.Shard(W.WORKLOADS["tiny"], 3, 0, "seq")        # T = 256 < 3 x 128
     sh = bench.Shard(W.WORKLOADS["express32k"], 8, 7, "seq")
     assert sh.q_range == (28672, 32768) and sh.rows == (28672, 32768)
+
+
+class _FakeNodes:
+    """A stand-in for a thin_split handle's batch coresets on the CPU: n_b blocks of bpb bytes, the
+    owned ones filled by 'phase 1' with a pattern of (batch, byte), the others zero until imported."""
+
+    def __init__(self, k0, k1, n_b, bpb):
+        self.k0, self.k1, self.n_b, self.bpb = k0, k1, n_b, bpb
+        self.device = torch.device("cpu")
+        self.blocks = torch.zeros(n_b, bpb, dtype=torch.uint8)
+        for kk in range(k0, k1):
+            self.blocks[kk] = (torch.arange(bpb) * 7 + kk * 13) % 251
+
+    def nodes_layout(self, g=2):
+        return self.k0, self.k1, self.n_b, self.bpb
+
+    def nodes_export(self, dst, g=2):
+        dst[:(self.k1 - self.k0) * self.bpb] = self.blocks[self.k0:self.k1].reshape(-1)
+
+    def nodes_import(self, src, a, b, g=2):
+        self.blocks[a:b] = src[:(b - a) * self.bpb].reshape(b - a, self.bpb)
+
+
+def _rank_exchange(rank, world, port, q, owned):
+    import datetime
+    import thinned_softmax_attention_b200 as TA
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        k0, k1 = owned[rank]
+        h = _FakeNodes(k0, k1, owned[-1][1], 96)
+        TA.exchange_batch_coresets(h, 2, dist)
+        q.put((rank, h.blocks.numpy()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("owned", [[(0, 3), (3, 7)], [(0, 0), (0, 4), (4, 5)]])
+def test_batch_coreset_exchange_over_ranks(owned):
+    """exchange_batch_coresets on gloo ranks (the thin_split handles replaced by CPU stand-ins with the
+    same three calls): after the all-gather every rank holds every batch's block, each from the rank
+    that owns it -- unequal ownership (padding) and a rank owning no batch included."""
+    ctx = mp.get_context("spawn")
+    qu = ctx.Queue()
+    port = _free_port()
+    world = len(owned)
+    procs = [ctx.Process(target=_rank_exchange, args=(r, world, port, qu, owned)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted((qu.get(timeout=300) for _ in range(world)), key=lambda r: r[0])
+    for p in procs:
+        p.join(60)
+    assert all(p.exitcode == 0 for p in procs)
+    n_b, bpb = owned[-1][1], 96
+    want = np.stack([((np.arange(bpb) * 7 + kk * 13) % 251).astype(np.uint8) for kk in range(n_b)])
+    for _, blocks in res:
+        np.testing.assert_array_equal(blocks, want)
