@@ -22,35 +22,6 @@ namespace {
 constexpr int kDecodeChunk = 128;     // keys per CTA
 constexpr int kDecodeThreads = 128;   // 4 warps x 32 keys
 
-template <typename T, int EPL>
-__device__ __forceinline__ void load_lane(const T* row, int lane, float (&x)[EPL]) {
-  if constexpr (sizeof(T) == 2) {
-    // EPL bf16 = EPL * 2 bytes per lane
-    if constexpr (EPL == 2) {
-      const uint32_t u = *(const uint32_t*)(row + lane * 2);
-      x[0] = __uint_as_float(u << 16);
-      x[1] = __uint_as_float(u & 0xFFFF0000u);
-    } else if constexpr (EPL == 4) {
-      const uint2 u = *(const uint2*)(row + lane * 4);
-      x[0] = __uint_as_float(u.x << 16);
-      x[1] = __uint_as_float(u.x & 0xFFFF0000u);
-      x[2] = __uint_as_float(u.y << 16);
-      x[3] = __uint_as_float(u.y & 0xFFFF0000u);
-    } else {
-      const uint4 u = *(const uint4*)(row + lane * 8);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        x[2 * i] = __uint_as_float(w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) x[i] = to_f(row[lane * EPL + i]);
-  }
-}
-
 // A lane's DPL elements of a value row, kept as loaded (bf16 pairs or fp32 words) until used, so that
 // a round of rows in flight costs half the registers in bf16.
 template <typename T, int DPL>
